@@ -1,0 +1,219 @@
+"""CPU oracle for the routed MoE expert FFN -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never does, and this
+package never imports the CUDA library: the two share nothing but the seeded
+input bytes produced by ``moe_inputs``.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, fp64); this module builds it
+with gcc and marshals numpy arrays through ctypes.  Each wrapper names the
+step it follows:
+
+* ``quant_x``      -- per-token FP8 activation quantisation (R0);
+* ``route``        -- top-k, renormalised softmax, histogram, scan and stable
+                      permutation (R1/R2; rocketrecap.com "FlyDSL kernels in
+                      JAX", timestamps 5:56 "dynamic expert sizes" and 8:14
+                      "top-2 routing");
+* ``moe_ffn``      -- the whole layer, routed or masked-dense form (paragraph 2
+                      and timestamp 5:56: gather, group GEMM, SwiGLU, scatter
+                      versus the masked dense GEMM path);
+* ``moe_ffn_tokens`` -- the same layer evaluated on a subset of tokens.
+
+Parity of these functions with the pages is pinned by ``tests/test_oracle.py``.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+BF16 = 0
+FP8 = 1
+
+
+def build(force=False):
+    """Compile liboracle.so next to its source (gcc, OpenMP, no fast-math)."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-fno-fast-math", "-ffp-contract=off",
+           _SRC, "-o", _LIB + ".tmp", "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        lib.oracle_e4m3_to_double.restype = ctypes.c_double
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_from_float.restype = ctypes.c_uint8
+        lib.oracle_e4m3_from_float.argtypes = [ctypes.c_float]
+        lib.oracle_bf16_from_double.restype = ctypes.c_uint16
+        lib.oracle_bf16_from_double.argtypes = [ctypes.c_double]
+        lib.oracle_bf16_to_double.restype = ctypes.c_double
+        lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        lib.oracle_mx_exponent.restype = I
+        lib.oracle_mx_exponent.argtypes = [ctypes.c_double]
+        lib.oracle_mx_quant_block.restype = I
+        lib.oracle_mx_quant_block.argtypes = [P, I, P]
+        lib.oracle_quant_x.restype = None
+        lib.oracle_quant_x.argtypes = [P, I, I, P, P]
+        lib.oracle_route.restype = I
+        lib.oracle_route.argtypes = [P, I, I, I, P, P, P, P, P, P]
+        lib.oracle_moe_ffn.restype = I
+        lib.oracle_moe_ffn.argtypes = [I, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, I]
+        lib.oracle_moe_ffn_tokens.restype = I
+        lib.oracle_moe_ffn_tokens.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, I, P, P, I]
+        lib.oracle_max_threads.restype = I
+        lib.oracle_max_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def max_threads():
+    return _load().oracle_max_threads()
+
+
+# -- number formats ---------------------------------------------------------
+
+def e4m3_to_double(code):
+    return _load().oracle_e4m3_to_double(int(code) & 0xFF)
+
+
+def e4m3_from_float(v):
+    return _load().oracle_e4m3_from_float(float(v))
+
+
+def bf16_from_double(v):
+    return _load().oracle_bf16_from_double(float(v))
+
+
+def bf16_to_double(b):
+    return _load().oracle_bf16_to_double(int(b) & 0xFFFF)
+
+
+def mx_exponent(amax):
+    return _load().oracle_mx_exponent(float(amax))
+
+
+def mx_quant_block(hb):
+    """Quantise one block of bf16 values (given as float64): (exponent, codes)."""
+    hb = _c(hb, np.float64)
+    codes = np.zeros(hb.shape[0], dtype=np.uint8)
+    e = _load().oracle_mx_quant_block(_ptr(hb), hb.shape[0], _ptr(codes))
+    return e, codes
+
+
+# -- R0 --------------------------------------------------------------------
+
+def quant_x(x_bf16_bits):
+    """x: uint16 [T,H] bf16 bit patterns -> (xq uint8 [T,H], sx float32 [T])."""
+    x = _c(x_bf16_bits, np.uint16)
+    T, H = x.shape
+    xq = np.zeros((T, H), dtype=np.uint8)
+    sx = np.zeros(T, dtype=np.float32)
+    _load().oracle_quant_x(_ptr(x), T, H, _ptr(xq), _ptr(sx))
+    return xq, sx
+
+
+# -- R1/R2 -----------------------------------------------------------------
+
+def route(logits, k):
+    """logits float32 [T,E] -> dict(ids, w, counts, offsets, perm, inv_perm)."""
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    A = T * k
+    ids = np.zeros(max(A, 1), dtype=np.int32)
+    w = np.zeros(max(A, 1), dtype=np.float64)
+    counts = np.zeros(E, dtype=np.int32)
+    offsets = np.zeros(E + 1, dtype=np.int32)
+    perm = np.zeros(max(A, 1), dtype=np.int32)
+    inv = np.zeros(max(A, 1), dtype=np.int32)
+    rc = _load().oracle_route(_ptr(lg), T, E, k, _ptr(ids), _ptr(w), _ptr(counts), _ptr(offsets),
+                              _ptr(perm), _ptr(inv))
+    if rc != 0:
+        raise ValueError("oracle_route: bad arguments")
+    return dict(ids=ids[:A].reshape(T, k), w=w[:A].reshape(T, k), counts=counts, offsets=offsets,
+                perm=perm[:A], inv_perm=inv[:A])
+
+
+# -- the layer --------------------------------------------------------------
+
+def _weights(case):
+    fp8 = case["dtype"] == "fp8"
+    wt = np.uint8 if fp8 else np.uint16
+    w1 = _c(case["w1"], wt)
+    w3 = _c(case["w3"], wt)
+    w2 = _c(case["w2"], wt)
+    s1 = _c(case.get("s1"), np.float32) if fp8 else None
+    s3 = _c(case.get("s3"), np.float32) if fp8 else None
+    s2 = _c(case.get("s2"), np.float32) if fp8 else None
+    return w1, w3, w2, s1, s3, s2, (FP8 if fp8 else BF16)
+
+
+def moe_ffn(case, mode="routed", nthreads=0, want_h=False):
+    """Whole layer on a case dict of numpy arrays (see ``moe_inputs.to_numpy``).
+
+    Returns dict(out=uint16 [T,H] bf16 bits, out64=float64 [T,H], h=optional
+    float64 [T*k,F] dequantised intermediate in sorted order)."""
+    x = _c(case["x"], np.uint16)
+    lg = _c(case["logits"], np.float32)
+    T, H = x.shape
+    E = lg.shape[1]
+    k = int(case["k"])
+    w1, w3, w2, s1, s3, s2, dt = _weights(case)
+    F = w1.shape[1]
+    out = np.zeros((T, H), dtype=np.uint16)
+    out64 = np.zeros((T, H), dtype=np.float64)
+    h = np.zeros((T * k, F), dtype=np.float64) if want_h else None
+    rc = _load().oracle_moe_ffn(0 if mode == "routed" else 1, _ptr(x), _ptr(lg), _ptr(w1), _ptr(w3),
+                                _ptr(s1), _ptr(s3), _ptr(w2), _ptr(s2), T, H, F, E, k, dt, _ptr(out),
+                                _ptr(out64), _ptr(h), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_moe_ffn: bad arguments")
+    return dict(out=out, out64=out64, h=h)
+
+
+def moe_ffn_tokens(case, tokens, nthreads=0):
+    """Output rows for the given token ids only: dict(out [n,H] bf16 bits, out64)."""
+    x = _c(case["x"], np.uint16)
+    lg = _c(case["logits"], np.float32)
+    T, H = x.shape
+    E = lg.shape[1]
+    k = int(case["k"])
+    w1, w3, w2, s1, s3, s2, dt = _weights(case)
+    F = w1.shape[1]
+    tok = _c(tokens, np.int32)
+    n = tok.shape[0]
+    out = np.zeros((n, H), dtype=np.uint16)
+    out64 = np.zeros((n, H), dtype=np.float64)
+    rc = _load().oracle_moe_ffn_tokens(_ptr(x), _ptr(lg), _ptr(w1), _ptr(w3), _ptr(s1), _ptr(s3),
+                                       _ptr(w2), _ptr(s2), T, H, F, E, k, dt, _ptr(tok), n, _ptr(out),
+                                       _ptr(out64), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_moe_ffn_tokens: bad arguments")
+    return dict(out=out, out64=out64)
+
+
+def bf16_bits_to_float(b):
+    """uint16 bf16 bit patterns -> float64 values (exact widening)."""
+    b = np.asarray(b, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

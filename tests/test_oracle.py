@@ -1,0 +1,344 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself -- library routines (torch's float8/bfloat16 casts, torch.softmax,
+fp64 matmuls, Python's stable sort), closed forms, invariants and brute force.
+
+The method is the routed MoE expert FFN of rocketrecap.com "FlyDSL kernels in
+JAX" (paragraph 2; timestamps 5:56 and 8:14).  Numeric readings the pages leave
+open (tie-break, softmax over the selected logits, FP8 quantisation points) are
+the ones stated in the oracle's header.
+"""
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+import oracle
+
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+def e4m3_lib(v):
+    """torch's float32 -> float8_e4m3fn cast (round to nearest even)."""
+    return int(torch.tensor([v], dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).item())
+
+
+def bf16_lib(v):
+    return int(torch.tensor([v], dtype=torch.float32).to(torch.bfloat16).view(torch.int16).item()) & 0xFFFF
+
+
+# ---------------------------------------------------------------- formats
+
+def test_e4m3_decode_all_codes_match_library():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    lib = codes.view(torch.float8_e4m3fn).float().double().numpy()
+    for c in range(256):
+        mine = oracle.e4m3_to_double(c)
+        if math.isnan(lib[c]):
+            assert math.isnan(mine), c
+        else:
+            assert mine == lib[c], (c, mine, lib[c])
+    assert oracle.e4m3_to_double(0x7E) == 448.0
+    assert oracle.e4m3_to_double(0x01) == 2.0 ** -9  # smallest subnormal
+
+
+def test_e4m3_encode_matches_library_in_range():
+    rng = np.random.default_rng(1)
+    vals = list(rng.normal(0, 50, 4000).astype(np.float32)) + list(rng.normal(0, 0.01, 2000).astype(np.float32))
+    # exact midpoints between neighbouring codes (ties) and values just beside them
+    pos = [oracle.e4m3_to_double(c) for c in range(0x7F)]
+    for a, b in zip(pos[:-1], pos[1:]):
+        m = np.float32((a + b) / 2)
+        vals += [m, -m, np.nextafter(m, np.float32(0)), np.nextafter(m, np.float32(1e9))]
+    for v in vals:
+        v = np.float32(v)
+        if abs(v) > 448:
+            continue
+        assert oracle.e4m3_from_float(v) == e4m3_lib(v), v
+
+
+def test_e4m3_ties_to_even_and_saturation():
+    assert oracle.e4m3_from_float(1.0625) == 0x38      # 1.0 (mantissa 000) beats 1.125
+    assert oracle.e4m3_from_float(1.1875) == 0x3A      # 1.25 (mantissa 010) beats 1.125
+    assert oracle.e4m3_from_float(448.0) == 0x7E
+    assert oracle.e4m3_from_float(470.0) == 0x7E       # satfinite clamps
+    assert oracle.e4m3_from_float(1e30) == 0x7E
+    assert oracle.e4m3_from_float(-1e30) == 0xFE
+    assert oracle.e4m3_from_float(float("inf")) == 0x7E
+    assert oracle.e4m3_from_float(float("nan")) == 0x7F
+    assert oracle.e4m3_from_float(-0.0) == 0x80
+    assert oracle.e4m3_from_float(2.0 ** -10) == 0x00  # half the smallest subnormal: tie to even (0)
+
+
+def test_bf16_round_matches_library_for_binary32_inputs():
+    rng = np.random.default_rng(2)
+    vals = np.concatenate([rng.normal(0, 1, 3000), rng.normal(0, 1e-30, 200), rng.normal(0, 1e30, 200)])
+    vals = vals.astype(np.float32)
+    # binary32 values halfway between two bf16 values
+    halfway = (rng.integers(0, 2 ** 15, 500, dtype=np.uint32) << 16 | 0x8000).view(np.float32)
+    for v in list(vals) + list(halfway):
+        if not np.isfinite(v):
+            continue
+        assert oracle.bf16_from_double(float(v)) == bf16_lib(float(v)), v
+
+
+def test_bf16_round_from_double_is_single_rounding():
+    # a double just above a bf16 tie must round up (a binary32 detour would
+    # land exactly on the tie and round to even = down)
+    lo = 1.0
+    ulp = 2.0 ** -7
+    v = lo + ulp / 2 + 2.0 ** -40
+    assert Fraction(v) > Fraction(lo) + Fraction(ulp) / 2
+    assert oracle.bf16_to_double(oracle.bf16_from_double(v)) == lo + ulp
+    assert oracle.bf16_to_double(oracle.bf16_from_double(lo + ulp / 2)) == lo   # exact tie -> even
+    assert oracle.bf16_to_double(oracle.bf16_from_double(lo + 3 * ulp / 2)) == lo + 2 * ulp
+
+
+# ---------------------------------------------------------------- R0
+
+def test_quant_x_properties():
+    rng = np.random.default_rng(3)
+    x = torch.tensor(rng.normal(0, 1, (6, 64)), dtype=torch.float32).to(torch.bfloat16)
+    x[2] = 0
+    x[3, 5] = -7.5  # dominating negative absmax
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    xq, sx = oracle.quant_x(bits)
+    xf = x.float().numpy()
+    assert sx[2] == 1.0 and np.all(xq[2] == 0)
+    for t in (0, 1, 3, 4, 5):
+        amax = np.abs(xf[t]).max()
+        # sx is the binary32 quotient absmax / 448
+        assert abs(float(sx[t]) * 448.0 - amax) <= amax * 2.0 ** -23
+        i = int(np.abs(xf[t]).argmax())
+        assert xq[t, i] in (0x7E, 0xFE)  # the absmax element maps to +-448
+        deq = np.array([oracle.e4m3_to_double(c) for c in xq[t]]) * float(sx[t])
+        # nearest-value rounding: error at most half the spacing of e4m3 at that magnitude
+        for v, d in zip(xf[t], deq):
+            mag = abs(v) / float(sx[t])
+            spacing = 2.0 ** (max(math.floor(math.log2(mag)), -6) - 3) if mag > 0 else 2.0 ** -9
+            assert abs(d - v) <= 0.5 * spacing * float(sx[t]) * (1 + 1e-6) + 1e-30
+    assert xq[3, 5] == 0xFE
+
+
+# ---------------------------------------------------------------- MX block quantisation of h
+
+@pytest.mark.parametrize("amax,expected", [
+    (448.0, 0), (224.0, -1), (896.0, 1), (448.0 * 2 ** -10, -10), (449.0, 1), (447.0, 0),
+    (1.0, -8), (1.75, -8), (1.7578125, -7), (0.0, 0), (1e-40, -127), (3e38, 120)])
+def test_mx_exponent_closed_form(amax, expected):
+    assert oracle.mx_exponent(amax) == expected
+
+
+def test_mx_quant_block_properties():
+    rng = np.random.default_rng(4)
+    for trial in range(50):
+        hb = torch.tensor(rng.normal(0, 10.0 ** rng.uniform(-6, 3), 32), dtype=torch.float32)
+        hb = hb.to(torch.bfloat16).double().numpy()
+        e, codes = oracle.mx_quant_block(hb)
+        amax = np.abs(hb).max()
+        assert amax / 2.0 ** e <= 448.0
+        assert amax / 2.0 ** e > 224.0  # smallest power of two that fits
+        for v, c in zip(hb, codes):
+            assert c == e4m3_lib(np.float32(v / 2.0 ** e))
+    e, codes = oracle.mx_quant_block(np.zeros(32))
+    assert e == 0 and np.all(codes == 0)
+
+
+# ---------------------------------------------------------------- R1/R2 routing
+
+def _brute_topk(l, k):
+    key = lambda e: (-(-math.inf if math.isnan(l[e]) else float(l[e])), e)  # noqa: E731
+    return sorted(range(len(l)), key=key)[:k]
+
+
+def _check_routing(logits, k):
+    r = oracle.route(logits, k)
+    T, E = logits.shape
+    for t in range(T):
+        assert list(r["ids"][t]) == _brute_topk(logits[t], k), t
+        sel = np.array([logits[t, e] for e in r["ids"][t]], dtype=np.float64)
+        if np.all(np.isfinite(sel)):
+            ref = torch.softmax(torch.tensor(sel), dim=0).numpy()
+            np.testing.assert_allclose(r["w"][t], ref, rtol=1e-14, atol=1e-15)
+        assert abs(r["w"][t].sum() - 1.0) < 1e-12
+    flat = r["ids"].reshape(-1)
+    np.testing.assert_array_equal(r["counts"], np.bincount(flat, minlength=E))
+    assert r["counts"].sum() == T * k
+    np.testing.assert_array_equal(r["offsets"], np.concatenate([[0], np.cumsum(r["counts"])]))
+    # stable sort of assignments by expert (Python's sort is stable)
+    np.testing.assert_array_equal(r["perm"], sorted(range(T * k), key=lambda a: flat[a]))
+    np.testing.assert_array_equal(r["inv_perm"][r["perm"]], np.arange(T * k))
+    return r
+
+
+@pytest.mark.parametrize("T,E,k", [(8, 4, 2), (8, 4, 1), (5, 3, 3), (7, 8, 2), (64, 8, 2), (33, 64, 8)])
+def test_route_matches_brute_force(T, E, k):
+    rng = np.random.default_rng(T * 100 + E * 10 + k)
+    _check_routing(rng.normal(0, 1, (T, E)).astype(np.float32), k)
+
+
+def test_route_ties_nan_and_signed_zero():
+    lg = np.array([
+        [1.0, 1.0, 1.0, 1.0],          # all equal -> experts 0, 1
+        [0.0, -0.0, 0.5, -1.0],        # 0.5 first, then +0 vs -0 tie -> lower index 0
+        [np.nan, -5.0, np.nan, -6.0],  # NaN ranks as -inf
+        [-np.inf, np.nan, -np.inf, np.nan],  # nothing finite -> index order
+        [2.0, 3.0, 3.0, 1.0],          # tie on the max -> 1 then 2
+    ], dtype=np.float32)
+    r = _check_routing(lg, 2)
+    assert r["ids"].tolist() == [[0, 1], [2, 0], [1, 3], [0, 1], [1, 2]]
+    np.testing.assert_allclose(r["w"][0], [0.5, 0.5])
+    np.testing.assert_allclose(r["w"][3], [0.5, 0.5])   # limit reading: equal shares
+    np.testing.assert_allclose(r["w"][4], [0.5, 0.5])
+
+
+def test_route_k_equals_e_and_k1():
+    rng = np.random.default_rng(7)
+    lg = rng.normal(0, 1, (9, 4)).astype(np.float32)
+    r = _check_routing(lg, 4)
+    np.testing.assert_array_equal(r["counts"], [9, 9, 9, 9])
+    r1 = _check_routing(lg, 1)
+    assert np.all(r1["w"] == 1.0)
+
+
+def test_route_skewed_shares():
+    lg = moe_inputs.make_logits(8192, 8, 3, skew=True).numpy()
+    r = oracle.route(lg, 2)
+    share = r["counts"] / r["counts"].sum()
+    assert share[0] > 0.40 and share[7] < 0.01 and np.all(np.diff(share) < 0)
+
+
+# ---------------------------------------------------------------- the layer
+
+def _bf16_round_vec(a):
+    return np.array([oracle.bf16_to_double(oracle.bf16_from_double(float(v))) for v in a.reshape(-1)]).reshape(a.shape)
+
+
+def _dense_swiglu_reference(case, tok):
+    """E=1, k=1: the layer is a dense SwiGLU MLP; fp64 torch matmuls."""
+    fp8 = case["dtype"] == "fp8"
+    x = case["x"].double()
+    if fp8:
+        xq, sx = oracle.quant_x(moe_inputs.to_numpy(case)["x"])
+        xd = torch.tensor(xq).view(torch.float8_e4m3fn).double() * torch.tensor(sx).double()[:, None]
+        deq = lambda w, s: w.double() * s.double()[..., None]  # noqa: E731
+        W1, W3, W2 = deq(case["w1"][0], case["s1"][0]), deq(case["w3"][0], case["s3"][0]), deq(case["w2"][0], case["s2"][0])
+    else:
+        xd = x
+        W1, W3, W2 = case["w1"][0].double(), case["w3"][0].double(), case["w2"][0].double()
+    xd = xd[tok]
+    g = xd @ W1.T
+    u = xd @ W3.T
+    h = _bf16_round_vec((g * torch.sigmoid(g) * u).numpy())
+    if fp8:
+        hq = np.empty_like(h)
+        for r in range(h.shape[0]):
+            for b in range(0, h.shape[1], 32):
+                e, codes = oracle.mx_quant_block(h[r, b:b + 32])
+                hq[r, b:b + 32] = [oracle.e4m3_to_double(c) * 2.0 ** e for c in codes]
+        h = hq
+    return (torch.tensor(h) @ W2.T).numpy()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_single_expert_equals_dense_swiglu_mlp(dtype):
+    case = moe_inputs.make_case(T=6, H=64, F=96, E=1, k=1, dtype=dtype, seed=11)
+    r = oracle.moe_ffn(moe_inputs.to_numpy(case))
+    ref = _dense_swiglu_reference(case, np.arange(6))
+    scale = np.sqrt(np.mean(ref ** 2))
+    assert np.max(np.abs(r["out64"] - ref)) <= 1e-12 * scale
+    np.testing.assert_array_equal(r["out"], np.array([[oracle.bf16_from_double(v) for v in row] for row in ref]))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_routed_equals_masked_dense(dtype):
+    case = moe_inputs.make_case(T=12, H=64, F=64, E=4, k=2, dtype=dtype, seed=12)
+    nc = moe_inputs.to_numpy(case)
+    a = oracle.moe_ffn(nc, mode="routed")
+    b = oracle.moe_ffn(nc, mode="masked_dense")
+    scale = np.sqrt(np.mean(a["out64"] ** 2))
+    assert np.max(np.abs(a["out64"] - b["out64"])) <= 1e-12 * scale
+    np.testing.assert_array_equal(a["out"], b["out"])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_token_permutation_permutes_output(dtype):
+    case = moe_inputs.make_case(T=10, H=32, F=64, E=4, k=2, dtype=dtype, seed=13)
+    nc = moe_inputs.to_numpy(case)
+    base = oracle.moe_ffn(nc)
+    p = np.random.default_rng(5).permutation(10)
+    nc2 = dict(nc)
+    nc2["x"] = nc["x"][p]
+    nc2["logits"] = nc["logits"][p]
+    perm_out = oracle.moe_ffn(nc2)
+    np.testing.assert_array_equal(perm_out["out"], base["out"][p])
+    r1, r2 = oracle.route(nc["logits"], 2), oracle.route(nc2["logits"], 2)
+    np.testing.assert_array_equal(r2["ids"], r1["ids"][p])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_token_subset_matches_full_layer(dtype):
+    case = moe_inputs.make_case(T=9, H=32, F=64, E=4, k=2, dtype=dtype, seed=14)
+    nc = moe_inputs.to_numpy(case)
+    full = oracle.moe_ffn(nc)
+    tok = np.array([7, 0, 3])
+    sub = oracle.moe_ffn_tokens(nc, tok)
+    np.testing.assert_array_equal(sub["out"], full["out"][tok])
+
+
+def test_one_hot_closed_form():
+    """x_t = v_t * onehot(i_t); w1 = a_e I, w3 = b_e I, w2 = c_e P (P a cyclic
+    shift, not an involution).  Then Y(e,t)[P(i_t)] = c_e * bf16(silu(a_e v) b_e v)
+    and every other output is zero."""
+    D, E, k, T = 16, 3, 2, 5
+    a = [0.5, 1.5, -2.0]
+    b = [0.25, -1.0, 3.0]
+    c = [2.0, 0.5, -1.0]
+    shift = lambda n: (n + 3) % D  # noqa: E731
+    w1 = torch.zeros(E, D, D)
+    w3 = torch.zeros(E, D, D)
+    w2 = torch.zeros(E, D, D)
+    for e in range(E):
+        for n in range(D):
+            w1[e, n, n] = a[e]
+            w3[e, n, n] = b[e]
+            w2[e, shift(n), n] = c[e]
+    idx = [1, 4, 9, 15, 0]
+    vals = [1.0, -0.5, 2.0, 0.75, -3.0]
+    x = torch.zeros(T, D)
+    for t in range(T):
+        x[t, idx[t]] = vals[t]
+    logits = torch.tensor([[0.1, 0.7, 0.3], [1.0, 1.0, -1.0], [-2.0, 0.0, 2.0], [0.0, 0.0, 0.0], [5.0, -5.0, 4.0]])
+    case = dict(x=x.to(torch.bfloat16), logits=logits, w1=w1.to(torch.bfloat16), w3=w3.to(torch.bfloat16),
+                w2=w2.to(torch.bfloat16), k=k, dtype="bf16")
+    r = oracle.moe_ffn(moe_inputs.to_numpy(case))
+    for t in range(T):
+        lg = logits[t].tolist()
+        sel = sorted(range(E), key=lambda e: (-lg[e], e))[:k]
+        ex = [math.exp(lg[e] - lg[sel[0]]) for e in sel]
+        wts = [v / sum(ex) for v in ex]
+        expect = np.zeros(D)
+        v = vals[t]
+        for wj, e in sorted(zip(wts, sel), key=lambda p: p[1]):
+            g = a[e] * v
+            hval = oracle.bf16_to_double(oracle.bf16_from_double(g / (1 + math.exp(-g)) * (b[e] * v)))
+            expect[shift(idx[t])] += wj * c[e] * hval
+        np.testing.assert_allclose(r["out64"][t], expect, rtol=1e-15, atol=1e-300)
+
+
+def test_golden_regression_record():
+    """The stored record was written by tests/golden/make_golden.py (oracle only)."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_routing_and_rows.json")
+    with open(path) as f:
+        g = json.load(f)
+    nc = moe_inputs.to_numpy(moe_inputs.make_config("tiny"))
+    r = oracle.route(nc["logits"], nc["k"])
+    assert r["ids"].tolist() == g["topk_ids"]
+    assert r["counts"].tolist() == g["counts"]
+    assert r["perm"].tolist() == g["perm"]
+    rows = oracle.moe_ffn_tokens(nc, g["tokens"])
+    assert rows["out"].tolist() == g["out_bits"]
