@@ -1,0 +1,185 @@
+/*
+ * moe.h -- C ABI of libmoe: the routed mixture-of-experts expert FFN on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (rocketrecap.com, "FlyDSL kernels in JAX" talk summary):
+ *   paragraph 2 and timestamp 5:56 -- a two-stage routed MoE GEMM: gather of
+ *     each expert's tokens, group GEMM with the gate/up projections (w1, w3),
+ *     SwiGLU, group GEMM with the down projection (w2), scatter back to token
+ *     order; it replaces a masked dense GEMM over all experts;
+ *   timestamp 8:14 -- Mixtral-8x7B, top-2 routing, FP8, a one-time load-time
+ *     preshuffle of the expert weights;
+ *   timestamps 4:07 and 5:05 -- the host boundary: buffers, scalars and a
+ *     stream handed to the kernel launcher.
+ *
+ * Conventions for every entry point
+ *   - Pointers marked "device" must point to memory of the current CUDA device;
+ *     pointers marked "host" to host memory.  The caller owns every buffer;
+ *     the library allocates no device memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued asynchronously; no entry point except moe_get_status waits for
+ *     the device.
+ *   - Arguments are validated on the host before anything is enqueued; on any
+ *     return other than MOE_OK nothing was enqueued and outputs are untouched.
+ *   - Faults a kernel detects (a wait that timed out, an index out of range)
+ *     are recorded in a device status word read by moe_get_status.  Outputs of
+ *     a call whose status is not MOE_OK are undefined.
+ *   - Every device pointer must be 16-byte aligned (MOE_ERR_ALIGNMENT).
+ *
+ * Shapes: T tokens, H = d_model, F = d_ff, E experts, k experts per token,
+ * A = T*k assignments (assignment a = t*k + j is token t's j-th choice).
+ * Limits: 1 <= k <= min(E, 8), E <= 64, H % 128 == 0, F % 128 == 0,
+ * 0 <= T, T*k <= 262144 (MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,    /* null pointer, bad dimension or k/E out of range */
+    MOE_ERR_UNSUPPORTED = -2,    /* valid request outside what the kernels implement */
+    MOE_ERR_ALIGNMENT = -3,      /* a device pointer is not 16-byte aligned */
+    MOE_ERR_WORKSPACE = -4,      /* ws_bytes < moe_workspace_size(...) */
+    MOE_ERR_CUDA = -5,           /* a CUDA runtime/driver call or launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = -6, /* a kernel's bounded wait ran out (device status) */
+    MOE_ERR_DEVICE_BOUNDS = -7   /* a kernel saw an index out of range (device status) */
+} moe_status;
+
+typedef enum {
+    MOE_BF16 = 0,     /* bf16 activations and weights */
+    MOE_FP8_E4M3 = 1  /* e4m3 weights with fp32 per-output-channel scales; bf16 activations
+                         quantised per token to e4m3 inside the layer */
+} moe_dtype;
+
+/* Bytes of device workspace moe_ffn_forward needs for this problem (0 on bad
+ * arguments).  The same workspace also serves moe_route. */
+size_t moe_workspace_size(int T, int H, int F, int E, int k, int dtype);
+
+/*
+ * One-time weight preshuffle (timestamp 8:14, "load-time preshuffle").
+ * Interleaves the gate and up projections so that one tile of the first group
+ * GEMM holds matching gate/up output channels:
+ *   w13[e][64*b + i]      = w1[e][32*b + i]   for i in [0,32)
+ *   w13[e][64*b + 32 + i] = w3[e][32*b + i]
+ * and the same for the scales s13 (FP8 only; NULL for BF16).
+ *   w1, w3   device, [E,F,H] row-major (bf16 or e4m3 bytes), read only
+ *   s1, s3   device, [E,F] fp32, read only (FP8) or NULL (BF16)
+ *   w13_out  device, [E,2F,H] (bf16 or e4m3), written
+ *   s13_out  device, [E,2F] fp32 (FP8) or NULL
+ */
+int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const float* s3, void* w13_out,
+                        float* s13_out, int E, int F, int H, int dtype, void* stream);
+
+/*
+ * Routing alone (timestamps 5:56 and 8:14): top-k selection, softmax over the
+ * k selected logits, expert histogram, exclusive scan and stable permutation.
+ *   logits    device, [T,E] fp32, read only.  Larger logit first; equal logits
+ *             go to the lower expert index; NaN ranks as -inf.
+ *   topk_ids  device, [T,k] int32, written: chosen experts, best first.
+ *   topk_w    device, [T,k] fp32, written: exp(l_j - l_max) / sum_i exp(l_i - l_max)
+ *             over the chosen logits (expf, so not bit-exact with an fp64 softmax).
+ *   counts    device, [E] int32, written: assignments per expert.
+ *   offsets   device, [E+1] int32, written: exclusive scan of counts.
+ *   perm      device, [T*k] int32, written: sorted position -> assignment,
+ *             grouped by expert, ascending assignment index within an expert.
+ *   inv_perm  device, [T*k] int32, written: assignment -> sorted position.
+ *   ws, ws_bytes  reserved; routing alone needs no workspace (may be NULL, 0).
+ * ids, counts, offsets, perm and inv_perm are deterministic (bit-identical
+ * from run to run).
+ */
+int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w, int32_t* counts,
+              int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The whole MoE layer: out = sum_j topk_w[t,j] * W2_e (silu(W1_e x_t) * (W3_e x_t)),
+ * e = topk_ids[t,j] (paragraph 2 and timestamp 5:56).
+ *   x        device, [T,H] bf16, read only.
+ *   logits   device, [T,E] fp32, read only (routed exactly as moe_route does).
+ *   w13      device, prepared by moe_prepare_weights: [E,2F,H] bf16 or e4m3.
+ *   s13      device, [E,2F] fp32 (FP8) or NULL (BF16).
+ *   w2       device, [E,H,F] bf16 or e4m3, read only.
+ *   s2       device, [E,H] fp32 (FP8) or NULL (BF16).
+ *   out      device, [T,H] bf16, written.
+ *   ws       device workspace, >= moe_workspace_size(T,H,F,E,k,dtype) bytes;
+ *            scratch, contents undefined afterwards (moe_workspace_region
+ *            gives the offsets of the intermediate buffers it holds).
+ * Numerics: products accumulate in fp32 on the tensor cores.  FP8 mode:
+ * x is quantised per token (sx = absmax/448 in IEEE fp32, e4m3 round to
+ * nearest even with saturation); the intermediate h is rounded to bf16 and
+ * re-quantised to e4m3 in blocks of 32 d_ff elements with a power-of-two
+ * scale 2^ceil(log2(absmax/448)).  BF16 mode: h is rounded to bf16.  The k
+ * weighted expert outputs are summed in fp32 and rounded once to bf16.
+ * The call makes no host<->device synchronisation and may be captured in a
+ * CUDA graph.
+ */
+int moe_ffn_forward(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
+                    const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* Waits for `stream`, then returns and clears the device status word:
+ * MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BOUNDS, or MOE_ERR_CUDA when
+ * the wait itself failed. */
+int moe_get_status(void* stream);
+
+/* Regions of the workspace that moe_ffn_forward fills (for inspection and
+ * tests).  Returns the byte offset of region `which` inside ws and its size in
+ * *bytes, or -1 for a bad argument. */
+typedef enum {
+    MOE_WS_TOPK_IDS = 0,   /* int32 [T*k] */
+    MOE_WS_TOPK_W = 1,     /* fp32 [T*k] */
+    MOE_WS_COUNTS = 2,     /* int32 [E] */
+    MOE_WS_OFFSETS = 3,    /* int32 [E+1] */
+    MOE_WS_PERM = 4,       /* int32 [T*k] */
+    MOE_WS_INV_PERM = 5,   /* int32 [T*k] */
+    MOE_WS_SLOT_OF = 6,    /* int32 [T*k]: assignment -> row of the expert-padded layout */
+    MOE_WS_XS = 7,         /* gathered activations, one row per padded slot: e4m3 or bf16 [S,H] */
+    MOE_WS_SX = 8,         /* fp32 [S]: per-row activation scale (FP8) */
+    MOE_WS_H = 9,          /* intermediate h [S,F]: e4m3 or bf16 */
+    MOE_WS_H_SF = 10,      /* UE8M0 block scales of h (FP8), tiled for the tensor cores */
+    MOE_WS_OUT32 = 11,     /* fp32 [T,H] combine buffer */
+    MOE_WS_NUM_MTILES = 12, /* int32: number of 128-row tiles in the padded layout */
+    MOE_WS_SLOT_ASSIGN = 13, /* int32 [S]: padded row -> assignment, -1 for a padding row */
+    MOE_WS_MTILE_EXPERT = 14 /* int32 [S/128]: 128-row tile -> expert */
+} moe_ws_region;
+
+long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int which, size_t* bytes);
+
+/* Kernel selection for tests and tuning (host-side setting, process-wide).
+ *   MOE_OPT_PATH:     0 = choose by problem size, 1 = force the throughput
+ *                     tiles, 2 = force the weight-streaming tiles.
+ *   MOE_OPT_SPLITK:   0 = automatic, n > 0 = split the second GEMM's K into n parts
+ *                     (must divide F/128).
+ *   MOE_OPT_TIMEOUT_MS: limit of every device-side wait (default 2000).
+ * Returns the previous value, or MOE_ERR_INVALID_ARG. */
+typedef enum { MOE_OPT_PATH = 0, MOE_OPT_SPLITK = 1, MOE_OPT_TIMEOUT_MS = 2 } moe_option;
+int moe_set_option(int option, int value);
+
+/* Per-kernel device timing (tracing aid).  While enabled, moe_ffn_forward
+ * records a pair of CUDA events around each kernel it enqueues.
+ * moe_profile_enable returns the previous setting.  moe_profile_read waits for
+ * the recorded events, adds up the elapsed time per kernel into
+ * ms_total[MOE_KERNEL_COUNT] and the number of launches into
+ * launches[MOE_KERNEL_COUNT] (both host arrays, either may be NULL), and
+ * forgets the records when `reset` is nonzero.  Returns MOE_OK or MOE_ERR_CUDA. */
+typedef enum {
+    MOE_KERNEL_ROUTE = 0,
+    MOE_KERNEL_GATHER = 1,
+    MOE_KERNEL_STAGE1 = 2, /* group GEMM with w1/w3 + SwiGLU */
+    MOE_KERNEL_STAGE2 = 3, /* group GEMM with w2 + weighted scatter-add */
+    MOE_KERNEL_FINALIZE = 4,
+    MOE_KERNEL_COUNT = 5
+} moe_kernel_id;
+int moe_profile_enable(int on);
+int moe_profile_read(double* ms_total, int* launches, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,189 @@
+"""Routed MoE expert FFN on one B200 (sm_100a): Python binding of libmoe.
+
+The layer (rocketrecap.com "FlyDSL kernels in JAX", paragraph 2 and
+timestamps 5:56 and 8:14): top-k routing, gather of each expert's tokens, group
+GEMM with w1/w3 fused with SwiGLU, group GEMM with w2 fused with the
+routing-weighted scatter back to token order; FP8 (e4m3 with fp32 scales) or
+BF16.
+
+This module only marshals arguments: every step of the layer runs in the CUDA
+kernels of ``libmoe.so`` (built in tree by ``build.py``).  The C entry points
+keep their names (``moe_route``, ``moe_ffn_forward``, ...) and take raw device
+pointers; the ``route``/``ffn_forward``/``prepare_weights`` helpers accept
+torch tensors and pass their pointers and the current CUDA stream.  There is no
+fallback: if the library cannot be loaded, importing this package fails.
+"""
+import ctypes
+import os
+
+__all__ = [
+    "lib", "MOE_OK", "MOE_BF16", "MOE_FP8_E4M3", "WS", "MoeError", "moe_workspace_size", "moe_workspace_region",
+    "moe_prepare_weights", "moe_route", "moe_ffn_forward", "moe_get_status", "moe_set_option", "prepare_weights",
+    "route", "ffn_forward", "workspace", "ws_view", "EXPORTS", "KERNELS", "moe_profile_enable",
+    "moe_profile_read",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_ALIGNMENT",
+                -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA", -6: "MOE_ERR_DEVICE_TIMEOUT",
+                -7: "MOE_ERR_DEVICE_BOUNDS"}
+MOE_BF16 = 0
+MOE_FP8_E4M3 = 1
+OPT_PATH, OPT_SPLITK, OPT_TIMEOUT_MS = 0, 1, 2
+
+# workspace regions (moe_ws_region)
+WS = dict(topk_ids=0, topk_w=1, counts=2, offsets=3, perm=4, inv_perm=5, slot_of=6, xs=7, sx=8, h=9, h_sf=10,
+          out32=11, num_mtiles=12, slot_assign=13, mtile_expert=14)
+
+# every symbol include/moe.h declares
+EXPORTS = ["moe_workspace_size", "moe_prepare_weights", "moe_route", "moe_ffn_forward", "moe_get_status",
+           "moe_workspace_region", "moe_set_option", "moe_profile_enable", "moe_profile_read"]
+KERNELS = ["route", "gather", "stage1_w13_swiglu", "stage2_w2_scatter", "finalize"]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libmoe.so is not built ({LIB_PATH}); run `python mixture_experts_routed_02_b200/build.py`")
+
+lib = ctypes.CDLL(LIB_PATH)
+_P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+lib.moe_workspace_size.restype = _Z
+lib.moe_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I]
+lib.moe_workspace_region.restype = ctypes.c_longlong
+lib.moe_workspace_region.argtypes = [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_Z)]
+lib.moe_prepare_weights.restype = _I
+lib.moe_prepare_weights.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]
+lib.moe_route.restype = _I
+lib.moe_route.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P]
+lib.moe_ffn_forward.restype = _I
+lib.moe_ffn_forward.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P]
+lib.moe_get_status.restype = _I
+lib.moe_get_status.argtypes = [_P]
+lib.moe_set_option.restype = _I
+lib.moe_set_option.argtypes = [_I, _I]
+lib.moe_profile_enable.restype = _I
+lib.moe_profile_enable.argtypes = [_I]
+lib.moe_profile_read.restype = _I
+lib.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I), _I]
+
+# raw entry points, same names as the C ABI
+moe_workspace_size = lib.moe_workspace_size
+moe_prepare_weights = lib.moe_prepare_weights
+moe_route = lib.moe_route
+moe_ffn_forward = lib.moe_ffn_forward
+moe_get_status = lib.moe_get_status
+moe_set_option = lib.moe_set_option
+moe_profile_enable = lib.moe_profile_enable
+
+
+def moe_profile_read(reset=True):
+    """{kernel name: (total ms, launches)} of the calls recorded while profiling was on."""
+    ms = (ctypes.c_double * len(KERNELS))()
+    n = (ctypes.c_int * len(KERNELS))()
+    _check("moe_profile_read", lib.moe_profile_read(ms, n, 1 if reset else 0))
+    return {name: (ms[i], n[i]) for i, name in enumerate(KERNELS)}
+
+
+def moe_workspace_region(T, H, F, E, k, dtype, which):
+    """(byte offset, byte size) of a workspace region (``WS`` names or ints)."""
+    n = ctypes.c_size_t(0)
+    w = WS[which] if isinstance(which, str) else int(which)
+    off = lib.moe_workspace_region(T, H, F, E, k, dtype, w, ctypes.byref(n))
+    if off < 0:
+        raise MoeError("moe_workspace_region", -1)
+    return int(off), int(n.value)
+
+
+# ---------------------------------------------------------------- torch helpers
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != MOE_OK:
+        raise MoeError(fn, rc)
+
+
+def dtype_code(dtype):
+    return MOE_FP8_E4M3 if dtype in ("fp8", MOE_FP8_E4M3) else MOE_BF16
+
+
+def workspace(T, H, F, E, k, dtype, device="cuda"):
+    """Allocate (with torch) a workspace large enough for one layer call."""
+    import torch
+    n = moe_workspace_size(T, H, F, E, k, dtype_code(dtype))
+    if n == 0:
+        raise MoeError("moe_workspace_size", -1)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def ws_view(ws, T, H, F, E, k, dtype, which, torch_dtype=None):
+    """A tensor view of one workspace region (for inspection)."""
+    import torch
+    off, n = moe_workspace_region(T, H, F, E, k, dtype_code(dtype), which)
+    v = ws[off:off + n]
+    return v.view(torch_dtype) if torch_dtype is not None else v
+
+
+def prepare_weights(w1, w3, s1=None, s3=None, stream=None):
+    """One-time preshuffle: returns (w13 [E,2F,H], s13 [E,2F] or None)."""
+    import torch
+    E, F, H = w1.shape
+    fp8 = w1.dtype == torch.float8_e4m3fn
+    w13 = torch.empty(E, 2 * F, H, dtype=w1.dtype, device=w1.device)
+    s13 = torch.empty(E, 2 * F, dtype=torch.float32, device=w1.device) if fp8 else None
+    rc = moe_prepare_weights(_ptr(w1), _ptr(w3), _ptr(s1) if fp8 else None, _ptr(s3) if fp8 else None, _ptr(w13),
+                             _ptr(s13), E, F, H, MOE_FP8_E4M3 if fp8 else MOE_BF16, _stream(stream))
+    _check("moe_prepare_weights", rc)
+    return w13, s13
+
+
+def route(logits, k, stream=None):
+    """Routing alone; returns dict of device tensors (ids, w, counts, offsets, perm, inv_perm)."""
+    import torch
+    T, E = logits.shape
+    dev = logits.device
+    A = T * k
+    out = dict(ids=torch.empty(T, k, dtype=torch.int32, device=dev), w=torch.empty(T, k, dtype=torch.float32, device=dev),
+               counts=torch.empty(E, dtype=torch.int32, device=dev), offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+               perm=torch.empty(max(A, 1), dtype=torch.int32, device=dev),
+               inv_perm=torch.empty(max(A, 1), dtype=torch.int32, device=dev))
+    rc = moe_route(_ptr(logits), T, E, k, _ptr(out["ids"]), _ptr(out["w"]), _ptr(out["counts"]), _ptr(out["offsets"]),
+                   _ptr(out["perm"]), _ptr(out["inv_perm"]), None, 0, _stream(stream))
+    _check("moe_route", rc)
+    out["perm"] = out["perm"][:A]
+    out["inv_perm"] = out["inv_perm"][:A]
+    return out
+
+
+def ffn_forward(x, logits, w13, s13, w2, s2, k, out=None, ws=None, stream=None):
+    """The whole layer; returns the bf16 output [T,H] (and fills ``ws``)."""
+    import torch
+    T, H = x.shape
+    E = logits.shape[1]
+    F = w13.shape[1] // 2
+    fp8 = w13.dtype == torch.float8_e4m3fn
+    dt = MOE_FP8_E4M3 if fp8 else MOE_BF16
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = workspace(T, H, F, E, k, dt, x.device)
+    rc = moe_ffn_forward(_ptr(x), _ptr(logits), _ptr(w13), _ptr(s13) if fp8 else None, _ptr(w2),
+                         _ptr(s2) if fp8 else None, T, H, F, E, k, dt, _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
+    _check("moe_ffn_forward", rc)
+    return out

@@ -1,0 +1,138 @@
+// elementwise.cu -- the memory-bound steps around the two grouped GEMMs:
+//   gather_kernel    gather of each expert's token rows into the expert-padded
+//                    layout (rocketrecap.com "FlyDSL kernels in JAX", paragraph
+//                    2: "gather"), fused with the per-token FP8 quantisation of
+//                    the activations and with zeroing the fp32 combine buffer;
+//   finalize_kernel  fp32 combine buffer -> bf16 output;
+//   interleave_kernel the one-time load-time preshuffle of w1/w3 (timestamp 8:14).
+#include <algorithm>
+
+#include "kernels.cuh"
+
+namespace moe {
+
+// One CTA (128 threads) per row of the padded layout.  Rows past the last
+// tile are skipped; padding rows are written as zeros so the tensor cores see
+// finite values there.
+template <bool kFP8>
+__global__ void __launch_bounds__(128) gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int k,
+                                                     const int* __restrict__ num_mtiles,
+                                                     const int* __restrict__ slot_assign, uint8_t* __restrict__ xs,
+                                                     float* __restrict__ sx_slot, float* __restrict__ out32,
+                                                     int* __restrict__ status) {
+    const int s = blockIdx.x;
+    if (s >= *num_mtiles * kBlockM) return;
+    const int tid = threadIdx.x;
+    const int a = slot_assign[s];
+    const int eb = kFP8 ? 1 : 2;
+    uint8_t* row_out = xs + (size_t)s * H * eb;
+    const int nvec_out = H * eb / 16;
+    if (a < 0 || a / k >= T) {
+        if (a >= 0) record_error(status, MOE_ERR_DEVICE_BOUNDS);
+        for (int i = tid; i < nvec_out; i += 128) reinterpret_cast<uint4*>(row_out)[i] = make_uint4(0, 0, 0, 0);
+        if (kFP8 && tid == 0) sx_slot[s] = 0.f;
+        return;
+    }
+    const int t = a / k;
+    if (a % k == 0) {
+        float4* o = reinterpret_cast<float4*>(out32 + (size_t)t * H);
+        for (int i = tid; i < H / 4; i += 128) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    const int nvec_in = H / 8;  // 8 bf16 per 16-byte vector
+    if (!kFP8) {
+        uint4* dst = reinterpret_cast<uint4*>(row_out);
+        for (int i = tid; i < nvec_in; i += 128) dst[i] = __ldg(src + i);
+        return;
+    }
+    // FP8: absmax over the row, then x / sx rounded to e4m3 (nearest even, saturating)
+    __shared__ float warp_max[4];
+    float amax = 0.f;
+    for (int i = tid; i < nvec_in; i += 128) {
+        const uint4 v = __ldg(src + i);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p[j]);
+            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+    if ((tid & 31) == 0) warp_max[tid >> 5] = amax;
+    __syncthreads();
+    amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
+    const float sx = (amax == 0.f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+    if (tid == 0) sx_slot[s] = sx;
+    uint2* dst = reinterpret_cast<uint2*>(row_out);
+    for (int i = tid; i < nvec_in; i += 128) {
+        const uint4 v = __ldg(src + i);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+        uint32_t packed[2];
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+            const float2 f0 = __bfloat1622float2(p[j]);
+            const float2 f1 = __bfloat1622float2(p[j + 1]);
+            const __nv_fp8x2_storage_t q0 =
+                __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f0.x, sx), __fdiv_rn(f0.y, sx)), __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8x2_storage_t q1 =
+                __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f1.x, sx), __fdiv_rn(f1.y, sx)), __NV_SATFINITE, __NV_E4M3);
+            packed[j / 2] = (uint32_t)q0 | ((uint32_t)q1 << 16);
+        }
+        dst[i] = make_uint2(packed[0], packed[1]);
+    }
+}
+
+cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, int S_max, const int* num_mtiles,
+                          const int* slot_assign, uint8_t* xs, float* sx_slot, float* out32, int* status,
+                          cudaStream_t stream) {
+    if (fp8)
+        gather_kernel<true><<<S_max, 128, 0, stream>>>(x, T, H, k, num_mtiles, slot_assign, xs, sx_slot, out32, status);
+    else
+        gather_kernel<false><<<S_max, 128, 0, stream>>>(x, T, H, k, num_mtiles, slot_assign, xs, sx_slot, out32, status);
+    return cudaGetLastError();
+}
+
+// out = bf16(out32), round to nearest even; n is a multiple of 8.
+__global__ void finalize_kernel(const float* __restrict__ out32, __nv_bfloat16* __restrict__ out, size_t n) {
+    const size_t nv = n / 8;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nv; i += (size_t)gridDim.x * blockDim.x) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(out32) + 2 * i);
+        const float4 b = __ldg(reinterpret_cast<const float4*>(out32) + 2 * i + 1);
+        __nv_bfloat162 r[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
+                               __floats2bfloat162_rn(b.x, b.y), __floats2bfloat162_rn(b.z, b.w)};
+        reinterpret_cast<uint4*>(out)[i] = *reinterpret_cast<uint4*>(r);
+    }
+}
+
+// w13[e][64b + i] = w1[e][32b + i], w13[e][64b + 32 + i] = w3[e][32b + i]; one
+// CTA per destination row.  row_bytes % 16 == 0.
+__global__ void interleave_kernel(const uint8_t* __restrict__ w1, const uint8_t* __restrict__ w3,
+                                  const float* __restrict__ s1, const float* __restrict__ s3, uint8_t* __restrict__ w13,
+                                  float* __restrict__ s13, int F, int row_bytes) {
+    const int e = blockIdx.y;
+    const int r = blockIdx.x;  // destination row in [0, 2F)
+    const int b = r / 64, i = r % 64;
+    const bool up = i >= 32;
+    const int src_row = 32 * b + (i & 31);
+    const uint8_t* src = (up ? w3 : w1) + ((size_t)e * F + src_row) * row_bytes;
+    uint8_t* dst = w13 + ((size_t)e * 2 * F + r) * row_bytes;
+    for (int v = threadIdx.x; v < row_bytes / 16; v += blockDim.x)
+        reinterpret_cast<uint4*>(dst)[v] = __ldg(reinterpret_cast<const uint4*>(src) + v);
+    if (s13 && threadIdx.x == 0) s13[(size_t)e * 2 * F + r] = (up ? s3 : s1)[(size_t)e * F + src_row];
+}
+
+cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream) {
+    const int blocks = (int)std::min<size_t>((n / 8 + 255) / 256, (size_t)num_sms * 8);
+    if (blocks == 0) return cudaSuccess;
+    finalize_kernel<<<blocks, 256, 0, stream>>>(out32, out, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_interleave(const uint8_t* w1, const uint8_t* w3, const float* s1, const float* s3, uint8_t* w13,
+                              float* s13, int E, int F, int row_bytes, cudaStream_t stream) {
+    interleave_kernel<<<dim3(2 * F, E), 128, 0, stream>>>(w1, w3, s1, s3, w13, s13, F, row_bytes);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,387 @@
+// gemm.cu -- persistent grouped GEMM on the sm_100a tensor cores (tcgen05 +
+// TMEM + TMA) for both stages of the routed expert FFN (rocketrecap.com
+// "FlyDSL kernels in JAX", paragraph 2 and timestamp 5:56: group GEMM with
+// w1/w3 fused with SwiGLU, then group GEMM with w2 fused with the scatter).
+//
+// Row space: the expert-padded layout built by the router -- expert e owns
+// whole 128-row tiles, so a tile never straddles two experts and its weight
+// operand is one expert's matrix.  A tile is (m-tile, n-tile, K split).
+//
+// Stage 1: D[128 x BN] = Xs[128 rows, H] * W13_e[BN rows, H]^T.  W13 holds w1
+//   and w3 rows interleaved in blocks of 32, so accumulator columns [64g, 64g+32)
+//   are gate channels and [64g+32, 64g+64) the matching up channels.  Epilogue:
+//   (FP8: scale by sx[row] * s13[col]) -> h = silu(g) * u -> bf16 -> (FP8:
+//   e4m3 with one power-of-two scale per 32 channels) -> h.
+// Stage 2: D[128 x BN] = H[128 rows, F] * W2_e[BN rows, F]^T; FP8 uses the
+//   block-scaled MMA with h's per-32 scales (w2's are 1) and applies s2 in the
+//   epilogue.  Epilogue: scale by the routing weight, fp32 atomic add into the
+//   token's row of the combine buffer (which also makes K splits free).
+//
+// Warp roles (192 threads): warp 0 lane 0 issues TMA loads into an NST-deep
+// shared-memory ring; warp 1 owns TMEM and lane 0 issues the MMAs; warps 2..5
+// drain the two TMEM accumulators (double buffered, so the epilogue of one
+// tile overlaps the main loop of the next).
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+template <int STAGE, bool FP8, int BN, int NST>
+struct Cfg {
+    static constexpr bool MX = (STAGE == 2) && FP8;
+    static constexpr int A_BYTES = kBlockM * 128;
+    static constexpr int B_BYTES = BN * 128;
+    static constexpr int SF_BYTES = MX ? 512 : 0;
+    static constexpr int TX_BYTES = A_BYTES + B_BYTES + SF_BYTES;
+    static constexpr int KE = FP8 ? 128 : 64;  // K elements per 128-byte K tile
+    static constexpr int SFA_COL = 2 * BN;
+    static constexpr int SFB_COL = SFA_COL + 4 * NST;
+    static constexpr int COLS_USED = MX ? SFB_COL + 8 : 2 * BN;
+    static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
+                                   : COLS_USED <= 256 ? 256 : 512;
+    static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
+    static_assert(BN % 64 == 0 && BN <= 256, "BN");
+    // shared memory: A ring, B ring, SF ring, constant B scales, barriers
+    static constexpr int OFF_B = NST * A_BYTES;
+    static constexpr int OFF_SF = OFF_B + NST * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SF + NST * SF_BYTES;
+    static constexpr int OFF_BAR = OFF_SFB + (MX ? 512 : 0);
+    static constexpr int NUM_BARS = 2 * NST + 5;
+    static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;  // + alignment slack
+    static constexpr uint32_t IDESC = FP8 ? idesc_e4m3(kBlockM, BN) : idesc_bf16(kBlockM, BN);
+};
+
+__device__ __forceinline__ void decode_tile(int tile, int num_mt, int n_tiles, int& m, int& n, int& split) {
+    m = tile % num_mt;
+    const int r = tile / num_mt;
+    n = r % n_tiles;
+    split = r / n_tiles;
+}
+
+}  // namespace
+
+template <int STAGE, bool FP8, int BN, int NST>
+__global__ void __launch_bounds__(192, 1)
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmArgs args) {
+    using C = Cfg<STAGE, FP8, BN, NST>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + NST;
+    uint64_t* tfull = bars + 2 * NST;
+    uint64_t* tempty = bars + 2 * NST + 2;
+    uint64_t* drain = bars + 2 * NST + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t limit = args.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NST; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (C::MX && warp >= 2) {
+        // constant UE8M0 scale 2^0 for every row of B (w2 carries fp32 per-channel scales instead)
+        reinterpret_cast<uint32_t*>(smem + C::OFF_SFB)[threadIdx.x - 64] = 0x7F7F7F7Fu;
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int num_mt = *args.num_mtiles;
+    const int total = num_mt * args.n_tiles * args.splits;
+    const int kps = args.k_tiles / args.splits;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_last();
+            const uint64_t pol_b = policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                int m, n, split;
+                decode_tile(tile, num_mt, args.n_tiles, m, n, split);
+                const int e = args.mtile_expert[m];
+                const int brow = e * args.rows_b + n * BN;
+                for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, limit, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+                    tma_load_2d(smem + stage * C::A_BYTES, &tmA, &full[stage], kt * C::KE, m * kBlockM, pol_a);
+                    tma_load_2d(smem + C::OFF_B + stage * C::B_BYTES, &tmB, &full[stage], kt * C::KE, brow, pol_b);
+                    if constexpr (C::MX)
+                        bulk_load(smem + C::OFF_SF + stage * C::SF_BYTES,
+                                  args.a_sf + ((size_t)m * args.f_tiles + kt) * 512, 512, &full[stage]);
+                    ++issued;
+                    if (++stage == NST) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            // do not leave while copies into this CTA's shared memory are in
+            // flight (this wait ignores the abort flag but keeps its time limit)
+            volatile int keep_waiting = 0;
+            for (int i = 1; i <= min(issued, NST); ++i) {
+                int s = stage - i;
+                uint32_t ph = phase;
+                if (s < 0) {
+                    s += NST;
+                    ph ^= 1;
+                }
+                mbar_wait(&full[s], ph, &keep_waiting, limit, args.status);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            if constexpr (C::MX) {
+                for (int c = 0; c < 8; c += 4) tmem_cp_32x128b_x4(tmem_base + C::SFB_COL + c, sdesc_sf(smem_u32(smem + C::OFF_SFB)));
+            }
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, limit, args.status)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                for (int kk = 0; kk < kps; ++kk) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag, limit, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + stage * C::A_BYTES);
+                    const uint32_t b_addr = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+                    if constexpr (C::MX)
+                        tmem_cp_32x128b_x4(tmem_base + C::SFA_COL + 4 * stage,
+                                           sdesc_sf(smem_u32(smem + C::OFF_SF + stage * C::SF_BYTES)));
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = sdesc_sw128(a_addr + ks * 32);
+                        const uint64_t bd = sdesc_sw128(b_addr + ks * 32);
+                        const uint32_t accum = (kk > 0 || ks > 0) ? 1u : 0u;
+                        if constexpr (C::MX)
+                            mma_mxfp8(d_tmem, ad, bd, idesc_mxe4m3(kBlockM, BN, ks, ks),
+                                      tmem_base + C::SFA_COL + 4 * stage, tmem_base + C::SFB_COL, accum);
+                        else if constexpr (FP8)
+                            mma_fp8(d_tmem, ad, bd, C::IDESC, accum);
+                        else
+                            mma_bf16(d_tmem, ad, bd, C::IDESC, accum);
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == NST) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&tfull[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1;
+                }
+            }
+            // every MMA issued by this thread has finished before TMEM is released
+            volatile int keep_waiting = 0;
+            tc_commit(drain);
+            mbar_wait(drain, 0, &keep_waiting, limit, args.status);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- epilogue warps 2..5
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            int m, n, split;
+            decode_tile(tile, num_mt, args.n_tiles, m, n, split);
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, limit, args.status)) break;
+            tc_fence_after();
+            const int e = args.mtile_expert[m];
+            const int slot = m * kBlockM + row;
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+            if constexpr (STAGE == 1) {
+                const float sxv = FP8 ? args.row_scale[slot] : 1.0f;
+#pragma unroll 1
+                for (int g = 0; g < BN / 64; ++g) {
+                    uint32_t rg[32], ru[32];
+                    tmem_ld_32cols(tbase + g * 64, rg);
+                    tmem_ld_32cols(tbase + g * 64 + 32, ru);
+                    tmem_ld_wait();
+                    const int hcol = n * (BN / 2) + g * 32;
+                    float hv[32];
+                    if constexpr (FP8) {
+                        const float* cs = args.col_scale + (size_t)e * args.rows_b + n * BN + g * 64;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float gv = __uint_as_float(rg[i]) * sxv * __ldg(cs + i);
+                            const float uv = __uint_as_float(ru[i]) * sxv * __ldg(cs + 32 + i);
+                            hv[i] = __bfloat162float(__float2bfloat16_rn(gv / (1.0f + __expf(-gv)) * uv));
+                        }
+                        float amax = 0.f;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(hv[i]));
+                        int ex = 0;
+                        if (amax > 0.f) {
+                            const uint32_t b = __float_as_uint(__fdiv_rn(amax, 448.0f));
+                            const int e8 = (int)((b >> 23) & 0xFF);
+                            const uint32_t man = b & 0x7FFFFFu;
+                            ex = (e8 == 0) ? ((man > 0x400000u) ? -126 : -127) : e8 - 127 + (man != 0u);
+                            ex = max(-127, min(127, ex));
+                        }
+                        const float inv = ldexpf(1.0f, -ex);
+                        uint32_t packed[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+                                make_float2(hv[4 * i] * inv, hv[4 * i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+                            const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+                                make_float2(hv[4 * i + 2] * inv, hv[4 * i + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+                            packed[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) +
+                                                              (size_t)slot * args.out_ld + hcol);
+                        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                        args.out_sf[((size_t)m * args.f_tiles + (hcol >> 7)) * 512 + (row & 31) * 16 + (row >> 5) * 4 +
+                                    ((hcol >> 5) & 3)] = (uint8_t)(ex + 127);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float gv = __uint_as_float(rg[i]);
+                            const float uv = __uint_as_float(ru[i]);
+                            hv[i] = gv / (1.0f + __expf(-gv)) * uv;
+                        }
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            __nv_bfloat162 p = __floats2bfloat162_rn(hv[2 * i], hv[2 * i + 1]);
+                            packed[i] = *reinterpret_cast<uint32_t*>(&p);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) +
+                                                              (size_t)slot * args.out_ld + hcol);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    }
+                }
+            } else {
+                const int a = args.slot_assign[slot];
+                int t = (a >= 0) ? a / args.topk : -1;
+                if (t >= args.T) {
+                    record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
+                    t = -1;
+                }
+                const float wgt = (t >= 0) ? args.topk_w[a] : 0.f;
+                float* orow = static_cast<float*>(args.out) + (size_t)(t >= 0 ? t : 0) * args.out_ld;
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32cols(tbase + c0, r);
+                    tmem_ld_wait();
+                    if (t >= 0) {
+                        const int col = n * BN + c0;
+                        const float* cs = FP8 ? args.col_scale + (size_t)e * args.rows_b + col : nullptr;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4) {
+                            float4 v;
+                            v.x = __uint_as_float(r[i]) * wgt;
+                            v.y = __uint_as_float(r[i + 1]) * wgt;
+                            v.z = __uint_as_float(r[i + 2]) * wgt;
+                            v.w = __uint_as_float(r[i + 3]) * wgt;
+                            if constexpr (FP8) {
+                                const float4 s = __ldg(reinterpret_cast<const float4*>(cs + i));
+                                v.x *= s.x;
+                                v.y *= s.y;
+                                v.z *= s.z;
+                                v.w *= s.w;
+                            }
+                            atomicAdd(reinterpret_cast<float4*>(orow + col + i), v);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1;
+            }
+        }
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+namespace {
+
+template <int STAGE, bool FP8, int BN, int NST>
+cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, int grid,
+                       cudaStream_t stream) {
+    using C = Cfg<STAGE, FP8, BN, NST>;
+    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, 192, C::SMEM_BYTES, stream>>>(ta, tb, args);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int gemm_block_n(int stage, bool fp8, int cfg) {
+    if (stage == 2 && fp8) return 128;
+    return cfg == 0 ? 256 : 128;
+}
+
+cudaError_t launch_gemm(int stage, bool fp8, int cfg, const CUtensorMap& ta, const CUtensorMap& tb,
+                        const GemmArgs& args, int grid, cudaStream_t stream) {
+    if (stage == 1) {
+        if (fp8) return cfg == 0 ? launch_one<1, true, 256, 4>(ta, tb, args, grid, stream)
+                                 : launch_one<1, true, 128, 6>(ta, tb, args, grid, stream);
+        return cfg == 0 ? launch_one<1, false, 256, 4>(ta, tb, args, grid, stream)
+                        : launch_one<1, false, 128, 6>(ta, tb, args, grid, stream);
+    }
+    if (fp8) return launch_one<2, true, 128, 6>(ta, tb, args, grid, stream);
+    return cfg == 0 ? launch_one<2, false, 256, 4>(ta, tb, args, grid, stream)
+                    : launch_one<2, false, 128, 6>(ta, tb, args, grid, stream);
+}
+
+}  // namespace moe

@@ -1,0 +1,72 @@
+// kernels.cuh -- shared constants, argument structs and host-side launchers of
+// the library's kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int kMaxExperts = 64;
+constexpr int kMaxTopK = 8;
+constexpr int kBlockM = 128;  // rows per tile of the expert-padded layout
+
+// Where the router writes.  slot_of / slot_assign / mtile_expert / num_mtiles
+// may be null (routing alone); otherwise they describe the expert-padded row
+// layout: expert e owns rows [128*mt_start[e], 128*mt_start[e+1]), its n_e
+// assignments first in sorted order, then padding rows marked -1.
+struct RouteOutputs {
+    int32_t* topk_ids;
+    float* topk_w;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* perm;
+    int32_t* inv_perm;
+    int32_t* slot_of;       // [A] assignment -> padded row
+    int32_t* slot_assign;   // [S_max] padded row -> assignment or -1
+    int32_t* mtile_expert;  // [MT_max] tile -> expert
+    int32_t* num_mtiles;    // [1]
+};
+
+// Host launchers (each defined next to its kernel).
+cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream);
+cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, int S_max, const int* num_mtiles,
+                          const int* slot_assign, uint8_t* xs, float* sx_slot, float* out32, int* status,
+                          cudaStream_t stream);
+cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream);
+cudaError_t launch_interleave(const uint8_t* w1, const uint8_t* w3, const float* s1, const float* s3, uint8_t* w13,
+                              float* s13, int E, int F, int row_bytes, cudaStream_t stream);
+
+// Arguments of the grouped GEMM (both stages).
+struct GemmArgs {
+    const int* num_mtiles;
+    const int* mtile_expert;
+    const int* slot_assign;
+    const float* row_scale;   // stage 1, FP8: per-row activation scale [S]
+    const float* col_scale;   // FP8: s13 [E*2F] (stage 1) or s2 [E*H] (stage 2)
+    const float* topk_w;      // stage 2: routing weight per assignment
+    const uint8_t* a_sf;      // stage 2, FP8: UE8M0 scales of h, tiled
+    void* out;                // stage 1: h [S, F]; stage 2: out32 [T, H]
+    uint8_t* out_sf;          // stage 1, FP8: UE8M0 scales of h, tiled
+    int rows_b;               // rows of B per expert: 2F (stage 1) or H (stage 2)
+    int n_tiles;              // rows_b / BN
+    int k_tiles;              // K / (128 bytes of K)
+    int splits;               // K splits (stage 2)
+    int out_ld;               // F (stage 1) or H (stage 2)
+    int f_tiles;              // F / 128: scale tiles per row block of h
+    int topk;
+    int T;
+    unsigned long long timeout_ns;
+    int* status;              // device status word
+};
+
+// Host launchers of the tcgen05 grouped GEMM; defined in gemm.cu.
+// cfg: 0 = throughput tiles (BN=256), 1 = weight-streaming tiles (BN=128).
+cudaError_t launch_gemm(int stage, bool fp8, int cfg, const CUtensorMap& ta, const CUtensorMap& tb,
+                        const GemmArgs& args, int grid, cudaStream_t stream);
+int gemm_block_n(int stage, bool fp8, int cfg);
+
+}  // namespace moe

@@ -1,0 +1,415 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: argument validation,
+// workspace layout, TMA tensor maps and the launch sequence of one layer.
+//
+// One call of moe_ffn_forward enqueues, on the caller's stream:
+//   route_kernel   top-k, softmax, histogram, scan, permutation, padded layout
+//   gather_kernel  gather (+ per-token e4m3 quantisation) and zeroing of out32
+//   stage-1 GEMM   gather-GEMM with w1/w3 + SwiGLU (+ MX quantisation of h)
+//   stage-2 GEMM   GEMM with w2 + routing-weighted scatter-add into out32
+//   finalize       out32 -> bf16 out
+// (rocketrecap.com "FlyDSL kernels in JAX", paragraph 2 and timestamp 5:56.)
+#include <algorithm>
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "kernels.cuh"
+
+namespace moe {
+
+__device__ int g_status_word = 0;
+
+namespace {
+
+std::atomic<int> g_opt_path{0};
+std::atomic<int> g_opt_splitk{0};
+std::atomic<int> g_opt_timeout_ms{2000};
+
+// ---------------------------------------------------------------- profiling
+
+struct ProfRecord {
+    int kernel;
+    cudaEvent_t start, stop;
+};
+std::atomic<int> g_prof_on{0};
+std::mutex g_prof_mutex;
+std::vector<ProfRecord> g_prof_records;
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+    if (!g_prof_pool.empty()) {
+        cudaEvent_t e = g_prof_pool.back();
+        g_prof_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Records events around one kernel launch when profiling is on.
+struct ProfScope {
+    int kernel;
+    cudaStream_t stream;
+    cudaEvent_t start = nullptr;
+    ProfScope(int k, cudaStream_t s) : kernel(k), stream(s) {
+        if (!g_prof_on.load()) return;
+        std::lock_guard<std::mutex> lock(g_prof_mutex);
+        start = prof_event();
+        if (start) cudaEventRecord(start, stream);
+    }
+    ~ProfScope() {
+        if (!start) return;
+        std::lock_guard<std::mutex> lock(g_prof_mutex);
+        cudaEvent_t stop = prof_event();
+        if (!stop) return;
+        cudaEventRecord(stop, stream);
+        g_prof_records.push_back({kernel, start, stop});
+    }
+};
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+int g_num_sms[kMaxDevices] = {0};
+std::mutex g_dev_mutex;
+
+// Address of this device's status word and its SM count (looked up once per device).
+int device_info(int** status, int* num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return MOE_ERR_CUDA;
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+        g_status_ptr[dev] = static_cast<int*>(p);
+        g_num_sms[dev] = sms;
+    }
+    *status = g_status_ptr[dev];
+    *num_sms = g_num_sms[dev];
+    return MOE_OK;
+}
+
+// ---------------------------------------------------------------- workspace
+
+constexpr int kRegions = 15;
+
+struct Layout {
+    size_t off[kRegions];
+    size_t size[kRegions];
+    size_t total;
+    int A, MT_max, S_max;
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool dims_ok(int T, int H, int F, int E, int k, int dtype) {
+    return T >= 0 && H > 0 && F > 0 && E >= 1 && E <= kMaxExperts && k >= 1 && k <= E && k <= kMaxTopK &&
+           (dtype == MOE_BF16 || dtype == MOE_FP8_E4M3);
+}
+
+Layout make_layout(int T, int H, int F, int E, int k, int dtype) {
+    Layout L{};
+    const size_t A = (size_t)T * k;
+    const size_t eb = (dtype == MOE_FP8_E4M3) ? 1 : 2;
+    L.A = (int)A;
+    L.MT_max = (int)((A + kBlockM - 1) / kBlockM) + E;  // sum over experts of ceil(n_e / 128)
+    L.S_max = L.MT_max * kBlockM;
+    const size_t S = L.S_max;
+    size_t sz[kRegions] = {};
+    sz[MOE_WS_TOPK_IDS] = 4 * A;
+    sz[MOE_WS_TOPK_W] = 4 * A;
+    sz[MOE_WS_COUNTS] = 4 * (size_t)E;
+    sz[MOE_WS_OFFSETS] = 4 * (size_t)(E + 1);
+    sz[MOE_WS_PERM] = 4 * A;
+    sz[MOE_WS_INV_PERM] = 4 * A;
+    sz[MOE_WS_SLOT_OF] = 4 * A;
+    sz[MOE_WS_XS] = S * H * eb;
+    sz[MOE_WS_SX] = 4 * S;
+    sz[MOE_WS_H] = S * F * eb;
+    sz[MOE_WS_H_SF] = (dtype == MOE_FP8_E4M3) ? (size_t)L.MT_max * (F / 128) * 512 : 0;
+    sz[MOE_WS_OUT32] = 4 * (size_t)T * H;
+    sz[MOE_WS_NUM_MTILES] = 4;
+    sz[MOE_WS_SLOT_ASSIGN] = 4 * S;
+    sz[MOE_WS_MTILE_EXPERT] = 4 * (size_t)L.MT_max;
+    size_t off = 0;
+    for (int r = 0; r < kRegions; ++r) {
+        L.off[r] = off;
+        L.size[r] = sz[r];
+        off = align_up(off + sz[r], 1024);
+    }
+    L.total = off;
+    return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// 2-D row-major matrix [rows, cols] of elements of `eb` bytes; box = 128 bytes
+// of K by box_rows rows, 128-byte swizzle (matches the MMA descriptors).
+bool make_map(CUtensorMap* map, const void* base, size_t rows, size_t cols, int eb, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * eb};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / eb), (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// K splits of the second GEMM: enough work units for every SM when the layer
+// is small (decode), 1 otherwise.  Must divide F/128.
+int choose_splits(int mt_est, int n_tiles, int k_tiles, int num_sms) {
+    const int forced = g_opt_splitk.load();
+    if (forced > 0) return forced;
+    for (int s = 1; s <= k_tiles / 4; ++s) {
+        if (k_tiles % s) continue;
+        if ((long)mt_est * n_tiles * s >= 6L * num_sms) return s;
+    }
+    return 1;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(int T, int H, int F, int E, int k, int dtype) {
+    if (!dims_ok(T, H, F, E, k, dtype)) return 0;
+    return make_layout(T, H, F, E, k, dtype).total;
+}
+
+long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int which, size_t* bytes) {
+    if (!dims_ok(T, H, F, E, k, dtype) || which < 0 || which >= kRegions) return -1;
+    const Layout L = make_layout(T, H, F, E, k, dtype);
+    if (bytes) *bytes = L.size[which];
+    return (long long)L.off[which];
+}
+
+int moe_set_option(int option, int value) {
+    switch (option) {
+        case MOE_OPT_PATH:
+            if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+            return g_opt_path.exchange(value);
+        case MOE_OPT_SPLITK:
+            if (value < 0) return MOE_ERR_INVALID_ARG;
+            return g_opt_splitk.exchange(value);
+        case MOE_OPT_TIMEOUT_MS:
+            if (value < 1) return MOE_ERR_INVALID_ARG;
+            return g_opt_timeout_ms.exchange(value);
+        default:
+            return MOE_ERR_INVALID_ARG;
+    }
+}
+
+int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const float* s3, void* w13_out,
+                        float* s13_out, int E, int F, int H, int dtype, void* stream) {
+    if (!w1 || !w3 || !w13_out || E < 1 || E > kMaxExperts || F <= 0 || H <= 0) return MOE_ERR_INVALID_ARG;
+    if (dtype != MOE_BF16 && dtype != MOE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+    const bool fp8 = dtype == MOE_FP8_E4M3;
+    if (fp8 && (!s1 || !s3 || !s13_out)) return MOE_ERR_INVALID_ARG;
+    if (F % 128 || H % 128) return MOE_ERR_UNSUPPORTED;
+    if (!aligned16(w1) || !aligned16(w3) || !aligned16(w13_out)) return MOE_ERR_ALIGNMENT;
+    const int eb = fp8 ? 1 : 2;
+    return launch_status(launch_interleave(static_cast<const uint8_t*>(w1), static_cast<const uint8_t*>(w3),
+                                           fp8 ? s1 : nullptr, fp8 ? s3 : nullptr, static_cast<uint8_t*>(w13_out),
+                                           fp8 ? s13_out : nullptr, E, F, H * eb, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w, int32_t* counts,
+              int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > E || k > kMaxTopK) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !topk_ids || !topk_w || !perm || !inv_perm)) return MOE_ERR_INVALID_ARG;
+    if ((long long)T * k > 262144) return MOE_ERR_UNSUPPORTED;
+    RouteOutputs o{topk_ids, topk_w, counts, offsets, perm, inv_perm, nullptr, nullptr, nullptr, nullptr};
+    return launch_status(launch_route(logits, T, E, k, o, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_ffn_forward(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
+                    const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
+                    size_t ws_bytes, void* stream) {
+    if (!dims_ok(T, H, F, E, k, dtype)) return MOE_ERR_INVALID_ARG;
+    const bool fp8 = dtype == MOE_FP8_E4M3;
+    if (!w13 || !w2 || !ws || (fp8 && (!s13 || !s2))) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !logits || !out)) return MOE_ERR_INVALID_ARG;
+    if (H % 128 || F % 128) return MOE_ERR_UNSUPPORTED;
+    if ((long long)T * k > 262144) return MOE_ERR_UNSUPPORTED;
+    const void* ptrs[] = {x, logits, w13, s13, w2, s2, out, ws};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+    const Layout L = make_layout(T, H, F, E, k, dtype);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (T == 0) return MOE_OK;
+
+    int* status = nullptr;
+    int num_sms = 0;
+    if (device_info(&status, &num_sms) != MOE_OK) return MOE_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    auto reg = [&](int r) { return w + L.off[r]; };
+    const int eb = fp8 ? 1 : 2;
+
+    // weight-streaming tiles when experts see few rows on average
+    int cfg = g_opt_path.load();
+    cfg = (cfg == 0) ? ((L.A <= 64 * E) ? 1 : 0) : cfg - 1;
+    const int bn1 = gemm_block_n(1, fp8, cfg);
+    const int bn2 = gemm_block_n(2, fp8, cfg);
+    if ((2 * F) % bn1 || H % bn2) return MOE_ERR_UNSUPPORTED;
+
+    CUtensorMap ta1, tb1, ta2, tb2;
+    if (!make_map(&ta1, reg(MOE_WS_XS), L.S_max, H, eb, kBlockM) ||
+        !make_map(&tb1, w13, (size_t)E * 2 * F, H, eb, bn1) ||
+        !make_map(&ta2, reg(MOE_WS_H), L.S_max, F, eb, kBlockM) ||
+        !make_map(&tb2, w2, (size_t)E * H, F, eb, bn2))
+        return MOE_ERR_CUDA;
+
+    // 1. routing and the expert-padded layout
+    RouteOutputs o{reinterpret_cast<int32_t*>(reg(MOE_WS_TOPK_IDS)), reinterpret_cast<float*>(reg(MOE_WS_TOPK_W)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_COUNTS)), reinterpret_cast<int32_t*>(reg(MOE_WS_OFFSETS)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_PERM)), reinterpret_cast<int32_t*>(reg(MOE_WS_INV_PERM)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_SLOT_OF)), reinterpret_cast<int32_t*>(reg(MOE_WS_SLOT_ASSIGN)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_MTILE_EXPERT)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_NUM_MTILES))};
+    {
+        ProfScope ps(MOE_KERNEL_ROUTE, st);
+        if (launch_route(logits, T, E, k, o, st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+
+    // 2. gather (+ quantise) and zero the combine buffer
+    const int* num_mt = o.num_mtiles;
+    float* out32 = reinterpret_cast<float*>(reg(MOE_WS_OUT32));
+    float* sx = reinterpret_cast<float*>(reg(MOE_WS_SX));
+    {
+        ProfScope ps(MOE_KERNEL_GATHER, st);
+        if (launch_gather(fp8, static_cast<const __nv_bfloat16*>(x), T, H, k, L.S_max, num_mt, o.slot_assign,
+                          reg(MOE_WS_XS), sx, out32, status, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+
+    const unsigned long long timeout_ns = (unsigned long long)g_opt_timeout_ms.load() * 1000000ull;
+
+    // 3. stage 1: gather-GEMM with w1/w3, SwiGLU epilogue
+    GemmArgs g1{};
+    g1.num_mtiles = num_mt;
+    g1.mtile_expert = o.mtile_expert;
+    g1.slot_assign = o.slot_assign;
+    g1.row_scale = fp8 ? sx : nullptr;
+    g1.col_scale = fp8 ? s13 : nullptr;
+    g1.out = reg(MOE_WS_H);
+    g1.out_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;
+    g1.rows_b = 2 * F;
+    g1.n_tiles = 2 * F / bn1;
+    g1.k_tiles = H * eb / 128;
+    g1.splits = 1;
+    g1.out_ld = F;
+    g1.f_tiles = F / 128;
+    g1.topk = k;
+    g1.T = T;
+    g1.timeout_ns = timeout_ns;
+    g1.status = status;
+    const long tiles1 = (long)L.MT_max * g1.n_tiles;
+    {
+        ProfScope ps(MOE_KERNEL_STAGE1, st);
+        if (launch_gemm(1, fp8, cfg, ta1, tb1, g1, (int)std::min<long>(tiles1, num_sms), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+
+    // 4. stage 2: GEMM with w2, weighted scatter-add epilogue
+    GemmArgs g2 = g1;
+    g2.row_scale = nullptr;
+    g2.col_scale = fp8 ? s2 : nullptr;
+    g2.topk_w = o.topk_w;
+    g2.a_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;
+    g2.out = out32;
+    g2.out_sf = nullptr;
+    g2.rows_b = H;
+    g2.n_tiles = H / bn2;
+    g2.k_tiles = F * eb / 128;
+    const int mt_est = std::min(L.MT_max, (L.A + kBlockM - 1) / kBlockM + std::min(E, L.A));
+    g2.splits = choose_splits(mt_est, g2.n_tiles, g2.k_tiles, num_sms);
+    if (g2.splits < 1 || g2.k_tiles % g2.splits) return MOE_ERR_UNSUPPORTED;
+    g2.out_ld = H;
+    const long tiles2 = (long)L.MT_max * g2.n_tiles * g2.splits;
+    {
+        ProfScope ps(MOE_KERNEL_STAGE2, st);
+        if (launch_gemm(2, fp8, cfg, ta2, tb2, g2, (int)std::min<long>(tiles2, num_sms), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+
+    // 5. fp32 -> bf16
+    ProfScope ps(MOE_KERNEL_FINALIZE, st);
+    return launch_status(launch_finalize(out32, static_cast<__nv_bfloat16*>(out), (size_t)T * H, num_sms, st));
+}
+
+int moe_profile_enable(int on) { return g_prof_on.exchange(on ? 1 : 0); }
+
+int moe_profile_read(double* ms_total, int* launches, int reset) {
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
+    if (ms_total)
+        for (int i = 0; i < MOE_KERNEL_COUNT; ++i) ms_total[i] = 0.0;
+    if (launches)
+        for (int i = 0; i < MOE_KERNEL_COUNT; ++i) launches[i] = 0;
+    int rc = MOE_OK;
+    for (const ProfRecord& r : g_prof_records) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+            rc = MOE_ERR_CUDA;
+            continue;
+        }
+        if (ms_total) ms_total[r.kernel] += ms;
+        if (launches) launches[r.kernel] += 1;
+    }
+    if (reset) {
+        for (const ProfRecord& r : g_prof_records) {
+            g_prof_pool.push_back(r.start);
+            g_prof_pool.push_back(r.stop);
+        }
+        g_prof_records.clear();
+    }
+    return rc;
+}
+
+int moe_get_status(void* stream) {
+    int* status = nullptr;
+    int num_sms = 0;
+    if (device_info(&status, &num_sms) != MOE_OK) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,92 @@
+"""The C ABI on the host (no GPU needed): the library loads, exports every
+entry point include/moe.h declares, and rejects bad arguments before touching
+the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:size_t|int|long long)\s+(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import mixture_experts_routed_02_b200 as m
+    return m
+
+
+def test_exports_every_declared_symbol(moe):
+    declared = _declared_functions()
+    assert set(declared) >= {"moe_route", "moe_ffn_forward", "moe_workspace_size", "moe_prepare_weights",
+                             "moe_get_status"}
+    raw = ctypes.CDLL(moe.LIB_PATH)
+    for name in declared:
+        assert hasattr(raw, name), name
+    assert sorted(moe.EXPORTS) == declared
+
+
+def test_workspace_layout(moe):
+    for (T, H, F, E, k, dt) in [(64, 256, 512, 8, 2, 0), (16, 4096, 14336, 8, 2, 1), (4096, 4096, 14336, 8, 2, 1),
+                                (8192, 4096, 14336, 8, 2, 0), (1, 128, 128, 1, 1, 1)]:
+        total = moe.moe_workspace_size(T, H, F, E, k, dt)
+        assert total > 0
+        regions = sorted(moe.moe_workspace_region(T, H, F, E, k, dt, w) for w in moe.WS)
+        end = 0
+        for off, n in regions:
+            assert off % 1024 == 0 and off >= end
+            end = off + n
+        assert end <= total
+    # assignment-sized regions grow with T
+    assert moe.moe_workspace_size(2000, 256, 512, 8, 2, 1) > moe.moe_workspace_size(1000, 256, 512, 8, 2, 1)
+
+
+@pytest.mark.parametrize("args", [
+    (16, 4096, 14336, 0, 2, 1),     # E = 0
+    (16, 4096, 14336, 65, 2, 1),    # E > 64
+    (16, 4096, 14336, 8, 0, 1),     # k = 0
+    (16, 4096, 14336, 8, 9, 1),     # k > E
+    (16, 4096, 14336, 8, 2, 7),     # unknown dtype
+    (-1, 4096, 14336, 8, 2, 1),     # T < 0
+])
+def test_bad_dimensions(moe, args):
+    assert moe.moe_workspace_size(*args) == 0
+    T, H, F, E, k, dt = args
+    rc = moe.moe_ffn_forward(None, None, None, None, None, None, T, H, F, E, k, dt, None, None, 0, None)
+    assert rc == -1
+
+
+def test_null_and_unsupported_before_device(moe):
+    P = 4096  # a fake, 16-byte aligned address: never dereferenced on these paths
+    # null weights
+    assert moe.moe_ffn_forward(P, P, None, None, P, None, 4, 128, 128, 2, 1, 0, P, P, 1 << 40, None) == -1
+    # FP8 without scales
+    assert moe.moe_ffn_forward(P, P, P, None, P, None, 4, 128, 128, 2, 1, 1, P, P, 1 << 40, None) == -1
+    # H not a multiple of 128
+    assert moe.moe_ffn_forward(P, P, P, None, P, None, 4, 200, 128, 2, 1, 0, P, P, 1 << 40, None) == -2
+    # too many assignments
+    assert moe.moe_ffn_forward(P, P, P, None, P, None, 200000, 128, 128, 8, 2, 0, P, P, 1 << 40, None) == -2
+    # misaligned pointer
+    assert moe.moe_ffn_forward(P + 4, P, P, None, P, None, 4, 128, 128, 2, 1, 0, P, P, 1 << 40, None) == -3
+    # workspace too small
+    assert moe.moe_ffn_forward(P, P, P, None, P, None, 4, 128, 128, 2, 1, 0, P, P, 10, None) == -4
+    # routing and preshuffle argument checks
+    assert moe.moe_route(None, 4, 0, 1, None, None, None, None, None, None, None, 0, None) == -1
+    assert moe.moe_route(P, 4, 8, 2, None, P, P, P, P, P, None, 0, None) == -1
+    assert moe.moe_prepare_weights(None, P, None, None, P, None, 2, 128, 128, 0, None) == -1
+    assert moe.moe_prepare_weights(P, P, None, None, P, None, 2, 100, 128, 0, None) == -2
+
+
+def test_options(moe):
+    old = moe.moe_set_option(moe.OPT_PATH, 2)
+    assert moe.moe_set_option(moe.OPT_PATH, old) == 2
+    assert moe.moe_set_option(moe.OPT_PATH, 5) == -1
+    assert moe.moe_set_option(99, 0) == -1
+    assert moe.moe_set_option(moe.OPT_TIMEOUT_MS, 0) == -1

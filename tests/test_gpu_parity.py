@@ -1,0 +1,213 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Routing (ids, counts, offsets, permutation) and the FP8 activation codes and
+scales must match bit for bit; the layer output must satisfy
+|gpu - ref| <= 1e-2*|ref| + 2e-3*rms(ref) element by element.  Small cases span
+several 128-row tiles, ragged tails, empty experts and both tile paths; the
+full-size workloads are checked on sampled tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+import oracle
+from helpers import bf16_bits_to_f64, check_close, out_as_f64, run_layer, small_case, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import mixture_experts_routed_02_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+@pytest.fixture(autouse=True)
+def _reset_options(moe):
+    yield
+    moe.moe_set_option(moe.OPT_PATH, 0)
+    moe.moe_set_option(moe.OPT_SPLITK, 0)
+
+
+# ---------------------------------------------------------------- routing
+
+def _route_cases():
+    rng = np.random.default_rng(0)
+    cases = []
+    for T, E, k in [(1, 8, 2), (5, 3, 3), (64, 8, 2), (1000, 8, 2), (333, 64, 8), (77, 16, 1), (4096, 8, 2)]:
+        cases.append((f"normal_T{T}_E{E}_k{k}", rng.normal(0, 1, (T, E)).astype(np.float32), k))
+    ties = rng.integers(-2, 3, (500, 8)).astype(np.float32)  # many exact ties
+    ties[::7, 3] = np.nan
+    ties[::11, :] = 0.0
+    ties[1::11, ::2] = -0.0
+    cases.append(("ties_nan_zeros", ties, 2))
+    cases.append(("skewed_T8192", moe_inputs.make_logits(8192, 8, 3, skew=True).numpy(), 2))
+    cases.append(("sweep_T16384", moe_inputs.make_logits(16384, 8, 4).numpy(), 2))
+    return cases
+
+
+@pytest.mark.parametrize("name,logits,k", _route_cases(), ids=lambda v: v if isinstance(v, str) else "")
+def test_route_bit_exact(moe, name, logits, k):
+    ref = oracle.route(logits, k)
+    out = moe.route(torch.from_numpy(logits).cuda(), k)
+    assert moe.moe_get_status(None) == 0
+    np.testing.assert_array_equal(out["ids"].cpu().numpy(), ref["ids"])
+    np.testing.assert_array_equal(out["counts"].cpu().numpy(), ref["counts"])
+    np.testing.assert_array_equal(out["offsets"].cpu().numpy(), ref["offsets"])
+    np.testing.assert_array_equal(out["perm"].cpu().numpy(), ref["perm"])
+    np.testing.assert_array_equal(out["inv_perm"].cpu().numpy(), ref["inv_perm"])
+    np.testing.assert_allclose(out["w"].cpu().numpy(), ref["w"], rtol=2e-6, atol=1e-7)
+
+
+def test_route_deterministic(moe):
+    lg = torch.from_numpy(moe_inputs.make_logits(16384, 8, 9).numpy()).cuda()
+    runs = [moe.route(lg, 2) for _ in range(3)]
+    for key in ("ids", "counts", "offsets", "perm", "inv_perm", "w"):
+        for r in runs[1:]:
+            assert torch.equal(r[key], runs[0][key]), key
+
+
+# ---------------------------------------------------------------- the layer, small sizes
+
+SMALL = [
+    # (T, H, F, E, k, dtype, seed, skew)
+    (64, 256, 512, 8, 2, "bf16", 0, False),     # the tiny workload
+    (64, 256, 512, 8, 2, "fp8", 0, False),
+    (1, 256, 512, 8, 2, "fp8", 5, False),
+    (3, 256, 256, 8, 2, "bf16", 6, False),
+    (200, 256, 512, 8, 2, "bf16", 7, False),    # several 128-row tiles, ragged tails
+    (300, 256, 512, 8, 2, "fp8", 8, True),      # skewed: big and empty experts
+    (37, 128, 256, 1, 1, "fp8", 9, False),      # E = 1, k = 1 (dense SwiGLU MLP)
+    (50, 128, 384, 4, 4, "bf16", 10, False),    # k = E
+    (129, 384, 640, 16, 3, "fp8", 11, False),   # odd multiples of 128
+]
+
+
+def _ids(p):
+    T, H, F, E, k, dt, seed, skew = p
+    return f"T{T}_H{H}_F{F}_E{E}_k{k}_{dt}" + ("_skew" if skew else "")
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["throughput_tiles", "streaming_tiles"])
+@pytest.mark.parametrize("p", SMALL, ids=_ids)
+def test_layer_small(moe, p, path):
+    T, H, F, E, k, dt, seed, skew = p
+    moe.moe_set_option(moe.OPT_PATH, path)
+    case = small_case(T, H, F, E, k, dt, seed, skew)
+    nc = moe_inputs.to_numpy(case)
+    ref = oracle.moe_ffn(nc)
+    dcase = to_device(case)
+    out, ws = run_layer(dcase)
+    check_close(out_as_f64(out), bf16_bits_to_f64(ref["out"]), f"layer {_ids(p)} path {path}")
+
+    # routing inside the layer is bit-exact too
+    r = oracle.route(nc["logits"], k)
+    A = T * k
+    dtc = moe.dtype_code(dt)
+    ids = moe.ws_view(ws, T, H, F, E, k, dtc, "topk_ids", torch.int32)[:A].cpu().numpy()
+    perm = moe.ws_view(ws, T, H, F, E, k, dtc, "perm", torch.int32)[:A].cpu().numpy()
+    np.testing.assert_array_equal(ids, r["ids"].reshape(-1))
+    np.testing.assert_array_equal(perm, r["perm"])
+    if dt == "fp8":
+        # R0: per-token e4m3 codes and scales, bitwise
+        xq_ref, sx_ref = oracle.quant_x(nc["x"])
+        slot_of = moe.ws_view(ws, T, H, F, E, k, dtc, "slot_of", torch.int32)[:A].cpu().numpy()
+        xs = moe.ws_view(ws, T, H, F, E, k, dtc, "xs").cpu().numpy().reshape(-1, H)
+        sx = moe.ws_view(ws, T, H, F, E, k, dtc, "sx", torch.float32).cpu().numpy()
+        for a in range(A):
+            t = a // k
+            np.testing.assert_array_equal(xs[slot_of[a]], xq_ref[t])
+            assert sx[slot_of[a]].view(np.uint32) == sx_ref[t].view(np.uint32)
+
+
+@pytest.mark.parametrize("splits", [2, 4])
+def test_layer_split_k(moe, splits):
+    moe.moe_set_option(moe.OPT_PATH, 2)
+    moe.moe_set_option(moe.OPT_SPLITK, splits)
+    case = small_case(40, 256, 1024, 8, 2, "fp8", 21)
+    ref = oracle.moe_ffn(moe_inputs.to_numpy(case))
+    out, _ = run_layer(to_device(case))
+    check_close(out_as_f64(out), bf16_bits_to_f64(ref["out"]), f"split-K {splits}")
+
+
+def test_layer_repeat_and_empty(moe):
+    case = small_case(70, 256, 512, 8, 2, "fp8", 22)
+    dcase = to_device(case)
+    a, ws = run_layer(dcase)
+    b, _ = run_layer(dcase, ws)  # the workspace is reused: nothing may leak from the first call
+    c, _ = run_layer(dcase, ws)
+    assert torch.equal(b, c)
+    ref = oracle.moe_ffn(moe_inputs.to_numpy(case))
+    check_close(out_as_f64(b), bf16_bits_to_f64(ref["out"]), "repeat")
+    import mixture_experts_routed_02_b200 as moe_mod
+    # T = 0: valid, nothing to do
+    rc = moe_mod.moe_ffn_forward(None, None, dcase["w13"].data_ptr(), dcase["s13"].data_ptr(),
+                                 dcase["w2"].data_ptr(), dcase["s2"].data_ptr(), 0, 256, 512, 8, 2, 1, None,
+                                 ws.data_ptr(), ws.numel(), None)
+    assert rc == 0
+
+
+def test_preshuffle_layout(moe):
+    case = small_case(4, 128, 256, 3, 2, "fp8", 23)
+    d = to_device(case)
+    w13 = d["w13"].view(torch.uint8).cpu().numpy()
+    s13 = d["s13"].cpu().numpy()
+    w1 = case["w1"].view(torch.uint8).numpy()
+    w3 = case["w3"].view(torch.uint8).numpy()
+    for e in range(3):
+        for r in range(512):
+            b, i = divmod(r, 64)
+            src = (w3 if i >= 32 else w1)[e, 32 * b + (i % 32)]
+            np.testing.assert_array_equal(w13[e, r], src)
+            assert s13[e, r] == (case["s3"] if i >= 32 else case["s1"])[e, 32 * b + (i % 32)]
+
+
+def test_host_errors(moe):
+    x = torch.zeros(16, 100, dtype=torch.bfloat16, device="cuda")
+    rc = moe.moe_ffn_forward(x.data_ptr(), x.data_ptr(), x.data_ptr(), None, x.data_ptr(), None, 16, 100, 256, 8, 2,
+                             0, x.data_ptr(), x.data_ptr(), 1 << 30, None)
+    assert rc == -2  # H % 128 != 0
+    rc = moe.moe_ffn_forward(x.data_ptr() + 2, x.data_ptr(), x.data_ptr(), None, x.data_ptr(), None, 16, 128, 256, 8,
+                             2, 0, x.data_ptr(), x.data_ptr(), 1 << 30, None)
+    assert rc == -3  # misaligned
+    rc = moe.moe_ffn_forward(x.data_ptr(), x.data_ptr(), x.data_ptr(), None, x.data_ptr(), None, 16, 128, 256, 8, 2,
+                             0, x.data_ptr(), x.data_ptr(), 16, None)
+    assert rc == -4  # workspace too small
+    assert moe.moe_get_status(None) == 0
+
+
+# ---------------------------------------------------------------- full-size workloads, sampled tokens
+
+FULL = [("decode", None), ("prefill", 6), ("skewed", 6), ("sweep_T1", None), ("sweep_T128", 6),
+        ("sweep_T1024", 4), ("sweep_T16384", 4)]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,nsample", FULL, ids=[f[0] for f in FULL])
+def test_layer_full_size_sampled(moe, name, nsample):
+    case = moe_inputs.make_config(name)
+    T = case["T"]
+    dcase = to_device(case)
+    out, ws = run_layer(dcase)
+    nc = moe_inputs.to_numpy(case)
+    r = oracle.route(nc["logits"], case["k"])
+    # routing over every token is bit-exact
+    A = T * case["k"]
+    dtc = moe.dtype_code(case["dtype"])
+    ids = moe.ws_view(ws, T, case["H"], case["F"], case["E"], case["k"], dtc, "topk_ids", torch.int32)[:A]
+    perm = moe.ws_view(ws, T, case["H"], case["F"], case["E"], case["k"], dtc, "perm", torch.int32)[:A]
+    np.testing.assert_array_equal(ids.cpu().numpy(), r["ids"].reshape(-1))
+    np.testing.assert_array_equal(perm.cpu().numpy(), r["perm"])
+    # sampled tokens: first, last, and tokens routed to the least used expert
+    if nsample is None or nsample >= T:
+        tokens = np.arange(T)
+    else:
+        rare = int(np.argmin(np.where(r["counts"] > 0, r["counts"], 1 << 30)))
+        rare_tok = [int(a // case["k"]) for a in r["perm"][r["offsets"][rare]:r["offsets"][rare + 1]]][:2]
+        rng = np.random.default_rng(1234)
+        tokens = np.unique(np.concatenate([[0, T - 1], rare_tok, rng.integers(0, T, nsample)]))
+    ref = oracle.moe_ffn_tokens(nc, tokens.astype(np.int32))
+    got = out_as_f64(out)[tokens]
+    check_close(got, bf16_bits_to_f64(ref["out"]), f"{name} sampled tokens {tokens.tolist()}")
