@@ -283,8 +283,10 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     // weight-streaming tiles when experts see few rows on average
     int cfg = g_opt_path.load();
     cfg = (cfg == 0) ? ((L.A <= 64 * E) ? 1 : 0) : cfg - 1;
-    const int bn1 = gemm_block_n(1, fp8, cfg);
-    const int bn2 = gemm_block_n(2, fp8, cfg);
+    const int cfg1 = ((2 * F) % gemm_block_n(1, fp8, cfg) == 0) ? cfg : 1;
+    const int cfg2 = (H % gemm_block_n(2, fp8, cfg) == 0) ? cfg : 1;  // 128-wide tiles when d_model % 256 != 0
+    const int bn1 = gemm_block_n(1, fp8, cfg1);
+    const int bn2 = gemm_block_n(2, fp8, cfg2);
     if ((2 * F) % bn1 || H % bn2) return MOE_ERR_UNSUPPORTED;
 
     CUtensorMap ta1, tb1, ta2, tb2;
@@ -341,7 +343,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     const long tiles1 = (long)L.MT_max * g1.n_tiles;
     {
         ProfScope ps(MOE_KERNEL_STAGE1, st);
-        if (launch_gemm(1, fp8, cfg, ta1, tb1, g1, (int)std::min<long>(tiles1, num_sms), st) != cudaSuccess)
+        if (launch_gemm(1, fp8, cfg1, ta1, tb1, g1, (int)std::min<long>(tiles1, num_sms), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 
@@ -363,7 +365,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     const long tiles2 = (long)L.MT_max * g2.n_tiles * g2.splits;
     {
         ProfScope ps(MOE_KERNEL_STAGE2, st);
-        if (launch_gemm(2, fp8, cfg, ta2, tb2, g2, (int)std::min<long>(tiles2, num_sms), st) != cudaSuccess)
+        if (launch_gemm(2, fp8, cfg2, ta2, tb2, g2, (int)std::min<long>(tiles2, num_sms), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 

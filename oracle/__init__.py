@@ -73,7 +73,7 @@ def _load():
         lib.oracle_moe_ffn.restype = I
         lib.oracle_moe_ffn.argtypes = [I, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, I]
         lib.oracle_moe_ffn_tokens.restype = I
-        lib.oracle_moe_ffn_tokens.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, I, P, P, I]
+        lib.oracle_moe_ffn_tokens.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, I, P, P, P, P, I]
         lib.oracle_max_threads.restype = I
         lib.oracle_max_threads.argtypes = []
         _lib = lib
@@ -192,8 +192,10 @@ def moe_ffn(case, mode="routed", nthreads=0, want_h=False):
     return dict(out=out, out64=out64, h=h)
 
 
-def moe_ffn_tokens(case, tokens, nthreads=0):
-    """Output rows for the given token ids only: dict(out [n,H] bf16 bits, out64)."""
+def moe_ffn_tokens(case, tokens, nthreads=0, want_h=False):
+    """Output rows for the given token ids only: dict(out [n,H] bf16 bits, out64),
+    plus with want_h the per-assignment intermediates h_deq and h_exact
+    [n*k, F] (row i*k + j = j-th expert of the i-th listed token)."""
     x = _c(case["x"], np.uint16)
     lg = _c(case["logits"], np.float32)
     T, H = x.shape
@@ -205,12 +207,14 @@ def moe_ffn_tokens(case, tokens, nthreads=0):
     n = tok.shape[0]
     out = np.zeros((n, H), dtype=np.uint16)
     out64 = np.zeros((n, H), dtype=np.float64)
+    h_deq = np.zeros((n * k, F), dtype=np.float64) if want_h else None
+    h_exact = np.zeros((n * k, F), dtype=np.float64) if want_h else None
     rc = _load().oracle_moe_ffn_tokens(_ptr(x), _ptr(lg), _ptr(w1), _ptr(w3), _ptr(s1), _ptr(s3),
                                        _ptr(w2), _ptr(s2), T, H, F, E, k, dt, _ptr(tok), n, _ptr(out),
-                                       _ptr(out64), int(nthreads))
+                                       _ptr(out64), _ptr(h_deq), _ptr(h_exact), int(nthreads))
     if rc != 0:
         raise ValueError("oracle_moe_ffn_tokens: bad arguments")
-    return dict(out=out, out64=out64)
+    return dict(out=out, out64=out64, h_deq=h_deq, h_exact=h_exact)
 
 
 def bf16_bits_to_float(b):

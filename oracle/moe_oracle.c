@@ -287,8 +287,9 @@ static double x_value(const ffn_ctx* c, int t, int i) {
 }
 
 /* y[H] = Y(e, t) in fp64.  h_out (optional, [F]) receives the dequantised
- * intermediate that enters the second GEMM. */
-static void expert_ffn(const ffn_ctx* c, int e, int t, double* y, double* h_out) {
+ * intermediate that enters the second GEMM; h_exact (optional, [F]) the exact
+ * value silu(g) * u before any rounding. */
+static void expert_ffn(const ffn_ctx* c, int e, int t, double* y, double* h_out, double* h_exact) {
     int H = c->H, F = c->F;
     double* hq = (double*)malloc(sizeof(double) * F);
     for (int n = 0; n < F; ++n) {
@@ -299,6 +300,7 @@ static void expert_ffn(const ffn_ctx* c, int e, int t, double* y, double* h_out)
             u += weight_value(c, c->w3, c->s3, e, n, i, F, H) * xv;
         }
         double silu = g / (1.0 + exp(-g));
+        if (h_exact) h_exact[n] = silu * u;
         hq[n] = oracle_bf16_to_double(oracle_bf16_from_double(silu * u));
     }
     if (c->dtype == ORACLE_FP8) {
@@ -374,7 +376,7 @@ int oracle_moe_ffn(int mode, const uint16_t* x, const float* logits, const void*
         for (long p = 0; p < A; ++p) {
             int32_t a = perm[p];
             int e = ids[a];
-            expert_ffn(&c, e, (int)(a / k), ybuf + (size_t)p * H, h_sorted ? h_sorted + (size_t)p * F : NULL);
+            expert_ffn(&c, e, (int)(a / k), ybuf + (size_t)p * H, h_sorted ? h_sorted + (size_t)p * F : NULL, NULL);
         }
         /* scatter-add in sorted order (deterministic) */
         for (long p = 0; p < A; ++p) {
@@ -391,7 +393,7 @@ int oracle_moe_ffn(int mode, const uint16_t* x, const float* logits, const void*
                 double mask = 0.0;
                 for (int j = 0; j < k; ++j)
                     if (ids[(size_t)t * k + j] == e) mask = w[(size_t)t * k + j];
-                expert_ffn(&c, e, t, y, NULL);
+                expert_ffn(&c, e, t, y, NULL, NULL);
                 for (int o = 0; o < H; ++o) acc[(size_t)t * H + o] += mask * y[o];
             }
             free(y);
@@ -408,12 +410,15 @@ int oracle_moe_ffn(int mode, const uint16_t* x, const float* logits, const void*
 
 /* Output rows for a list of tokens only (each token's result depends on its
  * own activations and logits alone), per-token routed form.  out: [ntok,H]
- * bf16; out64 optional [ntok,H].  Used for sampled checks at full size and for
- * the CPU timing sample. */
+ * bf16; out64 optional [ntok,H].  Optional per-assignment intermediates, row
+ * i*k + j for the j-th expert of the i-th listed token: h_deq [ntok*k, F] (the
+ * dequantised values entering the second GEMM) and h_exact [ntok*k, F] (silu(g)*u
+ * before rounding).  Used for sampled checks at full size and for the CPU
+ * timing sample. */
 int oracle_moe_ffn_tokens(const uint16_t* x, const float* logits, const void* w1, const void* w3,
                           const float* s1, const float* s3, const void* w2, const float* s2, int T, int H,
                           int F, int E, int k, int dtype, const int32_t* tokens, int ntok, uint16_t* out,
-                          double* out64, int nthreads) {
+                          double* out64, double* h_deq, double* h_exact, int nthreads) {
     ffn_ctx c;
     if (ctx_init(&c, x, w1, w3, s1, s3, w2, s2, T, H, F, E, k, dtype)) return -1;
     for (int i = 0; i < ntok; ++i)
@@ -441,7 +446,9 @@ int oracle_moe_ffn_tokens(const uint16_t* x, const float* logits, const void* w1
                      NULL, NULL, NULL);
     double* ybuf = (double*)malloc(sizeof(double) * (size_t)H * (work ? work : 1));
     #pragma omp parallel for schedule(dynamic, 1)
-    for (long q = 0; q < work; ++q) expert_ffn(&c, ids[q], tokens[q / k], ybuf + (size_t)q * H, NULL);
+    for (long q = 0; q < work; ++q)
+        expert_ffn(&c, ids[q], tokens[q / k], ybuf + (size_t)q * H, h_deq ? h_deq + (size_t)q * F : NULL,
+                   h_exact ? h_exact + (size_t)q * F : NULL);
     for (int i = 0; i < ntok; ++i) {
         for (int o = 0; o < H; ++o) {
             double acc = 0.0;

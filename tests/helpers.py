@@ -4,6 +4,7 @@ import numpy as np
 import torch
 
 import moe_inputs
+import oracle
 
 # |gpu - ref| <= REL * |ref| + ABS_RMS * rms(ref), element by element: the
 # tolerance stated for this layer (fp32 tensor-core accumulation and bf16/e4m3
@@ -62,3 +63,128 @@ def out_as_f64(out):
 
 def small_case(T, H=256, F=512, E=8, k=2, dtype="bf16", seed=0, skew=False):
     return moe_inputs.make_case(T, H, F, E, k, dtype, seed, skew)
+
+
+# ---------------------------------------------------------------- flip-aware layer check
+#
+# The intermediate h is rounded (bf16, and in FP8 mode e4m3 with a per-32
+# power-of-two scale) from a value the GPU forms with fp32 tensor-core
+# accumulation and the oracle in fp64.  Where that value lies within rounding
+# noise of a decision boundary both neighbouring codes are correct, and one
+# flipped e4m3 code moves the outputs of its row by |w2| * (one e4m3 step).
+# verify_layer therefore (1) compares the GPU's h with the oracle's h element
+# by element and accepts a difference only when it is such a flip -- the
+# oracle's exact value lies within RHO (relative) of the boundary between the
+# two codes -- and only when flips are rare; (2) checks every output element
+# against the stated tolerance plus the exact effect of the validated flips of
+# its token, computed from the oracle's w2 and routing weights.
+
+RHO = 2.0 ** -12          # admissible distance of a flipped decision from its boundary (relative)
+MAX_FLIP_FRACTION = 1e-2  # flips allowed per h row (a real defect changes most of a row)
+
+
+def _e4m3_values():
+    return torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+
+
+def gpu_h_rows(moe, ws, case, assignments):
+    """Dequantised GPU intermediate (float64 [n, F]) and, in FP8 mode, the block
+    exponents ([n, F/32]) of the given assignments."""
+    T, H, F, E, k, dt = (case[x] for x in ("T", "H", "F", "E", "k", "dtype"))
+    dc = moe.dtype_code(dt)
+    A = T * k
+    slot_of = moe.ws_view(ws, T, H, F, E, k, dc, "slot_of", torch.int32)[:A].cpu().numpy()
+    slots = torch.from_numpy(slot_of[np.asarray(assignments)].astype(np.int64)).to(ws.device)
+    hreg = moe.ws_view(ws, T, H, F, E, k, dc, "h")
+    if dt == "bf16":
+        rows = hreg.view(torch.bfloat16).view(-1, F)[slots].double().cpu().numpy()
+        return rows, None
+    codes = hreg.view(-1, F)[slots].cpu().numpy()
+    sf = moe.ws_view(ws, T, H, F, E, k, dc, "h_sf").cpu().numpy()
+    s = slots.cpu().numpy()
+    m, row = s // 128, s % 128
+    b = np.arange(F // 32)
+    idx = ((m[:, None] * (F // 128) + b[None, :] // 4) * 512 + (row[:, None] % 32) * 16 + (row[:, None] // 32) * 4
+           + b[None, :] % 4)
+    exps = sf[idx].astype(np.int64) - 127
+    vals = _e4m3_values()[codes] * np.repeat(2.0 ** exps, 32, axis=1)
+    return vals, exps
+
+
+def _quant_h(v, e, fp8):
+    """The oracle's rounding of one exact value: bf16, then (FP8) e4m3 at block exponent e."""
+    b = oracle.bf16_to_double(oracle.bf16_from_double(v))
+    if not fp8:
+        return b
+    return oracle.e4m3_to_double(oracle.e4m3_from_float(np.float32(b / 2.0 ** e))) * 2.0 ** e
+
+
+def _admissible(v, gpu_val, e_gpu, fp8, floor):
+    """Is gpu_val the rounding of some value within RHO of v?  (Rounding is
+    monotone, so it suffices to bracket gpu_val between the roundings of the
+    window's ends.)"""
+    w = RHO * max(abs(v), floor)
+    lo, hi = _quant_h(v - w, e_gpu, fp8), _quant_h(v + w, e_gpu, fp8)
+    return min(lo, hi) <= gpu_val <= max(lo, hi)
+
+
+def verify_layer(moe, ws, out, case, tokens=None, what=""):
+    """Check the GPU layer output (and its intermediate h) for the given tokens
+    against the oracle.  Returns a dict of statistics."""
+    nc = moe_inputs.to_numpy(case)
+    T, F, k = case["T"], case["F"], case["k"]
+    fp8 = case["dtype"] == "fp8"
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    ref = oracle.moe_ffn_tokens(nc, tokens.astype(np.int32), want_h=True)
+    r = oracle.route(nc["logits"], k)
+    assigns = (tokens[:, None] * k + np.arange(k)[None, :]).reshape(-1)
+    gh, gexp = gpu_h_rows(moe, ws, case, assigns)
+    rh, rx = ref["h_deq"], ref["h_exact"]
+    allow = np.zeros((len(tokens), case["H"]))
+    flips = 0
+    for q in range(len(assigns)):
+        d = np.nonzero(gh[q] != rh[q])[0]
+        if d.size == 0:
+            continue
+        assert d.size <= max(2, MAX_FLIP_FRACTION * F), f"{what}: {d.size} h elements differ in assignment {assigns[q]}"
+        floor = 1e-2 * float(np.sqrt(np.mean(rx[q] ** 2)))
+        for n in d:
+            e_gpu = int(gexp[q, n // 32]) if fp8 else 0
+            if fp8:
+                blk = slice(32 * (n // 32), 32 * (n // 32) + 32)
+                amax_i = 32 * (n // 32) + int(np.argmax(np.abs(rx[q, blk])))
+                e_ref = oracle.mx_exponent(max(abs(oracle.bf16_to_double(oracle.bf16_from_double(v)))
+                                               for v in rx[q, blk]))
+                if e_gpu != e_ref:
+                    # a block-scale flip: the block's absmax must sit at the exponent boundary
+                    va = rx[q, amax_i]
+                    wa = RHO * abs(va)
+                    cand = {oracle.mx_exponent(abs(oracle.bf16_to_double(oracle.bf16_from_double(va + s * wa))))
+                            for s in (-1, 1)}
+                    assert e_gpu in cand, f"{what}: block exponent {e_gpu} vs {e_ref} not at a boundary"
+            assert _admissible(rx[q, n], gh[q, n], e_gpu, fp8, floor), (
+                f"{what}: h[{assigns[q]}, {n}] gpu {gh[q, n]!r} oracle {rh[q, n]!r} exact {rx[q, n]!r}: not a "
+                f"rounding flip")
+        flips += d.size
+        # exact effect of the flips of this assignment on the token's outputs
+        t_i, j = divmod(q, k)
+        e = int(r["ids"][tokens[t_i], j])
+        wgt = float(r["w"][tokens[t_i], j])
+        if fp8:
+            col = _e4m3_values()[nc["w2"][e][:, d]] * nc["s2"][e][:, None].astype(np.float64)
+        else:
+            col = bf16_bits_to_f64(nc["w2"][e][:, d])
+        allow[t_i] += wgt * (np.abs(col) @ np.abs(gh[q, d] - rh[q, d]))
+    gpu = out.float().double().cpu().numpy()[tokens]
+    refv = bf16_bits_to_f64(ref["out"])
+    rms = float(np.sqrt(np.mean(refv ** 2)))
+    allowed = REL * np.abs(refv) + ABS_RMS * rms + allow
+    err = np.abs(gpu - refv)
+    bad = err > allowed
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} outputs out of tolerance; worst err "
+                           f"{err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}, rms(ref) {rms:.3e}, "
+                           f"h flips {flips}")
+    strict = err <= REL * np.abs(refv) + ABS_RMS * rms
+    return dict(flips=flips, h_elements=len(assigns) * F, outputs_needing_allowance=int((~strict).sum()),
+                max_err_over_tol=float((err / (REL * np.abs(refv) + ABS_RMS * rms)).max()))

@@ -12,7 +12,7 @@ import torch
 
 import moe_inputs
 import oracle
-from helpers import bf16_bits_to_f64, check_close, out_as_f64, run_layer, small_case, to_device
+from helpers import bf16_bits_to_f64, check_close, out_as_f64, run_layer, small_case, to_device, verify_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -97,10 +97,9 @@ def test_layer_small(moe, p, path):
     moe.moe_set_option(moe.OPT_PATH, path)
     case = small_case(T, H, F, E, k, dt, seed, skew)
     nc = moe_inputs.to_numpy(case)
-    ref = oracle.moe_ffn(nc)
     dcase = to_device(case)
     out, ws = run_layer(dcase)
-    check_close(out_as_f64(out), bf16_bits_to_f64(ref["out"]), f"layer {_ids(p)} path {path}")
+    verify_layer(moe, ws, out, case, what=f"layer {_ids(p)} path {path}")
 
     # routing inside the layer is bit-exact too
     r = oracle.route(nc["logits"], k)
@@ -127,9 +126,8 @@ def test_layer_split_k(moe, splits):
     moe.moe_set_option(moe.OPT_PATH, 2)
     moe.moe_set_option(moe.OPT_SPLITK, splits)
     case = small_case(40, 256, 1024, 8, 2, "fp8", 21)
-    ref = oracle.moe_ffn(moe_inputs.to_numpy(case))
-    out, _ = run_layer(to_device(case))
-    check_close(out_as_f64(out), bf16_bits_to_f64(ref["out"]), f"split-K {splits}")
+    out, ws = run_layer(to_device(case))
+    verify_layer(moe, ws, out, case, what=f"split-K {splits}")
 
 
 def test_layer_repeat_and_empty(moe):
@@ -139,8 +137,7 @@ def test_layer_repeat_and_empty(moe):
     b, _ = run_layer(dcase, ws)  # the workspace is reused: nothing may leak from the first call
     c, _ = run_layer(dcase, ws)
     assert torch.equal(b, c)
-    ref = oracle.moe_ffn(moe_inputs.to_numpy(case))
-    check_close(out_as_f64(b), bf16_bits_to_f64(ref["out"]), "repeat")
+    verify_layer(moe, ws, c, case, what="repeat")
     import mixture_experts_routed_02_b200 as moe_mod
     # T = 0: valid, nothing to do
     rc = moe_mod.moe_ffn_forward(None, None, dcase["w13"].data_ptr(), dcase["s13"].data_ptr(),
@@ -208,6 +205,5 @@ def test_layer_full_size_sampled(moe, name, nsample):
         rare_tok = [int(a // case["k"]) for a in r["perm"][r["offsets"][rare]:r["offsets"][rare + 1]]][:2]
         rng = np.random.default_rng(1234)
         tokens = np.unique(np.concatenate([[0, T - 1], rare_tok, rng.integers(0, T, nsample)]))
-    ref = oracle.moe_ffn_tokens(nc, tokens.astype(np.int32))
-    got = out_as_f64(out)[tokens]
-    check_close(got, bf16_bits_to_f64(ref["out"]), f"{name} sampled tokens {tokens.tolist()}")
+    stats = verify_layer(moe, ws, out, case, tokens, what=f"{name} sampled tokens {tokens.tolist()}")
+    print(name, stats)
