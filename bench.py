@@ -258,10 +258,10 @@ def main():
     fp8 = spec["dtype"] == "fp8"
     x = case["x"].to(dev)
     logits = case["logits"].to(dev)
-    w2 = case["w2"].to(dev)
     s2 = case["s2"].to(dev) if fp8 else None
-    w13, s13 = moe.prepare_weights(case["w1"].to(dev), case["w3"].to(dev),
-                                   case["s1"].to(dev) if fp8 else None, case["s3"].to(dev) if fp8 else None)
+    w13, s13, w2 = moe.prepare_weights(case["w1"].to(dev), case["w3"].to(dev),
+                                       case["s1"].to(dev) if fp8 else None, case["s3"].to(dev) if fp8 else None,
+                                       case["w2"].to(dev))
     del case
     torch.cuda.empty_cache()
     dt_code = moe.MOE_FP8_E4M3 if fp8 else moe.MOE_BF16
@@ -270,7 +270,7 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        moe.ffn_forward(x, logits, w13, s13, w2, s2, k, out=out, ws=ws, stream=stream)
+        moe.ffn_forward(x, logits, w13, s13, w2, s2, k, F, fp8, out=out, ws=ws, stream=stream)
 
     for _ in range(max(3, args.warmup)):
         step()

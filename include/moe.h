@@ -64,18 +64,28 @@ size_t moe_workspace_size(int T, int H, int F, int E, int k, int dtype);
 
 /*
  * One-time weight preshuffle (timestamp 8:14, "load-time preshuffle").
- * Interleaves the gate and up projections so that one tile of the first group
- * GEMM holds matching gate/up output channels:
- *   w13[e][64*b + i]      = w1[e][32*b + i]   for i in [0,32)
- *   w13[e][64*b + 32 + i] = w3[e][32*b + i]
- * and the same for the scales s13 (FP8 only; NULL for BF16).
+ * Produces the layout the group GEMMs stream from.  Each expert matrix
+ * [rows, K] (K-contiguous, `eb` = 1 byte for e4m3, 2 for bf16) is cut into
+ * blocks of 128 rows x 128 bytes of K, stored contiguously in the order
+ * [expert][row block][K block], 16384 bytes each.  Inside a block, the 16-byte
+ * chunk c of row r sits at byte r*128 + ((c ^ (r % 8)) * 16): the 128-byte
+ * swizzle of the tensor cores' shared-memory operand, so one bulk copy of a
+ * block is a ready operand tile.
+ * w13 holds the gate and up projections interleaved in groups of 32 rows, so
+ * that one tile of the first group GEMM holds matching gate/up channels:
+ *   row 64*b + i      of w13[e] = row 32*b + i of w1[e]   (i in [0,32))
+ *   row 64*b + 32 + i of w13[e] = row 32*b + i of w3[e]
+ * and s13 (FP8 only) is interleaved the same way, unblocked: [E, 2F] fp32.
  *   w1, w3   device, [E,F,H] row-major (bf16 or e4m3 bytes), read only
- *   s1, s3   device, [E,F] fp32, read only (FP8) or NULL (BF16)
- *   w13_out  device, [E,2F,H] (bf16 or e4m3), written
+ *   s1, s3   device, [E,F] fp32 (FP8) or NULL (BF16), read only
+ *   w2       device, [E,H,F] row-major, read only
+ *   w13_out  device, E*2F*H*eb bytes, written (blocked layout above)
  *   s13_out  device, [E,2F] fp32 (FP8) or NULL
+ *   w2_out   device, E*H*F*eb bytes, written (blocked layout above)
+ * The per-output-channel scales of w2 (s2, [E,H]) are used as they are.
  */
-int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const float* s3, void* w13_out,
-                        float* s13_out, int E, int F, int H, int dtype, void* stream);
+int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const float* s3, const void* w2,
+                        void* w13_out, float* s13_out, void* w2_out, int E, int F, int H, int dtype, void* stream);
 
 /*
  * Routing alone (timestamps 5:56 and 8:14): top-k selection, softmax over the
@@ -102,9 +112,9 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float
  * e = topk_ids[t,j] (paragraph 2 and timestamp 5:56).
  *   x        device, [T,H] bf16, read only.
  *   logits   device, [T,E] fp32, read only (routed exactly as moe_route does).
- *   w13      device, prepared by moe_prepare_weights: [E,2F,H] bf16 or e4m3.
- *   s13      device, [E,2F] fp32 (FP8) or NULL (BF16).
- *   w2       device, [E,H,F] bf16 or e4m3, read only.
+ *   w13      device, w1/w3 prepared by moe_prepare_weights (blocked, interleaved).
+ *   s13      device, [E,2F] fp32 (FP8) or NULL (BF16), from moe_prepare_weights.
+ *   w2       device, w2 prepared by moe_prepare_weights (blocked).
  *   s2       device, [E,H] fp32 (FP8) or NULL (BF16).
  *   out      device, [T,H] bf16, written.
  *   ws       device workspace, >= moe_workspace_size(T,H,F,E,k,dtype) bytes;

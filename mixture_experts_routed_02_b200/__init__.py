@@ -60,7 +60,7 @@ lib.moe_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I]
 lib.moe_workspace_region.restype = ctypes.c_longlong
 lib.moe_workspace_region.argtypes = [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_Z)]
 lib.moe_prepare_weights.restype = _I
-lib.moe_prepare_weights.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]
+lib.moe_prepare_weights.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]
 lib.moe_route.restype = _I
 lib.moe_route.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P]
 lib.moe_ffn_forward.restype = _I
@@ -140,17 +140,20 @@ def ws_view(ws, T, H, F, E, k, dtype, which, torch_dtype=None):
     return v.view(torch_dtype) if torch_dtype is not None else v
 
 
-def prepare_weights(w1, w3, s1=None, s3=None, stream=None):
-    """One-time preshuffle: returns (w13 [E,2F,H], s13 [E,2F] or None)."""
+def prepare_weights(w1, w3, s1, s3, w2, stream=None):
+    """One-time preshuffle: returns (w13, s13, w2p) in the blocked layouts the
+    kernels stream (w13/w2p are flat byte tensors; s13 [E,2F] or None)."""
     import torch
     E, F, H = w1.shape
     fp8 = w1.dtype == torch.float8_e4m3fn
-    w13 = torch.empty(E, 2 * F, H, dtype=w1.dtype, device=w1.device)
+    w13 = torch.empty(E * 2 * F * H * w1.element_size(), dtype=torch.uint8, device=w1.device)
+    w2p = torch.empty(w2.numel() * w2.element_size(), dtype=torch.uint8, device=w2.device)
     s13 = torch.empty(E, 2 * F, dtype=torch.float32, device=w1.device) if fp8 else None
-    rc = moe_prepare_weights(_ptr(w1), _ptr(w3), _ptr(s1) if fp8 else None, _ptr(s3) if fp8 else None, _ptr(w13),
-                             _ptr(s13), E, F, H, MOE_FP8_E4M3 if fp8 else MOE_BF16, _stream(stream))
+    rc = moe_prepare_weights(_ptr(w1), _ptr(w3), _ptr(s1) if fp8 else None, _ptr(s3) if fp8 else None, _ptr(w2),
+                             _ptr(w13), _ptr(s13), _ptr(w2p), E, F, H, MOE_FP8_E4M3 if fp8 else MOE_BF16,
+                             _stream(stream))
     _check("moe_prepare_weights", rc)
-    return w13, s13
+    return w13, s13, w2p
 
 
 def route(logits, k, stream=None):
@@ -171,19 +174,17 @@ def route(logits, k, stream=None):
     return out
 
 
-def ffn_forward(x, logits, w13, s13, w2, s2, k, out=None, ws=None, stream=None):
-    """The whole layer; returns the bf16 output [T,H] (and fills ``ws``)."""
+def ffn_forward(x, logits, w13, s13, w2p, s2, k, F, fp8, out=None, ws=None, stream=None):
+    """The whole layer on prepared weights; returns the bf16 output [T,H] (and fills ``ws``)."""
     import torch
     T, H = x.shape
     E = logits.shape[1]
-    F = w13.shape[1] // 2
-    fp8 = w13.dtype == torch.float8_e4m3fn
     dt = MOE_FP8_E4M3 if fp8 else MOE_BF16
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
     if ws is None:
         ws = workspace(T, H, F, E, k, dt, x.device)
-    rc = moe_ffn_forward(_ptr(x), _ptr(logits), _ptr(w13), _ptr(s13) if fp8 else None, _ptr(w2),
+    rc = moe_ffn_forward(_ptr(x), _ptr(logits), _ptr(w13), _ptr(s13) if fp8 else None, _ptr(w2p),
                          _ptr(s2) if fp8 else None, T, H, F, E, k, dt, _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
     _check("moe_ffn_forward", rc)
     return out

@@ -4,7 +4,9 @@
 //                    2: "gather"), fused with the per-token FP8 quantisation of
 //                    the activations and with zeroing the fp32 combine buffer;
 //   finalize_kernel  fp32 combine buffer -> bf16 output;
-//   interleave_kernel the one-time load-time preshuffle of w1/w3 (timestamp 8:14).
+//   preshuffle_kernel the one-time load-time preshuffle of the expert weights into
+//                    contiguous, pre-swizzled 128x128-byte operand blocks
+//                    (timestamp 8:14).
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -105,21 +107,49 @@ __global__ void finalize_kernel(const float* __restrict__ out32, __nv_bfloat16* 
     }
 }
 
-// w13[e][64b + i] = w1[e][32b + i], w13[e][64b + 32 + i] = w3[e][32b + i]; one
-// CTA per destination row.  row_bytes % 16 == 0.
-__global__ void interleave_kernel(const uint8_t* __restrict__ w1, const uint8_t* __restrict__ w3,
-                                  const float* __restrict__ s1, const float* __restrict__ s3, uint8_t* __restrict__ w13,
-                                  float* __restrict__ s13, int F, int row_bytes) {
-    const int e = blockIdx.y;
-    const int r = blockIdx.x;  // destination row in [0, 2F)
-    const int b = r / 64, i = r % 64;
-    const bool up = i >= 32;
-    const int src_row = 32 * b + (i & 31);
-    const uint8_t* src = (up ? w3 : w1) + ((size_t)e * F + src_row) * row_bytes;
-    uint8_t* dst = w13 + ((size_t)e * 2 * F + r) * row_bytes;
-    for (int v = threadIdx.x; v < row_bytes / 16; v += blockDim.x)
-        reinterpret_cast<uint4*>(dst)[v] = __ldg(reinterpret_cast<const uint4*>(src) + v);
-    if (s13 && threadIdx.x == 0) s13[(size_t)e * 2 * F + r] = (up ? s3 : s1)[(size_t)e * F + src_row];
+// One thread per destination 16-byte chunk, destinations in address order.
+// Destination chunk g: (expert e, row block nb, K block kt, row r, stored
+// chunk pc); it holds logical chunk c = pc ^ (r % 8) of destination row
+// R = 128*nb + r.  With `interleave` the destination rows are the w1/w3
+// interleave (groups of 32 rows from a, then b); otherwise row R of a.
+__global__ void preshuffle_kernel(const uint8_t* __restrict__ a, const uint8_t* __restrict__ b,
+                                  uint8_t* __restrict__ dst, int E, int src_rows, int dst_rows, int row_bytes,
+                                  bool interleave) {
+    const int kt_count = row_bytes / 128;
+    const int nb_count = dst_rows / kWBlockRows;
+    const size_t total = (size_t)E * dst_rows * row_bytes / 16;
+    for (size_t g = blockIdx.x * (size_t)blockDim.x + threadIdx.x; g < total; g += (size_t)gridDim.x * blockDim.x) {
+        const int pc = (int)(g & 7);
+        const int r = (int)((g >> 3) & 127);
+        size_t rest = g >> 10;
+        const int kt = (int)(rest % kt_count);
+        rest /= kt_count;
+        const int nb = (int)(rest % nb_count);
+        const int e = (int)(rest / nb_count);
+        const int c = pc ^ (r & 7);
+        const int R = nb * kWBlockRows + r;
+        const uint8_t* src = a;
+        int srow = R;
+        if (interleave) {
+            const int grp = R / 64, i = R % 64;
+            src = (i < 32) ? a : b;
+            srow = 32 * grp + (i & 31);
+        }
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + ((size_t)e * src_rows + srow) * row_bytes +
+                                                             kt * 128 + c * 16));
+        reinterpret_cast<uint4*>(dst)[g] = v;
+    }
+}
+
+__global__ void interleave_scales_kernel(const float* __restrict__ s1, const float* __restrict__ s3,
+                                         float* __restrict__ s13, int E, int F) {
+    const size_t total = (size_t)E * 2 * F;
+    for (size_t g = blockIdx.x * (size_t)blockDim.x + threadIdx.x; g < total; g += (size_t)gridDim.x * blockDim.x) {
+        const int e = (int)(g / (2 * F));
+        const int R = (int)(g % (2 * F));
+        const int grp = R / 64, i = R % 64;
+        s13[g] = ((i < 32) ? s1 : s3)[(size_t)e * F + 32 * grp + (i & 31)];
+    }
 }
 
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream) {
@@ -129,9 +159,17 @@ cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, in
     return cudaGetLastError();
 }
 
-cudaError_t launch_interleave(const uint8_t* w1, const uint8_t* w3, const float* s1, const float* s3, uint8_t* w13,
-                              float* s13, int E, int F, int row_bytes, cudaStream_t stream) {
-    interleave_kernel<<<dim3(2 * F, E), 128, 0, stream>>>(w1, w3, s1, s3, w13, s13, F, row_bytes);
+cudaError_t launch_preshuffle(const uint8_t* a, const uint8_t* b, uint8_t* dst, int E, int src_rows, int dst_rows,
+                              int row_bytes, bool interleave, cudaStream_t stream) {
+    const size_t chunks = (size_t)E * dst_rows * row_bytes / 16;
+    const int blocks = (int)std::min<size_t>((chunks + 255) / 256, 65535);
+    preshuffle_kernel<<<blocks, 256, 0, stream>>>(a, b, dst, E, src_rows, dst_rows, row_bytes, interleave);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_interleave_scales(const float* s1, const float* s3, float* s13, int E, int F, cudaStream_t stream) {
+    const size_t n = (size_t)E * 2 * F;
+    interleave_scales_kernel<<<(int)std::min<size_t>((n + 255) / 256, 65535), 256, 0, stream>>>(s1, s3, s13, E, F);
     return cudaGetLastError();
 }
 

@@ -41,7 +41,7 @@ struct Cfg {
     static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
                                    : COLS_USED <= 256 ? 256 : 512;
     static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
-    static_assert(BN % 64 == 0 && BN <= 256, "BN");
+    static_assert(BN % kWBlockRows == 0 && BN <= 256, "BN: whole 128-row weight blocks");
     // shared memory: A ring, B ring, SF ring, constant B scales, barriers
     static constexpr int OFF_B = NST * A_BYTES;
     static constexpr int OFF_SF = OFF_B + NST * B_BYTES;
@@ -63,8 +63,7 @@ __device__ __forceinline__ void decode_tile(int tile, int num_mt, int n_tiles, i
 
 template <int STAGE, bool FP8, int BN, int NST>
 __global__ void __launch_bounds__(192, 1)
-    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const GemmArgs args) {
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const GemmArgs args) {
     using C = Cfg<STAGE, FP8, BN, NST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -104,7 +103,6 @@ __global__ void __launch_bounds__(192, 1)
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
-        prefetch_tmap(&tmB);
     }
     tc_fence_before();
     __syncthreads();
@@ -118,7 +116,8 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol_a = policy_evict_last();
-            const uint64_t pol_b = policy_evict_first();
+            const uint64_t pol_b = args.b_evict_first ? policy_evict_first() : policy_evict_normal();
+            const int b_nblk = args.rows_b / kWBlockRows;
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
@@ -127,7 +126,9 @@ __global__ void __launch_bounds__(192, 1)
                 int m, n, split;
                 decode_tile(tile, num_mt, args.n_tiles, m, n, split);
                 const int e = args.mtile_expert[m];
-                const int brow = e * args.rows_b + n * BN;
+                // first weight block of this tile: expert e, row block n*BN/128, K block 0
+                const uint8_t* bsrc = args.b_blocks + (((size_t)e * b_nblk + n * (BN / kWBlockRows)) * args.k_tiles)
+                                                          * kWBlockBytes;
                 for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, limit, args.status)) {
                         ok = false;
@@ -135,7 +136,11 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
                     tma_load_2d(smem + stage * C::A_BYTES, &tmA, &full[stage], kt * C::KE, m * kBlockM, pol_a);
-                    tma_load_2d(smem + C::OFF_B + stage * C::B_BYTES, &tmB, &full[stage], kt * C::KE, brow, pol_b);
+#pragma unroll
+                    for (int j = 0; j < BN / kWBlockRows; ++j)
+                        bulk_load_hint(smem + C::OFF_B + stage * C::B_BYTES + j * kWBlockBytes,
+                                       bsrc + ((size_t)j * args.k_tiles + kt) * kWBlockBytes, kWBlockBytes,
+                                       &full[stage], pol_b);
                     if constexpr (C::MX)
                         bulk_load(smem + C::OFF_SF + stage * C::SF_BYTES,
                                   args.a_sf + ((size_t)m * args.f_tiles + kt) * 512, 512, &full[stage]);
@@ -354,13 +359,12 @@ __global__ void __launch_bounds__(192, 1)
 namespace {
 
 template <int STAGE, bool FP8, int BN, int NST>
-cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, int grid,
-                       cudaStream_t stream) {
+cudaError_t launch_one(const CUtensorMap& ta, const GemmArgs& args, int grid, cudaStream_t stream) {
     using C = Cfg<STAGE, FP8, BN, NST>;
     auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    kern<<<grid, 192, C::SMEM_BYTES, stream>>>(ta, tb, args);
+    kern<<<grid, 192, C::SMEM_BYTES, stream>>>(ta, args);
     return cudaGetLastError();
 }
 
@@ -371,17 +375,17 @@ int gemm_block_n(int stage, bool fp8, int cfg) {
     return cfg == 0 ? 256 : 128;
 }
 
-cudaError_t launch_gemm(int stage, bool fp8, int cfg, const CUtensorMap& ta, const CUtensorMap& tb,
-                        const GemmArgs& args, int grid, cudaStream_t stream) {
+cudaError_t launch_gemm(int stage, bool fp8, int cfg, const CUtensorMap& ta, const GemmArgs& args, int grid,
+                        cudaStream_t stream) {
     if (stage == 1) {
-        if (fp8) return cfg == 0 ? launch_one<1, true, 256, 4>(ta, tb, args, grid, stream)
-                                 : launch_one<1, true, 128, 6>(ta, tb, args, grid, stream);
-        return cfg == 0 ? launch_one<1, false, 256, 4>(ta, tb, args, grid, stream)
-                        : launch_one<1, false, 128, 6>(ta, tb, args, grid, stream);
+        if (fp8) return cfg == 0 ? launch_one<1, true, 256, 4>(ta, args, grid, stream)
+                                 : launch_one<1, true, 128, 6>(ta, args, grid, stream);
+        return cfg == 0 ? launch_one<1, false, 256, 4>(ta, args, grid, stream)
+                        : launch_one<1, false, 128, 6>(ta, args, grid, stream);
     }
-    if (fp8) return launch_one<2, true, 128, 6>(ta, tb, args, grid, stream);
-    return cfg == 0 ? launch_one<2, false, 256, 4>(ta, tb, args, grid, stream)
-                    : launch_one<2, false, 128, 6>(ta, tb, args, grid, stream);
+    if (fp8) return launch_one<2, true, 128, 6>(ta, args, grid, stream);
+    return cfg == 0 ? launch_one<2, false, 256, 4>(ta, args, grid, stream)
+                    : launch_one<2, false, 128, 6>(ta, args, grid, stream);
 }
 
 }  // namespace moe

@@ -37,8 +37,12 @@ cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k,
                           const int* slot_assign, uint8_t* xs, float* sx_slot, float* out32, int* status,
                           cudaStream_t stream);
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream);
-cudaError_t launch_interleave(const uint8_t* w1, const uint8_t* w3, const float* s1, const float* s3, uint8_t* w13,
-                              float* s13, int E, int F, int row_bytes, cudaStream_t stream);
+// Blocked, pre-swizzled weight layout (see moe_prepare_weights in moe.h).
+constexpr int kWBlockRows = 128;
+constexpr int kWBlockBytes = kWBlockRows * 128;
+cudaError_t launch_preshuffle(const uint8_t* a, const uint8_t* b, uint8_t* dst, int E, int src_rows, int dst_rows,
+                              int row_bytes, bool interleave, cudaStream_t stream);
+cudaError_t launch_interleave_scales(const float* s1, const float* s3, float* s13, int E, int F, cudaStream_t stream);
 
 // Arguments of the grouped GEMM (both stages).
 struct GemmArgs {
@@ -48,6 +52,8 @@ struct GemmArgs {
     const float* row_scale;   // stage 1, FP8: per-row activation scale [S]
     const float* col_scale;   // FP8: s13 [E*2F] (stage 1) or s2 [E*H] (stage 2)
     const float* topk_w;      // stage 2: routing weight per assignment
+    const uint8_t* b_blocks;  // weights in the blocked layout: [E][rows_b/128][k_tiles][16 KB]
+    int b_evict_first;        // stream weights with the L2 evict-first hint (each tile read once)
     const uint8_t* a_sf;      // stage 2, FP8: UE8M0 scales of h, tiled
     void* out;                // stage 1: h [S, F]; stage 2: out32 [T, H]
     uint8_t* out_sf;          // stage 1, FP8: UE8M0 scales of h, tiled
@@ -65,8 +71,8 @@ struct GemmArgs {
 
 // Host launchers of the tcgen05 grouped GEMM; defined in gemm.cu.
 // cfg: 0 = throughput tiles (BN=256), 1 = weight-streaming tiles (BN=128).
-cudaError_t launch_gemm(int stage, bool fp8, int cfg, const CUtensorMap& ta, const CUtensorMap& tb,
-                        const GemmArgs& args, int grid, cudaStream_t stream);
+cudaError_t launch_gemm(int stage, bool fp8, int cfg, const CUtensorMap& ta, const GemmArgs& args, int grid,
+                        cudaStream_t stream);
 int gemm_block_n(int stage, bool fp8, int cfg);
 
 }  // namespace moe

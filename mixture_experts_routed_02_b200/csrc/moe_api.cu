@@ -230,18 +230,27 @@ int moe_set_option(int option, int value) {
     }
 }
 
-int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const float* s3, void* w13_out,
-                        float* s13_out, int E, int F, int H, int dtype, void* stream) {
-    if (!w1 || !w3 || !w13_out || E < 1 || E > kMaxExperts || F <= 0 || H <= 0) return MOE_ERR_INVALID_ARG;
+int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const float* s3, const void* w2,
+                        void* w13_out, float* s13_out, void* w2_out, int E, int F, int H, int dtype, void* stream) {
+    if (!w1 || !w3 || !w2 || !w13_out || !w2_out || E < 1 || E > kMaxExperts || F <= 0 || H <= 0)
+        return MOE_ERR_INVALID_ARG;
     if (dtype != MOE_BF16 && dtype != MOE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
     const bool fp8 = dtype == MOE_FP8_E4M3;
     if (fp8 && (!s1 || !s3 || !s13_out)) return MOE_ERR_INVALID_ARG;
     if (F % 128 || H % 128) return MOE_ERR_UNSUPPORTED;
-    if (!aligned16(w1) || !aligned16(w3) || !aligned16(w13_out)) return MOE_ERR_ALIGNMENT;
+    const void* ptrs[] = {w1, w3, w2, w13_out, w2_out, fp8 ? s13_out : nullptr};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
     const int eb = fp8 ? 1 : 2;
-    return launch_status(launch_interleave(static_cast<const uint8_t*>(w1), static_cast<const uint8_t*>(w3),
-                                           fp8 ? s1 : nullptr, fp8 ? s3 : nullptr, static_cast<uint8_t*>(w13_out),
-                                           fp8 ? s13_out : nullptr, E, F, H * eb, static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (launch_preshuffle(static_cast<const uint8_t*>(w1), static_cast<const uint8_t*>(w3),
+                          static_cast<uint8_t*>(w13_out), E, F, 2 * F, H * eb, true, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (launch_preshuffle(static_cast<const uint8_t*>(w2), nullptr, static_cast<uint8_t*>(w2_out), E, H, H, F * eb,
+                          false, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (fp8 && launch_interleave_scales(s1, s3, s13_out, E, F, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
 }
 
 int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w, int32_t* counts,
@@ -289,11 +298,9 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     const int bn2 = gemm_block_n(2, fp8, cfg2);
     if ((2 * F) % bn1 || H % bn2) return MOE_ERR_UNSUPPORTED;
 
-    CUtensorMap ta1, tb1, ta2, tb2;
+    CUtensorMap ta1, ta2;
     if (!make_map(&ta1, reg(MOE_WS_XS), L.S_max, H, eb, kBlockM) ||
-        !make_map(&tb1, w13, (size_t)E * 2 * F, H, eb, bn1) ||
-        !make_map(&ta2, reg(MOE_WS_H), L.S_max, F, eb, kBlockM) ||
-        !make_map(&tb2, w2, (size_t)E * H, F, eb, bn2))
+        !make_map(&ta2, reg(MOE_WS_H), L.S_max, F, eb, kBlockM))
         return MOE_ERR_CUDA;
 
     // 1. routing and the expert-padded layout
@@ -328,6 +335,8 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     g1.slot_assign = o.slot_assign;
     g1.row_scale = fp8 ? sx : nullptr;
     g1.col_scale = fp8 ? s13 : nullptr;
+    g1.b_blocks = static_cast<const uint8_t*>(w13);
+    g1.b_evict_first = (cfg1 == 1) ? 1 : 0;  // weight-streaming tiles read each weight block once
     g1.out = reg(MOE_WS_H);
     g1.out_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;
     g1.rows_b = 2 * F;
@@ -343,7 +352,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     const long tiles1 = (long)L.MT_max * g1.n_tiles;
     {
         ProfScope ps(MOE_KERNEL_STAGE1, st);
-        if (launch_gemm(1, fp8, cfg1, ta1, tb1, g1, (int)std::min<long>(tiles1, num_sms), st) != cudaSuccess)
+        if (launch_gemm(1, fp8, cfg1, ta1, g1, (int)std::min<long>(tiles1, num_sms), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 
@@ -353,6 +362,8 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     g2.col_scale = fp8 ? s2 : nullptr;
     g2.topk_w = o.topk_w;
     g2.a_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;
+    g2.b_blocks = static_cast<const uint8_t*>(w2);
+    g2.b_evict_first = (cfg2 == 1) ? 1 : 0;
     g2.out = out32;
     g2.out_sf = nullptr;
     g2.rows_b = H;
@@ -365,7 +376,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     const long tiles2 = (long)L.MT_max * g2.n_tiles * g2.splits;
     {
         ProfScope ps(MOE_KERNEL_STAGE2, st);
-        if (launch_gemm(2, fp8, cfg2, ta2, tb2, g2, (int)std::min<long>(tiles2, num_sms), st) != cudaSuccess)
+        if (launch_gemm(2, fp8, cfg2, ta2, g2, (int)std::min<long>(tiles2, num_sms), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 

@@ -40,7 +40,7 @@ def to_device(case, device="cuda"):
     for key in ("x", "logits", "w1", "w3", "w2", "s1", "s3", "s2"):
         v = case.get(key)
         d[key] = None if v is None else v.to(device)
-    d["w13"], d["s13"] = moe.prepare_weights(d["w1"], d["w3"], d["s1"], d["s3"])
+    d["w13"], d["s13"], d["w2p"] = moe.prepare_weights(d["w1"], d["w3"], d["s1"], d["s3"], d["w2"])
     for key in ("T", "H", "F", "E", "k", "dtype"):
         d[key] = case[key]
     return d
@@ -50,8 +50,8 @@ def run_layer(dcase, ws=None):
     import mixture_experts_routed_02_b200 as moe
     if ws is None:
         ws = moe.workspace(dcase["T"], dcase["H"], dcase["F"], dcase["E"], dcase["k"], dcase["dtype"])
-    out = moe.ffn_forward(dcase["x"], dcase["logits"], dcase["w13"], dcase["s13"], dcase["w2"], dcase["s2"],
-                          dcase["k"], ws=ws)
+    out = moe.ffn_forward(dcase["x"], dcase["logits"], dcase["w13"], dcase["s13"], dcase["w2p"], dcase["s2"],
+                          dcase["k"], dcase["F"], dcase["dtype"] == "fp8", ws=ws)
     st = moe.moe_get_status(None)
     assert st == 0, f"device status {moe.STATUS_NAMES.get(st, st)}"
     return out, ws
@@ -79,7 +79,10 @@ def small_case(T, H=256, F=512, E=8, k=2, dtype="bf16", seed=0, skew=False):
 # against the stated tolerance plus the exact effect of the validated flips of
 # its token, computed from the oracle's w2 and routing weights.
 
-RHO = 2.0 ** -12          # admissible distance of a flipped decision from its boundary (relative)
+RHO = 2.0 ** -12          # admissible distance of a flipped decision from its boundary (relative) ...
+ABS_FLOOR = 2.0 ** -14    # ... plus this fraction of the row's rms: g and u are sums of ~K terms, so
+                          # fp32 accumulation leaves an absolute error that is large relative to h
+                          # wherever g or u cancels to nearly zero
 MAX_FLIP_FRACTION = 1e-2  # flips allowed per h row (a real defect changes most of a row)
 
 
@@ -123,7 +126,7 @@ def _admissible(v, gpu_val, e_gpu, fp8, floor):
     """Is gpu_val the rounding of some value within RHO of v?  (Rounding is
     monotone, so it suffices to bracket gpu_val between the roundings of the
     window's ends.)"""
-    w = RHO * max(abs(v), floor)
+    w = RHO * abs(v) + RHO * floor
     lo, hi = _quant_h(v - w, e_gpu, fp8), _quant_h(v + w, e_gpu, fp8)
     return min(lo, hi) <= gpu_val <= max(lo, hi)
 
@@ -147,7 +150,7 @@ def verify_layer(moe, ws, out, case, tokens=None, what=""):
         if d.size == 0:
             continue
         assert d.size <= max(2, MAX_FLIP_FRACTION * F), f"{what}: {d.size} h elements differ in assignment {assigns[q]}"
-        floor = 1e-2 * float(np.sqrt(np.mean(rx[q] ** 2)))
+        floor = (ABS_FLOOR / RHO) * float(np.sqrt(np.mean(rx[q] ** 2)))
         for n in d:
             e_gpu = int(gexp[q, n // 32]) if fp8 else 0
             if fp8:

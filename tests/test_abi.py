@@ -80,8 +80,11 @@ def test_null_and_unsupported_before_device(moe):
     # routing and preshuffle argument checks
     assert moe.moe_route(None, 4, 0, 1, None, None, None, None, None, None, None, 0, None) == -1
     assert moe.moe_route(P, 4, 8, 2, None, P, P, P, P, P, None, 0, None) == -1
-    assert moe.moe_prepare_weights(None, P, None, None, P, None, 2, 128, 128, 0, None) == -1
-    assert moe.moe_prepare_weights(P, P, None, None, P, None, 2, 100, 128, 0, None) == -2
+    assert moe.moe_prepare_weights(None, P, None, None, P, P, None, P, 2, 128, 128, 0, None) == -1
+    assert moe.moe_prepare_weights(P, P, None, None, None, P, None, P, 2, 128, 128, 0, None) == -1
+    assert moe.moe_prepare_weights(P, P, None, None, P, P, None, P, 2, 128, 128, 1, None) == -1  # FP8 needs scales
+    assert moe.moe_prepare_weights(P, P, None, None, P, P, None, P, 2, 100, 128, 0, None) == -2
+    assert moe.moe_prepare_weights(P, P, None, None, P + 8, P, None, P, 2, 128, 128, 0, None) == -3
 
 
 def test_options(moe):

@@ -141,24 +141,39 @@ def test_layer_repeat_and_empty(moe):
     import mixture_experts_routed_02_b200 as moe_mod
     # T = 0: valid, nothing to do
     rc = moe_mod.moe_ffn_forward(None, None, dcase["w13"].data_ptr(), dcase["s13"].data_ptr(),
-                                 dcase["w2"].data_ptr(), dcase["s2"].data_ptr(), 0, 256, 512, 8, 2, 1, None,
+                                 dcase["w2p"].data_ptr(), dcase["s2"].data_ptr(), 0, 256, 512, 8, 2, 1, None,
                                  ws.data_ptr(), ws.numel(), None)
     assert rc == 0
 
 
-def test_preshuffle_layout(moe):
-    case = small_case(4, 128, 256, 3, 2, "fp8", 23)
+def _unblock(blocks, E, rows, row_bytes):
+    """Invert the blocked, swizzled weight layout: [E][rows/128][row_bytes/128][128 x 128 B]."""
+    nb, kt = rows // 128, row_bytes // 128
+    b = blocks.reshape(E, nb, kt, 128, 8, 16)
+    r = np.arange(128)[:, None]
+    pc = np.arange(8)[None, :] ^ (r % 8)              # stored position of logical chunk c
+    logical = b[:, :, :, np.arange(128)[:, None], pc, :]  # [E, nb, kt, 128, 8, 16]
+    return logical.transpose(0, 1, 3, 2, 4, 5).reshape(E, rows, row_bytes)
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+def test_preshuffle_layout(moe, dtype):
+    case = small_case(4, 256, 384, 3, 2, dtype, 23)
     d = to_device(case)
-    w13 = d["w13"].view(torch.uint8).cpu().numpy()
-    s13 = d["s13"].cpu().numpy()
-    w1 = case["w1"].view(torch.uint8).numpy()
-    w3 = case["w3"].view(torch.uint8).numpy()
-    for e in range(3):
-        for r in range(512):
-            b, i = divmod(r, 64)
-            src = (w3 if i >= 32 else w1)[e, 32 * b + (i % 32)]
-            np.testing.assert_array_equal(w13[e, r], src)
-            assert s13[e, r] == (case["s3"] if i >= 32 else case["s1"])[e, 32 * b + (i % 32)]
+    eb = 1 if dtype == "fp8" else 2
+    E, F, H = 3, 384, 256
+    w13 = _unblock(d["w13"].cpu().numpy(), E, 2 * F, H * eb)
+    w2 = _unblock(d["w2p"].cpu().numpy(), E, H, F * eb)
+    raw = lambda t: t.contiguous().view(torch.uint8).numpy().reshape(t.shape[0], t.shape[1], -1)  # noqa: E731
+    w1, w3, w2_ref = raw(case["w1"]), raw(case["w3"]), raw(case["w2"])
+    np.testing.assert_array_equal(w2, w2_ref)
+    for r in range(2 * F):
+        b, i = divmod(r, 64)
+        src = (w3 if i >= 32 else w1)[:, 32 * b + (i % 32)]
+        np.testing.assert_array_equal(w13[:, r], src)
+        if dtype == "fp8":
+            np.testing.assert_array_equal(d["s13"][:, r].cpu().numpy(),
+                                          (case["s3"] if i >= 32 else case["s1"])[:, 32 * b + (i % 32)].numpy())
 
 
 def test_host_errors(moe):
