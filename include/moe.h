@@ -149,9 +149,10 @@ typedef enum {
     MOE_WS_PERM = 4,       /* int32 [T*k] */
     MOE_WS_INV_PERM = 5,   /* int32 [T*k] */
     MOE_WS_SLOT_OF = 6,    /* int32 [T*k]: assignment -> row of the expert-padded layout */
-    MOE_WS_XS = 7,         /* gathered activations, one row per padded slot: e4m3 or bf16 [S,H] */
+    MOE_WS_XS = 7,         /* gathered activations, one row per padded slot: e4m3 or bf16 [S,H],
+                              rows H*eb + 128 bytes apart */
     MOE_WS_SX = 8,         /* fp32 [S]: per-row activation scale (FP8) */
-    MOE_WS_H = 9,          /* intermediate h [S,F]: e4m3 or bf16 */
+    MOE_WS_H = 9,          /* intermediate h [S,F]: e4m3 or bf16, rows F*eb + 128 bytes apart */
     MOE_WS_H_SF = 10,      /* UE8M0 block scales of h (FP8), tiled for the tensor cores */
     MOE_WS_OUT32 = 11,     /* fp32 [T,H] combine buffer */
     MOE_WS_NUM_MTILES = 12, /* int32: number of 128-row tiles in the padded layout */

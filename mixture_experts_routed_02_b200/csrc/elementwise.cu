@@ -27,7 +27,7 @@ __global__ void __launch_bounds__(128) gather_kernel(const __nv_bfloat16* __rest
     const int tid = threadIdx.x;
     const int a = slot_assign[s];
     const int eb = kFP8 ? 1 : 2;
-    uint8_t* row_out = xs + (size_t)s * H * eb;
+    uint8_t* row_out = xs + (size_t)s * act_pitch((long)H * eb);
     const int nvec_out = H * eb / 16;
     if (a < 0 || a / k >= T) {
         if (a >= 0) record_error(status, MOE_ERR_DEVICE_BOUNDS);

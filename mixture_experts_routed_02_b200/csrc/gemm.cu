@@ -52,6 +52,12 @@ struct Cfg {
     static constexpr uint32_t IDESC = FP8 ? idesc_e4m3(kBlockM, BN) : idesc_bf16(kBlockM, BN);
 };
 
+// SiLU(g) = g / (1 + e^-g) (glossary entry "SwiGLU").  The quotient uses the
+// fast division (at most 2 ulp, far below the bf16 rounding that follows):
+// the correctly rounded division made the epilogue slower than the main loop.
+// For g -> -inf the denominator overflows to +inf and the result is -0.
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
 __device__ __forceinline__ void decode_tile(int tile, int num_mt, int n_tiles, int& m, int& n, int& split) {
     m = tile % num_mt;
     const int r = tile / num_mt;
@@ -247,12 +253,20 @@ __global__ void __launch_bounds__(192, 1)
                     const int hcol = n * (BN / 2) + g * 32;
                     float hv[32];
                     if constexpr (FP8) {
-                        const float* cs = args.col_scale + (size_t)e * args.rows_b + n * BN + g * 64;
+                        // per-channel scales of the 32 gate and 32 up columns (64 contiguous floats)
+                        const float4* cs4 = reinterpret_cast<const float4*>(args.col_scale + (size_t)e * args.rows_b +
+                                                                            n * BN + g * 64);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float gv = __uint_as_float(rg[i]) * sxv * __ldg(cs + i);
-                            const float uv = __uint_as_float(ru[i]) * sxv * __ldg(cs + 32 + i);
-                            hv[i] = __bfloat162float(__float2bfloat16_rn(gv / (1.0f + __expf(-gv)) * uv));
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 sg = __ldg(cs4 + i4), su = __ldg(cs4 + 8 + i4);
+                            const float sgv[4] = {sg.x, sg.y, sg.z, sg.w}, suv[4] = {su.x, su.y, su.z, su.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int i = 4 * i4 + j;
+                                const float gv = __uint_as_float(rg[i]) * (sxv * sgv[j]);
+                                const float uv = __uint_as_float(ru[i]) * (sxv * suv[j]);
+                                hv[i] = __bfloat162float(__float2bfloat16_rn(silu(gv) * uv));
+                            }
                         }
                         float amax = 0.f;
 #pragma unroll
@@ -276,7 +290,7 @@ __global__ void __launch_bounds__(192, 1)
                             packed[i] = (uint32_t)lo | ((uint32_t)hi << 16);
                         }
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) +
-                                                              (size_t)slot * args.out_ld + hcol);
+                                                              (size_t)slot * args.out_pitch + hcol);
                         dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
                         dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
                         args.out_sf[((size_t)m * args.f_tiles + (hcol >> 7)) * 512 + (row & 31) * 16 + (row >> 5) * 4 +
@@ -284,9 +298,7 @@ __global__ void __launch_bounds__(192, 1)
                     } else {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            const float gv = __uint_as_float(rg[i]);
-                            const float uv = __uint_as_float(ru[i]);
-                            hv[i] = gv / (1.0f + __expf(-gv)) * uv;
+                            hv[i] = silu(__uint_as_float(rg[i])) * __uint_as_float(ru[i]);
                         }
                         uint32_t packed[16];
 #pragma unroll
@@ -294,8 +306,8 @@ __global__ void __launch_bounds__(192, 1)
                             __nv_bfloat162 p = __floats2bfloat162_rn(hv[2 * i], hv[2 * i + 1]);
                             packed[i] = *reinterpret_cast<uint32_t*>(&p);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) +
-                                                              (size_t)slot * args.out_ld + hcol);
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) +
+                                                              (size_t)slot * args.out_pitch + hcol * 2);
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
@@ -309,7 +321,8 @@ __global__ void __launch_bounds__(192, 1)
                     t = -1;
                 }
                 const float wgt = (t >= 0) ? args.topk_w[a] : 0.f;
-                float* orow = static_cast<float*>(args.out) + (size_t)(t >= 0 ? t : 0) * args.out_ld;
+                float* orow = reinterpret_cast<float*>(static_cast<uint8_t*>(args.out) +
+                                                       (size_t)(t >= 0 ? t : 0) * args.out_pitch);
 #pragma unroll 1
                 for (int c0 = 0; c0 < BN; c0 += 32) {
                     uint32_t r[32];

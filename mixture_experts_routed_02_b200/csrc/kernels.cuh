@@ -13,6 +13,10 @@ namespace moe {
 constexpr int kMaxExperts = 64;
 constexpr int kMaxTopK = 8;
 constexpr int kBlockM = 128;  // rows per tile of the expert-padded layout
+// Row pitch of the gathered activations and of h: 128 bytes more than a row,
+// so that the 128 rows of an operand tile do not sit a power of two apart
+// (such rows crowd into few L2 slices).
+__host__ __device__ constexpr long act_pitch(long row_bytes) { return row_bytes + 128; }
 
 // Where the router writes.  slot_of / slot_assign / mtile_expert / num_mtiles
 // may be null (routing alone); otherwise they describe the expert-padded row
@@ -61,7 +65,7 @@ struct GemmArgs {
     int n_tiles;              // rows_b / BN
     int k_tiles;              // K / (128 bytes of K)
     int splits;               // K splits (stage 2)
-    int out_ld;               // F (stage 1) or H (stage 2)
+    long out_pitch;           // bytes between output rows: h (stage 1) or out32 (stage 2)
     int f_tiles;              // F / 128: scale tiles per row block of h
     int topk;
     int T;

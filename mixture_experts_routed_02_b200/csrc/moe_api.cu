@@ -127,9 +127,9 @@ Layout make_layout(int T, int H, int F, int E, int k, int dtype) {
     sz[MOE_WS_PERM] = 4 * A;
     sz[MOE_WS_INV_PERM] = 4 * A;
     sz[MOE_WS_SLOT_OF] = 4 * A;
-    sz[MOE_WS_XS] = S * H * eb;
+    sz[MOE_WS_XS] = S * act_pitch((long)H * eb);
     sz[MOE_WS_SX] = 4 * S;
-    sz[MOE_WS_H] = S * F * eb;
+    sz[MOE_WS_H] = S * act_pitch((long)F * eb);
     sz[MOE_WS_H_SF] = (dtype == MOE_FP8_E4M3) ? (size_t)L.MT_max * (F / 128) * 512 : 0;
     sz[MOE_WS_OUT32] = 4 * (size_t)T * H;
     sz[MOE_WS_NUM_MTILES] = 4;
@@ -165,13 +165,14 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D row-major matrix [rows, cols] of elements of `eb` bytes; box = 128 bytes
+// 2-D row-major matrix [rows, cols] of elements of `eb` bytes, rows `pitch`
+// bytes apart; box = 128 bytes
 // of K by box_rows rows, 128-byte swizzle (matches the MMA descriptors).
-bool make_map(CUtensorMap* map, const void* base, size_t rows, size_t cols, int eb, int box_rows) {
+bool make_map(CUtensorMap* map, const void* base, size_t rows, size_t cols, size_t pitch, int eb, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)cols * eb};
+    const cuuint64_t strides[1] = {(cuuint64_t)pitch};
     const cuuint32_t box[2] = {(cuuint32_t)(128 / eb), (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(map, eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
@@ -299,8 +300,8 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     if ((2 * F) % bn1 || H % bn2) return MOE_ERR_UNSUPPORTED;
 
     CUtensorMap ta1, ta2;
-    if (!make_map(&ta1, reg(MOE_WS_XS), L.S_max, H, eb, kBlockM) ||
-        !make_map(&ta2, reg(MOE_WS_H), L.S_max, F, eb, kBlockM))
+    if (!make_map(&ta1, reg(MOE_WS_XS), L.S_max, H, act_pitch((long)H * eb), eb, kBlockM) ||
+        !make_map(&ta2, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, kBlockM))
         return MOE_ERR_CUDA;
 
     // 1. routing and the expert-padded layout
@@ -343,7 +344,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     g1.n_tiles = 2 * F / bn1;
     g1.k_tiles = H * eb / 128;
     g1.splits = 1;
-    g1.out_ld = F;
+    g1.out_pitch = act_pitch((long)F * eb);
     g1.f_tiles = F / 128;
     g1.topk = k;
     g1.T = T;
@@ -372,7 +373,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     const int mt_est = std::min(L.MT_max, (L.A + kBlockM - 1) / kBlockM + std::min(E, L.A));
     g2.splits = choose_splits(mt_est, g2.n_tiles, g2.k_tiles, num_sms);
     if (g2.splits < 1 || g2.k_tiles % g2.splits) return MOE_ERR_UNSUPPORTED;
-    g2.out_ld = H;
+    g2.out_pitch = (long)H * 4;
     const long tiles2 = (long)L.MT_max * g2.n_tiles * g2.splits;
     {
         ProfScope ps(MOE_KERNEL_STAGE2, st);

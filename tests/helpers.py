@@ -99,10 +99,12 @@ def gpu_h_rows(moe, ws, case, assignments):
     slot_of = moe.ws_view(ws, T, H, F, E, k, dc, "slot_of", torch.int32)[:A].cpu().numpy()
     slots = torch.from_numpy(slot_of[np.asarray(assignments)].astype(np.int64)).to(ws.device)
     hreg = moe.ws_view(ws, T, H, F, E, k, dc, "h")
+    eb = 2 if dt == "bf16" else 1
+    pitch = F * eb + 128  # rows of h are 128 bytes longer than their data
+    hrows = hreg.view(-1, pitch)[slots][:, :F * eb].contiguous()
     if dt == "bf16":
-        rows = hreg.view(torch.bfloat16).view(-1, F)[slots].double().cpu().numpy()
-        return rows, None
-    codes = hreg.view(-1, F)[slots].cpu().numpy()
+        return hrows.view(torch.bfloat16).double().cpu().numpy(), None
+    codes = hrows.cpu().numpy()
     sf = moe.ws_view(ws, T, H, F, E, k, dc, "h_sf").cpu().numpy()
     s = slots.cpu().numpy()
     m, row = s // 128, s % 128

@@ -113,7 +113,7 @@ def test_layer_small(moe, p, path):
         # R0: per-token e4m3 codes and scales, bitwise
         xq_ref, sx_ref = oracle.quant_x(nc["x"])
         slot_of = moe.ws_view(ws, T, H, F, E, k, dtc, "slot_of", torch.int32)[:A].cpu().numpy()
-        xs = moe.ws_view(ws, T, H, F, E, k, dtc, "xs").cpu().numpy().reshape(-1, H)
+        xs = moe.ws_view(ws, T, H, F, E, k, dtc, "xs").cpu().numpy().reshape(-1, H + 128)[:, :H]
         sx = moe.ws_view(ws, T, H, F, E, k, dtc, "sx", torch.float32).cpu().numpy()
         for a in range(A):
             t = a // k
