@@ -19,15 +19,15 @@
 //
 // Warp roles (192 threads): warp 0 lane 0 issues TMA loads into an NST-deep
 // shared-memory ring; warp 1 owns TMEM and lane 0 issues the MMAs; warps 2..5
-// drain the two TMEM accumulators (double buffered, so the epilogue of one
-// tile overlaps the main loop of the next).
+// drain the TMEM accumulators (double buffered where TMEM has room, so the
+// epilogue of one tile overlaps the main loop of the next).
 #include "kernels.cuh"
 
 namespace moe {
 
 namespace {
 
-template <int STAGE, bool FP8, int BN, int NST>
+template <int STAGE, bool FP8, int BN, int NST, int NACC>
 struct Cfg {
     static constexpr bool MX = (STAGE == 2) && FP8;
     static constexpr int A_BYTES = kBlockM * 128;
@@ -35,9 +35,9 @@ struct Cfg {
     static constexpr int SF_BYTES = MX ? 512 : 0;
     static constexpr int TX_BYTES = A_BYTES + B_BYTES + SF_BYTES;
     static constexpr int KE = FP8 ? 128 : 64;  // K elements per 128-byte K tile
-    static constexpr int SFA_COL = 2 * BN;
+    static constexpr int SFA_COL = NACC * BN;
     static constexpr int SFB_COL = SFA_COL + 4 * NST;
-    static constexpr int COLS_USED = MX ? SFB_COL + 8 : 2 * BN;
+    static constexpr int COLS_USED = MX ? SFB_COL + 8 : NACC * BN;
     static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
                                    : COLS_USED <= 256 ? 256 : 512;
     static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
@@ -67,10 +67,10 @@ __device__ __forceinline__ void decode_tile(int tile, int num_mt, int n_tiles, i
 
 }  // namespace
 
-template <int STAGE, bool FP8, int BN, int NST>
+template <int STAGE, bool FP8, int BN, int NST, int NACC>
 __global__ void __launch_bounds__(192, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const GemmArgs args) {
-    using C = Cfg<STAGE, FP8, BN, NST>;
+    using C = Cfg<STAGE, FP8, BN, NST, NACC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 if (!ok) break;
                 tc_commit(&tfull[acc]);
-                if (++acc == 2) {
+                if (++acc == NACC) {
                     acc = 0;
                     acc_phase ^= 1;
                 }
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
-            if (++acc == 2) {
+            if (++acc == NACC) {
                 acc = 0;
                 acc_phase ^= 1;
             }
@@ -371,10 +371,10 @@ __global__ void __launch_bounds__(192, 1)
 
 namespace {
 
-template <int STAGE, bool FP8, int BN, int NST>
+template <int STAGE, bool FP8, int BN, int NST, int NACC = 2>
 cudaError_t launch_one(const CUtensorMap& ta, const GemmArgs& args, int grid, cudaStream_t stream) {
-    using C = Cfg<STAGE, FP8, BN, NST>;
-    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST>;
+    using C = Cfg<STAGE, FP8, BN, NST, NACC>;
+    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     kern<<<grid, 192, C::SMEM_BYTES, stream>>>(ta, args);
@@ -384,7 +384,8 @@ cudaError_t launch_one(const CUtensorMap& ta, const GemmArgs& args, int grid, cu
 }  // namespace
 
 int gemm_block_n(int stage, bool fp8, int cfg) {
-    if (stage == 2 && fp8) return 128;
+    (void)stage;
+    (void)fp8;
     return cfg == 0 ? 256 : 128;
 }
 
@@ -396,7 +397,10 @@ cudaError_t launch_gemm(int stage, bool fp8, int cfg, const CUtensorMap& ta, con
         return cfg == 0 ? launch_one<1, false, 256, 4>(ta, args, grid, stream)
                         : launch_one<1, false, 128, 6>(ta, args, grid, stream);
     }
-    if (fp8) return launch_one<2, true, 128, 6>(ta, args, grid, stream);
+    // block-scaled FP8: two 256-column accumulators leave no TMEM for the scale
+    // factors, so the wide tile keeps a single accumulator
+    if (fp8) return cfg == 0 ? launch_one<2, true, 256, 4, 1>(ta, args, grid, stream)
+                             : launch_one<2, true, 128, 6, 2>(ta, args, grid, stream);
     return cfg == 0 ? launch_one<2, false, 256, 4>(ta, args, grid, stream)
                     : launch_one<2, false, 128, 6>(ta, args, grid, stream);
 }
