@@ -177,6 +177,22 @@ def cpu_baseline(spec, name, seconds):
                       f"routing, both expert GEMMs, combine), {dt:.1f} s"}
 
 
+def rank_batch(spec, rank):
+    """Seed of rank r's token batch under weak scaling (the weights are shared)."""
+    return spec["seed"] + 100 * rank
+
+
+def max_over_ranks(value_ms, world, device=None):
+    """Largest elapsed time over all ranks (the timing of a multi-GPU run)."""
+    if world <= 1:
+        return value_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(args, spec, name, rank):
     """The oracle as it stands, on the host cores: each step is one oracle call on
     a small batch of the workload's tokens (sized so the run stays within a
@@ -251,8 +267,8 @@ def main():
     case = moe_inputs.make_case(spec["T"], spec["H"], spec["F"], spec["E"], spec["k"], spec["dtype"], spec["seed"],
                                 spec["skew"])
     if rank > 0:
-        case["x"] = moe_inputs.make_x(spec["T"], spec["H"], spec["seed"] + 100 * rank)
-        case["logits"] = moe_inputs.make_logits(spec["T"], spec["E"], spec["seed"] + 100 * rank, spec["skew"])
+        case["x"] = moe_inputs.make_x(spec["T"], spec["H"], rank_batch(spec, rank))
+        case["logits"] = moe_inputs.make_logits(spec["T"], spec["E"], rank_batch(spec, rank), spec["skew"])
     log(f"[rank {rank}] inputs generated in {time.perf_counter() - t0:.1f} s")
     T, H, F, E, k = spec["T"], spec["H"], spec["F"], spec["E"], spec["k"]
     fp8 = spec["dtype"] == "fp8"
@@ -301,11 +317,7 @@ def main():
     clk = clocks.stop()
     moe.moe_profile_enable(0)
     kern = moe.moe_profile_read(reset=True)
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     st = moe.moe_get_status(None)
     if st != 0:
         raise RuntimeError(f"device status {moe.STATUS_NAMES.get(st, st)} in the timed region")
@@ -333,11 +345,7 @@ def main():
         e2e_step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     e2e_value = T * world * args.steps / (e2e_ms / 1e3)
     del case_x_h
 

@@ -342,3 +342,25 @@ def test_golden_regression_record():
     assert r["perm"].tolist() == g["perm"]
     rows = oracle.moe_ffn_tokens(nc, g["tokens"])
     assert rows["out"].tolist() == g["out_bits"]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_per_assignment_intermediates(dtype):
+    """h_deq of the per-token form equals the routed form's h (sorted order), and
+    rounding h_exact (bf16, then the block quantiser) reproduces h_deq."""
+    case = moe_inputs.make_case(T=7, H=64, F=96, E=4, k=2, dtype=dtype, seed=15)
+    nc = moe_inputs.to_numpy(case)
+    full = oracle.moe_ffn(nc, want_h=True)
+    tok = np.arange(7)
+    sub = oracle.moe_ffn_tokens(nc, tok, want_h=True)
+    r = oracle.route(nc["logits"], 2)
+    for a in range(14):
+        np.testing.assert_array_equal(sub["h_deq"][a], full["h"][r["inv_perm"][a]])
+        hb = _bf16_round_vec(sub["h_exact"][a])
+        if dtype == "bf16":
+            np.testing.assert_array_equal(hb, sub["h_deq"][a])
+        else:
+            for b in range(0, 96, 32):
+                e, codes = oracle.mx_quant_block(hb[b:b + 32])
+                np.testing.assert_array_equal([oracle.e4m3_to_double(c) * 2.0 ** e for c in codes],
+                                              sub["h_deq"][a][b:b + 32])
