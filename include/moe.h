@@ -133,6 +133,32 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
                     const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
                     size_t ws_bytes, void* stream);
 
+/*
+ * The layer without a caller-supplied workspace, for callers that cannot
+ * allocate device memory: code running while a stream is captured into a CUDA
+ * graph (no cudaMalloc allowed then), hosts whose device memory belongs to an
+ * allocator they cannot call, runtimes with a fixed memory budget.  The pages
+ * have no counterpart of this entry point; it is a property of this library.
+ *   Arguments, results and numerics are those of moe_ffn_forward; the
+ *   workspace is a device array built into the library,
+ *   moe_static_workspace_bytes() long (64 MiB).  The driver reserves it on
+ *   every GPU that loads the library's device code and keeps it until the
+ *   process exits.  This call allocates nothing.
+ *   Returns MOE_ERR_WORKSPACE, before enqueuing anything, when the problem
+ *   needs more than that (moe_workspace_size(T,H,F,E,k,dtype) bytes); decode
+ *   batches of Mixtral-8x7B experts fit (T = 16: about 23 MB FP8, 45 MB BF16).
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before capturing a stream.
+ *   All calls on a device share the one array, which keeps the last call's
+ *   contents (every call rewrites all it reads; nothing needs to start at
+ *   zero).  Calls whose work overlaps on the GPU -- e.g. on two streams at
+ *   once -- race on it and give undefined results; serialise them.
+ */
+int moe_ffn_forward_static(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
+                           const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* stream);
+size_t moe_static_workspace_bytes(void);
+
 /* Waits for `stream`, then returns and clears the device status word:
  * MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BOUNDS, or MOE_ERR_CUDA when
  * the wait itself failed. */

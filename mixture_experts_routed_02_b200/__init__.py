@@ -40,7 +40,8 @@ WS = dict(topk_ids=0, topk_w=1, counts=2, offsets=3, perm=4, inv_perm=5, slot_of
 
 # every symbol include/moe.h declares
 EXPORTS = ["moe_workspace_size", "moe_prepare_weights", "moe_route", "moe_ffn_forward", "moe_get_status",
-           "moe_workspace_region", "moe_set_option", "moe_profile_enable", "moe_profile_read"]
+           "moe_workspace_region", "moe_set_option", "moe_profile_enable", "moe_profile_read",
+           "moe_ffn_forward_static", "moe_static_workspace_bytes"]
 KERNELS = ["route", "gather", "stage1_w13_swiglu", "stage2_w2_scatter", "finalize"]
 
 
@@ -69,6 +70,10 @@ lib.moe_get_status.restype = _I
 lib.moe_get_status.argtypes = [_P]
 lib.moe_set_option.restype = _I
 lib.moe_set_option.argtypes = [_I, _I]
+lib.moe_ffn_forward_static.restype = _I
+lib.moe_ffn_forward_static.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
+lib.moe_static_workspace_bytes.restype = _Z
+lib.moe_static_workspace_bytes.argtypes = []
 lib.moe_profile_enable.restype = _I
 lib.moe_profile_enable.argtypes = [_I]
 lib.moe_profile_read.restype = _I
@@ -82,6 +87,8 @@ moe_ffn_forward = lib.moe_ffn_forward
 moe_get_status = lib.moe_get_status
 moe_set_option = lib.moe_set_option
 moe_profile_enable = lib.moe_profile_enable
+moe_ffn_forward_static = lib.moe_ffn_forward_static
+moe_static_workspace_bytes = lib.moe_static_workspace_bytes
 
 
 def moe_profile_read(reset=True):

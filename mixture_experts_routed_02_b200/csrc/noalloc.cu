@@ -1,0 +1,65 @@
+// noalloc.cu -- moe_ffn_forward_static: the MoE layer for callers that cannot
+// allocate device memory.
+//
+// Some callers have no way to obtain a workspace: code that runs while a CUDA
+// stream is being captured into a graph (cudaMalloc is not allowed then), hosts
+// whose device memory is owned by another allocator they cannot call into, and
+// runtimes with a fixed, up-front memory budget.  For them this entry point
+// uses a workspace that is part of the library itself: a file-scope device
+// array of kStaticWorkspaceBytes.  The driver reserves it on a GPU when the
+// library's device code is loaded there, and it stays reserved until the
+// process exits.  Everything else is the ordinary layer call: this file only
+// supplies the buffer to moe_ffn_forward.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+// 64 MiB: enough for decode-sized batches of Mixtral-8x7B experts (T = 16,
+// d_model 4096, d_ff 14336, 8 experts, top-2 needs about 23 MB in FP8 and
+// 45 MB in BF16).
+constexpr size_t kStaticWorkspaceBytes = size_t(64) << 20;
+
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+constexpr int kMaxStaticDevices = 64;
+void* g_static_ptr[kMaxStaticDevices] = {nullptr};
+std::mutex g_static_mutex;
+
+// Device address of this device's copy of the array.  In host code the
+// array's name is only a stand-in, so the address is looked up, once per
+// device, with that device current.
+int static_workspace(void** ptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxStaticDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_mutex);
+    if (!g_static_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+        g_static_ptr[dev] = p;
+    }
+    *ptr = g_static_ptr[dev];
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" size_t moe_static_workspace_bytes(void) { return moe::kStaticWorkspaceBytes; }
+
+extern "C" int moe_ffn_forward_static(const void* x, const float* logits, const void* w13, const float* s13,
+                                      const void* w2, const float* s2, int T, int H, int F, int E, int k, int dtype,
+                                      void* out, void* stream) {
+    const size_t need = moe_workspace_size(T, H, F, E, k, dtype);
+    if (need == 0) return MOE_ERR_INVALID_ARG;
+    if (need > moe::kStaticWorkspaceBytes) return MOE_ERR_WORKSPACE;
+    void* ws = nullptr;
+    const int rc = moe::static_workspace(&ws);
+    if (rc != MOE_OK) return rc;
+    return moe_ffn_forward(x, logits, w13, s13, w2, s2, T, H, F, E, k, dtype, out, ws, moe::kStaticWorkspaceBytes,
+                           stream);
+}
