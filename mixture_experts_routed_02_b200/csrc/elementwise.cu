@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(128) gather_kernel(const __nv_bfloat16* __rest
                                                      const int* __restrict__ slot_assign, uint8_t* __restrict__ xs,
                                                      float* __restrict__ sx_slot, float* __restrict__ out32,
                                                      int* __restrict__ status) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int s = blockIdx.x;
     if (s >= *num_mtiles * kBlockM) return;
     const int tid = threadIdx.x;
@@ -89,14 +91,16 @@ cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k,
                           const int* slot_assign, uint8_t* xs, float* sx_slot, float* out32, int* status,
                           cudaStream_t stream) {
     if (fp8)
-        gather_kernel<true><<<S_max, 128, 0, stream>>>(x, T, H, k, num_mtiles, slot_assign, xs, sx_slot, out32, status);
-    else
-        gather_kernel<false><<<S_max, 128, 0, stream>>>(x, T, H, k, num_mtiles, slot_assign, xs, sx_slot, out32, status);
-    return cudaGetLastError();
+        return launch_dependent(gather_kernel<true>, dim3(S_max), dim3(128), 0, stream, x, T, H, k, num_mtiles,
+                                slot_assign, xs, sx_slot, out32, status);
+    return launch_dependent(gather_kernel<false>, dim3(S_max), dim3(128), 0, stream, x, T, H, k, num_mtiles,
+                            slot_assign, xs, sx_slot, out32, status);
+
 }
 
 // out = bf16(out32), round to nearest even; n is a multiple of 8.
 __global__ void finalize_kernel(const float* __restrict__ out32, __nv_bfloat16* __restrict__ out, size_t n) {
+    griddep_wait();
     const size_t nv = n / 8;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nv; i += (size_t)gridDim.x * blockDim.x) {
         const float4 a = __ldg(reinterpret_cast<const float4*>(out32) + 2 * i);
@@ -155,8 +159,7 @@ __global__ void interleave_scales_kernel(const float* __restrict__ s1, const flo
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream) {
     const int blocks = (int)std::min<size_t>((n / 8 + 255) / 256, (size_t)num_sms * 8);
     if (blocks == 0) return cudaSuccess;
-    finalize_kernel<<<blocks, 256, 0, stream>>>(out32, out, n);
-    return cudaGetLastError();
+    return launch_dependent(finalize_kernel, dim3(blocks), dim3(256), 0, stream, out32, out, n);
 }
 
 cudaError_t launch_preshuffle(const uint8_t* a, const uint8_t* b, uint8_t* dst, int E, int src_rows, int dst_rows,

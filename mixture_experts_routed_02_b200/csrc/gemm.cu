@@ -115,15 +115,44 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
+    // The routing tables were written two launches back, so they may be read
+    // before the wait for the previous kernel (see griddep_wait).
     const int num_mt = *args.num_mtiles;
     const int total = num_mt * args.n_tiles * args.splits;
     const int kps = args.k_tiles / args.splits;
+    const int b_nblk = args.rows_b / kWBlockRows;
+    const uint64_t pol_b = args.b_evict_first ? policy_evict_first() : policy_evict_normal();
+    // first weight block of a tile: expert e, row block n*BN/128, K block 0
+    auto weight_base = [&](int e, int n) {
+        return args.b_blocks + (((size_t)e * b_nblk + n * (BN / kWBlockRows)) * args.k_tiles) * kWBlockBytes;
+    };
+    auto load_weights = [&](int stage, const uint8_t* bsrc, int kt) {
+#pragma unroll
+        for (int j = 0; j < BN / kWBlockRows; ++j)
+            bulk_load_hint(smem + C::OFF_B + stage * C::B_BYTES + j * kWBlockBytes,
+                           bsrc + ((size_t)j * args.k_tiles + kt) * kWBlockBytes, kWBlockBytes, &full[stage], pol_b);
+    };
+
+    // Weights depend on nothing earlier in the call: the producer puts the
+    // first tile's first weight blocks in flight before waiting for the
+    // previous kernel (whose output is the activation operand).
+    int npre = 0;
+    if (warp == 0 && lane == 0 && (int)blockIdx.x < total) {
+        int m, n, split;
+        decode_tile(blockIdx.x, num_mt, args.n_tiles, m, n, split);
+        const uint8_t* bsrc = weight_base(args.mtile_expert[m], n);
+        npre = min(NST, kps);
+        for (int kk = 0; kk < npre; ++kk) {  // fresh stages: nothing to wait for
+            mbar_arrive_expect_tx(&full[kk], C::TX_BYTES);
+            load_weights(kk, bsrc, split * kps + kk);
+        }
+    }
+    griddep_wait();
+    griddep_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol_a = policy_evict_last();
-            const uint64_t pol_b = args.b_evict_first ? policy_evict_first() : policy_evict_normal();
-            const int b_nblk = args.rows_b / kWBlockRows;
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
@@ -131,22 +160,18 @@ __global__ void __launch_bounds__(192, 1)
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 int m, n, split;
                 decode_tile(tile, num_mt, args.n_tiles, m, n, split);
-                const int e = args.mtile_expert[m];
-                // first weight block of this tile: expert e, row block n*BN/128, K block 0
-                const uint8_t* bsrc = args.b_blocks + (((size_t)e * b_nblk + n * (BN / kWBlockRows)) * args.k_tiles)
-                                                          * kWBlockBytes;
+                const uint8_t* bsrc = weight_base(args.mtile_expert[m], n);
                 for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, limit, args.status)) {
-                        ok = false;
-                        break;
+                    const bool prefetched = (tile == (int)blockIdx.x) && (kt - split * kps) < npre;
+                    if (!prefetched) {
+                        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, limit, args.status)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+                        load_weights(stage, bsrc, kt);
                     }
-                    mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
                     tma_load_2d(smem + stage * C::A_BYTES, &tmA, &full[stage], kt * C::KE, m * kBlockM, pol_a);
-#pragma unroll
-                    for (int j = 0; j < BN / kWBlockRows; ++j)
-                        bulk_load_hint(smem + C::OFF_B + stage * C::B_BYTES + j * kWBlockBytes,
-                                       bsrc + ((size_t)j * args.k_tiles + kt) * kWBlockBytes, kWBlockBytes,
-                                       &full[stage], pol_b);
                     if constexpr (C::MX)
                         bulk_load(smem + C::OFF_SF + stage * C::SF_BYTES,
                                   args.a_sf + ((size_t)m * args.f_tiles + kt) * 512, 512, &full[stage]);
@@ -323,36 +348,46 @@ __global__ void __launch_bounds__(192, 1)
                 const float wgt = (t >= 0) ? args.topk_w[a] : 0.f;
                 float* orow = reinterpret_cast<float*>(static_cast<uint8_t*>(args.out) +
                                                        (size_t)(t >= 0 ? t : 0) * args.out_pitch);
+                // 64 columns per TMEM wait; the accumulator is released as soon as
+                // the last columns are in registers, before their atomics
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    uint32_t r[32];
-                    tmem_ld_32cols(tbase + c0, r);
+                for (int c0 = 0; c0 < BN; c0 += 64) {
+                    uint32_t r[64];
+                    tmem_ld_32cols(tbase + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+                    tmem_ld_32cols(tbase + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
                     tmem_ld_wait();
+                    if (c0 + 64 == BN) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[acc]);
+                    }
                     if (t >= 0) {
                         const int col = n * BN + c0;
                         const float* cs = FP8 ? args.col_scale + (size_t)e * args.rows_b + col : nullptr;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4) {
+                        for (int i = 0; i < 64; i += 4) {
                             float4 v;
                             v.x = __uint_as_float(r[i]) * wgt;
                             v.y = __uint_as_float(r[i + 1]) * wgt;
                             v.z = __uint_as_float(r[i + 2]) * wgt;
                             v.w = __uint_as_float(r[i + 3]) * wgt;
                             if constexpr (FP8) {
-                                const float4 s = __ldg(reinterpret_cast<const float4*>(cs + i));
-                                v.x *= s.x;
-                                v.y *= s.y;
-                                v.z *= s.z;
-                                v.w *= s.w;
+                                const float4 sc = __ldg(reinterpret_cast<const float4*>(cs + i));
+                                v.x *= sc.x;
+                                v.y *= sc.y;
+                                v.z *= sc.z;
+                                v.w *= sc.w;
                             }
                             atomicAdd(reinterpret_cast<float4*>(orow + col + i), v);
                         }
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
+            if constexpr (STAGE == 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+            }
             if (++acc == NACC) {
                 acc = 0;
                 acc_phase ^= 1;
@@ -377,8 +412,7 @@ cudaError_t launch_one(const CUtensorMap& ta, const GemmArgs& args, int grid, cu
     auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    kern<<<grid, 192, C::SMEM_BYTES, stream>>>(ta, args);
-    return cudaGetLastError();
+    return launch_dependent(kern, dim3(grid), dim3(192), C::SMEM_BYTES, stream, ta, args);
 }
 
 }  // namespace

@@ -26,6 +26,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// A kernel launched with programmatic stream serialization may start while
+// its predecessor in the stream is still running.  griddep_wait() blocks the
+// calling thread until the predecessor grid has completed and its memory is
+// visible (a no-op for an ordinary launch); griddep_launch_dependents() lets
+// the next such kernel be scheduled.  Every kernel of a layer call signals its
+// dependents only after its own wait has returned, so a kernel that starts
+// early may already read what the kernels two or more places before it wrote.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

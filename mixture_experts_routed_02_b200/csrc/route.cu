@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const float* __
     __shared__ int n_mtiles;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_launch_dependents();  // the gather may be scheduled; it waits for this grid
     for (int i = tid; i < kRouteWarps * kMaxExperts; i += kRouteThreads) {
         (&cnt_w[0][0])[i] = 0;
         (&run_w[0][0])[i] = 0;
