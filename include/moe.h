@@ -119,7 +119,8 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float
  *   out      device, [T,H] bf16, written.
  *   ws       device workspace, >= moe_workspace_size(T,H,F,E,k,dtype) bytes;
  *            scratch, contents undefined afterwards (moe_workspace_region
- *            gives the offsets of the intermediate buffers it holds).
+ *            gives the offsets of the intermediate buffers it holds; rows of
+ *            the padded layout that hold no assignment are left unspecified).
  * Numerics: products accumulate in fp32 on the tensor cores.  FP8 mode:
  * x is quantised per token (sx = absmax/448 in IEEE fp32, e4m3 round to
  * nearest even with saturation); the intermediate h is rounded to bf16 and

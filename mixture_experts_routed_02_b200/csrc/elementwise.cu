@@ -13,30 +13,27 @@
 
 namespace moe {
 
-// One CTA (128 threads) per row of the padded layout.  Rows past the last
-// tile are skipped; padding rows are written as zeros so the tensor cores see
-// finite values there.
+// One CTA (128 threads) per assignment a = t*k + j: copies (bf16) or
+// quantises (FP8) token t's row into a's row of the expert-padded layout.
+// Padding rows are not written: the tensor cores compute each output row from
+// its own input row only, and the outputs of padding rows are discarded.  The
+// CTA of each token's first assignment also zeroes the token's fp32 combine row.
 template <bool kFP8>
 __global__ void __launch_bounds__(128) gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int k,
-                                                     const int* __restrict__ num_mtiles,
-                                                     const int* __restrict__ slot_assign, uint8_t* __restrict__ xs,
+                                                     const int* __restrict__ slot_of, uint8_t* __restrict__ xs,
                                                      float* __restrict__ sx_slot, float* __restrict__ out32,
                                                      int* __restrict__ status) {
     griddep_wait();
     griddep_launch_dependents();
-    const int s = blockIdx.x;
-    if (s >= *num_mtiles * kBlockM) return;
+    const int a = blockIdx.x;
     const int tid = threadIdx.x;
-    const int a = slot_assign[s];
+    const int s = slot_of[a];
     const int eb = kFP8 ? 1 : 2;
-    uint8_t* row_out = xs + (size_t)s * act_pitch((long)H * eb);
-    const int nvec_out = H * eb / 16;
-    if (a < 0 || a / k >= T) {
-        if (a >= 0) record_error(status, MOE_ERR_DEVICE_BOUNDS);
-        for (int i = tid; i < nvec_out; i += 128) reinterpret_cast<uint4*>(row_out)[i] = make_uint4(0, 0, 0, 0);
-        if (kFP8 && tid == 0) sx_slot[s] = 0.f;
+    if (s < 0) {
+        if (tid == 0) record_error(status, MOE_ERR_DEVICE_BOUNDS);
         return;
     }
+    uint8_t* row_out = xs + (size_t)s * act_pitch((long)H * eb);
     const int t = a / k;
     if (a % k == 0) {
         float4* o = reinterpret_cast<float4*>(out32 + (size_t)t * H);
@@ -87,15 +84,14 @@ __global__ void __launch_bounds__(128) gather_kernel(const __nv_bfloat16* __rest
     }
 }
 
-cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, int S_max, const int* num_mtiles,
-                          const int* slot_assign, uint8_t* xs, float* sx_slot, float* out32, int* status,
-                          cudaStream_t stream) {
+cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
+                          float* sx_slot, float* out32, int* status, cudaStream_t stream) {
+    const int A = T * k;
     if (fp8)
-        return launch_dependent(gather_kernel<true>, dim3(S_max), dim3(128), 0, stream, x, T, H, k, num_mtiles,
-                                slot_assign, xs, sx_slot, out32, status);
-    return launch_dependent(gather_kernel<false>, dim3(S_max), dim3(128), 0, stream, x, T, H, k, num_mtiles,
-                            slot_assign, xs, sx_slot, out32, status);
-
+        return launch_dependent(gather_kernel<true>, dim3(A), dim3(128), 0, stream, x, T, H, k, slot_of, xs, sx_slot,
+                                out32, status);
+    return launch_dependent(gather_kernel<false>, dim3(A), dim3(128), 0, stream, x, T, H, k, slot_of, xs, sx_slot, out32,
+                            status);
 }
 
 // out = bf16(out32), round to nearest even; n is a multiple of 8.

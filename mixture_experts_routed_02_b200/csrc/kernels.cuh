@@ -57,9 +57,8 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 
 // Host launchers (each defined next to its kernel).
 cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream);
-cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, int S_max, const int* num_mtiles,
-                          const int* slot_assign, uint8_t* xs, float* sx_slot, float* out32, int* status,
-                          cudaStream_t stream);
+cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
+                          float* sx_slot, float* out32, int* status, cudaStream_t stream);
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream);
 // Blocked, pre-swizzled weight layout (see moe_prepare_weights in moe.h).
 constexpr int kWBlockRows = 128;

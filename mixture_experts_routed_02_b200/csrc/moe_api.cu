@@ -322,8 +322,8 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     float* sx = reinterpret_cast<float*>(reg(MOE_WS_SX));
     {
         ProfScope ps(MOE_KERNEL_GATHER, st);
-        if (launch_gather(fp8, static_cast<const __nv_bfloat16*>(x), T, H, k, L.S_max, num_mt, o.slot_assign,
-                          reg(MOE_WS_XS), sx, out32, status, st) != cudaSuccess)
+        if (launch_gather(fp8, static_cast<const __nv_bfloat16*>(x), T, H, k, o.slot_of, reg(MOE_WS_XS), sx, out32,
+                          status, st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 

@@ -13,8 +13,6 @@ namespace moe {
 
 namespace {
 
-constexpr int kRouteThreads = 1024;
-constexpr int kRouteWarps = kRouteThreads / 32;
 
 __device__ __forceinline__ float rank_value(float v) { return isnan(v) ? -INFINITY : v; }
 
@@ -26,8 +24,10 @@ __device__ __forceinline__ float rank_value(float v) { return isnan(v) ? -INFINI
 // gives every warp its base position per expert.  Phase 4: warps revisit their
 // range and place each assignment; within a 32-wide batch __match_any_sync
 // ranks lanes holding the same expert, so the order stays ascending in a.
-__global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const float* __restrict__ logits, int T, int E,
-                                                                 int k, RouteOutputs o) {
+template <int kRouteWarps>
+__global__ void __launch_bounds__(kRouteWarps * 32, 1) route_kernel(const float* __restrict__ logits, int T, int E,
+                                                                    int k, RouteOutputs o) {
+    constexpr int kRouteThreads = kRouteWarps * 32;
     __shared__ int cnt_w[kRouteWarps][kMaxExperts];
     __shared__ int base_w[kRouteWarps][kMaxExperts];
     __shared__ int run_w[kRouteWarps][kMaxExperts];
@@ -166,8 +166,13 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const float* __
     }
 }
 
+// Four warps for small batches (the phases are short and latency-bound), 32
+// for large ones.
 cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream) {
-    route_kernel<<<1, kRouteThreads, 0, stream>>>(logits, T, E, k, o);
+    if ((long)T * k <= 1024)
+        route_kernel<4><<<1, 4 * 32, 0, stream>>>(logits, T, E, k, o);
+    else
+        route_kernel<32><<<1, 32 * 32, 0, stream>>>(logits, T, E, k, o);
     return cudaGetLastError();
 }
 
