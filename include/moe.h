@@ -195,8 +195,13 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
  *   MOE_OPT_SPLITK:   0 = automatic, n > 0 = split the second GEMM's K into n parts
  *                     (must divide F/128).
  *   MOE_OPT_TIMEOUT_MS: limit of every device-side wait (default 2000).
+ *   MOE_OPT_TEST_STALL: 1 = test of the failure path: the first group GEMM
+ *                     leaves out one operand copy of one CTA, so that CTA's
+ *                     bounded waits run out, the call's outputs are undefined
+ *                     and moe_get_status reports MOE_ERR_DEVICE_TIMEOUT; the
+ *                     context stays usable.  0 (default) = off.
  * Returns the previous value, or MOE_ERR_INVALID_ARG. */
-typedef enum { MOE_OPT_PATH = 0, MOE_OPT_SPLITK = 1, MOE_OPT_TIMEOUT_MS = 2 } moe_option;
+typedef enum { MOE_OPT_PATH = 0, MOE_OPT_SPLITK = 1, MOE_OPT_TIMEOUT_MS = 2, MOE_OPT_TEST_STALL = 3 } moe_option;
 int moe_set_option(int option, int value);
 
 /* Per-kernel device timing (tracing aid).  While enabled, moe_ffn_forward

@@ -171,7 +171,11 @@ __global__ void __launch_bounds__(192, 1)
                         mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
                         load_weights(stage, bsrc, kt);
                     }
-                    tma_load_2d(smem + stage * C::A_BYTES, &tmA, &full[stage], kt * C::KE, m * kBlockM, pol_a);
+                    // failure-detection test hook: CTA 0 leaves the activation
+                    // copy of its first stage out, so that stage never completes
+                    // and the MMA's bounded wait runs out (see MOE_OPT_TEST_STALL)
+                    if (!(args.test_stall && blockIdx.x == 0 && issued == 0))
+                        tma_load_2d(smem + stage * C::A_BYTES, &tmA, &full[stage], kt * C::KE, m * kBlockM, pol_a);
                     if constexpr (C::MX)
                         bulk_load(smem + C::OFF_SF + stage * C::SF_BYTES,
                                   args.a_sf + ((size_t)m * args.f_tiles + kt) * 512, 512, &full[stage]);

@@ -90,6 +90,7 @@ struct GemmArgs {
     int T;
     unsigned long long timeout_ns;
     int* status;              // device status word
+    int test_stall;           // test hook: one copy of CTA 0 is left out (its waits must time out)
 };
 
 // Host launchers of the tcgen05 grouped GEMM; defined in gemm.cu.

@@ -26,6 +26,7 @@ namespace {
 std::atomic<int> g_opt_path{0};
 std::atomic<int> g_opt_splitk{0};
 std::atomic<int> g_opt_timeout_ms{2000};
+std::atomic<int> g_opt_test_stall{0};
 
 // ---------------------------------------------------------------- profiling
 
@@ -226,6 +227,9 @@ int moe_set_option(int option, int value) {
         case MOE_OPT_TIMEOUT_MS:
             if (value < 1) return MOE_ERR_INVALID_ARG;
             return g_opt_timeout_ms.exchange(value);
+        case MOE_OPT_TEST_STALL:
+            if (value < 0 || value > 1) return MOE_ERR_INVALID_ARG;
+            return g_opt_test_stall.exchange(value);
         default:
             return MOE_ERR_INVALID_ARG;
     }
@@ -350,6 +354,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     g1.T = T;
     g1.timeout_ns = timeout_ns;
     g1.status = status;
+    g1.test_stall = g_opt_test_stall.load();
     const long tiles1 = (long)L.MT_max * g1.n_tiles;
     {
         ProfScope ps(MOE_KERNEL_STAGE1, st);
@@ -360,6 +365,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     // 4. stage 2: GEMM with w2, weighted scatter-add epilogue
     GemmArgs g2 = g1;
     g2.row_scale = nullptr;
+    g2.test_stall = 0;
     g2.col_scale = fp8 ? s2 : nullptr;
     g2.topk_w = o.topk_w;
     g2.a_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;

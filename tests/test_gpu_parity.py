@@ -82,6 +82,8 @@ SMALL = [
     (37, 128, 256, 1, 1, "fp8", 9, False),      # E = 1, k = 1 (dense SwiGLU MLP)
     (50, 128, 384, 4, 4, "bf16", 10, False),    # k = E
     (129, 384, 640, 16, 3, "fp8", 11, False),   # odd multiples of 128
+    (16, 256, 512, 8, 2, "fp8", 12, False),     # a decode-shaped batch (32 assignments)
+    (16, 256, 512, 8, 2, "bf16", 13, False),
 ]
 
 
