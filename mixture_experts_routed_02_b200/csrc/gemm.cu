@@ -110,6 +110,25 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
     }
+    // Expert-major tile order: the first 128-row tile of each expert (a scan
+    // of the per-expert row counts; written by the routing step, two launches
+    // back, so readable before the wait for the previous kernel).
+    __shared__ int s_mt_first[kMaxExperts + 1];
+    if (args.group_m && warp == 2) {
+        int carry = 0;
+        for (int base = 0; base < args.num_experts; base += 32) {
+            const int e = base + lane;
+            int v = (e < args.num_experts) ? (args.counts[e] + kBlockM - 1) / kBlockM : 0;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, v, d);
+                if (lane >= d) v += y;
+            }
+            if (e < args.num_experts) s_mt_first[e + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (lane == 0) s_mt_first[0] = 0;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -120,6 +139,30 @@ __global__ void __launch_bounds__(192, 1)
     const int num_mt = *args.num_mtiles;
     const int total = num_mt * args.n_tiles * args.splits;
     const int kps = args.k_tiles / args.splits;
+    // Tile -> (m, n, split).  Default: m fastest over all m-tiles, so the CTAs
+    // of a wave that share a weight tile run side by side.  Expert-major
+    // (group_m): all tiles of one expert before the next, m fastest inside it,
+    // so a wave's activation rows and weights are both one expert's and each
+    // is fetched from DRAM about once even when the activations of all
+    // experts together do not fit in L2.
+    auto tile_coords = [&](int tile, int& m, int& n, int& split) {
+        if (args.group_m) {
+            const int ns = args.n_tiles * args.splits;
+            const int e = args.mtile_expert[tile / ns];
+            const int mf = (e >= 0 && e < args.num_experts) ? s_mt_first[e] : 0;
+            const int cnt = (e >= 0 && e < args.num_experts) ? s_mt_first[e + 1] - mf : 0;
+            if (cnt > 0 && tile >= mf * ns && tile < (mf + cnt) * ns) {
+                const int local = tile - mf * ns;
+                m = mf + local % cnt;
+                const int r = local / cnt;
+                n = r % args.n_tiles;
+                split = r / args.n_tiles;
+                return;
+            }
+            record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
+        }
+        decode_tile(tile, num_mt, args.n_tiles, m, n, split);
+    };
     const int b_nblk = args.rows_b / kWBlockRows;
     const uint64_t pol_b = args.b_evict_first ? policy_evict_first() : policy_evict_normal();
     // first weight block of a tile: expert e, row block n*BN/128, K block 0
@@ -139,7 +182,7 @@ __global__ void __launch_bounds__(192, 1)
     int npre = 0;
     if (warp == 0 && lane == 0 && (int)blockIdx.x < total) {
         int m, n, split;
-        decode_tile(blockIdx.x, num_mt, args.n_tiles, m, n, split);
+        tile_coords(blockIdx.x, m, n, split);
         const uint8_t* bsrc = weight_base(args.mtile_expert[m], n);
         npre = min(NST, kps);
         for (int kk = 0; kk < npre; ++kk) {  // fresh stages: nothing to wait for
@@ -159,7 +202,7 @@ __global__ void __launch_bounds__(192, 1)
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 int m, n, split;
-                decode_tile(tile, num_mt, args.n_tiles, m, n, split);
+                tile_coords(tile, m, n, split);
                 const uint8_t* bsrc = weight_base(args.mtile_expert[m], n);
                 for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
                     const bool prefetched = (tile == (int)blockIdx.x) && (kt - split * kps) < npre;
@@ -265,7 +308,7 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             int m, n, split;
-            decode_tile(tile, num_mt, args.n_tiles, m, n, split);
+            tile_coords(tile, m, n, split);
             if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, limit, args.status)) break;
             tc_fence_after();
             const int e = args.mtile_expert[m];

@@ -91,6 +91,9 @@ struct GemmArgs {
     unsigned long long timeout_ns;
     int* status;              // device status word
     int test_stall;           // test hook: one copy of CTA 0 is left out (its waits must time out)
+    int group_m;              // expert-major tile order (see tile_coords in gemm.cu)
+    const int* counts;        // rows per expert [num_experts] (for group_m)
+    int num_experts;
 };
 
 // Host launchers of the tcgen05 grouped GEMM; defined in gemm.cu.

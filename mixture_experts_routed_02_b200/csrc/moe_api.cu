@@ -355,6 +355,9 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     g1.timeout_ns = timeout_ns;
     g1.status = status;
     g1.test_stall = g_opt_test_stall.load();
+    g1.counts = o.counts;
+    g1.num_experts = E;
+    g1.group_m = (cfg1 == 0) ? 1 : 0;
     const long tiles1 = (long)L.MT_max * g1.n_tiles;
     {
         ProfScope ps(MOE_KERNEL_STAGE1, st);
@@ -366,6 +369,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     GemmArgs g2 = g1;
     g2.row_scale = nullptr;
     g2.test_stall = 0;
+    g2.group_m = (cfg2 == 0) ? 1 : 0;
     g2.col_scale = fp8 ? s2 : nullptr;
     g2.topk_w = o.topk_w;
     g2.a_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;
