@@ -191,7 +191,9 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
 
 /* Kernel selection for tests and tuning (host-side setting, process-wide).
  *   MOE_OPT_PATH:     0 = choose by problem size, 1 = force the throughput
- *                     tiles, 2 = force the weight-streaming tiles.
+ *                     tiles (256 x 256 tiles on pairs of SMs), 2 = force the
+ *                     weight-streaming tiles (128 x 128 on one SM), 3 = force
+ *                     128 x 256 tiles on one SM.
  *   MOE_OPT_SPLITK:   0 = automatic, n > 0 = split the second GEMM's K into n parts
  *                     (must divide F/128).
  *   MOE_OPT_TIMEOUT_MS: limit of every device-side wait (default 2000).

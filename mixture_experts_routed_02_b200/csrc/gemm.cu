@@ -21,27 +21,39 @@
 // shared-memory ring; warp 1 owns TMEM and lane 0 issues the MMAs; warps 2..5
 // drain the TMEM accumulators (double buffered where TMEM has room, so the
 // epilogue of one tile overlaps the main loop of the next).
+//
+// CTA pairs (PAIR): a cluster of two CTAs on two SMs computes a 256 x BN tile
+// with tcgen05.mma.cta_group::2.  Its two 128-row halves are two m-tiles of
+// the same expert (the second one repeats the first when the expert has an odd
+// number of m-tiles; that half's results are discarded).  Each CTA loads its
+// own 128 activation rows and one half of the BN weight rows, so per unit of
+// work a CTA moves a third less operand data through L2 and shared memory
+// than a 128 x BN tile on one SM; the even CTA issues the MMAs and every
+// operand load of the pair completes on its barriers.
 #include "kernels.cuh"
 
 namespace moe {
 
 namespace {
 
-template <int STAGE, bool FP8, int BN, int NST, int NACC>
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR>
 struct Cfg {
     static constexpr bool MX = (STAGE == 2) && FP8;
     static constexpr int A_BYTES = kBlockM * 128;
-    static constexpr int B_BYTES = BN * 128;
+    static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // weight rows held by one CTA
+    static constexpr int B_BYTES = B_ROWS * 128;
     static constexpr int SF_BYTES = MX ? 512 : 0;
-    static constexpr int TX_BYTES = A_BYTES + B_BYTES + SF_BYTES;
+    // bytes that complete one stage: both CTAs' copies count on the even CTA's barrier
+    static constexpr int TX_BYTES = (PAIR ? 2 : 1) * (A_BYTES + B_BYTES + SF_BYTES);
     static constexpr int KE = FP8 ? 128 : 64;  // K elements per 128-byte K tile
+    static constexpr int MMA_M = PAIR ? 2 * kBlockM : kBlockM;
     static constexpr int SFA_COL = NACC * BN;
     static constexpr int SFB_COL = SFA_COL + 4 * NST;
     static constexpr int COLS_USED = MX ? SFB_COL + 8 : NACC * BN;
     static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
                                    : COLS_USED <= 256 ? 256 : 512;
     static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
-    static_assert(BN % kWBlockRows == 0 && BN <= 256, "BN: whole 128-row weight blocks");
+    static_assert(B_ROWS % kWBlockRows == 0 && BN <= 256, "BN: whole 128-row weight blocks");
     // shared memory: A ring, B ring, SF ring, constant B scales, barriers
     static constexpr int OFF_B = NST * A_BYTES;
     static constexpr int OFF_SF = OFF_B + NST * B_BYTES;
@@ -49,7 +61,8 @@ struct Cfg {
     static constexpr int OFF_BAR = OFF_SFB + (MX ? 512 : 0);
     static constexpr int NUM_BARS = 2 * NST + 5;
     static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;  // + alignment slack
-    static constexpr uint32_t IDESC = FP8 ? idesc_e4m3(kBlockM, BN) : idesc_bf16(kBlockM, BN);
+    static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+    static constexpr uint32_t IDESC = FP8 ? idesc_e4m3(MMA_M, BN) : idesc_bf16(MMA_M, BN);
 };
 
 // SiLU(g) = g / (1 + e^-g) (glossary entry "SwiGLU").  The quotient uses the
@@ -67,10 +80,11 @@ __device__ __forceinline__ void decode_tile(int tile, int num_mt, int n_tiles, i
 
 }  // namespace
 
-template <int STAGE, bool FP8, int BN, int NST, int NACC>
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
-    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const GemmArgs args) {
-    using C = Cfg<STAGE, FP8, BN, NST, NACC>;
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmSF, const GemmArgs args) {
+    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -84,6 +98,17 @@ __global__ void __launch_bounds__(192, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t limit = args.timeout_ns;
+    // pair: rank 0 (even CTA) issues the MMAs; work units are per cluster
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const bool leader = (rank == 0);
+    const int unit0 = PAIR ? (int)blockIdx.x / 2 : (int)blockIdx.x;
+    const int ustep = PAIR ? (int)gridDim.x / 2 : (int)gridDim.x;
+    // a wait that gives up tells the other CTA of the pair to give up too
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+        const bool ok = mbar_wait(bar, parity, abort_flag, limit, args.status);
+        if (PAIR && !ok) st_cluster_u32(mapa_shared(smem_u32((const void*)abort_flag), rank ^ 1u), 1u);
+        return ok;
+    };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NST; ++i) {
@@ -92,7 +117,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 4);
+            mbar_init(&tempty[i], PAIR ? 8 : 4);  // the epilogue warps of both CTAs release a pair tile
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -104,90 +129,151 @@ __global__ void __launch_bounds__(192, 1)
         fence_proxy_async_smem();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
+        if constexpr (PAIR) {
+            prefetch_tmap(&tmB);
+            if constexpr (C::MX) prefetch_tmap(&tmSF);
+        }
     }
-    // Expert-major tile order: the first 128-row tile of each expert (a scan
-    // of the per-expert row counts; written by the routing step, two launches
-    // back, so readable before the wait for the previous kernel).
+    // Expert-major tile order: the first 128-row tile (and, for pairs, the
+    // first pair of tiles) of each expert, from a scan of the per-expert row
+    // counts (written by the routing step, two launches back, so readable
+    // before the wait for the previous kernel).
     __shared__ int s_mt_first[kMaxExperts + 1];
-    if (args.group_m && warp == 2) {
-        int carry = 0;
+    __shared__ int s_pair_first[kMaxExperts + 1];
+    if ((PAIR || args.group_m) && warp == 2) {
+        int carry = 0, carry_p = 0;
         for (int base = 0; base < args.num_experts; base += 32) {
             const int e = base + lane;
             int v = (e < args.num_experts) ? (args.counts[e] + kBlockM - 1) / kBlockM : 0;
+            int vp = (v + 1) / 2;
 #pragma unroll
             for (int d = 1; d < 32; d <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, v, d);
-                if (lane >= d) v += y;
+                const int yp = __shfl_up_sync(0xffffffffu, vp, d);
+                if (lane >= d) {
+                    v += y;
+                    vp += yp;
+                }
             }
-            if (e < args.num_experts) s_mt_first[e + 1] = carry + v;
+            if (e < args.num_experts) {
+                s_mt_first[e + 1] = carry + v;
+                s_pair_first[e + 1] = carry_p + vp;
+            }
             carry += __shfl_sync(0xffffffffu, v, 31);
+            carry_p += __shfl_sync(0xffffffffu, vp, 31);
         }
-        if (lane == 0) s_mt_first[0] = 0;
+        if (lane == 0) {
+            s_mt_first[0] = 0;
+            s_pair_first[0] = 0;
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrival
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     // The routing tables were written two launches back, so they may be read
     // before the wait for the previous kernel (see griddep_wait).
     const int num_mt = *args.num_mtiles;
-    const int total = num_mt * args.n_tiles * args.splits;
+    const int ns = args.n_tiles * args.splits;
+    const int units = PAIR ? s_pair_first[args.num_experts] * ns : num_mt * ns;
     const int kps = args.k_tiles / args.splits;
-    // Tile -> (m, n, split).  Default: m fastest over all m-tiles, so the CTAs
-    // of a wave that share a weight tile run side by side.  Expert-major
-    // (group_m): all tiles of one expert before the next, m fastest inside it,
-    // so a wave's activation rows and weights are both one expert's and each
-    // is fetched from DRAM about once even when the activations of all
-    // experts together do not fit in L2.
-    auto tile_coords = [&](int tile, int& m, int& n, int& split) {
-        if (args.group_m) {
-            const int ns = args.n_tiles * args.splits;
-            const int e = args.mtile_expert[tile / ns];
-            const int mf = (e >= 0 && e < args.num_experts) ? s_mt_first[e] : 0;
-            const int cnt = (e >= 0 && e < args.num_experts) ? s_mt_first[e + 1] - mf : 0;
-            if (cnt > 0 && tile >= mf * ns && tile < (mf + cnt) * ns) {
-                const int local = tile - mf * ns;
-                m = mf + local % cnt;
+    // Work unit -> (this CTA's m-tile, n, split); `dup` marks the second half
+    // of a pair that repeats the first (its results are not stored).
+    //   Default order: m fastest over all m-tiles, so the CTAs of a wave that
+    //   share a weight tile run side by side.
+    //   Expert-major (group_m, and always for pairs): all tiles of one expert
+    //   before the next, m fastest inside it, so a wave's activation rows and
+    //   weights are both one expert's and each is fetched from DRAM about once
+    //   even when the activations of all experts together do not fit in L2.
+    auto unit_coords = [&](int u, int& m, int& n, int& split, bool& dup) {
+        dup = false;
+        if constexpr (PAIR) {
+            const int p = u / ns;
+            int lo = 0, hi = args.num_experts;  // largest e with s_pair_first[e] <= p
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (s_pair_first[mid] <= p) lo = mid;
+                else hi = mid;
+            }
+            const int e = lo;
+            const int cnt = s_pair_first[e + 1] - s_pair_first[e];
+            if (cnt > 0 && p < s_pair_first[e + 1]) {
+                const int local = u - s_pair_first[e] * ns;
+                const int m0 = s_mt_first[e] + 2 * (local % cnt);
                 const int r = local / cnt;
                 n = r % args.n_tiles;
                 split = r / args.n_tiles;
+                const bool odd = (m0 + 1 >= s_mt_first[e + 1]);
+                m = (rank == 0 || odd) ? m0 : m0 + 1;
+                dup = (rank == 1) && odd;
                 return;
             }
             record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
+            m = 0;
+            n = 0;
+            split = 0;
+            dup = true;
+            return;
+        } else {
+            if (args.group_m) {
+                const int e = args.mtile_expert[u / ns];
+                const int mf = (e >= 0 && e < args.num_experts) ? s_mt_first[e] : 0;
+                const int cnt = (e >= 0 && e < args.num_experts) ? s_mt_first[e + 1] - mf : 0;
+                if (cnt > 0 && u >= mf * ns && u < (mf + cnt) * ns) {
+                    const int local = u - mf * ns;
+                    m = mf + local % cnt;
+                    const int r = local / cnt;
+                    n = r % args.n_tiles;
+                    split = r / args.n_tiles;
+                    return;
+                }
+                record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
+            }
+            decode_tile(u, num_mt, args.n_tiles, m, n, split);
         }
-        decode_tile(tile, num_mt, args.n_tiles, m, n, split);
     };
     const int b_nblk = args.rows_b / kWBlockRows;
     const uint64_t pol_b = args.b_evict_first ? policy_evict_first() : policy_evict_normal();
-    // first weight block of a tile: expert e, row block n*BN/128, K block 0
-    auto weight_base = [&](int e, int n) {
-        return args.b_blocks + (((size_t)e * b_nblk + n * (BN / kWBlockRows)) * args.k_tiles) * kWBlockBytes;
-    };
-    auto load_weights = [&](int stage, const uint8_t* bsrc, int kt) {
+    // This CTA's weight blocks for unit (e, n) at K tile kt: the BN rows of the
+    // tile, or this CTA's half of them in a pair.
+    auto load_weights = [&](int stage, int e, int n, int kt) {
+        const int rb0 = n * (BN / kWBlockRows) + (PAIR ? (int)rank * (C::B_ROWS / kWBlockRows) : 0);
 #pragma unroll
-        for (int j = 0; j < BN / kWBlockRows; ++j)
-            bulk_load_hint(smem + C::OFF_B + stage * C::B_BYTES + j * kWBlockBytes,
-                           bsrc + ((size_t)j * args.k_tiles + kt) * kWBlockBytes, kWBlockBytes, &full[stage], pol_b);
+        for (int j = 0; j < C::B_ROWS / kWBlockRows; ++j) {
+            const size_t blk = ((size_t)e * b_nblk + rb0 + j) * args.k_tiles + kt;
+            uint8_t* dst = smem + C::OFF_B + stage * C::B_BYTES + j * kWBlockBytes;
+            if constexpr (PAIR)
+                tma_load_2d_pair(dst, &tmB, mapa_shared(smem_u32(&full[stage]), 0), 0, (int)(blk * kWBlockRows), pol_b);
+            else
+                bulk_load_hint(dst, args.b_blocks + blk * kWBlockBytes, kWBlockBytes, &full[stage], pol_b);
+        }
     };
 
     // Weights depend on nothing earlier in the call: the producer puts the
-    // first tile's first weight blocks in flight before waiting for the
+    // first unit's first weight blocks in flight before waiting for the
     // previous kernel (whose output is the activation operand).
     int npre = 0;
-    if (warp == 0 && lane == 0 && (int)blockIdx.x < total) {
+    if (warp == 0 && lane == 0 && unit0 < units) {
         int m, n, split;
-        tile_coords(blockIdx.x, m, n, split);
-        const uint8_t* bsrc = weight_base(args.mtile_expert[m], n);
+        bool dup;
+        unit_coords(unit0, m, n, split, dup);
+        const int e = args.mtile_expert[m];
         npre = min(NST, kps);
         for (int kk = 0; kk < npre; ++kk) {  // fresh stages: nothing to wait for
-            mbar_arrive_expect_tx(&full[kk], C::TX_BYTES);
-            load_weights(kk, bsrc, split * kps + kk);
+            if (leader) mbar_arrive_expect_tx(&full[kk], C::TX_BYTES);
+            load_weights(kk, e, n, split * kps + kk);
         }
     }
     griddep_wait();
@@ -200,28 +286,39 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t phase = 0;
             int issued = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            for (int u = unit0; u < units && ok; u += ustep) {
                 int m, n, split;
-                tile_coords(tile, m, n, split);
-                const uint8_t* bsrc = weight_base(args.mtile_expert[m], n);
+                bool dup;
+                unit_coords(u, m, n, split, dup);
+                const int e = args.mtile_expert[m];
                 for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
-                    const bool prefetched = (tile == (int)blockIdx.x) && (kt - split * kps) < npre;
+                    const bool prefetched = (u == unit0) && (kt - split * kps) < npre;
                     if (!prefetched) {
-                        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, limit, args.status)) {
+                        if (!wait(&empty[stage], phase ^ 1)) {
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-                        load_weights(stage, bsrc, kt);
+                        if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+                        load_weights(stage, e, n, kt);
                     }
                     // failure-detection test hook: CTA 0 leaves the activation
                     // copy of its first stage out, so that stage never completes
                     // and the MMA's bounded wait runs out (see MOE_OPT_TEST_STALL)
-                    if (!(args.test_stall && blockIdx.x == 0 && issued == 0))
-                        tma_load_2d(smem + stage * C::A_BYTES, &tmA, &full[stage], kt * C::KE, m * kBlockM, pol_a);
-                    if constexpr (C::MX)
-                        bulk_load(smem + C::OFF_SF + stage * C::SF_BYTES,
-                                  args.a_sf + ((size_t)m * args.f_tiles + kt) * 512, 512, &full[stage]);
+                    const bool skip = args.test_stall && blockIdx.x == 0 && issued == 0;
+                    if constexpr (PAIR) {
+                        const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+                        if (!skip)
+                            tma_load_2d_pair(smem + stage * C::A_BYTES, &tmA, bar, kt * C::KE, m * kBlockM, pol_a);
+                        if constexpr (C::MX)
+                            tma_load_2d_pair(smem + C::OFF_SF + stage * C::SF_BYTES, &tmSF, bar, 0,
+                                             (m * args.f_tiles + kt) * 4, pol_a);
+                    } else {
+                        if (!skip)
+                            tma_load_2d(smem + stage * C::A_BYTES, &tmA, &full[stage], kt * C::KE, m * kBlockM, pol_a);
+                        if constexpr (C::MX)
+                            bulk_load(smem + C::OFF_SF + stage * C::SF_BYTES,
+                                      args.a_sf + ((size_t)m * args.f_tiles + kt) * 512, 512, &full[stage]);
+                    }
                     ++issued;
                     if (++stage == NST) {
                         stage = 0;
@@ -230,73 +327,126 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             // do not leave while copies into this CTA's shared memory are in
-            // flight (this wait ignores the abort flag but keeps its time limit)
+            // flight (these waits ignore the abort flag but keep their time limit)
             volatile int keep_waiting = 0;
-            for (int i = 1; i <= min(issued, NST); ++i) {
-                int s = stage - i;
-                uint32_t ph = phase;
-                if (s < 0) {
-                    s += NST;
-                    ph ^= 1;
+            if constexpr (PAIR) {
+                // a pair's copies complete on the even CTA's barriers: wait
+                // instead until the MMAs have released every stage (which also
+                // means no commit towards this CTA is still on its way)
+                for (int i = 0; i < NST; ++i) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, ok ? &keep_waiting : abort_flag, limit, args.status))
+                        break;
+                    if (++stage == NST) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
                 }
-                mbar_wait(&full[s], ph, &keep_waiting, limit, args.status);
+            } else {
+                for (int i = 1; i <= min(issued, NST); ++i) {
+                    int s = stage - i;
+                    uint32_t ph = phase;
+                    if (s < 0) {
+                        s += NST;
+                        ph ^= 1;
+                    }
+                    mbar_wait(&full[s], ph, &keep_waiting, limit, args.status);
+                }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             if constexpr (C::MX) {
-                for (int c = 0; c < 8; c += 4) tmem_cp_32x128b_x4(tmem_base + C::SFB_COL + c, sdesc_sf(smem_u32(smem + C::OFF_SFB)));
+                for (int c = 0; c < 8; c += 4) {
+                    if constexpr (PAIR)
+                        tmem_cp_32x128b_x4_pair(tmem_base + C::SFB_COL + c, sdesc_sf(smem_u32(smem + C::OFF_SFB)));
+                    else
+                        tmem_cp_32x128b_x4(tmem_base + C::SFB_COL + c, sdesc_sf(smem_u32(smem + C::OFF_SFB)));
+                }
             }
+            // arrival on a barrier of both CTAs (pair) or of this CTA
+            auto commit = [&](uint64_t* bar) {
+                if constexpr (PAIR) {
+                    tc_commit_pair(smem_u32(bar));
+                    tc_commit_pair(mapa_shared(smem_u32(bar), 1));
+                } else {
+                    tc_commit(bar);
+                }
+            };
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, limit, args.status)) break;
+            for (int u = unit0; u < units && ok; u += ustep) {
+                if (!wait(&tempty[acc], acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
                 for (int kk = 0; kk < kps; ++kk) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag, limit, args.status)) {
+                    if (!wait(&full[stage], phase)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + stage * C::A_BYTES);
                     const uint32_t b_addr = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
-                    if constexpr (C::MX)
-                        tmem_cp_32x128b_x4(tmem_base + C::SFA_COL + 4 * stage,
-                                           sdesc_sf(smem_u32(smem + C::OFF_SF + stage * C::SF_BYTES)));
+                    if constexpr (C::MX) {
+                        const uint64_t sd = sdesc_sf(smem_u32(smem + C::OFF_SF + stage * C::SF_BYTES));
+                        if constexpr (PAIR)
+                            tmem_cp_32x128b_x4_pair(tmem_base + C::SFA_COL + 4 * stage, sd);
+                        else
+                            tmem_cp_32x128b_x4(tmem_base + C::SFA_COL + 4 * stage, sd);
+                    }
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t ad = sdesc_sw128(a_addr + ks * 32);
                         const uint64_t bd = sdesc_sw128(b_addr + ks * 32);
                         const uint32_t accum = (kk > 0 || ks > 0) ? 1u : 0u;
-                        if constexpr (C::MX)
-                            mma_mxfp8(d_tmem, ad, bd, idesc_mxe4m3(kBlockM, BN, ks, ks),
-                                      tmem_base + C::SFA_COL + 4 * stage, tmem_base + C::SFB_COL, accum);
-                        else if constexpr (FP8)
-                            mma_fp8(d_tmem, ad, bd, C::IDESC, accum);
-                        else
-                            mma_bf16(d_tmem, ad, bd, C::IDESC, accum);
+                        if constexpr (C::MX) {
+                            const uint32_t id = idesc_mxe4m3(C::MMA_M, BN, ks, ks);
+                            if constexpr (PAIR)
+                                mma_mxfp8_pair(d_tmem, ad, bd, id, tmem_base + C::SFA_COL + 4 * stage,
+                                               tmem_base + C::SFB_COL, accum);
+                            else
+                                mma_mxfp8(d_tmem, ad, bd, id, tmem_base + C::SFA_COL + 4 * stage,
+                                          tmem_base + C::SFB_COL, accum);
+                        } else if constexpr (FP8) {
+                            if constexpr (PAIR) mma_fp8_pair(d_tmem, ad, bd, C::IDESC, accum);
+                            else mma_fp8(d_tmem, ad, bd, C::IDESC, accum);
+                        } else {
+                            if constexpr (PAIR) mma_bf16_pair(d_tmem, ad, bd, C::IDESC, accum);
+                            else mma_bf16(d_tmem, ad, bd, C::IDESC, accum);
+                        }
                     }
-                    tc_commit(&empty[stage]);
+                    commit(&empty[stage]);
                     if (++stage == NST) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
                 if (!ok) break;
-                tc_commit(&tfull[acc]);
+                commit(&tfull[acc]);
                 if (++acc == NACC) {
                     acc = 0;
                     acc_phase ^= 1;
                 }
             }
-            // every MMA issued by this thread has finished before TMEM is released
             volatile int keep_waiting = 0;
-            tc_commit(drain);
+            if constexpr (PAIR) {
+                // both CTAs' epilogues have released every accumulator, so no
+                // arrival from the other CTA is still on its way to this one
+                for (int i = 0; i < NACC; ++i) {
+                    if (!mbar_wait(&tempty[acc], acc_phase ^ 1, ok ? &keep_waiting : abort_flag, limit, args.status))
+                        break;
+                    if (++acc == NACC) {
+                        acc = 0;
+                        acc_phase ^= 1;
+                    }
+                }
+            }
+            // every MMA issued by this thread has finished before TMEM is released
+            if constexpr (PAIR) tc_commit_pair(smem_u32(drain));
+            else tc_commit(drain);
             mbar_wait(drain, 0, &keep_waiting, limit, args.status);
         }
         __syncwarp();
@@ -306,10 +456,20 @@ __global__ void __launch_bounds__(192, 1)
         const int row = q * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        // the accumulator may be overwritten (pairs: the even CTA counts both CTAs' warps)
+        auto release = [&](int a) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[a]), 0));
+                else mbar_arrive(&tempty[a]);
+            }
+        };
+        for (int u = unit0; u < units; u += ustep) {
             int m, n, split;
-            tile_coords(tile, m, n, split);
-            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, limit, args.status)) break;
+            bool dup;
+            unit_coords(u, m, n, split, dup);
+            if (!wait(&tfull[acc], acc_phase)) break;
             tc_fence_after();
             const int e = args.mtile_expert[m];
             const int slot = m * kBlockM + row;
@@ -317,7 +477,7 @@ __global__ void __launch_bounds__(192, 1)
             if constexpr (STAGE == 1) {
                 const float sxv = FP8 ? args.row_scale[slot] : 1.0f;
 #pragma unroll 1
-                for (int g = 0; g < BN / 64; ++g) {
+                for (int g = 0; g < BN / 64 && !dup; ++g) {
                     uint32_t rg[32], ru[32];
                     tmem_ld_32cols(tbase + g * 64, rg);
                     tmem_ld_32cols(tbase + g * 64 + 32, ru);
@@ -385,8 +545,9 @@ __global__ void __launch_bounds__(192, 1)
                             dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
                     }
                 }
+                release(acc);
             } else {
-                const int a = args.slot_assign[slot];
+                const int a = dup ? -1 : args.slot_assign[slot];
                 int t = (a >= 0) ? a / args.topk : -1;
                 if (t >= args.T) {
                     record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
@@ -403,11 +564,7 @@ __global__ void __launch_bounds__(192, 1)
                     tmem_ld_32cols(tbase + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
                     tmem_ld_32cols(tbase + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
                     tmem_ld_wait();
-                    if (c0 + 64 == BN) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&tempty[acc]);
-                    }
+                    if (c0 + 64 == BN) release(acc);
                     if (t >= 0) {
                         const int col = n * BN + c0;
                         const float* cs = FP8 ? args.col_scale + (size_t)e * args.rows_b + col : nullptr;
@@ -430,11 +587,6 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 }
             }
-            if constexpr (STAGE == 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[acc]);
-            }
             if (++acc == NACC) {
                 acc = 0;
                 acc_phase ^= 1;
@@ -445,21 +597,40 @@ __global__ void __launch_bounds__(192, 1)
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();  // no cross-CTA traffic after this point
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+        else tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
+    if constexpr (PAIR) cluster_sync_all();
 }
 
 namespace {
 
-template <int STAGE, bool FP8, int BN, int NST, int NACC = 2>
-cudaError_t launch_one(const CUtensorMap& ta, const GemmArgs& args, int grid, cudaStream_t stream) {
-    using C = Cfg<STAGE, FP8, BN, NST, NACC>;
-    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC>;
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR>
+cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, int grid, cudaStream_t stream) {
+    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR>;
+    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    return launch_dependent(kern, dim3(grid), dim3(192), C::SMEM_BYTES, stream, ta, args);
+    if constexpr (PAIR) {
+        if (grid < 2 || grid % 2) return cudaErrorInvalidValue;
+        if (!maps.b || (C::MX && !maps.sf)) return cudaErrorInvalidValue;
+        return launch_dependent_cluster(kern, dim3(grid), dim3(192), C::SMEM_BYTES, 2, stream, *maps.a, *maps.b,
+                                        C::MX ? *maps.sf : *maps.a, args);
+    } else {
+        return launch_dependent(kern, dim3(grid), dim3(192), C::SMEM_BYTES, stream, *maps.a, *maps.a, *maps.a, args);
+    }
+}
+
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR>
+int max_pairs_one() {
+    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR>;
+    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+        return 0;
+    return max_active_clusters(kern, 192, C::SMEM_BYTES, 2);
 }
 
 }  // namespace
@@ -467,23 +638,34 @@ cudaError_t launch_one(const CUtensorMap& ta, const GemmArgs& args, int grid, cu
 int gemm_block_n(int stage, bool fp8, int cfg) {
     (void)stage;
     (void)fp8;
-    return cfg == 0 ? 256 : 128;
+    return cfg == 1 ? 128 : 256;
 }
 
-cudaError_t launch_gemm(int stage, bool fp8, int cfg, const CUtensorMap& ta, const GemmArgs& args, int grid,
+// cfg 0: CTA pairs, 256 x 256 tiles; cfg 1: one CTA, 128 x 128 tiles
+// (weight streaming); cfg 2: one CTA, 128 x 256 tiles.
+cudaError_t launch_gemm(int stage, bool fp8, int cfg, const GemmMaps& maps, const GemmArgs& args, int grid,
                         cudaStream_t stream) {
     if (stage == 1) {
-        if (fp8) return cfg == 0 ? launch_one<1, true, 256, 4>(ta, args, grid, stream)
-                                 : launch_one<1, true, 128, 6>(ta, args, grid, stream);
-        return cfg == 0 ? launch_one<1, false, 256, 4>(ta, args, grid, stream)
-                        : launch_one<1, false, 128, 6>(ta, args, grid, stream);
+        if (fp8) return cfg == 0 ? launch_one<1, true, 256, 6, 2, true>(maps, args, grid, stream)
+                      : cfg == 1 ? launch_one<1, true, 128, 6, 2, false>(maps, args, grid, stream)
+                                 : launch_one<1, true, 256, 4, 2, false>(maps, args, grid, stream);
+        return cfg == 0 ? launch_one<1, false, 256, 6, 2, true>(maps, args, grid, stream)
+             : cfg == 1 ? launch_one<1, false, 128, 6, 2, false>(maps, args, grid, stream)
+                        : launch_one<1, false, 256, 4, 2, false>(maps, args, grid, stream);
     }
     // block-scaled FP8: two 256-column accumulators leave no TMEM for the scale
-    // factors, so the wide tile keeps a single accumulator
-    if (fp8) return cfg == 0 ? launch_one<2, true, 256, 4, 1>(ta, args, grid, stream)
-                             : launch_one<2, true, 128, 6, 2>(ta, args, grid, stream);
-    return cfg == 0 ? launch_one<2, false, 256, 4>(ta, args, grid, stream)
-                    : launch_one<2, false, 128, 6>(ta, args, grid, stream);
+    // factors, so the wide tiles keep a single accumulator
+    if (fp8) return cfg == 0 ? launch_one<2, true, 256, 6, 1, true>(maps, args, grid, stream)
+                  : cfg == 1 ? launch_one<2, true, 128, 6, 2, false>(maps, args, grid, stream)
+                             : launch_one<2, true, 256, 4, 1, false>(maps, args, grid, stream);
+    return cfg == 0 ? launch_one<2, false, 256, 6, 2, true>(maps, args, grid, stream)
+         : cfg == 1 ? launch_one<2, false, 128, 6, 2, false>(maps, args, grid, stream)
+                    : launch_one<2, false, 256, 4, 2, false>(maps, args, grid, stream);
+}
+
+int gemm_max_pairs(int stage, bool fp8) {
+    if (stage == 1) return fp8 ? max_pairs_one<1, true, 256, 6, 2, true>() : max_pairs_one<1, false, 256, 6, 2, true>();
+    return fp8 ? max_pairs_one<2, true, 256, 6, 1, true>() : max_pairs_one<2, false, 256, 6, 2, true>();
 }
 
 }  // namespace moe

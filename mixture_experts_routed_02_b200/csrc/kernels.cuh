@@ -55,6 +55,47 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The same for a kernel whose CTAs form clusters of `cluster` CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, int cluster,
+                                     cudaStream_t stream, Args&&... args) {
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// How many clusters of `cluster` CTAs of this kernel can be resident at once
+// (0 on error).
+template <typename... KArgs>
+int max_active_clusters(void (*kernel)(KArgs...), int threads, size_t smem, int cluster) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(cluster);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) return 0;
+    return n;
+}
+
 // Host launchers (each defined next to its kernel).
 cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream);
 cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
@@ -96,10 +137,23 @@ struct GemmArgs {
     int num_experts;
 };
 
+// Tensor maps of one GEMM launch: a = activation rows (128-row boxes, 128-byte
+// swizzle); for CTA pairs also b = blocked weights (16 KB boxes) and, for the
+// block-scaled stage 2, sf = h's scale chunks (512-byte boxes).
+struct GemmMaps {
+    const CUtensorMap* a;
+    const CUtensorMap* b;
+    const CUtensorMap* sf;
+};
+
 // Host launchers of the tcgen05 grouped GEMM; defined in gemm.cu.
-// cfg: 0 = throughput tiles (BN=256), 1 = weight-streaming tiles (BN=128).
-cudaError_t launch_gemm(int stage, bool fp8, int cfg, const CUtensorMap& ta, const GemmArgs& args, int grid,
+// cfg: 0 = CTA pairs, 256 x 256 tiles (grid even, clusters of 2);
+//      1 = one CTA, 128 x 128 tiles (weight streaming);
+//      2 = one CTA, 128 x 256 tiles.
+cudaError_t launch_gemm(int stage, bool fp8, int cfg, const GemmMaps& maps, const GemmArgs& args, int grid,
                         cudaStream_t stream);
 int gemm_block_n(int stage, bool fp8, int cfg);
+// Resident clusters of the pair kernel of a stage (0 if it cannot run).
+int gemm_max_pairs(int stage, bool fp8);
 
 }  // namespace moe

@@ -74,6 +74,7 @@ struct ProfScope {
 constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices] = {nullptr};
 int g_num_sms[kMaxDevices] = {0};
+int g_max_pairs[kMaxDevices][2][2];  // [device][stage-1][fp8]; valid once g_status_ptr is set
 std::mutex g_dev_mutex;
 
 // Address of this device's status word and its SM count (looked up once per device).
@@ -86,12 +87,22 @@ int device_info(int** status, int* num_sms) {
         if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return MOE_ERR_CUDA;
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+        for (int s = 0; s < 2; ++s)
+            for (int f = 0; f < 2; ++f) g_max_pairs[dev][s][f] = gemm_max_pairs(s + 1, f != 0);
         g_status_ptr[dev] = static_cast<int*>(p);
         g_num_sms[dev] = sms;
     }
     *status = g_status_ptr[dev];
     *num_sms = g_num_sms[dev];
     return MOE_OK;
+}
+
+// Resident CTA pairs of a stage's pair kernel on the current device (after device_info).
+int max_pairs(int stage, bool fp8) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    return g_status_ptr[dev] ? g_max_pairs[dev][stage - 1][fp8 ? 1 : 0] : 0;
 }
 
 // ---------------------------------------------------------------- workspace
@@ -183,6 +194,22 @@ bool make_map(CUtensorMap* map, const void* base, size_t rows, size_t cols, size
     return r == CUDA_SUCCESS;
 }
 
+// Map of a buffer of 128-byte rows copied as they are (no swizzle), box_rows
+// rows per copy: the preshuffled weight blocks (already in the operand's
+// shared-memory image) and the tiled scale chunks of h.
+bool make_map_rows(CUtensorMap* map, const void* base, size_t rows, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int launch_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // K splits of the second GEMM: enough work units for every SM when the layer
@@ -219,7 +246,7 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
 int moe_set_option(int option, int value) {
     switch (option) {
         case MOE_OPT_PATH:
-            if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+            if (value < 0 || value > 3) return MOE_ERR_INVALID_ARG;
             return g_opt_path.exchange(value);
         case MOE_OPT_SPLITK:
             if (value < 0) return MOE_ERR_INVALID_ARG;
@@ -294,19 +321,41 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     auto reg = [&](int r) { return w + L.off[r]; };
     const int eb = fp8 ? 1 : 2;
 
-    // weight-streaming tiles when experts see few rows on average
+    // Tile configuration (see launch_gemm): weight-streaming tiles when experts
+    // see at most 64 rows on average; CTA pairs from 512 rows per expert on
+    // (below that, an expert's last, lone 128-row tile makes the pairs compute
+    // too many rows twice); one-CTA 128 x 256 tiles in between and where the
+    // pair kernel cannot be resident; 128-wide tiles when a dimension is not a
+    // multiple of 256.
     int cfg = g_opt_path.load();
-    cfg = (cfg == 0) ? ((L.A <= 64 * E) ? 1 : 0) : cfg - 1;
-    const int cfg1 = ((2 * F) % gemm_block_n(1, fp8, cfg) == 0) ? cfg : 1;
-    const int cfg2 = (H % gemm_block_n(2, fp8, cfg) == 0) ? cfg : 1;  // 128-wide tiles when d_model % 256 != 0
+    cfg = (cfg == 0) ? ((L.A <= 64 * E) ? 1 : (L.A < 512 * E) ? 2 : 0) : cfg - 1;
+    int cfg1 = ((2 * F) % gemm_block_n(1, fp8, cfg) == 0) ? cfg : 1;
+    int cfg2 = (H % gemm_block_n(2, fp8, cfg) == 0) ? cfg : 1;
+    if (cfg1 == 0 && max_pairs(1, fp8) < 1) cfg1 = 2;
+    if (cfg2 == 0 && max_pairs(2, fp8) < 1) cfg2 = 2;
     const int bn1 = gemm_block_n(1, fp8, cfg1);
     const int bn2 = gemm_block_n(2, fp8, cfg2);
     if ((2 * F) % bn1 || H % bn2) return MOE_ERR_UNSUPPORTED;
 
-    CUtensorMap ta1, ta2;
+    CUtensorMap ta1, ta2, tb1, tb2, tsf2;
     if (!make_map(&ta1, reg(MOE_WS_XS), L.S_max, H, act_pitch((long)H * eb), eb, kBlockM) ||
         !make_map(&ta2, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, kBlockM))
         return MOE_ERR_CUDA;
+    if (cfg1 == 0 && !make_map_rows(&tb1, w13, (size_t)E * (2 * F) * (H * eb / 128), kWBlockRows))
+        return MOE_ERR_CUDA;
+    if (cfg2 == 0 && !make_map_rows(&tb2, w2, (size_t)E * H * (F * eb / 128), kWBlockRows)) return MOE_ERR_CUDA;
+    if (cfg2 == 0 && fp8 && !make_map_rows(&tsf2, reg(MOE_WS_H_SF), (size_t)L.MT_max * (F / 128) * 4, 4))
+        return MOE_ERR_CUDA;
+    const GemmMaps maps1{&ta1, cfg1 == 0 ? &tb1 : nullptr, nullptr};
+    const GemmMaps maps2{&ta2, cfg2 == 0 ? &tb2 : nullptr, (cfg2 == 0 && fp8) ? &tsf2 : nullptr};
+    // grid: one CTA per SM at most; pairs: whole clusters that can be resident
+    auto grid_for = [&](int stage, int c, long units_per_mtile) {
+        if (c == 0) {
+            const long clusters = std::min<long>((long)max_pairs(stage, fp8), (long)L.MT_max * units_per_mtile);
+            return (int)(2 * std::max<long>(clusters, 1));
+        }
+        return (int)std::min<long>((long)L.MT_max * units_per_mtile, num_sms);
+    };
 
     // 1. routing and the expert-padded layout
     RouteOutputs o{reinterpret_cast<int32_t*>(reg(MOE_WS_TOPK_IDS)), reinterpret_cast<float*>(reg(MOE_WS_TOPK_W)),
@@ -357,11 +406,10 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     g1.test_stall = g_opt_test_stall.load();
     g1.counts = o.counts;
     g1.num_experts = E;
-    g1.group_m = (cfg1 == 0) ? 1 : 0;
-    const long tiles1 = (long)L.MT_max * g1.n_tiles;
+    g1.group_m = (cfg1 != 1) ? 1 : 0;
     {
         ProfScope ps(MOE_KERNEL_STAGE1, st);
-        if (launch_gemm(1, fp8, cfg1, ta1, g1, (int)std::min<long>(tiles1, num_sms), st) != cudaSuccess)
+        if (launch_gemm(1, fp8, cfg1, maps1, g1, grid_for(1, cfg1, g1.n_tiles), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 
@@ -369,7 +417,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     GemmArgs g2 = g1;
     g2.row_scale = nullptr;
     g2.test_stall = 0;
-    g2.group_m = (cfg2 == 0) ? 1 : 0;
+    g2.group_m = (cfg2 != 1) ? 1 : 0;
     g2.col_scale = fp8 ? s2 : nullptr;
     g2.topk_w = o.topk_w;
     g2.a_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;
@@ -381,13 +429,13 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     g2.n_tiles = H / bn2;
     g2.k_tiles = F * eb / 128;
     const int mt_est = std::min(L.MT_max, (L.A + kBlockM - 1) / kBlockM + std::min(E, L.A));
-    g2.splits = choose_splits(mt_est, g2.n_tiles, g2.k_tiles, num_sms);
+    g2.splits = (cfg2 == 0) ? choose_splits((mt_est + 1) / 2, g2.n_tiles, g2.k_tiles, std::max(1, num_sms / 2))
+                            : choose_splits(mt_est, g2.n_tiles, g2.k_tiles, num_sms);
     if (g2.splits < 1 || g2.k_tiles % g2.splits) return MOE_ERR_UNSUPPORTED;
     g2.out_pitch = (long)H * 4;
-    const long tiles2 = (long)L.MT_max * g2.n_tiles * g2.splits;
     {
         ProfScope ps(MOE_KERNEL_STAGE2, st);
-        if (launch_gemm(2, fp8, cfg2, ta2, g2, (int)std::min<long>(tiles2, num_sms), st) != cudaSuccess)
+        if (launch_gemm(2, fp8, cfg2, maps2, g2, grid_for(2, cfg2, (long)g2.n_tiles * g2.splits), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 

@@ -84,6 +84,8 @@ SMALL = [
     (129, 384, 640, 16, 3, "fp8", 11, False),   # odd multiples of 128
     (16, 256, 512, 8, 2, "fp8", 12, False),     # a decode-shaped batch (32 assignments)
     (16, 256, 512, 8, 2, "bf16", 13, False),
+    (1000, 256, 512, 4, 2, "fp8", 14, False),   # 4 tiles per expert: whole CTA pairs
+    (700, 256, 512, 4, 2, "bf16", 15, False),   # 3 tiles per expert: a pair and a lone tile
 ]
 
 
@@ -92,7 +94,7 @@ def _ids(p):
     return f"T{T}_H{H}_F{F}_E{E}_k{k}_{dt}" + ("_skew" if skew else "")
 
 
-@pytest.mark.parametrize("path", [1, 2], ids=["throughput_tiles", "streaming_tiles"])
+@pytest.mark.parametrize("path", [1, 2, 3], ids=["pair_tiles", "streaming_tiles", "wide_tiles"])
 @pytest.mark.parametrize("p", SMALL, ids=_ids)
 def test_layer_small(moe, p, path):
     T, H, F, E, k, dt, seed, skew = p

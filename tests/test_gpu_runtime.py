@@ -17,9 +17,20 @@ def moe():
     return m
 
 
-def test_stalled_wait_times_out_and_context_survives(moe):
+PATHS = pytest.mark.parametrize("path", [2, 1, 3], ids=["streaming_tiles", "pair_tiles", "wide_tiles"])
+
+
+@pytest.fixture(autouse=True)
+def _reset_path(moe):
+    yield
+    moe.moe_set_option(moe.OPT_PATH, 0)
+
+
+@PATHS
+def test_stalled_wait_times_out_and_context_survives(moe, path):
     case = small_case(64, 256, 512, 8, 2, "fp8", 41)
     d = to_device(case)
+    moe.moe_set_option(moe.OPT_PATH, path)
     old_t = moe.moe_set_option(moe.OPT_TIMEOUT_MS, 50)
     old_s = moe.moe_set_option(moe.OPT_TEST_STALL, 1)
     try:
@@ -35,8 +46,10 @@ def test_stalled_wait_times_out_and_context_survives(moe):
     verify_layer(moe, ws, out, case, what="after a timed-out call")
 
 
+@PATHS
 @pytest.mark.parametrize("dtype", ["fp8", "bf16"])
-def test_cuda_graph_capture_and_replay(moe, dtype):
+def test_cuda_graph_capture_and_replay(moe, dtype, path):
+    moe.moe_set_option(moe.OPT_PATH, path)
     T, H, F, E, k = 48, 256, 512, 8, 2
     case = small_case(T, H, F, E, k, dtype, 42)
     d = to_device(case)
