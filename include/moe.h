@@ -184,7 +184,9 @@ typedef enum {
     MOE_WS_OUT32 = 11,     /* fp32 [T,H] combine buffer */
     MOE_WS_NUM_MTILES = 12, /* int32: number of 128-row tiles in the padded layout */
     MOE_WS_SLOT_ASSIGN = 13, /* int32 [S]: padded row -> assignment, -1 for a padding row */
-    MOE_WS_MTILE_EXPERT = 14 /* int32 [S/128]: 128-row tile -> expert */
+    MOE_WS_MTILE_EXPERT = 14, /* int32 [S/128]: 128-row tile -> expert */
+    MOE_WS_ROUTE_BLOCKS = 15  /* int32 [ceil(T/256), E]: assignments per expert of each 256-token
+                                 block (routing of large batches on many SMs) */
 } moe_ws_region;
 
 long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int which, size_t* bytes);

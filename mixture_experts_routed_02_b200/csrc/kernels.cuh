@@ -34,6 +34,7 @@ struct RouteOutputs {
     int32_t* slot_assign;   // [S_max] padded row -> assignment or -1
     int32_t* mtile_expert;  // [MT_max] tile -> expert
     int32_t* num_mtiles;    // [1]
+    int32_t* blk_counts;    // [ceil(T/256)][E] per-block expert counts (many-CTA routing), or null
 };
 
 // Launch with programmatic stream serialization: the kernel may start while
@@ -99,7 +100,7 @@ int max_active_clusters(void (*kernel)(KArgs...), int threads, size_t smem, int 
 // Host launchers (each defined next to its kernel).
 cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream);
 cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
-                          float* sx_slot, float* out32, int* status, cudaStream_t stream);
+                          float* sx_slot, float* out32, int* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream);
 // Blocked, pre-swizzled weight layout (see moe_prepare_weights in moe.h).
 constexpr int kWBlockRows = 128;

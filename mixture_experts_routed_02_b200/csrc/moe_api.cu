@@ -107,7 +107,7 @@ int max_pairs(int stage, bool fp8) {
 
 // ---------------------------------------------------------------- workspace
 
-constexpr int kRegions = 15;
+constexpr int kRegions = 16;
 
 struct Layout {
     size_t off[kRegions];
@@ -147,6 +147,7 @@ Layout make_layout(int T, int H, int F, int E, int k, int dtype) {
     sz[MOE_WS_NUM_MTILES] = 4;
     sz[MOE_WS_SLOT_ASSIGN] = 4 * S;
     sz[MOE_WS_MTILE_EXPERT] = 4 * (size_t)L.MT_max;
+    sz[MOE_WS_ROUTE_BLOCKS] = 4 * (size_t)((T + 255) / 256) * E;
     size_t off = 0;
     for (int r = 0; r < kRegions; ++r) {
         L.off[r] = off;
@@ -363,7 +364,8 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
                    reinterpret_cast<int32_t*>(reg(MOE_WS_PERM)), reinterpret_cast<int32_t*>(reg(MOE_WS_INV_PERM)),
                    reinterpret_cast<int32_t*>(reg(MOE_WS_SLOT_OF)), reinterpret_cast<int32_t*>(reg(MOE_WS_SLOT_ASSIGN)),
                    reinterpret_cast<int32_t*>(reg(MOE_WS_MTILE_EXPERT)),
-                   reinterpret_cast<int32_t*>(reg(MOE_WS_NUM_MTILES))};
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_NUM_MTILES)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_ROUTE_BLOCKS))};
     {
         ProfScope ps(MOE_KERNEL_ROUTE, st);
         if (launch_route(logits, T, E, k, o, st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -376,7 +378,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     {
         ProfScope ps(MOE_KERNEL_GATHER, st);
         if (launch_gather(fp8, static_cast<const __nv_bfloat16*>(x), T, H, k, o.slot_of, reg(MOE_WS_XS), sx, out32,
-                          status, st) != cudaSuccess)
+                          status, num_sms, st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 

@@ -125,6 +125,50 @@ def test_layer_small(moe, p, path):
             assert sx[slot_of[a]].view(np.uint32) == sx_ref[t].view(np.uint32)
 
 
+def _expected_layout(r, T, E, k):
+    """The expert-padded row layout from the oracle's routing: expert e owns
+    whole 128-row tiles, its assignments first in sorted order, then padding."""
+    counts = r["counts"].astype(np.int64)
+    tiles = -(-counts // 128)
+    mt_start = np.concatenate([[0], np.cumsum(tiles)])
+    A = T * k
+    slot_of = np.empty(A, np.int64)
+    slot_assign = np.full(int(mt_start[-1]) * 128, -1, np.int64)
+    for e in range(E):
+        members = r["perm"][r["offsets"][e]:r["offsets"][e + 1]]
+        slots = mt_start[e] * 128 + np.arange(len(members))
+        slot_of[members] = slots
+        slot_assign[slots] = members
+    mtile_expert = np.repeat(np.arange(E), tiles)
+    return slot_of, slot_assign, mtile_expert, int(mt_start[-1])
+
+
+@pytest.mark.parametrize("T,E,k,seed", [(1024, 8, 2, 51), (1300, 16, 3, 52), (5000, 64, 8, 53), (3000, 8, 1, 54)])
+def test_layer_routing_layout_many_ctas(moe, T, E, k, seed):
+    """Large batches route on many SMs: every routing and layout array of the
+    layer's workspace equals the oracle's routing and the padding rule."""
+    H = F = 128
+    case = small_case(T, H, F, E, k, "fp8", seed)
+    out, ws = run_layer(to_device(case))
+    nc = moe_inputs.to_numpy(case)
+    r = oracle.route(nc["logits"], k)
+    A = T * k
+    view = lambda name: moe.ws_view(ws, T, H, F, E, k, 1, name, torch.int32).cpu().numpy()
+    np.testing.assert_array_equal(view("topk_ids")[:A], r["ids"].reshape(-1))
+    np.testing.assert_allclose(moe.ws_view(ws, T, H, F, E, k, 1, "topk_w", torch.float32)[:A].cpu().numpy(),
+                               r["w"].reshape(-1), rtol=2e-6, atol=1e-7)
+    np.testing.assert_array_equal(view("counts")[:E], r["counts"])
+    np.testing.assert_array_equal(view("offsets")[:E + 1], r["offsets"])
+    np.testing.assert_array_equal(view("perm")[:A], r["perm"])
+    np.testing.assert_array_equal(view("inv_perm")[:A], r["inv_perm"])
+    slot_of, slot_assign, mtile_expert, n_mt = _expected_layout(r, T, E, k)
+    assert int(view("num_mtiles")[0]) == n_mt
+    np.testing.assert_array_equal(view("slot_of")[:A], slot_of)
+    np.testing.assert_array_equal(view("slot_assign")[:n_mt * 128], slot_assign)
+    np.testing.assert_array_equal(view("mtile_expert")[:n_mt], mtile_expert)
+    verify_layer(moe, ws, out, case, tokens=np.array([0, T // 2, T - 1]), what=f"many-CTA routing T={T}")
+
+
 @pytest.mark.parametrize("splits", [2, 4])
 def test_layer_split_k(moe, splits):
     moe.moe_set_option(moe.OPT_PATH, 2)
