@@ -126,12 +126,14 @@ class ClockSampler:
 
 
 def source_sha():
+    """Hash of the sources the grouped-GEMM kernels are compiled from (their
+    translation unit and the headers it includes)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixture_experts_routed_02_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for path in [os.path.join(csrc, n) for n in ("gemm.cu", "kernels.cuh", "ptx.cuh")] + \
+            [os.path.join(ROOT, "include", "moe.h")]:
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode() + f.read())
     return h.hexdigest()[:16]
 
 

@@ -209,7 +209,9 @@ typedef enum { MOE_OPT_PATH = 0, MOE_OPT_SPLITK = 1, MOE_OPT_TIMEOUT_MS = 2, MOE
 int moe_set_option(int option, int value);
 
 /* Per-kernel device timing (tracing aid).  While enabled, moe_ffn_forward
- * records a pair of CUDA events around each kernel it enqueues.
+ * records a pair of CUDA events around each step it enqueues (routing is one
+ * kernel for small batches and two from 1024 tokens on; both are counted in
+ * `launches` and timed together).
  * moe_profile_enable returns the previous setting.  moe_profile_read waits for
  * the recorded events, adds up the elapsed time per kernel into
  * ms_total[MOE_KERNEL_COUNT] and the number of launches into

@@ -82,8 +82,9 @@ __device__ __forceinline__ void decode_tile(int tile, int num_mt, int n_tiles, i
 
 template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
-    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmSF, const GemmArgs args) {
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
+                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmSF,
+                    const GemmArgs args) {
     using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -139,6 +140,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
+        if constexpr (!PAIR) prefetch_tmap(&tmA32);
         if constexpr (PAIR) {
             prefetch_tmap(&tmB);
             if constexpr (C::MX) prefetch_tmap(&tmSF);
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(192, 1)
     // before the wait for the previous kernel).
     __shared__ int s_mt_first[kMaxExperts + 1];
     __shared__ int s_pair_first[kMaxExperts + 1];
-    if ((PAIR || args.group_m) && warp == 2) {
+    if (warp == 2) {
         int carry = 0, carry_p = 0;
         for (int base = 0; base < args.num_experts; base += 32) {
             const int e = base + lane;
@@ -244,6 +246,20 @@ __global__ void __launch_bounds__(192, 1)
             decode_tile(u, num_mt, args.n_tiles, m, n, split);
         }
     };
+    // One-CTA tiles whose m-tile holds at most 32 rows in use (small batches:
+    // a few tokens per expert) copy only those 32 activation rows; the MMA
+    // still reads 128 rows, and the results of the rows not copied (stale
+    // shared memory) belong to padding rows and are discarded.
+    auto a_rows32 = [&](int m) {
+        if constexpr (PAIR) {
+            return false;
+        } else {
+            const int e = args.mtile_expert[m];
+            if (e < 0 || e >= args.num_experts) return false;
+            return args.counts[e] - (m - s_mt_first[e]) * kBlockM <= 32;
+        }
+    };
+    auto stage_tx = [&](bool small) { return C::TX_BYTES - (small ? (kBlockM - 32) * 128 : 0); };
     const int b_nblk = args.rows_b / kWBlockRows;
     const uint64_t pol_b = args.b_evict_first ? policy_evict_first() : policy_evict_normal();
     // This CTA's weight blocks for unit (e, n) at K tile kt: the BN rows of the
@@ -270,9 +286,10 @@ __global__ void __launch_bounds__(192, 1)
         bool dup;
         unit_coords(unit0, m, n, split, dup);
         const int e = args.mtile_expert[m];
+        const uint32_t tx = stage_tx(a_rows32(m));
         npre = min(NST, kps);
         for (int kk = 0; kk < npre; ++kk) {  // fresh stages: nothing to wait for
-            if (leader) mbar_arrive_expect_tx(&full[kk], C::TX_BYTES);
+            if (leader) mbar_arrive_expect_tx(&full[kk], tx);
             load_weights(kk, e, n, split * kps + kk);
         }
     }
@@ -291,6 +308,7 @@ __global__ void __launch_bounds__(192, 1)
                 bool dup;
                 unit_coords(u, m, n, split, dup);
                 const int e = args.mtile_expert[m];
+                const bool small = a_rows32(m);
                 for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
                     const bool prefetched = (u == unit0) && (kt - split * kps) < npre;
                     if (!prefetched) {
@@ -298,7 +316,7 @@ __global__ void __launch_bounds__(192, 1)
                             ok = false;
                             break;
                         }
-                        if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+                        if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx(small));
                         load_weights(stage, e, n, kt);
                     }
                     // failure-detection test hook: CTA 0 leaves the activation
@@ -314,7 +332,8 @@ __global__ void __launch_bounds__(192, 1)
                                              (m * args.f_tiles + kt) * 4, pol_a);
                     } else {
                         if (!skip)
-                            tma_load_2d(smem + stage * C::A_BYTES, &tmA, &full[stage], kt * C::KE, m * kBlockM, pol_a);
+                            tma_load_2d(smem + stage * C::A_BYTES, small ? &tmA32 : &tmA, &full[stage], kt * C::KE,
+                                        m * kBlockM, pol_a);
                         if constexpr (C::MX)
                             bulk_load(smem + C::OFF_SF + stage * C::SF_BYTES,
                                       args.a_sf + ((size_t)m * args.f_tiles + kt) * 512, 512, &full[stage]);
@@ -617,10 +636,12 @@ cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, int grid, cud
     if constexpr (PAIR) {
         if (grid < 2 || grid % 2) return cudaErrorInvalidValue;
         if (!maps.b || (C::MX && !maps.sf)) return cudaErrorInvalidValue;
-        return launch_dependent_cluster(kern, dim3(grid), dim3(192), C::SMEM_BYTES, 2, stream, *maps.a, *maps.b,
-                                        C::MX ? *maps.sf : *maps.a, args);
+        return launch_dependent_cluster(kern, dim3(grid), dim3(192), C::SMEM_BYTES, 2, stream, *maps.a, *maps.a,
+                                        *maps.b, C::MX ? *maps.sf : *maps.a, args);
     } else {
-        return launch_dependent(kern, dim3(grid), dim3(192), C::SMEM_BYTES, stream, *maps.a, *maps.a, *maps.a, args);
+        if (!maps.a32) return cudaErrorInvalidValue;
+        return launch_dependent(kern, dim3(grid), dim3(192), C::SMEM_BYTES, stream, *maps.a, *maps.a32, *maps.a,
+                                *maps.a, args);
     }
 }
 

@@ -99,6 +99,7 @@ int max_active_clusters(void (*kernel)(KArgs...), int threads, size_t smem, int 
 
 // Host launchers (each defined next to its kernel).
 cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream);
+int route_launches(int T, const RouteOutputs& o);  // kernels launch_route enqueues (1 or 2)
 cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
                           float* sx_slot, float* out32, int* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream);
@@ -139,10 +140,12 @@ struct GemmArgs {
 };
 
 // Tensor maps of one GEMM launch: a = activation rows (128-row boxes, 128-byte
-// swizzle); for CTA pairs also b = blocked weights (16 KB boxes) and, for the
-// block-scaled stage 2, sf = h's scale chunks (512-byte boxes).
+// swizzle) and a32 = the same with 32-row boxes (one-CTA tiles); for CTA pairs
+// also b = blocked weights (16 KB boxes) and, for the block-scaled stage 2,
+// sf = h's scale chunks (512-byte boxes).
 struct GemmMaps {
     const CUtensorMap* a;
+    const CUtensorMap* a32;
     const CUtensorMap* b;
     const CUtensorMap* sf;
 };

@@ -32,6 +32,7 @@ std::atomic<int> g_opt_test_stall{0};
 
 struct ProfRecord {
     int kernel;
+    int launches;  // kernel launches between the two events
     cudaEvent_t start, stop;
 };
 std::atomic<int> g_prof_on{0};
@@ -54,8 +55,9 @@ cudaEvent_t prof_event() {
 struct ProfScope {
     int kernel;
     cudaStream_t stream;
+    int launches;
     cudaEvent_t start = nullptr;
-    ProfScope(int k, cudaStream_t s) : kernel(k), stream(s) {
+    ProfScope(int k, cudaStream_t s, int n = 1) : kernel(k), stream(s), launches(n) {
         if (!g_prof_on.load()) return;
         std::lock_guard<std::mutex> lock(g_prof_mutex);
         start = prof_event();
@@ -67,7 +69,7 @@ struct ProfScope {
         cudaEvent_t stop = prof_event();
         if (!stop) return;
         cudaEventRecord(stop, stream);
-        g_prof_records.push_back({kernel, start, stop});
+        g_prof_records.push_back({kernel, launches, start, stop});
     }
 };
 
@@ -322,33 +324,45 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     auto reg = [&](int r) { return w + L.off[r]; };
     const int eb = fp8 ? 1 : 2;
 
-    // Tile configuration (see launch_gemm): weight-streaming tiles when experts
-    // see at most 64 rows on average; CTA pairs from 512 rows per expert on
-    // (below that, an expert's last, lone 128-row tile makes the pairs compute
-    // too many rows twice); one-CTA 128 x 256 tiles in between and where the
-    // pair kernel cannot be resident; 128-wide tiles when a dimension is not a
-    // multiple of 256.
-    int cfg = g_opt_path.load();
-    cfg = (cfg == 0) ? ((L.A <= 64 * E) ? 1 : (L.A < 512 * E) ? 2 : 0) : cfg - 1;
-    int cfg1 = ((2 * F) % gemm_block_n(1, fp8, cfg) == 0) ? cfg : 1;
-    int cfg2 = (H % gemm_block_n(2, fp8, cfg) == 0) ? cfg : 1;
+    // Tile configuration (see launch_gemm), by the average rows per expert:
+    //   <= 64 (decode-sized): the first GEMM on one-CTA 128 x 256 tiles, the
+    //     second on 128 x 128 tiles with K split so that every SM streams
+    //     weights (its long K would leave most SMs idle otherwise);
+    //   up to 512: 128 x 256 tiles for both;
+    //   from 512 on: CTA pairs (below that, an expert's last, lone 128-row
+    //     tile makes a pair compute too many rows twice).
+    // One-CTA 128 x 256 tiles where the pair kernel cannot be resident;
+    // 128-wide tiles when a dimension is not a multiple of 256.
+    const bool small_batch = L.A <= 64 * E;
+    const int opt_path = g_opt_path.load();
+    int cfg1, cfg2;
+    if (opt_path == 0) {
+        cfg1 = (L.A < 512 * E) ? 2 : 0;
+        cfg2 = small_batch ? 1 : cfg1;
+    } else {
+        cfg1 = cfg2 = opt_path - 1;
+    }
+    if ((2 * F) % gemm_block_n(1, fp8, cfg1)) cfg1 = 1;
+    if (H % gemm_block_n(2, fp8, cfg2)) cfg2 = 1;
     if (cfg1 == 0 && max_pairs(1, fp8) < 1) cfg1 = 2;
     if (cfg2 == 0 && max_pairs(2, fp8) < 1) cfg2 = 2;
     const int bn1 = gemm_block_n(1, fp8, cfg1);
     const int bn2 = gemm_block_n(2, fp8, cfg2);
     if ((2 * F) % bn1 || H % bn2) return MOE_ERR_UNSUPPORTED;
 
-    CUtensorMap ta1, ta2, tb1, tb2, tsf2;
+    CUtensorMap ta1, ta2, ta1s, ta2s, tb1, tb2, tsf2;
     if (!make_map(&ta1, reg(MOE_WS_XS), L.S_max, H, act_pitch((long)H * eb), eb, kBlockM) ||
-        !make_map(&ta2, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, kBlockM))
+        !make_map(&ta2, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, kBlockM) ||
+        !make_map(&ta1s, reg(MOE_WS_XS), L.S_max, H, act_pitch((long)H * eb), eb, 32) ||
+        !make_map(&ta2s, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, 32))
         return MOE_ERR_CUDA;
     if (cfg1 == 0 && !make_map_rows(&tb1, w13, (size_t)E * (2 * F) * (H * eb / 128), kWBlockRows))
         return MOE_ERR_CUDA;
     if (cfg2 == 0 && !make_map_rows(&tb2, w2, (size_t)E * H * (F * eb / 128), kWBlockRows)) return MOE_ERR_CUDA;
     if (cfg2 == 0 && fp8 && !make_map_rows(&tsf2, reg(MOE_WS_H_SF), (size_t)L.MT_max * (F / 128) * 4, 4))
         return MOE_ERR_CUDA;
-    const GemmMaps maps1{&ta1, cfg1 == 0 ? &tb1 : nullptr, nullptr};
-    const GemmMaps maps2{&ta2, cfg2 == 0 ? &tb2 : nullptr, (cfg2 == 0 && fp8) ? &tsf2 : nullptr};
+    const GemmMaps maps1{&ta1, &ta1s, cfg1 == 0 ? &tb1 : nullptr, nullptr};
+    const GemmMaps maps2{&ta2, &ta2s, cfg2 == 0 ? &tb2 : nullptr, (cfg2 == 0 && fp8) ? &tsf2 : nullptr};
     // grid: one CTA per SM at most; pairs: whole clusters that can be resident
     auto grid_for = [&](int stage, int c, long units_per_mtile) {
         if (c == 0) {
@@ -367,7 +381,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
                    reinterpret_cast<int32_t*>(reg(MOE_WS_NUM_MTILES)),
                    reinterpret_cast<int32_t*>(reg(MOE_WS_ROUTE_BLOCKS))};
     {
-        ProfScope ps(MOE_KERNEL_ROUTE, st);
+        ProfScope ps(MOE_KERNEL_ROUTE, st, route_launches(T, o));
         if (launch_route(logits, T, E, k, o, st) != cudaSuccess) return MOE_ERR_CUDA;
     }
 
@@ -392,7 +406,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     g1.row_scale = fp8 ? sx : nullptr;
     g1.col_scale = fp8 ? s13 : nullptr;
     g1.b_blocks = static_cast<const uint8_t*>(w13);
-    g1.b_evict_first = (cfg1 == 1) ? 1 : 0;  // weight-streaming tiles read each weight block once
+    g1.b_evict_first = small_batch ? 1 : 0;  // one m-tile per expert: each weight block is read once
     g1.out = reg(MOE_WS_H);
     g1.out_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;
     g1.rows_b = 2 * F;
@@ -424,7 +438,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     g2.topk_w = o.topk_w;
     g2.a_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;
     g2.b_blocks = static_cast<const uint8_t*>(w2);
-    g2.b_evict_first = (cfg2 == 1) ? 1 : 0;
+    g2.b_evict_first = small_batch ? 1 : 0;
     g2.out = out32;
     g2.out_sf = nullptr;
     g2.rows_b = H;
@@ -462,7 +476,7 @@ int moe_profile_read(double* ms_total, int* launches, int reset) {
             continue;
         }
         if (ms_total) ms_total[r.kernel] += ms;
-        if (launches) launches[r.kernel] += 1;
+        if (launches) launches[r.kernel] += r.launches;
     }
     if (reset) {
         for (const ProfRecord& r : g_prof_records) {

@@ -333,8 +333,13 @@ __global__ void __launch_bounds__(kRouteBlockTokens) route_place_kernel(int T, i
 
 // Four warps for small batches (the phases are short and latency-bound), 32
 // for large ones.
+// Large batches with the padded layout: two kernels on many SMs.
+static bool route_many_ctas(int T, const RouteOutputs& o) { return o.blk_counts && o.slot_of && T >= 1024; }
+
+int route_launches(int T, const RouteOutputs& o) { return route_many_ctas(T, o) ? 2 : 1; }
+
 cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream) {
-    if (o.blk_counts && o.slot_of && T >= 1024) {
+    if (route_many_ctas(T, o)) {
         const int nblk = (T + kRouteBlockTokens - 1) / kRouteBlockTokens;
         route_topk_kernel<<<nblk, kRouteBlockTokens, 0, stream>>>(logits, T, E, k, o);
         const cudaError_t err = cudaGetLastError();
