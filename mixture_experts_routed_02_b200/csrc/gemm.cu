@@ -189,8 +189,19 @@ __global__ void __launch_bounds__(192, 1)
     // before the wait for the previous kernel (see griddep_wait).
     const int num_mt = *args.num_mtiles;
     const int ns = args.n_tiles * args.splits;
-    const int units = PAIR ? s_pair_first[args.num_experts] * ns : num_mt * ns;
+    const int tiles = PAIR ? s_pair_first[args.num_experts] * ns : num_mt * ns;
     const int kps = args.k_tiles / args.splits;
+    // Stage 1 on one CTA per tile: when the last wave of tiles would keep at
+    // most a quarter of the CTAs busy, each of its tiles is cut into BN/64
+    // units of 64 weight rows (no K split, so nothing to add up afterwards),
+    // which spreads that wave's weight stream over BN/64 times as many SMs.
+    constexpr int kQ = BN / 64;
+    int full_tiles = tiles;
+    if constexpr (STAGE == 1 && !PAIR && kQ > 1) {
+        const int tail = tiles % (int)gridDim.x;
+        if (tail > 0 && tail * kQ <= (int)gridDim.x) full_tiles = tiles - tail;
+    }
+    const int units = full_tiles + (tiles - full_tiles) * kQ;
     // Work unit -> (this CTA's m-tile, n, split); `dup` marks the second half
     // of a pair that repeats the first (its results are not stored).
     //   Default order: m fastest over all m-tiles, so the CTAs of a wave that
@@ -199,8 +210,15 @@ __global__ void __launch_bounds__(192, 1)
     //   before the next, m fastest inside it, so a wave's activation rows and
     //   weights are both one expert's and each is fetched from DRAM about once
     //   even when the activations of all experts together do not fit in L2.
-    auto unit_coords = [&](int u, int& m, int& n, int& split, bool& dup) {
+    //   q4 >= 0: the unit is 64-row slice q4 of tile `t` (the last wave's cut).
+    auto unit_coords = [&](int u, int& m, int& n, int& split, bool& dup, int& q4) {
         dup = false;
+        q4 = -1;
+        if (u >= full_tiles) {
+            const int v = u - full_tiles;
+            q4 = v % kQ;
+            u = full_tiles + v / kQ;
+        }
         if constexpr (PAIR) {
             const int p = u / ns;
             int lo = 0, hi = args.num_experts;  // largest e with s_pair_first[e] <= p
@@ -259,12 +277,20 @@ __global__ void __launch_bounds__(192, 1)
             return args.counts[e] - (m - s_mt_first[e]) * kBlockM <= 32;
         }
     };
-    auto stage_tx = [&](bool small) { return C::TX_BYTES - (small ? (kBlockM - 32) * 128 : 0); };
+    auto stage_tx = [&](bool small, int q4) {
+        return C::TX_BYTES - (small ? (kBlockM - 32) * 128 : 0) - (q4 >= 0 ? C::B_BYTES - 64 * 128 : 0);
+    };
     const int b_nblk = args.rows_b / kWBlockRows;
     const uint64_t pol_b = args.b_evict_first ? policy_evict_first() : policy_evict_normal();
     // This CTA's weight blocks for unit (e, n) at K tile kt: the BN rows of the
     // tile, or this CTA's half of them in a pair.
-    auto load_weights = [&](int stage, int e, int n, int kt) {
+    auto load_weights = [&](int stage, int e, int n, int kt, int q4) {
+        if (!PAIR && q4 >= 0) {  // 64 rows: one half of one 16 KB block (its pre-swizzled rows 0-63 or 64-127)
+            const size_t blk = ((size_t)e * b_nblk + n * (BN / kWBlockRows) + (q4 >> 1)) * args.k_tiles + kt;
+            bulk_load_hint(smem + C::OFF_B + stage * C::B_BYTES, args.b_blocks + blk * kWBlockBytes + (q4 & 1) * 8192,
+                           8192, &full[stage], pol_b);
+            return;
+        }
         const int rb0 = n * (BN / kWBlockRows) + (PAIR ? (int)rank * (C::B_ROWS / kWBlockRows) : 0);
 #pragma unroll
         for (int j = 0; j < C::B_ROWS / kWBlockRows; ++j) {
@@ -282,15 +308,15 @@ __global__ void __launch_bounds__(192, 1)
     // previous kernel (whose output is the activation operand).
     int npre = 0;
     if (warp == 0 && lane == 0 && unit0 < units) {
-        int m, n, split;
+        int m, n, split, q4;
         bool dup;
-        unit_coords(unit0, m, n, split, dup);
+        unit_coords(unit0, m, n, split, dup, q4);
         const int e = args.mtile_expert[m];
-        const uint32_t tx = stage_tx(a_rows32(m));
+        const uint32_t tx = stage_tx(a_rows32(m), q4);
         npre = min(NST, kps);
         for (int kk = 0; kk < npre; ++kk) {  // fresh stages: nothing to wait for
             if (leader) mbar_arrive_expect_tx(&full[kk], tx);
-            load_weights(kk, e, n, split * kps + kk);
+            load_weights(kk, e, n, split * kps + kk, q4);
         }
     }
     griddep_wait();
@@ -304,9 +330,9 @@ __global__ void __launch_bounds__(192, 1)
             int issued = 0;
             bool ok = true;
             for (int u = unit0; u < units && ok; u += ustep) {
-                int m, n, split;
+                int m, n, split, q4;
                 bool dup;
-                unit_coords(u, m, n, split, dup);
+                unit_coords(u, m, n, split, dup, q4);
                 const int e = args.mtile_expert[m];
                 const bool small = a_rows32(m);
                 for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
@@ -316,8 +342,8 @@ __global__ void __launch_bounds__(192, 1)
                             ok = false;
                             break;
                         }
-                        if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx(small));
-                        load_weights(stage, e, n, kt);
+                        if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx(small, q4));
+                        load_weights(stage, e, n, kt, q4);
                     }
                     // failure-detection test hook: CTA 0 leaves the activation
                     // copy of its first stage out, so that stage never completes
@@ -398,6 +424,11 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int u = unit0; u < units && ok; u += ustep) {
+                int m_, n_, split_, q4;
+                bool dup_;
+                unit_coords(u, m_, n_, split_, dup_, q4);
+                // a 64-row slice: the same MMAs with N = 64
+                const uint32_t idesc = (q4 >= 0) ? ((C::IDESC & ~(0x3Fu << 17)) | ((64u >> 3) << 17)) : C::IDESC;
                 if (!wait(&tempty[acc], acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
@@ -431,10 +462,10 @@ __global__ void __launch_bounds__(192, 1)
                                           tmem_base + C::SFB_COL, accum);
                         } else if constexpr (FP8) {
                             if constexpr (PAIR) mma_fp8_pair(d_tmem, ad, bd, C::IDESC, accum);
-                            else mma_fp8(d_tmem, ad, bd, C::IDESC, accum);
+                            else mma_fp8(d_tmem, ad, bd, idesc, accum);
                         } else {
                             if constexpr (PAIR) mma_bf16_pair(d_tmem, ad, bd, C::IDESC, accum);
-                            else mma_bf16(d_tmem, ad, bd, C::IDESC, accum);
+                            else mma_bf16(d_tmem, ad, bd, idesc, accum);
                         }
                     }
                     commit(&empty[stage]);
@@ -485,9 +516,9 @@ __global__ void __launch_bounds__(192, 1)
             }
         };
         for (int u = unit0; u < units; u += ustep) {
-            int m, n, split;
+            int m, n, split, q4;
             bool dup;
-            unit_coords(u, m, n, split, dup);
+            unit_coords(u, m, n, split, dup, q4);
             if (!wait(&tfull[acc], acc_phase)) break;
             tc_fence_after();
             const int e = args.mtile_expert[m];
@@ -496,10 +527,14 @@ __global__ void __launch_bounds__(192, 1)
             if constexpr (STAGE == 1) {
                 const float sxv = FP8 ? args.row_scale[slot] : 1.0f;
 #pragma unroll 1
-                for (int g = 0; g < BN / 64 && !dup; ++g) {
+                // 64-column groups: all BN / 64 of a tile, or the one of a 64-row slice
+                const int g_first = (q4 >= 0) ? q4 : 0;
+                const int g_count = (q4 >= 0) ? 1 : BN / 64;
+                for (int gi = 0; gi < g_count && !dup; ++gi) {
+                    const int g = g_first + gi;
                     uint32_t rg[32], ru[32];
-                    tmem_ld_32cols(tbase + g * 64, rg);
-                    tmem_ld_32cols(tbase + g * 64 + 32, ru);
+                    tmem_ld_32cols(tbase + gi * 64, rg);
+                    tmem_ld_32cols(tbase + gi * 64 + 32, ru);
                     tmem_ld_wait();
                     const int hcol = n * (BN / 2) + g * 32;
                     float hv[32];

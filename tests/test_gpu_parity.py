@@ -178,6 +178,31 @@ def test_layer_split_k(moe, splits):
     verify_layer(moe, ws, out, case, what=f"split-K {splits}")
 
 
+def _last_wave_sliced(num_mt, T, F, E, k, bn, num_sms):
+    """Whether the first GEMM cuts its last wave into 64-row slices: one CTA per
+    SM at most; a last wave that, cut into bn/64 slices per tile, still fits
+    in the grid."""
+    n_tiles = 2 * F // bn
+    grid = min((-(-T * k // 128) + E) * n_tiles, num_sms)
+    tail = (num_mt * n_tiles) % grid
+    return tail > 0 and tail * (bn // 64) <= grid
+
+
+@pytest.mark.parametrize("path,dt", [(3, "fp8"), (3, "bf16"), (2, "fp8"), (2, "bf16")],
+                         ids=["wide_fp8", "wide_bf16", "streaming_fp8", "streaming_bf16"])
+def test_layer_last_wave_slices(moe, path, dt):
+    """The first GEMM's last, lightly filled wave runs as 64-row weight slices
+    (MMA N = 64); every slice's SwiGLU columns land in the right place."""
+    T, H, F, E, k = 16, 256, 2560, 8, 2
+    moe.moe_set_option(moe.OPT_PATH, path)
+    case = small_case(T, H, F, E, k, dt, 61)
+    out, ws = run_layer(to_device(case))
+    num_mt = int(moe.ws_view(ws, T, H, F, E, k, moe.dtype_code(dt), "num_mtiles", torch.int32)[0])
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert _last_wave_sliced(num_mt, T, F, E, k, 256 if path == 3 else 128, sms)
+    verify_layer(moe, ws, out, case, what=f"last-wave slices path {path} {dt}")
+
+
 def test_layer_repeat_and_empty(moe):
     case = small_case(70, 256, 512, 8, 2, "fp8", 22)
     dcase = to_device(case)
