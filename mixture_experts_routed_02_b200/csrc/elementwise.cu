@@ -18,96 +18,106 @@ namespace moe {
 // Padding rows are not written: the tensor cores compute each output row from
 // its own input row only, and the outputs of padding rows are discarded.  The
 // CTA of each token's first assignment also zeroes the token's fp32 combine
-// row.  FP8 rows of up to kRegVec*1024 elements are read once and kept in
-// registers between the absmax and the quantisation.
+// row.  Rows of up to kRegVec*1024 elements are read once, into registers,
+// and before the wait for the routing kernel: the tokens are the caller's
+// input and the combine buffer was last read by the previous call's finalize,
+// both complete before routing started; only the destination row needs the
+// routing result.
 constexpr int kRegVec = 4;
 
 template <bool kFP8>
-__global__ void __launch_bounds__(128, 10) gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int k,
+__global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int k,
                                                      const int* __restrict__ slot_of, uint8_t* __restrict__ xs,
                                                      float* __restrict__ sx_slot, float* __restrict__ out32,
                                                      int* __restrict__ status) {
-    griddep_wait();
-    griddep_launch_dependents();
     __shared__ float warp_max[4];
     const int tid = threadIdx.x;
-    const int A = T * k;
+    const int a = blockIdx.x;
+    const int t = a / k;
     const int eb = kFP8 ? 1 : 2;
     const int nvec_in = H / 8;  // 8 bf16 per 16-byte vector
-    for (int a = blockIdx.x; a < A; a += gridDim.x) {  // one pass: the grid covers every assignment
-        const int s = slot_of[a];
-        if (s < 0) {
-            if (tid == 0) record_error(status, MOE_ERR_DEVICE_BOUNDS);
-            continue;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    const bool in_regs = nvec_in <= 128 * kRegVec;
+    uint4 v[kRegVec];
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < kRegVec; ++r) {
+            const int i = tid + r * 128;
+            v[r] = (i < nvec_in) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
         }
-        uint8_t* row_out = xs + (size_t)s * act_pitch((long)H * eb);
-        const int t = a / k;
-        if (a % k == 0) {
-            float4* o = reinterpret_cast<float4*>(out32 + (size_t)t * H);
-            for (int i = tid; i < H / 4; i += 128) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-        if (!kFP8) {
-            uint4* dst = reinterpret_cast<uint4*>(row_out);
+    }
+    if (a % k == 0) {
+        float4* o = reinterpret_cast<float4*>(out32 + (size_t)t * H);
+        for (int i = tid; i < H / 4; i += 128) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+    const int s = slot_of[a];
+    if (s < 0) {
+        if (tid == 0) record_error(status, MOE_ERR_DEVICE_BOUNDS);
+        return;
+    }
+    uint8_t* row_out = xs + (size_t)s * act_pitch((long)H * eb);
+    if (!kFP8) {
+        uint4* dst = reinterpret_cast<uint4*>(row_out);
+        if (in_regs) {
+#pragma unroll
+            for (int r = 0; r < kRegVec; ++r) {
+                const int i = tid + r * 128;
+                if (i < nvec_in) dst[i] = v[r];
+            }
+        } else {
             for (int i = tid; i < nvec_in; i += 128) dst[i] = __ldg(src + i);
-            continue;
         }
-        // FP8: absmax over the row, then x / sx rounded to e4m3 (nearest even, saturating)
-        const bool in_regs = nvec_in <= 128 * kRegVec;
-        uint4 v[kRegVec];
-        float amax = 0.f;
-        auto absmax8 = [&](const uint4& u) {
-            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+        return;
+    }
+    // FP8: absmax over the row, then x / sx rounded to e4m3 (nearest even, saturating)
+    float amax = 0.f;
+    auto absmax8 = [&](const uint4& u) {
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = __bfloat1622float2(p[j]);
-                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-            }
-        };
-        if (in_regs) {
-#pragma unroll
-            for (int r = 0; r < kRegVec; ++r) {
-                const int i = tid + r * 128;
-                v[r] = (i < nvec_in) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int r = 0; r < kRegVec; ++r) absmax8(v[r]);
-        } else {
-            for (int i = tid; i < nvec_in; i += 128) absmax8(__ldg(src + i));
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p[j]);
+            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
         }
+    };
+    if (in_regs) {
 #pragma unroll
-        for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
-        if ((tid & 31) == 0) warp_max[tid >> 5] = amax;
-        __syncthreads();
-        amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
-        __syncthreads();  // warp_max is reused by the next assignment
-        const float sx = (amax == 0.f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-        if (tid == 0) sx_slot[s] = sx;
-        uint2* dst = reinterpret_cast<uint2*>(row_out);
-        auto quant8 = [&](const uint4& u) {
-            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
-            uint32_t packed[2];
+        for (int r = 0; r < kRegVec; ++r) absmax8(v[r]);
+    } else {
+        for (int i = tid; i < nvec_in; i += 128) absmax8(__ldg(src + i));
+    }
 #pragma unroll
-            for (int j = 0; j < 4; j += 2) {
-                const float2 f0 = __bfloat1622float2(p[j]);
-                const float2 f1 = __bfloat1622float2(p[j + 1]);
-                const __nv_fp8x2_storage_t q0 = __nv_cvt_float2_to_fp8x2(
-                    make_float2(__fdiv_rn(f0.x, sx), __fdiv_rn(f0.y, sx)), __NV_SATFINITE, __NV_E4M3);
-                const __nv_fp8x2_storage_t q1 = __nv_cvt_float2_to_fp8x2(
-                    make_float2(__fdiv_rn(f1.x, sx), __fdiv_rn(f1.y, sx)), __NV_SATFINITE, __NV_E4M3);
-                packed[j / 2] = (uint32_t)q0 | ((uint32_t)q1 << 16);
-            }
-            return make_uint2(packed[0], packed[1]);
-        };
-        if (in_regs) {
+    for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+    if ((tid & 31) == 0) warp_max[tid >> 5] = amax;
+    __syncthreads();
+    amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
+    const float sx = (amax == 0.f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+    if (tid == 0) sx_slot[s] = sx;
+    uint2* dst = reinterpret_cast<uint2*>(row_out);
+    auto quant8 = [&](const uint4& u) {
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+        uint32_t packed[2];
 #pragma unroll
-            for (int r = 0; r < kRegVec; ++r) {
-                const int i = tid + r * 128;
-                if (i < nvec_in) dst[i] = quant8(v[r]);
-            }
-        } else {
-            for (int i = tid; i < nvec_in; i += 128) dst[i] = quant8(__ldg(src + i));
+        for (int j = 0; j < 4; j += 2) {
+            const float2 f0 = __bfloat1622float2(p[j]);
+            const float2 f1 = __bfloat1622float2(p[j + 1]);
+            const __nv_fp8x2_storage_t q0 = __nv_cvt_float2_to_fp8x2(
+                make_float2(__fdiv_rn(f0.x, sx), __fdiv_rn(f0.y, sx)), __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8x2_storage_t q1 = __nv_cvt_float2_to_fp8x2(
+                make_float2(__fdiv_rn(f1.x, sx), __fdiv_rn(f1.y, sx)), __NV_SATFINITE, __NV_E4M3);
+            packed[j / 2] = (uint32_t)q0 | ((uint32_t)q1 << 16);
         }
+        return make_uint2(packed[0], packed[1]);
+    };
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < kRegVec; ++r) {
+            const int i = tid + r * 128;
+            if (i < nvec_in) dst[i] = quant8(v[r]);
+        }
+    } else {
+        for (int i = tid; i < nvec_in; i += 128) dst[i] = quant8(__ldg(src + i));
     }
 }
 

@@ -25,20 +25,42 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits, in
     uint64_t chosen = 0;
     int ids[kMaxTopK];
     float vals[kMaxTopK];
-    for (int j = 0; j < k; ++j) {
-        int best = -1;
-        float bv = 0.f;
-        for (int e = 0; e < E; ++e) {
-            if ((chosen >> e) & 1ull) continue;
-            const float v = rank_value(__ldg(l + e));
-            if (best < 0 || v > bv) {
-                best = e;
-                bv = v;
+    if (E <= 16) {
+        // up to 16 experts: all logits loaded at once into registers (the
+        // loads do not wait on one another), then the same selection passes
+        float lv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) lv[e] = (e < E) ? rank_value(__ldg(l + e)) : 0.f;
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            float bv = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                if (e < E && !((chosen >> e) & 1ull) && (best < 0 || lv[e] > bv)) {
+                    best = e;
+                    bv = lv[e];
+                }
             }
+            chosen |= 1ull << best;
+            ids[j] = best;
+            vals[j] = bv;
         }
-        chosen |= 1ull << best;
-        ids[j] = best;
-        vals[j] = bv;
+    } else {
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            float bv = 0.f;
+            for (int e = 0; e < E; ++e) {
+                if ((chosen >> e) & 1ull) continue;
+                const float v = rank_value(__ldg(l + e));
+                if (best < 0 || v > bv) {
+                    best = e;
+                    bv = v;
+                }
+            }
+            chosen |= 1ull << best;
+            ids[j] = best;
+            vals[j] = bv;
+        }
     }
     float w[kMaxTopK];
     const float lmax = vals[0];
