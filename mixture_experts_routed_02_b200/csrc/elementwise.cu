@@ -122,10 +122,9 @@ __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __r
 }
 
 cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
-                          float* sx_slot, float* out32, int* status, int num_sms, cudaStream_t stream) {
+                          float* sx_slot, float* out32, int* status, cudaStream_t stream) {
     const int A = T * k;
     const int grid = std::max(1, A);
-    (void)num_sms;
     if (fp8)
         return launch_dependent(gather_kernel<true>, dim3(grid), dim3(128), 0, stream, x, T, H, k, slot_of, xs,
                                 sx_slot, out32, status);

@@ -101,7 +101,7 @@ int max_active_clusters(void (*kernel)(KArgs...), int threads, size_t smem, int 
 cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream);
 int route_launches(int T, const RouteOutputs& o);  // kernels launch_route enqueues (1 or 2)
 cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
-                          float* sx_slot, float* out32, int* status, int num_sms, cudaStream_t stream);
+                          float* sx_slot, float* out32, int* status, cudaStream_t stream);
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream);
 // Blocked, pre-swizzled weight layout (see moe_prepare_weights in moe.h).
 constexpr int kWBlockRows = 128;

@@ -392,7 +392,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     {
         ProfScope ps(MOE_KERNEL_GATHER, st);
         if (launch_gather(fp8, static_cast<const __nv_bfloat16*>(x), T, H, k, o.slot_of, reg(MOE_WS_XS), sx, out32,
-                          status, num_sms, st) != cudaSuccess)
+                          status, st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 
