@@ -195,7 +195,9 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
  *   MOE_OPT_PATH:     0 = choose by problem size, 1 = force the throughput
  *                     tiles (256 x 256 tiles on pairs of SMs), 2 = force the
  *                     weight-streaming tiles (128 x 128 on one SM), 3 = force
- *                     128 x 256 tiles on one SM.
+ *                     128 x 256 tiles on one SM, 4 = force the tiny-batch
+ *                     tiles (32 activation rows per stage; only for at most
+ *                     32 assignments, else MOE_ERR_UNSUPPORTED).
  *   MOE_OPT_SPLITK:   0 = automatic, n > 0 = split the second GEMM's K into n parts
  *                     (must divide F/128).
  *   MOE_OPT_TIMEOUT_MS: limit of every device-side wait (default 2000).

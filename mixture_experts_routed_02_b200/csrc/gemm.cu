@@ -36,10 +36,15 @@ namespace moe {
 
 namespace {
 
-template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR>
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR>
 struct Cfg {
     static constexpr bool MX = (STAGE == 2) && FP8;
-    static constexpr int A_BYTES = kBlockM * 128;
+    // activation rows copied per stage: 128, or 32 when no m-tile holds more
+    // than 32 rows in use (the MMA still reads 128 rows from the stage's
+    // address; rows 32-127 then alias the next buffers and belong to padding
+    // rows, whose results are discarded)
+    static constexpr int A_BYTES = AR * 128;
+    static_assert(AR == kBlockM || (AR == 32 && !PAIR), "activation rows per stage");
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // weight rows held by one CTA
     static constexpr int B_BYTES = B_ROWS * 128;
     static constexpr int SF_BYTES = MX ? 512 : 0;
@@ -80,12 +85,12 @@ __device__ __forceinline__ void decode_tile(int tile, int num_mt, int n_tiles, i
 
 }  // namespace
 
-template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR>
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR>
 __global__ void __launch_bounds__(192, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmSF,
                     const GemmArgs args) {
-    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR>;
+    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -278,7 +283,8 @@ __global__ void __launch_bounds__(192, 1)
         }
     };
     auto stage_tx = [&](bool small, int q4) {
-        return C::TX_BYTES - (small ? (kBlockM - 32) * 128 : 0) - (q4 >= 0 ? C::B_BYTES - 64 * 128 : 0);
+        return C::TX_BYTES - ((small && AR == kBlockM) ? (kBlockM - 32) * 128 : 0) -
+               (q4 >= 0 ? C::B_BYTES - 64 * 128 : 0);
     };
     const int b_nblk = args.rows_b / kWBlockRows;
     const uint64_t pol_b = args.b_evict_first ? policy_evict_first() : policy_evict_normal();
@@ -335,6 +341,7 @@ __global__ void __launch_bounds__(192, 1)
                 unit_coords(u, m, n, split, dup, q4);
                 const int e = args.mtile_expert[m];
                 const bool small = a_rows32(m);
+                if (AR == 32 && !small) record_error(args.status, MOE_ERR_DEVICE_BOUNDS);  // host chose this wrongly
                 for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
                     const bool prefetched = (u == unit0) && (kt - split * kps) < npre;
                     if (!prefetched) {
@@ -358,7 +365,7 @@ __global__ void __launch_bounds__(192, 1)
                                              (m * args.f_tiles + kt) * 4, pol_a);
                     } else {
                         if (!skip)
-                            tma_load_2d(smem + stage * C::A_BYTES, small ? &tmA32 : &tmA, &full[stage], kt * C::KE,
+                            tma_load_2d(smem + stage * C::A_BYTES, (small || AR == 32) ? &tmA32 : &tmA, &full[stage], kt * C::KE,
                                         m * kBlockM, pol_a);
                         if constexpr (C::MX)
                             bulk_load(smem + C::OFF_SF + stage * C::SF_BYTES,
@@ -662,10 +669,10 @@ __global__ void __launch_bounds__(192, 1)
 
 namespace {
 
-template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR>
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR = kBlockM>
 cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, int grid, cudaStream_t stream) {
-    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR>;
-    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR>;
+    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR>;
+    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR, AR>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     if constexpr (PAIR) {
@@ -680,10 +687,10 @@ cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, int grid, cud
     }
 }
 
-template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR>
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR = kBlockM>
 int max_pairs_one() {
-    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR>;
-    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR>;
+    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR>;
+    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR, AR>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return 0;
     return max_active_clusters(kern, 192, C::SMEM_BYTES, 2);
@@ -692,15 +699,24 @@ int max_pairs_one() {
 }  // namespace
 
 int gemm_block_n(int stage, bool fp8, int cfg) {
-    (void)stage;
     (void)fp8;
+    if (cfg == 3) return stage == 1 ? 256 : 128;
     return cfg == 1 ? 128 : 256;
 }
 
 // cfg 0: CTA pairs, 256 x 256 tiles; cfg 1: one CTA, 128 x 128 tiles
-// (weight streaming); cfg 2: one CTA, 128 x 256 tiles.
+// (weight streaming); cfg 2: one CTA, 128 x 256 tiles; cfg 3 (no m-tile with
+// more than 32 rows in use): 32 activation rows per stage, which leaves room
+// for deeper pipelines -- stage 1 on 128 x 256 tiles, stage 2 on 128 x 128.
 cudaError_t launch_gemm(int stage, bool fp8, int cfg, const GemmMaps& maps, const GemmArgs& args, int grid,
                         cudaStream_t stream) {
+    if (cfg == 3) {
+        if (stage == 1)
+            return fp8 ? launch_one<1, true, 256, 6, 2, false, 32>(maps, args, grid, stream)
+                       : launch_one<1, false, 256, 6, 2, false, 32>(maps, args, grid, stream);
+        return fp8 ? launch_one<2, true, 128, 10, 2, false, 32>(maps, args, grid, stream)
+                   : launch_one<2, false, 128, 10, 2, false, 32>(maps, args, grid, stream);
+    }
     if (stage == 1) {
         if (fp8) return cfg == 0 ? launch_one<1, true, 256, 6, 2, true>(maps, args, grid, stream)
                       : cfg == 1 ? launch_one<1, true, 128, 6, 2, false>(maps, args, grid, stream)

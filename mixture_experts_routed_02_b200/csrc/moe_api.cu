@@ -249,7 +249,7 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
 int moe_set_option(int option, int value) {
     switch (option) {
         case MOE_OPT_PATH:
-            if (value < 0 || value > 3) return MOE_ERR_INVALID_ARG;
+            if (value < 0 || value > 4) return MOE_ERR_INVALID_ARG;
             return g_opt_path.exchange(value);
         case MOE_OPT_SPLITK:
             if (value < 0) return MOE_ERR_INVALID_ARG;
@@ -314,6 +314,8 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
         if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
     const Layout L = make_layout(T, H, F, E, k, dtype);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    const int opt_path = g_opt_path.load();  // read once per call
+    if (opt_path == 4 && L.A > 32) return MOE_ERR_UNSUPPORTED;  // forced tiny-batch tiles
     if (T == 0) return MOE_OK;
 
     int* status = nullptr;
@@ -333,12 +335,14 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     //     tile makes a pair compute too many rows twice).
     // One-CTA 128 x 256 tiles where the pair kernel cannot be resident;
     // 128-wide tiles when a dimension is not a multiple of 256.
+    // At most 32 assignments in all (decode of up to 16 tokens with top-2): no
+    // tile holds more than 32 rows, so both GEMMs copy 32 activation rows per
+    // stage and run deeper pipelines.
     const bool small_batch = L.A <= 64 * E;
-    const int opt_path = g_opt_path.load();
     int cfg1, cfg2;
     if (opt_path == 0) {
-        cfg1 = (L.A < 512 * E) ? 2 : 0;
-        cfg2 = small_batch ? 1 : cfg1;
+        cfg1 = (L.A <= 32) ? 3 : (L.A < 512 * E) ? 2 : 0;
+        cfg2 = (L.A <= 32) ? 3 : small_batch ? 1 : cfg1;
     } else {
         cfg1 = cfg2 = opt_path - 1;
     }
@@ -433,7 +437,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     GemmArgs g2 = g1;
     g2.row_scale = nullptr;
     g2.test_stall = 0;
-    g2.group_m = (cfg2 != 1) ? 1 : 0;
+    g2.group_m = (cfg2 == 0 || cfg2 == 2) ? 1 : 0;
     g2.col_scale = fp8 ? s2 : nullptr;
     g2.topk_w = o.topk_w;
     g2.a_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;

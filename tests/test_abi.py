@@ -91,5 +91,10 @@ def test_options(moe):
     old = moe.moe_set_option(moe.OPT_PATH, 2)
     assert moe.moe_set_option(moe.OPT_PATH, old) == 2
     assert moe.moe_set_option(moe.OPT_PATH, 5) == -1
+    old = moe.moe_set_option(moe.OPT_PATH, 4)
+    # tiny-batch tiles are refused, before the device is touched, for more than 32 assignments
+    P = 4096
+    assert moe.moe_ffn_forward(P, P, P, None, P, None, 64, 128, 128, 8, 2, 0, P, P, 1 << 40, None) == -2
+    moe.moe_set_option(moe.OPT_PATH, old)
     assert moe.moe_set_option(99, 0) == -1
     assert moe.moe_set_option(moe.OPT_TIMEOUT_MS, 0) == -1

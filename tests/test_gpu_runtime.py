@@ -17,7 +17,7 @@ def moe():
     return m
 
 
-PATHS = pytest.mark.parametrize("path", [2, 1, 3], ids=["streaming_tiles", "pair_tiles", "wide_tiles"])
+PATHS = pytest.mark.parametrize("path", [2, 1, 3, 4], ids=["streaming_tiles", "pair_tiles", "wide_tiles", "tiny_tiles"])
 
 
 @pytest.fixture(autouse=True)
@@ -28,7 +28,7 @@ def _reset_path(moe):
 
 @PATHS
 def test_stalled_wait_times_out_and_context_survives(moe, path):
-    case = small_case(64, 256, 512, 8, 2, "fp8", 41)
+    case = small_case(16 if path == 4 else 64, 256, 512, 8, 2, "fp8", 41)
     d = to_device(case)
     moe.moe_set_option(moe.OPT_PATH, path)
     old_t = moe.moe_set_option(moe.OPT_TIMEOUT_MS, 50)
@@ -50,7 +50,7 @@ def test_stalled_wait_times_out_and_context_survives(moe, path):
 @pytest.mark.parametrize("dtype", ["fp8", "bf16"])
 def test_cuda_graph_capture_and_replay(moe, dtype, path):
     moe.moe_set_option(moe.OPT_PATH, path)
-    T, H, F, E, k = 48, 256, 512, 8, 2
+    T, H, F, E, k = (16 if path == 4 else 48), 256, 512, 8, 2
     case = small_case(T, H, F, E, k, dtype, 42)
     d = to_device(case)
     fp8 = dtype == "fp8"
