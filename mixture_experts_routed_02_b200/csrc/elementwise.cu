@@ -13,27 +13,29 @@
 
 namespace moe {
 
-// One CTA (128 threads) per assignment a = t*k + j: copies (bf16) or
-// quantises (FP8) token t's row into a's row of the expert-padded layout.
-// Padding rows are not written: the tensor cores compute each output row from
-// its own input row only, and the outputs of padding rows are discarded.  The
-// CTA of each token's first assignment also zeroes the token's fp32 combine
-// row.  Rows of up to kRegVec*1024 elements are read once, into registers,
-// and before the wait for the routing kernel: the tokens are the caller's
-// input and the combine buffer was last read by the previous call's finalize,
-// both complete before routing started; only the destination row needs the
-// routing result.
+// One CTA (128 threads) per `per_cta` consecutive assignments a = t*k + j of
+// one token t (per_cta = k: the whole token; 1: one assignment, for small
+// batches where more CTAs shorten the critical path): reads the row once,
+// quantises it once (FP8: the scale is per token, so every copy is the same)
+// and writes it to the padded-layout row of each of those assignments; the
+// CTA holding the token's first assignment also zeroes its fp32 combine row.  Padding rows are not written: the
+// tensor cores compute each output row from its own input row only, and the
+// outputs of padding rows are discarded.  Rows of up to kRegVec*1024 elements
+// are read into registers before the wait for the routing kernel: the tokens
+// are the caller's input and the combine buffer was last read by the previous
+// call's finalize, both complete before routing started; only the destination
+// rows need the routing result.
 constexpr int kRegVec = 4;
 
 template <bool kFP8>
 __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int k,
-                                                     const int* __restrict__ slot_of, uint8_t* __restrict__ xs,
-                                                     float* __restrict__ sx_slot, float* __restrict__ out32,
-                                                     int* __restrict__ status) {
+                                                    const int* __restrict__ slot_of, uint8_t* __restrict__ xs,
+                                                    float* __restrict__ sx_slot, float* __restrict__ out32,
+                                                    int per_cta, int* __restrict__ status) {
     __shared__ float warp_max[4];
     const int tid = threadIdx.x;
-    const int a = blockIdx.x;
-    const int t = a / k;
+    const int a0 = blockIdx.x * per_cta;
+    const int t = a0 / k;
     const int eb = kFP8 ? 1 : 2;
     const int nvec_in = H / 8;  // 8 bf16 per 16-byte vector
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
@@ -46,28 +48,37 @@ __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __r
             v[r] = (i < nvec_in) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
         }
     }
-    if (a % k == 0) {
+    if (a0 % k == 0) {
         float4* o = reinterpret_cast<float4*>(out32 + (size_t)t * H);
         for (int i = tid; i < H / 4; i += 128) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     griddep_wait();
     griddep_launch_dependents();
-    const int s = slot_of[a];
-    if (s < 0) {
+    // destination rows of this CTA's assignments
+    const int n = per_cta;
+    int slots[kMaxTopK];
+    bool bad = false;
+    for (int j = 0; j < n; ++j) {
+        slots[j] = slot_of[a0 + j];
+        bad |= slots[j] < 0;
+    }
+    if (bad) {
         if (tid == 0) record_error(status, MOE_ERR_DEVICE_BOUNDS);
         return;
     }
-    uint8_t* row_out = xs + (size_t)s * act_pitch((long)H * eb);
+    const long pitch = act_pitch((long)H * eb);
     if (!kFP8) {
-        uint4* dst = reinterpret_cast<uint4*>(row_out);
-        if (in_regs) {
+        for (int j = 0; j < n; ++j) {
+            uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)slots[j] * pitch);
+            if (in_regs) {
 #pragma unroll
-            for (int r = 0; r < kRegVec; ++r) {
-                const int i = tid + r * 128;
-                if (i < nvec_in) dst[i] = v[r];
+                for (int r = 0; r < kRegVec; ++r) {
+                    const int i = tid + r * 128;
+                    if (i < nvec_in) dst[i] = v[r];
+                }
+            } else {
+                for (int i = tid; i < nvec_in; i += 128) dst[i] = __ldg(src + i);
             }
-        } else {
-            for (int i = tid; i < nvec_in; i += 128) dst[i] = __ldg(src + i);
         }
         return;
     }
@@ -93,8 +104,7 @@ __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __r
     __syncthreads();
     amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
     const float sx = (amax == 0.f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-    if (tid == 0) sx_slot[s] = sx;
-    uint2* dst = reinterpret_cast<uint2*>(row_out);
+    if (tid < n) sx_slot[slots[tid]] = sx;
     auto quant8 = [&](const uint4& u) {
         const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
         uint32_t packed[2];
@@ -114,22 +124,28 @@ __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __r
 #pragma unroll
         for (int r = 0; r < kRegVec; ++r) {
             const int i = tid + r * 128;
-            if (i < nvec_in) dst[i] = quant8(v[r]);
+            if (i < nvec_in) {
+                const uint2 q = quant8(v[r]);
+                for (int j = 0; j < n; ++j) reinterpret_cast<uint2*>(xs + (size_t)slots[j] * pitch)[i] = q;
+            }
         }
     } else {
-        for (int i = tid; i < nvec_in; i += 128) dst[i] = quant8(__ldg(src + i));
+        for (int i = tid; i < nvec_in; i += 128) {
+            const uint2 q = quant8(__ldg(src + i));
+            for (int j = 0; j < n; ++j) reinterpret_cast<uint2*>(xs + (size_t)slots[j] * pitch)[i] = q;
+        }
     }
 }
 
 cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
                           float* sx_slot, float* out32, int* status, cudaStream_t stream) {
-    const int A = T * k;
-    const int grid = std::max(1, A);
+    const int per_cta = (T >= 256) ? k : 1;  // a CTA per token for large batches
+    const int grid = std::max(1, T * k / per_cta);
     if (fp8)
         return launch_dependent(gather_kernel<true>, dim3(grid), dim3(128), 0, stream, x, T, H, k, slot_of, xs,
-                                sx_slot, out32, status);
+                                sx_slot, out32, per_cta, status);
     return launch_dependent(gather_kernel<false>, dim3(grid), dim3(128), 0, stream, x, T, H, k, slot_of, xs, sx_slot,
-                            out32, status);
+                            out32, per_cta, status);
 }
 
 // out = bf16(out32), round to nearest even; n is a multiple of 8.
