@@ -27,13 +27,14 @@ namespace moe {
 // rows need the routing result.
 constexpr int kRegVec = 4;
 
-template <bool kFP8>
+template <bool kFP8, bool kPerToken>
 __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int k,
                                                     const int* __restrict__ slot_of, uint8_t* __restrict__ xs,
                                                     float* __restrict__ sx_slot, float* __restrict__ out32,
-                                                    int per_cta, int* __restrict__ status) {
+                                                    int* __restrict__ status) {
     __shared__ float warp_max[4];
     const int tid = threadIdx.x;
+    const int per_cta = kPerToken ? k : 1;
     const int a0 = blockIdx.x * per_cta;
     const int t = a0 / k;
     const int eb = kFP8 ? 1 : 2;
@@ -54,9 +55,10 @@ __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __r
     }
     griddep_wait();
     griddep_launch_dependents();
-    // destination rows of this CTA's assignments
+    // destination rows of this CTA's assignments (kept in registers when there
+    // is one)
     const int n = per_cta;
-    int slots[kMaxTopK];
+    int slots[kPerToken ? kMaxTopK : 1];
     bool bad = false;
     for (int j = 0; j < n; ++j) {
         slots[j] = slot_of[a0 + j];
@@ -139,13 +141,19 @@ __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __r
 
 cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
                           float* sx_slot, float* out32, int* status, cudaStream_t stream) {
-    const int per_cta = (T >= 256) ? k : 1;  // a CTA per token for large batches
-    const int grid = std::max(1, T * k / per_cta);
+    // a CTA per token for large batches, per assignment (more CTAs, shorter
+    // critical path) for small ones
+    const bool per_token = T >= 256;
+    const dim3 grid(std::max(1, per_token ? T : T * k));
     if (fp8)
-        return launch_dependent(gather_kernel<true>, dim3(grid), dim3(128), 0, stream, x, T, H, k, slot_of, xs,
-                                sx_slot, out32, per_cta, status);
-    return launch_dependent(gather_kernel<false>, dim3(grid), dim3(128), 0, stream, x, T, H, k, slot_of, xs, sx_slot,
-                            out32, per_cta, status);
+        return per_token ? launch_dependent(gather_kernel<true, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
+                                            xs, sx_slot, out32, status)
+                         : launch_dependent(gather_kernel<true, false>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
+                                            xs, sx_slot, out32, status);
+    return per_token ? launch_dependent(gather_kernel<false, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of, xs,
+                                        sx_slot, out32, status)
+                     : launch_dependent(gather_kernel<false, false>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
+                                        xs, sx_slot, out32, status);
 }
 
 // out = bf16(out32), round to nearest even; n is a multiple of 8.

@@ -335,14 +335,14 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     //     tile makes a pair compute too many rows twice).
     // One-CTA 128 x 256 tiles where the pair kernel cannot be resident;
     // 128-wide tiles when a dimension is not a multiple of 256.
-    // At most 32 assignments in all (decode of up to 16 tokens with top-2): no
-    // tile holds more than 32 rows, so both GEMMs copy 32 activation rows per
-    // stage and run deeper pipelines.
+    // (The tiny-batch tiles, 32 activation rows per stage with deeper
+    // pipelines, are only used when forced: measured against the small-batch
+    // configuration at 16 tokens they were not faster.)
     const bool small_batch = L.A <= 64 * E;
     int cfg1, cfg2;
     if (opt_path == 0) {
-        cfg1 = (L.A <= 32) ? 3 : (L.A < 512 * E) ? 2 : 0;
-        cfg2 = (L.A <= 32) ? 3 : small_batch ? 1 : cfg1;
+        cfg1 = (L.A < 512 * E) ? 2 : 0;
+        cfg2 = small_batch ? 1 : cfg1;
     } else {
         cfg1 = cfg2 = opt_path - 1;
     }
