@@ -11,7 +11,7 @@ under torch.distributed.run) every rank runs its own batch against its own copy
 of the weights (weak scaling); the only collectives are the timing barrier and
 the max over ranks.
 
-``--impl reference`` times the CPU oracle (fp64, the machine's host cores) on a
+``--impl reference`` times the CPU oracle (fp64, the host's CPU cores) on a
 bounded sample of the same workload.
 """
 import argparse

@@ -3,6 +3,7 @@
 //
 // One call of moe_ffn_forward enqueues, on the caller's stream:
 //   route_kernel   top-k, softmax, histogram, scan, permutation, padded layout
+//                  (from 1024 tokens: route_topk_kernel + route_place_kernel)
 //   gather_kernel  gather (+ per-token e4m3 quantisation) and zeroing of out32
 //   stage-1 GEMM   gather-GEMM with w1/w3 + SwiGLU (+ MX quantisation of h)
 //   stage-2 GEMM   GEMM with w2 + routing-weighted scatter-add into out32
