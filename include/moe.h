@@ -127,8 +127,13 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float
  * re-quantised to e4m3 in blocks of 32 d_ff elements with a power-of-two
  * scale 2^ceil(log2(absmax/448)).  BF16 mode: h is rounded to bf16.  The k
  * weighted expert outputs are summed in fp32 and rounded once to bf16.
- * The call makes no host<->device synchronisation and may be captured in a
- * CUDA graph.
+ * Execution: five kernels (six from 1024 tokens on) chained on `stream` with
+ * programmatic dependent launch; to the rest of the stream the call is
+ * ordinary stream-ordered work (later work starts after `out` is written).
+ * The group GEMM tiles are chosen from the average rows per expert (see
+ * MOE_OPT_PATH): small batches stream weights on one-CTA tiles, large ones
+ * use 256 x 256 tiles on pairs of SMs.  The call makes no host<->device
+ * synchronisation and may be captured in a CUDA graph.
  */
 int moe_ffn_forward(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
                     const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
@@ -147,7 +152,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
  *   process exits.  This call allocates nothing.
  *   Returns MOE_ERR_WORKSPACE, before enqueuing anything, when the problem
  *   needs more than that (moe_workspace_size(T,H,F,E,k,dtype) bytes); decode
- *   batches of Mixtral-8x7B experts fit (T = 16: about 23 MB FP8, 45 MB BF16).
+ *   batches of Mixtral-8x7B experts fit (T = 16: about 22 MB FP8, 43 MB BF16).
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before capturing a stream.
