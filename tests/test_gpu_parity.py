@@ -171,6 +171,27 @@ def test_layer_routing_layout_many_ctas(moe, T, E, k, seed):
     verify_layer(moe, ws, out, case, tokens=np.array([0, T // 2, T - 1]), what=f"many-CTA routing T={T}")
 
 
+def test_layer_largest_batch(moe):
+    """The largest batch the library takes (T*k = 262144 assignments): routing
+    of every token is bit-exact, the padded layout is complete, and sampled
+    outputs match the oracle."""
+    T, H, F, E, k = 131072, 128, 256, 8, 2
+    case = small_case(T, H, F, E, k, "fp8", 71)
+    out, ws = run_layer(to_device(case))
+    nc = moe_inputs.to_numpy(case)
+    r = oracle.route(nc["logits"], k)
+    A = T * k
+    view = lambda name: moe.ws_view(ws, T, H, F, E, k, 1, name, torch.int32).cpu().numpy()
+    np.testing.assert_array_equal(view("topk_ids")[:A], r["ids"].reshape(-1))
+    np.testing.assert_array_equal(view("perm")[:A], r["perm"])
+    slot_of, slot_assign, mtile_expert, n_mt = _expected_layout(r, T, E, k)
+    np.testing.assert_array_equal(view("slot_of")[:A], slot_of)
+    np.testing.assert_array_equal(view("slot_assign")[:n_mt * 128], slot_assign)
+    rng = np.random.default_rng(72)
+    tokens = np.unique(np.concatenate([[0, T - 1], rng.integers(0, T, 12)]))
+    verify_layer(moe, ws, out, case, tokens=tokens, what="largest batch")
+
+
 @pytest.mark.parametrize("splits", [2, 4])
 def test_layer_split_k(moe, splits):
     moe.moe_set_option(moe.OPT_PATH, 2)
