@@ -1,0 +1,92 @@
+"""Host-side measurement logic of bench.py (no GPU): the algorithmic work the
+roofline divides by, the lookup of recorded ncu traffic, and the parsing of
+the clock samples taken during the timed region."""
+import os
+import shutil
+
+import pytest
+
+import bench
+
+DECODE = dict(T=16, H=4096, F=14336, E=8, k=2, dtype="fp8", skew=False)
+
+
+def test_algorithmic_work_of_the_decode_layer():
+    # all 8 experts active: per expert 3*H*F e4m3 weight bytes plus 4*(2F+H)
+    # bytes of fp32 channel scales; bf16 tokens in and out; fp32 logits
+    w = bench.algorithmic(DECODE, [4, 4, 4, 4, 4, 4, 4, 4])
+    H, F, T, E = 4096, 14336, 16, 8
+    assert w["layer_bytes"] == 8 * (3 * H * F + 4 * (2 * F + H)) + T * H * 4 + 4 * T * E
+    assert abs(w["layer_bytes"] - 1.4106e9) < 1e6
+    # 6*H*F FLOP per assignment (3.523e8), 32 assignments, plus the router's T*E
+    assert w["layer_flops"] == 6.0 * H * F * 32 + 2.0 * T * E
+    assert abs(6.0 * H * F - 3.523e8) < 1e5
+    assert w["s1_flops"] == 2 * w["s2_flops"]
+    # stage 1 streams w1 and w3, stage 2 streams w2: 2:1 in weight bytes
+    assert abs(w["s1_bytes"] / w["s2_bytes"] - 2.0) < 0.01
+
+
+def test_experts_without_tokens_read_no_weights():
+    full = bench.algorithmic(DECODE, [4] * 8)
+    two = bench.algorithmic(DECODE, [16, 16, 0, 0, 0, 0, 0, 0])
+    assert two["active"] == 2
+    per_expert = 3 * 4096 * 14336 + 4 * (2 * 14336 + 4096)
+    assert full["layer_bytes"] - two["layer_bytes"] == 6 * per_expert
+    assert full["layer_flops"] == two["layer_flops"]  # same assignments, same work
+
+
+def test_bf16_weights_count_two_bytes_and_no_scales():
+    spec = dict(DECODE, dtype="bf16")
+    w = bench.algorithmic(spec, [4] * 8)
+    assert w["layer_bytes"] == 8 * 3 * 4096 * 14336 * 2 + 16 * 4096 * 4 + 4 * 16 * 8
+
+
+def test_recorded_traffic_needs_the_same_kernel_code(monkeypatch):
+    assert bench.recorded_traffic("stage1_w13_swiglu", "no-such-workload") is None
+    monkeypatch.setattr(bench, "source_sha", lambda: "0000000000000000")
+    assert bench.recorded_traffic("stage1_w13_swiglu", "decode") is None
+
+
+def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    root = tmp_path / "repo"
+    for d in ("mixture_experts_routed_02_b200/csrc", "include"):
+        (root / d).mkdir(parents=True)
+    for rel in ("mixture_experts_routed_02_b200/csrc/gemm.cu", "mixture_experts_routed_02_b200/csrc/kernels.cuh",
+                "mixture_experts_routed_02_b200/csrc/ptx.cuh", "include/moe.h"):
+        shutil.copy(os.path.join(bench.ROOT, rel), root / rel)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    base = bench.source_sha()
+    gemm = root / "mixture_experts_routed_02_b200/csrc/gemm.cu"
+    text = gemm.read_text()
+    gemm.write_text("// a new comment line\n" + text.replace("\n", "\n\n", 3))
+    assert bench.source_sha() == base
+    gemm.write_text(text.replace("kBlockM", "kBlockM ", 1) + "\nstatic int extra_code = 1;\n")
+    assert bench.source_sha() != base
+
+
+class _FakeSmi:
+    def __init__(self, lines):
+        self.out = "\n".join(lines)
+
+    def terminate(self):
+        pass
+
+    def communicate(self, timeout=None):
+        return self.out, ""
+
+
+@pytest.mark.parametrize("lines,reasons,median", [
+    (["0, 1965, 1965, 700, 0x0, Not Active, Not Active, Not Active, Not Active"] * 3, [], 1965.0),
+    (["0, 1400, 1965, 1000, 0x4, Not Active, Not Active, Not Active, Active",
+      "0, 1350, 1965, 1000, 0x4, Not Active, Not Active, Not Active, Active",
+      "0, 1965, 1965, 900, 0x0, Not Active, Not Active, Not Active, Not Active"], ["sw_power_cap"], 1400.0),
+    (["0, 1200, 1965, 600, 0x40, Not Active, Active, Not Active, Not Active", "garbage"],
+     ["hw_thermal_slowdown"], 1200.0),
+])
+def test_clock_samples(lines, reasons, median):
+    s = bench.ClockSampler(0)
+    s.proc = _FakeSmi(lines)
+    clk = s.stop()
+    assert clk["reasons"] == reasons
+    assert clk["sm_mhz"] == median
+    assert clk["sm_max_mhz"] == 1965.0
