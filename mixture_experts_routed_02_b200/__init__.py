@@ -12,6 +12,18 @@ keep their names (``moe_route``, ``moe_ffn_forward``, ...) and take raw device
 pointers; the ``route``/``ffn_forward``/``prepare_weights`` helpers accept
 torch tensors and pass their pointers and the current CUDA stream.  There is no
 fallback: if the library cannot be loaded, importing this package fails.
+
+Use (FP8: e4m3 weights with fp32 per-output-channel scales)::
+
+    import mixture_experts_routed_02_b200 as moe
+    w13, s13, w2p = moe.prepare_weights(w1, w3, s1, s3, w2)   # once, at load time
+    ws = moe.workspace(T, H, F, E, k, "fp8")                    # reusable scratch
+    out = moe.ffn_forward(x, logits, w13, s13, w2p, s2, k, F, True, ws=ws)
+    assert moe.moe_get_status(None) == moe.MOE_OK             # device-side checks
+
+``moe_set_option(OPT_PATH, n)`` forces the tile configuration (0 = by size,
+1 = CTA pairs, 2 = weight streaming, 3 = 128 x 256 tiles, 4 = tiny batches);
+``moe_profile_enable``/``moe_profile_read`` time each kernel of the layer.
 """
 import ctypes
 import os
