@@ -104,6 +104,10 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 1) route_kernel(const float*
     __shared__ int poff[kMaxExperts + 1];  // first padded slot of each expert
     __shared__ int mt_start[kMaxExperts + 1];
     __shared__ int n_mtiles;
+    // the small variant (at most 1024 assignments) keeps the chosen experts in
+    // shared memory for the later phases instead of reading them back
+    constexpr bool kIdsInSmem = kRouteWarps <= 4;
+    __shared__ int s_ids[kIdsInSmem ? 1024 : 1];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     griddep_launch_dependents();  // the gather may be scheduled; it waits for this grid
@@ -113,8 +117,17 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 1) route_kernel(const float*
     }
 
     // ---- phase 1: top-k and weights
-    for (int t = tid; t < T; t += kRouteThreads) route_token(logits, t, E, k, o);
+    for (int t = tid; t < T; t += kRouteThreads) {
+        int ids[kMaxTopK];
+        route_token(logits, t, E, k, o, &ids);
+        if constexpr (kIdsInSmem)
+            for (int j = 0; j < k; ++j) s_ids[t * k + j] = ids[j];
+    }
     __syncthreads();
+    auto id_of = [&](int a) {
+        if constexpr (kIdsInSmem) return s_ids[a];
+        else return o.topk_ids[a];
+    };
 
     // ---- phase 2: per-warp histograms over contiguous assignment ranges
     const int A = T * k;
@@ -123,7 +136,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 1) route_kernel(const float*
     const int a_end = min(A, a_begin + chunk);
     for (int base = a_begin; base < a_end; base += 32) {
         const int a = base + lane;
-        const int e = (a < a_end) ? o.topk_ids[a] : -1;
+        const int e = (a < a_end) ? id_of(a) : -1;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         if (e >= 0 && lane == __ffs(peers) - 1) cnt_w[warp][e] += __popc(peers);
         __syncwarp();
@@ -160,7 +173,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 1) route_kernel(const float*
     // ---- phase 4: placement
     for (int base = a_begin; base < a_end; base += 32) {
         const int a = base + lane;
-        const int e = (a < a_end) ? o.topk_ids[a] : -1;
+        const int e = (a < a_end) ? id_of(a) : -1;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         const int leader = __ffs(peers) - 1;
         if (e >= 0) {
@@ -182,15 +195,9 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 1) route_kernel(const float*
 
     // ---- padded layout: tile -> expert, and padding rows marked -1
     if (o.slot_assign) {
-        for (int m = tid; m < n_mtiles; m += kRouteThreads) {
-            int e = 0;
-            while (e + 1 < E && mt_start[e + 1] <= m) ++e;
-            o.mtile_expert[m] = e;
-        }
-        for (int s = tid; s < n_mtiles * kBlockM; s += kRouteThreads) {
-            int e = 0;
-            while (e + 1 < E && poff[e + 1] <= s) ++e;
-            if (s - poff[e] >= cnt[e]) o.slot_assign[s] = -1;
+        for (int e = 0; e < E; ++e) {
+            for (int m = mt_start[e] + tid; m < mt_start[e + 1]; m += kRouteThreads) o.mtile_expert[m] = e;
+            for (int s = poff[e] + cnt[e] + tid; s < poff[e + 1]; s += kRouteThreads) o.slot_assign[s] = -1;
         }
     }
 }
