@@ -202,6 +202,76 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 1) route_kernel(const float*
     }
 }
 
+// ---------------------------------------------------------------- one warp
+// At most 32 assignments (decode batches): one warp, assignment a on lane a.
+// Lane t < T routes token t; each lane then takes its assignment's expert
+// from the routing lane, and the histogram, scan and stable ranks come from
+// warp votes (__ballot_sync / __match_any_sync over lanes in assignment
+// order), with no block-wide barrier on the way.
+__global__ void __launch_bounds__(32, 1) route_warp_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                           RouteOutputs o) {
+    __shared__ int s_cnt[kMaxExperts];
+    __shared__ int s_mt[kMaxExperts + 1];
+    griddep_launch_dependents();  // the gather may be scheduled; it waits for this grid
+    const unsigned full = 0xffffffffu;
+    const int lane = threadIdx.x;
+    const int A = T * k;
+    int ids[kMaxTopK];
+    for (int j = 0; j < kMaxTopK; ++j) ids[j] = -1;
+    if (lane < T) route_token(logits, lane, E, k, o, &ids);
+    // the expert of assignment a = lane, held by lane a / k at index a % k
+    int e_a = -1;
+    const int src = (lane < A) ? lane / k : 0;
+    for (int j = 0; j < k; ++j) {
+        const int v = __shfl_sync(full, ids[j], src);
+        if (lane < A && lane % k == j) e_a = v;
+    }
+    // counts, offsets and padded tile starts, expert by expert
+    int off_mine = 0, poff_mine = 0, run = 0, tiles_run = 0;
+    for (int e = 0; e < E; ++e) {
+        const int c = __popc(__ballot_sync(full, e_a == e));
+        const int tiles = (c + kBlockM - 1) / kBlockM;
+        if (lane == 0) {
+            o.counts[e] = c;
+            o.offsets[e] = run;
+            s_cnt[e] = c;
+            s_mt[e] = tiles_run;
+        }
+        if (e < e_a) {
+            off_mine += c;
+            poff_mine += tiles * kBlockM;
+        }
+        run += c;
+        tiles_run += tiles;
+    }
+    if (lane == 0) {
+        o.offsets[E] = run;
+        s_mt[E] = tiles_run;
+        if (o.num_mtiles) *o.num_mtiles = tiles_run;
+    }
+    // stable placement: rank among the lanes (assignments) before this one
+    const unsigned peers = __match_any_sync(full, e_a);
+    if (e_a >= 0) {
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int pos = off_mine + rank;
+        o.perm[pos] = lane;
+        o.inv_perm[lane] = pos;
+        if (o.slot_of) {
+            const int slot = poff_mine + rank;
+            o.slot_of[lane] = slot;
+            o.slot_assign[slot] = lane;
+        }
+    }
+    __syncwarp();
+    // padded layout: tile -> expert, padding rows -1
+    if (o.slot_assign) {
+        for (int e = 0; e < E; ++e) {
+            for (int m = s_mt[e] + lane; m < s_mt[e + 1]; m += 32) o.mtile_expert[m] = e;
+            for (int s = s_mt[e] * kBlockM + s_cnt[e] + lane; s < s_mt[e + 1] * kBlockM; s += 32) o.slot_assign[s] = -1;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- many CTAs
 // For large batches the same routing runs on many SMs in two launches.
 // route_topk_kernel: one thread per token (256 tokens per CTA) does phase 1
@@ -360,8 +430,9 @@ __global__ void __launch_bounds__(kRouteBlockTokens) route_place_kernel(int T, i
     }
 }
 
-// Four warps for small batches (the phases are short and latency-bound), 32
-// for large ones.
+// One warp for up to 32 assignments, four warps up to 1024 (the phases are
+// short and latency-bound), 32 warps above, two kernels on many SMs from 1024
+// tokens.
 // Large batches with the padded layout: two kernels on many SMs.
 static bool route_many_ctas(int T, const RouteOutputs& o) { return o.blk_counts && o.slot_of && T >= 1024; }
 
@@ -375,7 +446,9 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOu
         if (err != cudaSuccess) return err;
         return launch_dependent(route_place_kernel, dim3(nblk), dim3(kRouteBlockTokens), 0, stream, T, E, k, nblk, o);
     }
-    if ((long)T * k <= 1024)
+    if ((long)T * k <= 32)
+        route_warp_kernel<<<1, 32, 0, stream>>>(logits, T, E, k, o);
+    else if ((long)T * k <= 1024)
         route_kernel<4><<<1, 4 * 32, 0, stream>>>(logits, T, E, k, o);
     else
         route_kernel<32><<<1, 32 * 32, 0, stream>>>(logits, T, E, k, o);
