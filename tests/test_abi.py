@@ -48,6 +48,27 @@ def test_workspace_layout(moe):
     assert moe.moe_workspace_size(2000, 256, 512, 8, 2, 1) > moe.moe_workspace_size(1000, 256, 512, 8, 2, 1)
 
 
+@pytest.mark.parametrize("T,H,F,E,k,dt", [(16, 4096, 14336, 8, 2, 1), (4096, 4096, 14336, 8, 2, 1),
+                                          (300, 384, 640, 16, 3, 0), (1, 128, 128, 1, 1, 1)])
+def test_workspace_region_sizes(moe, T, H, F, E, k, dt):
+    """Each region has the size its description in moe.h gives: routing arrays
+    of T*k ints, the padded layout of S = 128*(ceil(T*k/128) + E) rows with a
+    row pitch of row bytes + 128, h's block scales as 512-byte chunks per
+    (128-row tile, 128-column block) in FP8, the fp32 combine buffer [T, H]."""
+    A = T * k
+    eb = 1 if dt == 1 else 2
+    mt_max = -(-A // 128) + E
+    S = 128 * mt_max
+    want = dict(topk_ids=4 * A, topk_w=4 * A, counts=4 * E, offsets=4 * (E + 1), perm=4 * A, inv_perm=4 * A,
+                slot_of=4 * A, xs=S * (H * eb + 128), sx=4 * S, h=S * (F * eb + 128),
+                h_sf=mt_max * (F // 128) * 512 if dt == 1 else 0, out32=4 * T * H, num_mtiles=4,
+                slot_assign=4 * S, mtile_expert=4 * mt_max, route_blocks=4 * (-(-T // 256)) * E)
+    assert set(want) == set(moe.WS)
+    for name, n in want.items():
+        off, size = moe.moe_workspace_region(T, H, F, E, k, dt, moe.WS[name])
+        assert size == n, name
+
+
 @pytest.mark.parametrize("args", [
     (16, 4096, 14336, 0, 2, 1),     # E = 0
     (16, 4096, 14336, 65, 2, 1),    # E > 64
