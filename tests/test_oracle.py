@@ -194,6 +194,26 @@ def test_route_ties_nan_and_signed_zero():
     np.testing.assert_allclose(r["w"][4], [0.5, 0.5])
 
 
+def test_route_random_shapes_with_ties():
+    """Random shapes (T from 0, E up to 16, every k) with logits drawn from a
+    small set that forces ties, signed zeros, infinities and NaN."""
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    values = st.sampled_from([0.0, -0.0, 1.0, -1.0, 0.5, 2.0, math.inf, -math.inf, math.nan])
+
+    @settings(max_examples=150, deadline=None, derandomize=True)
+    @given(st.data())
+    def check(data):
+        E = data.draw(st.integers(1, 16))
+        k = data.draw(st.integers(1, min(E, 8)))
+        T = data.draw(st.integers(0, 40))
+        flat = data.draw(st.lists(values, min_size=T * E, max_size=T * E))
+        _check_routing(np.array(flat, dtype=np.float32).reshape(T, E), k)
+
+    check()
+
+
 def test_route_k_equals_e_and_k1():
     rng = np.random.default_rng(7)
     lg = rng.normal(0, 1, (9, 4)).astype(np.float32)
