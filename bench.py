@@ -1,23 +1,30 @@
 """Benchmark of the routed MoE expert FFN layer (one JSON line on stdout).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME|all]
 
 A step is one pass of the whole layer -- routing, gather (+ FP8 quantisation),
 the w1/w3 + SwiGLU group GEMM, the w2 + scatter group GEMM and the bf16
 finalize -- over one batch of T tokens whose inputs are already resident in
-HBM.  The default workload is the Mixtral-8x7B-shaped FP8 decode layer
-(T=16, d_model=4096, d_ff=14336, E=8, top-2).  With N > 1 (one process per GPU
-under torch.distributed.run) every rank runs its own batch against its own copy
-of the weights (weak scaling); the only collectives are the timing barrier and
-the max over ranks.
+HBM.  The headline workload is the Mixtral-8x7B-shaped FP8 decode layer
+(T=16, d_model=4096, d_ff=14336, E=8, top-2); by default (``--config all``)
+the same run also times every other workload of the Mixtral expert shape
+(prefill T=4096 FP8, skewed-routing T=8192 BF16, and the FP8 batch sweep
+T = 1, 128, 1024, 16384) and reports each as a sub-record under ``configs``
+with its own step time, roofline, CPU baseline and end-to-end number.
+
+With N > 1, one process per GPU (under torch.distributed.run; ``--gpus N``
+without a launcher starts one itself) runs its own token batch against its
+own copy of the weights (weak scaling); the only collectives are the timing
+barriers and the max over ranks.
 
 ``--impl reference`` times the CPU oracle (fp64, the host's CPU cores) on a
-bounded sample of the same workload.
+bounded sample of the headline workload; under N ranks rank 0 alone runs it.
 """
 import argparse
 import hashlib
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -31,21 +38,38 @@ METRIC = "MoE-layer tokens/s (Mixtral-8x7B shape FP8, T=16 and T=4096); % of roo
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_PER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
+HEADLINE = "decode"
+# the workloads of one default run, headline first; the sweep points share one weight set
+ALL_CONFIGS = ["decode", "prefill", "skewed", "sweep_T1", "sweep_T128", "sweep_T1024", "sweep_T16384"]
+
 
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--config", default="decode")
-    p.add_argument("--cpu-sample-seconds", type=float, default=12.0)
+    p.add_argument("--config", default="all", help="a workload name, or 'all' (headline + every other workload)")
+    p.add_argument("--cpu-sample-seconds", type=float, default=12.0, help="oracle sample of the headline workload")
+    p.add_argument("--sub-cpu-sample-seconds", type=float, default=4.0, help="oracle sample of each other workload")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    return p.parse_args()
+    p.add_argument("--no-e2e", action="store_true", help="skip the end-to-end pass (profiling runs)")
+    return p.parse_args(argv)
+
+
+def config_names(arg):
+    if arg == "all":
+        return list(ALL_CONFIGS)
+    names = [n.strip() for n in arg.split(",") if n.strip()]
+    import moe_inputs
+    for n in names:
+        if n not in moe_inputs.CONFIGS:
+            raise SystemExit(f"unknown workload {n!r}; known: {sorted(moe_inputs.CONFIGS)}")
+    return names
 
 
 def load_peaks():
@@ -77,8 +101,43 @@ def algorithmic(spec, counts):
                 s1_bytes=float(s1_bytes), s2_bytes=float(s2_bytes), layer_bytes=float(layer_bytes), active=active)
 
 
+def roofline(spec, alg, dom, dom_ms, window_ms, peaks, peak_kind, name):
+    """Roofline record of the dominant kernel: algorithmic bytes (HBM-bound
+    shapes) or FLOPs (tensor-bound shapes) per launch over its average launch
+    time, against the measured peak."""
+    H, F = spec["H"], spec["F"]
+    fp8 = spec["dtype"] == "fp8"
+    decode_like = alg["active"] * 3 * H * F * (1 if fp8 else 2) / 6.5e12 > alg["layer_flops"] / (
+        (2 * 2.25e15) if fp8 else 2.25e15)
+    if not dom.startswith("stage"):
+        return {"bound": "hbm", "achieved": None, "peak": float(peaks.get("hbm_gbs", 6650.0)), "unit": "GB/s",
+                "frac": None, "traffic": None, "kernel": dom, "kernel_ms": dom_ms}
+    per = "s1" if dom.startswith("stage1") else "s2"
+    if decode_like:
+        ach = alg[per + "_bytes"] / (dom_ms / 1e3) / 1e9
+        peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                "traffic": recorded_traffic(dom, name), "peak_source": f"{peak_kind} HBM copy bandwidth",
+                "algorithmic_per_launch": alg[per + "_bytes"]}
+    else:
+        ach = alg[per + "_flops"] / (dom_ms / 1e3) / 1e12
+        # a timed region of a second or more runs under the power cap: sustained peak; else burst
+        long_run = window_ms >= 1000.0
+        key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
+        base = float(peaks.get(key, FALLBACK_PEAKS[key]))
+        peak = base * (FP8_PER_BF16 if fp8 else 1.0)
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                "traffic": recorded_traffic(dom, name),
+                "peak_source": f"{peak_kind} {'sustained' if long_run else 'burst'} bf16 cuBLAS"
+                               + (" x 2 (fp8/bf16 nominal ratio)" if fp8 else ""),
+                "algorithmic_per_launch": alg[per + "_flops"]}
+    roof["kernel"] = dom
+    roof["kernel_ms"] = dom_ms
+    return roof
+
+
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi samples of SM clock and throttle reasons while GPU work runs."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -87,6 +146,7 @@ class ClockSampler:
     def __init__(self, device_index):
         self.dev = device_index
         self.proc = None
+        self.t0 = None
 
     def start(self):
         try:
@@ -95,10 +155,12 @@ class ClockSampler:
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        self.t0 = time.perf_counter()
 
     def stop(self):
         if self.proc is None:
             return None
+        window = (time.perf_counter() - self.t0) * 1e3 if self.t0 else None
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
@@ -121,8 +183,11 @@ class ClockSampler:
                     reasons.add(name)
         if not sms:
             return None
-        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
-                "samples": len(sms)}
+        rec = {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
+               "samples": len(sms)}
+        if window is not None:
+            rec["window_ms"] = round(window, 1)
+        return rec
 
 
 def source_sha():
@@ -158,29 +223,38 @@ def recorded_traffic(kernel, workload):
     return None
 
 
-def cpu_baseline(spec, name, seconds):
+def host_cores():
+    """CPU cores this process may run on (the oracle's thread count; a launcher
+    such as torch.distributed.run sets OMP_NUM_THREADS=1, which the oracle
+    would otherwise inherit)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(case, spec, name, seconds):
     """Time the oracle (as it stands) on whole-token samples of the workload."""
     import numpy as np
 
     import moe_inputs
     import oracle
-    case = moe_inputs.make_case(spec["T"], spec["H"], spec["F"], spec["E"], spec["k"], spec["dtype"], spec["seed"],
-                                spec["skew"])
     nc = moe_inputs.to_numpy(case)
     T = spec["T"]
     batch = max(1, min(T, 8))
+    cores = host_cores()
     tokens_done = 0
     t0 = time.perf_counter()
     i = 0
     while True:
         tok = (np.arange(batch) + i * batch) % T
-        oracle.moe_ffn_tokens(nc, tok.astype(np.int32))
+        oracle.moe_ffn_tokens(nc, tok.astype(np.int32), nthreads=cores)
         tokens_done += batch
         i += 1
         if time.perf_counter() - t0 >= seconds:
             break
     dt = time.perf_counter() - t0
-    return {"value": tokens_done / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+    return {"value": tokens_done / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{tokens_done} tokens of the {name} workload ({batch}-token batches, whole layer per token: "
                       f"routing, both expert GEMMs, combine), {dt:.1f} s"}
 
@@ -201,23 +275,41 @@ def max_over_ranks(value_ms, world, device=None):
     return float(t.item())
 
 
-def run_reference(args, spec, name, rank):
+def _free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(argv, n):
+    """Re-run this script as n ranks (one per GPU) under torch.distributed.run
+    on 127.0.0.1; returns the exit status of the launcher."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={_free_port()}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def run_reference(args, rank):
     """The oracle as it stands, on the host cores: each step is one oracle call on
-    a small batch of the workload's tokens (sized so the run stays within a
-    couple of minutes)."""
+    a small batch of the headline workload's tokens (sized so the run stays
+    within a couple of minutes)."""
     if rank != 0:
         return 0
     import numpy as np
 
     import moe_inputs
     import oracle
+    names = config_names(args.config)
+    name = HEADLINE if HEADLINE in names else names[0]
+    spec = moe_inputs.CONFIGS[name]
     case = moe_inputs.make_case(spec["T"], spec["H"], spec["F"], spec["E"], spec["k"], spec["dtype"], spec["seed"],
                                 spec["skew"])
     nc = moe_inputs.to_numpy(case)
     T = spec["T"]
     batch = max(1, min(T, 8))
+    cores = host_cores()
     t0 = time.perf_counter()
-    oracle.moe_ffn_tokens(nc, np.arange(batch, dtype=np.int32))
+    oracle.moe_ffn_tokens(nc, np.arange(batch, dtype=np.int32), nthreads=cores)
     per_call = time.perf_counter() - t0
     budget = 120.0
     while batch > 1 and per_call * (args.steps + args.warmup) > budget:
@@ -225,13 +317,13 @@ def run_reference(args, spec, name, rank):
         per_call /= 2
     calls = [((np.arange(batch) + i * batch) % T).astype(np.int32) for i in range(args.warmup + args.steps)]
     for tok in calls[:args.warmup]:
-        oracle.moe_ffn_tokens(nc, tok)
+        oracle.moe_ffn_tokens(nc, tok, nthreads=cores)
     t0 = time.perf_counter()
     for tok in calls[args.warmup:]:
-        oracle.moe_ffn_tokens(nc, tok)
+        oracle.moe_ffn_tokens(nc, tok, nthreads=cores)
     dt = time.perf_counter() - t0
     value = batch * args.steps / dt
-    cb = {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+    cb = {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
           "sample": f"{args.steps} oracle calls of {batch} tokens each from the {name} workload (whole layer per "
                     f"token), {dt:.1f} s"}
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
@@ -245,49 +337,53 @@ def run_reference(args, spec, name, rank):
     return 0
 
 
-def main():
-    args = parse()
-    import moe_inputs
-    name = args.config
-    spec = moe_inputs.CONFIGS[name]
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        return run_reference(args, spec, name, rank)
+class Weights:
+    """Device weights of one (shape, dtype, seed), prepared once and shared by
+    every workload drawn from the same weight seed (the sweep points)."""
 
+    def __init__(self):
+        self.key = None
+        self.w = None
+
+    def get(self, moe, case, spec, dev):
+        import torch
+        key = (spec["H"], spec["F"], spec["E"], spec["dtype"], spec["seed"])
+        if key != self.key:
+            self.w = None
+            torch.cuda.empty_cache()
+            fp8 = spec["dtype"] == "fp8"
+            w13, s13, w2 = moe.prepare_weights(case["w1"].to(dev), case["w3"].to(dev),
+                                               case["s1"].to(dev) if fp8 else None,
+                                               case["s3"].to(dev) if fp8 else None, case["w2"].to(dev))
+            s2 = case["s2"].to(dev) if fp8 else None
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+            self.key, self.w = key, (w13, s13, w2, s2)
+        return self.w
+
+
+def run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_seconds):
+    """Time one workload: the device-timed region (K steps, inputs resident),
+    a per-kernel pass, and the end-to-end pass through the public call with
+    host buffers.  Returns its record."""
     import torch
     import torch.distributed as dist
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    # the CPU baseline runs first, before the GPU is busy (rank 0, one GPU only)
-    cb = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(spec, name, args.cpu_sample_seconds)
-
-    import mixture_experts_routed_02_b200 as moe
-    t0 = time.perf_counter()
-    # weak scaling: each rank its own batch (seed offset by rank), the same weights
-    case = moe_inputs.make_case(spec["T"], spec["H"], spec["F"], spec["E"], spec["k"], spec["dtype"], spec["seed"],
-                                spec["skew"])
-    if rank > 0:
-        case["x"] = moe_inputs.make_x(spec["T"], spec["H"], rank_batch(spec, rank))
-        case["logits"] = moe_inputs.make_logits(spec["T"], spec["E"], rank_batch(spec, rank), spec["skew"])
-    log(f"[rank {rank}] inputs generated in {time.perf_counter() - t0:.1f} s")
     T, H, F, E, k = spec["T"], spec["H"], spec["F"], spec["E"], spec["k"]
     fp8 = spec["dtype"] == "fp8"
-    x = case["x"].to(dev)
-    logits = case["logits"].to(dev)
-    s2 = case["s2"].to(dev) if fp8 else None
-    w13, s13, w2 = moe.prepare_weights(case["w1"].to(dev), case["w3"].to(dev),
-                                       case["s1"].to(dev) if fp8 else None, case["s3"].to(dev) if fp8 else None,
-                                       case["w2"].to(dev))
-    del case
-    torch.cuda.empty_cache()
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and cpu_seconds > 0:
+        cb = cpu_baseline(case, spec, name, cpu_seconds)
+
+    w13, s13, w2, s2 = weights.get(moe, case, spec, dev)
+    if rank > 0:  # weak scaling: each rank its own batch (seed offset by rank), the same weights
+        import moe_inputs
+        x_cpu = moe_inputs.make_x(T, H, rank_batch(spec, rank))
+        lg_cpu = moe_inputs.make_logits(T, E, rank_batch(spec, rank), spec["skew"])
+    else:
+        x_cpu, lg_cpu = case["x"], case["logits"]
+    x = x_cpu.to(dev)
+    logits = lg_cpu.to(dev)
     dt_code = moe.MOE_FP8_E4M3 if fp8 else moe.MOE_BF16
     ws = moe.workspace(T, H, F, E, k, dt_code, dev)
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
@@ -301,12 +397,14 @@ def main():
     torch.cuda.synchronize()
     st = moe.moe_get_status(None)
     if st != 0:
-        raise RuntimeError(f"device status {moe.STATUS_NAMES.get(st, st)} after warm-up")
+        raise RuntimeError(f"{name}: device status {moe.STATUS_NAMES.get(st, st)} after warm-up")
     counts = moe.ws_view(ws, T, H, F, E, k, dt_code, "counts", torch.int32).cpu().tolist()
 
     # ---------------- device-timed region (inputs resident in HBM).  No events
     # between the kernels here: an event recorded between two kernels would
-    # stop the next one from starting while the previous one drains.
+    # stop the next one from starting while the previous one drains.  The
+    # clock sampler runs from just before this region to the end of the
+    # end-to-end pass (all of this workload's GPU work).
     clocks = ClockSampler(torch.cuda.current_device())
     if world > 1:
         dist.barrier()
@@ -322,7 +420,6 @@ def main():
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop()
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
 
     # ---------------- per-kernel durations: the same K steps again, with a CUDA
@@ -336,7 +433,7 @@ def main():
     kern = moe.moe_profile_read(reset=True)
     st = moe.moe_get_status(None)
     if st != 0:
-        raise RuntimeError(f"device status {moe.STATUS_NAMES.get(st, st)} in the timed region")
+        raise RuntimeError(f"{name}: device status {moe.STATUS_NAMES.get(st, st)} in the timed region")
     ms_step = ms_total / args.steps
     value = T * world * args.steps / (ms_total / 1e3)
 
@@ -344,51 +441,59 @@ def main():
     # A serving loop's pipeline: two sets of device buffers; step i's inputs go
     # up on one copy stream and step i-1's result comes down on another while
     # the layer runs, each step waiting only for the copies it needs.
-    x_h = x.cpu().pin_memory()
-    lg_h = logits.cpu().pin_memory()
-    outs_h = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    xs_d, lgs_d, outs_d = [x, x.clone()], [logits, logits.clone()], [out, torch.empty_like(out)]
-    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev = lambda: torch.cuda.Event()  # noqa: E731
-    h2d_done, comp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
-    for e in comp_done + d2h_done:
-        e.record(stream)
+    e2e = None
+    if not args.no_e2e:
+        x_h = x.cpu().pin_memory()
+        lg_h = logits.cpu().pin_memory()
+        outs_h = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        xs_d, lgs_d, outs_d = [x, x.clone()], [logits, logits.clone()], [out, torch.empty_like(out)]
+        h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        h2d_done, comp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        for e in comp_done + d2h_done:
+            e.record(stream)
 
-    def e2e_step(i):
-        b = i % 2
-        h2d_s.wait_event(comp_done[b])  # the layer two steps back has read these inputs
-        with torch.cuda.stream(h2d_s):
-            xs_d[b].copy_(x_h, non_blocking=True)
-            lgs_d[b].copy_(lg_h, non_blocking=True)
-        h2d_done[b].record(h2d_s)
-        stream.wait_event(h2d_done[b])
-        stream.wait_event(d2h_done[b])  # the result two steps back has been read out
-        moe.ffn_forward(xs_d[b], lgs_d[b], w13, s13, w2, s2, k, F, fp8, out=outs_d[b], ws=ws, stream=stream)
-        comp_done[b].record(stream)
-        d2h_s.wait_event(comp_done[b])
-        with torch.cuda.stream(d2h_s):
-            outs_h[b].copy_(outs_d[b], non_blocking=True)
-        d2h_done[b].record(d2h_s)
+        def e2e_step(i):
+            b = i % 2
+            h2d_s.wait_event(comp_done[b])  # the layer two steps back has read these inputs
+            with torch.cuda.stream(h2d_s):
+                xs_d[b].copy_(x_h, non_blocking=True)
+                lgs_d[b].copy_(lg_h, non_blocking=True)
+            h2d_done[b].record(h2d_s)
+            stream.wait_event(h2d_done[b])
+            stream.wait_event(d2h_done[b])  # the result two steps back has been read out
+            moe.ffn_forward(xs_d[b], lgs_d[b], w13, s13, w2, s2, k, F, fp8, out=outs_d[b], ws=ws, stream=stream)
+            comp_done[b].record(stream)
+            d2h_s.wait_event(comp_done[b])
+            with torch.cuda.stream(d2h_s):
+                outs_h[b].copy_(outs_d[b], non_blocking=True)
+            d2h_done[b].record(d2h_s)
 
-    for i in range(max(3, args.warmup)):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ev0.record(stream)
-    h2d_s.wait_event(ev0)  # no copy of the timed steps starts before the clock does
-    d2h_s.wait_event(ev0)
-    for i in range(args.steps):
-        e2e_step(i)
-    for e in d2h_done:
-        stream.wait_event(e)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
-    e2e_value = T * world * args.steps / (e2e_ms / 1e3)
-    last = (args.steps - 1) % 2
-    if not torch.equal(outs_h[last], outs_d[last].cpu()):
-        raise RuntimeError("the result read back to the host is not the last step's output")
+        for i in range(max(3, args.warmup)):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ev0.record(stream)
+        h2d_s.wait_event(ev0)  # no copy of the timed steps starts before the clock does
+        d2h_s.wait_event(ev0)
+        for i in range(args.steps):
+            e2e_step(i)
+        for e in d2h_done:
+            stream.wait_event(e)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        last = (args.steps - 1) % 2
+        if not torch.equal(outs_h[last], outs_d[last].cpu()):
+            raise RuntimeError(f"{name}: the result read back to the host is not the last step's output")
+        e2e = {"value": T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 2,
+               "ms_per_step": e2e_ms / args.steps}
+        st = moe.moe_get_status(None)
+        if st != 0:
+            raise RuntimeError(f"{name}: device status {moe.STATUS_NAMES.get(st, st)} in the end-to-end pass")
+    clk = clocks.stop()
 
     # ---------------- roofline of the dominant kernel
     peaks, peak_kind = load_peaks()
@@ -396,42 +501,15 @@ def main():
     names = moe.KERNELS
     dom = max(names, key=lambda n: kern[n][0])
     dom_ms = kern[dom][0] / max(1, kern[dom][1])
-    decode_like = alg["active"] * 3 * H * F * (1 if fp8 else 2) / 6.5e12 > alg["layer_flops"] / (
-        (2 * 2.25e15) if fp8 else 2.25e15)
-    if dom.startswith("stage"):
-        per = "s1" if dom.startswith("stage1") else "s2"
-        if decode_like:
-            ach = alg[per + "_bytes"] / (dom_ms / 1e3) / 1e9
-            peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-            roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                    "traffic": recorded_traffic(dom, name),
-                    "peak_source": f"{peak_kind} HBM copy bandwidth"}
-        else:
-            ach = alg[per + "_flops"] / (dom_ms / 1e3) / 1e12
-            # a timed region of a second or more runs under the power cap: sustained peak; else burst
-            long_run = ms_total >= 1000.0
-            key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
-            base = float(peaks.get(key, FALLBACK_PEAKS[key]))
-            peak = base * (FP8_PER_BF16 if fp8 else 1.0)
-            roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                    "traffic": recorded_traffic(dom, name),
-                    "peak_source": f"{peak_kind} {'sustained' if long_run else 'burst'} bf16 cuBLAS"
-                                   + (" x 2 (fp8/bf16 nominal ratio)" if fp8 else "")}
-    else:
-        roof = {"bound": "hbm", "achieved": None, "peak": float(peaks.get("hbm_gbs", 6650.0)), "unit": "GB/s",
-                "frac": None, "traffic": None}
-    roof["kernel"] = dom
-    roof["kernel_ms"] = dom_ms
-
+    roof = roofline(spec, alg, dom, dom_ms, ms_total, peaks, peak_kind, name)
     launches = sum(v[1] for v in kern.values())  # K steps, the same count as the timed region
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)" if fp8 else "bf16 (fp32 accumulate)",
-        "data": "synthetic (seeded; random-init weights of the Mixtral-8x7B expert shape)",
+    rec = {
+        "value": value, "unit": "tokens/s", "ms_per_step": ms_step, "steps": args.steps, "warmup": args.warmup,
+        "dtype": "fp8_e4m3 (fp32 accumulate)" if fp8 else "bf16 (fp32 accumulate)",
         "config": {"workload": workload_desc(spec, name), "T": T, "d_model": H, "d_ff": F, "experts": E, "top_k": k,
                    "weights": spec["dtype"], "parallelism": f"weak-scaling replicas x{world}" if world > 1 else "1 GPU",
-                   "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (alg["active"] * 3 * H * F * (1 if fp8 else 2) / 1e9),
+                   "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (
+                       alg["active"] * 3 * H * F * (1 if fp8 else 2) / 1e9),
                    "expert_counts": counts},
         "roofline": roof,
         "layer": {"tflops": alg["layer_flops"] / (ms_step / 1e3) / 1e12,
@@ -440,11 +518,74 @@ def main():
         "kernels_ms_per_step": {n: kern[n][0] / args.steps for n in names},
         "kernel_timing": "separate pass of the same K steps with an event pair around each kernel",
         "cpu_baseline": cb,
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2 + T * E * 4,
-                "d2h_bytes_per_step": T * H * 2},
+        "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk,
     }
+    del ws, out, x, logits
+    return rec
+
+
+def main(argv=None):
+    raw_argv = sys.argv[1:] if argv is None else list(argv)
+    args = parse(raw_argv)
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        # no launcher: start one process per GPU ourselves
+        return launch_ranks(raw_argv, args.gpus)
+    world = int(env_world or "1")
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} does not match WORLD_SIZE={world}")
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+
+    import moe_inputs
+    import torch
+    import torch.distributed as dist
+    names = config_names(args.config)
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    import mixture_experts_routed_02_b200 as moe
+    weights = Weights()
+    host_w = {}  # host weights of the last (shape, dtype, seed): the sweep points share them
+    records = {}
+    for i, name in enumerate(names):
+        spec = moe_inputs.CONFIGS[name]
+        t0 = time.perf_counter()
+        wkey = (spec["H"], spec["F"], spec["E"], spec["dtype"], spec["seed"])
+        if wkey not in host_w:
+            host_w = {wkey: moe_inputs.make_weights(spec["H"], spec["F"], spec["E"], spec["dtype"], spec["seed"])}
+        case = moe_inputs.make_case(spec["T"], spec["H"], spec["F"], spec["E"], spec["k"], spec["dtype"],
+                                    spec["seed"], spec["skew"], weights=host_w[wkey])
+        log(f"[rank {rank}] {name}: inputs generated in {time.perf_counter() - t0:.1f} s")
+        cpu_s = args.cpu_sample_seconds if i == 0 else args.sub_cpu_sample_seconds
+        records[name] = run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_s)
+        del case
+        r = records[name]
+        log(f"[rank {rank}] {name}: {r['ms_per_step'] * 1e3:.1f} us/step, {r['value']:.0f} tokens/s, "
+            f"{r['roofline']['kernel']} at {r['roofline']['frac']:.3f} of {r['roofline']['unit']} peak")
+
+    head = names[0]
+    h = records[head]
+    line = {
+        "metric": METRIC, "value": h["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": h["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": h["dtype"],
+        "data": "synthetic (seeded; random-init weights of the Mixtral-8x7B expert shape)",
+        "config": h["config"], "roofline": h["roofline"], "layer": h["layer"],
+        "kernels_ms_per_step": h["kernels_ms_per_step"], "kernel_timing": h["kernel_timing"],
+        "cpu_baseline": h["cpu_baseline"], "e2e": h["e2e"], "gpu_launches": h["gpu_launches"], "clocks": h["clocks"],
+    }
+    if len(names) > 1:
+        line["configs"] = {n: records[n] for n in names[1:]}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -91,19 +91,29 @@ def _weight(E, rows, cols, seed, stream, dtype):
     return codes, scales
 
 
-def make_case(T, H, F, E, k, dtype="bf16", seed=0, skew=False):
-    """All inputs of one layer call as torch CPU tensors.
-
-    Returns dict(x bf16 [T,H], logits f32 [T,E], w1/w3 [E,F,H], w2 [E,H,F]
-    (bf16 or float8_e4m3fn), s1/s3 f32 [E,F], s2 f32 [E,H] (fp8 only, else
-    None), and the scalars T,H,F,E,k,dtype,seed)."""
+def make_weights(H, F, E, dtype="bf16", seed=0):
+    """The expert weights of a case alone: dict(w1, w3, s1, s3, w2, s2) as in
+    ``make_case`` (the same draws for the same shape, dtype and seed)."""
     if dtype not in ("bf16", "fp8"):
         raise ValueError(dtype)
     w1, s1 = _weight(E, F, H, seed, _S_W1, dtype)
     w3, s3 = _weight(E, F, H, seed, _S_W3, dtype)
     w2, s2 = _weight(E, H, F, seed, _S_W2, dtype)
-    return dict(x=make_x(T, H, seed), logits=make_logits(T, E, seed, skew), w1=w1, w3=w3, w2=w2, s1=s1,
-                s3=s3, s2=s2, T=T, H=H, F=F, E=E, k=k, dtype=dtype, seed=seed)
+    return dict(w1=w1, w3=w3, w2=w2, s1=s1, s3=s3, s2=s2)
+
+
+def make_case(T, H, F, E, k, dtype="bf16", seed=0, skew=False, weights=None):
+    """All inputs of one layer call as torch CPU tensors.
+
+    Returns dict(x bf16 [T,H], logits f32 [T,E], w1/w3 [E,F,H], w2 [E,H,F]
+    (bf16 or float8_e4m3fn), s1/s3 f32 [E,F], s2 f32 [E,H] (fp8 only, else
+    None), and the scalars T,H,F,E,k,dtype,seed).  ``weights``, if given, is
+    the result of ``make_weights(H, F, E, dtype, seed)`` (reused, not redrawn)."""
+    if dtype not in ("bf16", "fp8"):
+        raise ValueError(dtype)
+    w = weights if weights is not None else make_weights(H, F, E, dtype, seed)
+    return dict(x=make_x(T, H, seed), logits=make_logits(T, E, seed, skew), **w,
+                T=T, H=H, F=F, E=E, k=k, dtype=dtype, seed=seed)
 
 
 def make_config(name):

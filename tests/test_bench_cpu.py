@@ -90,3 +90,29 @@ def test_clock_samples(lines, reasons, median):
     assert clk["reasons"] == reasons
     assert clk["sm_mhz"] == median
     assert clk["sm_max_mhz"] == 1965.0
+
+
+def test_default_run_times_every_mixtral_workload():
+    """The default bench run (`--config all`) times the headline decode layer
+    first and every other Mixtral-shaped workload after it."""
+    import moe_inputs
+    names = bench.config_names("all")
+    assert names[0] == bench.HEADLINE == "decode"
+    assert set(names) == set(moe_inputs.CONFIGS) - {"tiny"}
+    assert bench.config_names("prefill,sweep_T1") == ["prefill", "sweep_T1"]
+    with pytest.raises(SystemExit):
+        bench.config_names("no-such-workload")
+
+
+def test_tensor_bound_roofline_uses_fp8_peak_from_bf16():
+    spec = dict(T=4096, H=4096, F=14336, E=8, k=2, dtype="fp8", skew=False)
+    alg = bench.algorithmic(spec, [1024] * 8)
+    peaks = {"hbm_gbs": 6540.0, "bf16_tflops": 1633.0, "bf16_tflops_sustained": 1374.0}
+    r = bench.roofline(spec, alg, "stage1_w13_swiglu", 1.0, 30.0, peaks, "measured", "prefill")
+    assert r["bound"] == "tensor" and r["peak"] == 2 * 1633.0
+    assert abs(r["achieved"] - alg["s1_flops"] / 1e-3 / 1e12) < 1e-6
+    r = bench.roofline(spec, alg, "stage1_w13_swiglu", 1.0, 2000.0, peaks, "measured", "prefill")
+    assert r["peak"] == 2 * 1374.0  # a long timed region runs under the power cap
+    d = bench.roofline(dict(spec, T=16), bench.algorithmic(dict(spec, T=16), [4] * 8), "stage1_w13_swiglu", 0.15,
+                       5.0, peaks, "measured", "decode")
+    assert d["bound"] == "hbm" and d["unit"] == "GB/s"

@@ -1,6 +1,7 @@
 """The multi-process plumbing of bench.py on CPU: two gloo ranks (world size 2)
 agree on the max-over-ranks time, draw different token batches for the same
-weights, and the reference arm runs on rank 0 only."""
+weights, the reference arm runs on rank 0 only, and ``bench.py --gpus 2``
+without a launcher starts two ranks itself and prints one line."""
 import json
 import os
 import subprocess
@@ -64,3 +65,29 @@ def test_reference_arm_rank_behaviour(rank):
         assert d["cpu_baseline"]["kind"] == "oracle"
     else:
         assert lines == []
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` with no launcher in the environment starts two
+    ranks under torch.distributed.run (127.0.0.1); rank 0 alone prints, and
+    the line reports both ranks."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR",
+                                                             "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                        "--steps", "2", "--warmup", "1", "--gpus", "2"], capture_output=True, text=True, env=env,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["impl"] == "reference"
+    assert d["cpu_baseline"]["cores"] >= 1
+
+
+def test_gpus_flag_must_match_the_launcher():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                        "--steps", "1", "--warmup", "1", "--gpus", "4"], capture_output=True, text=True, env=env,
+                       timeout=120)
+    assert r.returncode != 0
+    assert "does not match WORLD_SIZE" in r.stderr
