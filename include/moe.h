@@ -145,7 +145,9 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
  * graph (no cudaMalloc allowed then), hosts whose device memory belongs to an
  * allocator they cannot call, runtimes with a fixed memory budget.  The pages
  * have no counterpart of this entry point; it is a property of this library.
- *   Arguments, results and numerics are those of moe_ffn_forward; the
+ *   Arguments, results and numerics are those of moe_ffn_forward, and the
+ *   arguments are checked in the same order (MOE_ERR_INVALID_ARG,
+ *   MOE_ERR_UNSUPPORTED, MOE_ERR_ALIGNMENT before MOE_ERR_WORKSPACE); the
  *   workspace is a device array built into the library,
  *   moe_static_workspace_bytes() long (64 MiB).  The driver reserves it on
  *   every GPU that loads the library's device code and keeps it until the
@@ -153,9 +155,11 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
  *   Returns MOE_ERR_WORKSPACE, before enqueuing anything, when the problem
  *   needs more than that (moe_workspace_size(T,H,F,E,k,dtype) bytes); decode
  *   batches of Mixtral-8x7B experts fit (T = 16: about 22 MB FP8, 43 MB BF16).
- *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before capturing a stream.
+ *   The first call in each CUDA context looks up the array's device address
+ *   (cudaGetSymbolAddress) with that context current; make that first call
+ *   before capturing a stream.  A device reset (cudaDeviceReset) ends the
+ *   context: the next call is again a first call and looks the address up
+ *   in the new context.
  *   All calls on a device share the one array, which keeps the last call's
  *   contents (every call rewrites all it reads; nothing needs to start at
  *   zero).  Calls whose work overlaps on the GPU -- e.g. on two streams at
@@ -211,8 +215,24 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
  *                     bounded waits run out, the call's outputs are undefined
  *                     and moe_get_status reports MOE_ERR_DEVICE_TIMEOUT; the
  *                     context stays usable.  0 (default) = off.
+ *   MOE_OPT_TEST_CORRUPT: test of the bounds checks: after routing, the host
+ *                     enqueues a 4-byte write of bytes 0x7F (an index far out
+ *                     of range) over the first entry of one routing table --
+ *                     1 = assignment -> padded row (read by the gather),
+ *                     2 = padded row -> assignment (read by the second GEMM's
+ *                     scatter), 3 = 128-row tile -> expert (read by both
+ *                     GEMMs).  The kernel that reads it records
+ *                     MOE_ERR_DEVICE_BOUNDS and skips the access; the call's
+ *                     outputs are undefined and the context stays usable.
+ *                     0 (default) = off.
  * Returns the previous value, or MOE_ERR_INVALID_ARG. */
-typedef enum { MOE_OPT_PATH = 0, MOE_OPT_SPLITK = 1, MOE_OPT_TIMEOUT_MS = 2, MOE_OPT_TEST_STALL = 3 } moe_option;
+typedef enum {
+    MOE_OPT_PATH = 0,
+    MOE_OPT_SPLITK = 1,
+    MOE_OPT_TIMEOUT_MS = 2,
+    MOE_OPT_TEST_STALL = 3,
+    MOE_OPT_TEST_CORRUPT = 4
+} moe_option;
 int moe_set_option(int option, int value);
 
 /* Per-kernel device timing (tracing aid).  While enabled, moe_ffn_forward

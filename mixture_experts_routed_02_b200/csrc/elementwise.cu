@@ -29,7 +29,8 @@ constexpr int kRegVec = 4;
 
 template <bool kFP8, bool kPerToken>
 __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int k,
-                                                    const int* __restrict__ slot_of, uint8_t* __restrict__ xs,
+                                                    const int* __restrict__ slot_of, int num_slots,
+                                                    uint8_t* __restrict__ xs,
                                                     float* __restrict__ sx_slot, float* __restrict__ out32,
                                                     int* __restrict__ status) {
     __shared__ float warp_max[4];
@@ -62,7 +63,7 @@ __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __r
     bool bad = false;
     for (int j = 0; j < n; ++j) {
         slots[j] = slot_of[a0 + j];
-        bad |= slots[j] < 0;
+        bad |= slots[j] < 0 || slots[j] >= num_slots;  // never from the router: a corrupted table
     }
     if (bad) {
         if (tid == 0) record_error(status, MOE_ERR_DEVICE_BOUNDS);
@@ -139,20 +140,20 @@ __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __r
     }
 }
 
-cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
-                          float* sx_slot, float* out32, int* status, cudaStream_t stream) {
+cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, int num_slots,
+                          uint8_t* xs, float* sx_slot, float* out32, int* status, cudaStream_t stream) {
     // a CTA per token for large batches, per assignment (more CTAs, shorter
     // critical path) for small ones
     const bool per_token = T >= 256;
     const dim3 grid(std::max(1, per_token ? T : T * k));
     if (fp8)
-        return per_token ? launch_dependent(gather_kernel<true, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
+        return per_token ? launch_dependent(gather_kernel<true, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of, num_slots,
                                             xs, sx_slot, out32, status)
-                         : launch_dependent(gather_kernel<true, false>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
+                         : launch_dependent(gather_kernel<true, false>, grid, dim3(128), 0, stream, x, T, H, k, slot_of, num_slots,
                                             xs, sx_slot, out32, status);
-    return per_token ? launch_dependent(gather_kernel<false, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of, xs,
+    return per_token ? launch_dependent(gather_kernel<false, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of, num_slots, xs,
                                         sx_slot, out32, status)
-                     : launch_dependent(gather_kernel<false, false>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
+                     : launch_dependent(gather_kernel<false, false>, grid, dim3(128), 0, stream, x, T, H, k, slot_of, num_slots,
                                         xs, sx_slot, out32, status);
 }
 

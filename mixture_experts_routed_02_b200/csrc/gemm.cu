@@ -192,7 +192,11 @@ __global__ void __launch_bounds__(192, 1)
 
     // The routing tables were written two launches back, so they may be read
     // before the wait for the previous kernel (see griddep_wait).
-    const int num_mt = *args.num_mtiles;
+    int num_mt = *args.num_mtiles;
+    if (num_mt < 0 || num_mt > args.mt_max) {  // never from the router: a corrupted table
+        if (threadIdx.x == 0) record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
+        num_mt = 0;
+    }
     const int ns = args.n_tiles * args.splits;
     const int tiles = PAIR ? s_pair_first[args.num_experts] * ns : num_mt * ns;
     const int kps = args.k_tiles / args.splits;
@@ -269,6 +273,16 @@ __global__ void __launch_bounds__(192, 1)
             decode_tile(u, num_mt, args.n_tiles, m, n, split);
         }
     };
+    // Expert of m-tile m; an index out of range (never from the router) is
+    // recorded and replaced by expert 0, so no access leaves the weights.
+    auto expert_of = [&](int m) {
+        int e = args.mtile_expert[m];
+        if (e < 0 || e >= args.num_experts) {
+            record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
+            e = 0;
+        }
+        return e;
+    };
     // One-CTA tiles whose m-tile holds at most 32 rows in use (small batches:
     // a few tokens per expert) copy only those 32 activation rows; the MMA
     // still reads 128 rows, and the results of the rows not copied (stale
@@ -317,7 +331,7 @@ __global__ void __launch_bounds__(192, 1)
         int m, n, split, q4;
         bool dup;
         unit_coords(unit0, m, n, split, dup, q4);
-        const int e = args.mtile_expert[m];
+        const int e = expert_of(m);
         const uint32_t tx = stage_tx(a_rows32(m), q4);
         npre = min(NST, kps);
         for (int kk = 0; kk < npre; ++kk) {  // fresh stages: nothing to wait for
@@ -339,7 +353,7 @@ __global__ void __launch_bounds__(192, 1)
                 int m, n, split, q4;
                 bool dup;
                 unit_coords(u, m, n, split, dup, q4);
-                const int e = args.mtile_expert[m];
+                const int e = expert_of(m);
                 const bool small = a_rows32(m);
                 if (AR == 32 && !small) record_error(args.status, MOE_ERR_DEVICE_BOUNDS);  // host chose this wrongly
                 for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
@@ -528,7 +542,7 @@ __global__ void __launch_bounds__(192, 1)
             unit_coords(u, m, n, split, dup, q4);
             if (!wait(&tfull[acc], acc_phase)) break;
             tc_fence_after();
-            const int e = args.mtile_expert[m];
+            const int e = expert_of(m);
             const int slot = m * kBlockM + row;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             if constexpr (STAGE == 1) {
@@ -610,7 +624,7 @@ __global__ void __launch_bounds__(192, 1)
             } else {
                 const int a = dup ? -1 : args.slot_assign[slot];
                 int t = (a >= 0) ? a / args.topk : -1;
-                if (t >= args.T) {
+                if (t >= args.T || a < -1) {
                     record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
                     t = -1;
                 }

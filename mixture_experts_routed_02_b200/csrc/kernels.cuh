@@ -97,11 +97,20 @@ int max_active_clusters(void (*kernel)(KArgs...), int threads, size_t smem, int 
     return n;
 }
 
+// Host-side helpers of the entry points (moe_api.cu).
+// Key of the CUDA context current on the calling thread: the driver's
+// context id, never reused (false if no context is current).
+bool context_key(unsigned long long* key);
+// The host-side argument checks of a layer call (everything but the
+// workspace size), in the order the layer entry points apply them.
+int check_forward_args(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
+                       const float* s2, int T, int H, int F, int E, int k, int dtype, const void* out, const void* ws);
+
 // Host launchers (each defined next to its kernel).
 cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream);
 int route_launches(int T, const RouteOutputs& o);  // kernels launch_route enqueues (1 or 2)
-cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, uint8_t* xs,
-                          float* sx_slot, float* out32, int* status, cudaStream_t stream);
+cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, int num_slots,
+                          uint8_t* xs, float* sx_slot, float* out32, int* status, cudaStream_t stream);
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream);
 // Blocked, pre-swizzled weight layout (see moe_prepare_weights in moe.h).
 constexpr int kWBlockRows = 128;
@@ -137,6 +146,7 @@ struct GemmArgs {
     int group_m;              // expert-major tile order (see tile_coords in gemm.cu)
     const int* counts;        // rows per expert [num_experts] (for group_m)
     int num_experts;
+    int mt_max;               // bound of *num_mtiles (a larger value is a corrupted table)
 };
 
 // Tensor maps of one GEMM launch: a = activation rows (128-row boxes, 128-byte

@@ -28,6 +28,7 @@ std::atomic<int> g_opt_path{0};
 std::atomic<int> g_opt_splitk{0};
 std::atomic<int> g_opt_timeout_ms{2000};
 std::atomic<int> g_opt_test_stall{0};
+std::atomic<int> g_opt_test_corrupt{0};
 
 // ---------------------------------------------------------------- profiling
 
@@ -74,38 +75,85 @@ struct ProfScope {
     }
 };
 
-constexpr int kMaxDevices = 64;
-int* g_status_ptr[kMaxDevices] = {nullptr};
-int g_num_sms[kMaxDevices] = {0};
-int g_max_pairs[kMaxDevices][2][2];  // [device][stage-1][fp8]; valid once g_status_ptr is set
-std::mutex g_dev_mutex;
+// ---------------------------------------------------------------- per-context state
+// The status word's device address, the SM count and the resident CTA pairs
+// are looked up once per CUDA context (not per device ordinal: after a device
+// reset, or under another driver-API context on the same device, an address
+// taken in the old context is no longer valid).  A context is identified by
+// the driver's unique context id (cuCtxGetId), which is never reused.
 
-// Address of this device's status word and its SM count (looked up once per device).
-int device_info(int** status, int* num_sms) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_dev_mutex);
-    if (!g_status_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return MOE_ERR_CUDA;
-        int sms = 0;
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
-        for (int s = 0; s < 2; ++s)
-            for (int f = 0; f < 2; ++f) g_max_pairs[dev][s][f] = gemm_max_pairs(s + 1, f != 0);
-        g_status_ptr[dev] = static_cast<int*>(p);
-        g_num_sms[dev] = sms;
-    }
-    *status = g_status_ptr[dev];
-    *num_sms = g_num_sms[dev];
-    return MOE_OK;
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(p);
 }
 
-// Resident CTA pairs of a stage's pair kernel on the current device (after device_info).
-int max_pairs(int stage, bool fp8) {
+}  // namespace
+
+// Key of the context current on this thread: the driver's context id, which
+// is never reused (or, where the driver offers no ids, one key per device
+// ordinal).  False when no context is current yet.
+bool context_key(unsigned long long* key) {
+    static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-    std::lock_guard<std::mutex> lock(g_dev_mutex);
-    return g_status_ptr[dev] ? g_max_pairs[dev][stage - 1][fp8 ? 1 : 0] : 0;
+    if (get_current) {
+        CUcontext ctx = nullptr;
+        if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+        if (get_id && get_id(ctx, key) == CUDA_SUCCESS) return true;
+    }
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    *key = ~0ull - (unsigned long long)dev;
+    return true;
+}
+
+namespace {
+
+struct CtxInfo {
+    unsigned long long ctx_id;
+    int* status;
+    int num_sms;
+    int max_pairs[2][2];  // [stage-1][fp8]
+};
+constexpr int kMaxContexts = 64;
+CtxInfo g_ctx[kMaxContexts];
+int g_ctx_count = 0, g_ctx_next = 0;
+std::mutex g_ctx_mutex;
+
+// Per-context state of the current context, looked up (and its context made
+// current by the runtime, if none was) on first use.
+int context_info(CtxInfo* out) {
+    std::lock_guard<std::mutex> lock(g_ctx_mutex);
+    unsigned long long key = 0;
+    if (context_key(&key)) {
+        for (int i = 0; i < g_ctx_count; ++i)
+            if (g_ctx[i].ctx_id == key) {
+                *out = g_ctx[i];
+                return MOE_OK;
+            }
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    CtxInfo c{};
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    for (int st = 0; st < 2; ++st)
+        for (int f = 0; f < 2; ++f) c.max_pairs[st][f] = gemm_max_pairs(st + 1, f != 0);
+    c.status = static_cast<int*>(p);
+    if (!context_key(&key)) return MOE_ERR_CUDA;  // the lookup above made a context current
+    c.ctx_id = key;
+    g_ctx[g_ctx_next] = c;
+    g_ctx_next = (g_ctx_next + 1) % kMaxContexts;
+    if (g_ctx_count < kMaxContexts) ++g_ctx_count;
+    *out = c;
+    return MOE_OK;
 }
 
 // ---------------------------------------------------------------- workspace
@@ -216,6 +264,72 @@ bool make_map_rows(CUtensorMap* map, const void* base, size_t rows, int box_rows
 
 int launch_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// ---------------------------------------------------------------- tensor-map cache
+// The tensor maps of a call depend only on the buffers' addresses and the
+// problem's shape, so they are encoded once per (workspace, weights, shape,
+// tile configuration) and reused by later calls with the same arguments.
+
+struct MapKey {
+    const void* ws;
+    const void* w13;
+    const void* w2;
+    int T, H, F, E, k, dtype, cfg1, cfg2;
+    bool operator==(const MapKey& o) const {
+        return ws == o.ws && w13 == o.w13 && w2 == o.w2 && T == o.T && H == o.H && F == o.F && E == o.E &&
+               k == o.k && dtype == o.dtype && cfg1 == o.cfg1 && cfg2 == o.cfg2;
+    }
+};
+struct MapSet {
+    CUtensorMap ta1, ta2, ta1s, ta2s, tb1, tb2, tsf2;
+};
+constexpr int kMapCache = 16;
+struct MapEntry {
+    MapKey key;
+    MapSet maps;
+    bool valid;
+};
+MapEntry g_maps[kMapCache];
+int g_maps_next = 0;
+std::mutex g_maps_mutex;
+
+bool find_maps(const MapKey& key, MapSet* out) {
+    std::lock_guard<std::mutex> lock(g_maps_mutex);
+    for (const MapEntry& m : g_maps)
+        if (m.valid && m.key == key) {
+            *out = m.maps;
+            return true;
+        }
+    return false;
+}
+
+void store_maps(const MapKey& key, const MapSet& maps) {
+    std::lock_guard<std::mutex> lock(g_maps_mutex);
+    g_maps[g_maps_next] = {key, maps, true};
+    g_maps_next = (g_maps_next + 1) % kMapCache;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- argument checks
+// The host-side checks of a layer call, in the order both layer entry points
+// apply them (dimensions, null pointers, supported shapes, alignment); the
+// workspace size is checked after them.
+int check_forward_args(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
+                       const float* s2, int T, int H, int F, int E, int k, int dtype, const void* out, const void* ws) {
+    if (!dims_ok(T, H, F, E, k, dtype)) return MOE_ERR_INVALID_ARG;
+    const bool fp8 = dtype == MOE_FP8_E4M3;
+    if (!w13 || !w2 || !ws || (fp8 && (!s13 || !s2))) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !logits || !out)) return MOE_ERR_INVALID_ARG;
+    if (H % 128 || F % 128) return MOE_ERR_UNSUPPORTED;
+    if ((long long)T * k > 262144) return MOE_ERR_UNSUPPORTED;
+    const void* ptrs[] = {x, logits, w13, s13, w2, s2, out, ws};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+    return MOE_OK;
+}
+
+namespace {
+
 // K splits of the second GEMM: enough work units for every SM when the layer
 // is small (decode), 1 otherwise.  Must divide F/128.
 int choose_splits(int mt_est, int n_tiles, int k_tiles, int num_sms) {
@@ -261,6 +375,9 @@ int moe_set_option(int option, int value) {
         case MOE_OPT_TEST_STALL:
             if (value < 0 || value > 1) return MOE_ERR_INVALID_ARG;
             return g_opt_test_stall.exchange(value);
+        case MOE_OPT_TEST_CORRUPT:
+            if (value < 0 || value > 3) return MOE_ERR_INVALID_ARG;
+            return g_opt_test_corrupt.exchange(value);
         default:
             return MOE_ERR_INVALID_ARG;
     }
@@ -304,24 +421,20 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float
 int moe_ffn_forward(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
                     const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
                     size_t ws_bytes, void* stream) {
-    if (!dims_ok(T, H, F, E, k, dtype)) return MOE_ERR_INVALID_ARG;
+    const int rc_args = check_forward_args(x, logits, w13, s13, w2, s2, T, H, F, E, k, dtype, out, ws);
+    if (rc_args != MOE_OK) return rc_args;
     const bool fp8 = dtype == MOE_FP8_E4M3;
-    if (!w13 || !w2 || !ws || (fp8 && (!s13 || !s2))) return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (!x || !logits || !out)) return MOE_ERR_INVALID_ARG;
-    if (H % 128 || F % 128) return MOE_ERR_UNSUPPORTED;
-    if ((long long)T * k > 262144) return MOE_ERR_UNSUPPORTED;
-    const void* ptrs[] = {x, logits, w13, s13, w2, s2, out, ws};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
     const Layout L = make_layout(T, H, F, E, k, dtype);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     const int opt_path = g_opt_path.load();  // read once per call
     if (opt_path == 4 && L.A > 32) return MOE_ERR_UNSUPPORTED;  // forced tiny-batch tiles
     if (T == 0) return MOE_OK;
 
-    int* status = nullptr;
-    int num_sms = 0;
-    if (device_info(&status, &num_sms) != MOE_OK) return MOE_ERR_CUDA;
+    CtxInfo ctx{};
+    if (context_info(&ctx) != MOE_OK) return MOE_ERR_CUDA;
+    int* status = ctx.status;
+    const int num_sms = ctx.num_sms;
+    auto max_pairs = [&](int stage, bool f8) { return ctx.max_pairs[stage - 1][f8 ? 1 : 0]; };
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* w = static_cast<uint8_t*>(ws);
     auto reg = [&](int r) { return w + L.off[r]; };
@@ -355,19 +468,24 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     const int bn2 = gemm_block_n(2, fp8, cfg2);
     if ((2 * F) % bn1 || H % bn2) return MOE_ERR_UNSUPPORTED;
 
-    CUtensorMap ta1, ta2, ta1s, ta2s, tb1, tb2, tsf2;
-    if (!make_map(&ta1, reg(MOE_WS_XS), L.S_max, H, act_pitch((long)H * eb), eb, kBlockM) ||
-        !make_map(&ta2, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, kBlockM) ||
-        !make_map(&ta1s, reg(MOE_WS_XS), L.S_max, H, act_pitch((long)H * eb), eb, 32) ||
-        !make_map(&ta2s, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, 32))
-        return MOE_ERR_CUDA;
-    if (cfg1 == 0 && !make_map_rows(&tb1, w13, (size_t)E * (2 * F) * (H * eb / 128), kWBlockRows))
-        return MOE_ERR_CUDA;
-    if (cfg2 == 0 && !make_map_rows(&tb2, w2, (size_t)E * H * (F * eb / 128), kWBlockRows)) return MOE_ERR_CUDA;
-    if (cfg2 == 0 && fp8 && !make_map_rows(&tsf2, reg(MOE_WS_H_SF), (size_t)L.MT_max * (F / 128) * 4, 4))
-        return MOE_ERR_CUDA;
-    const GemmMaps maps1{&ta1, &ta1s, cfg1 == 0 ? &tb1 : nullptr, nullptr};
-    const GemmMaps maps2{&ta2, &ta2s, cfg2 == 0 ? &tb2 : nullptr, (cfg2 == 0 && fp8) ? &tsf2 : nullptr};
+    const MapKey mkey{ws, w13, w2, T, H, F, E, k, dtype, cfg1, cfg2};
+    MapSet ms;
+    if (!find_maps(mkey, &ms)) {
+        if (!make_map(&ms.ta1, reg(MOE_WS_XS), L.S_max, H, act_pitch((long)H * eb), eb, kBlockM) ||
+            !make_map(&ms.ta2, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, kBlockM) ||
+            !make_map(&ms.ta1s, reg(MOE_WS_XS), L.S_max, H, act_pitch((long)H * eb), eb, 32) ||
+            !make_map(&ms.ta2s, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, 32))
+            return MOE_ERR_CUDA;
+        if (cfg1 == 0 && !make_map_rows(&ms.tb1, w13, (size_t)E * (2 * F) * (H * eb / 128), kWBlockRows))
+            return MOE_ERR_CUDA;
+        if (cfg2 == 0 && !make_map_rows(&ms.tb2, w2, (size_t)E * H * (F * eb / 128), kWBlockRows))
+            return MOE_ERR_CUDA;
+        if (cfg2 == 0 && fp8 && !make_map_rows(&ms.tsf2, reg(MOE_WS_H_SF), (size_t)L.MT_max * (F / 128) * 4, 4))
+            return MOE_ERR_CUDA;
+        store_maps(mkey, ms);
+    }
+    const GemmMaps maps1{&ms.ta1, &ms.ta1s, cfg1 == 0 ? &ms.tb1 : nullptr, nullptr};
+    const GemmMaps maps2{&ms.ta2, &ms.ta2s, cfg2 == 0 ? &ms.tb2 : nullptr, (cfg2 == 0 && fp8) ? &ms.tsf2 : nullptr};
     // grid: one CTA per SM at most; pairs: whole clusters that can be resident
     auto grid_for = [&](int stage, int c, long units_per_mtile) {
         if (c == 0) {
@@ -389,6 +507,13 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
         ProfScope ps(MOE_KERNEL_ROUTE, st, route_launches(T, o));
         if (launch_route(logits, T, E, k, o, st) != cudaSuccess) return MOE_ERR_CUDA;
     }
+    // failure-detection test hook: overwrite one entry of a routing table with
+    // an index far out of range (bytes 0x7F), as a corrupted table would hold
+    const int corrupt = g_opt_test_corrupt.load();
+    if (corrupt) {
+        void* target = corrupt == 1 ? (void*)o.slot_of : corrupt == 2 ? (void*)o.slot_assign : (void*)o.mtile_expert;
+        if (cudaMemsetAsync(target, 0x7F, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
 
     // 2. gather (+ quantise) and zero the combine buffer
     const int* num_mt = o.num_mtiles;
@@ -396,8 +521,8 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     float* sx = reinterpret_cast<float*>(reg(MOE_WS_SX));
     {
         ProfScope ps(MOE_KERNEL_GATHER, st);
-        if (launch_gather(fp8, static_cast<const __nv_bfloat16*>(x), T, H, k, o.slot_of, reg(MOE_WS_XS), sx, out32,
-                          status, st) != cudaSuccess)
+        if (launch_gather(fp8, static_cast<const __nv_bfloat16*>(x), T, H, k, o.slot_of, L.S_max, reg(MOE_WS_XS), sx,
+                          out32, status, st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 
@@ -427,6 +552,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     g1.test_stall = g_opt_test_stall.load();
     g1.counts = o.counts;
     g1.num_experts = E;
+    g1.mt_max = L.MT_max;
     g1.group_m = (cfg1 != 1) ? 1 : 0;
     {
         ProfScope ps(MOE_KERNEL_STAGE1, st);
@@ -494,14 +620,13 @@ int moe_profile_read(double* ms_total, int* launches, int reset) {
 }
 
 int moe_get_status(void* stream) {
-    int* status = nullptr;
-    int num_sms = 0;
-    if (device_info(&status, &num_sms) != MOE_OK) return MOE_ERR_CUDA;
+    CtxInfo ctx{};
+    if (context_info(&ctx) != MOE_OK) return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
     int v = 0;
-    if (cudaMemcpy(&v, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpy(&v, ctx.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
     const int zero = 0;
-    if (cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpy(ctx.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
     return v;
 }
 

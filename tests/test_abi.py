@@ -119,3 +119,29 @@ def test_options(moe):
     moe.moe_set_option(moe.OPT_PATH, old)
     assert moe.moe_set_option(99, 0) == -1
     assert moe.moe_set_option(moe.OPT_TIMEOUT_MS, 0) == -1
+
+
+def test_static_entry_checks_arguments_before_size(moe):
+    """moe_ffn_forward_static applies moe_ffn_forward's checks first, in the
+    same order, and only then compares the problem with its built-in
+    workspace (nothing here touches the device)."""
+    P = 4096
+    big = (4096, 4096, 14336, 8, 2, 1)  # far more than the built-in workspace
+    assert moe.moe_workspace_size(*big) > moe.moe_static_workspace_bytes()
+    T, H, F, E, k, dt = big
+    # null weights on an oversized problem: invalid argument, not workspace
+    assert moe.moe_ffn_forward_static(P, P, None, P, P, P, T, H, F, E, k, dt, P, None) == -1
+    # misaligned pointer on an oversized problem: alignment
+    assert moe.moe_ffn_forward_static(P + 4, P, P, P, P, P, T, H, F, E, k, dt, P, None) == -3
+    # unsupported shape
+    assert moe.moe_ffn_forward_static(P, P, P, P, P, P, 4, 200, 128, 2, 1, 1, P, None) == -2
+    # bad dimensions
+    assert moe.moe_ffn_forward_static(P, P, P, P, P, P, 4, 128, 128, 0, 1, 1, P, None) == -1
+    # valid arguments, oversized problem: workspace
+    assert moe.moe_ffn_forward_static(P, P, P, P, P, P, T, H, F, E, k, dt, P, None) == -4
+
+
+def test_test_hook_options_range(moe):
+    assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, 4) == -1
+    assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, -1) == -1
+    assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, 0) == 0

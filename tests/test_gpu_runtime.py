@@ -1,7 +1,8 @@
 """Runtime behaviour of the CUDA path: failure detection through the device
 status word (a wait that runs out ends the kernel cleanly and leaves the
-context usable), capture of a layer call in a CUDA graph, and run-to-run
-determinism."""
+context usable; a routing-table index out of range is caught by the kernel
+that reads it, which skips the access), capture of a layer call in a CUDA
+graph, and run-to-run determinism."""
 import numpy as np
 import pytest
 import torch
@@ -85,3 +86,28 @@ def test_output_deterministic_without_k_splits(moe):
     d = to_device(case)
     outs = [run_layer(d)[0].clone() for _ in range(3)]
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+
+
+CORRUPT = pytest.mark.parametrize("table", [1, 2, 3], ids=["slot_of", "slot_assign", "mtile_expert"])
+
+
+@CORRUPT
+@PATHS
+def test_corrupted_routing_index_is_caught(moe, table, path):
+    """A routing-table entry far out of range (written on the host side of the
+    call, after routing) is caught by the kernel that reads it: the status word
+    says MOE_ERR_DEVICE_BOUNDS, nothing faults, and the next call is correct."""
+    T = 16 if path == 4 else 64
+    case = small_case(T, 256, 512, 8, 2, "fp8", 45)
+    d = to_device(case)
+    moe.moe_set_option(moe.OPT_PATH, path)
+    old = moe.moe_set_option(moe.OPT_TEST_CORRUPT, table)
+    try:
+        moe.ffn_forward(d["x"], d["logits"], d["w13"], d["s13"], d["w2p"], d["s2"], 2, 512, True)
+        st = moe.moe_get_status(None)
+        assert st == -7, f"expected MOE_ERR_DEVICE_BOUNDS, got {moe.STATUS_NAMES.get(st, st)}"
+    finally:
+        moe.moe_set_option(moe.OPT_TEST_CORRUPT, old)
+    torch.cuda.synchronize()
+    out, ws = run_layer(d)
+    verify_layer(moe, ws, out, case, what=f"after a corrupted table {table}")

@@ -122,6 +122,58 @@ def test_quant_x_properties():
     assert xq[3, 5] == 0xFE
 
 
+def _quant_x_torch(x_bf16):
+    """R0 restated with torch's IEEE binary32 arithmetic and float8 conversion:
+    sx = fp32(absmax / 448) (1 for a zero row), codes = e4m3(fp32(x / sx))."""
+    xf = x_bf16.float()
+    amax = xf.abs().amax(dim=1)
+    sx = torch.where(amax > 0, amax / torch.tensor(448.0, dtype=torch.float32), torch.ones_like(amax))
+    q = (xf / sx[:, None]).to(torch.float8_e4m3fn)
+    return q.view(torch.uint8).numpy(), sx.numpy()
+
+
+def test_quant_x_bitwise_against_binary32_division():
+    """Codes and scales equal, bit for bit, a division in binary32 followed by
+    a round-to-nearest-even e4m3 conversion -- on random rows of many
+    magnitudes, and on rows whose scale is a power of two so that quotients
+    land exactly on e4m3 ties (normal and subnormal), where a wrong rounding
+    rule, a reciprocal multiply or a scale computed in another precision
+    would show."""
+    rng = np.random.default_rng(31)
+    rows = [rng.normal(0, 10.0 ** rng.uniform(-8, 4), 256) for _ in range(60)]
+    rows += [rng.uniform(-1, 1, 256) * 10.0 ** rng.uniform(-3, 3) for _ in range(20)]
+    ties = []
+    for j in (-3, 0, 5):
+        scale = 2.0 ** j  # absmax 448 * 2^j gives sx = 2^j exactly
+        mids = []
+        for ex in range(-6, 8):      # normal e4m3 binades: spacing 2^(ex-3), ties at odd multiples of half of it
+            step = 2.0 ** (ex - 3)
+            mids += [(2.0 ** ex) + (i + 0.5) * step for i in range(8)]
+        mids += [(i + 0.5) * 2.0 ** -9 for i in range(8)]  # subnormal ties
+        row = np.array([448.0] + mids + [-m for m in mids[:40]]) * scale
+        ties.append(row)
+    x = torch.zeros(len(rows) + len(ties), 256, dtype=torch.float32)
+    for i, r in enumerate(rows + ties):
+        x[i, :len(r)] = torch.tensor(r[:256], dtype=torch.float32)
+    x = x.to(torch.bfloat16)
+    # the tie rows are exactly representable in bf16
+    for i, r in enumerate(ties):
+        np.testing.assert_array_equal(x[len(rows) + i, :len(r)].double().numpy(), r)
+    x[3] = 0  # a zero row: scale 1, all codes zero
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    xq, sx = oracle.quant_x(bits)
+    xq_t, sx_t = _quant_x_torch(x)
+    np.testing.assert_array_equal(sx.view(np.uint32), sx_t.view(np.uint32))
+    np.testing.assert_array_equal(xq, xq_t)
+    assert sx[3] == 1.0 and not xq[3].any()
+    # the ties did round to even: e.g. 1.0625 -> 1.0 (code 0x38), 1.1875 -> 1.25 (0x3A)
+    t0 = len(rows) + 1  # scale 2^0
+    vals = x[t0].double().numpy()
+    i1 = int(np.nonzero(vals == 1.0625)[0][0])
+    i2 = int(np.nonzero(vals == 1.1875)[0][0])
+    assert xq[t0, i1] == 0x38 and xq[t0, i2] == 0x3A
+
+
 # ---------------------------------------------------------------- MX block quantisation of h
 
 @pytest.mark.parametrize("amax,expected", [

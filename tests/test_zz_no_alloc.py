@@ -50,3 +50,37 @@ def test_static_workspace_rejects_oversized_problem():
     rc = moe.moe_ffn_forward_static(_p(x), _p(x), _p(x), _p(x), _p(x), _p(x), T, H, F, E, k, 1, _p(x), None)
     assert rc == -4  # MOE_ERR_WORKSPACE, nothing enqueued
     assert moe.moe_get_status(None) == 0
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+def test_static_workspace_in_a_captured_graph(dtype):
+    """Code under stream capture cannot allocate: the first call (outside the
+    capture) looks up the built-in array, later calls are captured into a CUDA
+    graph whose replays match the allocated-workspace output."""
+    import mixture_experts_routed_02_b200 as moe
+    T, H, F, E, k = 24, 256, 512, 8, 2
+    case = small_case(T, H, F, E, k, dtype, seed=32)
+    d = to_device(case)
+    dt = moe.dtype_code(dtype)
+    ref = moe.ffn_forward(d["x"], d["logits"], d["w13"], d["s13"], d["w2p"], d["s2"], k, F, dtype == "fp8")
+    assert moe.moe_get_status(None) == 0
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+
+    def call():
+        return moe.moe_ffn_forward_static(_p(d["x"]), _p(d["logits"]), _p(d["w13"]), _p(d["s13"]), _p(d["w2p"]),
+                                          _p(d["s2"]), T, H, F, E, k, dt, _p(out), ctypes.c_void_p(s.cuda_stream))
+
+    with torch.cuda.stream(s):
+        assert call() == 0  # first call in this context: outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        rc = call()
+    assert rc == 0
+    for _ in range(2):
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert moe.moe_get_status(None) == 0
+        check_close(out.float().double().cpu().numpy(), ref.float().double().cpu().numpy(), "captured static call")
