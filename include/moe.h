@@ -128,8 +128,11 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float
  * scale 2^ceil(log2(absmax/448)).  BF16 mode: h is rounded to bf16.  The k
  * weighted expert outputs are summed in fp32 and rounded once to bf16.
  * Execution: five kernels (six from 1024 tokens on) chained on `stream` with
- * programmatic dependent launch; to the rest of the stream the call is
- * ordinary stream-ordered work (later work starts after `out` is written).
+ * programmatic dependent launch -- routing, per-token quantisation, the first
+ * group GEMM (which gathers each expert's token rows by TMA), the second group
+ * GEMM with the scatter-add, and the bf16 rounding; to the rest of the stream
+ * the call is ordinary stream-ordered work (later work starts after `out` is
+ * written).
  * The group GEMM tiles are chosen from the average rows per expert (see
  * MOE_OPT_PATH): small batches stream weights on one-CTA tiles, large ones
  * use 256 x 256 tiles on pairs of SMs.  The call makes no host<->device
@@ -169,6 +172,54 @@ int moe_ffn_forward_static(const void* x, const float* logits, const void* w13, 
                            const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* stream);
 size_t moe_static_workspace_bytes(void);
 
+/*
+ * One rank's part of the d_ff-sharded layer (multi-GPU; the talk summary's
+ * deployment, timestamp 8:14, runs the layer on 16 shards).  Each of n_ranks
+ * GPUs holds an F_shard = d_ff / n_ranks slice of every expert: rows
+ * [r*F_shard, (r+1)*F_shard) of w1 and w3 and the same columns of w2,
+ * prepared by moe_prepare_weights with F = F_shard (F_shard % 128 == 0, so the
+ * FP8 blocks of 32 d_ff channels never straddle two shards and the sharded
+ * layer rounds h exactly as the whole layer does).  Every rank routes all T
+ * tokens (the routing is deterministic, so all ranks agree), runs both group
+ * GEMMs on its slice, and its second GEMM adds each token's partial output
+ * straight into the combine rows of the rank that owns the token: rank
+ * g = t / rows_per_rank owns tokens [g*rows_per_rank, (g+1)*rows_per_rank),
+ * rows_per_rank = ceil(T / n_ranks) -- a GEMM and reduce-scatter in one pass,
+ * through peer memory.  Then it adds 1 to every rank's arrival counter.
+ *   x, logits, s2, T, H, E, k, dtype, ws, ws_bytes as in moe_ffn_forward (s2 is
+ *            the full [E,H]); w13, s13, w2 are this rank's prepared slices.
+ *   peer_out32   host array of n_ranks device pointers: rank g's fp32 combine
+ *            rows [rows_per_rank, H] for this step (possibly another GPU's
+ *            memory, mapped for peer access).  They must be zero before the
+ *            first step; moe_dff_finalize zeroes the rows it rounds, so a
+ *            caller that alternates two sets of combine rows between steps
+ *            (set s % 2 at step s) always adds into zeroed rows.
+ *   peer_counter host array of n_ranks device pointers: rank g's uint32
+ *            arrival counter (zero before the first step).
+ * Returns as moe_ffn_forward; 1 <= n_ranks <= 16, 0 <= rank < n_ranks.
+ */
+int moe_ffn_forward_dff(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
+                        const float* s2, int T, int H, int F_shard, int E, int k, int dtype, int n_ranks, int rank,
+                        float* const* peer_out32, unsigned int* const* peer_counter, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/*
+ * Closes a step of the d_ff-sharded layer on this rank: waits (bounded, like
+ * every wait of this library) until this rank's arrival counter reaches
+ * `target` -- n_ranks * step for the step-th call, counting from 1 -- then
+ * rounds this rank's `rows` combine rows to bf16 into `out` [rows, H] and
+ * zeroes them.  Enqueue it after moe_ffn_forward_dff on this rank's stream;
+ * on one GPU standing in for several ranks, enqueue every rank's
+ * moe_ffn_forward_dff before any rank's moe_dff_finalize.
+ *   out32_rows  device, fp32 [rows, H]: this rank's combine rows of the step.
+ *   out         device, bf16 [rows, H], written.
+ *   counter     device, this rank's arrival counter.
+ * A wait that runs out records MOE_ERR_DEVICE_TIMEOUT and leaves `out`
+ * unwritten.
+ */
+int moe_dff_finalize(float* out32_rows, void* out, int rows, int H, const unsigned int* counter, unsigned int target,
+                     void* stream);
+
 /* Waits for `stream`, then returns and clears the device status word:
  * MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BOUNDS, or MOE_ERR_CUDA when
  * the wait itself failed. */
@@ -185,9 +236,10 @@ typedef enum {
     MOE_WS_PERM = 4,       /* int32 [T*k] */
     MOE_WS_INV_PERM = 5,   /* int32 [T*k] */
     MOE_WS_SLOT_OF = 6,    /* int32 [T*k]: assignment -> row of the expert-padded layout */
-    MOE_WS_XS = 7,         /* gathered activations, one row per padded slot: e4m3 or bf16 [S,H],
-                              rows H*eb + 128 bytes apart */
-    MOE_WS_SX = 8,         /* fp32 [S]: per-row activation scale (FP8) */
+    MOE_WS_XS = 7,         /* FP8: quantised activations, one row per token: e4m3 [T,H] (the first
+                              group GEMM gathers each expert's rows from here; BF16 gathers
+                              from x itself and this region is empty) */
+    MOE_WS_SX = 8,         /* FP8: fp32 [T] per-token activation scale (empty for BF16) */
     MOE_WS_H = 9,          /* intermediate h [S,F]: e4m3 or bf16, rows F*eb + 128 bytes apart */
     MOE_WS_H_SF = 10,      /* UE8M0 block scales of h (FP8), tiled for the tensor cores */
     MOE_WS_OUT32 = 11,     /* fp32 [T,H] combine buffer */
@@ -218,10 +270,10 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
  *   MOE_OPT_TEST_CORRUPT: test of the bounds checks: after routing, the host
  *                     enqueues a 4-byte write of bytes 0x7F (an index far out
  *                     of range) over the first entry of one routing table --
- *                     1 = assignment -> padded row (read by the gather),
- *                     2 = padded row -> assignment (read by the second GEMM's
- *                     scatter), 3 = 128-row tile -> expert (read by both
- *                     GEMMs).  The kernel that reads it records
+ *                     1 = padded row -> assignment (read by the first GEMM's
+ *                     token gather and the second GEMM's scatter),
+ *                     2 = 128-row tile -> expert, 3 = the number of 128-row
+ *                     tiles (both read by both GEMMs).  The kernel that reads it records
  *                     MOE_ERR_DEVICE_BOUNDS and skips the access; the call's
  *                     outputs are undefined and the context stays usable.
  *                     0 (default) = off.
@@ -246,7 +298,7 @@ int moe_set_option(int option, int value);
  * forgets the records when `reset` is nonzero.  Returns MOE_OK or MOE_ERR_CUDA. */
 typedef enum {
     MOE_KERNEL_ROUTE = 0,
-    MOE_KERNEL_GATHER = 1,
+    MOE_KERNEL_QUANT = 1,  /* per-token FP8 quantisation + zeroing of the combine buffer */
     MOE_KERNEL_STAGE1 = 2, /* group GEMM with w1/w3 + SwiGLU */
     MOE_KERNEL_STAGE2 = 3, /* group GEMM with w2 + weighted scatter-add */
     MOE_KERNEL_FINALIZE = 4,

@@ -53,8 +53,8 @@ WS = dict(topk_ids=0, topk_w=1, counts=2, offsets=3, perm=4, inv_perm=5, slot_of
 # every symbol include/moe.h declares
 EXPORTS = ["moe_workspace_size", "moe_prepare_weights", "moe_route", "moe_ffn_forward", "moe_get_status",
            "moe_workspace_region", "moe_set_option", "moe_profile_enable", "moe_profile_read",
-           "moe_ffn_forward_static", "moe_static_workspace_bytes"]
-KERNELS = ["route", "gather", "stage1_w13_swiglu", "stage2_w2_scatter", "finalize"]
+           "moe_ffn_forward_static", "moe_static_workspace_bytes", "moe_ffn_forward_dff", "moe_dff_finalize"]
+KERNELS = ["route", "quantize", "stage1_w13_swiglu", "stage2_w2_scatter", "finalize"]
 
 
 class MoeError(RuntimeError):
@@ -86,6 +86,10 @@ lib.moe_ffn_forward_static.restype = _I
 lib.moe_ffn_forward_static.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
 lib.moe_static_workspace_bytes.restype = _Z
 lib.moe_static_workspace_bytes.argtypes = []
+lib.moe_ffn_forward_dff.restype = _I
+lib.moe_ffn_forward_dff.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _Z, _P]
+lib.moe_dff_finalize.restype = _I
+lib.moe_dff_finalize.argtypes = [_P, _P, _I, _I, _P, ctypes.c_uint, _P]
 lib.moe_profile_enable.restype = _I
 lib.moe_profile_enable.argtypes = [_I]
 lib.moe_profile_read.restype = _I
@@ -101,6 +105,8 @@ moe_set_option = lib.moe_set_option
 moe_profile_enable = lib.moe_profile_enable
 moe_ffn_forward_static = lib.moe_ffn_forward_static
 moe_static_workspace_bytes = lib.moe_static_workspace_bytes
+moe_ffn_forward_dff = lib.moe_ffn_forward_dff
+moe_dff_finalize = lib.moe_dff_finalize
 
 
 def moe_profile_read(reset=True):
@@ -206,4 +212,59 @@ def ffn_forward(x, logits, w13, s13, w2p, s2, k, F, fp8, out=None, ws=None, stre
     rc = moe_ffn_forward(_ptr(x), _ptr(logits), _ptr(w13), _ptr(s13) if fp8 else None, _ptr(w2p),
                          _ptr(s2) if fp8 else None, T, H, F, E, k, dt, _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
     _check("moe_ffn_forward", rc)
+    return out
+
+
+# ---------------------------------------------------------------- d_ff-sharded layer
+
+def dff_rows(T, n_ranks, rank):
+    """(first token, number of tokens) that rank `rank` owns in the d_ff-sharded
+    layer: blocks of ceil(T / n_ranks) tokens, the last one possibly shorter."""
+    per = -(-T // n_ranks) if T > 0 else 0
+    first = min(T, rank * per)
+    return first, max(0, min(per, T - first))
+
+
+def dff_shard(w1, w3, s1, s3, w2, n_ranks, rank):
+    """This rank's d_ff slice of the expert weights (slicing only): rows
+    [r*Fs, (r+1)*Fs) of w1, w3 (and s1, s3) and the same columns of w2,
+    Fs = d_ff / n_ranks (a multiple of 128).  Works on torch tensors on any
+    device; returns contiguous copies (w1, w3, s1, s3, w2)."""
+    F = w1.shape[1]
+    if F % n_ranks or (F // n_ranks) % 128:
+        raise ValueError(f"d_ff={F} does not split into {n_ranks} shards of a multiple of 128")
+    fs = F // n_ranks
+    sl = slice(rank * fs, (rank + 1) * fs)
+    c = lambda t: None if t is None else t.contiguous()  # noqa: E731
+    return (c(w1[:, sl]), c(w3[:, sl]), c(None if s1 is None else s1[:, sl]), c(None if s3 is None else s3[:, sl]),
+            c(w2[:, :, sl]))
+
+
+def ffn_forward_dff(x, logits, w13, s13, w2p, s2, k, F_shard, fp8, n_ranks, rank, peer_out32, peer_counter,
+                    ws=None, stream=None):
+    """One rank's part of a d_ff-sharded layer step (see moe_ffn_forward_dff):
+    ``peer_out32`` / ``peer_counter`` are lists of n_ranks device tensors (or
+    raw device addresses) of every rank's combine rows and arrival counter."""
+    T, H = x.shape
+    E = logits.shape[1]
+    dt = MOE_FP8_E4M3 if fp8 else MOE_BF16
+    if ws is None:
+        ws = workspace(T, H, F_shard, E, k, dt, x.device)
+    addr = lambda t: t if isinstance(t, int) else t.data_ptr()  # noqa: E731
+    outs = (ctypes.c_void_p * n_ranks)(*[addr(t) for t in peer_out32])
+    ctrs = (ctypes.c_void_p * n_ranks)(*[addr(t) for t in peer_counter])
+    rc = moe_ffn_forward_dff(_ptr(x), _ptr(logits), _ptr(w13), _ptr(s13) if fp8 else None, _ptr(w2p),
+                             _ptr(s2) if fp8 else None, T, H, F_shard, E, k, dt, n_ranks, rank, outs, ctrs, _ptr(ws),
+                             ws.numel(), _stream(stream))
+    _check("moe_ffn_forward_dff", rc)
+    return ws
+
+
+def dff_finalize(out32_rows, out, counter, target, stream=None):
+    """Round this rank's combine rows to bf16 once every rank has signalled
+    (see moe_dff_finalize); ``out32_rows`` [rows, H] fp32, ``out`` [rows, H] bf16."""
+    rows, H = out.shape
+    rc = moe_dff_finalize(_ptr(out32_rows), _ptr(out), rows, H, _ptr(counter), int(target) & 0xFFFFFFFF,
+                          _stream(stream))
+    _check("moe_dff_finalize", rc)
     return out

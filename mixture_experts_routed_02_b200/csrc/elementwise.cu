@@ -1,8 +1,8 @@
 // elementwise.cu -- the memory-bound steps around the two grouped GEMMs:
-//   gather_kernel    gather of each expert's token rows into the expert-padded
-//                    layout (rocketrecap.com "FlyDSL kernels in JAX", paragraph
-//                    2: "gather"), fused with the per-token FP8 quantisation of
-//                    the activations and with zeroing the fp32 combine buffer;
+//   quant_kernel     per-token FP8 quantisation of the activations (the first
+//                    GEMM gathers each expert's token rows from its output;
+//                    rocketrecap.com "FlyDSL kernels in JAX", paragraph 2:
+//                    "gather") and zeroing of the fp32 combine buffer;
 //   finalize_kernel  fp32 combine buffer -> bf16 output;
 //   preshuffle_kernel the one-time load-time preshuffle of the expert weights into
 //                    contiguous, pre-swizzled 128x128-byte operand blocks
@@ -13,148 +13,98 @@
 
 namespace moe {
 
-// One CTA (128 threads) per `per_cta` consecutive assignments a = t*k + j of
-// one token t (per_cta = k: the whole token; 1: one assignment, for small
-// batches where more CTAs shorten the critical path): reads the row once,
-// quantises it once (FP8: the scale is per token, so every copy is the same)
-// and writes it to the padded-layout row of each of those assignments; the
-// CTA holding the token's first assignment also zeroes its fp32 combine row.  Padding rows are not written: the
-// tensor cores compute each output row from its own input row only, and the
-// outputs of padding rows are discarded.  Rows of up to kRegVec*1024 elements
-// are read into registers before the wait for the routing kernel: the tokens
-// are the caller's input and the combine buffer was last read by the previous
-// call's finalize, both complete before routing started; only the destination
-// rows need the routing result.
+// One CTA (128 threads) per token t: zeroes the token's fp32 combine row and,
+// in FP8 mode, quantises the token's row once -- sx[t] = absmax/448 (IEEE
+// division, 1 for a zero row) and xq[t, i] = e4m3_rn_satfinite(x[t, i] / sx[t])
+// -- for the first GEMM, which gathers the rows of each expert's tokens from
+// xq (FP8) or straight from x (BF16) by TMA.  Nothing here depends on the
+// routing: the kernel runs beside the router and waits for it only at the end,
+// before it lets the first GEMM start, so that GEMM may read the routing
+// tables as soon as it starts.  Rows of up to kRegVec*1024 elements are held
+// in registers between the absmax pass and the quantisation pass.
 constexpr int kRegVec = 4;
 
-template <bool kFP8, bool kPerToken>
-__global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int k,
-                                                    const int* __restrict__ slot_of, int num_slots,
-                                                    uint8_t* __restrict__ xs,
-                                                    float* __restrict__ sx_slot, float* __restrict__ out32,
-                                                    int* __restrict__ status) {
+template <bool kFP8>
+__global__ void __launch_bounds__(128, 8) quant_kernel(const __nv_bfloat16* __restrict__ x, int H,
+                                                   uint8_t* __restrict__ xq, float* __restrict__ sx_tok,
+                                                   float* __restrict__ out32) {
     __shared__ float warp_max[4];
     const int tid = threadIdx.x;
-    const int per_cta = kPerToken ? k : 1;
-    const int a0 = blockIdx.x * per_cta;
-    const int t = a0 / k;
-    const int eb = kFP8 ? 1 : 2;
-    const int nvec_in = H / 8;  // 8 bf16 per 16-byte vector
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-    const bool in_regs = nvec_in <= 128 * kRegVec;
-    uint4 v[kRegVec];
-    if (in_regs) {
-#pragma unroll
-        for (int r = 0; r < kRegVec; ++r) {
-            const int i = tid + r * 128;
-            v[r] = (i < nvec_in) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
-    if (a0 % k == 0) {
+    const int t = blockIdx.x;
+    if (out32) {  // (the d_ff-sharded layer keeps its combine rows zero itself)
         float4* o = reinterpret_cast<float4*>(out32 + (size_t)t * H);
         for (int i = tid; i < H / 4; i += 128) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    griddep_wait();
-    griddep_launch_dependents();
-    // destination rows of this CTA's assignments (kept in registers when there
-    // is one)
-    const int n = per_cta;
-    int slots[kPerToken ? kMaxTopK : 1];
-    bool bad = false;
-    for (int j = 0; j < n; ++j) {
-        slots[j] = slot_of[a0 + j];
-        bad |= slots[j] < 0 || slots[j] >= num_slots;  // never from the router: a corrupted table
-    }
-    if (bad) {
-        if (tid == 0) record_error(status, MOE_ERR_DEVICE_BOUNDS);
-        return;
-    }
-    const long pitch = act_pitch((long)H * eb);
-    if (!kFP8) {
-        for (int j = 0; j < n; ++j) {
-            uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)slots[j] * pitch);
-            if (in_regs) {
+    if constexpr (kFP8) {
+        const int nvec_in = H / 8;  // 8 bf16 per 16-byte vector
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+        const bool in_regs = nvec_in <= 128 * kRegVec;
+        uint4 v[kRegVec];
+        if (in_regs) {
 #pragma unroll
-                for (int r = 0; r < kRegVec; ++r) {
-                    const int i = tid + r * 128;
-                    if (i < nvec_in) dst[i] = v[r];
-                }
-            } else {
-                for (int i = tid; i < nvec_in; i += 128) dst[i] = __ldg(src + i);
+            for (int r = 0; r < kRegVec; ++r) {
+                const int i = tid + r * 128;
+                v[r] = (i < nvec_in) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
             }
         }
-        return;
-    }
-    // FP8: absmax over the row, then x / sx rounded to e4m3 (nearest even, saturating)
-    float amax = 0.f;
-    auto absmax8 = [&](const uint4& u) {
-        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+        // absmax over the row, then x / sx rounded to e4m3 (nearest even, saturating)
+        float amax = 0.f;
+        auto absmax8 = [&](const uint4& u) {
+            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 f = __bfloat1622float2(p[j]);
-            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-        }
-    };
-    if (in_regs) {
-#pragma unroll
-        for (int r = 0; r < kRegVec; ++r) absmax8(v[r]);
-    } else {
-        for (int i = tid; i < nvec_in; i += 128) absmax8(__ldg(src + i));
-    }
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
-    if ((tid & 31) == 0) warp_max[tid >> 5] = amax;
-    __syncthreads();
-    amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
-    const float sx = (amax == 0.f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-    if (tid < n) sx_slot[slots[tid]] = sx;
-    auto quant8 = [&](const uint4& u) {
-        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
-        uint32_t packed[2];
-#pragma unroll
-        for (int j = 0; j < 4; j += 2) {
-            const float2 f0 = __bfloat1622float2(p[j]);
-            const float2 f1 = __bfloat1622float2(p[j + 1]);
-            const __nv_fp8x2_storage_t q0 = __nv_cvt_float2_to_fp8x2(
-                make_float2(__fdiv_rn(f0.x, sx), __fdiv_rn(f0.y, sx)), __NV_SATFINITE, __NV_E4M3);
-            const __nv_fp8x2_storage_t q1 = __nv_cvt_float2_to_fp8x2(
-                make_float2(__fdiv_rn(f1.x, sx), __fdiv_rn(f1.y, sx)), __NV_SATFINITE, __NV_E4M3);
-            packed[j / 2] = (uint32_t)q0 | ((uint32_t)q1 << 16);
-        }
-        return make_uint2(packed[0], packed[1]);
-    };
-    if (in_regs) {
-#pragma unroll
-        for (int r = 0; r < kRegVec; ++r) {
-            const int i = tid + r * 128;
-            if (i < nvec_in) {
-                const uint2 q = quant8(v[r]);
-                for (int j = 0; j < n; ++j) reinterpret_cast<uint2*>(xs + (size_t)slots[j] * pitch)[i] = q;
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(p[j]);
+                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
             }
+        };
+        if (in_regs) {
+#pragma unroll
+            for (int r = 0; r < kRegVec; ++r) absmax8(v[r]);
+        } else {
+            for (int i = tid; i < nvec_in; i += 128) absmax8(__ldg(src + i));
         }
-    } else {
-        for (int i = tid; i < nvec_in; i += 128) {
-            const uint2 q = quant8(__ldg(src + i));
-            for (int j = 0; j < n; ++j) reinterpret_cast<uint2*>(xs + (size_t)slots[j] * pitch)[i] = q;
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+        if ((tid & 31) == 0) warp_max[tid >> 5] = amax;
+        __syncthreads();
+        amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
+        const float sx = (amax == 0.f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+        if (tid == 0) sx_tok[t] = sx;
+        auto quant8 = [&](const uint4& u) {
+            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+            uint32_t packed[2];
+#pragma unroll
+            for (int j = 0; j < 4; j += 2) {
+                const float2 f0 = __bfloat1622float2(p[j]);
+                const float2 f1 = __bfloat1622float2(p[j + 1]);
+                const __nv_fp8x2_storage_t q0 = __nv_cvt_float2_to_fp8x2(
+                    make_float2(__fdiv_rn(f0.x, sx), __fdiv_rn(f0.y, sx)), __NV_SATFINITE, __NV_E4M3);
+                const __nv_fp8x2_storage_t q1 = __nv_cvt_float2_to_fp8x2(
+                    make_float2(__fdiv_rn(f1.x, sx), __fdiv_rn(f1.y, sx)), __NV_SATFINITE, __NV_E4M3);
+                packed[j / 2] = (uint32_t)q0 | ((uint32_t)q1 << 16);
+            }
+            return make_uint2(packed[0], packed[1]);
+        };
+        uint2* dst = reinterpret_cast<uint2*>(xq + (size_t)t * H);
+        if (in_regs) {
+#pragma unroll
+            for (int r = 0; r < kRegVec; ++r) {
+                const int i = tid + r * 128;
+                if (i < nvec_in) dst[i] = quant8(v[r]);
+            }
+        } else {
+            for (int i = tid; i < nvec_in; i += 128) dst[i] = quant8(__ldg(src + i));
         }
     }
+    griddep_wait();  // the router has completed ...
+    griddep_launch_dependents();  // ... before the first GEMM may start
 }
 
-cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, int num_slots,
-                          uint8_t* xs, float* sx_slot, float* out32, int* status, cudaStream_t stream) {
-    // a CTA per token for large batches, per assignment (more CTAs, shorter
-    // critical path) for small ones
-    const bool per_token = T >= 256;
-    const dim3 grid(std::max(1, per_token ? T : T * k));
-    if (fp8)
-        return per_token ? launch_dependent(gather_kernel<true, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of, num_slots,
-                                            xs, sx_slot, out32, status)
-                         : launch_dependent(gather_kernel<true, false>, grid, dim3(128), 0, stream, x, T, H, k, slot_of, num_slots,
-                                            xs, sx_slot, out32, status);
-    return per_token ? launch_dependent(gather_kernel<false, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of, num_slots, xs,
-                                        sx_slot, out32, status)
-                     : launch_dependent(gather_kernel<false, false>, grid, dim3(128), 0, stream, x, T, H, k, slot_of, num_slots,
-                                        xs, sx_slot, out32, status);
+cudaError_t launch_quant(bool fp8, const __nv_bfloat16* x, int T, int H, uint8_t* xq, float* sx_tok, float* out32,
+                         cudaStream_t stream) {
+    if (T == 0) return cudaSuccess;
+    return fp8 ? launch_dependent(quant_kernel<true>, dim3(T), dim3(128), 0, stream, x, H, xq, sx_tok, out32)
+               : launch_dependent(quant_kernel<false>, dim3(T), dim3(128), 0, stream, x, H, xq, sx_tok, out32);
 }
 
 // out = bf16(out32), round to nearest even; n is a multiple of 8.
@@ -168,6 +118,77 @@ __global__ void finalize_kernel(const float* __restrict__ out32, __nv_bfloat16* 
                                __floats2bfloat162_rn(b.x, b.y), __floats2bfloat162_rn(b.z, b.w)};
         reinterpret_cast<uint4*>(out)[i] = *reinterpret_cast<uint4*>(r);
     }
+}
+
+// ---------------------------------------------------------------- d_ff-sharded layer
+// Each rank's second GEMM adds its partial sums of every token straight into
+// the combine rows of the rank that owns the token (peer memory), which makes
+// the GEMM and the reduce-scatter one pass.  The two kernels below close a
+// step: every rank tells every rank that its additions are done (one system-
+// scope increment of each rank's arrival counter, after a system-scope fence),
+// and each rank rounds its own rows once all n_ranks increments of this step
+// have arrived, zeroing them for the step after next (the caller alternates
+// two sets of combine rows).
+
+__global__ void dff_signal_kernel(PeerCounters counters, int n_ranks) {
+    griddep_wait();  // the second GEMM's additions are complete
+    __threadfence_system();
+    if ((int)threadIdx.x < n_ranks) atomicAdd_system(counters.c[threadIdx.x], 1u);
+}
+
+__device__ __forceinline__ unsigned int ld_acquire_sys(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__global__ void dff_finalize_kernel(float* __restrict__ out32, __nv_bfloat16* __restrict__ out, size_t n,
+                                    const unsigned int* counter, unsigned int target, unsigned long long timeout_ns,
+                                    int* status) {
+    __shared__ int s_ok;
+    griddep_wait();
+    if (threadIdx.x == 0) {
+        // bounded wait for every rank's signal of this step (counters only grow;
+        // the comparison is modulo 2^32)
+        int ok = 1;
+        if ((int)(ld_acquire_sys(counter) - target) < 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while ((int)(ld_acquire_sys(counter) - target) < 0) {
+                if (globaltimer_ns() - t0 > timeout_ns) {
+                    record_error(status, MOE_ERR_DEVICE_TIMEOUT);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(200);
+            }
+        }
+        s_ok = ok;
+    }
+    __syncthreads();
+    if (!s_ok) return;
+    const size_t nv = n / 8;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nv; i += (size_t)gridDim.x * blockDim.x) {
+        float4* src = reinterpret_cast<float4*>(out32) + 2 * i;
+        const float4 a = src[0];
+        const float4 b = src[1];
+        __nv_bfloat162 r[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
+                               __floats2bfloat162_rn(b.x, b.y), __floats2bfloat162_rn(b.z, b.w)};
+        reinterpret_cast<uint4*>(out)[i] = *reinterpret_cast<uint4*>(r);
+        src[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        src[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+cudaError_t launch_dff_signal(const PeerCounters& counters, int n_ranks, cudaStream_t stream) {
+    return launch_dependent(dff_signal_kernel, dim3(1), dim3(32), 0, stream, counters, n_ranks);
+}
+
+cudaError_t launch_dff_finalize(float* out32_rows, __nv_bfloat16* out, size_t n, const unsigned int* counter,
+                                unsigned int target, unsigned long long timeout_ns, int* status, int num_sms,
+                                cudaStream_t stream) {
+    const int blocks = (int)std::max<size_t>(1, std::min<size_t>((n / 8 + 255) / 256, (size_t)num_sms * 8));
+    return launch_dependent(dff_finalize_kernel, dim3(blocks), dim3(256), 0, stream, out32_rows, out, n, counter,
+                            target, timeout_ns, status);
 }
 
 // One thread per destination 16-byte chunk, destinations in address order.

@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
-        if constexpr (!PAIR) prefetch_tmap(&tmA32);
+        if constexpr (!PAIR && STAGE == 2) prefetch_tmap(&tmA32);
         if constexpr (PAIR) {
             prefetch_tmap(&tmB);
             if constexpr (C::MX) prefetch_tmap(&tmSF);
@@ -200,15 +200,17 @@ __global__ void __launch_bounds__(192, 1)
     const int ns = args.n_tiles * args.splits;
     const int tiles = PAIR ? s_pair_first[args.num_experts] * ns : num_mt * ns;
     const int kps = args.k_tiles / args.splits;
-    // Stage 1 on one CTA per tile: when the last wave of tiles would keep at
-    // most a quarter of the CTAs busy, each of its tiles is cut into BN/64
-    // units of 64 weight rows (no K split, so nothing to add up afterwards),
-    // which spreads that wave's weight stream over BN/64 times as many SMs.
+    // Stage 1 on one CTA per tile: when the last wave of tiles would leave
+    // CTAs idle and cutting its tiles finishes sooner, each of its tiles is cut
+    // into kQ = BN/64 units of 64 weight rows (no K split, so nothing to add
+    // up afterwards), which spreads that wave's weight stream over more SMs.
+    // The cut pays when its ceil(tail*kQ/grid) waves of quarter-size units take
+    // less than one whole wave: tail*kQ <= (kQ-1)*grid.
     constexpr int kQ = BN / 64;
     int full_tiles = tiles;
     if constexpr (STAGE == 1 && !PAIR && kQ > 1) {
         const int tail = tiles % (int)gridDim.x;
-        if (tail > 0 && tail * kQ <= (int)gridDim.x) full_tiles = tiles - tail;
+        if (tail > 0 && tail * kQ <= (kQ - 1) * (int)gridDim.x) full_tiles = tiles - tail;
     }
     const int units = full_tiles + (tiles - full_tiles) * kQ;
     // Work unit -> (this CTA's m-tile, n, split); `dup` marks the second half
@@ -283,6 +285,17 @@ __global__ void __launch_bounds__(192, 1)
         }
         return e;
     };
+    // Token of padded row `slot` (-1 for a padding row); an assignment out of
+    // range (never from the router) is recorded and read as a padding row.
+    auto token_of = [&](int slot) {
+        const int a = args.slot_assign[slot];
+        if (a == -1) return -1;
+        if (a < 0 || a >= args.T * args.topk) {
+            record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
+            return -1;
+        }
+        return a / args.topk;
+    };
     // One-CTA tiles whose m-tile holds at most 32 rows in use (small batches:
     // a few tokens per expert) copy only those 32 activation rows; the MMA
     // still reads 128 rows, and the results of the rows not copied (stale
@@ -343,33 +356,61 @@ __global__ void __launch_bounds__(192, 1)
     griddep_launch_dependents();
 
     if (warp == 0) {
-        if (lane == 0) {
-            const uint64_t pol_a = policy_evict_last();
-            int stage = 0;
-            uint32_t phase = 0;
-            int issued = 0;
-            bool ok = true;
-            for (int u = unit0; u < units && ok; u += ustep) {
-                int m, n, split, q4;
-                bool dup;
-                unit_coords(u, m, n, split, dup, q4);
-                const int e = expert_of(m);
-                const bool small = a_rows32(m);
-                if (AR == 32 && !small) record_error(args.status, MOE_ERR_DEVICE_BOUNDS);  // host chose this wrongly
-                for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
-                    const bool prefetched = (u == unit0) && (kt - split * kps) < npre;
-                    if (!prefetched) {
-                        if (!wait(&empty[stage], phase ^ 1)) {
-                            ok = false;
-                            break;
+        // Producer warp.  Lane 0 waits for a free stage and copies the weights
+        // (and stage 2's activation tile and scales); in stage 1 the lanes
+        // then gather the activation rows of the tile, four token rows per
+        // lane, straight from the per-token rows (xq or x) by TMA.
+        const uint64_t pol_a = policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        bool ok = true;
+        for (int u = unit0; u < units && ok; u += ustep) {
+            int m, n, split, q4;
+            bool dup;
+            unit_coords(u, m, n, split, dup, q4);
+            const int e = expert_of(m);
+            const bool small = a_rows32(m);
+            if (AR == 32 && !small && lane == 0) record_error(args.status, MOE_ERR_DEVICE_BOUNDS);  // host chose this wrongly
+            // stage 1: token rows behind this lane's four rows of the m-tile
+            // (a padding row reads token 0; its results are discarded)
+            const int rows_in = (small || AR == 32) ? 32 : kBlockM;
+            const bool gathers = (STAGE == 1) && 4 * lane < rows_in;
+            int tok[4] = {0, 0, 0, 0};
+            if (STAGE == 1 && gathers) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tok[j] = max(token_of(m * kBlockM + 4 * lane + j), 0);
+            }
+            for (int kt = split * kps; kt < (split + 1) * kps; ++kt) {
+                const bool prefetched = (u == unit0) && (kt - split * kps) < npre;
+                if (!prefetched) {
+                    int good = 1;
+                    if (lane == 0) {
+                        good = wait(&empty[stage], phase ^ 1) ? 1 : 0;
+                        if (good) {
+                            if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx(small, q4));
+                            load_weights(stage, e, n, kt, q4);
                         }
-                        if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx(small, q4));
-                        load_weights(stage, e, n, kt, q4);
                     }
-                    // failure-detection test hook: CTA 0 leaves the activation
-                    // copy of its first stage out, so that stage never completes
-                    // and the MMA's bounded wait runs out (see MOE_OPT_TEST_STALL)
-                    const bool skip = args.test_stall && blockIdx.x == 0 && issued == 0;
+                    if (!__shfl_sync(0xffffffffu, good, 0)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                // failure-detection test hook: CTA 0 leaves the activation
+                // copy of its first stage out, so that stage never completes
+                // and the MMA's bounded wait runs out (see MOE_OPT_TEST_STALL)
+                const bool skip = args.test_stall && blockIdx.x == 0 && issued == 0;
+                if constexpr (STAGE == 1) {
+                    if (!skip && gathers) {
+                        uint8_t* dst = smem + stage * C::A_BYTES + lane * 4 * 128;
+                        if constexpr (PAIR)
+                            tma_gather4_pair(dst, &tmA, mapa_shared(smem_u32(&full[stage]), 0), kt * C::KE, tok[0],
+                                             tok[1], tok[2], tok[3], pol_a);
+                        else
+                            tma_gather4(dst, &tmA, &full[stage], kt * C::KE, tok[0], tok[1], tok[2], tok[3], pol_a);
+                    }
+                } else if (lane == 0) {
                     if constexpr (PAIR) {
                         const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
                         if (!skip)
@@ -379,21 +420,23 @@ __global__ void __launch_bounds__(192, 1)
                                              (m * args.f_tiles + kt) * 4, pol_a);
                     } else {
                         if (!skip)
-                            tma_load_2d(smem + stage * C::A_BYTES, (small || AR == 32) ? &tmA32 : &tmA, &full[stage], kt * C::KE,
-                                        m * kBlockM, pol_a);
+                            tma_load_2d(smem + stage * C::A_BYTES, (small || AR == 32) ? &tmA32 : &tmA, &full[stage],
+                                        kt * C::KE, m * kBlockM, pol_a);
                         if constexpr (C::MX)
                             bulk_load(smem + C::OFF_SF + stage * C::SF_BYTES,
                                       args.a_sf + ((size_t)m * args.f_tiles + kt) * 512, 512, &full[stage]);
                     }
-                    ++issued;
-                    if (++stage == NST) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
+                }
+                ++issued;
+                if (++stage == NST) {
+                    stage = 0;
+                    phase ^= 1;
                 }
             }
-            // do not leave while copies into this CTA's shared memory are in
-            // flight (these waits ignore the abort flag but keep their time limit)
+        }
+        // do not leave while copies into this CTA's shared memory are in
+        // flight (these waits ignore the abort flag but keep their time limit)
+        if (lane == 0) {
             volatile int keep_waiting = 0;
             if constexpr (PAIR) {
                 // a pair's copies complete on the even CTA's barriers: wait
@@ -546,7 +589,11 @@ __global__ void __launch_bounds__(192, 1)
             const int slot = m * kBlockM + row;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             if constexpr (STAGE == 1) {
-                const float sxv = FP8 ? args.row_scale[slot] : 1.0f;
+                float sxv = 1.0f;
+                if constexpr (FP8) {
+                    const int t = token_of(slot);
+                    sxv = (t >= 0) ? args.row_scale[t] : 0.0f;  // a padding row's results are discarded
+                }
 #pragma unroll 1
                 // 64-column groups: all BN / 64 of a tile, or the one of a 64-row slice
                 const int g_first = (q4 >= 0) ? q4 : 0;
@@ -623,14 +670,19 @@ __global__ void __launch_bounds__(192, 1)
                 release(acc);
             } else {
                 const int a = dup ? -1 : args.slot_assign[slot];
-                int t = (a >= 0) ? a / args.topk : -1;
-                if (t >= args.T || a < -1) {
-                    record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
-                    t = -1;
-                }
+                const int t = dup ? -1 : token_of(slot);
                 const float wgt = (t >= 0) ? args.topk_w[a] : 0.f;
+                // the combine row: this GPU's buffer, or (d_ff-sharded layer) the
+                // row of the rank that owns token t, possibly in a peer's memory
                 float* orow = reinterpret_cast<float*>(static_cast<uint8_t*>(args.out) +
                                                        (size_t)(t >= 0 ? t : 0) * args.out_pitch);
+                bool remote = false;
+                if (args.n_ranks > 0 && t >= 0) {
+                    const int g = t / args.rows_per_rank;
+                    orow = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(args.peer_out[g]) +
+                                                    (size_t)(t - g * args.rows_per_rank) * args.out_pitch);
+                    remote = g != args.rank;
+                }
                 // 64 columns per TMEM wait; the accumulator is released as soon as
                 // the last columns are in registers, before their atomics
 #pragma unroll 1
@@ -657,7 +709,14 @@ __global__ void __launch_bounds__(192, 1)
                                 v.z *= sc.z;
                                 v.w *= sc.w;
                             }
-                            atomicAdd(reinterpret_cast<float4*>(orow + col + i), v);
+                            if (remote) {  // scalar atomics through peer memory
+                                atomicAdd(orow + col + i, v.x);
+                                atomicAdd(orow + col + i + 1, v.y);
+                                atomicAdd(orow + col + i + 2, v.z);
+                                atomicAdd(orow + col + i + 3, v.w);
+                            } else {
+                                atomicAdd(reinterpret_cast<float4*>(orow + col + i), v);
+                            }
                         }
                     }
                 }

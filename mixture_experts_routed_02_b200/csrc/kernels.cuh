@@ -13,8 +13,9 @@ namespace moe {
 
 constexpr int kMaxExperts = 64;
 constexpr int kMaxTopK = 8;
+constexpr int kMaxRanks = 16;  // d_ff shards of the sharded layer
 constexpr int kBlockM = 128;  // rows per tile of the expert-padded layout
-// Row pitch of the gathered activations and of h: 128 bytes more than a row,
+// Row pitch of h: 128 bytes more than a row,
 // so that the 128 rows of an operand tile do not sit a power of two apart
 // (such rows crowd into few L2 slices).
 __host__ __device__ constexpr long act_pitch(long row_bytes) { return row_bytes + 128; }
@@ -97,6 +98,11 @@ int max_active_clusters(void (*kernel)(KArgs...), int threads, size_t smem, int 
     return n;
 }
 
+// Arrival counters of the ranks of a d_ff-sharded layer (kernel argument).
+struct PeerCounters {
+    unsigned int* c[kMaxRanks];
+};
+
 // Host-side helpers of the entry points (moe_api.cu).
 // Key of the CUDA context current on the calling thread: the driver's
 // context id, never reused (false if no context is current).
@@ -109,9 +115,16 @@ int check_forward_args(const void* x, const float* logits, const void* w13, cons
 // Host launchers (each defined next to its kernel).
 cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream);
 int route_launches(int T, const RouteOutputs& o);  // kernels launch_route enqueues (1 or 2)
-cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, int num_slots,
-                          uint8_t* xs, float* sx_slot, float* out32, int* status, cudaStream_t stream);
+cudaError_t launch_quant(bool fp8, const __nv_bfloat16* x, int T, int H, uint8_t* xq, float* sx_tok, float* out32,
+                         cudaStream_t stream);
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream);
+// d_ff-sharded layer: after the second GEMM, add 1 to every rank's arrival
+// counter (system scope); then this rank waits (bounded) until its counter
+// reaches `target`, rounds its own combine rows to bf16 and zeroes them.
+cudaError_t launch_dff_signal(const PeerCounters& counters, int n_ranks, cudaStream_t stream);
+cudaError_t launch_dff_finalize(float* out32_rows, __nv_bfloat16* out, size_t n, const unsigned int* counter,
+                                unsigned int target, unsigned long long timeout_ns, int* status, int num_sms,
+                                cudaStream_t stream);
 // Blocked, pre-swizzled weight layout (see moe_prepare_weights in moe.h).
 constexpr int kWBlockRows = 128;
 constexpr int kWBlockBytes = kWBlockRows * 128;
@@ -124,7 +137,7 @@ struct GemmArgs {
     const int* num_mtiles;
     const int* mtile_expert;
     const int* slot_assign;
-    const float* row_scale;   // stage 1, FP8: per-row activation scale [S]
+    const float* row_scale;   // stage 1, FP8: per-token activation scale [T]
     const float* col_scale;   // FP8: s13 [E*2F] (stage 1) or s2 [E*H] (stage 2)
     const float* topk_w;      // stage 2: routing weight per assignment
     const uint8_t* b_blocks;  // weights in the blocked layout: [E][rows_b/128][k_tiles][16 KB]
@@ -147,12 +160,22 @@ struct GemmArgs {
     const int* counts;        // rows per expert [num_experts] (for group_m)
     int num_experts;
     int mt_max;               // bound of *num_mtiles (a larger value is a corrupted table)
+    // d_ff-sharded layer, stage 2: with n_ranks > 0 token t's row is added into
+    // the combine rows of the rank that owns it (t / rows_per_rank), at
+    // peer_out[owner] + (t - owner * rows_per_rank) * H, through peer memory
+    int n_ranks;
+    int rank;
+    int rows_per_rank;
+    float* peer_out[kMaxRanks];
 };
 
-// Tensor maps of one GEMM launch: a = activation rows (128-row boxes, 128-byte
-// swizzle) and a32 = the same with 32-row boxes (one-CTA tiles); for CTA pairs
-// also b = blocked weights (16 KB boxes) and, for the block-scaled stage 2,
-// sf = h's scale chunks (512-byte boxes).
+
+// Tensor maps of one GEMM launch, all with 128-byte swizzle for the
+// activations.  Stage 1: a = the token rows (xq or x) with one-row boxes, read
+// by four-row TMA gathers.  Stage 2: a = rows of h (128-row boxes) and a32 =
+// the same with 32-row boxes (one-CTA tiles).  For CTA pairs also b = blocked
+// weights (16 KB boxes) and, for the block-scaled stage 2, sf = h's scale
+// chunks (512-byte boxes).
 struct GemmMaps {
     const CUtensorMap* a;
     const CUtensorMap* a32;

@@ -4,8 +4,9 @@
 // One call of moe_ffn_forward enqueues, on the caller's stream:
 //   route_kernel   top-k, softmax, histogram, scan, permutation, padded layout
 //                  (from 1024 tokens: route_topk_kernel + route_place_kernel)
-//   gather_kernel  gather (+ per-token e4m3 quantisation) and zeroing of out32
-//   stage-1 GEMM   gather-GEMM with w1/w3 + SwiGLU (+ MX quantisation of h)
+//   quant_kernel   per-token e4m3 quantisation (FP8) and zeroing of out32
+//   stage-1 GEMM   TMA gather of each expert's token rows, GEMM with w1/w3 +
+//                  SwiGLU (+ MX quantisation of h)
 //   stage-2 GEMM   GEMM with w2 + routing-weighted scatter-add into out32
 //   finalize       out32 -> bf16 out
 // (rocketrecap.com "FlyDSL kernels in JAX", paragraph 2 and timestamp 5:56.)
@@ -190,8 +191,8 @@ Layout make_layout(int T, int H, int F, int E, int k, int dtype) {
     sz[MOE_WS_PERM] = 4 * A;
     sz[MOE_WS_INV_PERM] = 4 * A;
     sz[MOE_WS_SLOT_OF] = 4 * A;
-    sz[MOE_WS_XS] = S * act_pitch((long)H * eb);
-    sz[MOE_WS_SX] = 4 * S;
+    sz[MOE_WS_XS] = (dtype == MOE_FP8_E4M3) ? (size_t)T * H : 0;  // per-token e4m3 rows (BF16 reads x itself)
+    sz[MOE_WS_SX] = (dtype == MOE_FP8_E4M3) ? 4 * (size_t)T : 0;
     sz[MOE_WS_H] = S * act_pitch((long)F * eb);
     sz[MOE_WS_H_SF] = (dtype == MOE_FP8_E4M3) ? (size_t)L.MT_max * (F / 128) * 512 : 0;
     sz[MOE_WS_OUT32] = 4 * (size_t)T * H;
@@ -270,17 +271,18 @@ int launch_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CU
 // tile configuration) and reused by later calls with the same arguments.
 
 struct MapKey {
+    const void* x;
     const void* ws;
     const void* w13;
     const void* w2;
     int T, H, F, E, k, dtype, cfg1, cfg2;
     bool operator==(const MapKey& o) const {
-        return ws == o.ws && w13 == o.w13 && w2 == o.w2 && T == o.T && H == o.H && F == o.F && E == o.E &&
+        return x == o.x && ws == o.ws && w13 == o.w13 && w2 == o.w2 && T == o.T && H == o.H && F == o.F && E == o.E &&
                k == o.k && dtype == o.dtype && cfg1 == o.cfg1 && cfg2 == o.cfg2;
     }
 };
 struct MapSet {
-    CUtensorMap ta1, ta2, ta1s, ta2s, tb1, tb2, tsf2;
+    CUtensorMap tg1, ta2, ta2s, tb1, tb2, tsf2;
 };
 constexpr int kMapCache = 16;
 struct MapEntry {
@@ -418,24 +420,41 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float
     return launch_status(launch_route(logits, T, E, k, o, static_cast<cudaStream_t>(stream)));
 }
 
-int moe_ffn_forward(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
-                    const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
-                    size_t ws_bytes, void* stream) {
-    const int rc_args = check_forward_args(x, logits, w13, s13, w2, s2, T, H, F, E, k, dtype, out, ws);
+}  // extern "C"
+
+namespace {
+
+// The d_ff-sharded layer's arguments (see moe_ffn_forward_dff).
+struct Dff {
+    int n_ranks, rank;
+    float* const* peer_out32;
+    unsigned int* const* peer_counter;
+};
+
+// The layer call: the whole layer (dff == nullptr), or one rank's part of the
+// d_ff-sharded layer (its GEMMs on its d_ff slice, the scatter-add into the
+// owners' combine rows, and the signal to every rank; no rounding).
+int forward_impl(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
+                 const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws, size_t ws_bytes,
+                 void* stream, const Dff* dff) {
+    const int rc_args = check_forward_args(x, logits, w13, s13, w2, s2, T, H, F, E, k, dtype, dff ? ws : out, ws);
     if (rc_args != MOE_OK) return rc_args;
     const bool fp8 = dtype == MOE_FP8_E4M3;
     const Layout L = make_layout(T, H, F, E, k, dtype);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     const int opt_path = g_opt_path.load();  // read once per call
     if (opt_path == 4 && L.A > 32) return MOE_ERR_UNSUPPORTED;  // forced tiny-batch tiles
-    if (T == 0) return MOE_OK;
+    PeerCounters counters{};
+    if (dff)
+        for (int g = 0; g < dff->n_ranks; ++g) counters.c[g] = dff->peer_counter[g];
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) return dff ? launch_status(launch_dff_signal(counters, dff->n_ranks, st)) : MOE_OK;
 
     CtxInfo ctx{};
     if (context_info(&ctx) != MOE_OK) return MOE_ERR_CUDA;
     int* status = ctx.status;
     const int num_sms = ctx.num_sms;
     auto max_pairs = [&](int stage, bool f8) { return ctx.max_pairs[stage - 1][f8 ? 1 : 0]; };
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* w = static_cast<uint8_t*>(ws);
     auto reg = [&](int r) { return w + L.off[r]; };
     const int eb = fp8 ? 1 : 2;
@@ -468,12 +487,14 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     const int bn2 = gemm_block_n(2, fp8, cfg2);
     if ((2 * F) % bn1 || H % bn2) return MOE_ERR_UNSUPPORTED;
 
-    const MapKey mkey{ws, w13, w2, T, H, F, E, k, dtype, cfg1, cfg2};
+    // stage 1 gathers token rows: from the per-token e4m3 rows (FP8) or from
+    // x itself (BF16), one-row boxes of 128 bytes
+    const void* a1_base = fp8 ? (const void*)reg(MOE_WS_XS) : x;
+    const MapKey mkey{a1_base, ws, w13, w2, T, H, F, E, k, dtype, cfg1, cfg2};
     MapSet ms;
     if (!find_maps(mkey, &ms)) {
-        if (!make_map(&ms.ta1, reg(MOE_WS_XS), L.S_max, H, act_pitch((long)H * eb), eb, kBlockM) ||
+        if (!make_map(&ms.tg1, a1_base, T, H, (size_t)H * eb, eb, 1) ||
             !make_map(&ms.ta2, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, kBlockM) ||
-            !make_map(&ms.ta1s, reg(MOE_WS_XS), L.S_max, H, act_pitch((long)H * eb), eb, 32) ||
             !make_map(&ms.ta2s, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, 32))
             return MOE_ERR_CUDA;
         if (cfg1 == 0 && !make_map_rows(&ms.tb1, w13, (size_t)E * (2 * F) * (H * eb / 128), kWBlockRows))
@@ -484,7 +505,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
             return MOE_ERR_CUDA;
         store_maps(mkey, ms);
     }
-    const GemmMaps maps1{&ms.ta1, &ms.ta1s, cfg1 == 0 ? &ms.tb1 : nullptr, nullptr};
+    const GemmMaps maps1{&ms.tg1, &ms.tg1, cfg1 == 0 ? &ms.tb1 : nullptr, nullptr};
     const GemmMaps maps2{&ms.ta2, &ms.ta2s, cfg2 == 0 ? &ms.tb2 : nullptr, (cfg2 == 0 && fp8) ? &ms.tsf2 : nullptr};
     // grid: one CTA per SM at most; pairs: whole clusters that can be resident
     auto grid_for = [&](int stage, int c, long units_per_mtile) {
@@ -511,29 +532,29 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
     // an index far out of range (bytes 0x7F), as a corrupted table would hold
     const int corrupt = g_opt_test_corrupt.load();
     if (corrupt) {
-        void* target = corrupt == 1 ? (void*)o.slot_of : corrupt == 2 ? (void*)o.slot_assign : (void*)o.mtile_expert;
+        void* target = corrupt == 1 ? (void*)o.slot_assign : corrupt == 2 ? (void*)o.mtile_expert : (void*)o.num_mtiles;
         if (cudaMemsetAsync(target, 0x7F, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
     }
 
-    // 2. gather (+ quantise) and zero the combine buffer
+    // 2. per-token quantisation (FP8) and zeroing of the combine buffer
     const int* num_mt = o.num_mtiles;
     float* out32 = reinterpret_cast<float*>(reg(MOE_WS_OUT32));
-    float* sx = reinterpret_cast<float*>(reg(MOE_WS_SX));
+    float* sx = fp8 ? reinterpret_cast<float*>(reg(MOE_WS_SX)) : nullptr;
     {
-        ProfScope ps(MOE_KERNEL_GATHER, st);
-        if (launch_gather(fp8, static_cast<const __nv_bfloat16*>(x), T, H, k, o.slot_of, L.S_max, reg(MOE_WS_XS), sx,
-                          out32, status, st) != cudaSuccess)
+        ProfScope ps(MOE_KERNEL_QUANT, st);
+        if (launch_quant(fp8, static_cast<const __nv_bfloat16*>(x), T, H, fp8 ? reg(MOE_WS_XS) : nullptr, sx,
+                         dff ? nullptr : out32, st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 
     const unsigned long long timeout_ns = (unsigned long long)g_opt_timeout_ms.load() * 1000000ull;
 
-    // 3. stage 1: gather-GEMM with w1/w3, SwiGLU epilogue
+    // 3. stage 1: GEMM with w1/w3 on the gathered token rows, SwiGLU epilogue
     GemmArgs g1{};
     g1.num_mtiles = num_mt;
     g1.mtile_expert = o.mtile_expert;
     g1.slot_assign = o.slot_assign;
-    g1.row_scale = fp8 ? sx : nullptr;
+    g1.row_scale = sx;
     g1.col_scale = fp8 ? s13 : nullptr;
     g1.b_blocks = static_cast<const uint8_t*>(w13);
     g1.b_evict_first = small_batch ? 1 : 0;  // one m-tile per expert: each weight block is read once
@@ -580,15 +601,63 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
                             : choose_splits(mt_est, g2.n_tiles, g2.k_tiles, num_sms);
     if (g2.splits < 1 || g2.k_tiles % g2.splits) return MOE_ERR_UNSUPPORTED;
     g2.out_pitch = (long)H * 4;
+    if (dff) {  // add into the owners' combine rows (peer memory)
+        g2.n_ranks = dff->n_ranks;
+        g2.rank = dff->rank;
+        g2.rows_per_rank = (T + dff->n_ranks - 1) / dff->n_ranks;
+        for (int g = 0; g < dff->n_ranks; ++g) g2.peer_out[g] = dff->peer_out32[g];
+        g2.out = dff->peer_out32[dff->rank];
+    }
     {
         ProfScope ps(MOE_KERNEL_STAGE2, st);
         if (launch_gemm(2, fp8, cfg2, maps2, g2, grid_for(2, cfg2, (long)g2.n_tiles * g2.splits), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
+    if (dff) return launch_status(launch_dff_signal(counters, dff->n_ranks, st));
 
     // 5. fp32 -> bf16
     ProfScope ps(MOE_KERNEL_FINALIZE, st);
     return launch_status(launch_finalize(out32, static_cast<__nv_bfloat16*>(out), (size_t)T * H, num_sms, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_ffn_forward(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
+                    const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
+                    size_t ws_bytes, void* stream) {
+    return forward_impl(x, logits, w13, s13, w2, s2, T, H, F, E, k, dtype, out, ws, ws_bytes, stream, nullptr);
+}
+
+int moe_ffn_forward_dff(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
+                        const float* s2, int T, int H, int F_shard, int E, int k, int dtype, int n_ranks, int rank,
+                        float* const* peer_out32, unsigned int* const* peer_counter, void* ws, size_t ws_bytes,
+                        void* stream) {
+    if (n_ranks < 1 || n_ranks > kMaxRanks || rank < 0 || rank >= n_ranks || !peer_out32 || !peer_counter)
+        return MOE_ERR_INVALID_ARG;
+    for (int g = 0; g < n_ranks; ++g) {
+        if (!peer_out32[g] || !peer_counter[g]) return MOE_ERR_INVALID_ARG;
+        if (!aligned16(peer_out32[g]) || (reinterpret_cast<uintptr_t>(peer_counter[g]) & 3u))
+            return MOE_ERR_ALIGNMENT;
+    }
+    const Dff dff{n_ranks, rank, peer_out32, peer_counter};
+    return forward_impl(x, logits, w13, s13, w2, s2, T, H, F_shard, E, k, dtype, nullptr, ws, ws_bytes, stream,
+                        &dff);
+}
+
+int moe_dff_finalize(float* out32_rows, void* out, int rows, int H, const unsigned int* counter, unsigned int target,
+                     void* stream) {
+    if (rows < 0 || H <= 0 || H % 128 || (rows > 0 && (!out32_rows || !out)) || !counter) return MOE_ERR_INVALID_ARG;
+    if ((out32_rows && !aligned16(out32_rows)) || (out && !aligned16(out)) ||
+        (reinterpret_cast<uintptr_t>(counter) & 3u))
+        return MOE_ERR_ALIGNMENT;
+    CtxInfo ctx{};
+    if (context_info(&ctx) != MOE_OK) return MOE_ERR_CUDA;
+    const unsigned long long timeout_ns = (unsigned long long)g_opt_timeout_ms.load() * 1000000ull;
+    return launch_status(launch_dff_finalize(out32_rows, static_cast<__nv_bfloat16*>(out), (size_t)rows * H, counter,
+                                             target, timeout_ns, ctx.status, ctx.num_sms,
+                                             static_cast<cudaStream_t>(stream)));
 }
 
 int moe_profile_enable(int on) { return g_prof_on.exchange(on ? 1 : 0); }

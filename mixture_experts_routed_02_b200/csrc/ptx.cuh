@@ -31,9 +31,10 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // its predecessor in the stream is still running.  griddep_wait() blocks the
 // calling thread until the predecessor grid has completed and its memory is
 // visible (a no-op for an ordinary launch); griddep_launch_dependents() lets
-// the next such kernel be scheduled.  Every kernel of a layer call signals its
-// dependents only after its own wait has returned, so a kernel that starts
-// early may already read what the kernels two or more places before it wrote.
+// the next such kernel be scheduled.  Every kernel of a layer call after the
+// first (the router, an ordinary launch) signals its dependents only after its
+// own wait has returned, so a kernel that starts early may already read what
+// the kernels two or more places before it wrote.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -103,6 +104,19 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+// TMA gather: four rows (y0..y3) of a 2-D tensor map whose box is one row
+// high, columns [x, x + box width), into four consecutive rows of shared
+// memory at smem_dst (the map's swizzle applies as for a tile load).
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y0,
+                                            int y1, int y2, int y3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
+        "l"(policy)
         : "memory");
 }
 
@@ -272,6 +286,18 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+// TMA gather of four rows into this CTA's shared memory, completing on an
+// mbarrier of either CTA of the pair (`bar_cluster`).
+__device__ __forceinline__ void tma_gather4_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y0, int y1, int y2, int y3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
+        "l"(policy)
         : "memory");
 }
 

@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32, 1) route_kernel(const float*
     __shared__ int s_ids[kIdsInSmem ? 1024 : 1];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    griddep_launch_dependents();  // the gather may be scheduled; it waits for this grid
+    griddep_launch_dependents();  // the quantisation may run beside; it waits for this grid at its end
     for (int i = tid; i < kRouteWarps * kMaxExperts; i += kRouteThreads) {
         (&cnt_w[0][0])[i] = 0;
         (&run_w[0][0])[i] = 0;
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(32, 1) route_warp_kernel(const float* __restri
                                                            RouteOutputs o) {
     __shared__ int s_cnt[kMaxExperts];
     __shared__ int s_mt[kMaxExperts + 1];
-    griddep_launch_dependents();  // the gather may be scheduled; it waits for this grid
+    griddep_launch_dependents();  // the quantisation may run beside; it waits for this grid at its end
     const unsigned full = 0xffffffffu;
     const int lane = threadIdx.x;
     const int A = T * k;

@@ -52,15 +52,16 @@ def test_workspace_layout(moe):
                                           (300, 384, 640, 16, 3, 0), (1, 128, 128, 1, 1, 1)])
 def test_workspace_region_sizes(moe, T, H, F, E, k, dt):
     """Each region has the size its description in moe.h gives: routing arrays
-    of T*k ints, the padded layout of S = 128*(ceil(T*k/128) + E) rows with a
-    row pitch of row bytes + 128, h's block scales as 512-byte chunks per
-    (128-row tile, 128-column block) in FP8, the fp32 combine buffer [T, H]."""
+    of T*k ints, per-token e4m3 rows and scales (FP8 only), h in the padded
+    layout of S = 128*(ceil(T*k/128) + E) rows with a row pitch of row bytes
+    + 128, h's block scales as 512-byte chunks per (128-row tile, 128-column
+    block) in FP8, the fp32 combine buffer [T, H]."""
     A = T * k
     eb = 1 if dt == 1 else 2
     mt_max = -(-A // 128) + E
     S = 128 * mt_max
     want = dict(topk_ids=4 * A, topk_w=4 * A, counts=4 * E, offsets=4 * (E + 1), perm=4 * A, inv_perm=4 * A,
-                slot_of=4 * A, xs=S * (H * eb + 128), sx=4 * S, h=S * (F * eb + 128),
+                slot_of=4 * A, xs=T * H if dt == 1 else 0, sx=4 * T if dt == 1 else 0, h=S * (F * eb + 128),
                 h_sf=mt_max * (F // 128) * 512 if dt == 1 else 0, out32=4 * T * H, num_mtiles=4,
                 slot_assign=4 * S, mtile_expert=4 * mt_max, route_blocks=4 * (-(-T // 256)) * E)
     assert set(want) == set(moe.WS)
@@ -145,3 +146,22 @@ def test_test_hook_options_range(moe):
     assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, 4) == -1
     assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, -1) == -1
     assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, 0) == 0
+
+
+def test_dff_entry_checks_arguments(moe):
+    """The d_ff-sharded entry points reject bad rank arguments and pointers
+    before touching the device."""
+    import ctypes
+    P = 4096
+    ptrs = lambda n, v=P: (ctypes.c_void_p * n)(*([v] * n))  # noqa: E731
+    args = (P, P, P, P, P, P, 4, 128, 128, 2, 1, 1)
+    assert moe.moe_ffn_forward_dff(*args, 0, 0, ptrs(1), ptrs(1), P, 1 << 40, None) == -1    # no ranks
+    assert moe.moe_ffn_forward_dff(*args, 17, 0, ptrs(17), ptrs(17), P, 1 << 40, None) == -1  # > 16 ranks
+    assert moe.moe_ffn_forward_dff(*args, 2, 2, ptrs(2), ptrs(2), P, 1 << 40, None) == -1    # rank >= n_ranks
+    assert moe.moe_ffn_forward_dff(*args, 2, 0, None, ptrs(2), P, 1 << 40, None) == -1
+    assert moe.moe_ffn_forward_dff(*args, 2, 0, ptrs(2, P + 8), ptrs(2), P, 1 << 40, None) == -3
+    assert moe.moe_ffn_forward_dff(*args, 2, 0, ptrs(2), ptrs(2, P + 2), P, 1 << 40, None) == -3
+    assert moe.moe_ffn_forward_dff(*args, 2, 0, ptrs(2), ptrs(2), P, 10, None) == -4          # workspace
+    assert moe.moe_dff_finalize(P, P, 4, 100, P, 2, None) == -1                               # H % 128
+    assert moe.moe_dff_finalize(P, P, 4, 128, None, 2, None) == -1
+    assert moe.moe_dff_finalize(P + 4, P, 4, 128, P, 2, None) == -3

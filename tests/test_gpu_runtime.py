@@ -88,7 +88,7 @@ def test_output_deterministic_without_k_splits(moe):
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
 
 
-CORRUPT = pytest.mark.parametrize("table", [1, 2, 3], ids=["slot_of", "slot_assign", "mtile_expert"])
+CORRUPT = pytest.mark.parametrize("table", [1, 2, 3], ids=["slot_assign", "mtile_expert", "num_mtiles"])
 
 
 @CORRUPT
