@@ -19,6 +19,8 @@ decode         16     4096   14336  8   2  fp8    1     weight-streaming shape
 prefill        4096   4096   14336  8   2  fp8    2     tensor-core shape
 skewed         8192   4096   14336  8   2  bf16   3     logits + 2*log(1/(e+1))
 sweep_T<n>     n      4096   14336  8   2  fp8    4     n in {1, 128, 1024, 16384}
+decode_mxfp4   16     4096   14336  8   2  mxfp4  5     MX FP4 expert weights
+prefill_mxfp4  4096   4096   14336  8   2  mxfp4  6     MX FP4 expert weights
 =============  =====  =====  =====  ==  =  =====  ====  =================================
 
 Distributions: x ~ N(0,1) rounded to bf16; router logits ~ N(0,1) fp32;
@@ -47,6 +49,9 @@ CONFIGS = {
 }
 for _n in (1, 128, 1024, 16384):
     CONFIGS[f"sweep_T{_n}"] = _spec(_n, H_MIXTRAL, F_MIXTRAL, 8, 2, "fp8", 4)
+# MX-scaled FP4 expert weights (e2m1 with a power-of-two scale per 32 values)
+CONFIGS["decode_mxfp4"] = _spec(16, H_MIXTRAL, F_MIXTRAL, 8, 2, "mxfp4", 5)
+CONFIGS["prefill_mxfp4"] = _spec(4096, H_MIXTRAL, F_MIXTRAL, 8, 2, "mxfp4", 6)
 
 # stream ids of the generators
 _S_X, _S_LOGITS, _S_W1, _S_W3, _S_W2 = range(5)
@@ -91,11 +96,44 @@ def _weight(E, rows, cols, seed, stream, dtype):
     return codes, scales
 
 
+def _weight_mxfp4(E, rows, cols, seed, stream):
+    """[E, rows, cols] weights ~ N(0, 0.02^2) -> bf16, then the MX FP4 format
+    (OCP Microscaling): each block of 32 consecutive elements along `cols`
+    (the contraction dimension) shares the power of two X = 2^(floor(log2
+    amax) - 2) (2 = the exponent of e2m1's largest value, 6 = 1.5 * 2^2; X = 1
+    for an all-zero block), and each element is the e2m1 code of w / X
+    (round to nearest, ties to even, saturating at +-6; ml_dtypes' float4
+    conversion).  Returns (codes uint8 [E, rows, cols/2], two per byte, the
+    even column in the low 4 bits; exponents uint8 [E, rows, cols/32] biased
+    by 127)."""
+    import ml_dtypes
+    g = _gen(seed, stream)
+    codes = torch.empty(E, rows, cols // 2, dtype=torch.uint8)
+    exps = torch.empty(E, rows, cols // 32, dtype=torch.uint8)
+    for e in range(E):
+        wb = (torch.randn(rows, cols, generator=g) * 0.02).to(torch.bfloat16).float().numpy()
+        blk = wb.reshape(rows, cols // 32, 32)
+        amax = np.abs(blk).max(axis=2)
+        with np.errstate(divide="ignore"):
+            ex = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 2, 0).astype(np.int32)
+        ex = np.clip(ex, -127, 127)
+        q = (blk / np.ldexp(np.float32(1.0), ex)[:, :, None]).astype(np.float32)  # exact: a power of two
+        c4 = q.astype(ml_dtypes.float4_e2m1fn).view(np.uint8).reshape(rows, cols) & 0xF
+        codes[e] = torch.from_numpy((c4[:, 0::2] | (c4[:, 1::2] << 4)).astype(np.uint8))
+        exps[e] = torch.from_numpy((ex + 127).astype(np.uint8))
+    return codes, exps
+
+
 def make_weights(H, F, E, dtype="bf16", seed=0):
     """The expert weights of a case alone: dict(w1, w3, s1, s3, w2, s2) as in
     ``make_case`` (the same draws for the same shape, dtype and seed)."""
-    if dtype not in ("bf16", "fp8"):
+    if dtype not in ("bf16", "fp8", "mxfp4"):
         raise ValueError(dtype)
+    if dtype == "mxfp4":
+        w1, s1 = _weight_mxfp4(E, F, H, seed, _S_W1)
+        w3, s3 = _weight_mxfp4(E, F, H, seed, _S_W3)
+        w2, s2 = _weight_mxfp4(E, H, F, seed, _S_W2)
+        return dict(w1=w1, w3=w3, w2=w2, s1=s1, s3=s3, s2=s2)
     w1, s1 = _weight(E, F, H, seed, _S_W1, dtype)
     w3, s3 = _weight(E, F, H, seed, _S_W3, dtype)
     w2, s2 = _weight(E, H, F, seed, _S_W2, dtype)
@@ -107,9 +145,11 @@ def make_case(T, H, F, E, k, dtype="bf16", seed=0, skew=False, weights=None):
 
     Returns dict(x bf16 [T,H], logits f32 [T,E], w1/w3 [E,F,H], w2 [E,H,F]
     (bf16 or float8_e4m3fn), s1/s3 f32 [E,F], s2 f32 [E,H] (fp8 only, else
-    None), and the scalars T,H,F,E,k,dtype,seed).  ``weights``, if given, is
+    None), and the scalars T,H,F,E,k,dtype,seed).  mxfp4: w1/w3 uint8
+    [E,F,H/2], w2 uint8 [E,H,F/2] (packed e2m1), s1/s3 uint8 [E,F,H/32], s2
+    uint8 [E,H,F/32] (block exponents, see ``_weight_mxfp4``).  ``weights``, if given, is
     the result of ``make_weights(H, F, E, dtype, seed)`` (reused, not redrawn)."""
-    if dtype not in ("bf16", "fp8"):
+    if dtype not in ("bf16", "fp8", "mxfp4"):
         raise ValueError(dtype)
     w = weights if weights is not None else make_weights(H, F, E, dtype, seed)
     return dict(x=make_x(T, H, seed), logits=make_logits(T, E, seed, skew), **w,

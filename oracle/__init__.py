@@ -10,6 +10,8 @@ with gcc and marshals numpy arrays through ctypes.  Each wrapper names the
 step it follows:
 
 * ``quant_x``      -- per-token FP8 activation quantisation (R0);
+* ``e2m1_to_double``, ``ue8m0_to_double`` -- the MX FP4 element and block
+                      scale formats (MX-scaled FP4 expert weights);
 * ``route``        -- top-k, renormalised softmax, histogram, scan and stable
                       permutation (R1/R2; rocketrecap.com "FlyDSL kernels in
                       JAX", timestamps 5:56 "dynamic expert sizes" and 8:14
@@ -34,6 +36,7 @@ _lib = None
 
 BF16 = 0
 FP8 = 1
+MXFP4 = 2
 
 
 def build(force=False):
@@ -60,6 +63,10 @@ def _load():
         lib.oracle_e4m3_from_float.argtypes = [ctypes.c_float]
         lib.oracle_bf16_from_double.restype = ctypes.c_uint16
         lib.oracle_bf16_from_double.argtypes = [ctypes.c_double]
+        lib.oracle_e2m1_to_double.restype = ctypes.c_double
+        lib.oracle_e2m1_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_ue8m0_to_double.restype = ctypes.c_double
+        lib.oracle_ue8m0_to_double.argtypes = [ctypes.c_uint8]
         lib.oracle_bf16_to_double.restype = ctypes.c_double
         lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
         lib.oracle_mx_exponent.restype = I
@@ -100,6 +107,14 @@ def e4m3_to_double(code):
 
 def e4m3_from_float(v):
     return _load().oracle_e4m3_from_float(float(v))
+
+
+def e2m1_to_double(code):
+    return _load().oracle_e2m1_to_double(int(code) & 0xF)
+
+
+def ue8m0_to_double(e):
+    return _load().oracle_ue8m0_to_double(int(e) & 0xFF)
 
 
 def bf16_from_double(v):
@@ -158,15 +173,17 @@ def route(logits, k):
 # -- the layer --------------------------------------------------------------
 
 def _weights(case):
-    fp8 = case["dtype"] == "fp8"
-    wt = np.uint8 if fp8 else np.uint16
+    """Weights and scales of a case: bf16 bits; e4m3 codes + fp32 channel
+    scales (fp8); packed e2m1 codes + uint8 block exponents (mxfp4)."""
+    dt = case["dtype"]
+    wt = np.uint16 if dt == "bf16" else np.uint8
+    st = {"bf16": None, "fp8": np.float32, "mxfp4": np.uint8}[dt]
     w1 = _c(case["w1"], wt)
     w3 = _c(case["w3"], wt)
     w2 = _c(case["w2"], wt)
-    s1 = _c(case.get("s1"), np.float32) if fp8 else None
-    s3 = _c(case.get("s3"), np.float32) if fp8 else None
-    s2 = _c(case.get("s2"), np.float32) if fp8 else None
-    return w1, w3, w2, s1, s3, s2, (FP8 if fp8 else BF16)
+    s1, s3, s2 = ((_c(case.get(n), st) if st is not None else None) for n in ("s1", "s3", "s2"))
+    return w1, w3, w2, s1, s3, s2, {"bf16": BF16, "fp8": FP8, "mxfp4": MXFP4}[dt]
+
 
 
 def moe_ffn(case, mode="routed", nthreads=0, want_h=False):

@@ -27,6 +27,12 @@
  *     d_ff elements with a power-of-two (UE8M0) scale 2^ceil(log2(absmax/448)),
  *     clamped to [2^-127, 2^127], scale 1 for an all-zero block;
  *   - BF16 mode: h rounded to bf16 and used as is;
+ *   - MXFP4 mode (MX-scaled FP4 expert weights, the kinachrichten.com page
+ *     "PyTorch erhaelt FlyDSL-Backend", its list of kernel benchmarks: MXFP4
+ *     scaled GEMM, E8M0 scales per 32 values): every weight is an OCP e2m1
+ *     code times the power of two 2^(s - 127) that its block of 32
+ *     consecutive K elements (along d_model for w1/w3, along d_ff for w2)
+ *     shares; x and h are quantised as in FP8 mode;
  *   - the combine is an fp64 sum, rounded once to bf16.
  *
  * Build: gcc -O2 -fopenmp -shared -fPIC -fno-fast-math -ffp-contract=off moe_oracle.c
@@ -42,6 +48,7 @@
 
 #define ORACLE_BF16 0
 #define ORACLE_FP8 1
+#define ORACLE_MXFP4 2
 
 /* ------------------------------------------------------------------------ */
 /* Number formats, written from their definitions.                          */
@@ -61,6 +68,21 @@ double oracle_e4m3_to_double(uint8_t code) {
         mag = ldexp(1.0 + (double)man / 8.0, ex - 7); /* normal: 1.man * 2^(ex-7) */
     return sign ? -mag : mag;
 }
+
+/* OCP e2m1 (the MX FP4 element): 1 sign, 2 exponent bits (bias 1), 1 mantissa
+ * bit, no infinities or NaN; exponent field 0 is subnormal (0.m * 2^0).  Only
+ * the low 4 bits of `code` are read.  Magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+double oracle_e2m1_to_double(uint8_t code) {
+    int sign = (code >> 3) & 1;
+    int ex = (code >> 1) & 3;
+    int man = code & 1;
+    double mag = (ex == 0) ? (double)man * 0.5 : ldexp(1.0 + (double)man * 0.5, ex - 1);
+    return sign ? -mag : mag;
+}
+
+/* UE8M0 (the MX block scale): an unsigned 8-bit biased exponent, value
+ * 2^(e - 127); e = 255 is NaN. */
+double oracle_ue8m0_to_double(uint8_t e) { return e == 255 ? NAN : ldexp(1.0, (int)e - 127); }
 
 /* Values of the 256 codes, filled once when the library is loaded. */
 static double e4m3_value[256];
@@ -261,23 +283,29 @@ int oracle_route(const float* logits, int T, int E, int k, int32_t* ids, double*
 
 typedef struct {
     const uint16_t* x;   /* [T,H] bf16 */
-    const void* w1;      /* [E,F,H] bf16 or e4m3 */
+    const void* w1;      /* [E,F,H] bf16 or e4m3; MXFP4: [E,F,H/2] packed e2m1 */
     const void* w3;      /* [E,F,H] */
-    const float* s1;     /* [E,F] (FP8) */
-    const float* s3;     /* [E,F] */
-    const void* w2;      /* [E,H,F] */
-    const float* s2;     /* [E,H] */
+    const void* s1;      /* FP8: fp32 [E,F] per output channel; MXFP4: uint8 [E,F,H/32] block exponents */
+    const void* s3;
+    const void* w2;      /* [E,H,F]; MXFP4: [E,H,F/2] */
+    const void* s2;      /* FP8: fp32 [E,H]; MXFP4: uint8 [E,H,F/32] */
     int T, H, F, E, k, dtype;
     double e4m3_table[256];
-    const uint8_t* xq;   /* [T,H] (FP8) */
+    const uint8_t* xq;   /* [T,H] (FP8, MXFP4) */
     const float* sx;     /* [T] */
 } ffn_ctx;
 
-static double weight_value(const ffn_ctx* c, const void* w, const float* s, int e, int row, int col,
+/* Element (row, col) of expert e's matrix [rows, cols] (cols = K).  MXFP4:
+ * two e2m1 codes per byte, the even column in the low 4 bits; the block
+ * exponent of (row, col / 32). */
+static double weight_value(const ffn_ctx* c, const void* w, const void* s, int e, int row, int col,
                            int rows, int cols) {
-    size_t i = ((size_t)e * rows + row) * cols + col;
-    if (c->dtype == ORACLE_BF16) return oracle_bf16_to_double(((const uint16_t*)w)[i]);
-    return c->e4m3_table[((const uint8_t*)w)[i]] * (double)s[(size_t)e * rows + row];
+    size_t r = (size_t)e * rows + row;
+    if (c->dtype == ORACLE_BF16) return oracle_bf16_to_double(((const uint16_t*)w)[r * cols + col]);
+    if (c->dtype == ORACLE_FP8) return c->e4m3_table[((const uint8_t*)w)[r * cols + col]] * (double)((const float*)s)[r];
+    uint8_t byte = ((const uint8_t*)w)[r * (cols / 2) + col / 2];
+    uint8_t code = (col & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+    return oracle_e2m1_to_double(code) * oracle_ue8m0_to_double(((const uint8_t*)s)[r * (cols / 32) + col / 32]);
 }
 
 static double x_value(const ffn_ctx* c, int t, int i) {
@@ -303,7 +331,7 @@ static void expert_ffn(const ffn_ctx* c, int e, int t, double* y, double* h_out,
         if (h_exact) h_exact[n] = silu * u;
         hq[n] = oracle_bf16_to_double(oracle_bf16_from_double(silu * u));
     }
-    if (c->dtype == ORACLE_FP8) {
+    if (c->dtype != ORACLE_BF16) {
         uint8_t codes[32];
         for (int b = 0; b < F; b += 32) {
             int n = (F - b < 32) ? F - b : 32;
@@ -320,12 +348,13 @@ static void expert_ffn(const ffn_ctx* c, int e, int t, double* y, double* h_out,
     free(hq);
 }
 
-static int ctx_init(ffn_ctx* c, const uint16_t* x, const void* w1, const void* w3, const float* s1,
-                    const float* s3, const void* w2, const float* s2, int T, int H, int F, int E, int k,
+static int ctx_init(ffn_ctx* c, const uint16_t* x, const void* w1, const void* w3, const void* s1,
+                    const void* s3, const void* w2, const void* s2, int T, int H, int F, int E, int k,
                     int dtype) {
     if (T < 0 || H < 1 || F < 1 || E < 1 || E > 64 || k < 1 || k > E) return -1;
-    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP8) return -1;
-    if (dtype == ORACLE_FP8 && (!s1 || !s3 || !s2)) return -1;
+    if (dtype != ORACLE_BF16 && dtype != ORACLE_FP8 && dtype != ORACLE_MXFP4) return -1;
+    if (dtype != ORACLE_BF16 && (!s1 || !s3 || !s2)) return -1;
+    if (dtype == ORACLE_MXFP4 && (H % 32 || F % 32)) return -1;
     c->x = x; c->w1 = w1; c->w3 = w3; c->s1 = s1; c->s3 = s3; c->w2 = w2; c->s2 = s2;
     c->T = T; c->H = H; c->F = F; c->E = E; c->k = k; c->dtype = dtype;
     for (int i = 0; i < 256; ++i) c->e4m3_table[i] = oracle_e4m3_to_double((uint8_t)i);
@@ -345,7 +374,7 @@ static int ctx_init(ffn_ctx* c, const uint16_t* x, const void* w1, const void* w
  * h_sorted (optional, routed mode): [T*k, F] dequantised intermediate in
  * sorted order.  Returns 0, or -1 on a bad argument. */
 int oracle_moe_ffn(int mode, const uint16_t* x, const float* logits, const void* w1, const void* w3,
-                   const float* s1, const float* s3, const void* w2, const float* s2, int T, int H, int F,
+                   const void* s1, const void* s3, const void* w2, const void* s2, int T, int H, int F,
                    int E, int k, int dtype, uint16_t* out, double* out64, double* h_sorted, int nthreads) {
     ffn_ctx c;
     if (ctx_init(&c, x, w1, w3, s1, s3, w2, s2, T, H, F, E, k, dtype)) return -1;
@@ -360,7 +389,7 @@ int oracle_moe_ffn(int mode, const uint16_t* x, const float* logits, const void*
     int32_t offsets[65];
     uint8_t* xq = NULL;
     float* sx = NULL;
-    if (dtype == ORACLE_FP8) {
+    if (dtype != ORACLE_BF16) {
         xq = (uint8_t*)malloc((size_t)T * H + 1);
         sx = (float*)malloc(sizeof(float) * (T ? T : 1));
         oracle_quant_x(x, T, H, xq, sx);
@@ -416,7 +445,7 @@ int oracle_moe_ffn(int mode, const uint16_t* x, const float* logits, const void*
  * before rounding).  Used for sampled checks at full size and for the CPU
  * timing sample. */
 int oracle_moe_ffn_tokens(const uint16_t* x, const float* logits, const void* w1, const void* w3,
-                          const float* s1, const float* s3, const void* w2, const float* s2, int T, int H,
+                          const void* s1, const void* s3, const void* w2, const void* s2, int T, int H,
                           int F, int E, int k, int dtype, const int32_t* tokens, int ntok, uint16_t* out,
                           double* out64, double* h_deq, double* h_exact, int nthreads) {
     ffn_ctx c;
@@ -431,7 +460,7 @@ int oracle_moe_ffn_tokens(const uint16_t* x, const float* logits, const void* w1
     double* w = (double*)malloc(sizeof(double) * (work ? work : 1));
     uint8_t* xq = NULL;
     float* sx = NULL;
-    if (dtype == ORACLE_FP8) {
+    if (dtype != ORACLE_BF16) {
         /* quantise only the sampled rows, indexed by their own token id */
         xq = (uint8_t*)calloc((size_t)T * H + 1, 1);
         sx = (float*)calloc((size_t)(T ? T : 1), sizeof(float));

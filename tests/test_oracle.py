@@ -282,20 +282,83 @@ def test_route_skewed_shares():
     assert share[0] > 0.40 and share[7] < 0.01 and np.all(np.diff(share) < 0)
 
 
+# ---------------------------------------------------------------- MX FP4 weight formats
+
+def test_e2m1_decode_all_codes():
+    """The 16 e2m1 codes against ml_dtypes' float4_e2m1fn (magnitudes 0, 0.5,
+    1, 1.5, 2, 3, 4, 6 and their negatives; -0 keeps its sign)."""
+    import ml_dtypes
+    ref = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    got = np.array([oracle.e2m1_to_double(c) for c in range(16)])
+    np.testing.assert_array_equal(got, ref)
+    assert math.copysign(1.0, oracle.e2m1_to_double(8)) == -1.0
+    assert oracle.e2m1_to_double(0x17) == oracle.e2m1_to_double(0x07) == 6.0  # only the low 4 bits count
+
+
+def test_ue8m0_decode_all_codes():
+    import ml_dtypes
+    ref = np.arange(256, dtype=np.uint8).view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    got = np.array([oracle.ue8m0_to_double(c) for c in range(256)])
+    np.testing.assert_array_equal(got[:255], ref[:255])
+    assert math.isnan(got[255]) and math.isnan(ref[255])
+    assert got[127] == 1.0 and got[0] == 2.0 ** -127 and got[254] == 2.0 ** 127
+
+
+def test_mxfp4_weights_are_an_mx_block_quantisation():
+    """The MX FP4 input format (OCP Microscaling): the block scale is
+    2^(floor(log2 amax) - 2), so a block's largest magnitude sits in [4, 8)
+    before rounding; every weight is within half an e2m1 step of the bf16
+    draw it encodes, except magnitudes above 6, which saturate at 6."""
+    E, rows, cols = 2, 64, 256
+    codes, exps = moe_inputs._weight_mxfp4(E, rows, cols, seed=21, stream=0)
+    g = moe_inputs._gen(21, 0)
+    for e in range(E):
+        wb = (torch.randn(rows, cols, generator=g) * 0.02).to(torch.bfloat16).double().numpy()
+        deq = _mx_fp4_dequant(codes[e], exps[e]).numpy()
+        scale = np.repeat(2.0 ** (exps[e].numpy().astype(np.int64) - 127), 32, axis=1)
+        q = deq / scale
+        assert np.abs(q).max() <= 6.0
+        # error at most half the e2m1 spacing at that magnitude (0.5 below 2, 1 in [2, 4), 2 in [4, 6])
+        mag = np.abs(wb / scale)
+        assert mag.max() < 8.0
+        spacing = np.where(mag < 2, 0.5, np.where(mag < 4, 1.0, 2.0))
+        allowed = np.where(mag > 6, mag - 6, 0.5 * spacing)
+        assert np.all(np.abs(q - wb / scale) <= allowed + 1e-12)
+        bmax = np.abs(q).reshape(rows, cols // 32, 32).max(axis=2)
+        assert np.all((bmax >= 4.0) & (bmax <= 6.0))
+
+
 # ---------------------------------------------------------------- the layer
 
 def _bf16_round_vec(a):
     return np.array([oracle.bf16_to_double(oracle.bf16_from_double(float(v))) for v in a.reshape(-1)]).reshape(a.shape)
 
 
+def _mx_fp4_dequant(codes, exps):
+    """Packed e2m1 codes [rows, K/2] and block exponents [rows, K/32] -> float64
+    [rows, K], decoded by ml_dtypes (an independent implementation of both
+    formats); the even column sits in the low 4 bits of each byte."""
+    import ml_dtypes
+    c = codes.numpy()
+    nib = np.empty((c.shape[0], c.shape[1] * 2), dtype=np.uint8)
+    nib[:, 0::2] = c & 0xF
+    nib[:, 1::2] = c >> 4
+    vals = nib.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    scale = exps.numpy().view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    return torch.tensor(vals * np.repeat(scale, 32, axis=1))
+
+
 def _dense_swiglu_reference(case, tok):
     """E=1, k=1: the layer is a dense SwiGLU MLP; fp64 torch matmuls."""
-    fp8 = case["dtype"] == "fp8"
+    fp8 = case["dtype"] in ("fp8", "mxfp4")
     x = case["x"].double()
     if fp8:
         xq, sx = oracle.quant_x(moe_inputs.to_numpy(case)["x"])
         xd = torch.tensor(xq).view(torch.float8_e4m3fn).double() * torch.tensor(sx).double()[:, None]
-        deq = lambda w, s: w.double() * s.double()[..., None]  # noqa: E731
+        if case["dtype"] == "fp8":
+            deq = lambda w, s: w.double() * s.double()[..., None]  # noqa: E731
+        else:
+            deq = _mx_fp4_dequant
         W1, W3, W2 = deq(case["w1"][0], case["s1"][0]), deq(case["w3"][0], case["s3"][0]), deq(case["w2"][0], case["s2"][0])
     else:
         xd = x
@@ -314,7 +377,7 @@ def _dense_swiglu_reference(case, tok):
     return (torch.tensor(h) @ W2.T).numpy()
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "mxfp4"])
 def test_single_expert_equals_dense_swiglu_mlp(dtype):
     case = moe_inputs.make_case(T=6, H=64, F=96, E=1, k=1, dtype=dtype, seed=11)
     r = oracle.moe_ffn(moe_inputs.to_numpy(case))
@@ -324,7 +387,7 @@ def test_single_expert_equals_dense_swiglu_mlp(dtype):
     np.testing.assert_array_equal(r["out"], np.array([[oracle.bf16_from_double(v) for v in row] for row in ref]))
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "mxfp4"])
 def test_routed_equals_masked_dense(dtype):
     case = moe_inputs.make_case(T=12, H=64, F=64, E=4, k=2, dtype=dtype, seed=12)
     nc = moe_inputs.to_numpy(case)
