@@ -87,16 +87,28 @@ def workload_desc(spec, name):
             f"top-{spec['k']}, {spec['dtype']}" + (", skewed routing" if spec["skew"] else ""))
 
 
+def weight_bytes(dtype, rows, cols):
+    """Bytes of one expert matrix [rows, cols] with its scales: bf16; e4m3 +
+    one fp32 scale per row; MX FP4 = half a byte per code + one byte per 32."""
+    if dtype == "bf16":
+        return 2 * rows * cols
+    if dtype == "fp8":
+        return rows * cols + 4 * rows
+    return rows * cols // 2 + rows * cols // 32
+
+
 def algorithmic(spec, counts):
     """Algorithmic FLOPs and bytes of the layer and of each GEMM kernel, from
     the routed expert counts (experts with no tokens read no weights)."""
     T, H, F, E, k = spec["T"], spec["H"], spec["F"], spec["E"], spec["k"]
-    bw = 1 if spec["dtype"] == "fp8" else 2
+    dt = spec["dtype"]
+    ba = 2 if dt == "bf16" else 1  # activation / h bytes per element
+    sf = (lambda n: n // 32) if dt != "bf16" else (lambda n: 0)  # h's block scales
     A = T * k
     active = sum(1 for c in counts if c > 0)
-    s1_bytes = active * (2 * F * H * bw + (8 * F if bw == 1 else 0)) + A * H * bw + A * F * bw + (A * F // 32 if bw == 1 else 0)
-    s2_bytes = active * (H * F * bw + (4 * H if bw == 1 else 0)) + A * F * bw + (A * F // 32 if bw == 1 else 0) + T * H * 4
-    layer_bytes = active * (3 * H * F * bw + (4 * (2 * F + H) if bw == 1 else 0)) + T * H * 2 * 2 + 4 * T * E
+    s1_bytes = active * weight_bytes(dt, 2 * F, H) + A * H * ba + A * F * ba + sf(A * F)
+    s2_bytes = active * weight_bytes(dt, H, F) + A * F * ba + sf(A * F) + T * H * 4
+    layer_bytes = active * (weight_bytes(dt, 2 * F, H) + weight_bytes(dt, H, F)) + T * H * 2 * 2 + 4 * T * E
     return dict(s1_flops=4.0 * H * F * A, s2_flops=2.0 * H * F * A, layer_flops=6.0 * H * F * A + 2.0 * T * E,
                 s1_bytes=float(s1_bytes), s2_bytes=float(s2_bytes), layer_bytes=float(layer_bytes), active=active)
 
@@ -106,9 +118,9 @@ def roofline(spec, alg, dom, dom_ms, window_ms, peaks, peak_kind, name):
     shapes) or FLOPs (tensor-bound shapes) per launch over its average launch
     time, against the measured peak."""
     H, F = spec["H"], spec["F"]
-    fp8 = spec["dtype"] == "fp8"
-    decode_like = alg["active"] * 3 * H * F * (1 if fp8 else 2) / 6.5e12 > alg["layer_flops"] / (
-        (2 * 2.25e15) if fp8 else 2.25e15)
+    fp8 = spec["dtype"] != "bf16"  # e4m3 activations: the FP8 tensor rate (MX FP4 weights too)
+    wb = weight_bytes(spec["dtype"], 3 * H, F)
+    decode_like = alg["active"] * wb / 6.5e12 > alg["layer_flops"] / ((2 * 2.25e15) if fp8 else 2.25e15)
     if not dom.startswith("stage"):
         return {"bound": "hbm", "achieved": None, "peak": float(peaks.get("hbm_gbs", 6650.0)), "unit": "GB/s",
                 "frac": None, "traffic": None, "kernel": dom, "kernel_ms": dom_ms}
@@ -352,10 +364,14 @@ class Weights:
             self.w = None
             torch.cuda.empty_cache()
             fp8 = spec["dtype"] == "fp8"
-            w13, s13, w2 = moe.prepare_weights(case["w1"].to(dev), case["w3"].to(dev),
-                                               case["s1"].to(dev) if fp8 else None,
-                                               case["s3"].to(dev) if fp8 else None, case["w2"].to(dev))
-            s2 = case["s2"].to(dev) if fp8 else None
+            if spec["dtype"] == "mxfp4":
+                w13, s13, w2, s2 = moe.prepare_weights_mx(*(case[n].to(dev) for n in ("w1", "w3", "s1", "s3", "w2",
+                                                                                        "s2")))
+            else:
+                w13, s13, w2 = moe.prepare_weights(case["w1"].to(dev), case["w3"].to(dev),
+                                                   case["s1"].to(dev) if fp8 else None,
+                                                   case["s3"].to(dev) if fp8 else None, case["w2"].to(dev))
+                s2 = case["s2"].to(dev) if fp8 else None
             torch.cuda.synchronize()
             torch.cuda.empty_cache()
             self.key, self.w = key, (w13, s13, w2, s2)
@@ -369,7 +385,7 @@ def run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_s
     import torch
     import torch.distributed as dist
     T, H, F, E, k = spec["T"], spec["H"], spec["F"], spec["E"], spec["k"]
-    fp8 = spec["dtype"] == "fp8"
+    fp8 = {"bf16": False, "fp8": True, "mxfp4": "mxfp4"}[spec["dtype"]]  # the binding's dtype argument
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and cpu_seconds > 0:
@@ -384,7 +400,7 @@ def run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_s
         x_cpu, lg_cpu = case["x"], case["logits"]
     x = x_cpu.to(dev)
     logits = lg_cpu.to(dev)
-    dt_code = moe.MOE_FP8_E4M3 if fp8 else moe.MOE_BF16
+    dt_code = moe.dtype_code(spec["dtype"])
     ws = moe.workspace(T, H, F, E, k, dt_code, dev)
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -505,11 +521,13 @@ def run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_s
     launches = sum(v[1] for v in kern.values())  # K steps, the same count as the timed region
     rec = {
         "value": value, "unit": "tokens/s", "ms_per_step": ms_step, "steps": args.steps, "warmup": args.warmup,
-        "dtype": "fp8_e4m3 (fp32 accumulate)" if fp8 else "bf16 (fp32 accumulate)",
+        "dtype": {"fp8": "fp8_e4m3 (fp32 accumulate)", "bf16": "bf16 (fp32 accumulate)",
+                  "mxfp4": "e2m1 weights with UE8M0 block scales x fp8_e4m3 activations (fp32 accumulate)"}[
+                      spec["dtype"]],
         "config": {"workload": workload_desc(spec, name), "T": T, "d_model": H, "d_ff": F, "experts": E, "top_k": k,
                    "weights": spec["dtype"], "parallelism": f"weak-scaling replicas x{world}" if world > 1 else "1 GPU",
                    "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (
-                       alg["active"] * 3 * H * F * (1 if fp8 else 2) / 1e9),
+                       alg["active"] * weight_bytes(spec["dtype"], 3 * H, F) / 1e9),
                    "expert_counts": counts},
         "roofline": roof,
         "layer": {"tflops": alg["layer_flops"] / (ms_step / 1e3) / 1e12,

@@ -53,9 +53,13 @@ typedef enum {
 } moe_status;
 
 typedef enum {
-    MOE_BF16 = 0,     /* bf16 activations and weights */
-    MOE_FP8_E4M3 = 1  /* e4m3 weights with fp32 per-output-channel scales; bf16 activations
-                         quantised per token to e4m3 inside the layer */
+    MOE_BF16 = 0,      /* bf16 activations and weights */
+    MOE_FP8_E4M3 = 1,  /* e4m3 weights with fp32 per-output-channel scales; bf16 activations
+                          quantised per token to e4m3 inside the layer */
+    MOE_MXFP4 = 2      /* MX FP4 weights: e2m1 codes with one UE8M0 (power-of-two) scale per 32
+                          consecutive contraction elements (the kinachrichten.com page "PyTorch
+                          erhaelt FlyDSL-Backend", its kernel list: MXFP4 scaled GEMM); activations
+                          and h as in MOE_FP8_E4M3 */
 } moe_dtype;
 
 /* Bytes of device workspace moe_ffn_forward needs for this problem (0 on bad
@@ -88,6 +92,31 @@ int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const f
                         void* w13_out, float* s13_out, void* w2_out, int E, int F, int H, int dtype, void* stream);
 
 /*
+ * One-time preparation of MX FP4 expert weights (MOE_MXFP4; the load-time
+ * preshuffle of timestamp 8:14 for this format).
+ *   w1, w3   device, [E,F,H/2] bytes: e2m1 codes, two per byte, the even
+ *            column (d_model index) in the low 4 bits; read only
+ *   s1, s3   device, [E,F,H/32] bytes: UE8M0 exponents (scale 2^(s-127)) of the
+ *            blocks of 32 consecutive columns; read only
+ *   w2       device, [E,H,F/2] bytes; s2 device, [E,H,F/32] bytes (blocks along d_ff)
+ *   w13_out  device, E*2F*H/2 bytes: w1/w3 rows interleaved in groups of 32 as
+ *            for moe_prepare_weights, still packed, row-major (read by TMA,
+ *            which spreads the codes to one per byte in shared memory);
+ *            32-byte aligned
+ *   s13_out  device, E*2F*H/32 bytes: the scales of those rows regrouped into
+ *            512-byte chunks per (expert, 128-row block, 128-column block),
+ *            byte (r%32)*16 + (r/32)*4 + b = row r of the block, 32-column
+ *            block b of the chunk (the order the MMA's scale copy takes)
+ *   w2_out   device, E*H*F/2 bytes (32-byte aligned); s2_out E*H*F/32 bytes,
+ *            the same chunks over [E,H] rows and d_ff columns
+ * The layer is then called with dtype MOE_MXFP4, w13 = w13_out, s13 = s13_out,
+ * w2 = w2_out, s2 = s2_out.
+ */
+int moe_prepare_weights_mx(const void* w1, const void* w3, const void* s1, const void* s3, const void* w2,
+                           const void* s2, void* w13_out, void* s13_out, void* w2_out, void* s2_out, int E, int F,
+                           int H, void* stream);
+
+/*
  * Routing alone (timestamps 5:56 and 8:14): top-k selection, softmax over the
  * k selected logits, expert histogram, exclusive scan and stable permutation.
  *   logits    device, [T,E] fp32, read only.  Larger logit first; equal logits
@@ -113,9 +142,11 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float
  *   x        device, [T,H] bf16, read only.
  *   logits   device, [T,E] fp32, read only (routed exactly as moe_route does).
  *   w13      device, w1/w3 prepared by moe_prepare_weights (blocked, interleaved).
- *   s13      device, [E,2F] fp32 (FP8) or NULL (BF16), from moe_prepare_weights.
- *   w2       device, w2 prepared by moe_prepare_weights (blocked).
- *   s2       device, [E,H] fp32 (FP8) or NULL (BF16).
+ *   s13      device, [E,2F] fp32 (FP8) or NULL (BF16), from moe_prepare_weights;
+ *            MXFP4: the scale chunks from moe_prepare_weights_mx.
+ *   w2       device, w2 prepared by moe_prepare_weights (blocked; MXFP4: by
+ *            moe_prepare_weights_mx).
+ *   s2       device, [E,H] fp32 (FP8) or NULL (BF16); MXFP4: prepared chunks.
  *   out      device, [T,H] bf16, written.
  *   ws       device workspace, >= moe_workspace_size(T,H,F,E,k,dtype) bytes;
  *            scratch, contents undefined afterwards (moe_workspace_region
@@ -125,7 +156,9 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float
  * x is quantised per token (sx = absmax/448 in IEEE fp32, e4m3 round to
  * nearest even with saturation); the intermediate h is rounded to bf16 and
  * re-quantised to e4m3 in blocks of 32 d_ff elements with a power-of-two
- * scale 2^ceil(log2(absmax/448)).  BF16 mode: h is rounded to bf16.  The k
+ * scale 2^ceil(log2(absmax/448)).  MXFP4 mode: the same, with the weights'
+ * block scales applied inside the MMAs (128 x 128 one-CTA tiles whatever
+ * MOE_OPT_PATH asks).  BF16 mode: h is rounded to bf16.  The k
  * weighted expert outputs are summed in fp32 and rounded once to bf16.
  * Execution: five kernels (six from 1024 tokens on) chained on `stream` with
  * programmatic dependent launch -- routing, per-token quantisation, the first
@@ -138,8 +171,8 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float
  * use 256 x 256 tiles on pairs of SMs.  The call makes no host<->device
  * synchronisation and may be captured in a CUDA graph.
  */
-int moe_ffn_forward(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
-                    const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
+int moe_ffn_forward(const void* x, const float* logits, const void* w13, const void* s13, const void* w2,
+                    const void* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
                     size_t ws_bytes, void* stream);
 
 /*
@@ -168,8 +201,8 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const f
  *   zero).  Calls whose work overlaps on the GPU -- e.g. on two streams at
  *   once -- race on it and give undefined results; serialise them.
  */
-int moe_ffn_forward_static(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
-                           const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* stream);
+int moe_ffn_forward_static(const void* x, const float* logits, const void* w13, const void* s13, const void* w2,
+                           const void* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* stream);
 size_t moe_static_workspace_bytes(void);
 
 /*
@@ -198,8 +231,8 @@ size_t moe_static_workspace_bytes(void);
  *            arrival counter (zero before the first step).
  * Returns as moe_ffn_forward; 1 <= n_ranks <= 16, 0 <= rank < n_ranks.
  */
-int moe_ffn_forward_dff(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
-                        const float* s2, int T, int H, int F_shard, int E, int k, int dtype, int n_ranks, int rank,
+int moe_ffn_forward_dff(const void* x, const float* logits, const void* w13, const void* s13, const void* w2,
+                        const void* s2, int T, int H, int F_shard, int E, int k, int dtype, int n_ranks, int rank,
                         float* const* peer_out32, unsigned int* const* peer_counter, void* ws, size_t ws_bytes,
                         void* stream);
 

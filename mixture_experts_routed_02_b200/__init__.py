@@ -44,6 +44,7 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
                 -7: "MOE_ERR_DEVICE_BOUNDS"}
 MOE_BF16 = 0
 MOE_FP8_E4M3 = 1
+MOE_MXFP4 = 2
 OPT_PATH, OPT_SPLITK, OPT_TIMEOUT_MS, OPT_TEST_STALL, OPT_TEST_CORRUPT = 0, 1, 2, 3, 4
 
 # workspace regions (moe_ws_region)
@@ -53,7 +54,8 @@ WS = dict(topk_ids=0, topk_w=1, counts=2, offsets=3, perm=4, inv_perm=5, slot_of
 # every symbol include/moe.h declares
 EXPORTS = ["moe_workspace_size", "moe_prepare_weights", "moe_route", "moe_ffn_forward", "moe_get_status",
            "moe_workspace_region", "moe_set_option", "moe_profile_enable", "moe_profile_read",
-           "moe_ffn_forward_static", "moe_static_workspace_bytes", "moe_ffn_forward_dff", "moe_dff_finalize"]
+           "moe_ffn_forward_static", "moe_static_workspace_bytes", "moe_ffn_forward_dff", "moe_dff_finalize",
+           "moe_prepare_weights_mx"]
 KERNELS = ["route", "quantize", "stage1_w13_swiglu", "stage2_w2_scatter", "finalize"]
 
 
@@ -74,6 +76,8 @@ lib.moe_workspace_region.restype = ctypes.c_longlong
 lib.moe_workspace_region.argtypes = [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_Z)]
 lib.moe_prepare_weights.restype = _I
 lib.moe_prepare_weights.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]
+lib.moe_prepare_weights_mx.restype = _I
+lib.moe_prepare_weights_mx.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P]
 lib.moe_route.restype = _I
 lib.moe_route.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P]
 lib.moe_ffn_forward.restype = _I
@@ -98,6 +102,7 @@ lib.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER
 # raw entry points, same names as the C ABI
 moe_workspace_size = lib.moe_workspace_size
 moe_prepare_weights = lib.moe_prepare_weights
+moe_prepare_weights_mx = lib.moe_prepare_weights_mx
 moe_route = lib.moe_route
 moe_ffn_forward = lib.moe_ffn_forward
 moe_get_status = lib.moe_get_status
@@ -145,7 +150,12 @@ def _check(fn, rc):
 
 
 def dtype_code(dtype):
-    return MOE_FP8_E4M3 if dtype in ("fp8", MOE_FP8_E4M3) else MOE_BF16
+    """"bf16" / "fp8" / "mxfp4" (or True = fp8, False = bf16, or the codes) -> the moe_dtype code."""
+    if dtype in ("mxfp4", MOE_MXFP4) and dtype is not True:
+        return MOE_MXFP4
+    if dtype is True or dtype in ("fp8", MOE_FP8_E4M3):
+        return MOE_FP8_E4M3
+    return MOE_BF16
 
 
 def workspace(T, H, F, E, k, dtype, device="cuda"):
@@ -163,6 +173,24 @@ def ws_view(ws, T, H, F, E, k, dtype, which, torch_dtype=None):
     off, n = moe_workspace_region(T, H, F, E, k, dtype_code(dtype), which)
     v = ws[off:off + n]
     return v.view(torch_dtype) if torch_dtype is not None else v
+
+
+def prepare_weights_mx(w1, w3, s1, s3, w2, s2, stream=None):
+    """One-time preparation of MX FP4 weights (uint8 tensors: packed e2m1
+    w1/w3 [E,F,H/2], w2 [E,H,F/2]; UE8M0 exponents s1/s3 [E,F,H/32], s2
+    [E,H,F/32]); returns (w13, s13, w2p, s2p) for ffn_forward(..., "mxfp4")."""
+    import torch
+    E, F, Hh = w1.shape
+    H = 2 * Hh
+    dev = w1.device
+    w13 = torch.empty(E * 2 * F * Hh, dtype=torch.uint8, device=dev)
+    s13 = torch.empty(E * 2 * F * (H // 32), dtype=torch.uint8, device=dev)
+    w2p = torch.empty_like(w2).view(-1)
+    s2p = torch.empty_like(s2).view(-1)
+    rc = moe_prepare_weights_mx(_ptr(w1), _ptr(w3), _ptr(s1), _ptr(s3), _ptr(w2), _ptr(s2), _ptr(w13), _ptr(s13),
+                                _ptr(w2p), _ptr(s2p), E, F, H, _stream(stream))
+    _check("moe_prepare_weights_mx", rc)
+    return w13, s13, w2p, s2p
 
 
 def prepare_weights(w1, w3, s1, s3, w2, stream=None):
@@ -200,11 +228,13 @@ def route(logits, k, stream=None):
 
 
 def ffn_forward(x, logits, w13, s13, w2p, s2, k, F, fp8, out=None, ws=None, stream=None):
-    """The whole layer on prepared weights; returns the bf16 output [T,H] (and fills ``ws``)."""
+    """The whole layer on prepared weights; returns the bf16 output [T,H] (and
+    fills ``ws``).  ``fp8``: True (e4m3 weights), False (bf16) or "mxfp4"."""
     import torch
     T, H = x.shape
     E = logits.shape[1]
-    dt = MOE_FP8_E4M3 if fp8 else MOE_BF16
+    dt = dtype_code(fp8)
+    fp8 = dt != MOE_BF16
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
     if ws is None:

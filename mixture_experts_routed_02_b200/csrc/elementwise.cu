@@ -236,6 +236,74 @@ __global__ void interleave_scales_kernel(const float* __restrict__ s1, const flo
     }
 }
 
+// MX FP4 weight preparation.  Rows of packed e2m1 codes (row_bytes each)
+// copied in 16-byte chunks; with `interleave` destination row R of an expert
+// is row 32*(R/64) + R%32 of a (R%64 < 32) or of b (the w1/w3 interleave of
+// the first GEMM), otherwise row R of a.
+__global__ void mx_rows_kernel(const uint8_t* __restrict__ a, const uint8_t* __restrict__ b,
+                               uint8_t* __restrict__ dst, int E, int src_rows, int dst_rows, int row_bytes,
+                               bool interleave) {
+    const int chunks = row_bytes / 16;
+    const size_t total = (size_t)E * dst_rows * chunks;
+    for (size_t g = blockIdx.x * (size_t)blockDim.x + threadIdx.x; g < total; g += (size_t)gridDim.x * blockDim.x) {
+        const int c = (int)(g % chunks);
+        const size_t rowg = g / chunks;
+        const int R = (int)(rowg % dst_rows);
+        const int e = (int)(rowg / dst_rows);
+        const uint8_t* src = a;
+        int srow = R;
+        if (interleave) {
+            src = (R % 64 < 32) ? a : b;
+            srow = 32 * (R / 64) + (R % 32);
+        }
+        reinterpret_cast<uint4*>(dst)[g] =
+            __ldg(reinterpret_cast<const uint4*>(src + ((size_t)e * src_rows + srow) * row_bytes) + c);
+    }
+}
+
+// The weights' UE8M0 block scales ([rows, K/32] per expert) regrouped into
+// one 512-byte chunk per (expert, 128-row block, 128-element K tile), in the
+// order the MMA's scale copy into TMEM takes (the same as h's scale chunks):
+// byte (r % 32) * 16 + (r / 32) * 4 + kb holds the scale of row r of the
+// block and K block kb of the tile.  Rows interleaved as in mx_rows_kernel.
+__global__ void mx_scale_chunks_kernel(const uint8_t* __restrict__ sa, const uint8_t* __restrict__ sb,
+                                       uint8_t* __restrict__ dst, int E, int src_rows, int dst_rows, int k_tiles,
+                                       bool interleave) {
+    const int nblk = dst_rows / 128;
+    const size_t total = (size_t)E * nblk * k_tiles * 512;
+    for (size_t g = blockIdx.x * (size_t)blockDim.x + threadIdx.x; g < total; g += (size_t)gridDim.x * blockDim.x) {
+        const int p = (int)(g % 512);
+        const size_t c = g / 512;
+        const int kt = (int)(c % k_tiles);
+        const int nb = (int)((c / k_tiles) % nblk);
+        const int e = (int)(c / ((size_t)k_tiles * nblk));
+        const int r = (p / 16) + 32 * ((p % 16) / 4);
+        const int kb = p % 4;
+        const int R = nb * 128 + r;
+        const uint8_t* src = sa;
+        int srow = R;
+        if (interleave) {
+            src = (R % 64 < 32) ? sa : sb;
+            srow = 32 * (R / 64) + (R % 32);
+        }
+        dst[g] = src[((size_t)e * src_rows + srow) * (k_tiles * 4) + kt * 4 + kb];
+    }
+}
+
+cudaError_t launch_mx_prepare(const uint8_t* a, const uint8_t* b, const uint8_t* sa, const uint8_t* sb,
+                              uint8_t* w_out, uint8_t* s_out, int E, int src_rows, int dst_rows, int K,
+                              bool interleave, cudaStream_t stream) {
+    const size_t nrow = (size_t)E * dst_rows * (K / 2) / 16;
+    mx_rows_kernel<<<(int)std::min<size_t>((nrow + 255) / 256, 65535), 256, 0, stream>>>(
+        a, b, w_out, E, src_rows, dst_rows, K / 2, interleave);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    const size_t nsf = (size_t)E * dst_rows * (K / 32);
+    mx_scale_chunks_kernel<<<(int)std::min<size_t>((nsf + 255) / 256, 65535), 256, 0, stream>>>(
+        sa, sb, s_out, E, src_rows, dst_rows, K / 128, interleave);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream) {
     const int blocks = (int)std::min<size_t>((n / 8 + 255) / 256, (size_t)num_sms * 8);
     if (blocks == 0) return cudaSuccess;

@@ -36,9 +36,18 @@ namespace moe {
 
 namespace {
 
-template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR>
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR, bool MXW>
 struct Cfg {
-    static constexpr bool MX = (STAGE == 2) && FP8;
+    // Block-scaled MMA (kind::mxf8f6f4, one UE8M0 scale per 32 K elements of
+    // every row of A and B): stage 2 in FP8 (h carries per-32 scales; w2's
+    // are 1), and both stages with MX FP4 weights (MXW: e2m1 weights with
+    // their own per-32 scales; stage 1's activation scales are 1, the per-token
+    // scale is applied in the epilogue).
+    static constexpr bool MX = ((STAGE == 2) && FP8) || MXW;
+    static constexpr bool SFA_VAR = MX && STAGE == 2;  // A scales copied per stage (h's)
+    static constexpr bool SFB_VAR = MXW;               // B scales copied per stage (the weights')
+    static constexpr bool HAS_SFC = MX && !(SFA_VAR && SFB_VAR);  // a constant all-ones scale block
+    static_assert(!MXW || (FP8 && !PAIR), "MX FP4 weights: e4m3 activations, one-CTA tiles");
     // activation rows copied per stage: 128, or 32 when no m-tile holds more
     // than 32 rows in use (the MMA still reads 128 rows from the stage's
     // address; rows 32-127 then alias the next buffers and belong to padding
@@ -46,28 +55,38 @@ struct Cfg {
     static constexpr int A_BYTES = AR * 128;
     static_assert(AR == kBlockM || (AR == 32 && !PAIR), "activation rows per stage");
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // weight rows held by one CTA
-    static constexpr int B_BYTES = B_ROWS * 128;
-    static constexpr int SF_BYTES = MX ? 512 : 0;
+    static constexpr int B_BYTES = B_ROWS * 128;       // shared memory (e2m1: one byte per element)
+    // bytes a weight row brings in: MX FP4 rows are copied packed (two codes
+    // per byte) and spread to one code per byte in shared memory by the copy
+    static constexpr int B_ROW_TX = MXW ? 64 : 128;
+    static constexpr int SFA_BYTES = SFA_VAR ? 512 : 0;
+    static constexpr int SFB_BYTES = SFB_VAR ? 512 * (B_ROWS / 128) : 0;
     // bytes that complete one stage: both CTAs' copies count on the even CTA's barrier
-    static constexpr int TX_BYTES = (PAIR ? 2 : 1) * (A_BYTES + B_BYTES + SF_BYTES);
+    static constexpr int TX_BYTES = (PAIR ? 2 : 1) * (A_BYTES + B_ROWS * B_ROW_TX + SFA_BYTES + SFB_BYTES);
     static constexpr int KE = FP8 ? 128 : 64;  // K elements per 128-byte K tile
     static constexpr int MMA_M = PAIR ? 2 * kBlockM : kBlockM;
+    // TMEM columns: accumulators, then A scales (4 per stage, or 4 constant),
+    // then B scales (BN/32 per stage, or 8 constant)
     static constexpr int SFA_COL = NACC * BN;
-    static constexpr int SFB_COL = SFA_COL + 4 * NST;
-    static constexpr int COLS_USED = MX ? SFB_COL + 8 : NACC * BN;
+    static constexpr int SFA_NCOL = SFA_VAR ? 4 * NST : (MX ? 4 : 0);
+    static constexpr int SFB_COL = SFA_COL + SFA_NCOL;
+    static constexpr int SFB_NCOL = SFB_VAR ? (BN / 32) * NST : (MX ? 8 : 0);
+    static constexpr int COLS_USED = SFB_COL + SFB_NCOL;
     static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
                                    : COLS_USED <= 256 ? 256 : 512;
     static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
     static_assert(B_ROWS % kWBlockRows == 0 && BN <= 256, "BN: whole 128-row weight blocks");
-    // shared memory: A ring, B ring, SF ring, constant B scales, barriers
+    // shared memory: A ring, B ring, A-scale ring, B-scale ring, constant scales, barriers
     static constexpr int OFF_B = NST * A_BYTES;
-    static constexpr int OFF_SF = OFF_B + NST * B_BYTES;
-    static constexpr int OFF_SFB = OFF_SF + NST * SF_BYTES;
-    static constexpr int OFF_BAR = OFF_SFB + (MX ? 512 : 0);
+    static constexpr int OFF_SFA = OFF_B + NST * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + NST * SFA_BYTES;
+    static constexpr int OFF_SFC = OFF_SFB + NST * SFB_BYTES;
+    static constexpr int OFF_BAR = OFF_SFC + (HAS_SFC ? 512 : 0);
     static constexpr int NUM_BARS = 2 * NST + 5;
     static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;  // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
     static constexpr uint32_t IDESC = FP8 ? idesc_e4m3(MMA_M, BN) : idesc_bf16(MMA_M, BN);
+    static constexpr uint32_t B_FMT = MXW ? kFmtE2M1 : kFmtE4M3;  // B operand format of the block-scaled MMA
 };
 
 // SiLU(g) = g / (1 + e^-g) (glossary entry "SwiGLU").  The quotient uses the
@@ -85,12 +104,12 @@ __device__ __forceinline__ void decode_tile(int tile, int num_mt, int n_tiles, i
 
 }  // namespace
 
-template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR>
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR, bool MXW>
 __global__ void __launch_bounds__(192, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmSF,
                     const GemmArgs args) {
-    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR>;
+    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR, MXW>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -129,9 +148,11 @@ __global__ void __launch_bounds__(192, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (C::MX && warp >= 2) {
-        // constant UE8M0 scale 2^0 for every row of B (w2 carries fp32 per-channel scales instead)
-        reinterpret_cast<uint32_t*>(smem + C::OFF_SFB)[threadIdx.x - 64] = 0x7F7F7F7Fu;
+    if (C::HAS_SFC && warp >= 2) {
+        // constant UE8M0 scale 2^0 for every row of the operand without block
+        // scales (FP8 stage 2: B, w2 has fp32 per-channel scales instead; MX
+        // FP4 stage 1: A, the activations have one fp32 scale per token)
+        reinterpret_cast<uint32_t*>(smem + C::OFF_SFC)[threadIdx.x - 64] = 0x7F7F7F7Fu;
         fence_proxy_async_smem();
     }
     if (warp == 1) {
@@ -146,10 +167,8 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
         if constexpr (!PAIR && STAGE == 2) prefetch_tmap(&tmA32);
-        if constexpr (PAIR) {
-            prefetch_tmap(&tmB);
-            if constexpr (C::MX) prefetch_tmap(&tmSF);
-        }
+        if constexpr (PAIR || MXW) prefetch_tmap(&tmB);
+        if constexpr (PAIR && C::SFA_VAR) prefetch_tmap(&tmSF);
     }
     // Expert-major tile order: the first 128-row tile (and, for pairs, the
     // first pair of tiles) of each expert, from a scan of the per-expert row
@@ -311,13 +330,31 @@ __global__ void __launch_bounds__(192, 1)
     };
     auto stage_tx = [&](bool small, int q4) {
         return C::TX_BYTES - ((small && AR == kBlockM) ? (kBlockM - 32) * 128 : 0) -
-               (q4 >= 0 ? C::B_BYTES - 64 * 128 : 0);
+               (q4 >= 0 ? (C::B_ROWS - 64) * C::B_ROW_TX : 0);
     };
     const int b_nblk = args.rows_b / kWBlockRows;
     const uint64_t pol_b = args.b_evict_first ? policy_evict_first() : policy_evict_normal();
     // This CTA's weight blocks for unit (e, n) at K tile kt: the BN rows of the
     // tile, or this CTA's half of them in a pair.
     auto load_weights = [&](int stage, int e, int n, int kt, int q4) {
+        if constexpr (MXW) {
+            // MX FP4: packed e2m1 rows by TMA (64-row boxes, spread to one code
+            // per byte, 128-byte swizzle), then the B scale chunk of each
+            // 128-row block (512 bytes, already in the layout TMEM takes)
+            uint8_t* dst = smem + C::OFF_B + stage * C::B_BYTES;
+            const int row0 = e * args.rows_b + n * BN + (q4 >= 0 ? 64 * q4 : 0);
+            const int boxes = (q4 >= 0) ? 1 : C::B_ROWS / 64;
+            for (int j = 0; j < boxes; ++j)
+                tma_load_2d(dst + j * 64 * 128, &tmB, &full[stage], kt * C::KE, row0 + 64 * j, pol_b);
+            const int rb0 = (n * BN + (q4 >= 0 ? 64 * q4 : 0)) / kWBlockRows;
+            const int nchunks = (q4 >= 0) ? 1 : C::B_ROWS / kWBlockRows;
+            for (int j = 0; j < nchunks; ++j) {
+                const size_t chunk = ((size_t)e * b_nblk + rb0 + j) * args.k_tiles + kt;
+                bulk_load_hint(smem + C::OFF_SFB + stage * C::SFB_BYTES + 512 * j, args.b_sf + chunk * 512, 512,
+                               &full[stage], pol_b);
+            }
+            return;
+        }
         if (!PAIR && q4 >= 0) {  // 64 rows: one half of one 16 KB block (its pre-swizzled rows 0-63 or 64-127)
             const size_t blk = ((size_t)e * b_nblk + n * (BN / kWBlockRows) + (q4 >> 1)) * args.k_tiles + kt;
             bulk_load_hint(smem + C::OFF_B + stage * C::B_BYTES, args.b_blocks + blk * kWBlockBytes + (q4 & 1) * 8192,
@@ -415,15 +452,15 @@ __global__ void __launch_bounds__(192, 1)
                         const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
                         if (!skip)
                             tma_load_2d_pair(smem + stage * C::A_BYTES, &tmA, bar, kt * C::KE, m * kBlockM, pol_a);
-                        if constexpr (C::MX)
-                            tma_load_2d_pair(smem + C::OFF_SF + stage * C::SF_BYTES, &tmSF, bar, 0,
+                        if constexpr (C::SFA_VAR)
+                            tma_load_2d_pair(smem + C::OFF_SFA + stage * C::SFA_BYTES, &tmSF, bar, 0,
                                              (m * args.f_tiles + kt) * 4, pol_a);
                     } else {
                         if (!skip)
                             tma_load_2d(smem + stage * C::A_BYTES, (small || AR == 32) ? &tmA32 : &tmA, &full[stage],
                                         kt * C::KE, m * kBlockM, pol_a);
-                        if constexpr (C::MX)
-                            bulk_load(smem + C::OFF_SF + stage * C::SF_BYTES,
+                        if constexpr (C::SFA_VAR)
+                            bulk_load(smem + C::OFF_SFA + stage * C::SFA_BYTES,
                                       args.a_sf + ((size_t)m * args.f_tiles + kt) * 512, 512, &full[stage]);
                     }
                 }
@@ -465,12 +502,15 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0 && leader) {
-            if constexpr (C::MX) {
-                for (int c = 0; c < 8; c += 4) {
-                    if constexpr (PAIR)
-                        tmem_cp_32x128b_x4_pair(tmem_base + C::SFB_COL + c, sdesc_sf(smem_u32(smem + C::OFF_SFB)));
-                    else
-                        tmem_cp_32x128b_x4(tmem_base + C::SFB_COL + c, sdesc_sf(smem_u32(smem + C::OFF_SFB)));
+            if constexpr (C::HAS_SFC) {  // the constant scales, once
+                const uint64_t sd = sdesc_sf(smem_u32(smem + C::OFF_SFC));
+                if constexpr (!C::SFB_VAR) {
+                    for (int c = 0; c < 8; c += 4) {
+                        if constexpr (PAIR) tmem_cp_32x128b_x4_pair(tmem_base + C::SFB_COL + c, sd);
+                        else tmem_cp_32x128b_x4(tmem_base + C::SFB_COL + c, sd);
+                    }
+                } else {
+                    tmem_cp_32x128b_x4(tmem_base + C::SFA_COL, sd);
                 }
             }
             // arrival on a barrier of both CTAs (pair) or of this CTA
@@ -491,8 +531,12 @@ __global__ void __launch_bounds__(192, 1)
                 int m_, n_, split_, q4;
                 bool dup_;
                 unit_coords(u, m_, n_, split_, dup_, q4);
-                // a 64-row slice: the same MMAs with N = 64
+                // a 64-row slice: the same MMAs with N = 64 (and, with MX FP4
+                // weights, the B scales of that half of the 128-row block:
+                // TMEM column j of a block's scales holds its rows 32j..32j+31)
                 const uint32_t idesc = (q4 >= 0) ? ((C::IDESC & ~(0x3Fu << 17)) | ((64u >> 3) << 17)) : C::IDESC;
+                const int mma_n = (q4 >= 0) ? 64 : BN;
+                const uint32_t sfb_half = (MXW && q4 >= 0) ? 2u * (uint32_t)(q4 & 1) : 0u;
                 if (!wait(&tempty[acc], acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
@@ -504,26 +548,30 @@ __global__ void __launch_bounds__(192, 1)
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + stage * C::A_BYTES);
                     const uint32_t b_addr = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
-                    if constexpr (C::MX) {
-                        const uint64_t sd = sdesc_sf(smem_u32(smem + C::OFF_SF + stage * C::SF_BYTES));
+                    if constexpr (C::SFA_VAR) {
+                        const uint64_t sd = sdesc_sf(smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES));
                         if constexpr (PAIR)
                             tmem_cp_32x128b_x4_pair(tmem_base + C::SFA_COL + 4 * stage, sd);
                         else
                             tmem_cp_32x128b_x4(tmem_base + C::SFA_COL + 4 * stage, sd);
                     }
+                    if constexpr (C::SFB_VAR) {
+#pragma unroll
+                        for (int j = 0; j < C::B_ROWS / 128; ++j)
+                            tmem_cp_32x128b_x4(tmem_base + C::SFB_COL + (BN / 32) * stage + 4 * j,
+                                               sdesc_sf(smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES + 512 * j)));
+                    }
+                    const uint32_t sfa = tmem_base + C::SFA_COL + (C::SFA_VAR ? 4 * stage : 0);
+                    const uint32_t sfb = tmem_base + C::SFB_COL + (C::SFB_VAR ? (BN / 32) * stage : 0) + sfb_half;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t ad = sdesc_sw128(a_addr + ks * 32);
                         const uint64_t bd = sdesc_sw128(b_addr + ks * 32);
                         const uint32_t accum = (kk > 0 || ks > 0) ? 1u : 0u;
                         if constexpr (C::MX) {
-                            const uint32_t id = idesc_mxe4m3(C::MMA_M, BN, ks, ks);
-                            if constexpr (PAIR)
-                                mma_mxfp8_pair(d_tmem, ad, bd, id, tmem_base + C::SFA_COL + 4 * stage,
-                                               tmem_base + C::SFB_COL, accum);
-                            else
-                                mma_mxfp8(d_tmem, ad, bd, id, tmem_base + C::SFA_COL + 4 * stage,
-                                          tmem_base + C::SFB_COL, accum);
+                            const uint32_t id = idesc_mx(C::MMA_M, mma_n, C::B_FMT, ks, ks);
+                            if constexpr (PAIR) mma_mxfp8_pair(d_tmem, ad, bd, id, sfa, sfb, accum);
+                            else mma_mxfp8(d_tmem, ad, bd, id, sfa, sfb, accum);
                         } else if constexpr (FP8) {
                             if constexpr (PAIR) mma_fp8_pair(d_tmem, ad, bd, C::IDESC, accum);
                             else mma_fp8(d_tmem, ad, bd, idesc, accum);
@@ -607,12 +655,14 @@ __global__ void __launch_bounds__(192, 1)
                     const int hcol = n * (BN / 2) + g * 32;
                     float hv[32];
                     if constexpr (FP8) {
-                        // per-channel scales of the 32 gate and 32 up columns (64 contiguous floats)
+                        // per-channel scales of the 32 gate and 32 up columns (64 contiguous
+                        // floats); MX FP4 weights carry their scales inside the MMA
                         const float4* cs4 = reinterpret_cast<const float4*>(args.col_scale + (size_t)e * args.rows_b +
                                                                             n * BN + g * 64);
 #pragma unroll
                         for (int i4 = 0; i4 < 8; ++i4) {
-                            const float4 sg = __ldg(cs4 + i4), su = __ldg(cs4 + 8 + i4);
+                            const float4 one = make_float4(1.f, 1.f, 1.f, 1.f);
+                            const float4 sg = MXW ? one : __ldg(cs4 + i4), su = MXW ? one : __ldg(cs4 + 8 + i4);
                             const float sgv[4] = {sg.x, sg.y, sg.z, sg.w}, suv[4] = {su.x, su.y, su.z, su.w};
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
@@ -694,7 +744,7 @@ __global__ void __launch_bounds__(192, 1)
                     if (c0 + 64 == BN) release(acc);
                     if (t >= 0) {
                         const int col = n * BN + c0;
-                        const float* cs = FP8 ? args.col_scale + (size_t)e * args.rows_b + col : nullptr;
+                        const float* cs = (FP8 && !MXW) ? args.col_scale + (size_t)e * args.rows_b + col : nullptr;
 #pragma unroll
                         for (int i = 0; i < 64; i += 4) {
                             float4 v;
@@ -702,7 +752,7 @@ __global__ void __launch_bounds__(192, 1)
                             v.y = __uint_as_float(r[i + 1]) * wgt;
                             v.z = __uint_as_float(r[i + 2]) * wgt;
                             v.w = __uint_as_float(r[i + 3]) * wgt;
-                            if constexpr (FP8) {
+                            if constexpr (FP8 && !MXW) {
                                 const float4 sc = __ldg(reinterpret_cast<const float4*>(cs + i));
                                 v.x *= sc.x;
                                 v.y *= sc.y;
@@ -742,28 +792,28 @@ __global__ void __launch_bounds__(192, 1)
 
 namespace {
 
-template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR = kBlockM>
+template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR = kBlockM, bool MXW = false>
 cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, int grid, cudaStream_t stream) {
-    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR>;
-    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR, AR>;
+    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR, MXW>;
+    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR, AR, MXW>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     if constexpr (PAIR) {
         if (grid < 2 || grid % 2) return cudaErrorInvalidValue;
-        if (!maps.b || (C::MX && !maps.sf)) return cudaErrorInvalidValue;
+        if (!maps.b || (C::SFA_VAR && !maps.sf)) return cudaErrorInvalidValue;
         return launch_dependent_cluster(kern, dim3(grid), dim3(192), C::SMEM_BYTES, 2, stream, *maps.a, *maps.a,
-                                        *maps.b, C::MX ? *maps.sf : *maps.a, args);
+                                        *maps.b, C::SFA_VAR ? *maps.sf : *maps.a, args);
     } else {
-        if (!maps.a32) return cudaErrorInvalidValue;
-        return launch_dependent(kern, dim3(grid), dim3(192), C::SMEM_BYTES, stream, *maps.a, *maps.a32, *maps.a,
-                                *maps.a, args);
+        if (!maps.a32 || (MXW && !maps.b)) return cudaErrorInvalidValue;
+        return launch_dependent(kern, dim3(grid), dim3(192), C::SMEM_BYTES, stream, *maps.a, *maps.a32,
+                                MXW ? *maps.b : *maps.a, *maps.a, args);
     }
 }
 
 template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR = kBlockM>
 int max_pairs_one() {
-    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR>;
-    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR, AR>;
+    using C = Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR, false>;
+    auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR, AR, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return 0;
     return max_active_clusters(kern, 192, C::SMEM_BYTES, 2);
@@ -781,8 +831,15 @@ int gemm_block_n(int stage, bool fp8, int cfg) {
 // (weight streaming); cfg 2: one CTA, 128 x 256 tiles; cfg 3 (no m-tile with
 // more than 32 rows in use): 32 activation rows per stage, which leaves room
 // for deeper pipelines -- stage 1 on 128 x 256 tiles, stage 2 on 128 x 128.
+// MX FP4 weights (mxw) run on cfg 1 only: two 128-column accumulators leave
+// room in TMEM for the per-stage scales of both operands.
 cudaError_t launch_gemm(int stage, bool fp8, int cfg, const GemmMaps& maps, const GemmArgs& args, int grid,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, bool mxw) {
+    if (mxw) {
+        if (cfg != 1 || !fp8) return cudaErrorInvalidValue;
+        return stage == 1 ? launch_one<1, true, 128, 6, 2, false, kBlockM, true>(maps, args, grid, stream)
+                          : launch_one<2, true, 128, 6, 2, false, kBlockM, true>(maps, args, grid, stream);
+    }
     if (cfg == 3) {
         if (stage == 1)
             return fp8 ? launch_one<1, true, 256, 6, 2, false, 32>(maps, args, grid, stream)

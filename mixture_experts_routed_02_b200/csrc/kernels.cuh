@@ -109,8 +109,8 @@ struct PeerCounters {
 bool context_key(unsigned long long* key);
 // The host-side argument checks of a layer call (everything but the
 // workspace size), in the order the layer entry points apply them.
-int check_forward_args(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
-                       const float* s2, int T, int H, int F, int E, int k, int dtype, const void* out, const void* ws);
+int check_forward_args(const void* x, const float* logits, const void* w13, const void* s13, const void* w2,
+                       const void* s2, int T, int H, int F, int E, int k, int dtype, const void* out, const void* ws);
 
 // Host launchers (each defined next to its kernel).
 cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOutputs& o, cudaStream_t stream);
@@ -131,6 +131,11 @@ constexpr int kWBlockBytes = kWBlockRows * 128;
 cudaError_t launch_preshuffle(const uint8_t* a, const uint8_t* b, uint8_t* dst, int E, int src_rows, int dst_rows,
                               int row_bytes, bool interleave, cudaStream_t stream);
 cudaError_t launch_interleave_scales(const float* s1, const float* s3, float* s13, int E, int F, cudaStream_t stream);
+// MX FP4 weights: packed e2m1 rows (interleaved w1/w3 rows for the first
+// GEMM) and their block scales as 512-byte TMEM-order chunks.
+cudaError_t launch_mx_prepare(const uint8_t* a, const uint8_t* b, const uint8_t* sa, const uint8_t* sb,
+                              uint8_t* w_out, uint8_t* s_out, int E, int src_rows, int dst_rows, int K,
+                              bool interleave, cudaStream_t stream);
 
 // Arguments of the grouped GEMM (both stages).
 struct GemmArgs {
@@ -143,6 +148,7 @@ struct GemmArgs {
     const uint8_t* b_blocks;  // weights in the blocked layout: [E][rows_b/128][k_tiles][16 KB]
     int b_evict_first;        // stream weights with the L2 evict-first hint (each tile read once)
     const uint8_t* a_sf;      // stage 2, FP8: UE8M0 scales of h, tiled
+    const uint8_t* b_sf;      // MX FP4 weights: UE8M0 scales, 512-byte chunks [E][rows_b/128][k_tiles]
     void* out;                // stage 1: h [S, F]; stage 2: out32 [T, H]
     uint8_t* out_sf;          // stage 1, FP8: UE8M0 scales of h, tiled
     int rows_b;               // rows of B per expert: 2F (stage 1) or H (stage 2)
@@ -170,6 +176,8 @@ struct GemmArgs {
 };
 
 
+// (With MX FP4 weights, b is the packed e2m1 weight rows, read with 64-row
+// boxes and spread to one code per byte.)
 // Tensor maps of one GEMM launch, all with 128-byte swizzle for the
 // activations.  Stage 1: a = the token rows (xq or x) with one-row boxes, read
 // by four-row TMA gathers.  Stage 2: a = rows of h (128-row boxes) and a32 =
@@ -188,7 +196,7 @@ struct GemmMaps {
 //      1 = one CTA, 128 x 128 tiles (weight streaming);
 //      2 = one CTA, 128 x 256 tiles.
 cudaError_t launch_gemm(int stage, bool fp8, int cfg, const GemmMaps& maps, const GemmArgs& args, int grid,
-                        cudaStream_t stream);
+                        cudaStream_t stream, bool mxw = false);
 int gemm_block_n(int stage, bool fp8, int cfg);
 // Resident clusters of the pair kernel of a stage (0 if it cannot run).
 int gemm_max_pairs(int stage, bool fp8);

@@ -172,13 +172,16 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 bool dims_ok(int T, int H, int F, int E, int k, int dtype) {
     return T >= 0 && H > 0 && F > 0 && E >= 1 && E <= kMaxExperts && k >= 1 && k <= E && k <= kMaxTopK &&
-           (dtype == MOE_BF16 || dtype == MOE_FP8_E4M3);
+           (dtype == MOE_BF16 || dtype == MOE_FP8_E4M3 || dtype == MOE_MXFP4);
 }
+
+// e4m3 activations and h (FP8 and MX FP4 weights) or bf16 throughout
+bool e4m3_acts(int dtype) { return dtype != MOE_BF16; }
 
 Layout make_layout(int T, int H, int F, int E, int k, int dtype) {
     Layout L{};
     const size_t A = (size_t)T * k;
-    const size_t eb = (dtype == MOE_FP8_E4M3) ? 1 : 2;
+    const size_t eb = e4m3_acts(dtype) ? 1 : 2;
     L.A = (int)A;
     L.MT_max = (int)((A + kBlockM - 1) / kBlockM) + E;  // sum over experts of ceil(n_e / 128)
     L.S_max = L.MT_max * kBlockM;
@@ -191,10 +194,10 @@ Layout make_layout(int T, int H, int F, int E, int k, int dtype) {
     sz[MOE_WS_PERM] = 4 * A;
     sz[MOE_WS_INV_PERM] = 4 * A;
     sz[MOE_WS_SLOT_OF] = 4 * A;
-    sz[MOE_WS_XS] = (dtype == MOE_FP8_E4M3) ? (size_t)T * H : 0;  // per-token e4m3 rows (BF16 reads x itself)
-    sz[MOE_WS_SX] = (dtype == MOE_FP8_E4M3) ? 4 * (size_t)T : 0;
+    sz[MOE_WS_XS] = e4m3_acts(dtype) ? (size_t)T * H : 0;  // per-token e4m3 rows (BF16 reads x itself)
+    sz[MOE_WS_SX] = e4m3_acts(dtype) ? 4 * (size_t)T : 0;
     sz[MOE_WS_H] = S * act_pitch((long)F * eb);
-    sz[MOE_WS_H_SF] = (dtype == MOE_FP8_E4M3) ? (size_t)L.MT_max * (F / 128) * 512 : 0;
+    sz[MOE_WS_H_SF] = e4m3_acts(dtype) ? (size_t)L.MT_max * (F / 128) * 512 : 0;
     sz[MOE_WS_OUT32] = 4 * (size_t)T * H;
     sz[MOE_WS_NUM_MTILES] = 4;
     sz[MOE_WS_SLOT_ASSIGN] = 4 * S;
@@ -244,6 +247,23 @@ bool make_map(CUtensorMap* map, const void* base, size_t rows, size_t cols, size
                           const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Map of packed MX FP4 weight rows [rows, cols] (two e2m1 codes per byte, row
+// pitch cols/2 bytes) whose copies spread each code to a byte of shared
+// memory (the 4-bit operand form of the block-scaled MMA), 128 codes by
+// box_rows rows per copy, 128-byte swizzle.
+bool make_map_fp4(CUtensorMap* map, const void* base, size_t rows, size_t cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(cols / 2)};
+    const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -316,10 +336,10 @@ void store_maps(const MapKey& key, const MapSet& maps) {
 // The host-side checks of a layer call, in the order both layer entry points
 // apply them (dimensions, null pointers, supported shapes, alignment); the
 // workspace size is checked after them.
-int check_forward_args(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
-                       const float* s2, int T, int H, int F, int E, int k, int dtype, const void* out, const void* ws) {
+int check_forward_args(const void* x, const float* logits, const void* w13, const void* s13, const void* w2,
+                       const void* s2, int T, int H, int F, int E, int k, int dtype, const void* out, const void* ws) {
     if (!dims_ok(T, H, F, E, k, dtype)) return MOE_ERR_INVALID_ARG;
-    const bool fp8 = dtype == MOE_FP8_E4M3;
+    const bool fp8 = e4m3_acts(dtype);
     if (!w13 || !w2 || !ws || (fp8 && (!s13 || !s2))) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !logits || !out)) return MOE_ERR_INVALID_ARG;
     if (H % 128 || F % 128) return MOE_ERR_UNSUPPORTED;
@@ -408,6 +428,29 @@ int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const f
     return MOE_OK;
 }
 
+int moe_prepare_weights_mx(const void* w1, const void* w3, const void* s1, const void* s3, const void* w2,
+                           const void* s2, void* w13_out, void* s13_out, void* w2_out, void* s2_out, int E, int F,
+                           int H, void* stream) {
+    if (!w1 || !w3 || !s1 || !s3 || !w2 || !s2 || !w13_out || !s13_out || !w2_out || !s2_out || E < 1 ||
+        E > kMaxExperts || F <= 0 || H <= 0)
+        return MOE_ERR_INVALID_ARG;
+    if (F % 128 || H % 128) return MOE_ERR_UNSUPPORTED;
+    const void* ptrs[] = {w1, w3, s1, s3, w2, s2, w13_out, s13_out, w2_out, s2_out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_ALIGNMENT;
+    // the packed rows are read by TMA: 32-byte aligned bases
+    if ((reinterpret_cast<uintptr_t>(w13_out) | reinterpret_cast<uintptr_t>(w2_out)) & 31u) return MOE_ERR_ALIGNMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    auto u8 = [](const void* p) { return static_cast<const uint8_t*>(p); };
+    if (launch_mx_prepare(u8(w1), u8(w3), u8(s1), u8(s3), static_cast<uint8_t*>(w13_out),
+                          static_cast<uint8_t*>(s13_out), E, F, 2 * F, H, true, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (launch_mx_prepare(u8(w2), nullptr, u8(s2), nullptr, static_cast<uint8_t*>(w2_out),
+                          static_cast<uint8_t*>(s2_out), E, H, H, F, false, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w, int32_t* counts,
               int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes, void* stream) {
     (void)ws;
@@ -434,12 +477,13 @@ struct Dff {
 // The layer call: the whole layer (dff == nullptr), or one rank's part of the
 // d_ff-sharded layer (its GEMMs on its d_ff slice, the scatter-add into the
 // owners' combine rows, and the signal to every rank; no rounding).
-int forward_impl(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
-                 const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws, size_t ws_bytes,
+int forward_impl(const void* x, const float* logits, const void* w13, const void* s13, const void* w2,
+                 const void* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws, size_t ws_bytes,
                  void* stream, const Dff* dff) {
     const int rc_args = check_forward_args(x, logits, w13, s13, w2, s2, T, H, F, E, k, dtype, dff ? ws : out, ws);
     if (rc_args != MOE_OK) return rc_args;
-    const bool fp8 = dtype == MOE_FP8_E4M3;
+    const bool fp8 = e4m3_acts(dtype);          // e4m3 activations and h
+    const bool mxw = dtype == MOE_MXFP4;        // MX FP4 weights with block scales
     const Layout L = make_layout(T, H, F, E, k, dtype);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     const int opt_path = g_opt_path.load();  // read once per call
@@ -479,6 +523,7 @@ int forward_impl(const void* x, const float* logits, const void* w13, const floa
     } else {
         cfg1 = cfg2 = opt_path - 1;
     }
+    if (mxw) cfg1 = cfg2 = 1;  // MX FP4 weights: 128 x 128 one-CTA tiles (room in TMEM for both operands' scales)
     if ((2 * F) % gemm_block_n(1, fp8, cfg1)) cfg1 = 1;
     if (H % gemm_block_n(2, fp8, cfg2)) cfg2 = 1;
     if (cfg1 == 0 && max_pairs(1, fp8) < 1) cfg1 = 2;
@@ -497,6 +542,10 @@ int forward_impl(const void* x, const float* logits, const void* w13, const floa
             !make_map(&ms.ta2, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, kBlockM) ||
             !make_map(&ms.ta2s, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, 32))
             return MOE_ERR_CUDA;
+        if (mxw) {
+            if (!make_map_fp4(&ms.tb1, w13, (size_t)E * 2 * F, H, 64) || !make_map_fp4(&ms.tb2, w2, (size_t)E * H, F, 64))
+                return MOE_ERR_CUDA;
+        }
         if (cfg1 == 0 && !make_map_rows(&ms.tb1, w13, (size_t)E * (2 * F) * (H * eb / 128), kWBlockRows))
             return MOE_ERR_CUDA;
         if (cfg2 == 0 && !make_map_rows(&ms.tb2, w2, (size_t)E * H * (F * eb / 128), kWBlockRows))
@@ -505,8 +554,9 @@ int forward_impl(const void* x, const float* logits, const void* w13, const floa
             return MOE_ERR_CUDA;
         store_maps(mkey, ms);
     }
-    const GemmMaps maps1{&ms.tg1, &ms.tg1, cfg1 == 0 ? &ms.tb1 : nullptr, nullptr};
-    const GemmMaps maps2{&ms.ta2, &ms.ta2s, cfg2 == 0 ? &ms.tb2 : nullptr, (cfg2 == 0 && fp8) ? &ms.tsf2 : nullptr};
+    const GemmMaps maps1{&ms.tg1, &ms.tg1, (cfg1 == 0 || mxw) ? &ms.tb1 : nullptr, nullptr};
+    const GemmMaps maps2{&ms.ta2, &ms.ta2s, (cfg2 == 0 || mxw) ? &ms.tb2 : nullptr,
+                         (cfg2 == 0 && fp8) ? &ms.tsf2 : nullptr};
     // grid: one CTA per SM at most; pairs: whole clusters that can be resident
     auto grid_for = [&](int stage, int c, long units_per_mtile) {
         if (c == 0) {
@@ -555,7 +605,8 @@ int forward_impl(const void* x, const float* logits, const void* w13, const floa
     g1.mtile_expert = o.mtile_expert;
     g1.slot_assign = o.slot_assign;
     g1.row_scale = sx;
-    g1.col_scale = fp8 ? s13 : nullptr;
+    g1.col_scale = (fp8 && !mxw) ? static_cast<const float*>(s13) : nullptr;
+    g1.b_sf = mxw ? static_cast<const uint8_t*>(s13) : nullptr;
     g1.b_blocks = static_cast<const uint8_t*>(w13);
     g1.b_evict_first = small_batch ? 1 : 0;  // one m-tile per expert: each weight block is read once
     g1.out = reg(MOE_WS_H);
@@ -577,7 +628,7 @@ int forward_impl(const void* x, const float* logits, const void* w13, const floa
     g1.group_m = (cfg1 != 1) ? 1 : 0;
     {
         ProfScope ps(MOE_KERNEL_STAGE1, st);
-        if (launch_gemm(1, fp8, cfg1, maps1, g1, grid_for(1, cfg1, g1.n_tiles), st) != cudaSuccess)
+        if (launch_gemm(1, fp8, cfg1, maps1, g1, grid_for(1, cfg1, g1.n_tiles), st, mxw) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 
@@ -586,7 +637,8 @@ int forward_impl(const void* x, const float* logits, const void* w13, const floa
     g2.row_scale = nullptr;
     g2.test_stall = 0;
     g2.group_m = (cfg2 == 0 || cfg2 == 2) ? 1 : 0;
-    g2.col_scale = fp8 ? s2 : nullptr;
+    g2.col_scale = (fp8 && !mxw) ? static_cast<const float*>(s2) : nullptr;
+    g2.b_sf = mxw ? static_cast<const uint8_t*>(s2) : nullptr;
     g2.topk_w = o.topk_w;
     g2.a_sf = fp8 ? reg(MOE_WS_H_SF) : nullptr;
     g2.b_blocks = static_cast<const uint8_t*>(w2);
@@ -610,7 +662,8 @@ int forward_impl(const void* x, const float* logits, const void* w13, const floa
     }
     {
         ProfScope ps(MOE_KERNEL_STAGE2, st);
-        if (launch_gemm(2, fp8, cfg2, maps2, g2, grid_for(2, cfg2, (long)g2.n_tiles * g2.splits), st) != cudaSuccess)
+        if (launch_gemm(2, fp8, cfg2, maps2, g2, grid_for(2, cfg2, (long)g2.n_tiles * g2.splits), st, mxw) !=
+            cudaSuccess)
             return MOE_ERR_CUDA;
     }
     if (dff) return launch_status(launch_dff_signal(counters, dff->n_ranks, st));
@@ -624,14 +677,14 @@ int forward_impl(const void* x, const float* logits, const void* w13, const floa
 
 extern "C" {
 
-int moe_ffn_forward(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
-                    const float* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
+int moe_ffn_forward(const void* x, const float* logits, const void* w13, const void* s13, const void* w2,
+                    const void* s2, int T, int H, int F, int E, int k, int dtype, void* out, void* ws,
                     size_t ws_bytes, void* stream) {
     return forward_impl(x, logits, w13, s13, w2, s2, T, H, F, E, k, dtype, out, ws, ws_bytes, stream, nullptr);
 }
 
-int moe_ffn_forward_dff(const void* x, const float* logits, const void* w13, const float* s13, const void* w2,
-                        const float* s2, int T, int H, int F_shard, int E, int k, int dtype, int n_ranks, int rank,
+int moe_ffn_forward_dff(const void* x, const float* logits, const void* w13, const void* s13, const void* w2,
+                        const void* s2, int T, int H, int F_shard, int E, int k, int dtype, int n_ranks, int rank,
                         float* const* peer_out32, unsigned int* const* peer_counter, void* ws, size_t ws_bytes,
                         void* stream) {
     if (n_ranks < 1 || n_ranks > kMaxRanks || rank < 0 || rank >= n_ranks || !peer_out32 || !peer_counter)

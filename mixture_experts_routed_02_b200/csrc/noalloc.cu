@@ -66,8 +66,8 @@ int static_workspace(void** ptr) {
 
 extern "C" size_t moe_static_workspace_bytes(void) { return moe::kStaticWorkspaceBytes; }
 
-extern "C" int moe_ffn_forward_static(const void* x, const float* logits, const void* w13, const float* s13,
-                                      const void* w2, const float* s2, int T, int H, int F, int E, int k, int dtype,
+extern "C" int moe_ffn_forward_static(const void* x, const float* logits, const void* w13, const void* s13,
+                                      const void* w2, const void* s2, int T, int H, int F, int E, int k, int dtype,
                                       void* out, void* stream) {
     // the checks of moe_ffn_forward first, in its order (the workspace pointer
     // is the built-in array, never null), then the size against the array

@@ -385,10 +385,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
     return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-// Block-scaled e4m3 with UE8M0 scales: B scale-factor id at bits 4-5, scale
-// format (1 = UE8M0) at bit 23, A scale-factor id at bits 29-30.
-__host__ __device__ constexpr uint32_t idesc_mxe4m3(int M, int N, uint32_t a_sf_id, uint32_t b_sf_id) {
-    return (b_sf_id << 4) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) | (a_sf_id << 29);
+// Block-scaled kind::mxf8f6f4 with UE8M0 scales, A e4m3 and B of format
+// b_fmt (kFmtE4M3 or kFmtE2M1, at bits 10-12): B scale-factor id at bits
+// 4-5, scale format (1 = UE8M0) at bit 23, A scale-factor id at bits 29-30.
+constexpr uint32_t kFmtE4M3 = 0;
+constexpr uint32_t kFmtE2M1 = 5;
+__host__ __device__ constexpr uint32_t idesc_mx(int M, int N, uint32_t b_fmt, uint32_t a_sf_id, uint32_t b_sf_id) {
+    return (b_sf_id << 4) | (b_fmt << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) |
+           (a_sf_id << 29);
 }
 
 }  // namespace moe

@@ -40,7 +40,12 @@ def to_device(case, device="cuda"):
     for key in ("x", "logits", "w1", "w3", "w2", "s1", "s3", "s2"):
         v = case.get(key)
         d[key] = None if v is None else v.to(device)
-    d["w13"], d["s13"], d["w2p"] = moe.prepare_weights(d["w1"], d["w3"], d["s1"], d["s3"], d["w2"])
+    if case["dtype"] == "mxfp4":
+        d["w13"], d["s13"], d["w2p"], d["s2p"] = moe.prepare_weights_mx(d["w1"], d["w3"], d["s1"], d["s3"], d["w2"],
+                                                                         d["s2"])
+    else:
+        d["w13"], d["s13"], d["w2p"] = moe.prepare_weights(d["w1"], d["w3"], d["s1"], d["s3"], d["w2"])
+        d["s2p"] = d["s2"]
     for key in ("T", "H", "F", "E", "k", "dtype"):
         d[key] = case[key]
     return d
@@ -50,8 +55,8 @@ def run_layer(dcase, ws=None):
     import mixture_experts_routed_02_b200 as moe
     if ws is None:
         ws = moe.workspace(dcase["T"], dcase["H"], dcase["F"], dcase["E"], dcase["k"], dcase["dtype"])
-    out = moe.ffn_forward(dcase["x"], dcase["logits"], dcase["w13"], dcase["s13"], dcase["w2p"], dcase["s2"],
-                          dcase["k"], dcase["F"], dcase["dtype"] == "fp8", ws=ws)
+    out = moe.ffn_forward(dcase["x"], dcase["logits"], dcase["w13"], dcase["s13"], dcase["w2p"], dcase["s2p"],
+                          dcase["k"], dcase["F"], dcase["dtype"], ws=ws)
     st = moe.moe_get_status(None)
     assert st == 0, f"device status {moe.STATUS_NAMES.get(st, st)}"
     return out, ws
@@ -84,6 +89,20 @@ ABS_FLOOR = 2.0 ** -14    # ... plus this fraction of the row's rms: g and u are
                           # fp32 accumulation leaves an absolute error that is large relative to h
                           # wherever g or u cancels to nearly zero
 MAX_FLIP_FRACTION = 1e-2  # flips allowed per h row (a real defect changes most of a row)
+
+
+def w2_columns(nc, dtype, e, cols):
+    """Dequantised columns `cols` (d_ff indices) of expert e's w2 [H, len(cols)],
+    from the oracle's number formats."""
+    cols = np.asarray(cols)
+    if dtype == "fp8":
+        return _e4m3_values()[nc["w2"][e][:, cols]] * nc["s2"][e][:, None].astype(np.float64)
+    if dtype == "bf16":
+        return bf16_bits_to_f64(nc["w2"][e][:, cols])
+    byte = nc["w2"][e][:, cols // 2]
+    code = np.where(cols % 2 == 1, byte >> 4, byte & 15)
+    vals = np.array([oracle.e2m1_to_double(c) for c in range(16)])[code]
+    return vals * np.array([oracle.ue8m0_to_double(v) for v in range(256)])[nc["s2"][e][:, cols // 32]]
 
 
 def _e4m3_values():
@@ -138,7 +157,7 @@ def verify_layer(moe, ws, out, case, tokens=None, what=""):
     against the oracle.  Returns a dict of statistics."""
     nc = moe_inputs.to_numpy(case)
     T, F, k = case["T"], case["F"], case["k"]
-    fp8 = case["dtype"] == "fp8"
+    fp8 = case["dtype"] in ("fp8", "mxfp4")  # h is e4m3 with block scales
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     ref = oracle.moe_ffn_tokens(nc, tokens.astype(np.int32), want_h=True)
     r = oracle.route(nc["logits"], k)
@@ -175,10 +194,7 @@ def verify_layer(moe, ws, out, case, tokens=None, what=""):
         t_i, j = divmod(q, k)
         e = int(r["ids"][tokens[t_i], j])
         wgt = float(r["w"][tokens[t_i], j])
-        if fp8:
-            col = _e4m3_values()[nc["w2"][e][:, d]] * nc["s2"][e][:, None].astype(np.float64)
-        else:
-            col = bf16_bits_to_f64(nc["w2"][e][:, d])
+        col = w2_columns(nc, case["dtype"], e, d)
         allow[t_i] += wgt * (np.abs(col) @ np.abs(gh[q, d] - rh[q, d]))
     gpu = out.float().double().cpu().numpy()[tokens]
     refv = bf16_bits_to_f64(ref["out"])

@@ -116,3 +116,17 @@ def test_tensor_bound_roofline_uses_fp8_peak_from_bf16():
     d = bench.roofline(dict(spec, T=16), bench.algorithmic(dict(spec, T=16), [4] * 8), "stage1_w13_swiglu", 0.15,
                        5.0, peaks, "measured", "decode")
     assert d["bound"] == "hbm" and d["unit"] == "GB/s"
+
+
+def test_mxfp4_weight_bytes():
+    """MX FP4 expert weights: half a byte per code plus one exponent byte per
+    32 codes -- 0.53125 bytes per weight, against 1 (+ channel scales) for e4m3."""
+    H, F = 4096, 14336
+    assert bench.weight_bytes("mxfp4", 3 * H, F) == 3 * H * F * 17 // 32
+    assert bench.weight_bytes("fp8", 3 * H, F) == 3 * H * F + 4 * 3 * H
+    assert bench.weight_bytes("bf16", 3 * H, F) == 6 * H * F
+    spec = dict(DECODE, dtype="mxfp4")
+    w = bench.algorithmic(spec, [4] * 8)
+    fp8 = bench.algorithmic(DECODE, [4] * 8)
+    assert 0.5 < w["layer_bytes"] / fp8["layer_bytes"] < 0.55
+    assert w["layer_flops"] == fp8["layer_flops"]

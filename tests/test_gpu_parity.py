@@ -124,13 +124,68 @@ def test_layer_small(moe, p, path):
     perm = moe.ws_view(ws, T, H, F, E, k, dtc, "perm", torch.int32)[:A].cpu().numpy()
     np.testing.assert_array_equal(ids, r["ids"].reshape(-1))
     np.testing.assert_array_equal(perm, r["perm"])
-    if dt == "fp8":
+    if dt in ("fp8", "mxfp4"):
         # R0: per-token e4m3 codes and scales, bitwise
         xq_ref, sx_ref = oracle.quant_x(nc["x"])
         xs = moe.ws_view(ws, T, H, F, E, k, dtc, "xs").cpu().numpy().reshape(T, H)
         sx = moe.ws_view(ws, T, H, F, E, k, dtc, "sx", torch.float32).cpu().numpy()
         np.testing.assert_array_equal(xs, xq_ref)
         np.testing.assert_array_equal(sx.view(np.uint32), sx_ref.view(np.uint32))
+
+
+MXFP4 = [
+    # (T, H, F, E, k, seed, skew): MX FP4 weights run on 128 x 128 one-CTA tiles
+    (64, 256, 512, 8, 2, 30, False),
+    (1, 256, 512, 8, 2, 31, False),
+    (16, 256, 512, 8, 2, 32, False),       # decode-shaped: 32 activation rows per stage
+    (200, 384, 640, 8, 2, 33, False),      # several m-tiles, ragged tails, odd multiples of 128
+    (300, 256, 512, 8, 2, 34, True),       # skewed: big and empty experts
+    (37, 128, 256, 1, 1, 35, False),       # E = 1, k = 1
+    (16, 256, 2560, 8, 2, 36, False),      # last wave cut into 64-row slices (half-block scales)
+]
+
+
+@pytest.mark.parametrize("p", MXFP4, ids=lambda p: f"T{p[0]}_H{p[1]}_F{p[2]}_E{p[3]}_k{p[4]}" + ("_skew" if p[6] else ""))
+def test_layer_small_mxfp4(moe, p):
+    T, H, F, E, k, seed, skew = p
+    case = small_case(T, H, F, E, k, "mxfp4", seed, skew)
+    nc = moe_inputs.to_numpy(case)
+    out, ws = run_layer(to_device(case))
+    verify_layer(moe, ws, out, case, what=f"mxfp4 layer T={T} H={H} F={F}")
+    xq_ref, sx_ref = oracle.quant_x(nc["x"])
+    xs = moe.ws_view(ws, T, H, F, E, k, moe.MOE_MXFP4, "xs").cpu().numpy().reshape(T, H)
+    np.testing.assert_array_equal(xs, xq_ref)
+
+
+def test_prepare_weights_mx_layout(moe):
+    """moe_prepare_weights_mx: w13 rows interleaved in groups of 32 (w1 then
+    w3), still packed; the scales regrouped into 512-byte chunks per (expert,
+    128-row block, 128-column block), byte (r%32)*16 + (r/32)*4 + b."""
+    E, F, H = 2, 256, 384
+    case = small_case(3, H, F, E, 2, "mxfp4", 37)
+    d = to_device(case)
+    w13 = d["w13"].cpu().numpy().reshape(E, 2 * F, H // 2)
+    w1, w3 = case["w1"].numpy(), case["w3"].numpy()
+    src_rows = lambda R: (w3 if R % 64 >= 32 else w1, 32 * (R // 64) + R % 32)  # noqa: E731
+    for R in range(2 * F):
+        src, r = src_rows(R)
+        np.testing.assert_array_equal(w13[:, R], src[:, r])
+    np.testing.assert_array_equal(d["w2p"].cpu().numpy().reshape(E, H, F // 2), case["w2"].numpy())
+    s13 = d["s13"].cpu().numpy().reshape(E, 2 * F // 128, H // 128, 512)
+    s1, s3 = case["s1"].numpy(), case["s3"].numpy()
+    for R in range(2 * F):
+        src, r = (s3 if R % 64 >= 32 else s1), 32 * (R // 64) + R % 32
+        nb, rr = divmod(R, 128)
+        for kt in range(H // 128):
+            for b in range(4):
+                assert s13[:, nb, kt, (rr % 32) * 16 + (rr // 32) * 4 + b].tolist() == src[:, r, 4 * kt + b].tolist()
+    s2p = d["s2p"].cpu().numpy().reshape(E, H // 128, F // 128, 512)
+    s2 = case["s2"].numpy()
+    for R in range(0, H, 7):
+        nb, rr = divmod(R, 128)
+        for kt in range(F // 128):
+            np.testing.assert_array_equal(s2p[:, nb, kt, (rr % 32) * 16 + (rr // 32) * 4 + np.arange(4)],
+                                          s2[:, R, 4 * kt:4 * kt + 4])
 
 
 def _expected_layout(r, T, E, k):
@@ -295,7 +350,8 @@ def test_host_errors(moe):
 
 # ---------------------------------------------------------------- full-size workloads, sampled tokens
 
-FULL = ["decode", "prefill", "skewed", "sweep_T1", "sweep_T128", "sweep_T1024", "sweep_T16384"]
+FULL = ["decode", "prefill", "skewed", "sweep_T1", "sweep_T128", "sweep_T1024", "sweep_T16384", "decode_mxfp4",
+        "prefill_mxfp4"]
 
 
 def _tokens_per_mtile(r, k, T, rng):
