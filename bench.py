@@ -58,7 +58,52 @@ def parse(argv=None):
     p.add_argument("--sub-cpu-sample-seconds", type=float, default=4.0, help="oracle sample of each other workload")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true", help="skip the end-to-end pass (profiling runs)")
+    p.add_argument("--fp8-peak-probe", action="store_true",
+                   help="measure the dense e4m3 GEMM rate of torch._scaled_mm (context for the FP8 roofline) and exit")
     return p.parse_args(argv)
+
+
+def fp8_peak_probe(n=8192, burst_reps=10, sustained_s=3.0):
+    """Dense e4m3 x e4m3 -> bf16 GEMM rate of the library GEMM (torch._scaled_mm,
+    per-tensor scales) at n^3: best of `burst_reps` single calls (burst) and
+    the average over a loop of about `sustained_s` seconds (under the power
+    cap), CUDA events on the current stream, clocks sampled meanwhile.  A
+    reference figure for the FP8 fractions, beside bf16 x 2."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device())
+    g = torch.Generator(device=dev).manual_seed(0)
+    a = (torch.randn(n, n, device=dev, generator=g) * 0.5).to(torch.float8_e4m3fn)
+    b = (torch.randn(n, n, device=dev, generator=g) * 0.5).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=dev)
+    mm = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)  # noqa: E731
+    for _ in range(5):
+        mm()
+    torch.cuda.synchronize()
+    flop = 2.0 * n ** 3
+    best = float("inf")
+    for _ in range(burst_reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    reps = max(10, int(sustained_s * 1e3 / best))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        mm()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    sust = e0.elapsed_time(e1) / reps
+    return {"probe": "torch._scaled_mm e4m3 x e4m3 -> bf16, per-tensor scales", "n": n,
+            "burst_tflops": flop / (best / 1e3) / 1e12, "burst_ms": best,
+            "sustained_tflops": flop / (sust / 1e3) / 1e12, "sustained_ms": sust, "sustained_reps": reps,
+            "clocks": clk}
 
 
 def config_names(arg):
@@ -564,6 +609,11 @@ def main(argv=None):
     import moe_inputs
     import torch
     import torch.distributed as dist
+    if args.fp8_peak_probe:
+        torch.cuda.set_device(local_rank)
+        if rank == 0:
+            print(json.dumps(fp8_peak_probe()), flush=True)
+        return 0
     names = config_names(args.config)
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
