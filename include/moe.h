@@ -101,7 +101,7 @@ int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const f
  *   w2       device, [E,H,F/2] bytes; s2 device, [E,H,F/32] bytes (blocks along d_ff)
  *   w13_out  device, E*2F*H/2 bytes: w1/w3 rows interleaved in groups of 32 as
  *            for moe_prepare_weights, still packed, row-major (read by TMA,
- *            which spreads the codes to one per byte in shared memory);
+ *            which puts every 16 codes into 16 bytes of shared memory);
  *            32-byte aligned
  *   s13_out  device, E*2F*H/32 bytes: the scales of those rows regrouped into
  *            512-byte chunks per (expert, 128-row block, 128-column block),

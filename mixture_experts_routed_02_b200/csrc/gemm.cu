@@ -57,7 +57,8 @@ struct Cfg {
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // weight rows held by one CTA
     static constexpr int B_BYTES = B_ROWS * 128;       // shared memory (e2m1: one byte per element)
     // bytes a weight row brings in: MX FP4 rows are copied packed (two codes
-    // per byte) and spread to one code per byte in shared memory by the copy
+    // per byte); in shared memory every 16 codes take 16 bytes (8 bytes of
+    // codes, 8 of padding: the 4-bit operand form of the block-scaled MMA)
     static constexpr int B_ROW_TX = MXW ? 64 : 128;
     static constexpr int SFA_BYTES = SFA_VAR ? 512 : 0;
     static constexpr int SFB_BYTES = SFB_VAR ? 512 * (B_ROWS / 128) : 0;
@@ -338,8 +339,8 @@ __global__ void __launch_bounds__(192, 1)
     // tile, or this CTA's half of them in a pair.
     auto load_weights = [&](int stage, int e, int n, int kt, int q4) {
         if constexpr (MXW) {
-            // MX FP4: packed e2m1 rows by TMA (64-row boxes, spread to one code
-            // per byte, 128-byte swizzle), then the B scale chunk of each
+            // MX FP4: packed e2m1 rows by TMA (64-row boxes, 16 codes per 16
+            // bytes of shared memory, 128-byte swizzle), then the B scale chunk of each
             // 128-row block (512 bytes, already in the layout TMEM takes)
             uint8_t* dst = smem + C::OFF_B + stage * C::B_BYTES;
             const int row0 = e * args.rows_b + n * BN + (q4 >= 0 ? 64 * q4 : 0);

@@ -177,7 +177,7 @@ struct GemmArgs {
 
 
 // (With MX FP4 weights, b is the packed e2m1 weight rows, read with 64-row
-// boxes and spread to one code per byte.)
+// boxes, every 16 codes into 16 bytes of shared memory.)
 // Tensor maps of one GEMM launch, all with 128-byte swizzle for the
 // activations.  Stage 1: a = the token rows (xq or x) with one-row boxes, read
 // by four-row TMA gathers.  Stage 2: a = rows of h (128-row boxes) and a32 =

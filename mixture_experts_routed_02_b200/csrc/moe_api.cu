@@ -251,8 +251,9 @@ bool make_map(CUtensorMap* map, const void* base, size_t rows, size_t cols, size
 }
 
 // Map of packed MX FP4 weight rows [rows, cols] (two e2m1 codes per byte, row
-// pitch cols/2 bytes) whose copies spread each code to a byte of shared
-// memory (the 4-bit operand form of the block-scaled MMA), 128 codes by
+// pitch cols/2 bytes) whose copies put every 16 codes into 16 bytes of shared
+// memory, 8 of codes and 8 of padding (the 4-bit operand form of the
+// block-scaled MMA), 128 codes by
 // box_rows rows per copy, 128-byte swizzle.
 bool make_map_fp4(CUtensorMap* map, const void* base, size_t rows, size_t cols, int box_rows) {
     EncodeTiledFn fn = encode_fn();
