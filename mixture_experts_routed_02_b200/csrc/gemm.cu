@@ -377,14 +377,15 @@ __global__ void __launch_bounds__(192, 1)
     // Weights depend on nothing earlier in the call: the producer puts the
     // first unit's first weight blocks in flight before waiting for the
     // previous kernel (whose output is the activation operand).
-    int npre = 0;
+    // (Every lane of the producer warp knows npre: the producer loop below
+    // runs warp-wide and its lanes must agree on which stages were issued here.)
+    const int npre = (unit0 < units) ? min(NST, kps) : 0;
     if (warp == 0 && lane == 0 && unit0 < units) {
         int m, n, split, q4;
         bool dup;
         unit_coords(unit0, m, n, split, dup, q4);
         const int e = expert_of(m);
         const uint32_t tx = stage_tx(a_rows32(m), q4);
-        npre = min(NST, kps);
         for (int kk = 0; kk < npre; ++kk) {  // fresh stages: nothing to wait for
             if (leader) mbar_arrive_expect_tx(&full[kk], tx);
             load_weights(kk, e, n, split * kps + kk, q4);
