@@ -269,9 +269,9 @@ typedef enum {
     MOE_WS_PERM = 4,       /* int32 [T*k] */
     MOE_WS_INV_PERM = 5,   /* int32 [T*k] */
     MOE_WS_SLOT_OF = 6,    /* int32 [T*k]: assignment -> row of the expert-padded layout */
-    MOE_WS_XS = 7,         /* FP8: quantised activations, one row per token: e4m3 [T,H] (the first
-                              group GEMM gathers each expert's rows from here; BF16 gathers
-                              from x itself and this region is empty) */
+    MOE_WS_XS = 7,         /* FP8: quantised activations, one row per token: e4m3 [T,H], written
+                              when the first group GEMM gathers each expert's rows itself
+                              (MOE_OPT_GATHER 1; BF16 then gathers from x itself); empty for BF16 */
     MOE_WS_SX = 8,         /* FP8: fp32 [T] per-token activation scale (empty for BF16) */
     MOE_WS_H = 9,          /* intermediate h [S,F]: e4m3 or bf16, rows F*eb + 128 bytes apart */
     MOE_WS_H_SF = 10,      /* UE8M0 block scales of h (FP8), tiled for the tensor cores */
@@ -279,8 +279,11 @@ typedef enum {
     MOE_WS_NUM_MTILES = 12, /* int32: number of 128-row tiles in the padded layout */
     MOE_WS_SLOT_ASSIGN = 13, /* int32 [S]: padded row -> assignment, -1 for a padding row */
     MOE_WS_MTILE_EXPERT = 14, /* int32 [S/128]: 128-row tile -> expert */
-    MOE_WS_ROUTE_BLOCKS = 15  /* int32 [ceil(T/256), E]: assignments per expert of each 256-token
+    MOE_WS_ROUTE_BLOCKS = 15, /* int32 [ceil(T/256), E]: assignments per expert of each 256-token
                                  block (routing of large batches on many SMs) */
+    MOE_WS_XG = 16            /* gathered activations, one row per padded slot: e4m3 or bf16 [S,H],
+                                 rows H*eb + 128 bytes apart (written by the gather pass; padding
+                                 rows unspecified) */
 } moe_ws_region;
 
 long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int which, size_t* bytes);
@@ -310,13 +313,21 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
  *                     MOE_ERR_DEVICE_BOUNDS and skips the access; the call's
  *                     outputs are undefined and the context stays usable.
  *                     0 (default) = off.
+ *   MOE_OPT_GATHER:   how the first group GEMM gets each expert's token rows:
+ *                     0 = automatic (currently 2), 1 = the GEMM gathers them
+ *                     itself with TMA tile::gather4 (four rows per copy) from
+ *                     the per-token rows (MOE_WS_XS, or x for BF16) after a
+ *                     per-token quantisation pass, 2 = a gather pass writes
+ *                     them into the expert-padded layout (MOE_WS_XG) and the
+ *                     GEMM copies whole tiles.
  * Returns the previous value, or MOE_ERR_INVALID_ARG. */
 typedef enum {
     MOE_OPT_PATH = 0,
     MOE_OPT_SPLITK = 1,
     MOE_OPT_TIMEOUT_MS = 2,
     MOE_OPT_TEST_STALL = 3,
-    MOE_OPT_TEST_CORRUPT = 4
+    MOE_OPT_TEST_CORRUPT = 4,
+    MOE_OPT_GATHER = 5
 } moe_option;
 int moe_set_option(int option, int value);
 

@@ -1,8 +1,10 @@
 // elementwise.cu -- the memory-bound steps around the two grouped GEMMs:
-//   quant_kernel     per-token FP8 quantisation of the activations (the first
-//                    GEMM gathers each expert's token rows from its output;
-//                    rocketrecap.com "FlyDSL kernels in JAX", paragraph 2:
-//                    "gather") and zeroing of the fp32 combine buffer;
+//   gather_kernel    gather of each expert's token rows into the expert-padded
+//                    layout (rocketrecap.com "FlyDSL kernels in JAX", paragraph
+//                    2: "gather"), fused with the per-token FP8 quantisation and
+//                    with zeroing the fp32 combine buffer;
+//   quant_kernel     per-token FP8 quantisation alone (for the first GEMM's
+//                    own TMA gather of token rows) and zeroing of out32;
 //   finalize_kernel  fp32 combine buffer -> bf16 output;
 //   preshuffle_kernel the one-time load-time preshuffle of the expert weights into
 //                    contiguous, pre-swizzled 128x128-byte operand blocks
@@ -98,6 +100,147 @@ __global__ void __launch_bounds__(128, 8) quant_kernel(const __nv_bfloat16* __re
     }
     griddep_wait();  // the router has completed ...
     griddep_launch_dependents();  // ... before the first GEMM may start
+}
+
+// The gather pass (the first GEMM then reads 128- or 32-row tiles of the
+// gathered rows with one TMA tile copy each; for tiles of many rows that is
+// far cheaper for the copy engine than 32 four-row gathers per K step).  One
+// CTA (128 threads) per `per_cta` consecutive assignments a = t*k + j of one
+// token t (per_cta = k: the whole token; 1: one assignment, for small batches
+// where more CTAs shorten the critical path): reads the row once, quantises it
+// once (FP8: the scale is per token, written once to sx[t]) and writes it to
+// the padded-layout row of each of those assignments; the CTA holding the
+// token's first assignment also zeroes its fp32 combine row.  Padding rows are
+// not written: the tensor cores compute each output row from its own input row
+// only, and the outputs of padding rows are discarded.  The row is read into
+// registers before the wait for the routing kernel (the tokens are the
+// caller's input and the combine buffer was last read by the previous call's
+// finalize, both complete before routing started); only the destination rows
+// need the routing result.
+template <bool kFP8, bool kPerToken>
+__global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int k,
+                                                    const int* __restrict__ slot_of, int num_slots,
+                                                    uint8_t* __restrict__ xs, float* __restrict__ sx_tok,
+                                                    float* __restrict__ out32, int* __restrict__ status) {
+    __shared__ float warp_max[4];
+    const int tid = threadIdx.x;
+    const int per_cta = kPerToken ? k : 1;
+    const int a0 = blockIdx.x * per_cta;
+    const int t = a0 / k;
+    const int eb = kFP8 ? 1 : 2;
+    const int nvec_in = H / 8;  // 8 bf16 per 16-byte vector
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    const bool in_regs = nvec_in <= 128 * kRegVec;
+    uint4 v[kRegVec];
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < kRegVec; ++r) {
+            const int i = tid + r * 128;
+            v[r] = (i < nvec_in) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    if (a0 % k == 0 && out32) {
+        float4* o = reinterpret_cast<float4*>(out32 + (size_t)t * H);
+        for (int i = tid; i < H / 4; i += 128) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+    const int n = per_cta;
+    int slots[kPerToken ? kMaxTopK : 1];
+    bool bad = false;
+    for (int j = 0; j < n; ++j) {
+        slots[j] = slot_of[a0 + j];
+        bad |= slots[j] < 0 || slots[j] >= num_slots;  // never from the router: a corrupted table
+    }
+    if (bad) {
+        if (tid == 0) record_error(status, MOE_ERR_DEVICE_BOUNDS);
+        return;
+    }
+    const long pitch = act_pitch((long)H * eb);
+    if (!kFP8) {
+        for (int j = 0; j < n; ++j) {
+            uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)slots[j] * pitch);
+            if (in_regs) {
+#pragma unroll
+                for (int r = 0; r < kRegVec; ++r) {
+                    const int i = tid + r * 128;
+                    if (i < nvec_in) dst[i] = v[r];
+                }
+            } else {
+                for (int i = tid; i < nvec_in; i += 128) dst[i] = __ldg(src + i);
+            }
+        }
+        return;
+    }
+    float amax = 0.f;
+    auto absmax8 = [&](const uint4& u) {
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p[j]);
+            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    };
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < kRegVec; ++r) absmax8(v[r]);
+    } else {
+        for (int i = tid; i < nvec_in; i += 128) absmax8(__ldg(src + i));
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+    if ((tid & 31) == 0) warp_max[tid >> 5] = amax;
+    __syncthreads();
+    amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
+    const float sx = (amax == 0.f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+    if (tid == 0 && a0 % k == 0) sx_tok[t] = sx;
+    auto quant8 = [&](const uint4& u) {
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+        uint32_t packed[2];
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+            const float2 f0 = __bfloat1622float2(p[j]);
+            const float2 f1 = __bfloat1622float2(p[j + 1]);
+            const __nv_fp8x2_storage_t q0 = __nv_cvt_float2_to_fp8x2(
+                make_float2(__fdiv_rn(f0.x, sx), __fdiv_rn(f0.y, sx)), __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8x2_storage_t q1 = __nv_cvt_float2_to_fp8x2(
+                make_float2(__fdiv_rn(f1.x, sx), __fdiv_rn(f1.y, sx)), __NV_SATFINITE, __NV_E4M3);
+            packed[j / 2] = (uint32_t)q0 | ((uint32_t)q1 << 16);
+        }
+        return make_uint2(packed[0], packed[1]);
+    };
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < kRegVec; ++r) {
+            const int i = tid + r * 128;
+            if (i < nvec_in) {
+                const uint2 q = quant8(v[r]);
+                for (int j = 0; j < n; ++j) reinterpret_cast<uint2*>(xs + (size_t)slots[j] * pitch)[i] = q;
+            }
+        }
+    } else {
+        for (int i = tid; i < nvec_in; i += 128) {
+            const uint2 q = quant8(__ldg(src + i));
+            for (int j = 0; j < n; ++j) reinterpret_cast<uint2*>(xs + (size_t)slots[j] * pitch)[i] = q;
+        }
+    }
+}
+
+cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, int num_slots,
+                          uint8_t* xs, float* sx_tok, float* out32, int* status, cudaStream_t stream) {
+    // a CTA per token for large batches, per assignment (more CTAs, shorter
+    // critical path) for small ones
+    const bool per_token = T >= 256;
+    const dim3 grid(std::max(1, per_token ? T : T * k));
+    if (fp8)
+        return per_token ? launch_dependent(gather_kernel<true, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
+                                            num_slots, xs, sx_tok, out32, status)
+                         : launch_dependent(gather_kernel<true, false>, grid, dim3(128), 0, stream, x, T, H, k,
+                                            slot_of, num_slots, xs, sx_tok, out32, status);
+    return per_token ? launch_dependent(gather_kernel<false, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
+                                        num_slots, xs, sx_tok, out32, status)
+                     : launch_dependent(gather_kernel<false, false>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
+                                        num_slots, xs, sx_tok, out32, status);
 }
 
 cudaError_t launch_quant(bool fp8, const __nv_bfloat16* x, int T, int H, uint8_t* xq, float* sx_tok, float* out32,

@@ -167,9 +167,9 @@ __global__ void __launch_bounds__(192, 1)
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
-        if constexpr (!PAIR && STAGE == 2) prefetch_tmap(&tmA32);
+        if constexpr (!PAIR) prefetch_tmap(&tmA32);
         if constexpr (PAIR || MXW) prefetch_tmap(&tmB);
-        if constexpr (PAIR && C::SFA_VAR) prefetch_tmap(&tmSF);
+        if ((PAIR && C::SFA_VAR) || (STAGE == 1 && args.a_gather)) prefetch_tmap(&tmSF);
     }
     // Expert-major tile order: the first 128-row tile (and, for pairs, the
     // first pair of tiles) of each expert, from a scan of the per-expert row
@@ -396,9 +396,11 @@ __global__ void __launch_bounds__(192, 1)
 
     if (warp == 0) {
         // Producer warp.  Lane 0 waits for a free stage and copies the weights
-        // (and stage 2's activation tile and scales); in stage 1 the lanes
-        // then gather the activation rows of the tile, four token rows per
-        // lane, straight from the per-token rows (xq or x) by TMA.
+        // and the activation tile (rows of the padded layout: the gather pass's
+        // output in stage 1, h in stage 2) and scales; with a_gather, stage 1's
+        // lanes instead gather the activation rows of the tile, four token rows
+        // per lane, straight from the per-token rows (xq or x) by TMA.
+        const bool tma_gather = (STAGE == 1) && args.a_gather != 0;
         const uint64_t pol_a = policy_evict_last();
         int stage = 0;
         uint32_t phase = 0;
@@ -414,9 +416,9 @@ __global__ void __launch_bounds__(192, 1)
             // stage 1: token rows behind this lane's four rows of the m-tile
             // (a padding row reads token 0; its results are discarded)
             const int rows_in = (small || AR == 32) ? 32 : kBlockM;
-            const bool gathers = (STAGE == 1) && 4 * lane < rows_in;
+            const bool gathers = tma_gather && 4 * lane < rows_in;
             int tok[4] = {0, 0, 0, 0};
-            if (STAGE == 1 && gathers) {
+            if (gathers) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) tok[j] = max(token_of(m * kBlockM + 4 * lane + j), 0);
             }
@@ -440,14 +442,14 @@ __global__ void __launch_bounds__(192, 1)
                 // copy of its first stage out, so that stage never completes
                 // and the MMA's bounded wait runs out (see MOE_OPT_TEST_STALL)
                 const bool skip = args.test_stall && blockIdx.x == 0 && issued == 0;
-                if constexpr (STAGE == 1) {
+                if (tma_gather) {
                     if (!skip && gathers) {
                         uint8_t* dst = smem + stage * C::A_BYTES + lane * 4 * 128;
                         if constexpr (PAIR)
-                            tma_gather4_pair(dst, &tmA, mapa_shared(smem_u32(&full[stage]), 0), kt * C::KE, tok[0],
+                            tma_gather4_pair(dst, &tmSF, mapa_shared(smem_u32(&full[stage]), 0), kt * C::KE, tok[0],
                                              tok[1], tok[2], tok[3], pol_a);
                         else
-                            tma_gather4(dst, &tmA, &full[stage], kt * C::KE, tok[0], tok[1], tok[2], tok[3], pol_a);
+                            tma_gather4(dst, &tmSF, &full[stage], kt * C::KE, tok[0], tok[1], tok[2], tok[3], pol_a);
                     }
                 } else if (lane == 0) {
                     if constexpr (PAIR) {
@@ -800,15 +802,19 @@ cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, int grid, cud
     auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR, AR, MXW>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
+    // the fourth map: h's scale chunks (block-scaled stage 2 on CTA pairs) or
+    // the per-token rows for the TMA gather (stage 1 with a_gather)
+    if ((PAIR && C::SFA_VAR && !maps.sf) || (STAGE == 1 && args.a_gather && !maps.sf)) return cudaErrorInvalidValue;
+    const CUtensorMap& m4 = maps.sf ? *maps.sf : *maps.a;
     if constexpr (PAIR) {
         if (grid < 2 || grid % 2) return cudaErrorInvalidValue;
-        if (!maps.b || (C::SFA_VAR && !maps.sf)) return cudaErrorInvalidValue;
+        if (!maps.b) return cudaErrorInvalidValue;
         return launch_dependent_cluster(kern, dim3(grid), dim3(192), C::SMEM_BYTES, 2, stream, *maps.a, *maps.a,
-                                        *maps.b, C::SFA_VAR ? *maps.sf : *maps.a, args);
+                                        *maps.b, m4, args);
     } else {
         if (!maps.a32 || (MXW && !maps.b)) return cudaErrorInvalidValue;
         return launch_dependent(kern, dim3(grid), dim3(192), C::SMEM_BYTES, stream, *maps.a, *maps.a32,
-                                MXW ? *maps.b : *maps.a, *maps.a, args);
+                                MXW ? *maps.b : *maps.a, m4, args);
     }
 }
 

@@ -117,6 +117,8 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, const RouteOu
 int route_launches(int T, const RouteOutputs& o);  // kernels launch_route enqueues (1 or 2)
 cudaError_t launch_quant(bool fp8, const __nv_bfloat16* x, int T, int H, uint8_t* xq, float* sx_tok, float* out32,
                          cudaStream_t stream);
+cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, int num_slots,
+                          uint8_t* xs, float* sx_tok, float* out32, int* status, cudaStream_t stream);
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream);
 // d_ff-sharded layer: after the second GEMM, add 1 to every rank's arrival
 // counter (system scope); then this rank waits (bounded) until its counter
@@ -166,6 +168,8 @@ struct GemmArgs {
     const int* counts;        // rows per expert [num_experts] (for group_m)
     int num_experts;
     int mt_max;               // bound of *num_mtiles (a larger value is a corrupted table)
+    int a_gather;             // stage 1: 1 = gather token rows by TMA (tile::gather4); 0 = tile copies of
+                              // the rows a gather pass wrote in the expert-padded layout
     // d_ff-sharded layer, stage 2: with n_ranks > 0 token t's row is added into
     // the combine rows of the rank that owns it (t / rows_per_rank), at
     // peer_out[owner] + (t - owner * rows_per_rank) * H, through peer memory
@@ -179,11 +183,12 @@ struct GemmArgs {
 // (With MX FP4 weights, b is the packed e2m1 weight rows, read with 64-row
 // boxes, every 16 codes into 16 bytes of shared memory.)
 // Tensor maps of one GEMM launch, all with 128-byte swizzle for the
-// activations.  Stage 1: a = the token rows (xq or x) with one-row boxes, read
-// by four-row TMA gathers.  Stage 2: a = rows of h (128-row boxes) and a32 =
-// the same with 32-row boxes (one-CTA tiles).  For CTA pairs also b = blocked
-// weights (16 KB boxes) and, for the block-scaled stage 2, sf = h's scale
-// chunks (512-byte boxes).
+// activations.  a = rows of the padded layout (gathered activations in stage
+// 1, h in stage 2) with 128-row boxes and a32 = the same with 32-row boxes
+// (one-CTA tiles).  For CTA pairs (and MX FP4 weights) also b = the weights.
+// sf: for the block-scaled stage 2, h's scale chunks (512-byte boxes); for
+// stage 1, the per-token rows (xq or x) with one-row boxes, read by four-row
+// TMA gathers when GemmArgs::a_gather is set.
 struct GemmMaps {
     const CUtensorMap* a;
     const CUtensorMap* a32;

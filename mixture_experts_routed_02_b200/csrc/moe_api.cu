@@ -30,6 +30,7 @@ std::atomic<int> g_opt_splitk{0};
 std::atomic<int> g_opt_timeout_ms{2000};
 std::atomic<int> g_opt_test_stall{0};
 std::atomic<int> g_opt_test_corrupt{0};
+std::atomic<int> g_opt_gather{0};
 
 // ---------------------------------------------------------------- profiling
 
@@ -159,7 +160,7 @@ int context_info(CtxInfo* out) {
 
 // ---------------------------------------------------------------- workspace
 
-constexpr int kRegions = 16;
+constexpr int kRegions = 17;
 
 struct Layout {
     size_t off[kRegions];
@@ -203,6 +204,7 @@ Layout make_layout(int T, int H, int F, int E, int k, int dtype) {
     sz[MOE_WS_SLOT_ASSIGN] = 4 * S;
     sz[MOE_WS_MTILE_EXPERT] = 4 * (size_t)L.MT_max;
     sz[MOE_WS_ROUTE_BLOCKS] = 4 * (size_t)((T + 255) / 256) * E;
+    sz[MOE_WS_XG] = S * act_pitch((long)H * eb);
     size_t off = 0;
     for (int r = 0; r < kRegions; ++r) {
         L.off[r] = off;
@@ -303,7 +305,7 @@ struct MapKey {
     }
 };
 struct MapSet {
-    CUtensorMap tg1, ta2, ta2s, tb1, tb2, tsf2;
+    CUtensorMap tg1, ta1, ta1s, ta2, ta2s, tb1, tb2, tsf2;
 };
 constexpr int kMapCache = 16;
 struct MapEntry {
@@ -401,6 +403,9 @@ int moe_set_option(int option, int value) {
         case MOE_OPT_TEST_CORRUPT:
             if (value < 0 || value > 3) return MOE_ERR_INVALID_ARG;
             return g_opt_test_corrupt.exchange(value);
+        case MOE_OPT_GATHER:
+            if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+            return g_opt_gather.exchange(value);
         default:
             return MOE_ERR_INVALID_ARG;
     }
@@ -540,6 +545,8 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
     MapSet ms;
     if (!find_maps(mkey, &ms)) {
         if (!make_map(&ms.tg1, a1_base, T, H, (size_t)H * eb, eb, 1) ||
+            !make_map(&ms.ta1, reg(MOE_WS_XG), L.S_max, H, act_pitch((long)H * eb), eb, kBlockM) ||
+            !make_map(&ms.ta1s, reg(MOE_WS_XG), L.S_max, H, act_pitch((long)H * eb), eb, 32) ||
             !make_map(&ms.ta2, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, kBlockM) ||
             !make_map(&ms.ta2s, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, 32))
             return MOE_ERR_CUDA;
@@ -555,7 +562,14 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
             return MOE_ERR_CUDA;
         store_maps(mkey, ms);
     }
-    const GemmMaps maps1{&ms.tg1, &ms.tg1, (cfg1 == 0 || mxw) ? &ms.tb1 : nullptr, nullptr};
+    // The first GEMM's activation rows: gathered by TMA inside the GEMM from
+    // the per-token rows, or tile copies of the rows a gather pass wrote in the
+    // padded layout.  A tile of many rows needs 32 four-row gathers per K
+    // step, which keeps the copy engine from feeding the tensor cores, so the
+    // gather pass is the default (MOE_OPT_GATHER selects either).
+    const int opt_gather = g_opt_gather.load();
+    const bool tma_gather = (opt_gather == 1);
+    const GemmMaps maps1{&ms.ta1, &ms.ta1s, (cfg1 == 0 || mxw) ? &ms.tb1 : nullptr, tma_gather ? &ms.tg1 : nullptr};
     const GemmMaps maps2{&ms.ta2, &ms.ta2s, (cfg2 == 0 || mxw) ? &ms.tb2 : nullptr,
                          (cfg2 == 0 && fp8) ? &ms.tsf2 : nullptr};
     // grid: one CTA per SM at most; pairs: whole clusters that can be resident
@@ -587,15 +601,20 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
         if (cudaMemsetAsync(target, 0x7F, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
     }
 
-    // 2. per-token quantisation (FP8) and zeroing of the combine buffer
+    // 2. per-token quantisation (FP8) -- with the gather into the padded
+    // layout, or alone for the first GEMM's TMA gather -- and zeroing of the
+    // combine buffer
     const int* num_mt = o.num_mtiles;
     float* out32 = reinterpret_cast<float*>(reg(MOE_WS_OUT32));
     float* sx = fp8 ? reinterpret_cast<float*>(reg(MOE_WS_SX)) : nullptr;
     {
         ProfScope ps(MOE_KERNEL_QUANT, st);
-        if (launch_quant(fp8, static_cast<const __nv_bfloat16*>(x), T, H, fp8 ? reg(MOE_WS_XS) : nullptr, sx,
-                         dff ? nullptr : out32, st) != cudaSuccess)
-            return MOE_ERR_CUDA;
+        const cudaError_t e =
+            tma_gather ? launch_quant(fp8, static_cast<const __nv_bfloat16*>(x), T, H, fp8 ? reg(MOE_WS_XS) : nullptr,
+                                      sx, dff ? nullptr : out32, st)
+                       : launch_gather(fp8, static_cast<const __nv_bfloat16*>(x), T, H, k, o.slot_of, L.S_max,
+                                       reg(MOE_WS_XG), sx, dff ? nullptr : out32, status, st);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
 
     const unsigned long long timeout_ns = (unsigned long long)g_opt_timeout_ms.load() * 1000000ull;
@@ -626,6 +645,7 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
     g1.counts = o.counts;
     g1.num_experts = E;
     g1.mt_max = L.MT_max;
+    g1.a_gather = tma_gather ? 1 : 0;
     g1.group_m = (cfg1 != 1) ? 1 : 0;
     {
         ProfScope ps(MOE_KERNEL_STAGE1, st);

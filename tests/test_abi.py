@@ -63,7 +63,8 @@ def test_workspace_region_sizes(moe, T, H, F, E, k, dt):
     want = dict(topk_ids=4 * A, topk_w=4 * A, counts=4 * E, offsets=4 * (E + 1), perm=4 * A, inv_perm=4 * A,
                 slot_of=4 * A, xs=T * H if dt == 1 else 0, sx=4 * T if dt == 1 else 0, h=S * (F * eb + 128),
                 h_sf=mt_max * (F // 128) * 512 if dt == 1 else 0, out32=4 * T * H, num_mtiles=4,
-                slot_assign=4 * S, mtile_expert=4 * mt_max, route_blocks=4 * (-(-T // 256)) * E)
+                slot_assign=4 * S, mtile_expert=4 * mt_max, route_blocks=4 * (-(-T // 256)) * E,
+                xg=S * (H * eb + 128))
     assert set(want) == set(moe.WS)
     for name, n in want.items():
         off, size = moe.moe_workspace_region(T, H, F, E, k, dt, moe.WS[name])
@@ -146,6 +147,8 @@ def test_test_hook_options_range(moe):
     assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, 4) == -1
     assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, -1) == -1
     assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, 0) == 0
+    assert moe.moe_set_option(moe.OPT_GATHER, 3) == -1
+    assert moe.moe_set_option(moe.OPT_GATHER, 0) == 0
 
 
 def test_dff_entry_checks_arguments(moe):

@@ -29,6 +29,29 @@ def _reset_options(moe):
     yield
     moe.moe_set_option(moe.OPT_PATH, 0)
     moe.moe_set_option(moe.OPT_SPLITK, 0)
+    moe.moe_set_option(moe.OPT_GATHER, 0)
+
+
+GATHER = pytest.mark.parametrize("gather", [2, 1], ids=["gather_pass", "tma_gather"])
+
+
+def check_r0(moe, ws, case, nc, gather):
+    """R0 bitwise: the per-token e4m3 codes (in the rows the first GEMM reads:
+    per-token rows for the TMA gather, gather = 1; the padded layout written by
+    the gather pass otherwise) and the per-token scales equal the oracle's."""
+    T, H, F, E, k, dt = (case[n] for n in ("T", "H", "F", "E", "k", "dtype"))
+    dtc = moe.dtype_code(dt)
+    xq_ref, sx_ref = oracle.quant_x(nc["x"])
+    sx = moe.ws_view(ws, T, H, F, E, k, dtc, "sx", torch.float32)[:T].cpu().numpy()
+    np.testing.assert_array_equal(sx.view(np.uint32), sx_ref.view(np.uint32))
+    if gather == 1:
+        xs = moe.ws_view(ws, T, H, F, E, k, dtc, "xs").cpu().numpy().reshape(T, H)
+        np.testing.assert_array_equal(xs, xq_ref)
+    else:
+        A = T * k
+        slot_of = moe.ws_view(ws, T, H, F, E, k, dtc, "slot_of", torch.int32)[:A].cpu().numpy()
+        xg = moe.ws_view(ws, T, H, F, E, k, dtc, "xg").cpu().numpy().reshape(-1, H + 128)[:, :H]
+        np.testing.assert_array_equal(xg[slot_of], xq_ref[np.arange(A) // k])
 
 
 # ---------------------------------------------------------------- routing
@@ -103,13 +126,15 @@ def _ids(p):
     return f"T{T}_H{H}_F{F}_E{E}_k{k}_{dt}" + ("_skew" if skew else "")
 
 
+@GATHER
 @pytest.mark.parametrize("path", [1, 2, 3, 4], ids=["pair_tiles", "streaming_tiles", "wide_tiles", "tiny_tiles"])
 @pytest.mark.parametrize("p", SMALL, ids=_ids)
-def test_layer_small(moe, p, path):
+def test_layer_small(moe, p, path, gather):
     T, H, F, E, k, dt, seed, skew = p
     if path == 4 and T * k > 32:
         pytest.skip("the tiny-batch tiles take at most 32 assignments")
     moe.moe_set_option(moe.OPT_PATH, path)
+    moe.moe_set_option(moe.OPT_GATHER, gather)
     case = small_case(T, H, F, E, k, dt, seed, skew)
     nc = moe_inputs.to_numpy(case)
     dcase = to_device(case)
@@ -125,12 +150,7 @@ def test_layer_small(moe, p, path):
     np.testing.assert_array_equal(ids, r["ids"].reshape(-1))
     np.testing.assert_array_equal(perm, r["perm"])
     if dt in ("fp8", "mxfp4"):
-        # R0: per-token e4m3 codes and scales, bitwise
-        xq_ref, sx_ref = oracle.quant_x(nc["x"])
-        xs = moe.ws_view(ws, T, H, F, E, k, dtc, "xs").cpu().numpy().reshape(T, H)
-        sx = moe.ws_view(ws, T, H, F, E, k, dtc, "sx", torch.float32).cpu().numpy()
-        np.testing.assert_array_equal(xs, xq_ref)
-        np.testing.assert_array_equal(sx.view(np.uint32), sx_ref.view(np.uint32))
+        check_r0(moe, ws, case, nc, gather)
 
 
 MXFP4 = [
@@ -145,16 +165,16 @@ MXFP4 = [
 ]
 
 
+@GATHER
 @pytest.mark.parametrize("p", MXFP4, ids=lambda p: f"T{p[0]}_H{p[1]}_F{p[2]}_E{p[3]}_k{p[4]}" + ("_skew" if p[6] else ""))
-def test_layer_small_mxfp4(moe, p):
+def test_layer_small_mxfp4(moe, p, gather):
     T, H, F, E, k, seed, skew = p
+    moe.moe_set_option(moe.OPT_GATHER, gather)
     case = small_case(T, H, F, E, k, "mxfp4", seed, skew)
     nc = moe_inputs.to_numpy(case)
     out, ws = run_layer(to_device(case))
     verify_layer(moe, ws, out, case, what=f"mxfp4 layer T={T} H={H} F={F}")
-    xq_ref, sx_ref = oracle.quant_x(nc["x"])
-    xs = moe.ws_view(ws, T, H, F, E, k, moe.MOE_MXFP4, "xs").cpu().numpy().reshape(T, H)
-    np.testing.assert_array_equal(xs, xq_ref)
+    check_r0(moe, ws, case, nc, gather)
 
 
 def test_prepare_weights_mx_layout(moe):
@@ -273,13 +293,15 @@ def _last_wave_sliced(num_mt, T, F, E, k, bn, num_sms):
     return tail > 0 and tail * q <= (q - 1) * grid
 
 
+@GATHER
 @pytest.mark.parametrize("path,dt", [(3, "fp8"), (3, "bf16"), (2, "fp8"), (2, "bf16")],
                          ids=["wide_fp8", "wide_bf16", "streaming_fp8", "streaming_bf16"])
-def test_layer_last_wave_slices(moe, path, dt):
+def test_layer_last_wave_slices(moe, path, dt, gather):
     """The first GEMM's last, lightly filled wave runs as 64-row weight slices
     (MMA N = 64); every slice's SwiGLU columns land in the right place."""
     T, H, F, E, k = 16, 256, 2560, 8, 2
     moe.moe_set_option(moe.OPT_PATH, path)
+    moe.moe_set_option(moe.OPT_GATHER, gather)
     case = small_case(T, H, F, E, k, dt, 61)
     out, ws = run_layer(to_device(case))
     num_mt = int(moe.ws_view(ws, T, H, F, E, k, moe.dtype_code(dt), "num_mtiles", torch.int32)[0])
