@@ -8,8 +8,9 @@ finalize -- over one batch of T tokens whose inputs are already resident in
 HBM.  The headline workload is the Mixtral-8x7B-shaped FP8 decode layer
 (T=16, d_model=4096, d_ff=14336, E=8, top-2); by default (``--config all``)
 the same run also times every other workload of the Mixtral expert shape
-(prefill T=4096 FP8, skewed-routing T=8192 BF16, and the FP8 batch sweep
-T = 1, 128, 1024, 16384) and reports each as a sub-record under ``configs``
+(prefill T=4096 FP8, skewed-routing T=8192 BF16, the FP8 batch sweep
+T = 1, 128, 1024, 16384, and decode / prefill with MX FP4 expert weights) and
+reports each as a sub-record under ``configs``
 with its own step time, roofline, CPU baseline and end-to-end number.
 
 With N > 1, one process per GPU (under torch.distributed.run; ``--gpus N``
@@ -40,7 +41,8 @@ FP8_PER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 HEADLINE = "decode"
 # the workloads of one default run, headline first; the sweep points share one weight set
-ALL_CONFIGS = ["decode", "prefill", "skewed", "sweep_T1", "sweep_T128", "sweep_T1024", "sweep_T16384"]
+ALL_CONFIGS = ["decode", "prefill", "skewed", "sweep_T1", "sweep_T128", "sweep_T1024", "sweep_T16384",
+               "decode_mxfp4", "prefill_mxfp4"]
 
 
 def log(*a):
