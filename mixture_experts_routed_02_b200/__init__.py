@@ -182,6 +182,12 @@ def prepare_weights_mx(w1, w3, s1, s3, w2, s2, stream=None):
     import torch
     E, F, Hh = w1.shape
     H = 2 * Hh
+    for t in (w1, w3, s1, s3, w2, s2):
+        if t.dtype != torch.uint8 or not t.is_contiguous():
+            raise ValueError("prepare_weights_mx takes contiguous uint8 tensors (packed e2m1 codes, UE8M0 exponents)")
+    if (w3.shape != (E, F, Hh) or w2.shape != (E, H, F // 2) or s1.shape != (E, F, H // 32)
+            or s3.shape != (E, F, H // 32) or s2.shape != (E, H, F // 32)):
+        raise ValueError("MX FP4 weight or scale shapes do not match")
     dev = w1.device
     w13 = torch.empty(E * 2 * F * Hh, dtype=torch.uint8, device=dev)
     s13 = torch.empty(E * 2 * F * (H // 32), dtype=torch.uint8, device=dev)
@@ -197,7 +203,13 @@ def prepare_weights(w1, w3, s1, s3, w2, stream=None):
     """One-time preshuffle: returns (w13, s13, w2p) in the blocked layouts the
     kernels stream (w13/w2p are flat byte tensors; s13 [E,2F] or None)."""
     import torch
+    for t in (w1, w3, w2):
+        if t.dtype not in (torch.bfloat16, torch.float8_e4m3fn) or t.dtype != w1.dtype or not t.is_contiguous():
+            raise ValueError("prepare_weights takes contiguous bf16 or float8_e4m3fn weights of one dtype "
+                             "(MX FP4 weights: prepare_weights_mx)")
     E, F, H = w1.shape
+    if w3.shape != (E, F, H) or w2.shape != (E, H, F):
+        raise ValueError(f"weight shapes {tuple(w1.shape)}, {tuple(w3.shape)}, {tuple(w2.shape)} do not match")
     fp8 = w1.dtype == torch.float8_e4m3fn
     w13 = torch.empty(E * 2 * F * H * w1.element_size(), dtype=torch.uint8, device=w1.device)
     w2p = torch.empty(w2.numel() * w2.element_size(), dtype=torch.uint8, device=w2.device)
