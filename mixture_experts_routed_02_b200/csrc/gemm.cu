@@ -220,17 +220,17 @@ __global__ void __launch_bounds__(192, 1)
     const int ns = args.n_tiles * args.splits;
     const int tiles = PAIR ? s_pair_first[args.num_experts] * ns : num_mt * ns;
     const int kps = args.k_tiles / args.splits;
-    // Stage 1 on one CTA per tile: when the last wave of tiles would leave
-    // CTAs idle and cutting its tiles finishes sooner, each of its tiles is cut
-    // into kQ = BN/64 units of 64 weight rows (no K split, so nothing to add
-    // up afterwards), which spreads that wave's weight stream over more SMs.
-    // The cut pays when its ceil(tail*kQ/grid) waves of quarter-size units take
-    // less than one whole wave: tail*kQ <= (kQ-1)*grid.
+    // Stage 1 on one CTA per tile: when the last wave of tiles would keep at
+    // most 1/kQ of the CTAs busy, each of its tiles is cut into kQ = BN/64
+    // units of 64 weight rows (no K split, so nothing to add up afterwards),
+    // which spreads that wave's weight stream over kQ times as many SMs.  (Cutting
+    // a fuller last wave, whose cut units then take several waves, was measured
+    // slower: with 76 of 148 CTAs in the last wave, 50 -> 64 us at one token.)
     constexpr int kQ = BN / 64;
     int full_tiles = tiles;
     if constexpr (STAGE == 1 && !PAIR && kQ > 1) {
         const int tail = tiles % (int)gridDim.x;
-        if (tail > 0 && tail * kQ <= (kQ - 1) * (int)gridDim.x) full_tiles = tiles - tail;
+        if (tail > 0 && tail * kQ <= (int)gridDim.x) full_tiles = tiles - tail;
     }
     const int units = full_tiles + (tiles - full_tiles) * kQ;
     // Work unit -> (this CTA's m-tile, n, split); `dup` marks the second half
@@ -747,29 +747,40 @@ __global__ void __launch_bounds__(192, 1)
                     tmem_ld_wait();
                     if (c0 + 64 == BN) release(acc);
                     if (t >= 0) {
+                        // the 64 weighted (and, FP8, channel-scaled) values first, all
+                        // scale loads in flight together; then one branch around two
+                        // straight runs of atomics (a branch inside the run keeps the
+                        // compiler from hoisting the loads)
                         const int col = n * BN + c0;
-                        const float* cs = (FP8 && !MXW) ? args.col_scale + (size_t)e * args.rows_b + col : nullptr;
+                        float4 v[16];
 #pragma unroll
-                        for (int i = 0; i < 64; i += 4) {
-                            float4 v;
-                            v.x = __uint_as_float(r[i]) * wgt;
-                            v.y = __uint_as_float(r[i + 1]) * wgt;
-                            v.z = __uint_as_float(r[i + 2]) * wgt;
-                            v.w = __uint_as_float(r[i + 3]) * wgt;
-                            if constexpr (FP8 && !MXW) {
-                                const float4 sc = __ldg(reinterpret_cast<const float4*>(cs + i));
-                                v.x *= sc.x;
-                                v.y *= sc.y;
-                                v.z *= sc.z;
-                                v.w *= sc.w;
+                        for (int i4 = 0; i4 < 16; ++i4)
+                            v[i4] = make_float4(__uint_as_float(r[4 * i4]) * wgt, __uint_as_float(r[4 * i4 + 1]) * wgt,
+                                                __uint_as_float(r[4 * i4 + 2]) * wgt,
+                                                __uint_as_float(r[4 * i4 + 3]) * wgt);
+                        if constexpr (FP8 && !MXW) {
+                            const float4* cs4 =
+                                reinterpret_cast<const float4*>(args.col_scale + (size_t)e * args.rows_b + col);
+#pragma unroll
+                            for (int i4 = 0; i4 < 16; ++i4) {
+                                const float4 sc = __ldg(cs4 + i4);
+                                v[i4].x *= sc.x;
+                                v[i4].y *= sc.y;
+                                v[i4].z *= sc.z;
+                                v[i4].w *= sc.w;
                             }
-                            if (remote) {  // scalar atomics through peer memory
-                                atomicAdd(orow + col + i, v.x);
-                                atomicAdd(orow + col + i + 1, v.y);
-                                atomicAdd(orow + col + i + 2, v.z);
-                                atomicAdd(orow + col + i + 3, v.w);
-                            } else {
-                                atomicAdd(reinterpret_cast<float4*>(orow + col + i), v);
+                        }
+                        if (!remote) {
+#pragma unroll
+                            for (int i4 = 0; i4 < 16; ++i4)
+                                atomicAdd(reinterpret_cast<float4*>(orow + col + 4 * i4), v[i4]);
+                        } else {  // scalar atomics through peer memory
+#pragma unroll
+                            for (int i4 = 0; i4 < 16; ++i4) {
+                                atomicAdd(orow + col + 4 * i4, v[i4].x);
+                                atomicAdd(orow + col + 4 * i4 + 1, v[i4].y);
+                                atomicAdd(orow + col + 4 * i4 + 2, v[i4].z);
+                                atomicAdd(orow + col + 4 * i4 + 3, v[i4].w);
                             }
                         }
                     }
@@ -829,8 +840,9 @@ int max_pairs_one() {
 
 }  // namespace
 
-int gemm_block_n(int stage, bool fp8, int cfg) {
+int gemm_block_n(int stage, bool fp8, int cfg, bool mxw) {
     (void)fp8;
+    if (mxw) return 128;
     if (cfg == 3) return stage == 1 ? 256 : 128;
     return cfg == 1 ? 128 : 256;
 }
@@ -839,12 +851,18 @@ int gemm_block_n(int stage, bool fp8, int cfg) {
 // (weight streaming); cfg 2: one CTA, 128 x 256 tiles; cfg 3 (no m-tile with
 // more than 32 rows in use): 32 activation rows per stage, which leaves room
 // for deeper pipelines -- stage 1 on 128 x 256 tiles, stage 2 on 128 x 128.
-// MX FP4 weights (mxw) run on cfg 1 only: two 128-column accumulators leave
-// room in TMEM for the per-stage scales of both operands.
+// MX FP4 weights (mxw) run on 128 x 128 one-CTA tiles (two 128-column
+// accumulators leave room in TMEM for the per-stage scales of both operands):
+// cfg 1, or cfg 3 (at most 32 assignments in all) with 32 activation rows per
+// stage and 10 stages -- a stage of 4-bit weights brings only half the bytes
+// of an e4m3 one from HBM, so more stages keep enough in flight.
 cudaError_t launch_gemm(int stage, bool fp8, int cfg, const GemmMaps& maps, const GemmArgs& args, int grid,
                         cudaStream_t stream, bool mxw) {
     if (mxw) {
-        if (cfg != 1 || !fp8) return cudaErrorInvalidValue;
+        if ((cfg != 1 && cfg != 3) || !fp8) return cudaErrorInvalidValue;
+        if (cfg == 3)
+            return stage == 1 ? launch_one<1, true, 128, 10, 2, false, 32, true>(maps, args, grid, stream)
+                              : launch_one<2, true, 128, 10, 2, false, 32, true>(maps, args, grid, stream);
         return stage == 1 ? launch_one<1, true, 128, 6, 2, false, kBlockM, true>(maps, args, grid, stream)
                           : launch_one<2, true, 128, 6, 2, false, kBlockM, true>(maps, args, grid, stream);
     }

@@ -202,7 +202,7 @@ struct GemmMaps {
 //      2 = one CTA, 128 x 256 tiles.
 cudaError_t launch_gemm(int stage, bool fp8, int cfg, const GemmMaps& maps, const GemmArgs& args, int grid,
                         cudaStream_t stream, bool mxw = false);
-int gemm_block_n(int stage, bool fp8, int cfg);
+int gemm_block_n(int stage, bool fp8, int cfg, bool mxw = false);
 // Resident clusters of the pair kernel of a stage (0 if it cannot run).
 int gemm_max_pairs(int stage, bool fp8);
 

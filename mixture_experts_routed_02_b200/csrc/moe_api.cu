@@ -529,13 +529,16 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
     } else {
         cfg1 = cfg2 = opt_path - 1;
     }
-    if (mxw) cfg1 = cfg2 = 1;  // MX FP4 weights: 128 x 128 one-CTA tiles (room in TMEM for both operands' scales)
-    if ((2 * F) % gemm_block_n(1, fp8, cfg1)) cfg1 = 1;
-    if (H % gemm_block_n(2, fp8, cfg2)) cfg2 = 1;
+    // MX FP4 weights: 128 x 128 one-CTA tiles (room in TMEM for both operands'
+    // scales), with 32 activation rows per stage and deeper pipelines when the
+    // whole batch has at most 32 assignments
+    if (mxw) cfg1 = cfg2 = (L.A <= 32) ? 3 : 1;
+    if ((2 * F) % gemm_block_n(1, fp8, cfg1, mxw)) cfg1 = 1;
+    if (H % gemm_block_n(2, fp8, cfg2, mxw)) cfg2 = 1;
     if (cfg1 == 0 && max_pairs(1, fp8) < 1) cfg1 = 2;
     if (cfg2 == 0 && max_pairs(2, fp8) < 1) cfg2 = 2;
-    const int bn1 = gemm_block_n(1, fp8, cfg1);
-    const int bn2 = gemm_block_n(2, fp8, cfg2);
+    const int bn1 = gemm_block_n(1, fp8, cfg1, mxw);
+    const int bn2 = gemm_block_n(2, fp8, cfg2, mxw);
     if ((2 * F) % bn1 || H % bn2) return MOE_ERR_UNSUPPORTED;
 
     // stage 1 gathers token rows: from the per-token e4m3 rows (FP8) or from

@@ -284,13 +284,12 @@ def test_layer_split_k(moe, splits):
 
 def _last_wave_sliced(num_mt, T, F, E, k, bn, num_sms):
     """Whether the first GEMM cuts its last wave into 64-row slices: one CTA per
-    SM at most; a last wave whose slices take fewer waves than the number of
-    slices per tile (tail * q <= (q - 1) * grid, q = bn / 64)."""
+    SM at most; a last wave that, cut into bn/64 slices per tile, still fits
+    in the grid."""
     n_tiles = 2 * F // bn
     grid = min((-(-T * k // 128) + E) * n_tiles, num_sms)
     tail = (num_mt * n_tiles) % grid
-    q = bn // 64
-    return tail > 0 and tail * q <= (q - 1) * grid
+    return tail > 0 and tail * (bn // 64) <= grid
 
 
 @GATHER
