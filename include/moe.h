@@ -281,9 +281,10 @@ typedef enum {
     MOE_WS_MTILE_EXPERT = 14, /* int32 [S/128]: 128-row tile -> expert */
     MOE_WS_ROUTE_BLOCKS = 15, /* int32 [ceil(T/256), E]: assignments per expert of each 256-token
                                  block (routing of large batches on many SMs) */
-    MOE_WS_XG = 16            /* gathered activations, one row per padded slot: e4m3 or bf16 [S,H],
+    MOE_WS_XG = 16,           /* gathered activations, one row per padded slot: e4m3 or bf16 [S,H],
                                  rows H*eb + 128 bytes apart (written by the gather pass; padding
                                  rows unspecified) */
+    MOE_WS_SX_SLOT = 17       /* FP8: fp32 [S] activation scale of each padded row (gather pass) */
 } moe_ws_region;
 
 long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int which, size_t* bytes);

@@ -49,7 +49,7 @@ OPT_PATH, OPT_SPLITK, OPT_TIMEOUT_MS, OPT_TEST_STALL, OPT_TEST_CORRUPT, OPT_GATH
 
 # workspace regions (moe_ws_region)
 WS = dict(topk_ids=0, topk_w=1, counts=2, offsets=3, perm=4, inv_perm=5, slot_of=6, xs=7, sx=8, h=9, h_sf=10,
-          out32=11, num_mtiles=12, slot_assign=13, mtile_expert=14, route_blocks=15, xg=16)
+          out32=11, num_mtiles=12, slot_assign=13, mtile_expert=14, route_blocks=15, xg=16, sx_slot=17)
 
 # every symbol include/moe.h declares
 EXPORTS = ["moe_workspace_size", "moe_prepare_weights", "moe_route", "moe_ffn_forward", "moe_get_status",

@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(128, 8) quant_kernel(const __nv_bfloat16* __re
 // CTA (128 threads) per `per_cta` consecutive assignments a = t*k + j of one
 // token t (per_cta = k: the whole token; 1: one assignment, for small batches
 // where more CTAs shorten the critical path): reads the row once, quantises it
-// once (FP8: the scale is per token, written once to sx[t]) and writes it to
+// once (FP8: the scale is per token, written to sx[t] and to each of its
+// padded rows) and writes it to
 // the padded-layout row of each of those assignments; the CTA holding the
 // token's first assignment also zeroes its fp32 combine row.  Padding rows are
 // not written: the tensor cores compute each output row from its own input row
@@ -121,7 +122,8 @@ template <bool kFP8, bool kPerToken>
 __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int k,
                                                     const int* __restrict__ slot_of, int num_slots,
                                                     uint8_t* __restrict__ xs, float* __restrict__ sx_tok,
-                                                    float* __restrict__ out32, int* __restrict__ status) {
+                                                    float* __restrict__ sx_slot, float* __restrict__ out32,
+                                                    int* __restrict__ status) {
     __shared__ float warp_max[4];
     const int tid = threadIdx.x;
     const int per_cta = kPerToken ? k : 1;
@@ -194,6 +196,7 @@ __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __r
     amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
     const float sx = (amax == 0.f) ? 1.0f : __fdiv_rn(amax, 448.0f);
     if (tid == 0 && a0 % k == 0) sx_tok[t] = sx;
+    if (tid < n) sx_slot[slots[tid]] = sx;  // per padded row too: the first GEMM's epilogue reads it there
     auto quant8 = [&](const uint4& u) {
         const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
         uint32_t packed[2];
@@ -227,20 +230,20 @@ __global__ void __launch_bounds__(128, 8) gather_kernel(const __nv_bfloat16* __r
 }
 
 cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, int num_slots,
-                          uint8_t* xs, float* sx_tok, float* out32, int* status, cudaStream_t stream) {
+                          uint8_t* xs, float* sx_tok, float* sx_slot, float* out32, int* status, cudaStream_t stream) {
     // a CTA per token for large batches, per assignment (more CTAs, shorter
     // critical path) for small ones
     const bool per_token = T >= 256;
     const dim3 grid(std::max(1, per_token ? T : T * k));
     if (fp8)
         return per_token ? launch_dependent(gather_kernel<true, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
-                                            num_slots, xs, sx_tok, out32, status)
+                                            num_slots, xs, sx_tok, sx_slot, out32, status)
                          : launch_dependent(gather_kernel<true, false>, grid, dim3(128), 0, stream, x, T, H, k,
-                                            slot_of, num_slots, xs, sx_tok, out32, status);
+                                            slot_of, num_slots, xs, sx_tok, sx_slot, out32, status);
     return per_token ? launch_dependent(gather_kernel<false, true>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
-                                        num_slots, xs, sx_tok, out32, status)
+                                        num_slots, xs, sx_tok, sx_slot, out32, status)
                      : launch_dependent(gather_kernel<false, false>, grid, dim3(128), 0, stream, x, T, H, k, slot_of,
-                                        num_slots, xs, sx_tok, out32, status);
+                                        num_slots, xs, sx_tok, sx_slot, out32, status);
 }
 
 cudaError_t launch_quant(bool fp8, const __nv_bfloat16* x, int T, int H, uint8_t* xq, float* sx_tok, float* out32,

@@ -641,10 +641,16 @@ __global__ void __launch_bounds__(192, 1)
             const int slot = m * kBlockM + row;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             if constexpr (STAGE == 1) {
+                // the activation scale of the row: per padded row as the gather
+                // pass wrote it, or per token for the GEMM's own TMA gather
                 float sxv = 1.0f;
                 if constexpr (FP8) {
-                    const int t = token_of(slot);
-                    sxv = (t >= 0) ? args.row_scale[t] : 0.0f;  // a padding row's results are discarded
+                    if (args.a_gather) {
+                        const int t = token_of(slot);
+                        sxv = (t >= 0) ? args.row_scale[t] : 0.0f;  // a padding row's results are discarded
+                    } else {
+                        sxv = args.row_scale_slot[slot];
+                    }
                 }
 #pragma unroll 1
                 // 64-column groups: all BN / 64 of a tile, or the one of a 64-row slice
@@ -724,7 +730,11 @@ __global__ void __launch_bounds__(192, 1)
                 release(acc);
             } else {
                 const int a = dup ? -1 : args.slot_assign[slot];
-                const int t = dup ? -1 : token_of(slot);
+                int t = (a >= 0) ? a / args.topk : -1;
+                if (t >= args.T || a < -1) {  // never from the router: a corrupted table
+                    record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
+                    t = -1;
+                }
                 const float wgt = (t >= 0) ? args.topk_w[a] : 0.f;
                 // the combine row: this GPU's buffer, or (d_ff-sharded layer) the
                 // row of the rank that owns token t, possibly in a peer's memory

@@ -118,7 +118,7 @@ int route_launches(int T, const RouteOutputs& o);  // kernels launch_route enque
 cudaError_t launch_quant(bool fp8, const __nv_bfloat16* x, int T, int H, uint8_t* xq, float* sx_tok, float* out32,
                          cudaStream_t stream);
 cudaError_t launch_gather(bool fp8, const __nv_bfloat16* x, int T, int H, int k, const int* slot_of, int num_slots,
-                          uint8_t* xs, float* sx_tok, float* out32, int* status, cudaStream_t stream);
+                          uint8_t* xs, float* sx_tok, float* sx_slot, float* out32, int* status, cudaStream_t stream);
 cudaError_t launch_finalize(const float* out32, __nv_bfloat16* out, size_t n, int num_sms, cudaStream_t stream);
 // d_ff-sharded layer: after the second GEMM, add 1 to every rank's arrival
 // counter (system scope); then this rank waits (bounded) until its counter
@@ -144,7 +144,8 @@ struct GemmArgs {
     const int* num_mtiles;
     const int* mtile_expert;
     const int* slot_assign;
-    const float* row_scale;   // stage 1, FP8: per-token activation scale [T]
+    const float* row_scale;   // stage 1, FP8: per-token activation scale [T] (TMA gather)
+    const float* row_scale_slot;  // stage 1, FP8: the same per padded row [S] (gather pass)
     const float* col_scale;   // FP8: s13 [E*2F] (stage 1) or s2 [E*H] (stage 2)
     const float* topk_w;      // stage 2: routing weight per assignment
     const uint8_t* b_blocks;  // weights in the blocked layout: [E][rows_b/128][k_tiles][16 KB]

@@ -160,7 +160,7 @@ int context_info(CtxInfo* out) {
 
 // ---------------------------------------------------------------- workspace
 
-constexpr int kRegions = 17;
+constexpr int kRegions = 18;
 
 struct Layout {
     size_t off[kRegions];
@@ -205,6 +205,7 @@ Layout make_layout(int T, int H, int F, int E, int k, int dtype) {
     sz[MOE_WS_MTILE_EXPERT] = 4 * (size_t)L.MT_max;
     sz[MOE_WS_ROUTE_BLOCKS] = 4 * (size_t)((T + 255) / 256) * E;
     sz[MOE_WS_XG] = S * act_pitch((long)H * eb);
+    sz[MOE_WS_SX_SLOT] = e4m3_acts(dtype) ? 4 * S : 0;
     size_t off = 0;
     for (int r = 0; r < kRegions; ++r) {
         L.off[r] = off;
@@ -616,7 +617,8 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
             tma_gather ? launch_quant(fp8, static_cast<const __nv_bfloat16*>(x), T, H, fp8 ? reg(MOE_WS_XS) : nullptr,
                                       sx, dff ? nullptr : out32, st)
                        : launch_gather(fp8, static_cast<const __nv_bfloat16*>(x), T, H, k, o.slot_of, L.S_max,
-                                       reg(MOE_WS_XG), sx, dff ? nullptr : out32, status, st);
+                                       reg(MOE_WS_XG), sx, fp8 ? reinterpret_cast<float*>(reg(MOE_WS_SX_SLOT)) : nullptr,
+                                       dff ? nullptr : out32, status, st);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
 
@@ -628,6 +630,7 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
     g1.mtile_expert = o.mtile_expert;
     g1.slot_assign = o.slot_assign;
     g1.row_scale = sx;
+    g1.row_scale_slot = fp8 ? reinterpret_cast<const float*>(reg(MOE_WS_SX_SLOT)) : nullptr;
     g1.col_scale = (fp8 && !mxw) ? static_cast<const float*>(s13) : nullptr;
     g1.b_sf = mxw ? static_cast<const uint8_t*>(s13) : nullptr;
     g1.b_blocks = static_cast<const uint8_t*>(w13);

@@ -64,7 +64,7 @@ def test_workspace_region_sizes(moe, T, H, F, E, k, dt):
                 slot_of=4 * A, xs=T * H if dt == 1 else 0, sx=4 * T if dt == 1 else 0, h=S * (F * eb + 128),
                 h_sf=mt_max * (F // 128) * 512 if dt == 1 else 0, out32=4 * T * H, num_mtiles=4,
                 slot_assign=4 * S, mtile_expert=4 * mt_max, route_blocks=4 * (-(-T // 256)) * E,
-                xg=S * (H * eb + 128))
+                xg=S * (H * eb + 128), sx_slot=4 * S if dt == 1 else 0)
     assert set(want) == set(moe.WS)
     for name, n in want.items():
         off, size = moe.moe_workspace_region(T, H, F, E, k, dt, moe.WS[name])
