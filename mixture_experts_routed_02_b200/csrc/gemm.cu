@@ -401,12 +401,16 @@ __global__ void __launch_bounds__(192, 1)
         // lanes instead gather the activation rows of the tile, four token rows
         // per lane, straight from the per-token rows (xq or x) by TMA.
         const bool tma_gather = (STAGE == 1) && args.a_gather != 0;
+        // without the TMA gather lane 0 alone runs the loop (the other lanes
+        // wait at the end), as the copies it issues need no other lane
+        const bool in_loop = tma_gather || lane == 0;
+        const unsigned loop_mask = tma_gather ? 0xffffffffu : 1u;
         const uint64_t pol_a = policy_evict_last();
         int stage = 0;
         uint32_t phase = 0;
         int issued = 0;
         bool ok = true;
-        for (int u = unit0; u < units && ok; u += ustep) {
+        for (int u = unit0; in_loop && u < units && ok; u += ustep) {
             int m, n, split, q4;
             bool dup;
             unit_coords(u, m, n, split, dup, q4);
@@ -433,7 +437,7 @@ __global__ void __launch_bounds__(192, 1)
                             load_weights(stage, e, n, kt, q4);
                         }
                     }
-                    if (!__shfl_sync(0xffffffffu, good, 0)) {
+                    if (!__shfl_sync(loop_mask, good, 0)) {
                         ok = false;
                         break;
                     }
