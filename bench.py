@@ -640,8 +640,10 @@ def main(argv=None):
         records[name] = run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_s)
         del case
         r = records[name]
+        frac = r["roofline"]["frac"]
         log(f"[rank {rank}] {name}: {r['ms_per_step'] * 1e3:.1f} us/step, {r['value']:.0f} tokens/s, "
-            f"{r['roofline']['kernel']} at {r['roofline']['frac']:.3f} of {r['roofline']['unit']} peak")
+            f"{r['roofline']['kernel']} at " + (f"{frac:.3f}" if frac is not None else "n/a") +
+            f" of {r['roofline']['unit']} peak")
 
     head = names[0]
     h = records[head]
