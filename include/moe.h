@@ -100,15 +100,17 @@ int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const f
  *            blocks of 32 consecutive columns; read only
  *   w2       device, [E,H,F/2] bytes; s2 device, [E,H,F/32] bytes (blocks along d_ff)
  *   w13_out  device, E*2F*H/2 bytes: w1/w3 rows interleaved in groups of 32 as
- *            for moe_prepare_weights, still packed, row-major (read by TMA,
- *            which puts every 16 codes into 16 bytes of shared memory);
- *            32-byte aligned
+ *            for moe_prepare_weights, still packed, cut into contiguous
+ *            blocks of 128 rows x 64 bytes (128 codes of K) in the order
+ *            [expert][128-row block][128-column block], so that a TMA copy of
+ *            half a block reads 4 KB in one run (it puts every 16 codes into
+ *            16 bytes of shared memory); 32-byte aligned
  *   s13_out  device, E*2F*H/32 bytes: the scales of those rows regrouped into
  *            512-byte chunks per (expert, 128-row block, 128-column block),
  *            byte (r%32)*16 + (r/32)*4 + b = row r of the block, 32-column
  *            block b of the chunk (the order the MMA's scale copy takes)
- *   w2_out   device, E*H*F/2 bytes (32-byte aligned); s2_out E*H*F/32 bytes,
- *            the same chunks over [E,H] rows and d_ff columns
+ *   w2_out   device, E*H*F/2 bytes, the same blocks over [E,H] rows and d_ff
+ *            columns (32-byte aligned); s2_out E*H*F/32 bytes, the same chunks
  * The layer is then called with dtype MOE_MXFP4, w13 = w13_out, s13 = s13_out,
  * w2 = w2_out, s2 = s2_out.
  */

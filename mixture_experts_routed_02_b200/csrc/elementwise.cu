@@ -382,20 +382,28 @@ __global__ void interleave_scales_kernel(const float* __restrict__ s1, const flo
     }
 }
 
-// MX FP4 weight preparation.  Rows of packed e2m1 codes (row_bytes each)
-// copied in 16-byte chunks; with `interleave` destination row R of an expert
-// is row 32*(R/64) + R%32 of a (R%64 < 32) or of b (the w1/w3 interleave of
-// the first GEMM), otherwise row R of a.
+// MX FP4 weight preparation.  Packed e2m1 rows (K/2 bytes each) regrouped
+// into contiguous blocks of 128 rows x 64 bytes (128 codes of K) in the order
+// [expert][128-row block][128-column K block], so that each TMA copy of the
+// first (64-row) or second half of a block reads 4 KB in one run (row-major
+// rows would be read as 64-byte pieces 2 KB apart, far too small to keep HBM
+// busy).  One thread per 16-byte chunk of the destination.  With `interleave`
+// destination row R of an expert is row 32*(R/64) + R%32 of a (R%64 < 32) or
+// of b (the w1/w3 interleave of the first GEMM), otherwise row R of a.
 __global__ void mx_rows_kernel(const uint8_t* __restrict__ a, const uint8_t* __restrict__ b,
                                uint8_t* __restrict__ dst, int E, int src_rows, int dst_rows, int row_bytes,
                                bool interleave) {
-    const int chunks = row_bytes / 16;
-    const size_t total = (size_t)E * dst_rows * chunks;
+    const int k_tiles = row_bytes / 64;
+    const size_t total = (size_t)E * dst_rows * row_bytes / 16;
     for (size_t g = blockIdx.x * (size_t)blockDim.x + threadIdx.x; g < total; g += (size_t)gridDim.x * blockDim.x) {
-        const int c = (int)(g % chunks);
-        const size_t rowg = g / chunks;
-        const int R = (int)(rowg % dst_rows);
-        const int e = (int)(rowg / dst_rows);
+        const int c4 = (int)(g & 3);                   // 16-byte chunk of the block row
+        const int r = (int)((g >> 2) & 127);           // row inside the block
+        size_t rest = g >> 9;                          // (expert, block, K block)
+        const int kt = (int)(rest % k_tiles);
+        rest /= k_tiles;
+        const int nb = (int)(rest % (dst_rows / 128));
+        const int e = (int)(rest / (dst_rows / 128));
+        const int R = nb * 128 + r;
         const uint8_t* src = a;
         int srow = R;
         if (interleave) {
@@ -403,7 +411,7 @@ __global__ void mx_rows_kernel(const uint8_t* __restrict__ a, const uint8_t* __r
             srow = 32 * (R / 64) + (R % 32);
         }
         reinterpret_cast<uint4*>(dst)[g] =
-            __ldg(reinterpret_cast<const uint4*>(src + ((size_t)e * src_rows + srow) * row_bytes) + c);
+            __ldg(reinterpret_cast<const uint4*>(src + ((size_t)e * src_rows + srow) * row_bytes + kt * 64) + c4);
     }
 }
 

@@ -339,14 +339,19 @@ __global__ void __launch_bounds__(192, 1)
     // tile, or this CTA's half of them in a pair.
     auto load_weights = [&](int stage, int e, int n, int kt, int q4) {
         if constexpr (MXW) {
-            // MX FP4: packed e2m1 rows by TMA (64-row boxes, 16 codes per 16
-            // bytes of shared memory, 128-byte swizzle), then the B scale chunk of each
-            // 128-row block (512 bytes, already in the layout TMEM takes)
+            // MX FP4: packed e2m1 rows by TMA from the blocked layout (each
+            // 64-row half of a 128-row x 64-byte block is 4 KB in one run; 16
+            // codes per 16 bytes of shared memory, 128-byte swizzle), then the
+            // B scale chunk of each 128-row block (512 bytes, already in the
+            // layout TMEM takes)
             uint8_t* dst = smem + C::OFF_B + stage * C::B_BYTES;
-            const int row0 = e * args.rows_b + n * BN + (q4 >= 0 ? 64 * q4 : 0);
+            const int half0 = (n * BN + (q4 >= 0 ? 64 * q4 : 0)) / 64;  // first 64-row half of the unit
             const int boxes = (q4 >= 0) ? 1 : C::B_ROWS / 64;
-            for (int j = 0; j < boxes; ++j)
-                tma_load_2d(dst + j * 64 * 128, &tmB, &full[stage], kt * C::KE, row0 + 64 * j, pol_b);
+            for (int j = 0; j < boxes; ++j) {
+                const int h = half0 + j;
+                const int brow = (int)((((size_t)e * b_nblk + h / 2) * args.k_tiles + kt) * kWBlockRows) + 64 * (h & 1);
+                tma_load_2d(dst + j * 64 * 128, &tmB, &full[stage], 0, brow, pol_b);
+            }
             const int rb0 = (n * BN + (q4 >= 0 ? 64 * q4 : 0)) / kWBlockRows;
             const int nchunks = (q4 >= 0) ? 1 : C::B_ROWS / kWBlockRows;
             for (int j = 0; j < nchunks; ++j) {

@@ -253,14 +253,14 @@ bool make_map(CUtensorMap* map, const void* base, size_t rows, size_t cols, size
     return r == CUDA_SUCCESS;
 }
 
-// Map of packed MX FP4 weight rows [rows, cols] (two e2m1 codes per byte, row
-// pitch cols/2 bytes) whose copies put every 16 codes into 16 bytes of shared
-// memory, 8 of codes and 8 of padding (the 4-bit operand form of the
-// block-scaled MMA), 128 codes by
-// box_rows rows per copy, 128-byte swizzle.
-bool make_map_fp4(CUtensorMap* map, const void* base, size_t rows, size_t cols, int box_rows) {
+// Map of the blocked MX FP4 weights seen as rows of 128 packed e2m1 codes (64
+// bytes each; see moe_prepare_weights_mx) whose copies put every 16 codes into
+// 16 bytes of shared memory, 8 of codes and 8 of padding (the 4-bit operand
+// form of the block-scaled MMA): box_rows rows per copy, 128-byte swizzle.
+bool make_map_fp4(CUtensorMap* map, const void* base, size_t rows, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    const size_t cols = 128;
     const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)(cols / 2)};
     const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
@@ -555,7 +555,8 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
             !make_map(&ms.ta2s, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, 32))
             return MOE_ERR_CUDA;
         if (mxw) {
-            if (!make_map_fp4(&ms.tb1, w13, (size_t)E * 2 * F, H, 64) || !make_map_fp4(&ms.tb2, w2, (size_t)E * H, F, 64))
+            if (!make_map_fp4(&ms.tb1, w13, (size_t)E * 2 * F * (H / 128), 64) ||
+                !make_map_fp4(&ms.tb2, w2, (size_t)E * H * (F / 128), 64))
                 return MOE_ERR_CUDA;
         }
         if (cfg1 == 0 && !make_map_rows(&ms.tb1, w13, (size_t)E * (2 * F) * (H * eb / 128), kWBlockRows))

@@ -179,18 +179,21 @@ def test_layer_small_mxfp4(moe, p, gather):
 
 def test_prepare_weights_mx_layout(moe):
     """moe_prepare_weights_mx: w13 rows interleaved in groups of 32 (w1 then
-    w3), still packed; the scales regrouped into 512-byte chunks per (expert,
-    128-row block, 128-column block), byte (r%32)*16 + (r/32)*4 + b."""
+    w3), still packed, in contiguous blocks of 128 rows x 64 bytes ordered
+    [expert][row block][K block]; the scales regrouped into 512-byte chunks
+    per (expert, 128-row block, 128-column block), byte (r%32)*16 + (r/32)*4 + b."""
     E, F, H = 2, 256, 384
     case = small_case(3, H, F, E, 2, "mxfp4", 37)
     d = to_device(case)
-    w13 = d["w13"].cpu().numpy().reshape(E, 2 * F, H // 2)
+    unblock = lambda t, rows, cols: (t.cpu().numpy().reshape(E, rows // 128, cols // 128, 128, 64)  # noqa: E731
+                                     .transpose(0, 1, 3, 2, 4).reshape(E, rows, cols // 2))
+    w13 = unblock(d["w13"], 2 * F, H)
     w1, w3 = case["w1"].numpy(), case["w3"].numpy()
     src_rows = lambda R: (w3 if R % 64 >= 32 else w1, 32 * (R // 64) + R % 32)  # noqa: E731
     for R in range(2 * F):
         src, r = src_rows(R)
         np.testing.assert_array_equal(w13[:, R], src[:, r])
-    np.testing.assert_array_equal(d["w2p"].cpu().numpy().reshape(E, H, F // 2), case["w2"].numpy())
+    np.testing.assert_array_equal(unblock(d["w2p"], H, F), case["w2"].numpy())
     s13 = d["s13"].cpu().numpy().reshape(E, 2 * F // 128, H // 128, 512)
     s1, s3 = case["s1"].numpy(), case["s3"].numpy()
     for R in range(2 * F):
