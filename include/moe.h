@@ -323,6 +323,9 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
  *                     per-token quantisation pass, 2 = a gather pass writes
  *                     them into the expert-padded layout (MOE_WS_XG) and the
  *                     GEMM copies whole tiles.
+ *   MOE_OPT_MX_BOX:   MX FP4 weights: rows per TMA copy of the packed weights,
+ *                     0 = automatic (128), 64 or 128 (64-row copies also let
+ *                     the first GEMM cut its last wave into 64-row slices).
  * Returns the previous value, or MOE_ERR_INVALID_ARG. */
 typedef enum {
     MOE_OPT_PATH = 0,
@@ -330,7 +333,8 @@ typedef enum {
     MOE_OPT_TIMEOUT_MS = 2,
     MOE_OPT_TEST_STALL = 3,
     MOE_OPT_TEST_CORRUPT = 4,
-    MOE_OPT_GATHER = 5
+    MOE_OPT_GATHER = 5,
+    MOE_OPT_MX_BOX = 6
 } moe_option;
 int moe_set_option(int option, int value);
 

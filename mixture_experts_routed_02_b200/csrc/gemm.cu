@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(192, 1)
     // slower: with 76 of 148 CTAs in the last wave, 50 -> 64 us at one token.)
     constexpr int kQ = BN / 64;
     int full_tiles = tiles;
-    if constexpr (STAGE == 1 && !PAIR && kQ > 1) {
+    if (STAGE == 1 && !PAIR && kQ > 1 && (!MXW || args.b_box_rows == 64)) {  // (128-row copies: whole tiles)
         const int tail = tiles % (int)gridDim.x;
         if (tail > 0 && tail * kQ <= (int)gridDim.x) full_tiles = tiles - tail;
     }
@@ -345,12 +345,14 @@ __global__ void __launch_bounds__(192, 1)
             // B scale chunk of each 128-row block (512 bytes, already in the
             // layout TMEM takes)
             uint8_t* dst = smem + C::OFF_B + stage * C::B_BYTES;
-            const int half0 = (n * BN + (q4 >= 0 ? 64 * q4 : 0)) / 64;  // first 64-row half of the unit
-            const int boxes = (q4 >= 0) ? 1 : C::B_ROWS / 64;
+            const int box = args.b_box_rows;                            // 64 or 128 rows per copy
+            const int piece0 = (n * BN + (q4 >= 0 ? 64 * q4 : 0)) / box;  // first box of the unit
+            const int boxes = (q4 >= 0) ? 1 : C::B_ROWS / box;
             for (int j = 0; j < boxes; ++j) {
-                const int h = half0 + j;
-                const int brow = (int)((((size_t)e * b_nblk + h / 2) * args.k_tiles + kt) * kWBlockRows) + 64 * (h & 1);
-                tma_load_2d(dst + j * 64 * 128, &tmB, &full[stage], 0, brow, pol_b);
+                const int p = piece0 + j, per_blk = kWBlockRows / box;
+                const int brow = (int)((((size_t)e * b_nblk + p / per_blk) * args.k_tiles + kt) * kWBlockRows) +
+                                 box * (p % per_blk);
+                tma_load_2d(dst + j * box * 128, &tmB, &full[stage], 0, brow, pol_b);
             }
             const int rb0 = (n * BN + (q4 >= 0 ? 64 * q4 : 0)) / kWBlockRows;
             const int nchunks = (q4 >= 0) ? 1 : C::B_ROWS / kWBlockRows;

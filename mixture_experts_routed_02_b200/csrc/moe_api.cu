@@ -31,6 +31,7 @@ std::atomic<int> g_opt_timeout_ms{2000};
 std::atomic<int> g_opt_test_stall{0};
 std::atomic<int> g_opt_test_corrupt{0};
 std::atomic<int> g_opt_gather{0};
+std::atomic<int> g_opt_mx_box{0};
 
 // ---------------------------------------------------------------- profiling
 
@@ -299,10 +300,10 @@ struct MapKey {
     const void* ws;
     const void* w13;
     const void* w2;
-    int T, H, F, E, k, dtype, cfg1, cfg2;
+    int T, H, F, E, k, dtype, cfg1, cfg2, mx_box;
     bool operator==(const MapKey& o) const {
         return x == o.x && ws == o.ws && w13 == o.w13 && w2 == o.w2 && T == o.T && H == o.H && F == o.F && E == o.E &&
-               k == o.k && dtype == o.dtype && cfg1 == o.cfg1 && cfg2 == o.cfg2;
+               k == o.k && dtype == o.dtype && cfg1 == o.cfg1 && cfg2 == o.cfg2 && mx_box == o.mx_box;
     }
 };
 struct MapSet {
@@ -407,6 +408,9 @@ int moe_set_option(int option, int value) {
         case MOE_OPT_GATHER:
             if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
             return g_opt_gather.exchange(value);
+        case MOE_OPT_MX_BOX:
+            if (value != 0 && value != 64 && value != 128) return MOE_ERR_INVALID_ARG;
+            return g_opt_mx_box.exchange(value);
         default:
             return MOE_ERR_INVALID_ARG;
     }
@@ -545,7 +549,8 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
     // stage 1 gathers token rows: from the per-token e4m3 rows (FP8) or from
     // x itself (BF16), one-row boxes of 128 bytes
     const void* a1_base = fp8 ? (const void*)reg(MOE_WS_XS) : x;
-    const MapKey mkey{a1_base, ws, w13, w2, T, H, F, E, k, dtype, cfg1, cfg2};
+    const int mx_box = (g_opt_mx_box.load() == 64) ? 64 : 128;  // rows per copy of MX FP4 weights
+    const MapKey mkey{a1_base, ws, w13, w2, T, H, F, E, k, dtype, cfg1, cfg2, mx_box};
     MapSet ms;
     if (!find_maps(mkey, &ms)) {
         if (!make_map(&ms.tg1, a1_base, T, H, (size_t)H * eb, eb, 1) ||
@@ -555,8 +560,8 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
             !make_map(&ms.ta2s, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, 32))
             return MOE_ERR_CUDA;
         if (mxw) {
-            if (!make_map_fp4(&ms.tb1, w13, (size_t)E * 2 * F * (H / 128), 64) ||
-                !make_map_fp4(&ms.tb2, w2, (size_t)E * H * (F / 128), 64))
+            if (!make_map_fp4(&ms.tb1, w13, (size_t)E * 2 * F * (H / 128), mx_box) ||
+                !make_map_fp4(&ms.tb2, w2, (size_t)E * H * (F / 128), mx_box))
                 return MOE_ERR_CUDA;
         }
         if (cfg1 == 0 && !make_map_rows(&ms.tb1, w13, (size_t)E * (2 * F) * (H * eb / 128), kWBlockRows))
@@ -653,6 +658,7 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
     g1.num_experts = E;
     g1.mt_max = L.MT_max;
     g1.a_gather = tma_gather ? 1 : 0;
+    g1.b_box_rows = mx_box;
     g1.group_m = (cfg1 != 1) ? 1 : 0;
     {
         ProfScope ps(MOE_KERNEL_STAGE1, st);

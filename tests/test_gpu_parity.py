@@ -177,6 +177,21 @@ def test_layer_small_mxfp4(moe, p, gather):
     check_r0(moe, ws, case, nc, gather)
 
 
+@pytest.mark.parametrize("box", [64, 128])
+def test_layer_mxfp4_copy_rows(moe, box):
+    """MX FP4 weight copies of 64 rows (the first GEMM then cuts its last wave
+    into 64-row slices, whose B scales are half a 128-row chunk) and of 128
+    rows, at a decode shape whose last wave is lightly filled."""
+    old = moe.moe_set_option(moe.OPT_MX_BOX, box)
+    try:
+        T, H, F, E, k = 16, 256, 2560, 8, 2
+        case = small_case(T, H, F, E, k, "mxfp4", 38)
+        out, ws = run_layer(to_device(case))
+        verify_layer(moe, ws, out, case, what=f"mxfp4 copies of {box} rows")
+    finally:
+        moe.moe_set_option(moe.OPT_MX_BOX, old)
+
+
 def test_prepare_weights_mx_layout(moe):
     """moe_prepare_weights_mx: w13 rows interleaved in groups of 32 (w1 then
     w3), still packed, in contiguous blocks of 128 rows x 64 bytes ordered
