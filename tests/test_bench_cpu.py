@@ -52,7 +52,7 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     for d in ("mixture_experts_routed_02_b200/csrc", "include"):
         (root / d).mkdir(parents=True)
     for rel in ("mixture_experts_routed_02_b200/csrc/gemm.cu", "mixture_experts_routed_02_b200/csrc/kernels.cuh",
-                "mixture_experts_routed_02_b200/csrc/ptx.cuh", "include/moe.h"):
+                "mixture_experts_routed_02_b200/csrc/ptx.cuh"):
         shutil.copy(os.path.join(bench.ROOT, rel), root / rel)
     monkeypatch.setattr(bench, "ROOT", str(root))
     base = bench.source_sha()
