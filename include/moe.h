@@ -163,9 +163,11 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float
  * MOE_OPT_PATH asks).  BF16 mode: h is rounded to bf16.  The k
  * weighted expert outputs are summed in fp32 and rounded once to bf16.
  * Execution: five kernels (six from 1024 tokens on) chained on `stream` with
- * programmatic dependent launch -- routing, per-token quantisation, the first
- * group GEMM (which gathers each expert's token rows by TMA), the second group
- * GEMM with the scatter-add, and the bf16 rounding; to the rest of the stream
+ * programmatic dependent launch -- routing, the gather of each expert's token
+ * rows into the expert-padded layout (with their per-token quantisation), the
+ * first group GEMM, the second group GEMM with the scatter-add, and the bf16
+ * rounding (MOE_OPT_GATHER can instead let the first GEMM gather the rows
+ * itself by TMA after a quantisation pass); to the rest of the stream
  * the call is ordinary stream-ordered work (later work starts after `out` is
  * written).
  * The group GEMM tiles are chosen from the average rows per expert (see
@@ -297,7 +299,9 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
  *                     weight-streaming tiles (128 x 128 on one SM), 3 = force
  *                     128 x 256 tiles on one SM, 4 = force the tiny-batch
  *                     tiles (32 activation rows per stage; only for at most
- *                     32 assignments, else MOE_ERR_UNSUPPORTED).
+ *                     32 assignments, else MOE_ERR_UNSUPPORTED).  MX FP4
+ *                     weights run on 128 x 128 one-SM tiles only: 4 forces
+ *                     their tiny-batch form, 1-3 the other one.
  *   MOE_OPT_SPLITK:   0 = automatic, n > 0 = split the second GEMM's K into n parts
  *                     (must divide F/128).
  *   MOE_OPT_TIMEOUT_MS: limit of every device-side wait (default 2000).
@@ -323,9 +327,6 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
  *                     per-token quantisation pass, 2 = a gather pass writes
  *                     them into the expert-padded layout (MOE_WS_XG) and the
  *                     GEMM copies whole tiles.
- *   MOE_OPT_MX_BOX:   MX FP4 weights: rows per TMA copy of the packed weights,
- *                     0 = automatic (128), 64 or 128 (64-row copies also let
- *                     the first GEMM cut its last wave into 64-row slices).
  * Returns the previous value, or MOE_ERR_INVALID_ARG. */
 typedef enum {
     MOE_OPT_PATH = 0,
@@ -333,8 +334,7 @@ typedef enum {
     MOE_OPT_TIMEOUT_MS = 2,
     MOE_OPT_TEST_STALL = 3,
     MOE_OPT_TEST_CORRUPT = 4,
-    MOE_OPT_GATHER = 5,
-    MOE_OPT_MX_BOX = 6
+    MOE_OPT_GATHER = 5
 } moe_option;
 int moe_set_option(int option, int value);
 

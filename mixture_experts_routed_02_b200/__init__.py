@@ -45,7 +45,7 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
 MOE_BF16 = 0
 MOE_FP8_E4M3 = 1
 MOE_MXFP4 = 2
-OPT_PATH, OPT_SPLITK, OPT_TIMEOUT_MS, OPT_TEST_STALL, OPT_TEST_CORRUPT, OPT_GATHER, OPT_MX_BOX = range(7)
+OPT_PATH, OPT_SPLITK, OPT_TIMEOUT_MS, OPT_TEST_STALL, OPT_TEST_CORRUPT, OPT_GATHER = range(6)
 
 # workspace regions (moe_ws_region)
 WS = dict(topk_ids=0, topk_w=1, counts=2, offsets=3, perm=4, inv_perm=5, slot_of=6, xs=7, sx=8, h=9, h_sf=10,

@@ -20,7 +20,9 @@
 // Warp roles (192 threads): warp 0 lane 0 issues TMA loads into an NST-deep
 // shared-memory ring; warp 1 owns TMEM and lane 0 issues the MMAs; warps 2..5
 // drain the TMEM accumulators (double buffered where TMEM has room, so the
-// epilogue of one tile overlaps the main loop of the next).
+// epilogue of one tile overlaps the main loop of the next).  With MX FP4
+// weights warps 6 and 7 (256 threads) spread each stage's packed weight rows
+// into the 4-bit operand form before the stage counts as full.
 //
 // CTA pairs (PAIR): a cluster of two CTAs on two SMs computes a 256 x BN tile
 // with tcgen05.mma.cta_group::2.  Its two 128-row halves are two m-tiles of
@@ -55,11 +57,16 @@ struct Cfg {
     static constexpr int A_BYTES = AR * 128;
     static_assert(AR == kBlockM || (AR == 32 && !PAIR), "activation rows per stage");
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // weight rows held by one CTA
-    static constexpr int B_BYTES = B_ROWS * 128;       // shared memory (e2m1: one byte per element)
-    // bytes a weight row brings in: MX FP4 rows are copied packed (two codes
-    // per byte); in shared memory every 16 codes take 16 bytes (8 bytes of
-    // codes, 8 of padding: the 4-bit operand form of the block-scaled MMA)
-    static constexpr int B_ROW_TX = MXW ? 64 : 128;
+    static constexpr int B_BYTES = B_ROWS * 128;       // shared memory (e2m1: every 16 codes in 16 bytes)
+    // MX FP4 weights come in packed (two codes per byte, 64 bytes a row) into a
+    // staging ring that completes on its own barriers; two converter warps
+    // then write every 16 codes into 16 bytes of the operand (8 bytes of
+    // codes, 8 of padding: the 4-bit operand form of the block-scaled MMA) and
+    // arrive on the stage's full barrier.  So B adds no bytes to it.
+    static constexpr int B_ROW_TX = MXW ? 0 : 128;
+    static constexpr int STG_BYTES = MXW ? B_ROWS * 64 : 0;
+    static constexpr int NCONV = MXW ? 2 : 0;               // converter warps (6, 7)
+    static constexpr int THREADS = 192 + 32 * NCONV;
     static constexpr int SFA_BYTES = SFA_VAR ? 512 : 0;
     static constexpr int SFB_BYTES = SFB_VAR ? 512 * (B_ROWS / 128) : 0;
     // bytes that complete one stage: both CTAs' copies count on the even CTA's barrier
@@ -81,9 +88,10 @@ struct Cfg {
     static constexpr int OFF_B = NST * A_BYTES;
     static constexpr int OFF_SFA = OFF_B + NST * B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + NST * SFA_BYTES;
-    static constexpr int OFF_SFC = OFF_SFB + NST * SFB_BYTES;
+    static constexpr int OFF_STG = OFF_SFB + NST * SFB_BYTES;
+    static constexpr int OFF_SFC = OFF_STG + NST * STG_BYTES;
     static constexpr int OFF_BAR = OFF_SFC + (HAS_SFC ? 512 : 0);
-    static constexpr int NUM_BARS = 2 * NST + 5;
+    static constexpr int NUM_BARS = 2 * NST + 5 + (MXW ? NST : 0);
     static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;  // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
     static constexpr uint32_t IDESC = FP8 ? idesc_e4m3(MMA_M, BN) : idesc_bf16(MMA_M, BN);
@@ -106,7 +114,7 @@ __device__ __forceinline__ void decode_tile(int tile, int num_mt, int n_tiles, i
 }  // namespace
 
 template <int STAGE, bool FP8, int BN, int NST, int NACC, bool PAIR, int AR, bool MXW>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR, MXW>::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmSF,
                     const GemmArgs args) {
@@ -119,6 +127,7 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* tfull = bars + 2 * NST;
     uint64_t* tempty = bars + 2 * NST + 2;
     uint64_t* drain = bars + 2 * NST + 4;
+    uint64_t* raw = bars + 2 * NST + 5;  // MX FP4: packed weights landed in the staging ring
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -138,8 +147,9 @@ __global__ void __launch_bounds__(192, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NST; ++i) {
-            mbar_init(&full[i], 1);
+            mbar_init(&full[i], 1 + C::NCONV);  // (MX FP4: the producer and the converter warps)
             mbar_init(&empty[i], 1);
+            if constexpr (MXW) mbar_init(&raw[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
@@ -149,7 +159,7 @@ __global__ void __launch_bounds__(192, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (C::HAS_SFC && warp >= 2) {
+    if (C::HAS_SFC && warp >= 2 && warp < 6) {
         // constant UE8M0 scale 2^0 for every row of the operand without block
         // scales (FP8 stage 2: B, w2 has fp32 per-channel scales instead; MX
         // FP4 stage 1: A, the activations have one fp32 scale per token)
@@ -168,7 +178,7 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
         if constexpr (!PAIR) prefetch_tmap(&tmA32);
-        if constexpr (PAIR || MXW) prefetch_tmap(&tmB);
+        if constexpr (PAIR) prefetch_tmap(&tmB);
         if ((PAIR && C::SFA_VAR) || (STAGE == 1 && args.a_gather)) prefetch_tmap(&tmSF);
     }
     // Expert-major tile order: the first 128-row tile (and, for pairs, the
@@ -228,7 +238,7 @@ __global__ void __launch_bounds__(192, 1)
     // slower: with 76 of 148 CTAs in the last wave, 50 -> 64 us at one token.)
     constexpr int kQ = BN / 64;
     int full_tiles = tiles;
-    if (STAGE == 1 && !PAIR && kQ > 1 && (!MXW || args.b_box_rows == 64)) {  // (128-row copies: whole tiles)
+    if constexpr (STAGE == 1 && !PAIR && kQ > 1) {
         const int tail = tiles % (int)gridDim.x;
         if (tail > 0 && tail * kQ <= (int)gridDim.x) full_tiles = tiles - tail;
     }
@@ -339,20 +349,20 @@ __global__ void __launch_bounds__(192, 1)
     // tile, or this CTA's half of them in a pair.
     auto load_weights = [&](int stage, int e, int n, int kt, int q4) {
         if constexpr (MXW) {
-            // MX FP4: packed e2m1 rows by TMA from the blocked layout (each
-            // 64-row half of a 128-row x 64-byte block is 4 KB in one run; 16
-            // codes per 16 bytes of shared memory, 128-byte swizzle), then the
-            // B scale chunk of each 128-row block (512 bytes, already in the
-            // layout TMEM takes)
-            uint8_t* dst = smem + C::OFF_B + stage * C::B_BYTES;
-            const int box = args.b_box_rows;                            // 64 or 128 rows per copy
-            const int piece0 = (n * BN + (q4 >= 0 ? 64 * q4 : 0)) / box;  // first box of the unit
-            const int boxes = (q4 >= 0) ? 1 : C::B_ROWS / box;
-            for (int j = 0; j < boxes; ++j) {
-                const int p = piece0 + j, per_blk = kWBlockRows / box;
-                const int brow = (int)((((size_t)e * b_nblk + p / per_blk) * args.k_tiles + kt) * kWBlockRows) +
-                                 box * (p % per_blk);
-                tma_load_2d(dst + j * box * 128, &tmB, &full[stage], 0, brow, pol_b);
+            // MX FP4: the packed rows of each 128-row block of the unit (8 KB
+            // in one run in the blocked layout; a 64-row slice is half of one)
+            // by bulk copy into the staging ring, for the converter warps; then
+            // the B scale chunk of each 128-row block (512 bytes, already in
+            // the layout TMEM takes)
+            uint8_t* dst = smem + C::OFF_STG + stage * C::STG_BYTES;
+            const int row0 = n * BN + (q4 >= 0 ? 64 * q4 : 0);
+            const uint32_t bytes = (q4 >= 0) ? 64 * 64 : C::STG_BYTES;
+            mbar_arrive_expect_tx(&raw[stage], bytes);
+            for (int j = 0; j < (q4 >= 0 ? 1 : C::B_ROWS / kWBlockRows); ++j) {
+                const size_t blk = ((size_t)e * b_nblk + row0 / kWBlockRows + j) * args.k_tiles + kt;
+                const uint8_t* src = args.b_blocks + blk * (kWBlockRows * 64) + (row0 % kWBlockRows) * 64;
+                bulk_load_hint(dst + j * kWBlockRows * 64, src, q4 >= 0 ? 64 * 64 : kWBlockRows * 64, &raw[stage],
+                               pol_b);
             }
             const int rb0 = (n * BN + (q4 >= 0 ? 64 * q4 : 0)) / kWBlockRows;
             const int nchunks = (q4 >= 0) ? 1 : C::B_ROWS / kWBlockRows;
@@ -627,7 +637,62 @@ __global__ void __launch_bounds__(192, 1)
             mbar_wait(drain, 0, &keep_waiting, limit, args.status);
         }
         __syncwarp();
-    } else {
+    } else if (MXW && warp >= 6) {
+        // ---------------- converter warps (MX FP4 weights): each stage's
+        // packed rows (64 bytes = 128 codes) into the operand form, 16 codes
+        // per 16 bytes (codes first, then 8 bytes of padding), with the
+        // 128-byte swizzle of the K-major operand tile (16-byte chunk c of row
+        // r at r*128 + (c ^ (r % 8))*16); each warp takes half the rows, and
+        // every lane loads all its packed pieces before it stores, so the
+        // shared-memory latencies overlap.  Then the stage's full barrier
+        // hears from both warps.
+        constexpr int kConv = C::NCONV > 0 ? C::NCONV : 1;  // (the other kernels never come here)
+        constexpr int kMaxPieces = C::B_ROWS * 4 / (32 * kConv);  // 16-byte packed pieces per lane
+        const int cw = warp - 6;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int u = unit0; u < units && ok; u += ustep) {
+            int m, n, split, q4;
+            bool dup;
+            unit_coords(u, m, n, split, dup, q4);
+            const int pieces = ((q4 >= 0) ? 64 : C::B_ROWS) * 4 / kConv;  // this warp's pieces of the stage
+            const int p0 = cw * pieces;
+            for (int kk = 0; kk < kps; ++kk) {
+                if (!wait(&raw[stage], phase)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* stg = smem + C::OFF_STG + stage * C::STG_BYTES;
+                uint8_t* opb = smem + C::OFF_B + stage * C::B_BYTES;
+                uint4 v[kMaxPieces];
+#pragma unroll
+                for (int j = 0; j < kMaxPieces; ++j) {
+                    const int i = lane + 32 * j;
+                    if (i < pieces) v[j] = *reinterpret_cast<const uint4*>(stg + (p0 + i) * 16);
+                }
+#pragma unroll
+                for (int j = 0; j < kMaxPieces; ++j) {
+                    const int i = lane + 32 * j;
+                    if (i < pieces) {
+                        const int r = (p0 + i) >> 2, pc = (p0 + i) & 3;  // row, piece of 32 codes in it
+                        uint8_t* rowp = opb + r * 128;
+                        *reinterpret_cast<uint4*>(rowp + (((2 * pc) ^ (r & 7)) * 16)) = make_uint4(v[j].x, v[j].y, 0u, 0u);
+                        *reinterpret_cast<uint4*>(rowp + (((2 * pc + 1) ^ (r & 7)) * 16)) =
+                            make_uint4(v[j].z, v[j].w, 0u, 0u);
+                    }
+                }
+                fence_proxy_async_smem();  // the tensor core reads these bytes through the async proxy
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[stage]);
+                if (++stage == NST) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp < 6) {
         // ---------------- epilogue warps 2..5
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;
@@ -663,10 +728,10 @@ __global__ void __launch_bounds__(192, 1)
                         sxv = args.row_scale_slot[slot];
                     }
                 }
-#pragma unroll 1
                 // 64-column groups: all BN / 64 of a tile, or the one of a 64-row slice
                 const int g_first = (q4 >= 0) ? q4 : 0;
                 const int g_count = (q4 >= 0) ? 1 : BN / 64;
+#pragma unroll 1
                 for (int gi = 0; gi < g_count && !dup; ++gi) {
                     const int g = g_first + gi;
                     uint32_t rg[32], ru[32];
@@ -841,12 +906,12 @@ cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, int grid, cud
     if constexpr (PAIR) {
         if (grid < 2 || grid % 2) return cudaErrorInvalidValue;
         if (!maps.b) return cudaErrorInvalidValue;
-        return launch_dependent_cluster(kern, dim3(grid), dim3(192), C::SMEM_BYTES, 2, stream, *maps.a, *maps.a,
+        return launch_dependent_cluster(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, 2, stream, *maps.a, *maps.a,
                                         *maps.b, m4, args);
     } else {
-        if (!maps.a32 || (MXW && !maps.b)) return cudaErrorInvalidValue;
-        return launch_dependent(kern, dim3(grid), dim3(192), C::SMEM_BYTES, stream, *maps.a, *maps.a32,
-                                MXW ? *maps.b : *maps.a, m4, args);
+        if (!maps.a32) return cudaErrorInvalidValue;
+        return launch_dependent(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream, *maps.a, *maps.a32,
+                                *maps.a, m4, args);
     }
 }
 
@@ -856,7 +921,7 @@ int max_pairs_one() {
     auto kern = moe_gemm_kernel<STAGE, FP8, BN, NST, NACC, PAIR, AR, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return 0;
-    return max_active_clusters(kern, 192, C::SMEM_BYTES, 2);
+    return max_active_clusters(kern, C::THREADS, C::SMEM_BYTES, 2);
 }
 
 }  // namespace
@@ -874,18 +939,19 @@ int gemm_block_n(int stage, bool fp8, int cfg, bool mxw) {
 // for deeper pipelines -- stage 1 on 128 x 256 tiles, stage 2 on 128 x 128.
 // MX FP4 weights (mxw) run on 128 x 128 one-CTA tiles (two 128-column
 // accumulators leave room in TMEM for the per-stage scales of both operands):
-// cfg 1, or cfg 3 (at most 32 assignments in all) with 32 activation rows per
-// stage and 10 stages -- a stage of 4-bit weights brings only half the bytes
-// of an e4m3 one from HBM, so more stages keep enough in flight.
+// cfg 1 (5 stages), or cfg 3 (at most 32 assignments in all) with 32
+// activation rows per stage and 7 stages -- a stage of 4-bit weights brings
+// only half the bytes of an e4m3 one from HBM, so more stages keep enough in
+// flight (each stage also holds the packed rows, 8 KB).
 cudaError_t launch_gemm(int stage, bool fp8, int cfg, const GemmMaps& maps, const GemmArgs& args, int grid,
                         cudaStream_t stream, bool mxw) {
     if (mxw) {
         if ((cfg != 1 && cfg != 3) || !fp8) return cudaErrorInvalidValue;
         if (cfg == 3)
-            return stage == 1 ? launch_one<1, true, 128, 10, 2, false, 32, true>(maps, args, grid, stream)
-                              : launch_one<2, true, 128, 10, 2, false, 32, true>(maps, args, grid, stream);
-        return stage == 1 ? launch_one<1, true, 128, 6, 2, false, kBlockM, true>(maps, args, grid, stream)
-                          : launch_one<2, true, 128, 6, 2, false, kBlockM, true>(maps, args, grid, stream);
+            return stage == 1 ? launch_one<1, true, 128, 7, 2, false, 32, true>(maps, args, grid, stream)
+                              : launch_one<2, true, 128, 7, 2, false, 32, true>(maps, args, grid, stream);
+        return stage == 1 ? launch_one<1, true, 128, 5, 2, false, kBlockM, true>(maps, args, grid, stream)
+                          : launch_one<2, true, 128, 5, 2, false, kBlockM, true>(maps, args, grid, stream);
     }
     if (cfg == 3) {
         if (stage == 1)

@@ -171,7 +171,6 @@ struct GemmArgs {
     int mt_max;               // bound of *num_mtiles (a larger value is a corrupted table)
     int a_gather;             // stage 1: 1 = gather token rows by TMA (tile::gather4); 0 = tile copies of
                               // the rows a gather pass wrote in the expert-padded layout
-    int b_box_rows;           // MX FP4 weights: rows per TMA copy of the packed weights (64 or 128)
     // d_ff-sharded layer, stage 2: with n_ranks > 0 token t's row is added into
     // the combine rows of the rank that owns it (t / rows_per_rank), at
     // peer_out[owner] + (t - owner * rows_per_rank) * H, through peer memory

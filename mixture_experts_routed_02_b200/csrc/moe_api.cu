@@ -31,7 +31,6 @@ std::atomic<int> g_opt_timeout_ms{2000};
 std::atomic<int> g_opt_test_stall{0};
 std::atomic<int> g_opt_test_corrupt{0};
 std::atomic<int> g_opt_gather{0};
-std::atomic<int> g_opt_mx_box{0};
 
 // ---------------------------------------------------------------- profiling
 
@@ -254,24 +253,6 @@ bool make_map(CUtensorMap* map, const void* base, size_t rows, size_t cols, size
     return r == CUDA_SUCCESS;
 }
 
-// Map of the blocked MX FP4 weights seen as rows of 128 packed e2m1 codes (64
-// bytes each; see moe_prepare_weights_mx) whose copies put every 16 codes into
-// 16 bytes of shared memory, 8 of codes and 8 of padding (the 4-bit operand
-// form of the block-scaled MMA): box_rows rows per copy, 128-byte swizzle.
-bool make_map_fp4(CUtensorMap* map, const void* base, size_t rows, int box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const size_t cols = 128;
-    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)(cols / 2)};
-    const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box,
-                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 // Map of a buffer of 128-byte rows copied as they are (no swizzle), box_rows
 // rows per copy: the preshuffled weight blocks (already in the operand's
 // shared-memory image) and the tiled scale chunks of h.
@@ -300,10 +281,10 @@ struct MapKey {
     const void* ws;
     const void* w13;
     const void* w2;
-    int T, H, F, E, k, dtype, cfg1, cfg2, mx_box;
+    int T, H, F, E, k, dtype, cfg1, cfg2;
     bool operator==(const MapKey& o) const {
         return x == o.x && ws == o.ws && w13 == o.w13 && w2 == o.w2 && T == o.T && H == o.H && F == o.F && E == o.E &&
-               k == o.k && dtype == o.dtype && cfg1 == o.cfg1 && cfg2 == o.cfg2 && mx_box == o.mx_box;
+               k == o.k && dtype == o.dtype && cfg1 == o.cfg1 && cfg2 == o.cfg2;
     }
 };
 struct MapSet {
@@ -408,9 +389,6 @@ int moe_set_option(int option, int value) {
         case MOE_OPT_GATHER:
             if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
             return g_opt_gather.exchange(value);
-        case MOE_OPT_MX_BOX:
-            if (value != 0 && value != 64 && value != 128) return MOE_ERR_INVALID_ARG;
-            return g_opt_mx_box.exchange(value);
         default:
             return MOE_ERR_INVALID_ARG;
     }
@@ -535,9 +513,10 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
         cfg1 = cfg2 = opt_path - 1;
     }
     // MX FP4 weights: 128 x 128 one-CTA tiles (room in TMEM for both operands'
-    // scales), with 32 activation rows per stage and deeper pipelines when the
-    // whole batch has at most 32 assignments
-    if (mxw) cfg1 = cfg2 = (L.A <= 32) ? 3 : 1;
+    // scales); the tiny-batch form (32 activation rows per stage, deeper
+    // pipelines) only when forced: at 16 tokens it measured 284 us a layer
+    // against 274 us for the 128-row form
+    if (mxw) cfg1 = cfg2 = (opt_path == 4) ? 3 : 1;
     if ((2 * F) % gemm_block_n(1, fp8, cfg1, mxw)) cfg1 = 1;
     if (H % gemm_block_n(2, fp8, cfg2, mxw)) cfg2 = 1;
     if (cfg1 == 0 && max_pairs(1, fp8) < 1) cfg1 = 2;
@@ -549,8 +528,7 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
     // stage 1 gathers token rows: from the per-token e4m3 rows (FP8) or from
     // x itself (BF16), one-row boxes of 128 bytes
     const void* a1_base = fp8 ? (const void*)reg(MOE_WS_XS) : x;
-    const int mx_box = (g_opt_mx_box.load() == 64) ? 64 : 128;  // rows per copy of MX FP4 weights
-    const MapKey mkey{a1_base, ws, w13, w2, T, H, F, E, k, dtype, cfg1, cfg2, mx_box};
+    const MapKey mkey{a1_base, ws, w13, w2, T, H, F, E, k, dtype, cfg1, cfg2};
     MapSet ms;
     if (!find_maps(mkey, &ms)) {
         if (!make_map(&ms.tg1, a1_base, T, H, (size_t)H * eb, eb, 1) ||
@@ -559,11 +537,6 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
             !make_map(&ms.ta2, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, kBlockM) ||
             !make_map(&ms.ta2s, reg(MOE_WS_H), L.S_max, F, act_pitch((long)F * eb), eb, 32))
             return MOE_ERR_CUDA;
-        if (mxw) {
-            if (!make_map_fp4(&ms.tb1, w13, (size_t)E * 2 * F * (H / 128), mx_box) ||
-                !make_map_fp4(&ms.tb2, w2, (size_t)E * H * (F / 128), mx_box))
-                return MOE_ERR_CUDA;
-        }
         if (cfg1 == 0 && !make_map_rows(&ms.tb1, w13, (size_t)E * (2 * F) * (H * eb / 128), kWBlockRows))
             return MOE_ERR_CUDA;
         if (cfg2 == 0 && !make_map_rows(&ms.tb2, w2, (size_t)E * H * (F * eb / 128), kWBlockRows))
@@ -579,8 +552,8 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
     // gather pass is the default (MOE_OPT_GATHER selects either).
     const int opt_gather = g_opt_gather.load();
     const bool tma_gather = (opt_gather == 1);
-    const GemmMaps maps1{&ms.ta1, &ms.ta1s, (cfg1 == 0 || mxw) ? &ms.tb1 : nullptr, tma_gather ? &ms.tg1 : nullptr};
-    const GemmMaps maps2{&ms.ta2, &ms.ta2s, (cfg2 == 0 || mxw) ? &ms.tb2 : nullptr,
+    const GemmMaps maps1{&ms.ta1, &ms.ta1s, cfg1 == 0 ? &ms.tb1 : nullptr, tma_gather ? &ms.tg1 : nullptr};
+    const GemmMaps maps2{&ms.ta2, &ms.ta2s, cfg2 == 0 ? &ms.tb2 : nullptr,
                          (cfg2 == 0 && fp8) ? &ms.tsf2 : nullptr};
     // grid: one CTA per SM at most; pairs: whole clusters that can be resident
     auto grid_for = [&](int stage, int c, long units_per_mtile) {
@@ -658,7 +631,6 @@ int forward_impl(const void* x, const float* logits, const void* w13, const void
     g1.num_experts = E;
     g1.mt_max = L.MT_max;
     g1.a_gather = tma_gather ? 1 : 0;
-    g1.b_box_rows = mx_box;
     g1.group_m = (cfg1 != 1) ? 1 : 0;
     {
         ProfScope ps(MOE_KERNEL_STAGE1, st);

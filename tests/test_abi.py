@@ -149,8 +149,7 @@ def test_test_hook_options_range(moe):
     assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, 0) == 0
     assert moe.moe_set_option(moe.OPT_GATHER, 3) == -1
     assert moe.moe_set_option(moe.OPT_GATHER, 0) == 0
-    assert moe.moe_set_option(moe.OPT_MX_BOX, 32) == -1
-    assert moe.moe_set_option(moe.OPT_MX_BOX, 0) == 0
+    assert moe.moe_set_option(6, 0) == -1  # no option 6
 
 
 def test_dff_entry_checks_arguments(moe):

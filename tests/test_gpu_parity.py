@@ -157,7 +157,7 @@ MXFP4 = [
     # (T, H, F, E, k, seed, skew): MX FP4 weights run on 128 x 128 one-CTA tiles
     (64, 256, 512, 8, 2, 30, False),
     (1, 256, 512, 8, 2, 31, False),
-    (16, 256, 512, 8, 2, 32, False),       # decode-shaped: 32 activation rows per stage
+    (16, 256, 512, 8, 2, 32, False),       # decode-shaped (32 assignments)
     (200, 384, 640, 8, 2, 33, False),      # several m-tiles, ragged tails, odd multiples of 128
     (300, 256, 512, 8, 2, 34, True),       # skewed: big and empty experts
     (37, 128, 256, 1, 1, 35, False),       # E = 1, k = 1
@@ -166,9 +166,13 @@ MXFP4 = [
 
 
 @GATHER
+@pytest.mark.parametrize("path", [0, 4], ids=["auto_tiles", "tiny_tiles"])
 @pytest.mark.parametrize("p", MXFP4, ids=lambda p: f"T{p[0]}_H{p[1]}_F{p[2]}_E{p[3]}_k{p[4]}" + ("_skew" if p[6] else ""))
-def test_layer_small_mxfp4(moe, p, gather):
+def test_layer_small_mxfp4(moe, p, path, gather):
     T, H, F, E, k, seed, skew = p
+    if path == 4 and T * k > 32:
+        pytest.skip("the tiny-batch tiles take at most 32 assignments")
+    moe.moe_set_option(moe.OPT_PATH, path)
     moe.moe_set_option(moe.OPT_GATHER, gather)
     case = small_case(T, H, F, E, k, "mxfp4", seed, skew)
     nc = moe_inputs.to_numpy(case)
@@ -177,19 +181,14 @@ def test_layer_small_mxfp4(moe, p, gather):
     check_r0(moe, ws, case, nc, gather)
 
 
-@pytest.mark.parametrize("box", [64, 128])
-def test_layer_mxfp4_copy_rows(moe, box):
-    """MX FP4 weight copies of 64 rows (the first GEMM then cuts its last wave
-    into 64-row slices, whose B scales are half a 128-row chunk) and of 128
-    rows, at a decode shape whose last wave is lightly filled."""
-    old = moe.moe_set_option(moe.OPT_MX_BOX, box)
-    try:
-        T, H, F, E, k = 16, 256, 2560, 8, 2
-        case = small_case(T, H, F, E, k, "mxfp4", 38)
-        out, ws = run_layer(to_device(case))
-        verify_layer(moe, ws, out, case, what=f"mxfp4 copies of {box} rows")
-    finally:
-        moe.moe_set_option(moe.OPT_MX_BOX, old)
+def test_layer_mxfp4_sliced_last_wave(moe):
+    """MX FP4 at a decode shape whose last wave of first-GEMM tiles is lightly
+    filled, so that wave runs as 64-row slices: each slice's packed rows are
+    half of a 128-row block and its B scales half of a 128-row chunk."""
+    T, H, F, E, k = 16, 256, 2560, 8, 2
+    case = small_case(T, H, F, E, k, "mxfp4", 38)
+    out, ws = run_layer(to_device(case))
+    verify_layer(moe, ws, out, case, what="mxfp4 sliced last wave")
 
 
 def test_prepare_weights_mx_layout(moe):
