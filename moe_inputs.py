@@ -24,6 +24,7 @@ prefill_mxfp4  4096   4096   14336  8   2  mxfp4  6     MX FP4 expert weights
 =============  =====  =====  =====  ==  =  =====  ====  =================================
 
 Distributions: x ~ N(0,1) rounded to bf16; router logits ~ N(0,1) fp32;
+upstream gradient of the backward pass dy ~ N(0,1) rounded to bf16;
 weights ~ N(0, 0.02^2) rounded to bf16 (and quantised per output channel for
 fp8).  Every draw comes from its own torch CPU generator seeded with
 ``seed * 1000 + stream`` so that each tensor can be regenerated alone.
@@ -54,7 +55,7 @@ CONFIGS["decode_mxfp4"] = _spec(16, H_MIXTRAL, F_MIXTRAL, 8, 2, "mxfp4", 5)
 CONFIGS["prefill_mxfp4"] = _spec(4096, H_MIXTRAL, F_MIXTRAL, 8, 2, "mxfp4", 6)
 
 # stream ids of the generators
-_S_X, _S_LOGITS, _S_W1, _S_W3, _S_W2 = range(5)
+_S_X, _S_LOGITS, _S_W1, _S_W3, _S_W2, _S_DY = range(6)
 
 
 def _gen(seed, stream):
@@ -68,6 +69,11 @@ def skew_bias(E):
 
 def make_x(T, H, seed):
     return torch.randn(T, H, generator=_gen(seed, _S_X)).to(torch.bfloat16)
+
+
+def make_dy(T, H, seed):
+    """Upstream gradient of the layer output for the backward pass: N(0,1) -> bf16 [T,H]."""
+    return torch.randn(T, H, generator=_gen(seed, _S_DY)).to(torch.bfloat16)
 
 
 def make_logits(T, E, seed, skew=False):

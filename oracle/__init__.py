@@ -19,7 +19,12 @@ step it follows:
 * ``moe_ffn``      -- the whole layer, routed or masked-dense form (paragraph 2
                       and timestamp 5:56: gather, group GEMM, SwiGLU, scatter
                       versus the masked dense GEMM path);
-* ``moe_ffn_tokens`` -- the same layer evaluated on a subset of tokens.
+* ``moe_ffn_tokens`` -- the same layer evaluated on a subset of tokens;
+* ``ffn64``, ``ffn_bwd64``, ``ffn_bwd64_sampled`` -- the BF16 layer on fp64
+                      inputs and its gradients (the custom VJP for training
+                      that timestamp 10:07 names as the next step): dx, dw1,
+                      dw3, dw2 and the router logits' gradient, in full or
+                      sampled at full size.
 
 Parity of these functions with the pages is pinned by ``tests/test_oracle.py``.
 """
@@ -83,6 +88,13 @@ def _load():
         lib.oracle_moe_ffn_tokens.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, I, P, P, P, P, I]
         lib.oracle_max_threads.restype = I
         lib.oracle_max_threads.argtypes = []
+        lib.oracle_moe_ffn64.restype = I
+        lib.oracle_moe_ffn64.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, I]
+        lib.oracle_moe_ffn_bwd64.restype = I
+        lib.oracle_moe_ffn_bwd64.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, P, P, I]
+        lib.oracle_moe_ffn_bwd64_sampled.restype = I
+        lib.oracle_moe_ffn_bwd64_sampled.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, I, P, P, P, I, P, P, P,
+                                                     I]
         _lib = lib
     return _lib
 
@@ -238,3 +250,67 @@ def bf16_bits_to_float(b):
     """uint16 bf16 bit patterns -> float64 values (exact widening)."""
     b = np.asarray(b, dtype=np.uint16)
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# -- backward (custom VJP) of the BF16 layer -------------------------------
+
+def bf16_bits_to_f64(bits):
+    """bf16 bit patterns (uint16) -> float64 values (exact)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _dims64(x, w1, logits, k):
+    T, H = x.shape
+    E, F, H1 = w1.shape
+    if H1 != H or logits.shape != (T, E) or not 1 <= k <= E:
+        raise ValueError("inconsistent shapes")
+    return T, H, F, E
+
+
+def ffn64(x, logits, w1, w3, w2, k, round_h=False, nthreads=0):
+    """The layer on fp64 inputs: y [T,H] fp64 (not rounded); h rounded to bf16
+    when round_h, as the BF16 forward does."""
+    x, lg, w1, w3, w2 = (_c(a, np.float64) for a in (x, logits, w1, w3, w2))
+    T, H, F, E = _dims64(x, w1, lg, k)
+    y = np.zeros((T, H))
+    rc = _load().oracle_moe_ffn64(_ptr(x), _ptr(lg), _ptr(w1), _ptr(w3), _ptr(w2), T, H, F, E, k, int(round_h),
+                                  _ptr(y), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_moe_ffn64: bad arguments")
+    return y
+
+
+def ffn_bwd64(x, logits, w1, w3, w2, dy, k, round_h=True, nthreads=0):
+    """Gradients of <dy, layer(x)>: dict(dx [T,H], dw1 [E,F,H], dw3 [E,F,H],
+    dw2 [E,H,F], dlogits [T,E], dwa [T,k] routing-weight gradients), fp64."""
+    x, lg, w1, w3, w2, dy = (_c(a, np.float64) for a in (x, logits, w1, w3, w2, dy))
+    T, H, F, E = _dims64(x, w1, lg, k)
+    out = dict(dx=np.zeros((T, H)), dw1=np.zeros((E, F, H)), dw3=np.zeros((E, F, H)), dw2=np.zeros((E, H, F)),
+               dlogits=np.zeros((T, E)), dwa=np.zeros(max(T * k, 1)))
+    rc = _load().oracle_moe_ffn_bwd64(_ptr(x), _ptr(lg), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(dy), T, H, F, E, k,
+                                      int(round_h), _ptr(out["dx"]), _ptr(out["dw1"]), _ptr(out["dw3"]),
+                                      _ptr(out["dw2"]), _ptr(out["dlogits"]), _ptr(out["dwa"]), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_moe_ffn_bwd64: bad arguments")
+    out["dwa"] = out["dwa"][:T * k].reshape(T, k)
+    return out
+
+
+def ffn_bwd64_sampled(x, logits, w1, w3, w2, dy, k, tokens, feats, round_h=True, nthreads=0):
+    """Sampled gradients: dx [ntok,H] and dlogits [ntok,E] of the listed
+    tokens; for each (e, n) in feats, dw1[e, n, :], dw3[e, n, :] and
+    dw2[e, :, n] ([nfeat,H] each)."""
+    x, lg, w1, w3, w2, dy = (_c(a, np.float64) for a in (x, logits, w1, w3, w2, dy))
+    T, H, F, E = _dims64(x, w1, lg, k)
+    tok = _c(tokens, np.int32).reshape(-1)
+    ft = _c(feats, np.int32).reshape(-1, 2)
+    out = dict(dx=np.zeros((len(tok), H)), dlogits=np.zeros((len(tok), E)), dw1=np.zeros((len(ft), H)),
+               dw3=np.zeros((len(ft), H)), dw2=np.zeros((len(ft), H)))
+    rc = _load().oracle_moe_ffn_bwd64_sampled(_ptr(x), _ptr(lg), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(dy), T, H, F, E,
+                                              k, int(round_h), _ptr(tok), len(tok), _ptr(out["dx"]),
+                                              _ptr(out["dlogits"]), _ptr(ft), len(ft), _ptr(out["dw1"]),
+                                              _ptr(out["dw3"]), _ptr(out["dw2"]), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_moe_ffn_bwd64_sampled: bad arguments")
+    return out

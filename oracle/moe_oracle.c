@@ -35,6 +35,10 @@
  *     shares; x and h are quantised as in FP8 mode;
  *   - the combine is an fp64 sum, rounded once to bf16.
  *
+ * The last section holds the backward pass (custom VJP) of the BF16 layer on
+ * fp64 inputs: the gradients of <dy, out> with respect to x, w1, w3, w2 and
+ * the router logits (timestamp 10:07 names it as the next step).
+ *
  * Build: gcc -O2 -fopenmp -shared -fPIC -fno-fast-math -ffp-contract=off moe_oracle.c
  *        -o liboracle.so -lm
  */
@@ -499,4 +503,324 @@ int oracle_max_threads(void) {
 #else
     return 1;
 #endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* Backward (custom VJP) of the BF16 layer, fp64.                           */
+/* ------------------------------------------------------------------------ */
+/*
+ * The pages list a custom VJP for training as the next step of the routed
+ * kernel (rocketrecap.com "FlyDSL kernels in JAX", timestamp 10:07) and do not
+ * define it; what is computed here is the gradient of the BF16 layer above
+ * with respect to x, w1, w3, w2 and the router logits, for an upstream
+ * gradient dy = dL/dout.  For each assignment a = (t, j) of token t to expert
+ * e with routing weight w_a:
+ *
+ *   g = W1_e x_t,  u = W3_e x_t,  h = silu(g) * u   (rounded to bf16 when
+ *       round_h, as the forward rounds it; the rounding passes gradients
+ *       through unchanged),  o = W2_e h
+ *   dw_a = <dy_t, o>,   dO = w_a dy_t,   dh = W2_e^T dO
+ *   du = dh * silu(g),  dg = dh * u * silu'(g),  silu'(g) = s(g) (1 + g (1 - s(g)))
+ *       with s the logistic function
+ *   dx_t  += W1_e^T dg + W3_e^T du
+ *   dW1_e += dg x_t^T,  dW3_e += du x_t^T,  dW2_e += dO h^T
+ *
+ * Router: w = softmax over the k chosen logits, so for the chosen experts
+ * dlogit[t, e_j] = w_j (dw_j - sum_i w_i dw_i), and 0 for the others (the
+ * choice itself is piecewise constant in the logits).
+ *
+ * Inputs are fp64 so that finite differences can perturb them.  The choice of
+ * experts follows the forward's ranking rule (larger logit first, lower index
+ * on a tie, NaN as -inf); gradients are defined for finite logits.
+ */
+
+typedef struct {
+    const double *x, *w1, *w3, *w2;  /* [T,H], [E,F,H], [E,F,H], [E,H,F] */
+    int T, H, F, E, k, round_h;
+} bctx;
+
+static double ranked64(double l) { return isnan(l) ? -INFINITY : l; }
+
+/* top-k and the softmax over the chosen logits of one token (fp64 logits) */
+static void topk64(const double* l, int E, int k, int32_t* ids, double* w) {
+    char chosen[64];
+    memset(chosen, 0, sizeof(chosen));
+    for (int j = 0; j < k; ++j) {
+        int best = -1;
+        for (int e = 0; e < E; ++e) {
+            if (chosen[e]) continue;
+            if (best < 0 || ranks_before(ranked64(l[e]), e, ranked64(l[best]), best)) best = e;
+        }
+        chosen[best] = 1;
+        ids[j] = best;
+    }
+    double lmax = ranked64(l[ids[0]]);
+    if (isinf(lmax)) {
+        int n = 0;
+        for (int j = 0; j < k; ++j) n += (ranked64(l[ids[j]]) == lmax);
+        for (int j = 0; j < k; ++j) w[j] = (ranked64(l[ids[j]]) == lmax) ? 1.0 / n : 0.0;
+        return;
+    }
+    double den = 0.0;
+    for (int j = 0; j < k; ++j) den += exp(ranked64(l[ids[j]]) - lmax);
+    for (int j = 0; j < k; ++j) w[j] = exp(ranked64(l[ids[j]]) - lmax) / den;
+}
+
+static int bctx_init(bctx* c, const double* x, const double* w1, const double* w3, const double* w2, int T,
+                     int H, int F, int E, int k, int round_h) {
+    if (T < 0 || H < 1 || F < 1 || E < 1 || E > 64 || k < 1 || k > E) return -1;
+    c->x = x; c->w1 = w1; c->w3 = w3; c->w2 = w2;
+    c->T = T; c->H = H; c->F = F; c->E = E; c->k = k; c->round_h = round_h;
+    return 0;
+}
+
+/* g, u, h [F] and o [H] of token t through expert e */
+static void fwd_assign(const bctx* c, int e, int t, double* g, double* u, double* h, double* o) {
+    int H = c->H, F = c->F;
+    const double* xt = c->x + (size_t)t * H;
+    for (int n = 0; n < F; ++n) {
+        const double* r1 = c->w1 + ((size_t)e * F + n) * H;
+        const double* r3 = c->w3 + ((size_t)e * F + n) * H;
+        double gv = 0.0, uv = 0.0;
+        for (int i = 0; i < H; ++i) {
+            gv += r1[i] * xt[i];
+            uv += r3[i] * xt[i];
+        }
+        double hv = gv / (1.0 + exp(-gv)) * uv;
+        if (c->round_h) hv = oracle_bf16_to_double(oracle_bf16_from_double(hv));
+        g[n] = gv; u[n] = uv; h[n] = hv;
+    }
+    for (int m = 0; m < H; ++m) {
+        const double* r2 = c->w2 + ((size_t)e * H + m) * F;
+        double acc = 0.0;
+        for (int n = 0; n < F; ++n) acc += r2[n] * h[n];
+        o[m] = acc;
+    }
+}
+
+/* dg, du [F] from dh and the forward values */
+static void swiglu_bwd(int F, const double* g, const double* u, const double* dh, double* dg, double* du) {
+    for (int n = 0; n < F; ++n) {
+        double s = 1.0 / (1.0 + exp(-g[n]));
+        du[n] = dh[n] * (g[n] / (1.0 + exp(-g[n])));
+        dg[n] = dh[n] * u[n] * (s * (1.0 + g[n] * (1.0 - s)));
+    }
+}
+
+/* y [T,H] (fp64, not rounded) of the layer on fp64 inputs; the combine adds
+ * each token's expert outputs in ascending expert order, as the routed form */
+int oracle_moe_ffn64(const double* x, const double* logits, const double* w1, const double* w3, const double* w2,
+                     int T, int H, int F, int E, int k, int round_h, double* y, int nthreads) {
+    bctx c;
+    if (bctx_init(&c, x, w1, w3, w2, T, H, F, E, k, round_h)) return -1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < T; ++t) {
+        int32_t ids[64];
+        double w[64];
+        double *g = malloc(sizeof(double) * F), *u = malloc(sizeof(double) * F), *h = malloc(sizeof(double) * F);
+        double** o = malloc(sizeof(double*) * k);
+        topk64(logits + (size_t)t * E, E, k, ids, w);
+        for (int j = 0; j < k; ++j) {
+            o[j] = malloc(sizeof(double) * H);
+            fwd_assign(&c, ids[j], t, g, u, h, o[j]);
+        }
+        for (int m = 0; m < H; ++m) {
+            double acc = 0.0;
+            for (int e = 0; e < E; ++e)
+                for (int j = 0; j < k; ++j)
+                    if (ids[j] == e) acc += w[j] * o[j][m];
+            y[(size_t)t * H + m] = acc;
+        }
+        for (int j = 0; j < k; ++j) free(o[j]);
+        free(o); free(g); free(u); free(h);
+    }
+    return 0;
+}
+
+/* Full gradients: dx [T,H], dw1/dw3 [E,F,H], dw2 [E,H,F], dlogits [T,E]; dwa
+ * (optional) [T*k] the gradients of the routing weights.  Experts run in
+ * parallel; inside one, assignments in ascending order. */
+int oracle_moe_ffn_bwd64(const double* x, const double* logits, const double* w1, const double* w3,
+                         const double* w2, const double* dy, int T, int H, int F, int E, int k, int round_h,
+                         double* dx, double* dw1, double* dw3, double* dw2, double* dlogits, double* dwa_out,
+                         int nthreads) {
+    bctx c;
+    if (bctx_init(&c, x, w1, w3, w2, T, H, F, E, k, round_h)) return -1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+    long A = (long)T * k;
+    int32_t* ids = malloc(sizeof(int32_t) * (A ? A : 1));
+    double* w = malloc(sizeof(double) * (A ? A : 1));
+    double* dwa = calloc(A ? A : 1, sizeof(double));
+    double* dxa = calloc((size_t)(A ? A : 1) * H, sizeof(double));
+    for (int t = 0; t < T; ++t) topk64(logits + (size_t)t * E, E, k, ids + (size_t)t * k, w + (size_t)t * k);
+    memset(dw1, 0, sizeof(double) * (size_t)E * F * H);
+    memset(dw3, 0, sizeof(double) * (size_t)E * F * H);
+    memset(dw2, 0, sizeof(double) * (size_t)E * H * F);
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int e = 0; e < E; ++e) {
+        double *g = malloc(sizeof(double) * F), *u = malloc(sizeof(double) * F), *h = malloc(sizeof(double) * F);
+        double *dh = malloc(sizeof(double) * F), *dg = malloc(sizeof(double) * F), *du = malloc(sizeof(double) * F);
+        double *o = malloc(sizeof(double) * H), *dO = malloc(sizeof(double) * H);
+        for (long a = 0; a < A; ++a) {
+            if (ids[a] != e) continue;
+            int t = (int)(a / k);
+            const double* dyt = dy + (size_t)t * H;
+            const double* xt = x + (size_t)t * H;
+            fwd_assign(&c, e, t, g, u, h, o);
+            double s = 0.0;
+            for (int m = 0; m < H; ++m) s += dyt[m] * o[m];
+            dwa[a] = s;
+            for (int m = 0; m < H; ++m) dO[m] = w[a] * dyt[m];
+            for (int n = 0; n < F; ++n) {
+                double acc = 0.0;
+                for (int m = 0; m < H; ++m) acc += w2[((size_t)e * H + m) * F + n] * dO[m];
+                dh[n] = acc;
+            }
+            swiglu_bwd(F, g, u, dh, dg, du);
+            double* dxr = dxa + (size_t)a * H;
+            for (int i = 0; i < H; ++i) {
+                double acc = 0.0;
+                for (int n = 0; n < F; ++n)
+                    acc += w1[((size_t)e * F + n) * H + i] * dg[n] + w3[((size_t)e * F + n) * H + i] * du[n];
+                dxr[i] = acc;
+            }
+            for (int n = 0; n < F; ++n) {
+                double* r1 = dw1 + ((size_t)e * F + n) * H;
+                double* r3 = dw3 + ((size_t)e * F + n) * H;
+                for (int i = 0; i < H; ++i) {
+                    r1[i] += dg[n] * xt[i];
+                    r3[i] += du[n] * xt[i];
+                }
+            }
+            for (int m = 0; m < H; ++m) {
+                double* r2 = dw2 + ((size_t)e * H + m) * F;
+                for (int n = 0; n < F; ++n) r2[n] += dO[m] * h[n];
+            }
+        }
+        free(g); free(u); free(h); free(dh); free(dg); free(du); free(o); free(dO);
+    }
+    for (int t = 0; t < T; ++t) {
+        for (int i = 0; i < H; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < k; ++j) acc += dxa[((size_t)t * k + j) * H + i];
+            dx[(size_t)t * H + i] = acc;
+        }
+        double sw = 0.0;
+        for (int j = 0; j < k; ++j) sw += w[(size_t)t * k + j] * dwa[(size_t)t * k + j];
+        for (int e = 0; e < E; ++e) dlogits[(size_t)t * E + e] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            size_t a = (size_t)t * k + j;
+            dlogits[(size_t)t * E + ids[a]] = w[a] * (dwa[a] - sw);
+        }
+    }
+    if (dwa_out) memcpy(dwa_out, dwa, sizeof(double) * A);
+    free(ids); free(w); free(dwa); free(dxa);
+    return 0;
+}
+
+/* Sampled gradients, for sizes where the full form takes too long: dx and
+ * dlogits of the listed tokens ([ntok,H], [ntok,E]); for each listed pair
+ * (e, n) of feats [nfeat,2], row n of dW1_e and of dW3_e and column n of
+ * dW2_e ([nfeat,H] each).  Same arithmetic and order as the full form. */
+int oracle_moe_ffn_bwd64_sampled(const double* x, const double* logits, const double* w1, const double* w3,
+                                 const double* w2, const double* dy, int T, int H, int F, int E, int k,
+                                 int round_h, const int32_t* tokens, int ntok, double* dx_s, double* dl_s,
+                                 const int32_t* feats, int nfeat, double* dw1_s, double* dw3_s, double* dw2_s,
+                                 int nthreads) {
+    bctx c;
+    if (bctx_init(&c, x, w1, w3, w2, T, H, F, E, k, round_h)) return -1;
+    for (int i = 0; i < ntok; ++i)
+        if (tokens[i] < 0 || tokens[i] >= T) return -1;
+    for (int i = 0; i < nfeat; ++i)
+        if (feats[2 * i] < 0 || feats[2 * i] >= E || feats[2 * i + 1] < 0 || feats[2 * i + 1] >= F) return -1;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+    long A = (long)T * k;
+    int32_t* ids = malloc(sizeof(int32_t) * (A ? A : 1));
+    double* w = malloc(sizeof(double) * (A ? A : 1));
+    for (int t = 0; t < T; ++t) topk64(logits + (size_t)t * E, E, k, ids + (size_t)t * k, w + (size_t)t * k);
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int q = 0; q < ntok; ++q) {
+        int t = tokens[q];
+        const double* dyt = dy + (size_t)t * H;
+        double *g = malloc(sizeof(double) * F), *u = malloc(sizeof(double) * F), *h = malloc(sizeof(double) * F);
+        double *dh = malloc(sizeof(double) * F), *dg = malloc(sizeof(double) * F), *du = malloc(sizeof(double) * F);
+        double *o = malloc(sizeof(double) * H), *dO = malloc(sizeof(double) * H);
+        double* dxa = calloc((size_t)k * H, sizeof(double));
+        double dwa[64];
+        for (int j = 0; j < k; ++j) {
+            size_t a = (size_t)t * k + j;
+            int e = ids[a];
+            fwd_assign(&c, e, t, g, u, h, o);
+            double s = 0.0;
+            for (int m = 0; m < H; ++m) s += dyt[m] * o[m];
+            dwa[j] = s;
+            for (int m = 0; m < H; ++m) dO[m] = w[a] * dyt[m];
+            for (int n = 0; n < F; ++n) {
+                double acc = 0.0;
+                for (int m = 0; m < H; ++m) acc += w2[((size_t)e * H + m) * F + n] * dO[m];
+                dh[n] = acc;
+            }
+            swiglu_bwd(F, g, u, dh, dg, du);
+            for (int i = 0; i < H; ++i) {
+                double acc = 0.0;
+                for (int n = 0; n < F; ++n)
+                    acc += w1[((size_t)e * F + n) * H + i] * dg[n] + w3[((size_t)e * F + n) * H + i] * du[n];
+                dxa[(size_t)j * H + i] = acc;
+            }
+        }
+        for (int i = 0; i < H; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < k; ++j) acc += dxa[(size_t)j * H + i];
+            dx_s[(size_t)q * H + i] = acc;
+        }
+        double sw = 0.0;
+        for (int j = 0; j < k; ++j) sw += w[(size_t)t * k + j] * dwa[j];
+        for (int e = 0; e < E; ++e) dl_s[(size_t)q * E + e] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            size_t a = (size_t)t * k + j;
+            dl_s[(size_t)q * E + ids[a]] = w[a] * (dwa[j] - sw);
+        }
+        free(g); free(u); free(h); free(dh); free(dg); free(du); free(o); free(dO); free(dxa);
+    }
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int q = 0; q < nfeat; ++q) {
+        int e = feats[2 * q], n = feats[2 * q + 1];
+        double* r1 = dw1_s + (size_t)q * H;
+        double* r3 = dw3_s + (size_t)q * H;
+        double* c2 = dw2_s + (size_t)q * H;
+        for (int i = 0; i < H; ++i) r1[i] = r3[i] = c2[i] = 0.0;
+        const double* w1r = w1 + ((size_t)e * F + n) * H;
+        const double* w3r = w3 + ((size_t)e * F + n) * H;
+        for (long a = 0; a < A; ++a) {
+            if (ids[a] != e) continue;
+            int t = (int)(a / k);
+            const double* xt = x + (size_t)t * H;
+            const double* dyt = dy + (size_t)t * H;
+            double gv = 0.0, uv = 0.0;
+            for (int i = 0; i < H; ++i) {
+                gv += w1r[i] * xt[i];
+                uv += w3r[i] * xt[i];
+            }
+            double hv = gv / (1.0 + exp(-gv)) * uv;
+            if (round_h) hv = oracle_bf16_to_double(oracle_bf16_from_double(hv));
+            double dhv = 0.0;
+            for (int m = 0; m < H; ++m) dhv += w2[((size_t)e * H + m) * F + n] * (w[a] * dyt[m]);
+            double dgv, duv;
+            swiglu_bwd(1, &gv, &uv, &dhv, &dgv, &duv);
+            for (int i = 0; i < H; ++i) {
+                r1[i] += dgv * xt[i];
+                r3[i] += duv * xt[i];
+            }
+            for (int m = 0; m < H; ++m) c2[m] += (w[a] * dyt[m]) * hv;
+        }
+    }
+    free(ids); free(w);
+    return 0;
 }

@@ -499,3 +499,140 @@ def test_per_assignment_intermediates(dtype):
                 e, codes = oracle.mx_quant_block(hb[b:b + 32])
                 np.testing.assert_array_equal([oracle.e4m3_to_double(c) * 2.0 ** e for c in codes],
                                               sub["h_deq"][a][b:b + 32])
+
+
+# ---------------------------------------------------------------- backward (custom VJP)
+
+def _bwd_inputs(T, H, F, E, seed, wscale=0.3):
+    rng = np.random.default_rng(seed)
+    return dict(x=rng.standard_normal((T, H)), logits=rng.standard_normal((T, E)),
+                w1=rng.standard_normal((E, F, H)) * wscale, w3=rng.standard_normal((E, F, H)) * wscale,
+                w2=rng.standard_normal((E, H, F)) * wscale, dy=rng.standard_normal((T, H)))
+
+
+def test_ffn64_equals_forward_oracle_on_bf16_inputs():
+    """The fp64-input layer with h rounded to bf16 is the BF16 forward oracle
+    (pinned above) on bf16-representable inputs: the same sums in the same
+    order, so equal to the last bit."""
+    case = moe_inputs.make_case(23, 128, 256, 8, 2, "bf16", 41)
+    nc = moe_inputs.to_numpy(case)
+    ref = oracle.moe_ffn(nc)["out64"]
+    f = oracle.bf16_bits_to_f64
+    y = oracle.ffn64(f(nc["x"]), nc["logits"].astype(np.float64), f(nc["w1"]), f(nc["w3"]), f(nc["w2"]), 2,
+                     round_h=True)
+    np.testing.assert_array_equal(y, ref)
+
+
+@pytest.mark.parametrize("T,H,F,E,k", [(5, 8, 12, 4, 2), (3, 6, 10, 3, 3), (4, 8, 8, 1, 1)])
+def test_bwd_matches_finite_differences(T, H, F, E, k):
+    """Every entry of dx, dw1, dw3, dw2 and dlogits against a central
+    difference of L = <dy, layer(x)> (fp64, h not rounded), step 1e-6: a
+    dropped term, a sign, a transposed operand or a wrong index fails."""
+    d = _bwd_inputs(T, H, F, E, seed=7 * T + E)
+    g = oracle.ffn_bwd64(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], k, round_h=False)
+    names = ["x", "logits", "w1", "w3", "w2"]
+    grads = {"x": "dx", "logits": "dlogits", "w1": "dw1", "w3": "dw3", "w2": "dw2"}
+    eps = 1e-6
+
+    def loss(args):
+        return float((oracle.ffn64(*(args[n] for n in names), k) * d["dy"]).sum())
+
+    for n in names:
+        for idx in np.ndindex(d[n].shape):
+            p = {m: d[m] for m in names}
+            p[n] = d[n].copy()
+            p[n][idx] += eps
+            lp = loss(p)
+            p[n][idx] -= 2 * eps
+            lm = loss(p)
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - g[grads[n]][idx]) < 1e-7 * (1 + abs(fd)), (n, idx, fd, g[grads[n]][idx])
+
+
+def test_bwd_dense_mlp_against_autograd():
+    """E = 1, k = 1: the layer is a dense SwiGLU MLP with routing weight 1;
+    its gradients from torch.autograd (fp64) and dlogits = 0."""
+    T, H, F = 9, 16, 24
+    d = _bwd_inputs(T, H, F, 1, seed=3)
+    g = oracle.ffn_bwd64(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], 1, round_h=False)
+    x, w1, w3, w2 = (torch.tensor(d[n], requires_grad=True) for n in ("x", "w1", "w3", "w2"))
+    y = (torch.nn.functional.silu(x @ w1[0].T) * (x @ w3[0].T)) @ w2[0].T
+    (y * torch.tensor(d["dy"])).sum().backward()
+    for mine, lib in ((g["dx"], x.grad), (g["dw1"], w1.grad), (g["dw3"], w3.grad), (g["dw2"], w2.grad)):
+        np.testing.assert_allclose(mine, lib.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.all(g["dlogits"] == 0.0)
+
+
+def test_bwd_all_experts_chosen_against_autograd():
+    """k = E: every expert is chosen and the weights are the softmax over all
+    logits, so the layer is sum_e softmax(l)_e FFN_e(x); torch.autograd of
+    that (fp64) gives every gradient, the logits' included."""
+    T, H, F, E = 7, 12, 20, 3
+    d = _bwd_inputs(T, H, F, E, seed=11)
+    g = oracle.ffn_bwd64(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], E, round_h=False)
+    x, lg, w1, w3, w2 = (torch.tensor(d[n], requires_grad=True) for n in ("x", "logits", "w1", "w3", "w2"))
+    p = torch.softmax(lg, dim=1)
+    y = sum(p[:, e:e + 1] * ((torch.nn.functional.silu(x @ w1[e].T) * (x @ w3[e].T)) @ w2[e].T) for e in range(E))
+    (y * torch.tensor(d["dy"])).sum().backward()
+    for mine, lib in ((g["dx"], x.grad), (g["dlogits"], lg.grad), (g["dw1"], w1.grad), (g["dw3"], w3.grad),
+                      (g["dw2"], w2.grad)):
+        np.testing.assert_allclose(mine, lib.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_bwd_router_gradient_invariants():
+    """Softmax is invariant to a shift of the chosen logits: each token's
+    logit gradients sum to 0; experts not chosen get exactly 0; and dlogit_j =
+    w_j (dw_j - sum_i w_i dw_i) with dw_a = <dy_t, expert output>."""
+    T, H, F, E, k = 40, 16, 32, 8, 2
+    d = _bwd_inputs(T, H, F, E, seed=5)
+    g = oracle.ffn_bwd64(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], k)
+    np.testing.assert_allclose(g["dlogits"].sum(axis=1), 0.0, atol=1e-12)
+    r = oracle.route(d["logits"].astype(np.float32), k)
+    for t in range(T):
+        chosen = set(r["ids"][t].tolist())
+        for e in range(E):
+            if e not in chosen:
+                assert g["dlogits"][t, e] == 0.0
+    # dw_a from the expert outputs y_e computed by the forward with one-hot logits
+    big = 1e4
+    for t in range(0, T, 7):
+        for j in range(k):
+            e = int(r["ids"][t, j])
+            onehot = np.full((1, E), -big)
+            onehot[0, e] = 0.0
+            ye = oracle.ffn64(d["x"][t:t + 1], onehot, d["w1"], d["w3"], d["w2"], 1, round_h=True)
+            assert abs(g["dwa"][t, j] - float(ye[0] @ d["dy"][t])) < 1e-12 * (1 + abs(g["dwa"][t, j]))
+
+
+def test_bwd_rounded_h_close_to_exact():
+    """Rounding h to bf16 (the forward's intermediate) moves the gradients by
+    about the bf16 unit (2^-9 relative) and no more."""
+    d = _bwd_inputs(30, 16, 32, 4, seed=9)
+    a = oracle.ffn_bwd64(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], 2, round_h=True)
+    b = oracle.ffn_bwd64(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], 2, round_h=False)
+    for n in ("dx", "dw1", "dw3", "dw2", "dlogits"):
+        rel = np.linalg.norm(a[n] - b[n]) / np.linalg.norm(b[n])
+        assert rel < 2.0 ** -8, (n, rel)
+    # dx, dw1 and dw3 see h only through dw_a (the router) -- not at all with k = 1 and E = 1
+    d1 = _bwd_inputs(10, 8, 16, 1, seed=2)
+    a1 = oracle.ffn_bwd64(d1["x"], d1["logits"], d1["w1"], d1["w3"], d1["w2"], d1["dy"], 1, round_h=True)
+    b1 = oracle.ffn_bwd64(d1["x"], d1["logits"], d1["w1"], d1["w3"], d1["w2"], d1["dy"], 1, round_h=False)
+    for n in ("dx", "dw1", "dw3"):
+        np.testing.assert_array_equal(a1[n], b1[n])
+
+
+def test_bwd_sampled_equals_full():
+    """The sampled form (used at full size) gives the full form's values for
+    the rows and columns it samples, to the last bit."""
+    T, H, F, E, k = 33, 16, 24, 4, 2
+    d = _bwd_inputs(T, H, F, E, seed=13)
+    full = oracle.ffn_bwd64(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], k)
+    tok = np.array([0, 5, 32, 17], dtype=np.int32)
+    feats = np.array([[0, 0], [3, 23], [2, 7], [1, 11]], dtype=np.int32)
+    s = oracle.ffn_bwd64_sampled(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], k, tok, feats)
+    np.testing.assert_array_equal(s["dx"], full["dx"][tok])
+    np.testing.assert_array_equal(s["dlogits"], full["dlogits"][tok])
+    for q, (e, n) in enumerate(feats):
+        np.testing.assert_array_equal(s["dw1"][q], full["dw1"][e, n])
+        np.testing.assert_array_equal(s["dw3"][q], full["dw3"][e, n])
+        np.testing.assert_array_equal(s["dw2"][q], full["dw2"][e, :, n])
