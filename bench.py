@@ -561,7 +561,7 @@ def run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_s
     # ---------------- roofline of the dominant kernel
     peaks, peak_kind = load_peaks()
     alg = algorithmic(spec, counts)
-    names = moe.KERNELS
+    names = moe.FWD_KERNELS
     dom = max(names, key=lambda n: kern[n][0])
     dom_ms = kern[dom][0] / max(1, kern[dom][1])
     roof = roofline(spec, alg, dom, dom_ms, ms_total, peaks, peak_kind, name)

@@ -339,9 +339,11 @@ typedef enum {
 int moe_set_option(int option, int value);
 
 /* Per-kernel device timing (tracing aid).  While enabled, moe_ffn_forward
- * records a pair of CUDA events around each step it enqueues (routing is one
- * kernel for small batches and two from 1024 tokens on; both are counted in
- * `launches` and timed together).
+ * and moe_ffn_backward record a pair of CUDA events around each step they
+ * enqueue (routing is one kernel for small batches and two from 1024 tokens
+ * on; both are counted in `launches` and timed together; the backward's
+ * routing, gathers, transposes, rounding of dx and router gradient are timed
+ * together as MOE_KERNEL_BWD_AUX).
  * moe_profile_enable returns the previous setting.  moe_profile_read waits for
  * the recorded events, adds up the elapsed time per kernel into
  * ms_total[MOE_KERNEL_COUNT] and the number of launches into
@@ -353,10 +355,64 @@ typedef enum {
     MOE_KERNEL_STAGE1 = 2, /* group GEMM with w1/w3 + SwiGLU */
     MOE_KERNEL_STAGE2 = 3, /* group GEMM with w2 + weighted scatter-add */
     MOE_KERNEL_FINALIZE = 4,
-    MOE_KERNEL_COUNT = 5
+    MOE_KERNEL_BWD_GU = 5,   /* backward: g, u, h recomputed (group GEMM with w1/w3) */
+    MOE_KERNEL_BWD_DH = 6,   /* backward: dh = W2^T dy -> dg, du, routing-weight gradients */
+    MOE_KERNEL_BWD_DX = 7,   /* backward: dx = W1^T dg + W3^T du, scatter-add per token */
+    MOE_KERNEL_BWD_DW2 = 8,  /* backward: dW2 per expert */
+    MOE_KERNEL_BWD_DW13 = 9, /* backward: dW1, dW3 per expert */
+    MOE_KERNEL_BWD_AUX = 10, /* backward: routing, gathers, transposes, dx rounding, router gradient */
+    MOE_KERNEL_COUNT = 11
 } moe_kernel_id;
 int moe_profile_enable(int on);
 int moe_profile_read(double* ms_total, int* launches, int reset);
+
+/*
+ * Backward pass (custom VJP) of the BF16 layer, for training.  The pages name
+ * a custom VJP as the next step of the routed kernel without defining it
+ * (rocketrecap.com "FlyDSL kernels in JAX", timestamp 10:07); this is the
+ * gradient of the BF16 layer of moe_ffn_forward (h rounded to bf16 there;
+ * the rounding passes gradients through unchanged) for an upstream gradient
+ * dy = dL/dout.  For each assignment a = (t, j) of token t to expert e with
+ * routing weight w_a, g = W1_e x_t, u = W3_e x_t, h = silu(g) u:
+ *   dw_a = <dy_t, W2_e h>,  dh = w_a W2_e^T dy_t,  du = dh silu(g),
+ *   dg = dh u s(g) (1 + g (1 - s(g)))  (s the logistic function),
+ *   dx_t = sum_j (W1_e^T dg + W3_e^T du),
+ *   dW1_e = sum dg x_t^T,  dW3_e = sum du x_t^T,  dW2_e = sum w_a dy_t h^T,
+ *   dlogits[t, e_j] = w_j (dw_j - sum_i w_i dw_i) for the chosen experts, 0
+ *   for the others (the routing weights are the softmax over the chosen
+ *   logits; the choice is piecewise constant).
+ * g and u are recomputed from x and w1/w3 (the forward keeps no
+ * intermediates).  Arithmetic: bf16 operands, fp32 accumulation; g, u, h, dg,
+ * du, w_a dy_t are rounded to bf16 where they are stored between kernels; dx
+ * is summed over the k experts in fp32 and rounded once.
+ *
+ * moe_backward_workspace_size: bytes of `ws` for moe_ffn_backward (0 if the
+ *   dimensions are unsupported: bf16 only, d_model and d_ff multiples of 128,
+ *   1 <= E <= 64, 1 <= k <= min(E, 8)).
+ * moe_prepare_weights_bwd: the transposed weight copies the backward reads,
+ *   bf16, device pointers, enqueued on `stream`:
+ *     w13t [E, H, 2F]: w13t[e][h][f] = w1[e][f][h], w13t[e][h][F + f] = w3[e][f][h]
+ *     w2t  [E, F, H]:  w2t[e][f][h] = w2[e][h][f]
+ *   from w1, w3 [E, F, H] and w2 [E, H, F] (row-major, as moe_prepare_weights
+ *   takes them).  Redo after every weight update.  All pointers 16-byte
+ *   aligned (MOE_ERR_ALIGNMENT), the buffers the caller's; nothing is freed.
+ * moe_ffn_backward: x [T, H], dy [T, H] bf16, logits [T, E] fp32 (finite),
+ *   w1, w3 [E, F, H] bf16 (row-major, as given to moe_prepare_weights),
+ *   w13t, w2t from moe_prepare_weights_bwd; outputs dx [T, H] bf16, dw1, dw3
+ *   [E, F, H] and dw2 [E, H, F] bf16 (fully written: zero for an expert with
+ *   no tokens), dlogits [T, E] fp32.  Device pointers, 16-byte aligned
+ *   (logits and dlogits 4-byte); ws >= moe_backward_workspace_size bytes.
+ *   Enqueued on `stream` (no host synchronisation; may be captured in a CUDA
+ *   graph).  Returns MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_ALIGNMENT,
+ *   MOE_ERR_WORKSPACE or MOE_ERR_CUDA (a launch failed; device-side faults
+ *   surface through moe_get_status as for the forward).
+ */
+size_t moe_backward_workspace_size(int T, int H, int F, int E, int k);
+int moe_prepare_weights_bwd(const void* w1, const void* w3, const void* w2, void* w13t_out, void* w2t_out, int E,
+                            int F, int H, void* stream);
+int moe_ffn_backward(const void* x, const float* logits, const void* w1, const void* w3, const void* w13t,
+                     const void* w2t, const void* dy, int T, int H, int F, int E, int k, void* dx, void* dw1,
+                     void* dw3, void* dw2, float* dlogits, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -17,6 +17,7 @@
 #include <mutex>
 #include <vector>
 
+#include "bwd.cuh"
 #include "kernels.cuh"
 
 namespace moe {
@@ -756,6 +757,292 @@ int moe_get_status(void* stream) {
     const int zero = 0;
     if (cudaMemcpy(ctx.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
     return v;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- backward pass
+// Workspace: the forward layout of the BF16 layer (routing tables, gathered x,
+// h, the fp32 row buffer -- here dx32) followed by the backward's own regions.
+
+namespace {
+
+enum BwdRegion { kBwGU = 0, kBwDYG, kBwDGU, kBwDOT, kBwXT, kBwHT, kBwDW, kBwRegions };
+
+struct BwdLayout {
+    Layout fwd;
+    size_t off[kBwRegions];
+    size_t total;
+};
+
+BwdLayout make_bwd_layout(int T, int H, int F, int E, int k) {
+    BwdLayout B{};
+    B.fwd = make_layout(T, H, F, E, k, MOE_BF16);
+    const size_t S = B.fwd.S_max;
+    size_t sz[kBwRegions];
+    sz[kBwGU] = S * act_pitch(4L * F);  // g|u rows [S, 2F]; later dg|du transposed [2F, S]
+    sz[kBwDYG] = S * act_pitch(2L * H);  // dy gathered into the slot layout [S, H]
+    sz[kBwDGU] = S * act_pitch(4L * F);  // dg|du [S, 2F]
+    sz[kBwDOT] = (size_t)H * S * 2;      // (w_a dy_t) transposed [H, S]
+    sz[kBwXT] = (size_t)H * S * 2;       // x transposed [H, S]
+    sz[kBwHT] = (size_t)F * S * 2;       // h transposed [F, S]
+    sz[kBwDW] = 4 * (size_t)B.fwd.A;     // routing-weight gradients
+    size_t off = B.fwd.total;
+    for (int r = 0; r < kBwRegions; ++r) {
+        B.off[r] = off;
+        off = align_up(off + sz[r], 1024);
+    }
+    B.total = off;
+    return B;
+}
+
+bool bwd_dims_ok(int T, int H, int F, int E, int k) {
+    return dims_ok(T, H, F, E, k, MOE_BF16) && H % 128 == 0 && F % 128 == 0;
+}
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_backward_workspace_size(int T, int H, int F, int E, int k) {
+    if (!bwd_dims_ok(T, H, F, E, k)) return 0;
+    return make_bwd_layout(T, H, F, E, k).total;
+}
+
+int moe_prepare_weights_bwd(const void* w1, const void* w3, const void* w2, void* w13t_out, void* w2t_out, int E,
+                            int F, int H, void* stream) {
+    if (E < 1 || E > kMaxExperts || F <= 0 || H <= 0 || F % 128 || H % 128) return MOE_ERR_INVALID_ARG;
+    if (!w1 || !w3 || !w2 || !w13t_out || !w2t_out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w1) || !aligned16(w3) || !aligned16(w2) || !aligned16(w13t_out) || !aligned16(w2t_out))
+        return MOE_ERR_ALIGNMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TransposeArgs p{};
+    // w13t[e][h][c] = w1[e][c][h] (c < F), w3[e][c - F][h] (c >= F)
+    p.src_pitch = H;
+    p.src_batch = (long)F * H;
+    p.rows = F;
+    p.out = w13t_out;
+    p.out_pitch = 2L * F;
+    p.out_batch = 2L * F * H;
+    p.src = w1;
+    p.out_col = 0;
+    if (launch_transpose(kSrcRows, p, H, F, E, st) != cudaSuccess) return MOE_ERR_CUDA;
+    p.src = w3;
+    p.out_col = F;
+    if (launch_transpose(kSrcRows, p, H, F, E, st) != cudaSuccess) return MOE_ERR_CUDA;
+    // w2t[e][f][h] = w2[e][h][f]
+    TransposeArgs q{};
+    q.src = w2;
+    q.src_pitch = F;
+    q.src_batch = (long)H * F;
+    q.rows = H;
+    q.out = w2t_out;
+    q.out_pitch = H;
+    q.out_batch = (long)F * H;
+    if (launch_transpose(kSrcRows, q, F, H, E, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int moe_ffn_backward(const void* x, const float* logits, const void* w1, const void* w3, const void* w13t,
+                     const void* w2t, const void* dy, int T, int H, int F, int E, int k, void* dx, void* dw1,
+                     void* dw3, void* dw2, float* dlogits, void* ws, size_t ws_bytes, void* stream) {
+    if (!bwd_dims_ok(T, H, F, E, k)) return MOE_ERR_INVALID_ARG;
+    if (!w1 || !w3 || !w13t || !w2t || !dw1 || !dw3 || !dw2 || !ws) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !logits || !dy || !dx || !dlogits)) return MOE_ERR_INVALID_ARG;
+    for (const void* ptr : {(const void*)w1, w3, w13t, w2t, (const void*)dw1, (const void*)dw3, (const void*)dw2,
+                            (const void*)ws})
+        if (!aligned16(ptr)) return MOE_ERR_ALIGNMENT;
+    if (T > 0 && (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || !aligned4(logits) || !aligned4(dlogits)))
+        return MOE_ERR_ALIGNMENT;
+    const BwdLayout B = make_bwd_layout(T, H, F, E, k);
+    const Layout& L = B.fwd;
+    if (ws_bytes < B.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {  // no tokens: every weight gradient is zero
+        const size_t n = (size_t)E * F * H * 2;
+        if (cudaMemsetAsync(dw1, 0, n, st) != cudaSuccess || cudaMemsetAsync(dw3, 0, n, st) != cudaSuccess ||
+            cudaMemsetAsync(dw2, 0, n, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    CtxInfo ctx{};
+    if (context_info(&ctx) != MOE_OK) return MOE_ERR_CUDA;
+    int* status = ctx.status;
+    const int num_sms = ctx.num_sms;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    auto reg = [&](int r) { return w + L.off[r]; };
+    auto breg = [&](int r) { return w + B.off[r]; };
+    const int S = L.S_max;
+    const unsigned long long timeout_ns = (unsigned long long)g_opt_timeout_ms.load() * 1000000ull;
+
+    // 1. the forward's routing and slot layout, x and dy gathered into it
+    RouteOutputs o{reinterpret_cast<int32_t*>(reg(MOE_WS_TOPK_IDS)), reinterpret_cast<float*>(reg(MOE_WS_TOPK_W)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_COUNTS)), reinterpret_cast<int32_t*>(reg(MOE_WS_OFFSETS)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_PERM)), reinterpret_cast<int32_t*>(reg(MOE_WS_INV_PERM)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_SLOT_OF)), reinterpret_cast<int32_t*>(reg(MOE_WS_SLOT_ASSIGN)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_MTILE_EXPERT)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_NUM_MTILES)),
+                   reinterpret_cast<int32_t*>(reg(MOE_WS_ROUTE_BLOCKS))};
+    float* dx32 = reinterpret_cast<float*>(reg(MOE_WS_OUT32));
+    float* dwa = reinterpret_cast<float*>(breg(kBwDW));
+    {
+        ProfScope ps(MOE_KERNEL_BWD_AUX, st, route_launches(T, o) + 2);
+        if (launch_route(logits, T, E, k, o, st) != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_gather(false, static_cast<const __nv_bfloat16*>(x), T, H, k, o.slot_of, S, reg(MOE_WS_XG), nullptr,
+                          nullptr, nullptr, status, st) != cudaSuccess ||
+            launch_gather(false, static_cast<const __nv_bfloat16*>(dy), T, H, k, o.slot_of, S, breg(kBwDYG), nullptr,
+                          nullptr, nullptr, status, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(dx32, 0, (size_t)T * H * 4, st) != cudaSuccess ||
+            cudaMemsetAsync(dwa, 0, (size_t)L.A * 4, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+
+    // tensor maps: K-major bf16 operands, 64-element x 128-row boxes
+    CUtensorMap mXg, mW1, mW3, mDyg, mW2t, mDgu, mW13t, mDot, mHt, mDgut, mXt;
+    const long p2H = act_pitch(2L * H), p4F = act_pitch(4L * F), p2F = act_pitch(2L * F);
+    if (!make_map(&mXg, reg(MOE_WS_XG), S, H, p2H, 2, 128) ||
+        !make_map(&mW1, w1, (size_t)E * F, H, (size_t)H * 2, 2, 128) ||
+        !make_map(&mW3, w3, (size_t)E * F, H, (size_t)H * 2, 2, 128) ||
+        !make_map(&mDyg, breg(kBwDYG), S, H, p2H, 2, 128) ||
+        !make_map(&mW2t, w2t, (size_t)E * F, H, (size_t)H * 2, 2, 128) ||
+        !make_map(&mDgu, breg(kBwDGU), S, 2L * F, p4F, 2, 128) ||
+        !make_map(&mW13t, w13t, (size_t)E * H, 2L * F, (size_t)F * 4, 2, 128) ||
+        !make_map(&mDot, breg(kBwDOT), H, S, (size_t)S * 2, 2, 128) ||
+        !make_map(&mHt, breg(kBwHT), F, S, (size_t)S * 2, 2, 128) ||
+        !make_map(&mDgut, breg(kBwGU), 2L * F, S, (size_t)S * 2, 2, 128) ||
+        !make_map(&mXt, breg(kBwXT), H, S, (size_t)S * 2, 2, 128))
+        return MOE_ERR_CUDA;
+
+    BwdArgs base{};
+    base.num_mtiles = o.num_mtiles;
+    base.mtile_expert = o.mtile_expert;
+    base.slot_assign = o.slot_assign;
+    base.counts = o.counts;
+    base.topk_w = o.topk_w;
+    base.num_experts = E;
+    base.mt_max = L.MT_max;
+    base.topk = k;
+    base.T = T;
+    base.F = F;
+    base.timeout_ns = timeout_ns;
+    base.status = status;
+    auto row_grid = [&](int n_tiles) { return (int)std::min<long>((long)L.MT_max * n_tiles, num_sms); };
+
+    // 2. g, u, h recomputed
+    {
+        BwdArgs a = base;
+        a.n_tiles = F / 128;
+        a.k_tiles = H / 64;
+        a.b_rows = F;
+        a.out = breg(kBwGU);
+        a.out_pitch = p4F;
+        a.out2 = reg(MOE_WS_H);
+        a.out2_pitch = p2F;
+        ProfScope ps(MOE_KERNEL_BWD_GU, st);
+        if (launch_bwd_gemm(kBwdGU, 256, mXg, mW1, mW3, a, row_grid(a.n_tiles), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    // 3. dh -> dg, du and the routing-weight gradients
+    {
+        const int bn = (F % 256 == 0) ? 256 : 128;
+        BwdArgs a = base;
+        a.n_tiles = F / bn;
+        a.k_tiles = H / 64;
+        a.b_rows = F;
+        a.out = breg(kBwDGU);
+        a.out_pitch = p4F;
+        a.gu = breg(kBwGU);
+        a.gu_pitch = p4F;
+        a.hbuf = reg(MOE_WS_H);
+        a.h_pitch = p2F;
+        a.dw = dwa;
+        ProfScope ps(MOE_KERNEL_BWD_DH, st);
+        if (launch_bwd_gemm(kBwdDH, bn, mDyg, mW2t, mW2t, a, row_grid(a.n_tiles), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    // 4. dx: the k experts' contributions meet in fp32, then one rounding
+    {
+        const int bn = (H % 256 == 0) ? 256 : 128;
+        BwdArgs a = base;
+        a.n_tiles = H / bn;
+        a.k_tiles = 2 * F / 64;
+        a.b_rows = H;
+        a.out = dx32;
+        a.out_pitch = (long)H * 4;
+        ProfScope ps(MOE_KERNEL_BWD_DX, st);
+        if (launch_bwd_gemm(kBwdDX, bn, mDgu, mW13t, mW13t, a, row_grid(a.n_tiles), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    {
+        ProfScope ps(MOE_KERNEL_BWD_AUX, st, 5);
+        if (launch_finalize(dx32, static_cast<__nv_bfloat16*>(dx), (size_t)T * H, num_sms, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        // transposed operands of the weight gradients: w_a dy_t and x_t per slot, h
+        TransposeArgs p{};
+        p.num_mtiles = o.num_mtiles;
+        p.mt_max = L.MT_max;
+        p.slot_assign = o.slot_assign;
+        p.num_assign = L.A;
+        p.topk = k;
+        p.out_pitch = S;
+        p.status = status;
+        p.src = dy;
+        p.src_pitch = H;
+        p.scale = o.topk_w;
+        p.out = breg(kBwDOT);
+        if (launch_transpose(kSrcTokens, p, H, S, 1, st) != cudaSuccess) return MOE_ERR_CUDA;
+        p.src = x;
+        p.scale = nullptr;
+        p.out = breg(kBwXT);
+        if (launch_transpose(kSrcTokens, p, H, S, 1, st) != cudaSuccess) return MOE_ERR_CUDA;
+        p.src = reg(MOE_WS_H);
+        p.src_pitch = p2F / 2;
+        p.out = breg(kBwHT);
+        if (launch_transpose(kSrcSlots, p, F, S, 1, st) != cudaSuccess) return MOE_ERR_CUDA;
+        // dg|du transposed, over g|u (read by step 3 only)
+        p.src = breg(kBwDGU);
+        p.src_pitch = p4F / 2;
+        p.out = breg(kBwGU);
+        if (launch_transpose(kSrcSlots, p, 2 * F, S, 1, st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    // 5. dW2_e = (w dy)^T h and [dW1_e; dW3_e] = [dg; du]^T x over each expert's slots
+    {
+        const int bn = (F % 256 == 0) ? 256 : 128;
+        BwdArgs a = base;
+        a.m_tiles = H / 128;
+        a.n_tiles = F / bn;
+        a.out = dw2;
+        a.out2 = dw2;
+        a.out_pitch = (long)F * 2;
+        a.split = H;
+        a.expert_stride = (long)H * F * 2;
+        const int grid = (int)std::min<long>((long)E * a.m_tiles * a.n_tiles, num_sms);
+        ProfScope ps(MOE_KERNEL_BWD_DW2, st);
+        if (launch_bwd_gemm(kBwdDW, bn, mDot, mHt, mHt, a, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    {
+        const int bn = (H % 256 == 0) ? 256 : 128;
+        BwdArgs a = base;
+        a.m_tiles = 2 * F / 128;
+        a.n_tiles = H / bn;
+        a.out = dw1;
+        a.out2 = dw3;
+        a.out_pitch = (long)H * 2;
+        a.split = F;
+        a.expert_stride = (long)F * H * 2;
+        const int grid = (int)std::min<long>((long)E * a.m_tiles * a.n_tiles, num_sms);
+        ProfScope ps(MOE_KERNEL_BWD_DW13, st);
+        if (launch_bwd_gemm(kBwdDW, bn, mDgut, mXt, mXt, a, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    // 6. router
+    {
+        ProfScope ps(MOE_KERNEL_BWD_AUX, st);
+        if (launch_dlogits(o.topk_ids, o.topk_w, dwa, T, E, k, dlogits, st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
 }
 
 }  // extern "C"

@@ -21,6 +21,7 @@ skewed         8192   4096   14336  8   2  bf16   3     logits + 2*log(1/(e+1))
 sweep_T<n>     n      4096   14336  8   2  fp8    4     n in {1, 128, 1024, 16384}
 decode_mxfp4   16     4096   14336  8   2  mxfp4  5     MX FP4 expert weights
 prefill_mxfp4  4096   4096   14336  8   2  mxfp4  6     MX FP4 expert weights
+train_prefill  4096   4096   14336  8   2  bf16   7     backward pass (BWD_CONFIGS)
 =============  =====  =====  =====  ==  =  =====  ====  =================================
 
 Distributions: x ~ N(0,1) rounded to bf16; router logits ~ N(0,1) fp32;
@@ -53,6 +54,11 @@ for _n in (1, 128, 1024, 16384):
 # MX-scaled FP4 expert weights (e2m1 with a power-of-two scale per 32 values)
 CONFIGS["decode_mxfp4"] = _spec(16, H_MIXTRAL, F_MIXTRAL, 8, 2, "mxfp4", 5)
 CONFIGS["prefill_mxfp4"] = _spec(4096, H_MIXTRAL, F_MIXTRAL, 8, 2, "mxfp4", 6)
+
+# backward pass (training) workloads: BF16 weights, an upstream gradient dy
+BWD_CONFIGS = {
+    "train_prefill": _spec(4096, H_MIXTRAL, F_MIXTRAL, 8, 2, "bf16", 7),
+}
 
 # stream ids of the generators
 _S_X, _S_LOGITS, _S_W1, _S_W3, _S_W2, _S_DY = range(6)

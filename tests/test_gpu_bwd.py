@@ -1,0 +1,149 @@
+"""Parity of the backward pass (custom VJP) of the BF16 layer with the fp64
+oracle: dx, dw1, dw3, dw2 and the router-logit gradients, element by element
+at small sizes (several tiles, ragged tails, empty experts, k = E, E = 1,
+d_ff not a multiple of 256), sampled rows and columns at the Mixtral expert
+shape, and the transposed weight copies bit for bit.
+
+Tolerance, element by element: |gpu - ref| <= REL |ref| + ABS_RMS rms(ref).
+The GPU rounds to bf16 what it stores between kernels (g, u, h, dg, du and
+w_a dy_t) and every output but dlogits, each rounding at most 2^-9 relative,
+and accumulates in fp32; REL = 2^-6 and ABS_RMS = 2^-7 leave a factor of 8
+(4 for the cancellation term) over one such rounding.  The oracle rounds h
+to bf16 as the forward does (round_h) and is exact otherwise."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+REL = 2.0 ** -6
+ABS_RMS = 2.0 ** -7
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import mixture_experts_routed_02_b200 as m
+    return m
+
+
+def close(gpu, ref, what):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite values"
+    if ref.size == 0:
+        return
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    err = np.abs(gpu - ref)
+    bad = err > REL * np.abs(ref) + ABS_RMS * rms
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} out of tolerance; worst {err.max():.3e} at "
+                           f"{np.unravel_index(err.argmax(), err.shape)}, rms(ref) {rms:.3e}")
+
+
+def f64(t):
+    """A bf16 or fp32 torch tensor (any device) -> float64 numpy."""
+    return t.detach().float().cpu().double().numpy()
+
+
+def run_bwd(moe, case, dy):
+    dev = "cuda"
+    x, lg = case["x"].to(dev), case["logits"].to(dev)
+    w1, w3, w2 = case["w1"].to(dev), case["w3"].to(dev), case["w2"].to(dev)
+    w13t, w2t = moe.prepare_weights_bwd(w1, w3, w2)
+    out = moe.ffn_backward(x, lg, w1, w3, w13t, w2t, dy.to(dev), case["k"])
+    torch.cuda.synchronize()
+    st = moe.moe_get_status(None)
+    assert st == 0, moe.STATUS_NAMES.get(st, st)
+    return out
+
+
+def oracle_inputs(case, dy):
+    nc = moe_inputs.to_numpy(case)
+    f = oracle.bf16_bits_to_f64
+    return (f(nc["x"]), nc["logits"].astype(np.float64), f(nc["w1"]), f(nc["w3"]), f(nc["w2"]),
+            f(moe_inputs.to_numpy({"dy": dy})["dy"]))
+
+
+SMALL = [
+    # (T, H, F, E, k, seed, skew)
+    (64, 256, 512, 8, 2, 50, False),
+    (200, 256, 512, 8, 2, 51, False),     # several m-tiles per expert, ragged tails
+    (300, 256, 512, 8, 2, 52, True),      # skewed: big and empty experts (zero weight gradients)
+    (129, 384, 640, 4, 3, 53, False),     # d_ff and d_model not multiples of 256: 128-wide tiles
+    (37, 128, 256, 1, 1, 54, False),      # E = 1, k = 1: a dense SwiGLU MLP (dlogits = 0)
+    (50, 128, 384, 4, 4, 55, False),      # k = E
+    (1, 256, 512, 8, 2, 56, False),       # one token
+    (700, 256, 512, 4, 2, 57, False),     # several full tiles per expert
+]
+
+
+@pytest.mark.parametrize("p", SMALL, ids=lambda p: f"T{p[0]}_H{p[1]}_F{p[2]}_E{p[3]}_k{p[4]}" + ("_skew" if p[6] else ""))
+def test_backward_small(moe, p):
+    T, H, F, E, k, seed, skew = p
+    case = moe_inputs.make_case(T, H, F, E, k, "bf16", seed, skew)
+    dy = moe_inputs.make_dy(T, H, seed)
+    out = run_bwd(moe, case, dy)
+    ref = oracle.ffn_bwd64(*oracle_inputs(case, dy), k, round_h=True)
+    for name in ("dx", "dw1", "dw3", "dw2", "dlogits"):
+        close(f64(out[name]), ref[name], f"{name} T={T} H={H} F={F} E={E} k={k}")
+    if skew:
+        counts = np.bincount(oracle.route(case["logits"].numpy(), k)["ids"].reshape(-1), minlength=E)
+        for e in np.flatnonzero(counts == 0):
+            for name in ("dw1", "dw3", "dw2"):
+                assert torch.count_nonzero(out[name][e]).item() == 0, (name, e)
+
+
+def test_backward_no_tokens(moe):
+    """T = 0: every weight gradient is zero (written, not left as it was)."""
+    H, F, E, k = 128, 256, 4, 2
+    case = moe_inputs.make_case(0, H, F, E, k, "bf16", 58)
+    dev = "cuda"
+    w1, w3, w2 = case["w1"].to(dev), case["w3"].to(dev), case["w2"].to(dev)
+    w13t, w2t = moe.prepare_weights_bwd(w1, w3, w2)
+    out = {n: torch.full(s, 7.0, dtype=torch.bfloat16, device=dev)
+           for n, s in (("dw1", (E, F, H)), ("dw3", (E, F, H)), ("dw2", (E, H, F)))}
+    out["dx"] = torch.empty(0, H, dtype=torch.bfloat16, device=dev)
+    out["dlogits"] = torch.empty(0, E, dtype=torch.float32, device=dev)
+    x = torch.empty(0, H, dtype=torch.bfloat16, device=dev)
+    lg = torch.empty(0, E, dtype=torch.float32, device=dev)
+    moe.ffn_backward(x, lg, w1, w3, w13t, w2t, x, k, out=out)
+    torch.cuda.synchronize()
+    for n in ("dw1", "dw3", "dw2"):
+        assert torch.count_nonzero(out[n]).item() == 0, n
+
+
+def test_prepare_weights_bwd_layout(moe):
+    """w13t[e] = [w1[e]^T | w3[e]^T] and w2t[e] = w2[e]^T, bit for bit."""
+    E, F, H = 3, 384, 256
+    w = moe_inputs.make_weights(H, F, E, "bf16", 59)
+    w1, w3, w2 = (w[n].cuda() for n in ("w1", "w3", "w2"))
+    w13t, w2t = moe.prepare_weights_bwd(w1, w3, w2)
+    torch.cuda.synchronize()
+    ref13 = torch.cat([w["w1"].transpose(1, 2), w["w3"].transpose(1, 2)], dim=2)
+    assert torch.equal(w13t.cpu().view(torch.int16), ref13.contiguous().view(torch.int16))
+    assert torch.equal(w2t.cpu().view(torch.int16), w["w2"].transpose(1, 2).contiguous().view(torch.int16))
+
+
+def test_backward_full_size_sampled(moe):
+    """The Mixtral expert shape at the training workload's size (T = 4096,
+    d_model 4096, d_ff 14336, 8 experts, top-2), in the launch configuration
+    the benchmark times: dx and dlogits of sampled tokens, rows of dW1/dW3
+    and columns of dW2 of sampled (expert, feature) pairs, against the
+    oracle's sampled form."""
+    spec = moe_inputs.BWD_CONFIGS["train_prefill"]
+    T, H, F, E, k = spec["T"], spec["H"], spec["F"], spec["E"], spec["k"]
+    case = moe_inputs.make_case(T, H, F, E, k, "bf16", spec["seed"])
+    dy = moe_inputs.make_dy(T, H, spec["seed"])
+    out = run_bwd(moe, case, dy)
+    tokens = np.array([0, 1, 1023, 2048, T - 1], dtype=np.int32)
+    feats = np.array([[0, 0], [1, 7000], [3, F - 1], [5, 4097], [7, 128]], dtype=np.int32)
+    ref = oracle.ffn_bwd64_sampled(*oracle_inputs(case, dy), k, tokens, feats, round_h=True)
+    close(f64(out["dx"][torch.from_numpy(tokens).long()]), ref["dx"], "dx (sampled tokens)")
+    close(f64(out["dlogits"][torch.from_numpy(tokens).long()]), ref["dlogits"], "dlogits (sampled tokens)")
+    for q, (e, n) in enumerate(feats):
+        close(f64(out["dw1"][e, n]), ref["dw1"][q], f"dw1[{e}, {n}, :]")
+        close(f64(out["dw3"][e, n]), ref["dw3"][q], f"dw3[{e}, {n}, :]")
+        close(f64(out["dw2"][e, :, n]), ref["dw2"][q], f"dw2[{e}, :, {n}]")
