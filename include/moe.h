@@ -382,9 +382,10 @@ int moe_profile_read(double* ms_total, int* launches, int reset);
  *   for the others (the routing weights are the softmax over the chosen
  *   logits; the choice is piecewise constant).
  * g and u are recomputed from x and w1/w3 (the forward keeps no
- * intermediates).  Arithmetic: bf16 operands, fp32 accumulation; g, u, h, dg,
- * du, w_a dy_t are rounded to bf16 where they are stored between kernels; dx
- * is summed over the k experts in fp32 and rounded once.
+ * intermediates).  Arithmetic: bf16 operands, fp32 accumulation; g and u are
+ * kept in fp32, h (as in the forward), dg, du and the w_a dy_t entering dW2 are
+ * rounded to bf16 where they are stored between kernels; dx is summed over
+ * the k experts in fp32 and rounded once.
  *
  * moe_backward_workspace_size: bytes of `ws` for moe_ffn_backward (0 if the
  *   dimensions are unsupported: bf16 only, d_model and d_ff multiples of 128,

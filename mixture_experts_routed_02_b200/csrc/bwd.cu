@@ -15,7 +15,7 @@
 // swizzle (no preshuffled weights: training changes them every step):
 //   GU   [slots x 2F]: xg . [W1_e; W3_e]^T -- g and u recomputed (activation
 //        recomputation: the forward keeps nothing but its output); the
-//        epilogue stores g, u and h = bf16(silu(g) u);
+//        epilogue stores g and u in fp32 and h = bf16(silu(g) u);
 //   DH   [slots x F]:  dyg . (W2_e^T)^T, K = H -- epilogue: dw_a (sum over the
 //        tile's columns of dh_unweighted * h, one fp32 atomic per row and tile),
 //        dh = w_a * acc, then dg and du into dGU [slots x 2F];
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             if constexpr (MODE == kBwdGU) {
-                // g, u (bf16) into gu[slot] at columns f and F + f, h into hbuf[slot]
+                // g, u (fp32) into gu[slot] at columns f and F + f, h (bf16) into hbuf[slot]
 #pragma unroll 1
                 for (int c0 = 0; c0 < 128; c0 += 32) {
                     uint32_t rg[32], ru[32];
@@ -306,16 +306,18 @@ __global__ void __launch_bounds__(192, 1)
                             uv[i] = __uint_as_float(ru[i]);
                             hv[i] = __fdividef(gv[i], 1.0f + __expf(-gv[i])) * uv[i];
                         }
-                        uint4* dg = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) + (size_t)slot * args.out_pitch) + f / 8;
-                        uint4* du = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) + (size_t)slot * args.out_pitch) +
-                                    (args.F + f) / 8;
-                        uint4* dh = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out2) + (size_t)slot * args.out2_pitch) + f / 8;
+                        float4* og = reinterpret_cast<float4*>(static_cast<uint8_t*>(args.out) + (size_t)slot * args.out_pitch) +
+                                     f / 4;
+                        float4* ou = reinterpret_cast<float4*>(static_cast<uint8_t*>(args.out) + (size_t)slot * args.out_pitch) +
+                                     (args.F + f) / 4;
+                        uint4* oh = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out2) + (size_t)slot * args.out2_pitch) + f / 8;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            dg[i] = pack8(gv + 8 * i);
-                            du[i] = pack8(uv + 8 * i);
-                            dh[i] = pack8(hv + 8 * i);
+                        for (int i = 0; i < 8; ++i) {
+                            og[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
+                            ou[i] = make_float4(uv[4 * i], uv[4 * i + 1], uv[4 * i + 2], uv[4 * i + 3]);
                         }
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) oh[i] = pack8(hv + 8 * i);
                     }
                 }
             } else if constexpr (MODE == kBwdDH) {
@@ -331,17 +333,19 @@ __global__ void __launch_bounds__(192, 1)
                     if (a >= 0) {
                         const int f = n * BN + c0;
                         const uint8_t* gurow = static_cast<const uint8_t*>(args.gu) + (size_t)slot * args.gu_pitch;
-                        const uint4* gp = reinterpret_cast<const uint4*>(gurow) + f / 8;
-                        const uint4* up = reinterpret_cast<const uint4*>(gurow) + (args.F + f) / 8;
+                        const float4* gp = reinterpret_cast<const float4*>(gurow) + f / 4;
+                        const float4* up = reinterpret_cast<const float4*>(gurow) + (args.F + f) / 4;
                         const uint4* hp =
                             reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(args.hbuf) + (size_t)slot * args.h_pitch) + f / 8;
                         float gv[32], uv[32], hv[32];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            unpack8(__ldg(gp + i), gv + 8 * i);
-                            unpack8(__ldg(up + i), uv + 8 * i);
-                            unpack8(__ldg(hp + i), hv + 8 * i);
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 g4 = __ldg(gp + i), u4 = __ldg(up + i);
+                            gv[4 * i] = g4.x; gv[4 * i + 1] = g4.y; gv[4 * i + 2] = g4.z; gv[4 * i + 3] = g4.w;
+                            uv[4 * i] = u4.x; uv[4 * i + 1] = u4.y; uv[4 * i + 2] = u4.z; uv[4 * i + 3] = u4.w;
                         }
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) unpack8(__ldg(hp + i), hv + 8 * i);
                         float dgv[32], duv[32];
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
@@ -430,10 +434,14 @@ __global__ void __launch_bounds__(192, 1)
 //   kSrcSlots: src row s of the slot layout, 0 for a padding slot;
 //   kSrcTokens: the token row of slot s's assignment (t = a / topk), times
 //              topk_w[a] if scaled, 0 for a padding slot.
-// Reads are 128 bytes per row of the tile, writes 128 bytes per output row.
+// Each thread reads 16-byte pieces of source rows (a warp covers four rows of
+// 128 bytes) and writes 16-byte pieces of output rows (eight consecutive
+// slots); the tile crosses shared memory with a row pitch of 66 elements so
+// that the column reads of one warp fall on distinct banks but for pairs.
 template <int SRC>
 __global__ void __launch_bounds__(256) transpose_kernel(TransposeArgs p) {
-    __shared__ uint16_t tile[64][65];
+    constexpr int kPitch = 66;
+    __shared__ __align__(16) uint16_t tile[64 * kPitch];
     const int c0 = blockIdx.x * 64, s0 = blockIdx.y * 64, z = blockIdx.z;
     int rows = p.rows;
     if (SRC != kSrcRows) {
@@ -443,26 +451,29 @@ __global__ void __launch_bounds__(256) transpose_kernel(TransposeArgs p) {
     if (s0 >= rows) return;
     const uint16_t* src = static_cast<const uint16_t*>(p.src) + (size_t)z * p.src_batch;
     uint16_t* out = static_cast<uint16_t*>(p.out) + (size_t)z * p.out_batch;
-    for (int i = threadIdx.x; i < 64 * 64; i += 256) {
-        const int r = i >> 6, c = i & 63;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int q = threadIdx.x + 256 * i;  // 512 pieces: 64 rows x 8 pieces of 8 elements
+        const int r = q >> 3, c8 = (q & 7) * 8;
         const int s = s0 + r;
-        uint16_t v = 0;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (s < rows) {
             if constexpr (SRC == kSrcRows) {
-                v = src[(size_t)s * p.src_pitch + c0 + c];
+                v = *reinterpret_cast<const uint4*>(src + (size_t)s * p.src_pitch + c0 + c8);
             } else {
                 const int a = p.slot_assign[s];
                 if (a >= 0 && a < p.num_assign) {
                     if constexpr (SRC == kSrcSlots) {
-                        v = src[(size_t)s * p.src_pitch + c0 + c];
+                        v = *reinterpret_cast<const uint4*>(src + (size_t)s * p.src_pitch + c0 + c8);
                     } else {
-                        const uint16_t raw = src[(size_t)(a / p.topk) * p.src_pitch + c0 + c];
+                        v = *reinterpret_cast<const uint4*>(src + (size_t)(a / p.topk) * p.src_pitch + c0 + c8);
                         if (p.scale) {
-                            const float f = __uint_as_float((uint32_t)raw << 16) * p.scale[a];
-                            __nv_bfloat16 b = __float2bfloat16_rn(f);
-                            v = *reinterpret_cast<uint16_t*>(&b);
-                        } else {
-                            v = raw;
+                            const float sc = p.scale[a];
+                            float f[8];
+                            unpack8(v, f);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) f[j] *= sc;
+                            v = pack8(f);
                         }
                     }
                 } else if (a < -1 || a >= p.num_assign) {
@@ -470,12 +481,32 @@ __global__ void __launch_bounds__(256) transpose_kernel(TransposeArgs p) {
                 }
             }
         }
-        tile[r][c] = v;
+        uint32_t* t32 = reinterpret_cast<uint32_t*>(tile + r * kPitch + c8);  // 4-byte aligned (kPitch even)
+        t32[0] = v.x;
+        t32[1] = v.y;
+        t32[2] = v.z;
+        t32[3] = v.w;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < 64 * 64; i += 256) {
-        const int c = i >> 6, r = i & 63;
-        if (s0 + r < rows) out[(size_t)(c0 + c) * p.out_pitch + p.out_col + s0 + r] = tile[r][c];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int q = threadIdx.x + 256 * i;  // 512 pieces: 64 output rows x 8 pieces of 8 slots
+        const int c = q >> 3, r8 = (q & 7) * 8;
+        if (s0 + r8 >= rows) continue;  // rows is a multiple of 64 for slot sources
+        uint16_t e[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) e[j] = tile[(r8 + j) * kPitch + c];
+        uint16_t* dst = out + (size_t)(c0 + c) * p.out_pitch + p.out_col + s0 + r8;
+        if (s0 + r8 + 8 <= rows) {
+            uint4 w;
+            w.x = e[0] | ((uint32_t)e[1] << 16);
+            w.y = e[2] | ((uint32_t)e[3] << 16);
+            w.z = e[4] | ((uint32_t)e[5] << 16);
+            w.w = e[6] | ((uint32_t)e[7] << 16);
+            *reinterpret_cast<uint4*>(dst) = w;
+        } else {
+            for (int j = 0; j < 8 && s0 + r8 + j < rows; ++j) dst[j] = e[j];
+        }
     }
 }
 
@@ -532,7 +563,11 @@ cudaError_t launch_bwd_gemm(int mode, int bn, const CUtensorMap& a, const CUtens
 
 cudaError_t launch_transpose(int src_kind, const TransposeArgs& p, int cols, int rows_max, int batch,
                              cudaStream_t stream) {
-    if (cols % 64 || rows_max < 0 || batch < 1) return cudaErrorInvalidValue;
+    // 16-byte pieces: the source pitch, the output pitch and column offset in
+    // whole pieces of 8 elements (the bases are 16-byte aligned by contract)
+    if (cols % 64 || rows_max < 0 || batch < 1 || p.src_pitch % 8 || p.out_pitch % 8 || p.out_col % 8 ||
+        p.src_batch % 8 || p.out_batch % 8)
+        return cudaErrorInvalidValue;
     if (rows_max == 0 || cols == 0) return cudaSuccess;
     const dim3 grid(cols / 64, (rows_max + 63) / 64, batch);
     switch (src_kind) {

@@ -23,11 +23,11 @@ struct BwdArgs {
     int m_tiles;   // DW: output rows / 128
     int b_rows;    // rows of B per expert (GU: F, DH: F, DX: H)
     int F;         // d_ff (GU, DH: column offset of u and du)
-    void* out;     // GU: g|u [S, 2F]; DH: dg|du [S, 2F]; DX: fp32 dx [T, H]; DW: dW (first part)
+    void* out;     // GU: fp32 g|u [S, 2F]; DH: dg|du [S, 2F]; DX: fp32 dx [T, H]; DW: dW (first part)
     long out_pitch;  // bytes
     void* out2;    // GU: h [S, F]; DW: rows >= split (dW3)
     long out2_pitch;
-    const void* gu;  // DH: g|u
+    const void* gu;  // DH: fp32 g|u
     long gu_pitch;
     const void* hbuf;  // DH: h
     long h_pitch;

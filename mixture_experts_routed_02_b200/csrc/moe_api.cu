@@ -780,7 +780,7 @@ BwdLayout make_bwd_layout(int T, int H, int F, int E, int k) {
     B.fwd = make_layout(T, H, F, E, k, MOE_BF16);
     const size_t S = B.fwd.S_max;
     size_t sz[kBwRegions];
-    sz[kBwGU] = S * act_pitch(4L * F);  // g|u rows [S, 2F]; later dg|du transposed [2F, S]
+    sz[kBwGU] = S * act_pitch(8L * F);  // fp32 g|u rows [S, 2F]; later bf16 dg|du transposed [2F, S]
     sz[kBwDYG] = S * act_pitch(2L * H);  // dy gathered into the slot layout [S, H]
     sz[kBwDGU] = S * act_pitch(4L * F);  // dg|du [S, 2F]
     sz[kBwDOT] = (size_t)H * S * 2;      // (w_a dy_t) transposed [H, S]
@@ -902,7 +902,7 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
 
     // tensor maps: K-major bf16 operands, 64-element x 128-row boxes
     CUtensorMap mXg, mW1, mW3, mDyg, mW2t, mDgu, mW13t, mDot, mHt, mDgut, mXt;
-    const long p2H = act_pitch(2L * H), p4F = act_pitch(4L * F), p2F = act_pitch(2L * F);
+    const long p2H = act_pitch(2L * H), p4F = act_pitch(4L * F), p2F = act_pitch(2L * F), p8F = act_pitch(8L * F);
     if (!make_map(&mXg, reg(MOE_WS_XG), S, H, p2H, 2, 128) ||
         !make_map(&mW1, w1, (size_t)E * F, H, (size_t)H * 2, 2, 128) ||
         !make_map(&mW3, w3, (size_t)E * F, H, (size_t)H * 2, 2, 128) ||
@@ -938,7 +938,7 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.k_tiles = H / 64;
         a.b_rows = F;
         a.out = breg(kBwGU);
-        a.out_pitch = p4F;
+        a.out_pitch = p8F;
         a.out2 = reg(MOE_WS_H);
         a.out2_pitch = p2F;
         ProfScope ps(MOE_KERNEL_BWD_GU, st);
@@ -955,7 +955,7 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.out = breg(kBwDGU);
         a.out_pitch = p4F;
         a.gu = breg(kBwGU);
-        a.gu_pitch = p4F;
+        a.gu_pitch = p8F;
         a.hbuf = reg(MOE_WS_H);
         a.h_pitch = p2F;
         a.dw = dwa;

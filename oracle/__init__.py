@@ -91,10 +91,11 @@ def _load():
         lib.oracle_moe_ffn64.restype = I
         lib.oracle_moe_ffn64.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, I]
         lib.oracle_moe_ffn_bwd64.restype = I
-        lib.oracle_moe_ffn_bwd64.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, P, P, I]
+        lib.oracle_moe_ffn_bwd64.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P,
+                                             I]
         lib.oracle_moe_ffn_bwd64_sampled.restype = I
         lib.oracle_moe_ffn_bwd64_sampled.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, I, P, P, P, I, P, P, P,
-                                                     I]
+                                                     P, P, P, P, P, I]
         _lib = lib
     return _lib
 
@@ -260,6 +261,10 @@ def bf16_bits_to_f64(bits):
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+def _round(round_h, round_inter=False):
+    return (1 if round_h else 0) | (2 if round_inter else 0)
+
+
 def _dims64(x, w1, logits, k):
     T, H = x.shape
     E, F, H1 = w1.shape
@@ -274,43 +279,57 @@ def ffn64(x, logits, w1, w3, w2, k, round_h=False, nthreads=0):
     x, lg, w1, w3, w2 = (_c(a, np.float64) for a in (x, logits, w1, w3, w2))
     T, H, F, E = _dims64(x, w1, lg, k)
     y = np.zeros((T, H))
-    rc = _load().oracle_moe_ffn64(_ptr(x), _ptr(lg), _ptr(w1), _ptr(w3), _ptr(w2), T, H, F, E, k, int(round_h),
+    rc = _load().oracle_moe_ffn64(_ptr(x), _ptr(lg), _ptr(w1), _ptr(w3), _ptr(w2), T, H, F, E, k, _round(round_h),
                                   _ptr(y), nthreads)
     if rc != 0:
         raise ValueError("oracle_moe_ffn64: bad arguments")
     return y
 
 
-def ffn_bwd64(x, logits, w1, w3, w2, dy, k, round_h=True, nthreads=0):
+def ffn_bwd64(x, logits, w1, w3, w2, dy, k, round_h=True, round_inter=False, want_abs=False, nthreads=0):
     """Gradients of <dy, layer(x)>: dict(dx [T,H], dw1 [E,F,H], dw3 [E,F,H],
-    dw2 [E,H,F], dlogits [T,E], dwa [T,k] routing-weight gradients), fp64."""
+    dw2 [E,H,F], dlogits [T,E], dwa [T,k] routing-weight gradients), fp64.
+    round_h: h rounded to bf16 as the forward does; round_inter: also dg, du
+    and the w_a dy_t entering dW2 (a bf16 implementation's storage points).
+    want_abs: also each entry's sum of absolute terms ("<name>_abs")."""
     x, lg, w1, w3, w2, dy = (_c(a, np.float64) for a in (x, logits, w1, w3, w2, dy))
     T, H, F, E = _dims64(x, w1, lg, k)
     out = dict(dx=np.zeros((T, H)), dw1=np.zeros((E, F, H)), dw3=np.zeros((E, F, H)), dw2=np.zeros((E, H, F)),
                dlogits=np.zeros((T, E)), dwa=np.zeros(max(T * k, 1)))
+    names = ("dx", "dw1", "dw3", "dw2", "dlogits")
+    if want_abs:
+        for n in names:
+            out[n + "_abs"] = np.zeros_like(out[n])
+    ab = [_ptr(out[n + "_abs"]) if want_abs else None for n in names]
     rc = _load().oracle_moe_ffn_bwd64(_ptr(x), _ptr(lg), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(dy), T, H, F, E, k,
-                                      int(round_h), _ptr(out["dx"]), _ptr(out["dw1"]), _ptr(out["dw3"]),
-                                      _ptr(out["dw2"]), _ptr(out["dlogits"]), _ptr(out["dwa"]), nthreads)
+                                      _round(round_h, round_inter), _ptr(out["dx"]), _ptr(out["dw1"]), _ptr(out["dw3"]),
+                                      _ptr(out["dw2"]), _ptr(out["dlogits"]), _ptr(out["dwa"]), *ab, nthreads)
     if rc != 0:
         raise ValueError("oracle_moe_ffn_bwd64: bad arguments")
     out["dwa"] = out["dwa"][:T * k].reshape(T, k)
     return out
 
 
-def ffn_bwd64_sampled(x, logits, w1, w3, w2, dy, k, tokens, feats, round_h=True, nthreads=0):
+def ffn_bwd64_sampled(x, logits, w1, w3, w2, dy, k, tokens, feats, round_h=True, round_inter=False, want_abs=False,
+                      nthreads=0):
     """Sampled gradients: dx [ntok,H] and dlogits [ntok,E] of the listed
     tokens; for each (e, n) in feats, dw1[e, n, :], dw3[e, n, :] and
-    dw2[e, :, n] ([nfeat,H] each)."""
+    dw2[e, :, n] ([nfeat,H] each); with want_abs their error scales too."""
     x, lg, w1, w3, w2, dy = (_c(a, np.float64) for a in (x, logits, w1, w3, w2, dy))
     T, H, F, E = _dims64(x, w1, lg, k)
     tok = _c(tokens, np.int32).reshape(-1)
     ft = _c(feats, np.int32).reshape(-1, 2)
     out = dict(dx=np.zeros((len(tok), H)), dlogits=np.zeros((len(tok), E)), dw1=np.zeros((len(ft), H)),
                dw3=np.zeros((len(ft), H)), dw2=np.zeros((len(ft), H)))
+    names = ("dx", "dlogits", "dw1", "dw3", "dw2")
+    if want_abs:
+        for n in names:
+            out[n + "_abs"] = np.zeros_like(out[n])
+    ab = [_ptr(out[n + "_abs"]) if want_abs else None for n in names]
     rc = _load().oracle_moe_ffn_bwd64_sampled(_ptr(x), _ptr(lg), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(dy), T, H, F, E,
-                                              k, int(round_h), _ptr(tok), len(tok), _ptr(out["dx"]),
+                                              k, _round(round_h, round_inter), _ptr(tok), len(tok), _ptr(out["dx"]),
                                               _ptr(out["dlogits"]), _ptr(ft), len(ft), _ptr(out["dw1"]),
-                                              _ptr(out["dw3"]), _ptr(out["dw2"]), nthreads)
+                                              _ptr(out["dw3"]), _ptr(out["dw2"]), *ab, nthreads)
     if rc != 0:
         raise ValueError("oracle_moe_ffn_bwd64_sampled: bad arguments")
     return out

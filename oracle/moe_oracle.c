@@ -516,9 +516,9 @@ int oracle_max_threads(void) {
  * gradient dy = dL/dout.  For each assignment a = (t, j) of token t to expert
  * e with routing weight w_a:
  *
- *   g = W1_e x_t,  u = W3_e x_t,  h = silu(g) * u   (rounded to bf16 when
- *       round_h, as the forward rounds it; the rounding passes gradients
- *       through unchanged),  o = W2_e h
+ *   g = W1_e x_t,  u = W3_e x_t,  h = silu(g) * u   (rounded to bf16 with
+ *       ORACLE_ROUND_H, as the forward rounds it; the rounding passes
+ *       gradients through unchanged),  o = W2_e h
  *   dw_a = <dy_t, o>,   dO = w_a dy_t,   dh = W2_e^T dO
  *   du = dh * silu(g),  dg = dh * u * silu'(g),  silu'(g) = s(g) (1 + g (1 - s(g)))
  *       with s the logistic function
@@ -532,12 +532,27 @@ int oracle_max_threads(void) {
  * Inputs are fp64 so that finite differences can perturb them.  The choice of
  * experts follows the forward's ranking rule (larger logit first, lower index
  * on a tie, NaN as -inf); gradients are defined for finite logits.
+ *
+ * `round` flags: ORACLE_ROUND_H rounds h to bf16 (the forward's rounding);
+ * ORACLE_ROUND_INTER also rounds to bf16 the values a bf16 implementation
+ * stores between its backward steps -- dg and du, and the products w_a dy_t
+ * that enter dW2 (dh uses w_a dy_t unrounded).  All else is exact.
+ *
+ * Optional error scales (`abs` outputs): each gradient entry's sum of the
+ * absolute values of its terms -- |W1|^T |dg| + |W3|^T |du| for dx, |dg| |x|^T
+ * for dW1, |du| |x|^T for dW3, |w_a dy| |h|^T for dW2, and for the router
+ * w_j (s_j + sum_i w_i s_i) with s_a = sum_f |dh_f / w_a| |h_f| -- the scale
+ * against which a perturbation of the individual terms is measured.
  */
+#define ORACLE_ROUND_H 1
+#define ORACLE_ROUND_INTER 2
 
 typedef struct {
     const double *x, *w1, *w3, *w2;  /* [T,H], [E,F,H], [E,F,H], [E,H,F] */
-    int T, H, F, E, k, round_h;
+    int T, H, F, E, k, round_h, round_inter;
 } bctx;
+
+static double bf16r(double v) { return oracle_bf16_to_double(oracle_bf16_from_double(v)); }
 
 static double ranked64(double l) { return isnan(l) ? -INFINITY : l; }
 
@@ -567,10 +582,12 @@ static void topk64(const double* l, int E, int k, int32_t* ids, double* w) {
 }
 
 static int bctx_init(bctx* c, const double* x, const double* w1, const double* w3, const double* w2, int T,
-                     int H, int F, int E, int k, int round_h) {
+                     int H, int F, int E, int k, int round) {
     if (T < 0 || H < 1 || F < 1 || E < 1 || E > 64 || k < 1 || k > E) return -1;
     c->x = x; c->w1 = w1; c->w3 = w3; c->w2 = w2;
-    c->T = T; c->H = H; c->F = F; c->E = E; c->k = k; c->round_h = round_h;
+    c->T = T; c->H = H; c->F = F; c->E = E; c->k = k;
+    c->round_h = (round & ORACLE_ROUND_H) != 0;
+    c->round_inter = (round & ORACLE_ROUND_INTER) != 0;
     return 0;
 }
 
@@ -587,7 +604,7 @@ static void fwd_assign(const bctx* c, int e, int t, double* g, double* u, double
             uv += r3[i] * xt[i];
         }
         double hv = gv / (1.0 + exp(-gv)) * uv;
-        if (c->round_h) hv = oracle_bf16_to_double(oracle_bf16_from_double(hv));
+        if (c->round_h) hv = bf16r(hv);
         g[n] = gv; u[n] = uv; h[n] = hv;
     }
     for (int m = 0; m < H; ++m) {
@@ -598,21 +615,26 @@ static void fwd_assign(const bctx* c, int e, int t, double* g, double* u, double
     }
 }
 
-/* dg, du [F] from dh and the forward values */
-static void swiglu_bwd(int F, const double* g, const double* u, const double* dh, double* dg, double* du) {
+/* dg, du [F] from dh and the forward values (rounded to bf16 with round_inter) */
+static void swiglu_bwd(int F, const double* g, const double* u, const double* dh, double* dg, double* du,
+                       int round_inter) {
     for (int n = 0; n < F; ++n) {
         double s = 1.0 / (1.0 + exp(-g[n]));
         du[n] = dh[n] * (g[n] / (1.0 + exp(-g[n])));
         dg[n] = dh[n] * u[n] * (s * (1.0 + g[n] * (1.0 - s)));
+        if (round_inter) {
+            du[n] = bf16r(du[n]);
+            dg[n] = bf16r(dg[n]);
+        }
     }
 }
 
 /* y [T,H] (fp64, not rounded) of the layer on fp64 inputs; the combine adds
  * each token's expert outputs in ascending expert order, as the routed form */
 int oracle_moe_ffn64(const double* x, const double* logits, const double* w1, const double* w3, const double* w2,
-                     int T, int H, int F, int E, int k, int round_h, double* y, int nthreads) {
+                     int T, int H, int F, int E, int k, int round, double* y, int nthreads) {
     bctx c;
-    if (bctx_init(&c, x, w1, w3, w2, T, H, F, E, k, round_h)) return -1;
+    if (bctx_init(&c, x, w1, w3, w2, T, H, F, E, k, round)) return -1;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
 #endif
@@ -641,14 +663,16 @@ int oracle_moe_ffn64(const double* x, const double* logits, const double* w1, co
 }
 
 /* Full gradients: dx [T,H], dw1/dw3 [E,F,H], dw2 [E,H,F], dlogits [T,E]; dwa
- * (optional) [T*k] the gradients of the routing weights.  Experts run in
+ * (optional) [T*k] the gradients of the routing weights; the error scales
+ * (optional, all or none) in arrays of the same shapes.  Experts run in
  * parallel; inside one, assignments in ascending order. */
 int oracle_moe_ffn_bwd64(const double* x, const double* logits, const double* w1, const double* w3,
-                         const double* w2, const double* dy, int T, int H, int F, int E, int k, int round_h,
+                         const double* w2, const double* dy, int T, int H, int F, int E, int k, int round,
                          double* dx, double* dw1, double* dw3, double* dw2, double* dlogits, double* dwa_out,
+                         double* dx_abs, double* dw1_abs, double* dw3_abs, double* dw2_abs, double* dl_abs,
                          int nthreads) {
     bctx c;
-    if (bctx_init(&c, x, w1, w3, w2, T, H, F, E, k, round_h)) return -1;
+    if (bctx_init(&c, x, w1, w3, w2, T, H, F, E, k, round)) return -1;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
 #endif
@@ -657,10 +681,18 @@ int oracle_moe_ffn_bwd64(const double* x, const double* logits, const double* w1
     double* w = malloc(sizeof(double) * (A ? A : 1));
     double* dwa = calloc(A ? A : 1, sizeof(double));
     double* dxa = calloc((size_t)(A ? A : 1) * H, sizeof(double));
+    const int want_abs = dx_abs != NULL;
+    double* dwabs = calloc(A ? A : 1, sizeof(double));
+    double* dxabs = want_abs ? calloc((size_t)(A ? A : 1) * H, sizeof(double)) : NULL;
     for (int t = 0; t < T; ++t) topk64(logits + (size_t)t * E, E, k, ids + (size_t)t * k, w + (size_t)t * k);
     memset(dw1, 0, sizeof(double) * (size_t)E * F * H);
     memset(dw3, 0, sizeof(double) * (size_t)E * F * H);
     memset(dw2, 0, sizeof(double) * (size_t)E * H * F);
+    if (want_abs) {
+        memset(dw1_abs, 0, sizeof(double) * (size_t)E * F * H);
+        memset(dw3_abs, 0, sizeof(double) * (size_t)E * F * H);
+        memset(dw2_abs, 0, sizeof(double) * (size_t)E * H * F);
+    }
     #pragma omp parallel for schedule(dynamic, 1)
     for (int e = 0; e < E; ++e) {
         double *g = malloc(sizeof(double) * F), *u = malloc(sizeof(double) * F), *h = malloc(sizeof(double) * F);
@@ -681,7 +713,7 @@ int oracle_moe_ffn_bwd64(const double* x, const double* logits, const double* w1
                 for (int m = 0; m < H; ++m) acc += w2[((size_t)e * H + m) * F + n] * dO[m];
                 dh[n] = acc;
             }
-            swiglu_bwd(F, g, u, dh, dg, du);
+            swiglu_bwd(F, g, u, dh, dg, du, c.round_inter);
             double* dxr = dxa + (size_t)a * H;
             for (int i = 0; i < H; ++i) {
                 double acc = 0.0;
@@ -699,7 +731,34 @@ int oracle_moe_ffn_bwd64(const double* x, const double* logits, const double* w1
             }
             for (int m = 0; m < H; ++m) {
                 double* r2 = dw2 + ((size_t)e * H + m) * F;
-                for (int n = 0; n < F; ++n) r2[n] += dO[m] * h[n];
+                const double dom = c.round_inter ? bf16r(dO[m]) : dO[m];
+                for (int n = 0; n < F; ++n) r2[n] += dom * h[n];
+            }
+            if (want_abs) {
+                double sa = 0.0;
+                for (int n = 0; n < F; ++n) sa += fabs(dh[n]) * fabs(h[n]);
+                dwabs[a] = (w[a] > 0.0) ? sa / w[a] : 0.0;
+                double* xr = dxabs + (size_t)a * H;
+                for (int i = 0; i < H; ++i) {
+                    double acc = 0.0;
+                    for (int n = 0; n < F; ++n)
+                        acc += fabs(w1[((size_t)e * F + n) * H + i] * dg[n]) +
+                               fabs(w3[((size_t)e * F + n) * H + i] * du[n]);
+                    xr[i] = acc;
+                }
+                for (int n = 0; n < F; ++n) {
+                    double* r1 = dw1_abs + ((size_t)e * F + n) * H;
+                    double* r3 = dw3_abs + ((size_t)e * F + n) * H;
+                    for (int i = 0; i < H; ++i) {
+                        r1[i] += fabs(dg[n] * xt[i]);
+                        r3[i] += fabs(du[n] * xt[i]);
+                    }
+                }
+                for (int m = 0; m < H; ++m) {
+                    double* r2 = dw2_abs + ((size_t)e * H + m) * F;
+                    const double dom = fabs(c.round_inter ? bf16r(dO[m]) : dO[m]);
+                    for (int n = 0; n < F; ++n) r2[n] += dom * fabs(h[n]);
+                }
             }
         }
         free(g); free(u); free(h); free(dh); free(dg); free(du); free(o); free(dO);
@@ -717,23 +776,39 @@ int oracle_moe_ffn_bwd64(const double* x, const double* logits, const double* w1
             size_t a = (size_t)t * k + j;
             dlogits[(size_t)t * E + ids[a]] = w[a] * (dwa[a] - sw);
         }
+        if (want_abs) {
+            for (int i = 0; i < H; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < k; ++j) acc += dxabs[((size_t)t * k + j) * H + i];
+                dx_abs[(size_t)t * H + i] = acc;
+            }
+            double swa = 0.0;
+            for (int j = 0; j < k; ++j) swa += w[(size_t)t * k + j] * dwabs[(size_t)t * k + j];
+            for (int e = 0; e < E; ++e) dl_abs[(size_t)t * E + e] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                size_t a = (size_t)t * k + j;
+                dl_abs[(size_t)t * E + ids[a]] = w[a] * (dwabs[a] + swa);
+            }
+        }
     }
     if (dwa_out) memcpy(dwa_out, dwa, sizeof(double) * A);
-    free(ids); free(w); free(dwa); free(dxa);
+    free(ids); free(w); free(dwa); free(dxa); free(dwabs); free(dxabs);
     return 0;
 }
 
 /* Sampled gradients, for sizes where the full form takes too long: dx and
  * dlogits of the listed tokens ([ntok,H], [ntok,E]); for each listed pair
  * (e, n) of feats [nfeat,2], row n of dW1_e and of dW3_e and column n of
- * dW2_e ([nfeat,H] each).  Same arithmetic and order as the full form. */
+ * dW2_e ([nfeat,H] each).  Same arithmetic and order as the full form; the
+ * error scales (optional, all or none) in arrays of the same shapes. */
 int oracle_moe_ffn_bwd64_sampled(const double* x, const double* logits, const double* w1, const double* w3,
                                  const double* w2, const double* dy, int T, int H, int F, int E, int k,
-                                 int round_h, const int32_t* tokens, int ntok, double* dx_s, double* dl_s,
+                                 int round, const int32_t* tokens, int ntok, double* dx_s, double* dl_s,
                                  const int32_t* feats, int nfeat, double* dw1_s, double* dw3_s, double* dw2_s,
+                                 double* dx_abs, double* dl_abs, double* dw1_abs, double* dw3_abs, double* dw2_abs,
                                  int nthreads) {
     bctx c;
-    if (bctx_init(&c, x, w1, w3, w2, T, H, F, E, k, round_h)) return -1;
+    if (bctx_init(&c, x, w1, w3, w2, T, H, F, E, k, round)) return -1;
     for (int i = 0; i < ntok; ++i)
         if (tokens[i] < 0 || tokens[i] >= T) return -1;
     for (int i = 0; i < nfeat; ++i)
@@ -753,7 +828,8 @@ int oracle_moe_ffn_bwd64_sampled(const double* x, const double* logits, const do
         double *dh = malloc(sizeof(double) * F), *dg = malloc(sizeof(double) * F), *du = malloc(sizeof(double) * F);
         double *o = malloc(sizeof(double) * H), *dO = malloc(sizeof(double) * H);
         double* dxa = calloc((size_t)k * H, sizeof(double));
-        double dwa[64];
+        double* dxab = calloc((size_t)k * H, sizeof(double));
+        double dwa[64], dwab[64];
         for (int j = 0; j < k; ++j) {
             size_t a = (size_t)t * k + j;
             int e = ids[a];
@@ -767,12 +843,24 @@ int oracle_moe_ffn_bwd64_sampled(const double* x, const double* logits, const do
                 for (int m = 0; m < H; ++m) acc += w2[((size_t)e * H + m) * F + n] * dO[m];
                 dh[n] = acc;
             }
-            swiglu_bwd(F, g, u, dh, dg, du);
+            swiglu_bwd(F, g, u, dh, dg, du, c.round_inter);
             for (int i = 0; i < H; ++i) {
                 double acc = 0.0;
                 for (int n = 0; n < F; ++n)
                     acc += w1[((size_t)e * F + n) * H + i] * dg[n] + w3[((size_t)e * F + n) * H + i] * du[n];
                 dxa[(size_t)j * H + i] = acc;
+            }
+            if (dx_abs) {
+                double sa = 0.0;
+                for (int n = 0; n < F; ++n) sa += fabs(dh[n]) * fabs(h[n]);
+                dwab[j] = (w[a] > 0.0) ? sa / w[a] : 0.0;
+                for (int i = 0; i < H; ++i) {
+                    double acc = 0.0;
+                    for (int n = 0; n < F; ++n)
+                        acc += fabs(w1[((size_t)e * F + n) * H + i] * dg[n]) +
+                               fabs(w3[((size_t)e * F + n) * H + i] * du[n]);
+                    dxab[(size_t)j * H + i] = acc;
+                }
             }
         }
         for (int i = 0; i < H; ++i) {
@@ -787,7 +875,21 @@ int oracle_moe_ffn_bwd64_sampled(const double* x, const double* logits, const do
             size_t a = (size_t)t * k + j;
             dl_s[(size_t)q * E + ids[a]] = w[a] * (dwa[j] - sw);
         }
-        free(g); free(u); free(h); free(dh); free(dg); free(du); free(o); free(dO); free(dxa);
+        if (dx_abs) {
+            for (int i = 0; i < H; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < k; ++j) acc += dxab[(size_t)j * H + i];
+                dx_abs[(size_t)q * H + i] = acc;
+            }
+            double swa = 0.0;
+            for (int j = 0; j < k; ++j) swa += w[(size_t)t * k + j] * dwab[j];
+            for (int e = 0; e < E; ++e) dl_abs[(size_t)q * E + e] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                size_t a = (size_t)t * k + j;
+                dl_abs[(size_t)q * E + ids[a]] = w[a] * (dwab[j] + swa);
+            }
+        }
+        free(g); free(u); free(h); free(dh); free(dg); free(du); free(o); free(dO); free(dxa); free(dxab);
     }
     #pragma omp parallel for schedule(dynamic, 1)
     for (int q = 0; q < nfeat; ++q) {
@@ -796,6 +898,11 @@ int oracle_moe_ffn_bwd64_sampled(const double* x, const double* logits, const do
         double* r3 = dw3_s + (size_t)q * H;
         double* c2 = dw2_s + (size_t)q * H;
         for (int i = 0; i < H; ++i) r1[i] = r3[i] = c2[i] = 0.0;
+        double* a1 = dw1_abs ? dw1_abs + (size_t)q * H : NULL;
+        double* a3 = dw1_abs ? dw3_abs + (size_t)q * H : NULL;
+        double* a2 = dw1_abs ? dw2_abs + (size_t)q * H : NULL;
+        if (a1)
+            for (int i = 0; i < H; ++i) a1[i] = a3[i] = a2[i] = 0.0;
         const double* w1r = w1 + ((size_t)e * F + n) * H;
         const double* w3r = w3 + ((size_t)e * F + n) * H;
         for (long a = 0; a < A; ++a) {
@@ -809,16 +916,24 @@ int oracle_moe_ffn_bwd64_sampled(const double* x, const double* logits, const do
                 uv += w3r[i] * xt[i];
             }
             double hv = gv / (1.0 + exp(-gv)) * uv;
-            if (round_h) hv = oracle_bf16_to_double(oracle_bf16_from_double(hv));
+            if (c.round_h) hv = bf16r(hv);
             double dhv = 0.0;
             for (int m = 0; m < H; ++m) dhv += w2[((size_t)e * H + m) * F + n] * (w[a] * dyt[m]);
             double dgv, duv;
-            swiglu_bwd(1, &gv, &uv, &dhv, &dgv, &duv);
+            swiglu_bwd(1, &gv, &uv, &dhv, &dgv, &duv, c.round_inter);
             for (int i = 0; i < H; ++i) {
                 r1[i] += dgv * xt[i];
                 r3[i] += duv * xt[i];
             }
-            for (int m = 0; m < H; ++m) c2[m] += (w[a] * dyt[m]) * hv;
+            for (int m = 0; m < H; ++m) c2[m] += (c.round_inter ? bf16r(w[a] * dyt[m]) : w[a] * dyt[m]) * hv;
+            if (a1) {
+                for (int i = 0; i < H; ++i) {
+                    a1[i] += fabs(dgv * xt[i]);
+                    a3[i] += fabs(duv * xt[i]);
+                }
+                for (int m = 0; m < H; ++m)
+                    a2[m] += fabs((c.round_inter ? bf16r(w[a] * dyt[m]) : w[a] * dyt[m]) * hv);
+            }
         }
     }
     free(ids); free(w);

@@ -4,12 +4,20 @@ at small sizes (several tiles, ragged tails, empty experts, k = E, E = 1,
 d_ff not a multiple of 256), sampled rows and columns at the Mixtral expert
 shape, and the transposed weight copies bit for bit.
 
-Tolerance, element by element: |gpu - ref| <= REL |ref| + ABS_RMS rms(ref).
-The GPU rounds to bf16 what it stores between kernels (g, u, h, dg, du and
-w_a dy_t) and every output but dlogits, each rounding at most 2^-9 relative,
-and accumulates in fp32; REL = 2^-6 and ABS_RMS = 2^-7 leave a factor of 8
-(4 for the cancellation term) over one such rounding.  The oracle rounds h
-to bf16 as the forward does (round_h) and is exact otherwise."""
+The oracle rounds to bf16 where the GPU stores bf16 between its kernels (h,
+as the forward does; dg, du and the w_a dy_t entering dW2: round_h and
+round_inter) and is exact otherwise.  What separates the two is then: the
+bf16 rounding of the GPU's outputs (dx and the weight gradients; at most half
+a unit, 2^-9 of the value); an intermediate that the GPU (fp32) and the oracle
+(fp64) round to neighbouring bf16 values, which moves that term of a sum by
+one unit (at most 2^-7 of the term; dW2's terms have two rounded factors);
+and the GPU's fp32 sums (K up to 2F terms: about 2^-9 of the sum of the
+absolute terms).  Tolerance, element by element:
+
+    |gpu - ref| <= REL |ref| + C |ref|_abs,
+
+|ref|_abs the oracle's sum of the absolute values of the entry's terms,
+REL = 2^-8, C = 2^-6 (2^-5 for dW2): twice the unit-flip and summation terms."""
 import numpy as np
 import pytest
 import torch
@@ -19,8 +27,8 @@ import oracle
 
 pytestmark = pytest.mark.gpu
 
-REL = 2.0 ** -6
-ABS_RMS = 2.0 ** -7
+REL = 2.0 ** -8
+C_ABS = {"dx": 2.0 ** -6, "dw1": 2.0 ** -6, "dw3": 2.0 ** -6, "dw2": 2.0 ** -5, "dlogits": 2.0 ** -6}
 
 
 @pytest.fixture(scope="module")
@@ -29,18 +37,19 @@ def moe():
     return m
 
 
-def close(gpu, ref, what):
+def close(gpu, ref, ref_abs, name, what):
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
-    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
+    assert gpu.shape == ref.shape == ref_abs.shape, (what, gpu.shape, ref.shape)
     assert np.all(np.isfinite(gpu)), f"{what}: non-finite values"
     if ref.size == 0:
         return
-    rms = float(np.sqrt(np.mean(ref ** 2)))
     err = np.abs(gpu - ref)
-    bad = err > REL * np.abs(ref) + ABS_RMS * rms
-    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} out of tolerance; worst {err.max():.3e} at "
-                           f"{np.unravel_index(err.argmax(), err.shape)}, rms(ref) {rms:.3e}")
+    allowed = REL * np.abs(ref) + C_ABS[name] * ref_abs
+    ratio = err / np.maximum(allowed, 1e-300)
+    bad = err > allowed
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} out of tolerance; worst {ratio.max():.2f}x "
+                           f"the allowance, at {np.unravel_index(ratio.argmax(), err.shape)}")
 
 
 def f64(t):
@@ -86,9 +95,9 @@ def test_backward_small(moe, p):
     case = moe_inputs.make_case(T, H, F, E, k, "bf16", seed, skew)
     dy = moe_inputs.make_dy(T, H, seed)
     out = run_bwd(moe, case, dy)
-    ref = oracle.ffn_bwd64(*oracle_inputs(case, dy), k, round_h=True)
+    ref = oracle.ffn_bwd64(*oracle_inputs(case, dy), k, round_h=True, round_inter=True, want_abs=True)
     for name in ("dx", "dw1", "dw3", "dw2", "dlogits"):
-        close(f64(out[name]), ref[name], f"{name} T={T} H={H} F={F} E={E} k={k}")
+        close(f64(out[name]), ref[name], ref[name + "_abs"], name, f"{name} T={T} H={H} F={F} E={E} k={k}")
     if skew:
         counts = np.bincount(oracle.route(case["logits"].numpy(), k)["ids"].reshape(-1), minlength=E)
         for e in np.flatnonzero(counts == 0):
@@ -140,10 +149,12 @@ def test_backward_full_size_sampled(moe):
     out = run_bwd(moe, case, dy)
     tokens = np.array([0, 1, 1023, 2048, T - 1], dtype=np.int32)
     feats = np.array([[0, 0], [1, 7000], [3, F - 1], [5, 4097], [7, 128]], dtype=np.int32)
-    ref = oracle.ffn_bwd64_sampled(*oracle_inputs(case, dy), k, tokens, feats, round_h=True)
-    close(f64(out["dx"][torch.from_numpy(tokens).long()]), ref["dx"], "dx (sampled tokens)")
-    close(f64(out["dlogits"][torch.from_numpy(tokens).long()]), ref["dlogits"], "dlogits (sampled tokens)")
+    ref = oracle.ffn_bwd64_sampled(*oracle_inputs(case, dy), k, tokens, feats, round_h=True, round_inter=True,
+                                   want_abs=True)
+    idx = torch.from_numpy(tokens).long()
+    close(f64(out["dx"][idx]), ref["dx"], ref["dx_abs"], "dx", "dx (sampled tokens)")
+    close(f64(out["dlogits"][idx]), ref["dlogits"], ref["dlogits_abs"], "dlogits", "dlogits (sampled tokens)")
     for q, (e, n) in enumerate(feats):
-        close(f64(out["dw1"][e, n]), ref["dw1"][q], f"dw1[{e}, {n}, :]")
-        close(f64(out["dw3"][e, n]), ref["dw3"][q], f"dw3[{e}, {n}, :]")
-        close(f64(out["dw2"][e, :, n]), ref["dw2"][q], f"dw2[{e}, :, {n}]")
+        close(f64(out["dw1"][e, n]), ref["dw1"][q], ref["dw1_abs"][q], "dw1", f"dw1[{e}, {n}, :]")
+        close(f64(out["dw3"][e, n]), ref["dw3"][q], ref["dw3_abs"][q], "dw3", f"dw3[{e}, {n}, :]")
+        close(f64(out["dw2"][e, :, n]), ref["dw2"][q], ref["dw2_abs"][q], "dw2", f"dw2[{e}, :, {n}]")

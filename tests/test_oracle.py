@@ -636,3 +636,52 @@ def test_bwd_sampled_equals_full():
         np.testing.assert_array_equal(s["dw1"][q], full["dw1"][e, n])
         np.testing.assert_array_equal(s["dw3"][q], full["dw3"][e, n])
         np.testing.assert_array_equal(s["dw2"][q], full["dw2"][e, :, n])
+
+
+def test_bwd_rounding_points_move_little():
+    """Rounding the backward's stored intermediates (g, u, dg, du, w_a dy_t)
+    to bf16 moves the gradients by about the bf16 unit, and rounds exactly
+    the values it names: with E = 1 and k = 1, dw1 from the rounded form is
+    the product of bf16 dg and x."""
+    d = _bwd_inputs(30, 16, 32, 4, seed=19)
+    a = oracle.ffn_bwd64(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], 2, round_h=True, round_inter=True)
+    b = oracle.ffn_bwd64(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], 2, round_h=True)
+    for n in ("dx", "dw1", "dw3", "dw2"):
+        rel = np.linalg.norm(a[n] - b[n]) / np.linalg.norm(b[n])
+        assert 0 < rel < 2.0 ** -7, (n, rel)
+    np.testing.assert_array_equal(a["dlogits"], b["dlogits"])  # dw_a sees neither rounding
+    # one token, one expert: dw1 = dg x^T with dg a bf16 value
+    d1 = _bwd_inputs(1, 8, 16, 1, seed=23)
+    g1 = oracle.ffn_bwd64(d1["x"], d1["logits"], d1["w1"], d1["w3"], d1["w2"], d1["dy"], 1, round_h=True,
+                          round_inter=True)
+    x = d1["x"][0]
+    i = int(np.argmax(np.abs(x)))
+    dg = g1["dw1"][0][:, i] / x[i]
+    bits = torch.tensor(dg, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+    np.testing.assert_allclose(dg, bits, rtol=1e-15, atol=0)
+
+
+def test_bwd_error_scales():
+    """The error scales are sums of absolute terms: at least |gradient|
+    everywhere, equal to it where a sum has one term (one token, one expert:
+    dW1 = dg x^T, dW3 = du x^T, dW2 = dO h^T), and the sampled form gives the
+    full form's scales."""
+    d = _bwd_inputs(25, 16, 24, 4, seed=29)
+    g = oracle.ffn_bwd64(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], 2, round_inter=True, want_abs=True)
+    for n in ("dx", "dw1", "dw3", "dw2", "dlogits"):
+        assert np.all(g[n + "_abs"] >= np.abs(g[n]) * (1 - 1e-12)), n
+    assert np.all(g["dx_abs"] > 0)
+    one = _bwd_inputs(1, 8, 16, 1, seed=31)
+    g1 = oracle.ffn_bwd64(one["x"], one["logits"], one["w1"], one["w3"], one["w2"], one["dy"], 1, want_abs=True)
+    for n in ("dw1", "dw3", "dw2"):
+        np.testing.assert_allclose(g1[n + "_abs"], np.abs(g1[n]), rtol=1e-14)
+    tok = np.array([3, 24], dtype=np.int32)
+    feats = np.array([[1, 5], [3, 23]], dtype=np.int32)
+    s = oracle.ffn_bwd64_sampled(d["x"], d["logits"], d["w1"], d["w3"], d["w2"], d["dy"], 2, tok, feats,
+                                 round_inter=True, want_abs=True)
+    np.testing.assert_allclose(s["dx_abs"], g["dx_abs"][tok], rtol=1e-13)
+    np.testing.assert_allclose(s["dlogits_abs"], g["dlogits_abs"][tok], rtol=1e-13)
+    for q, (e, n) in enumerate(feats):
+        np.testing.assert_allclose(s["dw1_abs"][q], g["dw1_abs"][e, n], rtol=1e-13)
+        np.testing.assert_allclose(s["dw3_abs"][q], g["dw3_abs"][e, n], rtol=1e-13)
+        np.testing.assert_allclose(s["dw2_abs"][q], g["dw2_abs"][e, :, n], rtol=1e-13)
