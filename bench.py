@@ -9,9 +9,10 @@ HBM.  The headline workload is the Mixtral-8x7B-shaped FP8 decode layer
 (T=16, d_model=4096, d_ff=14336, E=8, top-2); by default (``--config all``)
 the same run also times every other workload of the Mixtral expert shape
 (prefill T=4096 FP8, skewed-routing T=8192 BF16, the FP8 batch sweep
-T = 1, 128, 1024, 16384, and decode / prefill with MX FP4 expert weights) and
-reports each as a sub-record under ``configs``
-with its own step time, roofline, CPU baseline and end-to-end number.
+T = 1, 128, 1024, 16384, decode / prefill with MX FP4 expert weights, and a
+BF16 training step at T=4096: weight layouts, forward, backward) and reports
+each as a sub-record under ``configs`` with its own step time, roofline, CPU
+baseline and end-to-end number.
 
 With N > 1, one process per GPU (under torch.distributed.run; ``--gpus N``
 without a launcher starts one itself) runs its own token batch against its
@@ -42,7 +43,7 @@ FP8_PER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 HEADLINE = "decode"
 # the workloads of one default run, headline first; the sweep points share one weight set
 ALL_CONFIGS = ["decode", "prefill", "skewed", "sweep_T1", "sweep_T128", "sweep_T1024", "sweep_T16384",
-               "decode_mxfp4", "prefill_mxfp4"]
+               "decode_mxfp4", "prefill_mxfp4", "train_prefill"]
 
 
 def log(*a):
@@ -113,9 +114,10 @@ def config_names(arg):
         return list(ALL_CONFIGS)
     names = [n.strip() for n in arg.split(",") if n.strip()]
     import moe_inputs
+    known = {**moe_inputs.CONFIGS, **moe_inputs.BWD_CONFIGS}
     for n in names:
-        if n not in moe_inputs.CONFIGS:
-            raise SystemExit(f"unknown workload {n!r}; known: {sorted(moe_inputs.CONFIGS)}")
+        if n not in known:
+            raise SystemExit(f"unknown workload {n!r}; known: {sorted(known)}")
     return names
 
 
@@ -249,15 +251,18 @@ class ClockSampler:
         return rec
 
 
-def source_sha():
-    """Hash of the code the grouped-GEMM kernels are compiled from (their
-    translation unit and the library headers it includes; the public header
-    gives them only status codes), comments and blank space removed, so that
-    an edit to a comment keeps the recorded counters."""
+def source_sha(kernel="stage1_w13_swiglu"):
+    """Hash of the code a kernel is compiled from (the grouped GEMMs of the
+    forward: gemm.cu; of the backward: bwd.cu and bwd.cuh; both with the
+    library headers they include -- the public header gives them only status
+    codes), comments and blank space removed, so that an edit to a comment
+    keeps the recorded counters."""
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixture_experts_routed_02_b200", "csrc")
-    for path in [os.path.join(csrc, n) for n in ("gemm.cu", "kernels.cuh", "ptx.cuh")]:
+    files = ("bwd.cu", "bwd.cuh", "kernels.cuh", "ptx.cuh") if kernel.startswith("bwd") else (
+        "gemm.cu", "kernels.cuh", "ptx.cuh")
+    for path in [os.path.join(csrc, n) for n in files]:
         with open(path) as f:
             code = f.read()
         code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)
@@ -275,7 +280,7 @@ def recorded_traffic(kernel, workload):
             recs = json.load(f)
     except (OSError, ValueError):
         return None
-    sha = source_sha()
+    sha = source_sha(kernel)
     for r in recs:
         if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == sha:
             return r.get("dram_bytes_per_launch")
@@ -591,6 +596,186 @@ def run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_s
     return rec
 
 
+def train_cpu_baseline(case, dy, spec, name, seconds):
+    """Time the oracle's backward (as it stands) on sampled tokens of the
+    training workload: per token the forward of its k assignments, dh, the
+    SwiGLU derivative, dx and the router gradient (the sampled form leaves out
+    the weight-gradient outer products)."""
+    import numpy as np
+
+    import moe_inputs
+    import oracle
+    nc = moe_inputs.to_numpy(case)
+    f = oracle.bf16_bits_to_f64
+    args64 = (f(nc["x"]), nc["logits"].astype(np.float64), f(nc["w1"]), f(nc["w3"]), f(nc["w2"]),
+              f(moe_inputs.to_numpy({"dy": dy})["dy"]))
+    T = spec["T"]
+    cores = host_cores()
+    batch = max(1, min(T, cores))
+    done = 0
+    feats = np.zeros((0, 2), dtype=np.int32)
+    t0 = time.perf_counter()
+    i = 0
+    while True:
+        tok = ((np.arange(batch) + i * batch) % T).astype(np.int32)
+        oracle.ffn_bwd64_sampled(*args64, spec["k"], tok, feats, round_h=True, nthreads=cores)
+        done += batch
+        i += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} tokens of the {name} workload ({batch}-token batches): the oracle's sampled backward "
+                      f"(forward of the token's experts, dh, SwiGLU derivative, dx, router gradient; no weight "
+                      f"gradients), {dt:.1f} s"}
+
+
+def run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_seconds):
+    """Time one BF16 training step of the layer: the weight layouts both passes
+    read (redone every step, as weights change), the forward, and the
+    backward (custom VJP: dx, dw1, dw3, dw2, dlogits).  Same structure of
+    record as run_gpu_config."""
+    import torch
+    import torch.distributed as dist
+
+    import moe_inputs
+    T, H, F, E, k = spec["T"], spec["H"], spec["F"], spec["E"], spec["k"]
+    seed = rank_batch(spec, rank)
+    dy_cpu = moe_inputs.make_dy(T, H, seed)
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and cpu_seconds > 0:
+        cb = train_cpu_baseline(case, dy_cpu, spec, name, cpu_seconds)
+    if rank > 0:
+        x_cpu, lg_cpu = moe_inputs.make_x(T, H, seed), moe_inputs.make_logits(T, E, seed, spec["skew"])
+    else:
+        x_cpu, lg_cpu = case["x"], case["logits"]
+    x, logits, dy = x_cpu.to(dev), lg_cpu.to(dev), dy_cpu.to(dev)
+    w1, w3, w2 = case["w1"].to(dev), case["w3"].to(dev), case["w2"].to(dev)
+    prep_f = moe.prepare_weights(w1, w3, None, None, w2)
+    prep_b = moe.prepare_weights_bwd(w1, w3, w2)
+    ws_f = moe.workspace(T, H, F, E, k, "bf16", dev)
+    ws_b = moe.backward_workspace(T, H, F, E, k, dev)
+    y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    grads = moe.ffn_backward(x, logits, w1, w3, prep_b[0], prep_b[1], dy, k, ws=ws_b)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xx=x, lgg=logits, dyy=dy, g=grads):
+        moe.prepare_weights(w1, w3, None, None, w2, stream=stream, out=prep_f)
+        moe.ffn_forward(xx, lgg, prep_f[0], None, prep_f[2], None, k, F, False, out=y, ws=ws_f, stream=stream)
+        moe.prepare_weights_bwd(w1, w3, w2, stream=stream, out=prep_b)
+        moe.ffn_backward(xx, lgg, w1, w3, prep_b[0], prep_b[1], dyy, k, ws=ws_b, out=g, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    st = moe.moe_get_status(None)
+    if st != 0:
+        raise RuntimeError(f"{name}: device status {moe.STATUS_NAMES.get(st, st)} after warm-up")
+    counts = moe.ws_view(ws_f, T, H, F, E, k, "bf16", "counts", torch.int32).cpu().tolist()
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+
+    moe.moe_profile_read(reset=True)
+    moe.moe_profile_enable(1)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    moe.moe_profile_enable(0)
+    kern = moe.moe_profile_read(reset=True)
+    st = moe.moe_get_status(None)
+    if st != 0:
+        raise RuntimeError(f"{name}: device status {moe.STATUS_NAMES.get(st, st)} in the timed region")
+    ms_step = ms_total / args.steps
+    value = T * world * args.steps / (ms_total / 1e3)
+
+    # end to end: x, logits and dy up from pinned host memory, dx and dlogits back, every step
+    e2e = None
+    if not args.no_e2e:
+        x_h, lg_h, dy_h = (t.cpu().pin_memory() for t in (x_cpu, lg_cpu, dy_cpu))
+        dx_h = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+        dl_h = torch.empty(T, E, dtype=torch.float32).pin_memory()
+        xd, lgd, dyd = torch.empty_like(x), torch.empty_like(logits), torch.empty_like(dy)
+
+        def e2e_step():
+            xd.copy_(x_h, non_blocking=True)
+            lgd.copy_(lg_h, non_blocking=True)
+            dyd.copy_(dy_h, non_blocking=True)
+            step(xd, lgd, dyd, grads)
+            dx_h.copy_(grads["dx"], non_blocking=True)
+            dl_h.copy_(grads["dlogits"], non_blocking=True)
+
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        if not torch.equal(dx_h, grads["dx"].cpu()):
+            raise RuntimeError(f"{name}: the dx read back to the host is not the last step's")
+        e2e = {"value": T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": T * H * 2 * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 2 + T * E * 4,
+               "ms_per_step": e2e_ms / args.steps}
+    clk = clocks.stop()
+
+    # roofline of the dominant kernel (tensor-bound at this size): algorithmic
+    # FLOPs per launch from the routed assignments A = T k (padding rows excluded)
+    A = T * k
+    kflops = {"stage1_w13_swiglu": 4.0 * A * F * H, "stage2_w2_scatter": 2.0 * A * F * H,
+              "bwd_gu_recompute": 4.0 * A * F * H, "bwd_dh_swiglu": 2.0 * A * F * H,
+              "bwd_dx_scatter": 4.0 * A * F * H, "bwd_dw2": 2.0 * A * F * H, "bwd_dw13": 4.0 * A * F * H}
+    dom = max(kflops, key=lambda n: kern[n][0])
+    dom_ms = kern[dom][0] / max(1, kern[dom][1])
+    peaks, peak_kind = load_peaks()
+    long_run = ms_total >= 1000.0
+    key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
+    peak = float(peaks.get(key, FALLBACK_PEAKS[key]))
+    ach = kflops[dom] / (dom_ms / 1e3) / 1e12
+    roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+            "traffic": recorded_traffic(dom, name),
+            "peak_source": f"{peak_kind} {'sustained' if long_run else 'burst'} bf16 cuBLAS",
+            "algorithmic_per_launch": kflops[dom], "kernel": dom, "kernel_ms": dom_ms}
+    step_flops = 22.0 * A * F * H  # forward 6, recompute of g/u 4, dh 2, dx 4, dW2 2, dW1/dW3 4
+    launches = sum(v[1] for v in kern.values())
+    wbytes = 3 * E * F * H * 2
+    return {
+        "value": value, "unit": "tokens/s", "ms_per_step": ms_step, "steps": args.steps, "warmup": args.warmup,
+        "dtype": "bf16 (fp32 accumulate)",
+        "config": {"workload": workload_desc(spec, name) + "; training step: weight layouts, forward, backward "
+                   "(dx, dw1, dw3, dw2, dlogits)", "T": T, "d_model": H, "d_ff": F, "experts": E, "top_k": k,
+                   "weights": "bf16", "parallelism": f"weak-scaling replicas x{world}" if world > 1 else "1 GPU",
+                   "l2": "inputs larger than L2 (expert weights %.2f GB, read by several kernels per step)" % (
+                       wbytes / 1e9),
+                   "expert_counts": counts},
+        "roofline": roof,
+        "layer": {"tflops": step_flops / (ms_step / 1e3) / 1e12, "flops_per_step": step_flops},
+        "kernels_ms_per_step": {n: kern[n][0] / args.steps for n in moe.KERNELS if kern[n][1]},
+        "kernel_timing": "separate pass of the same K steps with an event pair around each kernel",
+        "cpu_baseline": cb,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+
+
 def main(argv=None):
     raw_argv = sys.argv[1:] if argv is None else list(argv)
     args = parse(raw_argv)
@@ -628,7 +813,8 @@ def main(argv=None):
     host_w = {}  # host weights of the last (shape, dtype, seed): the sweep points share them
     records = {}
     for i, name in enumerate(names):
-        spec = moe_inputs.CONFIGS[name]
+        train = name in moe_inputs.BWD_CONFIGS
+        spec = moe_inputs.BWD_CONFIGS[name] if train else moe_inputs.CONFIGS[name]
         t0 = time.perf_counter()
         wkey = (spec["H"], spec["F"], spec["E"], spec["dtype"], spec["seed"])
         if wkey not in host_w:
@@ -637,7 +823,12 @@ def main(argv=None):
                                     spec["seed"], spec["skew"], weights=host_w[wkey])
         log(f"[rank {rank}] {name}: inputs generated in {time.perf_counter() - t0:.1f} s")
         cpu_s = args.cpu_sample_seconds if i == 0 else args.sub_cpu_sample_seconds
-        records[name] = run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_s)
+        if train:
+            weights.w = weights.key = None  # the forward workloads' device weights are not needed here
+            torch.cuda.empty_cache()
+            records[name] = run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_s)
+        else:
+            records[name] = run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_s)
         del case
         r = records[name]
         frac = r["roofline"]["frac"]

@@ -338,9 +338,9 @@ typedef enum {
 } moe_option;
 int moe_set_option(int option, int value);
 
-/* Per-kernel device timing (tracing aid).  While enabled, moe_ffn_forward
- * and moe_ffn_backward record a pair of CUDA events around each step they
- * enqueue (routing is one kernel for small batches and two from 1024 tokens
+/* Per-kernel device timing (tracing aid).  While enabled, moe_ffn_forward,
+ * moe_ffn_backward and the weight preparations record a pair of CUDA events
+ * around each step they enqueue (routing is one kernel for small batches and two from 1024 tokens
  * on; both are counted in `launches` and timed together; the backward's
  * routing, gathers, transposes, rounding of dx and router gradient are timed
  * together as MOE_KERNEL_BWD_AUX).
@@ -361,7 +361,8 @@ typedef enum {
     MOE_KERNEL_BWD_DW2 = 8,  /* backward: dW2 per expert */
     MOE_KERNEL_BWD_DW13 = 9, /* backward: dW1, dW3 per expert */
     MOE_KERNEL_BWD_AUX = 10, /* backward: routing, gathers, transposes, dx rounding, router gradient */
-    MOE_KERNEL_COUNT = 11
+    MOE_KERNEL_PREPARE = 11, /* moe_prepare_weights, _mx and _bwd (weight layouts) */
+    MOE_KERNEL_COUNT = 12
 } moe_kernel_id;
 int moe_profile_enable(int on);
 int moe_profile_read(double* ms_total, int* launches, int reset);

@@ -59,7 +59,7 @@ EXPORTS = ["moe_workspace_size", "moe_prepare_weights", "moe_route", "moe_ffn_fo
 # kernel ids of moe_profile_read: the forward's five, then the backward's
 FWD_KERNELS = ["route", "quantize", "stage1_w13_swiglu", "stage2_w2_scatter", "finalize"]
 BWD_KERNELS = ["bwd_gu_recompute", "bwd_dh_swiglu", "bwd_dx_scatter", "bwd_dw2", "bwd_dw13", "bwd_aux"]
-KERNELS = FWD_KERNELS + BWD_KERNELS
+KERNELS = FWD_KERNELS + BWD_KERNELS + ["prepare_weights"]
 
 
 class MoeError(RuntimeError):
@@ -211,9 +211,10 @@ def prepare_weights_mx(w1, w3, s1, s3, w2, s2, stream=None):
     return w13, s13, w2p, s2p
 
 
-def prepare_weights(w1, w3, s1, s3, w2, stream=None):
+def prepare_weights(w1, w3, s1, s3, w2, stream=None, out=None):
     """One-time preshuffle: returns (w13, s13, w2p) in the blocked layouts the
-    kernels stream (w13/w2p are flat byte tensors; s13 [E,2F] or None)."""
+    kernels stream (w13/w2p are flat byte tensors; s13 [E,2F] or None).
+    ``out``: an earlier result to write into (training: every step)."""
     import torch
     for t in (w1, w3, w2):
         if t.dtype not in (torch.bfloat16, torch.float8_e4m3fn) or t.dtype != w1.dtype or not t.is_contiguous():
@@ -223,9 +224,12 @@ def prepare_weights(w1, w3, s1, s3, w2, stream=None):
     if w3.shape != (E, F, H) or w2.shape != (E, H, F):
         raise ValueError(f"weight shapes {tuple(w1.shape)}, {tuple(w3.shape)}, {tuple(w2.shape)} do not match")
     fp8 = w1.dtype == torch.float8_e4m3fn
-    w13 = torch.empty(E * 2 * F * H * w1.element_size(), dtype=torch.uint8, device=w1.device)
-    w2p = torch.empty(w2.numel() * w2.element_size(), dtype=torch.uint8, device=w2.device)
-    s13 = torch.empty(E, 2 * F, dtype=torch.float32, device=w1.device) if fp8 else None
+    if out is not None:
+        w13, s13, w2p = out
+    else:
+        w13 = torch.empty(E * 2 * F * H * w1.element_size(), dtype=torch.uint8, device=w1.device)
+        w2p = torch.empty(w2.numel() * w2.element_size(), dtype=torch.uint8, device=w2.device)
+        s13 = torch.empty(E, 2 * F, dtype=torch.float32, device=w1.device) if fp8 else None
     rc = moe_prepare_weights(_ptr(w1), _ptr(w3), _ptr(s1) if fp8 else None, _ptr(s3) if fp8 else None, _ptr(w2),
                              _ptr(w13), _ptr(s13), _ptr(w2p), E, F, H, MOE_FP8_E4M3 if fp8 else MOE_BF16,
                              _stream(stream))
@@ -326,9 +330,10 @@ def dff_finalize(out32_rows, out, counter, target, stream=None):
 
 # ---------------------------------------------------------------- backward pass (BF16)
 
-def prepare_weights_bwd(w1, w3, w2, stream=None):
+def prepare_weights_bwd(w1, w3, w2, stream=None, out=None):
     """Transposed copies the backward reads (redo after each weight update):
-    w13t [E,H,2F] = [w1^T | w3^T] per expert and w2t [E,F,H] = w2^T, bf16."""
+    w13t [E,H,2F] = [w1^T | w3^T] per expert and w2t [E,F,H] = w2^T, bf16.
+    ``out``: an earlier (w13t, w2t) to write into."""
     import torch
     for t in (w1, w3, w2):
         if t.dtype != torch.bfloat16 or not t.is_contiguous():
@@ -336,8 +341,11 @@ def prepare_weights_bwd(w1, w3, w2, stream=None):
     E, F, H = w1.shape
     if w3.shape != (E, F, H) or w2.shape != (E, H, F):
         raise ValueError("weight shapes do not match")
-    w13t = torch.empty(E, H, 2 * F, dtype=torch.bfloat16, device=w1.device)
-    w2t = torch.empty(E, F, H, dtype=torch.bfloat16, device=w1.device)
+    if out is not None:
+        w13t, w2t = out
+    else:
+        w13t = torch.empty(E, H, 2 * F, dtype=torch.bfloat16, device=w1.device)
+        w2t = torch.empty(E, F, H, dtype=torch.bfloat16, device=w1.device)
     _check("moe_prepare_weights_bwd", moe_prepare_weights_bwd(_ptr(w1), _ptr(w3), _ptr(w2), _ptr(w13t), _ptr(w2t),
                                                               E, F, H, _stream(stream)))
     return w13t, w2t

@@ -408,6 +408,7 @@ int moe_prepare_weights(const void* w1, const void* w3, const float* s1, const f
         if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
     const int eb = fp8 ? 1 : 2;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ProfScope ps(MOE_KERNEL_PREPARE, st, fp8 ? 3 : 2);
     if (launch_preshuffle(static_cast<const uint8_t*>(w1), static_cast<const uint8_t*>(w3),
                           static_cast<uint8_t*>(w13_out), E, F, 2 * F, H * eb, true, st) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -428,9 +429,8 @@ int moe_prepare_weights_mx(const void* w1, const void* w3, const void* s1, const
     const void* ptrs[] = {w1, w3, s1, s3, w2, s2, w13_out, s13_out, w2_out, s2_out};
     for (const void* p : ptrs)
         if (!aligned16(p)) return MOE_ERR_ALIGNMENT;
-    // the packed rows are read by TMA: 32-byte aligned bases
-    if ((reinterpret_cast<uintptr_t>(w13_out) | reinterpret_cast<uintptr_t>(w2_out)) & 31u) return MOE_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ProfScope ps(MOE_KERNEL_PREPARE, st, 4);
     auto u8 = [](const void* p) { return static_cast<const uint8_t*>(p); };
     if (launch_mx_prepare(u8(w1), u8(w3), u8(s1), u8(s3), static_cast<uint8_t*>(w13_out),
                           static_cast<uint8_t*>(s13_out), E, F, 2 * F, H, true, st) != cudaSuccess)
@@ -818,6 +818,7 @@ int moe_prepare_weights_bwd(const void* w1, const void* w3, const void* w2, void
     if (!aligned16(w1) || !aligned16(w3) || !aligned16(w2) || !aligned16(w13t_out) || !aligned16(w2t_out))
         return MOE_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ProfScope ps(MOE_KERNEL_PREPARE, st, 3);
     TransposeArgs p{};
     // w13t[e][h][c] = w1[e][c][h] (c < F), w3[e][c - F][h] (c >= F)
     p.src_pitch = H;

@@ -43,7 +43,7 @@ def test_bf16_weights_count_two_bytes_and_no_scales():
 
 def test_recorded_traffic_needs_the_same_kernel_code(monkeypatch):
     assert bench.recorded_traffic("stage1_w13_swiglu", "no-such-workload") is None
-    monkeypatch.setattr(bench, "source_sha", lambda: "0000000000000000")
+    monkeypatch.setattr(bench, "source_sha", lambda kernel="": "0000000000000000")
     assert bench.recorded_traffic("stage1_w13_swiglu", "decode") is None
 
 
@@ -94,12 +94,14 @@ def test_clock_samples(lines, reasons, median):
 
 def test_default_run_times_every_mixtral_workload():
     """The default bench run (`--config all`) times the headline decode layer
-    first and every other Mixtral-shaped workload after it."""
+    first and every other Mixtral-shaped workload after it, the training step
+    (forward + backward) included."""
     import moe_inputs
     names = bench.config_names("all")
     assert names[0] == bench.HEADLINE == "decode"
-    assert set(names) == set(moe_inputs.CONFIGS) - {"tiny"}
+    assert set(names) == (set(moe_inputs.CONFIGS) - {"tiny"}) | set(moe_inputs.BWD_CONFIGS)
     assert bench.config_names("prefill,sweep_T1") == ["prefill", "sweep_T1"]
+    assert bench.config_names("train_prefill") == ["train_prefill"]
     with pytest.raises(SystemExit):
         bench.config_names("no-such-workload")
 
