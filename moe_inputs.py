@@ -22,6 +22,7 @@ sweep_T<n>     n      4096   14336  8   2  fp8    4     n in {1, 128, 1024, 1638
 decode_mxfp4   16     4096   14336  8   2  mxfp4  5     MX FP4 expert weights
 prefill_mxfp4  4096   4096   14336  8   2  mxfp4  6     MX FP4 expert weights
 train_prefill  4096   4096   14336  8   2  bf16   7     backward pass (BWD_CONFIGS)
+train_small    1024   1024   3584   8   2  bf16   8     backward, small case for profiler captures
 =============  =====  =====  =====  ==  =  =====  ====  =================================
 
 Distributions: x ~ N(0,1) rounded to bf16; router logits ~ N(0,1) fp32;
@@ -58,6 +59,8 @@ CONFIGS["prefill_mxfp4"] = _spec(4096, H_MIXTRAL, F_MIXTRAL, 8, 2, "mxfp4", 6)
 # backward pass (training) workloads: BF16 weights, an upstream gradient dy
 BWD_CONFIGS = {
     "train_prefill": _spec(4096, H_MIXTRAL, F_MIXTRAL, 8, 2, "bf16", 7),
+    # a quarter-width expert shape: the small case for detailed profiler captures
+    "train_small": _spec(1024, 1024, 3584, 8, 2, "bf16", 8),
 }
 
 # stream ids of the generators

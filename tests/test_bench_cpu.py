@@ -99,9 +99,9 @@ def test_default_run_times_every_mixtral_workload():
     import moe_inputs
     names = bench.config_names("all")
     assert names[0] == bench.HEADLINE == "decode"
-    assert set(names) == (set(moe_inputs.CONFIGS) - {"tiny"}) | set(moe_inputs.BWD_CONFIGS)
+    assert set(names) == (set(moe_inputs.CONFIGS) - {"tiny"}) | {"train_prefill"}
     assert bench.config_names("prefill,sweep_T1") == ["prefill", "sweep_T1"]
-    assert bench.config_names("train_prefill") == ["train_prefill"]
+    assert bench.config_names("train_small") == ["train_small"]  # the profiler's small training case
     with pytest.raises(SystemExit):
         bench.config_names("no-such-workload")
 
