@@ -301,7 +301,10 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
  *                     tiles (32 activation rows per stage; only for at most
  *                     32 assignments, else MOE_ERR_UNSUPPORTED).  MX FP4
  *                     weights run on 128 x 128 one-SM tiles only: 4 forces
- *                     their tiny-batch form, 1-3 the other one.
+ *                     their tiny-batch form, 1-3 the other one.  The
+ *                     backward's GEMMs take 256 x 256 tiles on pairs of SMs
+ *                     where the tile is 256 wide (0, 1) or one-SM tiles
+ *                     only (2, 3, 4).
  *   MOE_OPT_SPLITK:   0 = automatic, n > 0 = split the second GEMM's K into n parts
  *                     (must divide F/128).
  *   MOE_OPT_TIMEOUT_MS: limit of every device-side wait (default 2000).

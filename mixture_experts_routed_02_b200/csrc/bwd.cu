@@ -36,17 +36,26 @@ namespace moe {
 
 namespace {
 
-template <int BN, int NST>
+// PAIR: a cluster of two CTAs on two SMs computes a 256 x BN tile with
+// tcgen05.mma.cta_group::2 -- each CTA copies its own 128 rows of A and half
+// of B's BN rows, all copies complete on the even CTA's barriers, the even
+// CTA issues the MMAs, and each CTA's TMEM receives its own 128 rows.  Per
+// unit of work a CTA moves a third less operand data than on one SM, and a
+// stage of 32 KB instead of 48 leaves room for six stages.
+template <int BN, int NST, bool PAIR>
 struct BCfg {
     static constexpr int A_BYTES = kBlockM * 128;  // 128 rows x 64 bf16
-    static constexpr int B_BYTES = BN * 128;
+    static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // this CTA's rows of B
+    static constexpr int B_BYTES = B_ROWS * 128;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;  // on the even CTA's full barrier
     static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;  // two accumulators
     static constexpr int OFF_BAR = NST * STAGE_BYTES;
     static constexpr int NUM_BARS = 2 * NST + 5;  // full, empty, tfull[2], tempty[2], drain
     static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-    static constexpr uint32_t IDESC = idesc_bf16(kBlockM, BN);
+    static_assert(B_ROWS % 128 == 0, "B copies of 128 rows");
+    static constexpr uint32_t IDESC = idesc_bf16(PAIR ? 2 * kBlockM : kBlockM, BN);
 };
 
 __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
@@ -75,11 +84,11 @@ __device__ __forceinline__ float logistic(float g) { return __fdividef(1.0f, 1.0
 
 }  // namespace
 
-template <int MODE, int BN, int NST>
+template <int MODE, int BN, int NST, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmB2, const BwdArgs args) {
-    using C = BCfg<BN, NST>;
+    using C = BCfg<BN, NST, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -92,7 +101,16 @@ __global__ void __launch_bounds__(192, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t limit = args.timeout_ns;
-    auto wait = [&](uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, abort_flag, limit, args.status); };
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit0 = PAIR ? (int)blockIdx.x / 2 : (int)blockIdx.x;
+    const int ustep = PAIR ? (int)gridDim.x / 2 : (int)gridDim.x;
+    // a wait that gives up tells the other CTA of the pair to give up too
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+        const bool ok = mbar_wait(bar, parity, abort_flag, limit, args.status);
+        if (PAIR && !ok) st_cluster_u32(mapa_shared(smem_u32((const void*)abort_flag), rank ^ 1u), 1u);
+        return ok;
+    };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NST; ++i) {
@@ -101,50 +119,70 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 4);
+            mbar_init(&tempty[i], PAIR ? 8 : 4);  // the epilogue warps of both CTAs release a pair tile
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
         if (MODE == kBwdGU) prefetch_tmap(&tmB2);
     }
-    // DW: first 128-row tile of each expert in the slot layout (scan of the
-    // per-expert tile counts)
+    // first 128-row tile of each expert in the slot layout (DW: K ranges; row
+    // modes on pairs: the pairs of an expert's tiles), and first pair of tiles
     __shared__ int s_mt_first[kMaxExperts + 1];
-    if (MODE == kBwdDW && warp == 2) {
-        int carry = 0;
+    __shared__ int s_pair_first[kMaxExperts + 1];
+    if ((MODE == kBwdDW || PAIR) && warp == 2) {
+        int carry = 0, carry_p = 0;
         for (int base = 0; base < args.num_experts; base += 32) {
             const int e = base + lane;
             int v = (e < args.num_experts) ? (args.counts[e] + kBlockM - 1) / kBlockM : 0;
+            int vp = (v + 1) / 2;
 #pragma unroll
             for (int d = 1; d < 32; d <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, v, d);
-                if (lane >= d) v += y;
+                const int yp = __shfl_up_sync(0xffffffffu, vp, d);
+                if (lane >= d) {
+                    v += y;
+                    vp += yp;
+                }
             }
-            if (e < args.num_experts) s_mt_first[e + 1] = carry + v;
+            if (e < args.num_experts) {
+                s_mt_first[e + 1] = carry + v;
+                s_pair_first[e + 1] = carry_p + vp;
+            }
             carry += __shfl_sync(0xffffffffu, v, 31);
+            carry_p += __shfl_sync(0xffffffffu, vp, 31);
         }
-        if (lane == 0) s_mt_first[0] = 0;
+        if (lane == 0) {
+            s_mt_first[0] = 0;
+            s_pair_first[0] = 0;
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrival
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    // work units: row modes -> (m-tile of slots, n-tile); DW -> (expert, m-tile
-    // of output rows, n-tile), experts slowest so a wave shares operands in L2
+    // work units: row modes -> (m-tile of slots, or pair of an expert's
+    // m-tiles; n-tile); DW -> (expert, m-tile or pair of m-tiles of output
+    // rows, n-tile), experts slowest so a wave shares operands in L2
     int units;
     int num_mt = 0;
     if constexpr (MODE == kBwdDW) {
-        units = args.num_experts * args.m_tiles * args.n_tiles;
+        units = args.num_experts * (PAIR ? args.m_tiles / 2 : args.m_tiles) * args.n_tiles;
         if (s_mt_first[args.num_experts] > args.mt_max) {  // never from the router: corrupted counts
             if (threadIdx.x == 0) record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
             units = 0;
@@ -155,18 +193,52 @@ __global__ void __launch_bounds__(192, 1)
             if (threadIdx.x == 0) record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
             num_mt = 0;
         }
-        units = num_mt * args.n_tiles;
+        units = PAIR ? s_pair_first[args.num_experts] * args.n_tiles : num_mt * args.n_tiles;
+        if (PAIR && s_mt_first[args.num_experts] != num_mt) {  // never from the router
+            if (threadIdx.x == 0) record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
+            units = 0;
+        }
     }
-    // unit -> (e, m, n, first K step, K steps)
-    auto unit_coords = [&](int u, int& e, int& m, int& n, int& k0, int& kc) {
+    // unit -> (e, this CTA's m-tile, n, first K step, K steps); `dup` marks the
+    // second half of a pair that repeats the first (an expert with an odd
+    // number of m-tiles: its results are not stored)
+    auto unit_coords = [&](int u, int& e, int& m, int& n, int& k0, int& kc, bool& dup) {
+        dup = false;
         if constexpr (MODE == kBwdDW) {
-            const int per_e = args.m_tiles * args.n_tiles;
+            const int mt = PAIR ? args.m_tiles / 2 : args.m_tiles;
+            const int per_e = mt * args.n_tiles;
             e = u / per_e;
             const int r = u - e * per_e;
-            m = r % args.m_tiles;
-            n = r / args.m_tiles;
+            m = PAIR ? 2 * (r % mt) + (int)rank : r % mt;
+            n = r / mt;
             k0 = 2 * s_mt_first[e];  // 64 slots per K step, 128 slots per tile
             kc = 2 * (s_mt_first[e + 1] - s_mt_first[e]);
+        } else if constexpr (PAIR) {
+            const int p = u / args.n_tiles;
+            int lo = 0, hi = args.num_experts;  // largest e with s_pair_first[e] <= p
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (s_pair_first[mid] <= p) lo = mid;
+                else hi = mid;
+            }
+            e = lo;
+            const int cnt = s_pair_first[e + 1] - s_pair_first[e];
+            k0 = 0;
+            kc = args.k_tiles;
+            if (cnt > 0 && p < s_pair_first[e + 1]) {
+                const int local = u - s_pair_first[e] * args.n_tiles;
+                const int m0 = s_mt_first[e] + 2 * (local % cnt);
+                n = local / cnt;
+                const bool odd = m0 + 1 >= s_mt_first[e + 1];
+                m = (rank == 0 || odd) ? m0 : m0 + 1;
+                dup = (rank == 1) && odd;
+                return;
+            }
+            record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
+            e = 0;
+            m = 0;
+            n = 0;
+            dup = true;
         } else {
             m = u % num_mt;
             n = u / num_mt;
@@ -187,9 +259,10 @@ __global__ void __launch_bounds__(192, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            for (int u = unit0; u < units && ok; u += ustep) {
                 int e, m, n, k0, kc;
-                unit_coords(u, e, m, n, k0, kc);
+                bool dup;
+                unit_coords(u, e, m, n, k0, kc, dup);
                 for (int kk = 0; kk < kc; ++kk) {
                     if (!wait(&empty[stage], phase ^ 1)) {
                         ok = false;
@@ -198,18 +271,33 @@ __global__ void __launch_bounds__(192, 1)
                     uint8_t* sa = smem + stage * C::STAGE_BYTES;
                     uint8_t* sb = sa + C::A_BYTES;
                     const int kx = (k0 + kk) * 64;
-                    mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-                    tma_load_2d(sa, &tmA, &full[stage], kx, m * kBlockM, pol_a);
-                    if constexpr (MODE == kBwdGU) {
-                        // 128 rows of W1_e and the same 128 rows of W3_e: the tile's
-                        // first 128 columns are g, the last 128 u, of the same features
-                        tma_load_2d(sb, &tmB, &full[stage], kx, e * args.b_rows + n * 128, pol_b);
-                        tma_load_2d(sb + 128 * 128, &tmB2, &full[stage], kx, e * args.b_rows + n * 128, pol_b);
-                    } else {
-                        const int brow = (MODE == kBwdDW ? 0 : e * args.b_rows) + n * BN;
+                    if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+                    // B rows of this CTA: GU -- 128 rows of W1_e and the same 128
+                    // rows of W3_e (the tile's first 128 columns are g, the last 128
+                    // u, of the same features; on a pair each CTA holds one of the
+                    // two); otherwise BN rows, or this CTA's half of them
+                    if constexpr (PAIR) {
+                        const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+                        tma_load_2d_pair(sa, &tmA, bar, kx, m * kBlockM, pol_a);
+                        if constexpr (MODE == kBwdGU) {
+                            tma_load_2d_pair(sb, rank == 0 ? &tmB : &tmB2, bar, kx, e * args.b_rows + n * 128, pol_b);
+                        } else {
+                            const int brow = (MODE == kBwdDW ? 0 : e * args.b_rows) + n * BN + (int)rank * C::B_ROWS;
 #pragma unroll
-                        for (int j = 0; j < BN / 128; ++j)
-                            tma_load_2d(sb + j * 128 * 128, &tmB, &full[stage], kx, brow + 128 * j, pol_b);
+                            for (int j = 0; j < C::B_ROWS / 128; ++j)
+                                tma_load_2d_pair(sb + j * 128 * 128, &tmB, bar, kx, brow + 128 * j, pol_b);
+                        }
+                    } else {
+                        tma_load_2d(sa, &tmA, &full[stage], kx, m * kBlockM, pol_a);
+                        if constexpr (MODE == kBwdGU) {
+                            tma_load_2d(sb, &tmB, &full[stage], kx, e * args.b_rows + n * 128, pol_b);
+                            tma_load_2d(sb + 128 * 128, &tmB2, &full[stage], kx, e * args.b_rows + n * 128, pol_b);
+                        } else {
+                            const int brow = (MODE == kBwdDW ? 0 : e * args.b_rows) + n * BN;
+#pragma unroll
+                            for (int j = 0; j < BN / 128; ++j)
+                                tma_load_2d(sb + j * 128 * 128, &tmB, &full[stage], kx, brow + 128 * j, pol_b);
+                        }
                     }
                     if (++stage == NST) {
                         stage = 0;
@@ -220,15 +308,25 @@ __global__ void __launch_bounds__(192, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && leader) {
+            // arrival on a barrier of both CTAs (pair) or of this CTA
+            auto commit = [&](uint64_t* bar) {
+                if constexpr (PAIR) {
+                    tc_commit_pair(smem_u32(bar));
+                    tc_commit_pair(mapa_shared(smem_u32(bar), 1));
+                } else {
+                    tc_commit(bar);
+                }
+            };
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            for (int u = unit0; u < units && ok; u += ustep) {
                 int e, m, n, k0, kc;
-                unit_coords(u, e, m, n, k0, kc);
+                bool dup;
+                unit_coords(u, e, m, n, k0, kc, dup);
                 if (!wait(&tempty[acc], acc_phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
@@ -241,24 +339,41 @@ __global__ void __launch_bounds__(192, 1)
                     const uint32_t a_addr = smem_u32(smem + stage * C::STAGE_BYTES);
                     const uint32_t b_addr = a_addr + C::A_BYTES;
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16(d_tmem, sdesc_sw128(a_addr + ks * 32), sdesc_sw128(b_addr + ks * 32), C::IDESC,
-                                 (kk > 0 || ks > 0) ? 1u : 0u);
-                    tc_commit(&empty[stage]);
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = sdesc_sw128(a_addr + ks * 32), bd = sdesc_sw128(b_addr + ks * 32);
+                        const uint32_t accum = (kk > 0 || ks > 0) ? 1u : 0u;
+                        if constexpr (PAIR) mma_bf16_pair(d_tmem, ad, bd, C::IDESC, accum);
+                        else mma_bf16(d_tmem, ad, bd, C::IDESC, accum);
+                    }
+                    commit(&empty[stage]);
                     if (++stage == NST) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
                 if (!ok) break;
-                tc_commit(&tfull[acc]);  // (no MMA for an expert without slots: the epilogue writes zeros)
+                commit(&tfull[acc]);  // (no MMA for an expert without slots: the epilogue writes zeros)
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1;
                 }
             }
             volatile int keep_waiting = 0;
-            tc_commit(drain);
+            if constexpr (PAIR) {
+                // both CTAs' epilogues have released every accumulator, so no
+                // arrival from the other CTA is still on its way to this one
+                for (int i = 0; i < 2; ++i) {
+                    if (!mbar_wait(&tempty[acc], acc_phase ^ 1, ok ? &keep_waiting : abort_flag, limit, args.status))
+                        break;
+                    if (++acc == 2) {
+                        acc = 0;
+                        acc_phase ^= 1;
+                    }
+                }
+            }
+            // every MMA issued by this thread has finished before TMEM is released
+            if constexpr (PAIR) tc_commit_pair(smem_u32(drain));
+            else tc_commit(drain);
             mbar_wait(drain, 0, &keep_waiting, limit, args.status);
         }
         __syncwarp();
@@ -271,18 +386,22 @@ __global__ void __launch_bounds__(192, 1)
         auto release = [&](int a) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[a]);
+            if (lane == 0) {
+                if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[a]), 0));
+                else mbar_arrive(&tempty[a]);
+            }
         };
-        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        for (int u = unit0; u < units; u += ustep) {
             int e, m, n, k0, kc;
-            unit_coords(u, e, m, n, k0, kc);
+            bool dup;
+            unit_coords(u, e, m, n, k0, kc, dup);
             if (!wait(&tfull[acc], acc_phase)) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             const int slot = m * kBlockM + row;
             int a = -1;
             if constexpr (MODE != kBwdDW) {
-                a = args.slot_assign[slot];
+                a = dup ? -1 : args.slot_assign[slot];
                 if (a < -1 || a >= args.T * args.topk) {  // never from the router
                     record_error(args.status, MOE_ERR_DEVICE_BOUNDS);
                     a = -1;
@@ -422,10 +541,13 @@ __global__ void __launch_bounds__(192, 1)
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();  // no cross-CTA traffic after this point
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+        else tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
+    if constexpr (PAIR) cluster_sync_all();
 }
 
 // ---------------------------------------------------------------- transposes
@@ -528,34 +650,80 @@ __global__ void dlogits_kernel(const int32_t* __restrict__ ids, const float* __r
 
 namespace {
 
-template <int MODE, int BN, int NST>
+template <int MODE, int BN, int NST, bool PAIR>
 cudaError_t launch_bwd_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const BwdArgs& args,
                            int grid, cudaStream_t stream) {
-    using C = BCfg<BN, NST>;
-    auto kern = bwd_gemm_kernel<MODE, BN, NST>;
+    using C = BCfg<BN, NST, PAIR>;
+    auto kern = bwd_gemm_kernel<MODE, BN, NST, PAIR>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    kern<<<grid, 192, C::SMEM_BYTES, stream>>>(a, b, b2, args);
-    return cudaGetLastError();
+    if constexpr (PAIR) {
+        if (grid < 2 || grid % 2) return cudaErrorInvalidValue;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(192);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kern, a, b, b2, args);
+    } else {
+        kern<<<grid, 192, C::SMEM_BYTES, stream>>>(a, b, b2, args);
+        return cudaGetLastError();
+    }
+}
+
+template <int MODE>
+int max_pairs_one() {
+    using C = BCfg<256, 6, true>;
+    auto kern = bwd_gemm_kernel<MODE, 256, 6, true>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+        return 0;
+    return max_active_clusters(kern, 192, C::SMEM_BYTES, 2);
 }
 
 }  // namespace
 
-cudaError_t launch_bwd_gemm(int mode, int bn, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
-                            const BwdArgs& args, int grid, cudaStream_t stream) {
+// Clusters of two CTAs of the 256 x 256 backward GEMM that can be resident
+// at once (0 if none can: then the one-SM tiles run).
+int bwd_max_pairs(int mode) {
+    switch (mode) {
+        case kBwdGU: return max_pairs_one<kBwdGU>();
+        case kBwdDH: return max_pairs_one<kBwdDH>();
+        case kBwdDX: return max_pairs_one<kBwdDX>();
+        case kBwdDW: return max_pairs_one<kBwdDW>();
+        default: return 0;
+    }
+}
+
+// bn = 256: 128 x 256 tiles on one SM, or 256 x 256 on a pair (pair); bn =
+// 128: 128 x 128 tiles on one SM (a dimension not a multiple of 256).
+cudaError_t launch_bwd_gemm(int mode, int bn, bool pair, const CUtensorMap& a, const CUtensorMap& b,
+                            const CUtensorMap& b2, const BwdArgs& args, int grid, cudaStream_t stream) {
     if (grid < 1) return cudaSuccess;
+    if (pair && bn != 256) return cudaErrorInvalidValue;
     switch (mode) {
         case kBwdGU:
-            return bn == 256 ? launch_bwd_one<kBwdGU, 256, 4>(a, b, b2, args, grid, stream) : cudaErrorInvalidValue;
+            if (bn != 256) return cudaErrorInvalidValue;
+            return pair ? launch_bwd_one<kBwdGU, 256, 6, true>(a, b, b2, args, grid, stream)
+                        : launch_bwd_one<kBwdGU, 256, 4, false>(a, b, b2, args, grid, stream);
         case kBwdDH:
-            return bn == 256 ? launch_bwd_one<kBwdDH, 256, 4>(a, b, b2, args, grid, stream)
-                             : launch_bwd_one<kBwdDH, 128, 6>(a, b, b2, args, grid, stream);
+            return pair ? launch_bwd_one<kBwdDH, 256, 6, true>(a, b, b2, args, grid, stream)
+                 : bn == 256 ? launch_bwd_one<kBwdDH, 256, 4, false>(a, b, b2, args, grid, stream)
+                             : launch_bwd_one<kBwdDH, 128, 6, false>(a, b, b2, args, grid, stream);
         case kBwdDX:
-            return bn == 256 ? launch_bwd_one<kBwdDX, 256, 4>(a, b, b2, args, grid, stream)
-                             : launch_bwd_one<kBwdDX, 128, 6>(a, b, b2, args, grid, stream);
+            return pair ? launch_bwd_one<kBwdDX, 256, 6, true>(a, b, b2, args, grid, stream)
+                 : bn == 256 ? launch_bwd_one<kBwdDX, 256, 4, false>(a, b, b2, args, grid, stream)
+                             : launch_bwd_one<kBwdDX, 128, 6, false>(a, b, b2, args, grid, stream);
         case kBwdDW:
-            return bn == 256 ? launch_bwd_one<kBwdDW, 256, 4>(a, b, b2, args, grid, stream)
-                             : launch_bwd_one<kBwdDW, 128, 6>(a, b, b2, args, grid, stream);
+            return pair ? launch_bwd_one<kBwdDW, 256, 6, true>(a, b, b2, args, grid, stream)
+                 : bn == 256 ? launch_bwd_one<kBwdDW, 256, 4, false>(a, b, b2, args, grid, stream)
+                             : launch_bwd_one<kBwdDW, 128, 6, false>(a, b, b2, args, grid, stream);
         default:
             return cudaErrorInvalidValue;
     }

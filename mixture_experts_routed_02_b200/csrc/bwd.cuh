@@ -37,8 +37,11 @@ struct BwdArgs {
     unsigned long long timeout_ns;
     int* status;
 };
-cudaError_t launch_bwd_gemm(int mode, int bn, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
-                            const BwdArgs& args, int grid, cudaStream_t stream);
+// bn = 256 (128 x 256 tiles on one SM, or 256 x 256 on a pair of SMs when
+// `pair`) or 128 (128 x 128 on one SM); grid = CTAs (pairs: an even number).
+cudaError_t launch_bwd_gemm(int mode, int bn, bool pair, const CUtensorMap& a, const CUtensorMap& b,
+                            const CUtensorMap& b2, const BwdArgs& args, int grid, cudaStream_t stream);
+int bwd_max_pairs(int mode);  // resident clusters of the pair kernel (0: none)
 
 // out[c][out_col + s] = row s of the source, column c (bf16, 64 x 64 tiles):
 enum TransposeSrc {

@@ -930,7 +930,27 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
     base.F = F;
     base.timeout_ns = timeout_ns;
     base.status = status;
-    auto row_grid = [&](int n_tiles) { return (int)std::min<long>((long)L.MT_max * n_tiles, num_sms); };
+    // one CTA per SM at most; pairs: whole clusters that can be resident.
+    // Pairs wherever the tile is 256 wide (DW: an even number of 128-row
+    // output tiles); the pair kernels' residency is looked up once per context.
+    const int opt_path = g_opt_path.load();  // 2, 3 or 4: one-SM tiles only
+    auto pairs_for = [&](int mode) {
+        if (opt_path >= 2) return 0;
+        static std::mutex mu;
+        static unsigned long long key[4] = {0, 0, 0, 0};
+        static int val[4] = {0, 0, 0, 0};
+        std::lock_guard<std::mutex> lock(mu);
+        if (key[mode] != ctx.ctx_id) {
+            val[mode] = bwd_max_pairs(mode);
+            key[mode] = ctx.ctx_id;
+        }
+        return val[mode];
+    };
+    auto grid_for = [&](int mode, bool pair, long units) {
+        if (pair) return (int)(2 * std::max<long>(1, std::min<long>(units, pairs_for(mode))));
+        return (int)std::max<long>(1, std::min<long>(units, num_sms));
+    };
+    const long mt_pairs = (L.MT_max + 1) / 2 + E;  // upper bound of the m-tile pairs over all experts
 
     // 2. g, u, h recomputed
     {
@@ -942,8 +962,10 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.out_pitch = p8F;
         a.out2 = reg(MOE_WS_H);
         a.out2_pitch = p2F;
+        const bool pair = pairs_for(kBwdGU) > 0;
         ProfScope ps(MOE_KERNEL_BWD_GU, st);
-        if (launch_bwd_gemm(kBwdGU, 256, mXg, mW1, mW3, a, row_grid(a.n_tiles), st) != cudaSuccess)
+        if (launch_bwd_gemm(kBwdGU, 256, pair, mXg, mW1, mW3, a,
+                            grid_for(kBwdGU, pair, (pair ? mt_pairs : L.MT_max) * a.n_tiles), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
     // 3. dh -> dg, du and the routing-weight gradients
@@ -960,8 +982,10 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.hbuf = reg(MOE_WS_H);
         a.h_pitch = p2F;
         a.dw = dwa;
+        const bool pair = bn == 256 && pairs_for(kBwdDH) > 0;
         ProfScope ps(MOE_KERNEL_BWD_DH, st);
-        if (launch_bwd_gemm(kBwdDH, bn, mDyg, mW2t, mW2t, a, row_grid(a.n_tiles), st) != cudaSuccess)
+        if (launch_bwd_gemm(kBwdDH, bn, pair, mDyg, mW2t, mW2t, a,
+                            grid_for(kBwdDH, pair, (pair ? mt_pairs : L.MT_max) * a.n_tiles), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
     // 4. dx: the k experts' contributions meet in fp32, then one rounding
@@ -973,8 +997,10 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.b_rows = H;
         a.out = dx32;
         a.out_pitch = (long)H * 4;
+        const bool pair = bn == 256 && pairs_for(kBwdDX) > 0;
         ProfScope ps(MOE_KERNEL_BWD_DX, st);
-        if (launch_bwd_gemm(kBwdDX, bn, mDgu, mW13t, mW13t, a, row_grid(a.n_tiles), st) != cudaSuccess)
+        if (launch_bwd_gemm(kBwdDX, bn, pair, mDgu, mW13t, mW13t, a,
+                            grid_for(kBwdDX, pair, (pair ? mt_pairs : L.MT_max) * a.n_tiles), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
     {
@@ -1020,9 +1046,11 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.out_pitch = (long)F * 2;
         a.split = H;
         a.expert_stride = (long)H * F * 2;
-        const int grid = (int)std::min<long>((long)E * a.m_tiles * a.n_tiles, num_sms);
+        const bool pair = bn == 256 && a.m_tiles % 2 == 0 && pairs_for(kBwdDW) > 0;
+        const long units = (long)E * (pair ? a.m_tiles / 2 : a.m_tiles) * a.n_tiles;
         ProfScope ps(MOE_KERNEL_BWD_DW2, st);
-        if (launch_bwd_gemm(kBwdDW, bn, mDot, mHt, mHt, a, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_bwd_gemm(kBwdDW, bn, pair, mDot, mHt, mHt, a, grid_for(kBwdDW, pair, units), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
     }
     {
         const int bn = (H % 256 == 0) ? 256 : 128;
@@ -1034,9 +1062,11 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.out_pitch = (long)H * 2;
         a.split = F;
         a.expert_stride = (long)F * H * 2;
-        const int grid = (int)std::min<long>((long)E * a.m_tiles * a.n_tiles, num_sms);
+        const bool pair = bn == 256 && a.m_tiles % 2 == 0 && pairs_for(kBwdDW) > 0;
+        const long units = (long)E * (pair ? a.m_tiles / 2 : a.m_tiles) * a.n_tiles;
         ProfScope ps(MOE_KERNEL_BWD_DW13, st);
-        if (launch_bwd_gemm(kBwdDW, bn, mDgut, mXt, mXt, a, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_bwd_gemm(kBwdDW, bn, pair, mDgut, mXt, mXt, a, grid_for(kBwdDW, pair, units), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
     }
     // 6. router
     {

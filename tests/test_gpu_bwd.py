@@ -89,9 +89,21 @@ SMALL = [
 ]
 
 
+@pytest.fixture(autouse=True)
+def _reset_path(moe):
+    yield
+    moe.moe_set_option(moe.OPT_PATH, 0)
+
+
+@pytest.mark.parametrize("path", [0, 3], ids=["pair_tiles", "one_sm_tiles"])
 @pytest.mark.parametrize("p", SMALL, ids=lambda p: f"T{p[0]}_H{p[1]}_F{p[2]}_E{p[3]}_k{p[4]}" + ("_skew" if p[6] else ""))
-def test_backward_small(moe, p):
+def test_backward_small(moe, p, path):
+    """Pairs of SMs on 256 x 256 tiles where the tile is 256 wide (an expert
+    with an odd number of 128-row tiles repeats its last one in the second
+    CTA; an odd number of 128-row weight-gradient tiles keeps one-SM tiles),
+    or one-SM tiles throughout."""
     T, H, F, E, k, seed, skew = p
+    moe.moe_set_option(moe.OPT_PATH, path)
     case = moe_inputs.make_case(T, H, F, E, k, "bf16", seed, skew)
     dy = moe_inputs.make_dy(T, H, seed)
     out = run_bwd(moe, case, dy)
