@@ -10,7 +10,7 @@ HBM.  The headline workload is the Mixtral-8x7B-shaped FP8 decode layer
 the same run also times every other workload of the Mixtral expert shape
 (prefill T=4096 FP8, skewed-routing T=8192 BF16, the FP8 batch sweep
 T = 1, 128, 1024, 16384, decode / prefill with MX FP4 expert weights, and a
-BF16 training step at T=4096: weight layouts, forward, backward) and reports
+BF16 training step at T=4096: weight layout, forward, backward) and reports
 each as a sub-record under ``configs`` with its own step time, roofline, CPU
 baseline and end-to-end number.
 
@@ -631,10 +631,10 @@ def train_cpu_baseline(case, dy, spec, name, seconds):
 
 
 def run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_seconds):
-    """Time one BF16 training step of the layer: the weight layouts both passes
-    read (redone every step, as weights change), the forward, and the
-    backward (custom VJP: dx, dw1, dw3, dw2, dlogits).  Same structure of
-    record as run_gpu_config."""
+    """Time one BF16 training step of the layer: the forward's weight layout
+    (redone every step, as weights change), the forward, and the backward
+    (custom VJP: dx, dw1, dw3, dw2, dlogits; it reads the weights as they
+    are).  Same structure of record as run_gpu_config."""
     import torch
     import torch.distributed as dist
 
@@ -652,18 +652,16 @@ def run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_seconds):
     x, logits, dy = x_cpu.to(dev), lg_cpu.to(dev), dy_cpu.to(dev)
     w1, w3, w2 = case["w1"].to(dev), case["w3"].to(dev), case["w2"].to(dev)
     prep_f = moe.prepare_weights(w1, w3, None, None, w2)
-    prep_b = moe.prepare_weights_bwd(w1, w3, w2)
     ws_f = moe.workspace(T, H, F, E, k, "bf16", dev)
     ws_b = moe.backward_workspace(T, H, F, E, k, dev)
     y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-    grads = moe.ffn_backward(x, logits, w1, w3, prep_b[0], prep_b[1], dy, k, ws=ws_b)
+    grads = moe.ffn_backward(x, logits, w1, w3, w2, dy, k, ws=ws_b)
     stream = torch.cuda.current_stream(dev)
 
     def step(xx=x, lgg=logits, dyy=dy, g=grads):
         moe.prepare_weights(w1, w3, None, None, w2, stream=stream, out=prep_f)
         moe.ffn_forward(xx, lgg, prep_f[0], None, prep_f[2], None, k, F, False, out=y, ws=ws_f, stream=stream)
-        moe.prepare_weights_bwd(w1, w3, w2, stream=stream, out=prep_b)
-        moe.ffn_backward(xx, lgg, w1, w3, prep_b[0], prep_b[1], dyy, k, ws=ws_b, out=g, stream=stream)
+        moe.ffn_backward(xx, lgg, w1, w3, w2, dyy, k, ws=ws_b, out=g, stream=stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -759,8 +757,8 @@ def run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_seconds):
     return {
         "value": value, "unit": "tokens/s", "ms_per_step": ms_step, "steps": args.steps, "warmup": args.warmup,
         "dtype": "bf16 (fp32 accumulate)",
-        "config": {"workload": workload_desc(spec, name) + "; training step: weight layouts, forward, backward "
-                   "(dx, dw1, dw3, dw2, dlogits)", "T": T, "d_model": H, "d_ff": F, "experts": E, "top_k": k,
+        "config": {"workload": workload_desc(spec, name) + "; training step: forward weight layout, forward, "
+                   "backward (dx, dw1, dw3, dw2, dlogits)", "T": T, "d_model": H, "d_ff": F, "experts": E, "top_k": k,
                    "weights": "bf16", "parallelism": f"weak-scaling replicas x{world}" if world > 1 else "1 GPU",
                    "l2": "inputs larger than L2 (expert weights %.2f GB, read by several kernels per step)" % (
                        wbytes / 1e9),

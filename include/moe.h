@@ -345,7 +345,7 @@ int moe_set_option(int option, int value);
  * moe_ffn_backward and the weight preparations record a pair of CUDA events
  * around each step they enqueue (routing is one kernel for small batches and two from 1024 tokens
  * on; both are counted in `launches` and timed together; the backward's
- * routing, gathers, transposes, rounding of dx and router gradient are timed
+ * routing, slot gather, rounding of dx and router gradient are timed
  * together as MOE_KERNEL_BWD_AUX).
  * moe_profile_enable returns the previous setting.  moe_profile_read waits for
  * the recorded events, adds up the elapsed time per kernel into
@@ -363,8 +363,8 @@ typedef enum {
     MOE_KERNEL_BWD_DX = 7,   /* backward: dx = W1^T dg + W3^T du, scatter-add per token */
     MOE_KERNEL_BWD_DW2 = 8,  /* backward: dW2 per expert */
     MOE_KERNEL_BWD_DW13 = 9, /* backward: dW1, dW3 per expert */
-    MOE_KERNEL_BWD_AUX = 10, /* backward: routing, gathers, transposes, dx rounding, router gradient */
-    MOE_KERNEL_PREPARE = 11, /* moe_prepare_weights, _mx and _bwd (weight layouts) */
+    MOE_KERNEL_BWD_AUX = 10, /* backward: routing, slot gather, dx rounding, router gradient */
+    MOE_KERNEL_PREPARE = 11, /* moe_prepare_weights and _mx (weight layouts) */
     MOE_KERNEL_COUNT = 12
 } moe_kernel_id;
 int moe_profile_enable(int on);
@@ -386,38 +386,33 @@ int moe_profile_read(double* ms_total, int* launches, int reset);
  *   for the others (the routing weights are the softmax over the chosen
  *   logits; the choice is piecewise constant).
  * g and u are recomputed from x and w1/w3 (the forward keeps no
- * intermediates).  Arithmetic: bf16 operands, fp32 accumulation; g and u are
- * kept in fp32, h (as in the forward), dg, du and the w_a dy_t entering dW2 are
- * rounded to bf16 where they are stored between kernels; dx is summed over
- * the k experts in fp32 and rounded once.
+ * intermediates).  Every grouped GEMM reads its operands as they lie -- the
+ * weights in the caller's row-major layout, the activations in the
+ * expert-padded slot layout -- K-major or MN-major, so nothing is
+ * transposed and the weights need no preparation.  Arithmetic: bf16
+ * operands, fp32 accumulation; g and u are kept in fp32, h (as in the
+ * forward), dg, du and the w_a dy_t entering dW2 are rounded to bf16 where
+ * they are stored between kernels; dx is summed over the k experts in fp32
+ * and rounded once.
  *
  * moe_backward_workspace_size: bytes of `ws` for moe_ffn_backward (0 if the
  *   dimensions are unsupported: bf16 only, d_model and d_ff multiples of 128,
  *   1 <= E <= 64, 1 <= k <= min(E, 8)).
- * moe_prepare_weights_bwd: the transposed weight copies the backward reads,
- *   bf16, device pointers, enqueued on `stream`:
- *     w13t [E, H, 2F]: w13t[e][h][f] = w1[e][f][h], w13t[e][h][F + f] = w3[e][f][h]
- *     w2t  [E, F, H]:  w2t[e][f][h] = w2[e][h][f]
- *   from w1, w3 [E, F, H] and w2 [E, H, F] (row-major, as moe_prepare_weights
- *   takes them).  Redo after every weight update.  All pointers 16-byte
- *   aligned (MOE_ERR_ALIGNMENT), the buffers the caller's; nothing is freed.
  * moe_ffn_backward: x [T, H], dy [T, H] bf16, logits [T, E] fp32 (finite),
- *   w1, w3 [E, F, H] bf16 (row-major, as given to moe_prepare_weights),
- *   w13t, w2t from moe_prepare_weights_bwd; outputs dx [T, H] bf16, dw1, dw3
- *   [E, F, H] and dw2 [E, H, F] bf16 (fully written: zero for an expert with
- *   no tokens), dlogits [T, E] fp32.  Device pointers, 16-byte aligned
- *   (logits and dlogits 4-byte); ws >= moe_backward_workspace_size bytes.
- *   Enqueued on `stream` (no host synchronisation; may be captured in a CUDA
- *   graph).  Returns MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_ALIGNMENT,
- *   MOE_ERR_WORKSPACE or MOE_ERR_CUDA (a launch failed; device-side faults
- *   surface through moe_get_status as for the forward).
+ *   w1, w3 [E, F, H] and w2 [E, H, F] bf16, row-major (as moe_prepare_weights
+ *   takes them); outputs dx [T, H] bf16, dw1, dw3 [E, F, H] and dw2 [E, H, F]
+ *   bf16 (fully written: zero for an expert with no tokens), dlogits [T, E]
+ *   fp32.  Device pointers, 16-byte aligned (logits and dlogits 4-byte); ws
+ *   >= moe_backward_workspace_size bytes.  Enqueued on `stream` (no host
+ *   synchronisation; may be captured in a CUDA graph).  Returns MOE_OK,
+ *   MOE_ERR_INVALID_ARG, MOE_ERR_ALIGNMENT, MOE_ERR_WORKSPACE or MOE_ERR_CUDA
+ *   (a launch failed; device-side faults surface through moe_get_status as
+ *   for the forward).
  */
 size_t moe_backward_workspace_size(int T, int H, int F, int E, int k);
-int moe_prepare_weights_bwd(const void* w1, const void* w3, const void* w2, void* w13t_out, void* w2t_out, int E,
-                            int F, int H, void* stream);
-int moe_ffn_backward(const void* x, const float* logits, const void* w1, const void* w3, const void* w13t,
-                     const void* w2t, const void* dy, int T, int H, int F, int E, int k, void* dx, void* dw1,
-                     void* dw3, void* dw2, float* dlogits, void* ws, size_t ws_bytes, void* stream);
+int moe_ffn_backward(const void* x, const float* logits, const void* w1, const void* w3, const void* w2,
+                     const void* dy, int T, int H, int F, int E, int k, void* dx, void* dw1, void* dw3, void* dw2,
+                     float* dlogits, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

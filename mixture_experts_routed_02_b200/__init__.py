@@ -55,7 +55,7 @@ WS = dict(topk_ids=0, topk_w=1, counts=2, offsets=3, perm=4, inv_perm=5, slot_of
 EXPORTS = ["moe_workspace_size", "moe_prepare_weights", "moe_route", "moe_ffn_forward", "moe_get_status",
            "moe_workspace_region", "moe_set_option", "moe_profile_enable", "moe_profile_read",
            "moe_ffn_forward_static", "moe_static_workspace_bytes", "moe_ffn_forward_dff", "moe_dff_finalize",
-           "moe_prepare_weights_mx", "moe_backward_workspace_size", "moe_prepare_weights_bwd", "moe_ffn_backward"]
+           "moe_prepare_weights_mx", "moe_backward_workspace_size", "moe_ffn_backward"]
 # kernel ids of moe_profile_read: the forward's five, then the backward's
 FWD_KERNELS = ["route", "quantize", "stage1_w13_swiglu", "stage2_w2_scatter", "finalize"]
 BWD_KERNELS = ["bwd_gu_recompute", "bwd_dh_swiglu", "bwd_dx_scatter", "bwd_dw2", "bwd_dw13", "bwd_aux"]
@@ -103,10 +103,8 @@ lib.moe_profile_read.restype = _I
 lib.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I), _I]
 lib.moe_backward_workspace_size.restype = _Z
 lib.moe_backward_workspace_size.argtypes = [_I, _I, _I, _I, _I]
-lib.moe_prepare_weights_bwd.restype = _I
-lib.moe_prepare_weights_bwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _P]
 lib.moe_ffn_backward.restype = _I
-lib.moe_ffn_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]
+lib.moe_ffn_backward.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]
 
 # raw entry points, same names as the C ABI
 moe_workspace_size = lib.moe_workspace_size
@@ -122,7 +120,6 @@ moe_static_workspace_bytes = lib.moe_static_workspace_bytes
 moe_ffn_forward_dff = lib.moe_ffn_forward_dff
 moe_dff_finalize = lib.moe_dff_finalize
 moe_backward_workspace_size = lib.moe_backward_workspace_size
-moe_prepare_weights_bwd = lib.moe_prepare_weights_bwd
 moe_ffn_backward = lib.moe_ffn_backward
 
 
@@ -330,27 +327,6 @@ def dff_finalize(out32_rows, out, counter, target, stream=None):
 
 # ---------------------------------------------------------------- backward pass (BF16)
 
-def prepare_weights_bwd(w1, w3, w2, stream=None, out=None):
-    """Transposed copies the backward reads (redo after each weight update):
-    w13t [E,H,2F] = [w1^T | w3^T] per expert and w2t [E,F,H] = w2^T, bf16.
-    ``out``: an earlier (w13t, w2t) to write into."""
-    import torch
-    for t in (w1, w3, w2):
-        if t.dtype != torch.bfloat16 or not t.is_contiguous():
-            raise ValueError("prepare_weights_bwd takes contiguous bf16 weights")
-    E, F, H = w1.shape
-    if w3.shape != (E, F, H) or w2.shape != (E, H, F):
-        raise ValueError("weight shapes do not match")
-    if out is not None:
-        w13t, w2t = out
-    else:
-        w13t = torch.empty(E, H, 2 * F, dtype=torch.bfloat16, device=w1.device)
-        w2t = torch.empty(E, F, H, dtype=torch.bfloat16, device=w1.device)
-    _check("moe_prepare_weights_bwd", moe_prepare_weights_bwd(_ptr(w1), _ptr(w3), _ptr(w2), _ptr(w13t), _ptr(w2t),
-                                                              E, F, H, _stream(stream)))
-    return w13t, w2t
-
-
 def backward_workspace(T, H, F, E, k, device="cuda"):
     import torch
     n = moe_backward_workspace_size(T, H, F, E, k)
@@ -359,11 +335,11 @@ def backward_workspace(T, H, F, E, k, device="cuda"):
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-def ffn_backward(x, logits, w1, w3, w13t, w2t, dy, k, ws=None, out=None, stream=None):
+def ffn_backward(x, logits, w1, w3, w2, dy, k, ws=None, out=None, stream=None):
     """Gradients of the BF16 layer for the upstream gradient dy: returns
     dict(dx [T,H] bf16, dw1 [E,F,H], dw3 [E,F,H], dw2 [E,H,F] bf16, dlogits
-    [T,E] fp32).  w1, w3: the row-major bf16 weights; w13t, w2t from
-    prepare_weights_bwd.  ``out``: an earlier result dict to write into."""
+    [T,E] fp32).  w1, w3 [E,F,H], w2 [E,H,F]: the row-major bf16 weights (no
+    preparation).  ``out``: an earlier result dict to write into."""
     import torch
     T, H = x.shape
     E, F, _ = w1.shape
@@ -376,7 +352,12 @@ def ffn_backward(x, logits, w1, w3, w13t, w2t, dy, k, ws=None, out=None, stream=
                    dw3=torch.empty(E, F, H, dtype=torch.bfloat16, device=dev),
                    dw2=torch.empty(E, H, F, dtype=torch.bfloat16, device=dev),
                    dlogits=torch.empty(T, E, dtype=torch.float32, device=dev))
-    rc = moe_ffn_backward(_ptr(x), _ptr(logits), _ptr(w1), _ptr(w3), _ptr(w13t), _ptr(w2t), _ptr(dy), T, H, F, E, k,
+    for t in (w1, w3, w2):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("ffn_backward takes contiguous bf16 weights")
+    if w3.shape != (E, F, H) or w2.shape != (E, H, F):
+        raise ValueError("weight shapes do not match")
+    rc = moe_ffn_backward(_ptr(x), _ptr(logits), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(dy), T, H, F, E, k,
                           _ptr(out["dx"]), _ptr(out["dw1"]), _ptr(out["dw3"]), _ptr(out["dw2"]), _ptr(out["dlogits"]),
                           _ptr(ws), ws.numel(), _stream(stream))
     _check("moe_ffn_backward", rc)

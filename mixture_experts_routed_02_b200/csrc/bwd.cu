@@ -11,19 +11,25 @@
 //   dlogit[t, e_j] = w_j (dw_j - sum_i w_i dw_i)   (softmax over the chosen logits)
 //
 // Five grouped GEMMs on the tensor cores (tcgen05, bf16 operands, fp32 in
-// TMEM), each operand a K-major bf16 matrix copied by 2-D TMA with the 128-byte
-// swizzle (no preshuffled weights: training changes them every step):
-//   GU   [slots x 2F]: xg . [W1_e; W3_e]^T -- g and u recomputed (activation
-//        recomputation: the forward keeps nothing but its output); the
-//        epilogue stores g and u in fp32 and h = bf16(silu(g) u);
-//   DH   [slots x F]:  dyg . (W2_e^T)^T, K = H -- epilogue: dw_a (sum over the
-//        tile's columns of dh_unweighted * h, one fp32 atomic per row and tile),
-//        dh = w_a * acc, then dg and du into dGU [slots x 2F];
-//   DX   [slots x H]:  dGU . ([W1_e; W3_e]^T)^T, K = 2F -- epilogue: fp32
-//        atomics into dx32[t] (the k experts of a token meet there);
-//   DW   [rows x cols] per expert, K = the expert's padded slots: dW2_e =
-//        dO^T h and [dW1_e; dW3_e] = dGU^T x, the transposed operands written
-//        by the transpose kernel below (rows of the slot layout -> columns).
+// TMEM), every operand copied by 2-D TMA with the 128-byte swizzle straight
+// from the matrix it is -- the weights as the caller holds them (no
+// preshuffle: training changes them every step), the activations in the
+// expert-padded slot layout -- and read by the MMA K-major (K contiguous) or
+// MN-major (M or N contiguous), as it lies, so nothing is transposed:
+//   GU   [slots x 2F]: xg . [W1_e; W3_e]^T, K = H, both K-major -- g and u
+//        recomputed (activation recomputation: the forward keeps nothing but
+//        its output); the epilogue stores g and u in fp32 and h =
+//        bf16(silu(g) u), zero rows for padding slots;
+//   DH   [slots x F]:  dyg . W2_e, K = H, W2_e [H, F] MN-major -- epilogue:
+//        dw_a (the tile's sum of dh_unweighted * h, one fp32 atomic per row
+//        and tile), dh = w_a * acc, then dg and du into dGU [slots x 2F];
+//   DX   [slots x H]:  dGU . [W1_e; W3_e], K = 2F, W1_e / W3_e [F, H]
+//        MN-major -- epilogue: fp32 atomics into dx32[t] (the k experts of a
+//        token meet there);
+//   DW   [rows x cols] per expert, K = the expert's padded slots, both
+//        operands MN-major: dW2_e = dO^T h with dO = w_a dy_t gathered per
+//        slot, and [dW1_e; dW3_e] = dGU^T xg (padding slots are zero in dO,
+//        h, dGU and xg, so they add nothing).
 // Warp roles as in the forward GEMM: warp 0 lane 0 issues the TMA copies into
 // an NST-deep ring, warp 1 owns TMEM and issues the MMAs, warps 2..5 drain the
 // two TMEM accumulators (the epilogue of one tile overlaps the next tile's
@@ -42,8 +48,11 @@ namespace {
 // CTA issues the MMAs, and each CTA's TMEM receives its own 128 rows.  Per
 // unit of work a CTA moves a third less operand data than on one SM, and a
 // stage of 32 KB instead of 48 leaves room for six stages.
-template <int BN, int NST, bool PAIR>
+template <int MODE, int BN, int NST, bool PAIR>
 struct BCfg {
+    // operand majorness: A MN-major in DW; B MN-major in DH, DX and DW
+    static constexpr bool A_MN = MODE == kBwdDW;
+    static constexpr bool B_MN = MODE != kBwdGU;
     static constexpr int A_BYTES = kBlockM * 128;  // 128 rows x 64 bf16
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // this CTA's rows of B
     static constexpr int B_BYTES = B_ROWS * 128;
@@ -54,9 +63,26 @@ struct BCfg {
     static constexpr int NUM_BARS = 2 * NST + 5;  // full, empty, tfull[2], tempty[2], drain
     static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-    static_assert(B_ROWS % 128 == 0, "B copies of 128 rows");
-    static constexpr uint32_t IDESC = idesc_bf16(PAIR ? 2 * kBlockM : kBlockM, BN);
+    static_assert(B_ROWS % 128 == 0, "B: whole boxes of 128 (K-major) or 64 (MN-major) columns");
+    // bits 15 and 16 of the instruction descriptor: A and B MN-major
+    static constexpr uint32_t IDESC =
+        idesc_bf16(PAIR ? 2 * kBlockM : kBlockM, BN) | ((A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16);
 };
+
+// Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
+// blocks of 64 MN elements x 64 K rows (one TMA box, 8 KB: K rows of 128
+// bytes, 8-row swizzle atoms 1024 bytes apart -- the stride byte offset),
+// consecutive MN blocks 8 KB apart (the leading byte offset).  One MMA reads
+// 16 K rows: the next one starts two atoms (2048 bytes) further.
+__device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);  // start address
+    d |= (uint64_t)(8192 >> 4) << 16;        // leading byte offset: next 64-element MN block
+    d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset: next 8 K rows
+    d |= (uint64_t)1 << 46;                  // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;                  // layout: 128-byte swizzle
+    return d;
+}
 
 __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
@@ -88,7 +114,7 @@ template <int MODE, int BN, int NST, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmB2, const BwdArgs args) {
-    using C = BCfg<BN, NST, PAIR>;
+    using C = BCfg<MODE, BN, NST, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -272,32 +298,48 @@ __global__ void __launch_bounds__(192, 1)
                     uint8_t* sb = sa + C::A_BYTES;
                     const int kx = (k0 + kk) * 64;
                     if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-                    // B rows of this CTA: GU -- 128 rows of W1_e and the same 128
-                    // rows of W3_e (the tile's first 128 columns are g, the last 128
-                    // u, of the same features; on a pair each CTA holds one of the
-                    // two); otherwise BN rows, or this CTA's half of them
-                    if constexpr (PAIR) {
-                        const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
-                        tma_load_2d_pair(sa, &tmA, bar, kx, m * kBlockM, pol_a);
-                        if constexpr (MODE == kBwdGU) {
-                            tma_load_2d_pair(sb, rank == 0 ? &tmB : &tmB2, bar, kx, e * args.b_rows + n * 128, pol_b);
+                    // every copy completes on the even CTA's barrier (a pair) or on this CTA's
+                    const uint32_t bar = PAIR ? mapa_shared(smem_u32(&full[stage]), 0) : smem_u32(&full[stage]);
+                    auto load = [&](void* dst, const CUtensorMap* map, int x, int y, uint64_t pol) {
+                        if constexpr (PAIR) tma_load_2d_pair(dst, map, bar, x, y, pol);
+                        else tma_load_2d(dst, map, &full[stage], x, y, pol);
+                    };
+                    // A: 128 rows of K-major data (one box of 64 K x 128 rows), or
+                    // (DW) the 128 output rows' columns of the slot layout, MN-major:
+                    // two boxes of 64 MN x 64 K
+                    if constexpr (C::A_MN) {
+                        load(sa, &tmA, m * kBlockM, kx, pol_a);
+                        load(sa + 8192, &tmA, m * kBlockM + 64, kx, pol_a);
+                    } else {
+                        load(sa, &tmA, kx, m * kBlockM, pol_a);
+                    }
+                    // B: this CTA's B_ROWS columns of the tile (all BN on one SM)
+                    const int ncol = n * BN + (PAIR ? (int)rank * C::B_ROWS : 0);
+                    if constexpr (MODE == kBwdGU) {
+                        // 128 rows of W1_e and the same 128 rows of W3_e (K-major): the
+                        // tile's first 128 columns are g, the last 128 u, of the same
+                        // features; on a pair each CTA holds one of the two
+                        if constexpr (PAIR) {
+                            load(sb, rank == 0 ? &tmB : &tmB2, kx, e * args.b_rows + n * 128, pol_b);
                         } else {
-                            const int brow = (MODE == kBwdDW ? 0 : e * args.b_rows) + n * BN + (int)rank * C::B_ROWS;
-#pragma unroll
-                            for (int j = 0; j < C::B_ROWS / 128; ++j)
-                                tma_load_2d_pair(sb + j * 128 * 128, &tmB, bar, kx, brow + 128 * j, pol_b);
+                            load(sb, &tmB, kx, e * args.b_rows + n * 128, pol_b);
+                            load(sb + 128 * 128, &tmB2, kx, e * args.b_rows + n * 128, pol_b);
                         }
                     } else {
-                        tma_load_2d(sa, &tmA, &full[stage], kx, m * kBlockM, pol_a);
-                        if constexpr (MODE == kBwdGU) {
-                            tma_load_2d(sb, &tmB, &full[stage], kx, e * args.b_rows + n * 128, pol_b);
-                            tma_load_2d(sb + 128 * 128, &tmB2, &full[stage], kx, e * args.b_rows + n * 128, pol_b);
-                        } else {
-                            const int brow = (MODE == kBwdDW ? 0 : e * args.b_rows) + n * BN;
-#pragma unroll
-                            for (int j = 0; j < BN / 128; ++j)
-                                tma_load_2d(sb + j * 128 * 128, &tmB, &full[stage], kx, brow + 128 * j, pol_b);
+                        // MN-major boxes of 64 columns x 64 K rows: DH from W2_e (rows
+                        // h = K), DX from W1_e for K < F and W3_e beyond (rows c = K),
+                        // DW from the slot layout (rows = slots = K)
+                        const CUtensorMap* mb = &tmB;
+                        int krow = kx;
+                        if constexpr (MODE == kBwdDH) {
+                            krow = e * args.b_rows + kx;
+                        } else if constexpr (MODE == kBwdDX) {
+                            const bool up = kx >= args.F;
+                            mb = up ? &tmB2 : &tmB;
+                            krow = e * args.F + (up ? kx - args.F : kx);
                         }
+#pragma unroll
+                        for (int j = 0; j < C::B_ROWS / 64; ++j) load(sb + j * 8192, mb, ncol + 64 * j, krow, pol_b);
                     }
                     if (++stage == NST) {
                         stage = 0;
@@ -340,7 +382,9 @@ __global__ void __launch_bounds__(192, 1)
                     const uint32_t b_addr = a_addr + C::A_BYTES;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = sdesc_sw128(a_addr + ks * 32), bd = sdesc_sw128(b_addr + ks * 32);
+                        // 16 K per MMA: 32 bytes along a K-major row, or two 8-row atoms MN-major
+                        const uint64_t ad = C::A_MN ? sdesc_sw128_mn(a_addr + ks * 2048) : sdesc_sw128(a_addr + ks * 32);
+                        const uint64_t bd = C::B_MN ? sdesc_sw128_mn(b_addr + ks * 2048) : sdesc_sw128(b_addr + ks * 32);
                         const uint32_t accum = (kk > 0 || ks > 0) ? 1u : 0u;
                         if constexpr (PAIR) mma_bf16_pair(d_tmem, ad, bd, C::IDESC, accum);
                         else mma_bf16(d_tmem, ad, bd, C::IDESC, accum);
@@ -416,6 +460,12 @@ __global__ void __launch_bounds__(192, 1)
                     tmem_ld_32cols(tbase + 128 + c0, ru);
                     tmem_ld_wait();
                     if (c0 + 32 == 128) release(acc);
+                    if (a < 0 && !dup) {  // a padding slot: h = 0 (the weight gradients read it)
+                        uint4* oh = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out2) +
+                                                             (size_t)slot * args.out2_pitch) + (n * 128 + c0) / 8;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) oh[i] = make_uint4(0u, 0u, 0u, 0u);
+                    }
                     if (a >= 0) {
                         const int f = n * 128 + c0;
                         float gv[32], uv[32], hv[32];
@@ -449,6 +499,13 @@ __global__ void __launch_bounds__(192, 1)
                     tmem_ld_32cols(tbase + c0, r);
                     tmem_ld_wait();
                     if (c0 + 32 == BN) release(acc);
+                    if (a < 0 && !dup) {  // a padding slot: dg = du = 0 (dW1 and dW3 read them)
+                        uint8_t* orow = static_cast<uint8_t*>(args.out) + (size_t)slot * args.out_pitch;
+                        uint4* og = reinterpret_cast<uint4*>(orow) + (n * BN + c0) / 8;
+                        uint4* ou = reinterpret_cast<uint4*>(orow) + (args.F + n * BN + c0) / 8;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) og[i] = ou[i] = make_uint4(0u, 0u, 0u, 0u);
+                    }
                     if (a >= 0) {
                         const int f = n * BN + c0;
                         const uint8_t* gurow = static_cast<const uint8_t*>(args.gu) + (size_t)slot * args.gu_pitch;
@@ -550,85 +607,44 @@ __global__ void __launch_bounds__(192, 1)
     if constexpr (PAIR) cluster_sync_all();
 }
 
-// ---------------------------------------------------------------- transposes
-// out[c][s] = v(s, c) for 64 x 64 tiles, bf16, where row s of the source is
-//   kSrcRows:  src row s (weights: a plain [rows, cols] matrix per batch z);
-//   kSrcSlots: src row s of the slot layout, 0 for a padding slot;
-//   kSrcTokens: the token row of slot s's assignment (t = a / topk), times
-//              topk_w[a] if scaled, 0 for a padding slot.
-// Each thread reads 16-byte pieces of source rows (a warp covers four rows of
-// 128 bytes) and writes 16-byte pieces of output rows (eight consecutive
-// slots); the tile crosses shared memory with a row pitch of 66 elements so
-// that the column reads of one warp fall on distinct banks but for pairs.
-template <int SRC>
-__global__ void __launch_bounds__(256) transpose_kernel(TransposeArgs p) {
-    constexpr int kPitch = 66;
-    __shared__ __align__(16) uint16_t tile[64 * kPitch];
-    const int c0 = blockIdx.x * 64, s0 = blockIdx.y * 64, z = blockIdx.z;
-    int rows = p.rows;
-    if (SRC != kSrcRows) {
-        const int nmt = *p.num_mtiles;
-        rows = (nmt >= 0 && nmt <= p.mt_max) ? nmt * kBlockM : 0;
+// ---------------------------------------------------------------- slot gather
+// Rows of the expert-padded slot layout for the backward's operands, zero for
+// padding slots (the weight gradients sum over every slot of an expert):
+// xg[s] = x[t], dyg[s] = dy[t], dog[s] = bf16(w_a dy[t]) for slot s holding
+// assignment a = (t, j); rows from num_mtiles * 128 on are left alone.  One
+// warp per slot row, 16-byte pieces.
+__global__ void __launch_bounds__(256) slot_gather_kernel(SlotGatherArgs p) {
+    const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    const int nmt = *p.num_mtiles;
+    const int rows = (nmt >= 0 && nmt <= p.mt_max) ? nmt * kBlockM : 0;
+    if (warp >= rows) return;
+    const int s = warp;
+    int a = p.slot_assign[s];
+    if (a < -1 || a >= p.num_assign) {  // never from the router: a corrupted table
+        if (lane == 0) record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+        a = -1;
     }
-    if (s0 >= rows) return;
-    const uint16_t* src = static_cast<const uint16_t*>(p.src) + (size_t)z * p.src_batch;
-    uint16_t* out = static_cast<uint16_t*>(p.out) + (size_t)z * p.out_batch;
+    const int t = a >= 0 ? a / p.topk : 0;
+    const float w = a >= 0 ? p.topk_w[a] : 0.0f;
+    const uint4* xr = reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H);
+    const uint4* dr = reinterpret_cast<const uint4*>(p.dy + (size_t)t * p.H);
+    uint4* xo = reinterpret_cast<uint4*>(p.xg + (size_t)s * p.pitch);
+    uint4* dyo = reinterpret_cast<uint4*>(p.dyg + (size_t)s * p.pitch);
+    uint4* doo = reinterpret_cast<uint4*>(p.dog + (size_t)s * p.pitch);
+    for (int i = lane; i < p.H / 8; i += 32) {
+        uint4 xv = make_uint4(0u, 0u, 0u, 0u), dv = xv, ov = xv;
+        if (a >= 0) {
+            xv = __ldg(xr + i);
+            dv = __ldg(dr + i);
+            float f[8];
+            unpack8(dv, f);
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int q = threadIdx.x + 256 * i;  // 512 pieces: 64 rows x 8 pieces of 8 elements
-        const int r = q >> 3, c8 = (q & 7) * 8;
-        const int s = s0 + r;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (s < rows) {
-            if constexpr (SRC == kSrcRows) {
-                v = *reinterpret_cast<const uint4*>(src + (size_t)s * p.src_pitch + c0 + c8);
-            } else {
-                const int a = p.slot_assign[s];
-                if (a >= 0 && a < p.num_assign) {
-                    if constexpr (SRC == kSrcSlots) {
-                        v = *reinterpret_cast<const uint4*>(src + (size_t)s * p.src_pitch + c0 + c8);
-                    } else {
-                        v = *reinterpret_cast<const uint4*>(src + (size_t)(a / p.topk) * p.src_pitch + c0 + c8);
-                        if (p.scale) {
-                            const float sc = p.scale[a];
-                            float f[8];
-                            unpack8(v, f);
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) f[j] *= sc;
-                            v = pack8(f);
-                        }
-                    }
-                } else if (a < -1 || a >= p.num_assign) {
-                    record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
-                }
-            }
+            for (int j = 0; j < 8; ++j) f[j] *= w;
+            ov = pack8(f);
         }
-        uint32_t* t32 = reinterpret_cast<uint32_t*>(tile + r * kPitch + c8);  // 4-byte aligned (kPitch even)
-        t32[0] = v.x;
-        t32[1] = v.y;
-        t32[2] = v.z;
-        t32[3] = v.w;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int q = threadIdx.x + 256 * i;  // 512 pieces: 64 output rows x 8 pieces of 8 slots
-        const int c = q >> 3, r8 = (q & 7) * 8;
-        if (s0 + r8 >= rows) continue;  // rows is a multiple of 64 for slot sources
-        uint16_t e[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) e[j] = tile[(r8 + j) * kPitch + c];
-        uint16_t* dst = out + (size_t)(c0 + c) * p.out_pitch + p.out_col + s0 + r8;
-        if (s0 + r8 + 8 <= rows) {
-            uint4 w;
-            w.x = e[0] | ((uint32_t)e[1] << 16);
-            w.y = e[2] | ((uint32_t)e[3] << 16);
-            w.z = e[4] | ((uint32_t)e[5] << 16);
-            w.w = e[6] | ((uint32_t)e[7] << 16);
-            *reinterpret_cast<uint4*>(dst) = w;
-        } else {
-            for (int j = 0; j < 8 && s0 + r8 + j < rows; ++j) dst[j] = e[j];
-        }
+        xo[i] = xv;
+        dyo[i] = dv;
+        doo[i] = ov;
     }
 }
 
@@ -653,7 +669,7 @@ namespace {
 template <int MODE, int BN, int NST, bool PAIR>
 cudaError_t launch_bwd_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const BwdArgs& args,
                            int grid, cudaStream_t stream) {
-    using C = BCfg<BN, NST, PAIR>;
+    using C = BCfg<MODE, BN, NST, PAIR>;
     auto kern = bwd_gemm_kernel<MODE, BN, NST, PAIR>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (err != cudaSuccess) return err;
@@ -680,7 +696,7 @@ cudaError_t launch_bwd_one(const CUtensorMap& a, const CUtensorMap& b, const CUt
 
 template <int MODE>
 int max_pairs_one() {
-    using C = BCfg<256, 6, true>;
+    using C = BCfg<MODE, 256, 6, true>;
     auto kern = bwd_gemm_kernel<MODE, 256, 6, true>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
         return 0;
@@ -729,21 +745,10 @@ cudaError_t launch_bwd_gemm(int mode, int bn, bool pair, const CUtensorMap& a, c
     }
 }
 
-cudaError_t launch_transpose(int src_kind, const TransposeArgs& p, int cols, int rows_max, int batch,
-                             cudaStream_t stream) {
-    // 16-byte pieces: the source pitch, the output pitch and column offset in
-    // whole pieces of 8 elements (the bases are 16-byte aligned by contract)
-    if (cols % 64 || rows_max < 0 || batch < 1 || p.src_pitch % 8 || p.out_pitch % 8 || p.out_col % 8 ||
-        p.src_batch % 8 || p.out_batch % 8)
-        return cudaErrorInvalidValue;
-    if (rows_max == 0 || cols == 0) return cudaSuccess;
-    const dim3 grid(cols / 64, (rows_max + 63) / 64, batch);
-    switch (src_kind) {
-        case kSrcRows: transpose_kernel<kSrcRows><<<grid, 256, 0, stream>>>(p); break;
-        case kSrcSlots: transpose_kernel<kSrcSlots><<<grid, 256, 0, stream>>>(p); break;
-        case kSrcTokens: transpose_kernel<kSrcTokens><<<grid, 256, 0, stream>>>(p); break;
-        default: return cudaErrorInvalidValue;
-    }
+cudaError_t launch_slot_gather(const SlotGatherArgs& p, int rows_max, cudaStream_t stream) {
+    if (p.H % 8 || p.pitch % 8) return cudaErrorInvalidValue;
+    if (rows_max <= 0) return cudaSuccess;
+    slot_gather_kernel<<<(rows_max + 7) / 8, 256, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

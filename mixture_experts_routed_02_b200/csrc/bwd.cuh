@@ -1,5 +1,7 @@
 // bwd.cuh -- argument structs and launchers of the backward pass (bwd.cu).
 #pragma once
+#include <cuda_bf16.h>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -7,7 +9,7 @@ namespace moe {
 // ---------------------------------------------------------------- backward pass
 // Grouped GEMMs of the backward pass (bwd.cu): GU recomputes g, u and h; DH
 // gives dg, du and the routing-weight gradients; DX scatters dx; DW forms the
-// weight gradients per expert from transposed operands.
+// weight gradients per expert (operands read K-major or MN-major as they lie).
 enum BwdMode { kBwdGU = 0, kBwdDH = 1, kBwdDX = 2, kBwdDW = 3 };
 
 struct BwdArgs {
@@ -21,8 +23,8 @@ struct BwdArgs {
     int n_tiles;   // output columns / BN (GU: F / 128)
     int k_tiles;   // K / 64 (GU, DH, DX)
     int m_tiles;   // DW: output rows / 128
-    int b_rows;    // rows of B per expert (GU: F, DH: F, DX: H)
-    int F;         // d_ff (GU, DH: column offset of u and du)
+    int b_rows;    // rows of B's matrix per expert (GU: F rows of W1 / W3; DH: H rows of W2)
+    int F;         // d_ff (GU, DH: column offset of u and du; DX: where K moves from W1 to W3)
     void* out;     // GU: fp32 g|u [S, 2F]; DH: dg|du [S, 2F]; DX: fp32 dx [T, H]; DW: dW (first part)
     long out_pitch;  // bytes
     void* out2;    // GU: h [S, F]; DW: rows >= split (dW3)
@@ -43,31 +45,25 @@ cudaError_t launch_bwd_gemm(int mode, int bn, bool pair, const CUtensorMap& a, c
                             const CUtensorMap& b2, const BwdArgs& args, int grid, cudaStream_t stream);
 int bwd_max_pairs(int mode);  // resident clusters of the pair kernel (0: none)
 
-// out[c][out_col + s] = row s of the source, column c (bf16, 64 x 64 tiles):
-enum TransposeSrc {
-    kSrcRows = 0,    // plain [rows, cols] matrices, batch z of p.batch
-    kSrcSlots = 1,   // rows of the slot layout, 0 for padding slots
-    kSrcTokens = 2   // the token row of each slot's assignment (optionally x topk_w), 0 for padding
-};
-struct TransposeArgs {
-    const void* src;
-    long src_pitch;   // elements
-    long src_batch;   // elements between batches (kSrcRows)
-    int rows;         // kSrcRows: source rows
-    const int* num_mtiles;  // slot sources: rows = num_mtiles * 128
+// Rows of the slot layout for the backward (zero for padding slots):
+// xg = x[t], dyg = dy[t], dog = bf16(w_a dy[t]); rows `pitch` elements apart.
+struct SlotGatherArgs {
+    const __nv_bfloat16* x;
+    const __nv_bfloat16* dy;
+    const int* num_mtiles;
     int mt_max;
     const int* slot_assign;
-    int num_assign;   // T * k
+    const float* topk_w;
+    int num_assign;  // T * k
     int topk;
-    const float* scale;     // kSrcTokens: per-assignment factor, or null
-    void* out;
-    long out_pitch;   // elements
-    long out_col;     // elements
-    long out_batch;   // elements
+    int H;
+    long pitch;  // elements
+    __nv_bfloat16* xg;
+    __nv_bfloat16* dyg;
+    __nv_bfloat16* dog;
     int* status;
 };
-cudaError_t launch_transpose(int src_kind, const TransposeArgs& p, int cols, int rows_max, int batch,
-                             cudaStream_t stream);
+cudaError_t launch_slot_gather(const SlotGatherArgs& p, int rows_max, cudaStream_t stream);
 cudaError_t launch_dlogits(const int32_t* ids, const float* w, const float* dw, int T, int E, int k, float* dlogits,
                            cudaStream_t stream);
 

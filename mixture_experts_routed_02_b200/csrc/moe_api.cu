@@ -767,7 +767,7 @@ int moe_get_status(void* stream) {
 
 namespace {
 
-enum BwdRegion { kBwGU = 0, kBwDYG, kBwDGU, kBwDOT, kBwXT, kBwHT, kBwDW, kBwRegions };
+enum BwdRegion { kBwGU = 0, kBwDYG, kBwDOG, kBwDGU, kBwDW, kBwRegions };
 
 struct BwdLayout {
     Layout fwd;
@@ -780,12 +780,10 @@ BwdLayout make_bwd_layout(int T, int H, int F, int E, int k) {
     B.fwd = make_layout(T, H, F, E, k, MOE_BF16);
     const size_t S = B.fwd.S_max;
     size_t sz[kBwRegions];
-    sz[kBwGU] = S * act_pitch(8L * F);  // fp32 g|u rows [S, 2F]; later bf16 dg|du transposed [2F, S]
-    sz[kBwDYG] = S * act_pitch(2L * H);  // dy gathered into the slot layout [S, H]
+    sz[kBwGU] = S * act_pitch(8L * F);   // fp32 g|u rows [S, 2F]
+    sz[kBwDYG] = S * act_pitch(2L * H);  // dy per slot [S, H]
+    sz[kBwDOG] = S * act_pitch(2L * H);  // w_a dy per slot [S, H]
     sz[kBwDGU] = S * act_pitch(4L * F);  // dg|du [S, 2F]
-    sz[kBwDOT] = (size_t)H * S * 2;      // (w_a dy_t) transposed [H, S]
-    sz[kBwXT] = (size_t)H * S * 2;       // x transposed [H, S]
-    sz[kBwHT] = (size_t)F * S * 2;       // h transposed [F, S]
     sz[kBwDW] = 4 * (size_t)B.fwd.A;     // routing-weight gradients
     size_t off = B.fwd.total;
     for (int r = 0; r < kBwRegions; ++r) {
@@ -811,49 +809,13 @@ size_t moe_backward_workspace_size(int T, int H, int F, int E, int k) {
     return make_bwd_layout(T, H, F, E, k).total;
 }
 
-int moe_prepare_weights_bwd(const void* w1, const void* w3, const void* w2, void* w13t_out, void* w2t_out, int E,
-                            int F, int H, void* stream) {
-    if (E < 1 || E > kMaxExperts || F <= 0 || H <= 0 || F % 128 || H % 128) return MOE_ERR_INVALID_ARG;
-    if (!w1 || !w3 || !w2 || !w13t_out || !w2t_out) return MOE_ERR_INVALID_ARG;
-    if (!aligned16(w1) || !aligned16(w3) || !aligned16(w2) || !aligned16(w13t_out) || !aligned16(w2t_out))
-        return MOE_ERR_ALIGNMENT;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    ProfScope ps(MOE_KERNEL_PREPARE, st, 3);
-    TransposeArgs p{};
-    // w13t[e][h][c] = w1[e][c][h] (c < F), w3[e][c - F][h] (c >= F)
-    p.src_pitch = H;
-    p.src_batch = (long)F * H;
-    p.rows = F;
-    p.out = w13t_out;
-    p.out_pitch = 2L * F;
-    p.out_batch = 2L * F * H;
-    p.src = w1;
-    p.out_col = 0;
-    if (launch_transpose(kSrcRows, p, H, F, E, st) != cudaSuccess) return MOE_ERR_CUDA;
-    p.src = w3;
-    p.out_col = F;
-    if (launch_transpose(kSrcRows, p, H, F, E, st) != cudaSuccess) return MOE_ERR_CUDA;
-    // w2t[e][f][h] = w2[e][h][f]
-    TransposeArgs q{};
-    q.src = w2;
-    q.src_pitch = F;
-    q.src_batch = (long)H * F;
-    q.rows = H;
-    q.out = w2t_out;
-    q.out_pitch = H;
-    q.out_batch = (long)F * H;
-    if (launch_transpose(kSrcRows, q, F, H, E, st) != cudaSuccess) return MOE_ERR_CUDA;
-    return MOE_OK;
-}
-
-int moe_ffn_backward(const void* x, const float* logits, const void* w1, const void* w3, const void* w13t,
-                     const void* w2t, const void* dy, int T, int H, int F, int E, int k, void* dx, void* dw1,
-                     void* dw3, void* dw2, float* dlogits, void* ws, size_t ws_bytes, void* stream) {
+int moe_ffn_backward(const void* x, const float* logits, const void* w1, const void* w3, const void* w2,
+                     const void* dy, int T, int H, int F, int E, int k, void* dx, void* dw1, void* dw3, void* dw2,
+                     float* dlogits, void* ws, size_t ws_bytes, void* stream) {
     if (!bwd_dims_ok(T, H, F, E, k)) return MOE_ERR_INVALID_ARG;
-    if (!w1 || !w3 || !w13t || !w2t || !dw1 || !dw3 || !dw2 || !ws) return MOE_ERR_INVALID_ARG;
+    if (!w1 || !w3 || !w2 || !dw1 || !dw3 || !dw2 || !ws) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !logits || !dy || !dx || !dlogits)) return MOE_ERR_INVALID_ARG;
-    for (const void* ptr : {(const void*)w1, w3, w13t, w2t, (const void*)dw1, (const void*)dw3, (const void*)dw2,
-                            (const void*)ws})
+    for (const void* ptr : {w1, w3, w2, (const void*)dw1, (const void*)dw3, (const void*)dw2, (const void*)ws})
         if (!aligned16(ptr)) return MOE_ERR_ALIGNMENT;
     if (T > 0 && (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || !aligned4(logits) || !aligned4(dlogits)))
         return MOE_ERR_ALIGNMENT;
@@ -877,8 +839,9 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
     auto breg = [&](int r) { return w + B.off[r]; };
     const int S = L.S_max;
     const unsigned long long timeout_ns = (unsigned long long)g_opt_timeout_ms.load() * 1000000ull;
+    const long p2H = act_pitch(2L * H), p4F = act_pitch(4L * F), p2F = act_pitch(2L * F), p8F = act_pitch(8L * F);
 
-    // 1. the forward's routing and slot layout, x and dy gathered into it
+    // 1. the forward's routing and slot layout; x, dy and w_a dy gathered into it
     RouteOutputs o{reinterpret_cast<int32_t*>(reg(MOE_WS_TOPK_IDS)), reinterpret_cast<float*>(reg(MOE_WS_TOPK_W)),
                    reinterpret_cast<int32_t*>(reg(MOE_WS_COUNTS)), reinterpret_cast<int32_t*>(reg(MOE_WS_OFFSETS)),
                    reinterpret_cast<int32_t*>(reg(MOE_WS_PERM)), reinterpret_cast<int32_t*>(reg(MOE_WS_INV_PERM)),
@@ -889,32 +852,44 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
     float* dx32 = reinterpret_cast<float*>(reg(MOE_WS_OUT32));
     float* dwa = reinterpret_cast<float*>(breg(kBwDW));
     {
-        ProfScope ps(MOE_KERNEL_BWD_AUX, st, route_launches(T, o) + 2);
+        ProfScope ps(MOE_KERNEL_BWD_AUX, st, route_launches(T, o) + 1);
         if (launch_route(logits, T, E, k, o, st) != cudaSuccess) return MOE_ERR_CUDA;
-        if (launch_gather(false, static_cast<const __nv_bfloat16*>(x), T, H, k, o.slot_of, S, reg(MOE_WS_XG), nullptr,
-                          nullptr, nullptr, status, st) != cudaSuccess ||
-            launch_gather(false, static_cast<const __nv_bfloat16*>(dy), T, H, k, o.slot_of, S, breg(kBwDYG), nullptr,
-                          nullptr, nullptr, status, st) != cudaSuccess)
-            return MOE_ERR_CUDA;
+        SlotGatherArgs g{};
+        g.x = static_cast<const __nv_bfloat16*>(x);
+        g.dy = static_cast<const __nv_bfloat16*>(dy);
+        g.num_mtiles = o.num_mtiles;
+        g.mt_max = L.MT_max;
+        g.slot_assign = o.slot_assign;
+        g.topk_w = o.topk_w;
+        g.num_assign = L.A;
+        g.topk = k;
+        g.H = H;
+        g.pitch = p2H / 2;
+        g.xg = reinterpret_cast<__nv_bfloat16*>(reg(MOE_WS_XG));
+        g.dyg = reinterpret_cast<__nv_bfloat16*>(breg(kBwDYG));
+        g.dog = reinterpret_cast<__nv_bfloat16*>(breg(kBwDOG));
+        g.status = status;
+        if (launch_slot_gather(g, S, st) != cudaSuccess) return MOE_ERR_CUDA;
         if (cudaMemsetAsync(dx32, 0, (size_t)T * H * 4, st) != cudaSuccess ||
             cudaMemsetAsync(dwa, 0, (size_t)L.A * 4, st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
 
-    // tensor maps: K-major bf16 operands, 64-element x 128-row boxes
-    CUtensorMap mXg, mW1, mW3, mDyg, mW2t, mDgu, mW13t, mDot, mHt, mDgut, mXt;
-    const long p2H = act_pitch(2L * H), p4F = act_pitch(4L * F), p2F = act_pitch(2L * F), p8F = act_pitch(8L * F);
+    // tensor maps: 64-element x 128-row boxes for K-major operands, 64 x 64
+    // for MN-major ones (all bf16, 128-byte swizzle)
+    CUtensorMap mXg, mW1, mW3, mDyg, mW2mn, mDgu, mW1mn, mW3mn, mDogmn, mHmn, mDgumn, mXgmn;
     if (!make_map(&mXg, reg(MOE_WS_XG), S, H, p2H, 2, 128) ||
         !make_map(&mW1, w1, (size_t)E * F, H, (size_t)H * 2, 2, 128) ||
         !make_map(&mW3, w3, (size_t)E * F, H, (size_t)H * 2, 2, 128) ||
         !make_map(&mDyg, breg(kBwDYG), S, H, p2H, 2, 128) ||
-        !make_map(&mW2t, w2t, (size_t)E * F, H, (size_t)H * 2, 2, 128) ||
+        !make_map(&mW2mn, w2, (size_t)E * H, F, (size_t)F * 2, 2, 64) ||
         !make_map(&mDgu, breg(kBwDGU), S, 2L * F, p4F, 2, 128) ||
-        !make_map(&mW13t, w13t, (size_t)E * H, 2L * F, (size_t)F * 4, 2, 128) ||
-        !make_map(&mDot, breg(kBwDOT), H, S, (size_t)S * 2, 2, 128) ||
-        !make_map(&mHt, breg(kBwHT), F, S, (size_t)S * 2, 2, 128) ||
-        !make_map(&mDgut, breg(kBwGU), 2L * F, S, (size_t)S * 2, 2, 128) ||
-        !make_map(&mXt, breg(kBwXT), H, S, (size_t)S * 2, 2, 128))
+        !make_map(&mW1mn, w1, (size_t)E * F, H, (size_t)H * 2, 2, 64) ||
+        !make_map(&mW3mn, w3, (size_t)E * F, H, (size_t)H * 2, 2, 64) ||
+        !make_map(&mDogmn, breg(kBwDOG), S, H, p2H, 2, 64) ||
+        !make_map(&mHmn, reg(MOE_WS_H), S, F, p2F, 2, 64) ||
+        !make_map(&mDgumn, breg(kBwDGU), S, 2L * F, p4F, 2, 64) ||
+        !make_map(&mXgmn, reg(MOE_WS_XG), S, H, p2H, 2, 64))
         return MOE_ERR_CUDA;
 
     BwdArgs base{};
@@ -968,13 +943,13 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
                             grid_for(kBwdGU, pair, (pair ? mt_pairs : L.MT_max) * a.n_tiles), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
-    // 3. dh -> dg, du and the routing-weight gradients
+    // 3. dh = w_a W2^T dy -> dg, du and the routing-weight gradients
     {
         const int bn = (F % 256 == 0) ? 256 : 128;
         BwdArgs a = base;
         a.n_tiles = F / bn;
         a.k_tiles = H / 64;
-        a.b_rows = F;
+        a.b_rows = H;
         a.out = breg(kBwDGU);
         a.out_pitch = p4F;
         a.gu = breg(kBwGU);
@@ -984,7 +959,7 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.dw = dwa;
         const bool pair = bn == 256 && pairs_for(kBwdDH) > 0;
         ProfScope ps(MOE_KERNEL_BWD_DH, st);
-        if (launch_bwd_gemm(kBwdDH, bn, pair, mDyg, mW2t, mW2t, a,
+        if (launch_bwd_gemm(kBwdDH, bn, pair, mDyg, mW2mn, mW2mn, a,
                             grid_for(kBwdDH, pair, (pair ? mt_pairs : L.MT_max) * a.n_tiles), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
@@ -994,46 +969,18 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         BwdArgs a = base;
         a.n_tiles = H / bn;
         a.k_tiles = 2 * F / 64;
-        a.b_rows = H;
         a.out = dx32;
         a.out_pitch = (long)H * 4;
         const bool pair = bn == 256 && pairs_for(kBwdDX) > 0;
         ProfScope ps(MOE_KERNEL_BWD_DX, st);
-        if (launch_bwd_gemm(kBwdDX, bn, pair, mDgu, mW13t, mW13t, a,
+        if (launch_bwd_gemm(kBwdDX, bn, pair, mDgu, mW1mn, mW3mn, a,
                             grid_for(kBwdDX, pair, (pair ? mt_pairs : L.MT_max) * a.n_tiles), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
     {
-        ProfScope ps(MOE_KERNEL_BWD_AUX, st, 5);
+        ProfScope ps(MOE_KERNEL_BWD_AUX, st);
         if (launch_finalize(dx32, static_cast<__nv_bfloat16*>(dx), (size_t)T * H, num_sms, st) != cudaSuccess)
             return MOE_ERR_CUDA;
-        // transposed operands of the weight gradients: w_a dy_t and x_t per slot, h
-        TransposeArgs p{};
-        p.num_mtiles = o.num_mtiles;
-        p.mt_max = L.MT_max;
-        p.slot_assign = o.slot_assign;
-        p.num_assign = L.A;
-        p.topk = k;
-        p.out_pitch = S;
-        p.status = status;
-        p.src = dy;
-        p.src_pitch = H;
-        p.scale = o.topk_w;
-        p.out = breg(kBwDOT);
-        if (launch_transpose(kSrcTokens, p, H, S, 1, st) != cudaSuccess) return MOE_ERR_CUDA;
-        p.src = x;
-        p.scale = nullptr;
-        p.out = breg(kBwXT);
-        if (launch_transpose(kSrcTokens, p, H, S, 1, st) != cudaSuccess) return MOE_ERR_CUDA;
-        p.src = reg(MOE_WS_H);
-        p.src_pitch = p2F / 2;
-        p.out = breg(kBwHT);
-        if (launch_transpose(kSrcSlots, p, F, S, 1, st) != cudaSuccess) return MOE_ERR_CUDA;
-        // dg|du transposed, over g|u (read by step 3 only)
-        p.src = breg(kBwDGU);
-        p.src_pitch = p4F / 2;
-        p.out = breg(kBwGU);
-        if (launch_transpose(kSrcSlots, p, 2 * F, S, 1, st) != cudaSuccess) return MOE_ERR_CUDA;
     }
     // 5. dW2_e = (w dy)^T h and [dW1_e; dW3_e] = [dg; du]^T x over each expert's slots
     {
@@ -1049,7 +996,7 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         const bool pair = bn == 256 && a.m_tiles % 2 == 0 && pairs_for(kBwdDW) > 0;
         const long units = (long)E * (pair ? a.m_tiles / 2 : a.m_tiles) * a.n_tiles;
         ProfScope ps(MOE_KERNEL_BWD_DW2, st);
-        if (launch_bwd_gemm(kBwdDW, bn, pair, mDot, mHt, mHt, a, grid_for(kBwdDW, pair, units), st) != cudaSuccess)
+        if (launch_bwd_gemm(kBwdDW, bn, pair, mDogmn, mHmn, mHmn, a, grid_for(kBwdDW, pair, units), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
     {
@@ -1065,7 +1012,8 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         const bool pair = bn == 256 && a.m_tiles % 2 == 0 && pairs_for(kBwdDW) > 0;
         const long units = (long)E * (pair ? a.m_tiles / 2 : a.m_tiles) * a.n_tiles;
         ProfScope ps(MOE_KERNEL_BWD_DW13, st);
-        if (launch_bwd_gemm(kBwdDW, bn, pair, mDgut, mXt, mXt, a, grid_for(kBwdDW, pair, units), st) != cudaSuccess)
+        if (launch_bwd_gemm(kBwdDW, bn, pair, mDgumn, mXgmn, mXgmn, a, grid_for(kBwdDW, pair, units), st) !=
+            cudaSuccess)
             return MOE_ERR_CUDA;
     }
     // 6. router

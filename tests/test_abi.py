@@ -177,8 +177,8 @@ def test_backward_entry_checks(moe):
     assert moe.moe_backward_workspace_size(16, 4000, 14336, 8, 2) == 0   # d_model not a multiple of 128
     assert moe.moe_backward_workspace_size(16, 4096, 14336, 8, 9) == 0   # k > E
     P = 4096
-    assert moe.moe_ffn_backward(P, P, P, P, P, P, P, 16, 4096, 14336, 8, 2, P, P, P, P, P, None, 0, None) == -1
-    assert moe.moe_ffn_backward(P, P, P + 8, P, P, P, P, 16, 4096, 14336, 8, 2, P, P, P, P, P, P, 1 << 40,
+    assert moe.moe_ffn_backward(P, P, P, P, P, P, 16, 4096, 14336, 8, 2, P, P, P, P, P, None, 0, None) == -1
+    assert moe.moe_ffn_backward(P, P, P + 8, P, P, P, 16, 4096, 14336, 8, 2, P, P, P, P, P, P, 1 << 40,
                                 None) == -3
     n = moe.moe_backward_workspace_size(16, 256, 512, 8, 2)
-    assert moe.moe_ffn_backward(P, P, P, P, P, P, P, 16, 256, 512, 8, 2, P, P, P, P, P, P, n - 1, None) == -4
+    assert moe.moe_ffn_backward(P, P, P, P, P, P, 16, 256, 512, 8, 2, P, P, P, P, P, P, n - 1, None) == -4
