@@ -231,12 +231,16 @@ __global__ void __launch_bounds__(192, 1)
     auto unit_coords = [&](int u, int& e, int& m, int& n, int& k0, int& kc, bool& dup) {
         dup = false;
         if constexpr (MODE == kBwdDW) {
+            // inside an expert, the index of the larger operand changes slowest
+            // (n_fast: A is the larger, so a wave shares its rows and reads B's
+            // small columns from L2; otherwise the other way round)
             const int mt = PAIR ? args.m_tiles / 2 : args.m_tiles;
             const int per_e = mt * args.n_tiles;
             e = u / per_e;
             const int r = u - e * per_e;
-            m = PAIR ? 2 * (r % mt) + (int)rank : r % mt;
-            n = r / mt;
+            const int mi = args.n_fast ? r / args.n_tiles : r % mt;
+            m = PAIR ? 2 * mi + (int)rank : mi;
+            n = args.n_fast ? r % args.n_tiles : r / mt;
             k0 = 2 * s_mt_first[e];  // 64 slots per K step, 128 slots per tile
             kc = 2 * (s_mt_first[e + 1] - s_mt_first[e]);
         } else if constexpr (PAIR) {

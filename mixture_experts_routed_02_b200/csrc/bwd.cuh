@@ -35,6 +35,7 @@ struct BwdArgs {
     long h_pitch;
     float* dw;     // DH: routing-weight gradients [T*k] (fp32 atomics)
     int split;     // DW: output rows from here on go to out2
+    int n_fast;    // DW: n-tiles fastest inside an expert (A, the M side, is the larger operand)
     long expert_stride;  // DW: bytes per expert of out / out2
     unsigned long long timeout_ns;
     int* status;

@@ -993,6 +993,7 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.out_pitch = (long)F * 2;
         a.split = H;
         a.expert_stride = (long)H * F * 2;
+        a.n_fast = H > F ? 1 : 0;
         const bool pair = bn == 256 && a.m_tiles % 2 == 0 && pairs_for(kBwdDW) > 0;
         const long units = (long)E * (pair ? a.m_tiles / 2 : a.m_tiles) * a.n_tiles;
         ProfScope ps(MOE_KERNEL_BWD_DW2, st);
@@ -1009,6 +1010,7 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.out_pitch = (long)H * 2;
         a.split = F;
         a.expert_stride = (long)F * H * 2;
+        a.n_fast = 2 * F > H ? 1 : 0;  // dg|du (2F columns) is read once, x's H columns from L2
         const bool pair = bn == 256 && a.m_tiles % 2 == 0 && pairs_for(kBwdDW) > 0;
         const long units = (long)E * (pair ? a.m_tiles / 2 : a.m_tiles) * a.n_tiles;
         ProfScope ps(MOE_KERNEL_BWD_DW13, st);
