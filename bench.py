@@ -10,7 +10,7 @@ HBM.  The headline workload is the Mixtral-8x7B-shaped FP8 decode layer
 the same run also times every other workload of the Mixtral expert shape
 (prefill T=4096 FP8, skewed-routing T=8192 BF16, the FP8 batch sweep
 T = 1, 128, 1024, 16384, decode / prefill with MX FP4 expert weights, and a
-BF16 training step at T=4096: weight layout, forward, backward) and reports
+BF16 training step at T=4096: forward and backward) and reports
 each as a sub-record under ``configs`` with its own step time, roofline, CPU
 baseline and end-to-end number.
 
@@ -631,10 +631,10 @@ def train_cpu_baseline(case, dy, spec, name, seconds):
 
 
 def run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_seconds):
-    """Time one BF16 training step of the layer: the forward's weight layout
-    (redone every step, as weights change), the forward, and the backward
-    (custom VJP: dx, dw1, dw3, dw2, dlogits; it reads the weights as they
-    are).  Same structure of record as run_gpu_config."""
+    """Time one BF16 training step of the layer: the training forward (from
+    the row-major weights, which change every step, keeping routing, x, g, u
+    and h) and the backward from what it kept (custom VJP: dx, dw1, dw3, dw2,
+    dlogits).  Same structure of record as run_gpu_config."""
     import torch
     import torch.distributed as dist
 
@@ -651,17 +651,14 @@ def run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_seconds):
         x_cpu, lg_cpu = case["x"], case["logits"]
     x, logits, dy = x_cpu.to(dev), lg_cpu.to(dev), dy_cpu.to(dev)
     w1, w3, w2 = case["w1"].to(dev), case["w3"].to(dev), case["w2"].to(dev)
-    prep_f = moe.prepare_weights(w1, w3, None, None, w2)
-    ws_f = moe.workspace(T, H, F, E, k, "bf16", dev)
-    ws_b = moe.backward_workspace(T, H, F, E, k, dev)
-    y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-    grads = moe.ffn_backward(x, logits, w1, w3, w2, dy, k, ws=ws_b)
+    ws = moe.backward_workspace(T, H, F, E, k, dev)
+    y, _ = moe.ffn_forward_train(x, logits, w1, w3, w2, k, ws=ws)
+    grads = moe.ffn_backward_saved(w1, w3, w2, dy, k, ws)
     stream = torch.cuda.current_stream(dev)
 
     def step(xx=x, lgg=logits, dyy=dy, g=grads):
-        moe.prepare_weights(w1, w3, None, None, w2, stream=stream, out=prep_f)
-        moe.ffn_forward(xx, lgg, prep_f[0], None, prep_f[2], None, k, F, False, out=y, ws=ws_f, stream=stream)
-        moe.ffn_backward(xx, lgg, w1, w3, w2, dyy, k, ws=ws_b, out=g, stream=stream)
+        moe.ffn_forward_train(xx, lgg, w1, w3, w2, k, ws=ws, out=y, stream=stream)
+        moe.ffn_backward_saved(w1, w3, w2, dyy, k, ws, out=g, stream=stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -669,7 +666,7 @@ def run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_seconds):
     st = moe.moe_get_status(None)
     if st != 0:
         raise RuntimeError(f"{name}: device status {moe.STATUS_NAMES.get(st, st)} after warm-up")
-    counts = moe.ws_view(ws_f, T, H, F, E, k, "bf16", "counts", torch.int32).cpu().tolist()
+    counts = moe.ws_view(ws, T, H, F, E, k, "bf16", "counts", torch.int32).cpu().tolist()
 
     clocks = ClockSampler(torch.cuda.current_device())
     if world > 1:
@@ -737,7 +734,7 @@ def run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_seconds):
     # roofline of the dominant kernel (tensor-bound at this size): algorithmic
     # FLOPs per launch from the routed assignments A = T k (padding rows excluded)
     A = T * k
-    kflops = {"stage1_w13_swiglu": 4.0 * A * F * H, "stage2_w2_scatter": 2.0 * A * F * H,
+    kflops = {"stage1_w13_swiglu": 4.0 * A * F * H, "stage2_w2_scatter": 2.0 * A * F * H,  # the training forward
               "bwd_gu_recompute": 4.0 * A * F * H, "bwd_dh_swiglu": 2.0 * A * F * H,
               "bwd_dx_scatter": 4.0 * A * F * H, "bwd_dw2": 2.0 * A * F * H, "bwd_dw13": 4.0 * A * F * H}
     dom = max(kflops, key=lambda n: kern[n][0])
@@ -751,14 +748,15 @@ def run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_seconds):
             "traffic": recorded_traffic(dom, name),
             "peak_source": f"{peak_kind} {'sustained' if long_run else 'burst'} bf16 cuBLAS",
             "algorithmic_per_launch": kflops[dom], "kernel": dom, "kernel_ms": dom_ms}
-    step_flops = 22.0 * A * F * H  # forward 6, recompute of g/u 4, dh 2, dx 4, dW2 2, dW1/dW3 4
+    step_flops = 18.0 * A * F * H  # forward 6 (g, u, h kept), dh 2, dx 4, dW2 2, dW1/dW3 4
     launches = sum(v[1] for v in kern.values())
     wbytes = 3 * E * F * H * 2
     return {
         "value": value, "unit": "tokens/s", "ms_per_step": ms_step, "steps": args.steps, "warmup": args.warmup,
         "dtype": "bf16 (fp32 accumulate)",
-        "config": {"workload": workload_desc(spec, name) + "; training step: forward weight layout, forward, "
-                   "backward (dx, dw1, dw3, dw2, dlogits)", "T": T, "d_model": H, "d_ff": F, "experts": E, "top_k": k,
+        "config": {"workload": workload_desc(spec, name) + "; training step: forward from the row-major weights "
+                   "keeping g/u/h, backward from them (dx, dw1, dw3, dw2, dlogits)", "T": T, "d_model": H, "d_ff": F,
+                   "experts": E, "top_k": k,
                    "weights": "bf16", "parallelism": f"weak-scaling replicas x{world}" if world > 1 else "1 GPU",
                    "l2": "inputs larger than L2 (expert weights %.2f GB, read by several kernels per step)" % (
                        wbytes / 1e9),

@@ -410,6 +410,23 @@ int moe_profile_read(double* ms_total, int* launches, int reset);
  *   for the forward).
  */
 size_t moe_backward_workspace_size(int T, int H, int F, int E, int k);
+/*
+ * Training pair.  moe_ffn_forward_train: the BF16 layer of moe_ffn_forward
+ *   (same output, same arithmetic: h rounded to bf16, fp32 combine rounded
+ *   once) computed from the caller's row-major w1, w3, w2 -- no
+ *   moe_prepare_weights, which a training step would have to redo after every
+ *   weight update -- and keeping in `ws` (moe_backward_workspace_size bytes)
+ *   the routing, the gathered x and g, u, h of this call.
+ * moe_ffn_backward_saved: the backward of the last moe_ffn_forward_train on
+ *   the same `ws`, from what it kept (no routing, no recompute of g and u; x
+ *   and logits are not needed again).  Same outputs and contract as
+ *   moe_ffn_backward; T, H, F, E, k and the weights must be the forward's.
+ */
+int moe_ffn_forward_train(const void* x, const float* logits, const void* w1, const void* w3, const void* w2, int T,
+                          int H, int F, int E, int k, void* out, void* ws, size_t ws_bytes, void* stream);
+int moe_ffn_backward_saved(const void* w1, const void* w3, const void* w2, const void* dy, int T, int H, int F, int E,
+                           int k, void* dx, void* dw1, void* dw3, void* dw2, float* dlogits, void* ws, size_t ws_bytes,
+                           void* stream);
 int moe_ffn_backward(const void* x, const float* logits, const void* w1, const void* w3, const void* w2,
                      const void* dy, int T, int H, int F, int E, int k, void* dx, void* dw1, void* dw3, void* dw2,
                      float* dlogits, void* ws, size_t ws_bytes, void* stream);

@@ -55,7 +55,8 @@ WS = dict(topk_ids=0, topk_w=1, counts=2, offsets=3, perm=4, inv_perm=5, slot_of
 EXPORTS = ["moe_workspace_size", "moe_prepare_weights", "moe_route", "moe_ffn_forward", "moe_get_status",
            "moe_workspace_region", "moe_set_option", "moe_profile_enable", "moe_profile_read",
            "moe_ffn_forward_static", "moe_static_workspace_bytes", "moe_ffn_forward_dff", "moe_dff_finalize",
-           "moe_prepare_weights_mx", "moe_backward_workspace_size", "moe_ffn_backward"]
+           "moe_prepare_weights_mx", "moe_backward_workspace_size", "moe_ffn_backward", "moe_ffn_forward_train",
+           "moe_ffn_backward_saved"]
 # kernel ids of moe_profile_read: the forward's five, then the backward's
 FWD_KERNELS = ["route", "quantize", "stage1_w13_swiglu", "stage2_w2_scatter", "finalize"]
 BWD_KERNELS = ["bwd_gu_recompute", "bwd_dh_swiglu", "bwd_dx_scatter", "bwd_dw2", "bwd_dw13", "bwd_aux"]
@@ -105,6 +106,10 @@ lib.moe_backward_workspace_size.restype = _Z
 lib.moe_backward_workspace_size.argtypes = [_I, _I, _I, _I, _I]
 lib.moe_ffn_backward.restype = _I
 lib.moe_ffn_backward.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]
+lib.moe_ffn_forward_train.restype = _I
+lib.moe_ffn_forward_train.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P]
+lib.moe_ffn_backward_saved.restype = _I
+lib.moe_ffn_backward_saved.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]
 
 # raw entry points, same names as the C ABI
 moe_workspace_size = lib.moe_workspace_size
@@ -121,6 +126,8 @@ moe_ffn_forward_dff = lib.moe_ffn_forward_dff
 moe_dff_finalize = lib.moe_dff_finalize
 moe_backward_workspace_size = lib.moe_backward_workspace_size
 moe_ffn_backward = lib.moe_ffn_backward
+moe_ffn_forward_train = lib.moe_ffn_forward_train
+moe_ffn_backward_saved = lib.moe_ffn_backward_saved
 
 
 def moe_profile_read(reset=True):
@@ -361,4 +368,51 @@ def ffn_backward(x, logits, w1, w3, w2, dy, k, ws=None, out=None, stream=None):
                           _ptr(out["dx"]), _ptr(out["dw1"]), _ptr(out["dw3"]), _ptr(out["dw2"]), _ptr(out["dlogits"]),
                           _ptr(ws), ws.numel(), _stream(stream))
     _check("moe_ffn_backward", rc)
+    return out
+
+
+def _bf16_weights(w1, w3, w2, fn):
+    import torch
+    for t in (w1, w3, w2):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{fn} takes contiguous bf16 weights")
+    E, F, H = w1.shape
+    if w3.shape != (E, F, H) or w2.shape != (E, H, F):
+        raise ValueError("weight shapes do not match")
+    return E, F, H
+
+
+def ffn_forward_train(x, logits, w1, w3, w2, k, ws=None, out=None, stream=None):
+    """The BF16 layer from the row-major weights (no preparation), keeping in
+    ``ws`` (a backward workspace) what ffn_backward_saved needs; returns
+    (out [T,H] bf16, ws)."""
+    import torch
+    T, H = x.shape
+    E, F, _ = _bf16_weights(w1, w3, w2, "ffn_forward_train")
+    if ws is None:
+        ws = backward_workspace(T, H, F, E, k, x.device)
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
+    _check("moe_ffn_forward_train", moe_ffn_forward_train(_ptr(x), _ptr(logits), _ptr(w1), _ptr(w3), _ptr(w2), T, H, F,
+                                                          E, k, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, ws
+
+
+def ffn_backward_saved(w1, w3, w2, dy, k, ws, out=None, stream=None):
+    """The backward of the last ffn_forward_train on ``ws``: same result dict
+    as ffn_backward."""
+    import torch
+    T, H = dy.shape
+    E, F, _ = _bf16_weights(w1, w3, w2, "ffn_backward_saved")
+    dev = dy.device
+    if out is None:
+        out = dict(dx=torch.empty(T, H, dtype=torch.bfloat16, device=dev),
+                   dw1=torch.empty(E, F, H, dtype=torch.bfloat16, device=dev),
+                   dw3=torch.empty(E, F, H, dtype=torch.bfloat16, device=dev),
+                   dw2=torch.empty(E, H, F, dtype=torch.bfloat16, device=dev),
+                   dlogits=torch.empty(T, E, dtype=torch.float32, device=dev))
+    rc = moe_ffn_backward_saved(_ptr(w1), _ptr(w3), _ptr(w2), _ptr(dy), T, H, F, E, k, _ptr(out["dx"]),
+                                _ptr(out["dw1"]), _ptr(out["dw3"]), _ptr(out["dw2"]), _ptr(out["dlogits"]), _ptr(ws),
+                                ws.numel(), _stream(stream))
+    _check("moe_ffn_backward_saved", rc)
     return out

@@ -50,9 +50,10 @@ namespace {
 // stage of 32 KB instead of 48 leaves room for six stages.
 template <int MODE, int BN, int NST, bool PAIR>
 struct BCfg {
-    // operand majorness: A MN-major in DW; B MN-major in DH, DX and DW
+    // operand majorness: A MN-major in DW; B MN-major in DH, DX and DW (GU
+    // and FwdW2 read weight rows, K-major)
     static constexpr bool A_MN = MODE == kBwdDW;
-    static constexpr bool B_MN = MODE != kBwdGU;
+    static constexpr bool B_MN = MODE == kBwdDH || MODE == kBwdDX || MODE == kBwdDW;
     static constexpr int A_BYTES = kBlockM * 128;  // 128 rows x 64 bf16
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // this CTA's rows of B
     static constexpr int B_BYTES = B_ROWS * 128;
@@ -329,6 +330,11 @@ __global__ void __launch_bounds__(192, 1)
                             load(sb, &tmB, kx, e * args.b_rows + n * 128, pol_b);
                             load(sb + 128 * 128, &tmB2, kx, e * args.b_rows + n * 128, pol_b);
                         }
+                    } else if constexpr (!C::B_MN) {
+                        // FwdW2: BN (or this CTA's B_ROWS) rows of W2_e, K-major
+#pragma unroll
+                        for (int j = 0; j < C::B_ROWS / 128; ++j)
+                            load(sb + j * 128 * 128, &tmB, kx, e * args.b_rows + ncol + 128 * j, pol_b);
                     } else {
                         // MN-major boxes of 64 columns x 64 K rows: DH from W2_e (rows
                         // h = K), DX from W1_e for K < F and W3_e beyond (rows c = K),
@@ -547,8 +553,11 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 }
                 if (a >= 0) atomicAdd(args.dw + a, part);
-            } else if constexpr (MODE == kBwdDX) {
+            } else if constexpr (MODE == kBwdDX || MODE == kFwdW2) {
+                // dx: the k experts of a token meet in fp32; FwdW2: the same with
+                // the routing weight (the forward's combine)
                 const int t = (a >= 0) ? a / args.topk : -1;
+                const float wa = (MODE == kFwdW2 && t >= 0) ? args.topk_w[a] : 1.0f;
                 float* orow = reinterpret_cast<float*>(static_cast<uint8_t*>(args.out) + (size_t)(t >= 0 ? t : 0) * args.out_pitch);
 #pragma unroll 1
                 for (int c0 = 0; c0 < BN; c0 += 64) {
@@ -562,8 +571,9 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                         for (int i4 = 0; i4 < 16; ++i4)
                             atomicAdd(reinterpret_cast<float4*>(orow + col + 4 * i4),
-                                      make_float4(__uint_as_float(r[4 * i4]), __uint_as_float(r[4 * i4 + 1]),
-                                                  __uint_as_float(r[4 * i4 + 2]), __uint_as_float(r[4 * i4 + 3])));
+                                      make_float4(__uint_as_float(r[4 * i4]) * wa, __uint_as_float(r[4 * i4 + 1]) * wa,
+                                                  __uint_as_float(r[4 * i4 + 2]) * wa,
+                                                  __uint_as_float(r[4 * i4 + 3]) * wa));
                     }
                 }
             } else {
@@ -614,8 +624,9 @@ __global__ void __launch_bounds__(192, 1)
 // ---------------------------------------------------------------- slot gather
 // Rows of the expert-padded slot layout for the backward's operands, zero for
 // padding slots (the weight gradients sum over every slot of an expert):
-// xg[s] = x[t], dyg[s] = dy[t], dog[s] = bf16(w_a dy[t]) for slot s holding
-// assignment a = (t, j); rows from num_mtiles * 128 on are left alone.  One
+// xg[s] = x[t] (if x is given), dyg[s] = dy[t] and dog[s] = bf16(w_a dy[t])
+// (if dy is given) for slot s holding assignment a = (t, j); rows from
+// num_mtiles * 128 on are left alone.  One
 // warp per slot row, 16-byte pieces.
 __global__ void __launch_bounds__(256) slot_gather_kernel(SlotGatherArgs p) {
     const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
@@ -636,19 +647,20 @@ __global__ void __launch_bounds__(256) slot_gather_kernel(SlotGatherArgs p) {
     uint4* dyo = reinterpret_cast<uint4*>(p.dyg + (size_t)s * p.pitch);
     uint4* doo = reinterpret_cast<uint4*>(p.dog + (size_t)s * p.pitch);
     for (int i = lane; i < p.H / 8; i += 32) {
-        uint4 xv = make_uint4(0u, 0u, 0u, 0u), dv = xv, ov = xv;
-        if (a >= 0) {
-            xv = __ldg(xr + i);
-            dv = __ldg(dr + i);
-            float f[8];
-            unpack8(dv, f);
+        if (p.x) xo[i] = a >= 0 ? __ldg(xr + i) : make_uint4(0u, 0u, 0u, 0u);
+        if (p.dy) {
+            uint4 dv = make_uint4(0u, 0u, 0u, 0u), ov = dv;
+            if (a >= 0) {
+                dv = __ldg(dr + i);
+                float f[8];
+                unpack8(dv, f);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) f[j] *= w;
-            ov = pack8(f);
+                for (int j = 0; j < 8; ++j) f[j] *= w;
+                ov = pack8(f);
+            }
+            dyo[i] = dv;
+            doo[i] = ov;
         }
-        xo[i] = xv;
-        dyo[i] = dv;
-        doo[i] = ov;
     }
 }
 
@@ -717,6 +729,7 @@ int bwd_max_pairs(int mode) {
         case kBwdDH: return max_pairs_one<kBwdDH>();
         case kBwdDX: return max_pairs_one<kBwdDX>();
         case kBwdDW: return max_pairs_one<kBwdDW>();
+        case kFwdW2: return max_pairs_one<kFwdW2>();
         default: return 0;
     }
 }
@@ -744,6 +757,10 @@ cudaError_t launch_bwd_gemm(int mode, int bn, bool pair, const CUtensorMap& a, c
             return pair ? launch_bwd_one<kBwdDW, 256, 6, true>(a, b, b2, args, grid, stream)
                  : bn == 256 ? launch_bwd_one<kBwdDW, 256, 4, false>(a, b, b2, args, grid, stream)
                              : launch_bwd_one<kBwdDW, 128, 6, false>(a, b, b2, args, grid, stream);
+        case kFwdW2:
+            return pair ? launch_bwd_one<kFwdW2, 256, 6, true>(a, b, b2, args, grid, stream)
+                 : bn == 256 ? launch_bwd_one<kFwdW2, 256, 4, false>(a, b, b2, args, grid, stream)
+                             : launch_bwd_one<kFwdW2, 128, 6, false>(a, b, b2, args, grid, stream);
         default:
             return cudaErrorInvalidValue;
     }

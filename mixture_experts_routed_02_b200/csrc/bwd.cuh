@@ -10,7 +10,9 @@ namespace moe {
 // Grouped GEMMs of the backward pass (bwd.cu): GU recomputes g, u and h; DH
 // gives dg, du and the routing-weight gradients; DX scatters dx; DW forms the
 // weight gradients per expert (operands read K-major or MN-major as they lie).
-enum BwdMode { kBwdGU = 0, kBwdDH = 1, kBwdDX = 2, kBwdDW = 3 };
+// (kFwdW2: the training forward's second GEMM, h . W2_e^T with the weighted
+// scatter-add, from the caller's row-major w2)
+enum BwdMode { kBwdGU = 0, kBwdDH = 1, kBwdDX = 2, kBwdDW = 3, kFwdW2 = 4 };
 
 struct BwdArgs {
     // the expert-padded slot layout (from the router)
@@ -25,7 +27,7 @@ struct BwdArgs {
     int m_tiles;   // DW: output rows / 128
     int b_rows;    // rows of B's matrix per expert (GU: F rows of W1 / W3; DH: H rows of W2)
     int F;         // d_ff (GU, DH: column offset of u and du; DX: where K moves from W1 to W3)
-    void* out;     // GU: fp32 g|u [S, 2F]; DH: dg|du [S, 2F]; DX: fp32 dx [T, H]; DW: dW (first part)
+    void* out;     // GU: fp32 g|u [S, 2F]; DH: dg|du [S, 2F]; DX, FwdW2: fp32 rows [T, H]; DW: dW (first part)
     long out_pitch;  // bytes
     void* out2;    // GU: h [S, F]; DW: rows >= split (dW3)
     long out2_pitch;
@@ -47,7 +49,8 @@ cudaError_t launch_bwd_gemm(int mode, int bn, bool pair, const CUtensorMap& a, c
 int bwd_max_pairs(int mode);  // resident clusters of the pair kernel (0: none)
 
 // Rows of the slot layout for the backward (zero for padding slots):
-// xg = x[t], dyg = dy[t], dog = bf16(w_a dy[t]); rows `pitch` elements apart.
+// xg = x[t] (when x is given), dyg = dy[t] and dog = bf16(w_a dy[t]) (when dy
+// is given); rows `pitch` elements apart.
 struct SlotGatherArgs {
     const __nv_bfloat16* x;
     const __nv_bfloat16* dy;

@@ -800,30 +800,39 @@ bool bwd_dims_ok(int T, int H, int F, int E, int k) {
 
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-}  // namespace
+enum TrainPart { kTrainForward = 0, kTrainBackwardSaved = 1, kTrainBackward = 2 };
 
-extern "C" {
-
-size_t moe_backward_workspace_size(int T, int H, int F, int E, int k) {
-    if (!bwd_dims_ok(T, H, F, E, k)) return 0;
-    return make_bwd_layout(T, H, F, E, k).total;
-}
-
-int moe_ffn_backward(const void* x, const float* logits, const void* w1, const void* w3, const void* w2,
-                     const void* dy, int T, int H, int F, int E, int k, void* dx, void* dw1, void* dw3, void* dw2,
-                     float* dlogits, void* ws, size_t ws_bytes, void* stream) {
+// The training forward and the two forms of the backward share one workspace
+// layout.  kTrainForward: routing, x gathered into the slot layout, g/u/h
+// (kept for the backward), the second GEMM with the weighted combine, the bf16
+// output.  kTrainBackwardSaved: the backward from what the forward kept.
+// kTrainBackward: the backward with its own routing and g/u/h recompute.
+int train_impl(int part, const void* x, const float* logits, const void* w1, const void* w3, const void* w2,
+               const void* dy, int T, int H, int F, int E, int k, void* out, void* dx, void* dw1, void* dw3,
+               void* dw2, float* dlogits, void* ws, size_t ws_bytes, void* stream) {
+    const bool fwd = part == kTrainForward;
+    const bool bwd = !fwd;
+    const bool recompute = part == kTrainBackward;
     if (!bwd_dims_ok(T, H, F, E, k)) return MOE_ERR_INVALID_ARG;
-    if (!w1 || !w3 || !w2 || !dw1 || !dw3 || !dw2 || !ws) return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (!x || !logits || !dy || !dx || !dlogits)) return MOE_ERR_INVALID_ARG;
-    for (const void* ptr : {w1, w3, w2, (const void*)dw1, (const void*)dw3, (const void*)dw2, (const void*)ws})
+    if (!w1 || !w3 || !w2 || !ws || (bwd && (!dw1 || !dw3 || !dw2))) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && ((part != kTrainBackwardSaved && (!x || !logits)) || (fwd && !out) || (bwd && (!dy || !dx || !dlogits))))
+        return MOE_ERR_INVALID_ARG;
+    for (const void* ptr : {w1, w3, w2, (const void*)ws})
         if (!aligned16(ptr)) return MOE_ERR_ALIGNMENT;
-    if (T > 0 && (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || !aligned4(logits) || !aligned4(dlogits)))
-        return MOE_ERR_ALIGNMENT;
+    if (bwd)
+        for (const void* ptr : {(const void*)dw1, (const void*)dw3, (const void*)dw2})
+            if (!aligned16(ptr)) return MOE_ERR_ALIGNMENT;
+    if (T > 0) {
+        if (part != kTrainBackwardSaved && (!aligned16(x) || !aligned4(logits))) return MOE_ERR_ALIGNMENT;
+        if (fwd && !aligned16(out)) return MOE_ERR_ALIGNMENT;
+        if (bwd && (!aligned16(dy) || !aligned16(dx) || !aligned4(dlogits))) return MOE_ERR_ALIGNMENT;
+    }
     const BwdLayout B = make_bwd_layout(T, H, F, E, k);
     const Layout& L = B.fwd;
     if (ws_bytes < B.total) return MOE_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (T == 0) {  // no tokens: every weight gradient is zero
+    if (T == 0) {  // no tokens: nothing to compute; every weight gradient is zero
+        if (fwd) return MOE_OK;
         const size_t n = (size_t)E * F * H * 2;
         if (cudaMemsetAsync(dw1, 0, n, st) != cudaSuccess || cudaMemsetAsync(dw3, 0, n, st) != cudaSuccess ||
             cudaMemsetAsync(dw2, 0, n, st) != cudaSuccess)
@@ -841,7 +850,6 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
     const unsigned long long timeout_ns = (unsigned long long)g_opt_timeout_ms.load() * 1000000ull;
     const long p2H = act_pitch(2L * H), p4F = act_pitch(4L * F), p2F = act_pitch(2L * F), p8F = act_pitch(8L * F);
 
-    // 1. the forward's routing and slot layout; x, dy and w_a dy gathered into it
     RouteOutputs o{reinterpret_cast<int32_t*>(reg(MOE_WS_TOPK_IDS)), reinterpret_cast<float*>(reg(MOE_WS_TOPK_W)),
                    reinterpret_cast<int32_t*>(reg(MOE_WS_COUNTS)), reinterpret_cast<int32_t*>(reg(MOE_WS_OFFSETS)),
                    reinterpret_cast<int32_t*>(reg(MOE_WS_PERM)), reinterpret_cast<int32_t*>(reg(MOE_WS_INV_PERM)),
@@ -849,14 +857,20 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
                    reinterpret_cast<int32_t*>(reg(MOE_WS_MTILE_EXPERT)),
                    reinterpret_cast<int32_t*>(reg(MOE_WS_NUM_MTILES)),
                    reinterpret_cast<int32_t*>(reg(MOE_WS_ROUTE_BLOCKS))};
-    float* dx32 = reinterpret_cast<float*>(reg(MOE_WS_OUT32));
+    float* rows32 = reinterpret_cast<float*>(reg(MOE_WS_OUT32));  // the forward's combine, or dx32
     float* dwa = reinterpret_cast<float*>(breg(kBwDW));
+
+    // 1. routing (the backward from saved activations reuses the forward's),
+    // and the slot gather: x (forward, recompute) and dy, w_a dy (backward)
     {
-        ProfScope ps(MOE_KERNEL_BWD_AUX, st, route_launches(T, o) + 1);
-        if (launch_route(logits, T, E, k, o, st) != cudaSuccess) return MOE_ERR_CUDA;
+        ProfScope ps(fwd ? MOE_KERNEL_ROUTE : MOE_KERNEL_BWD_AUX, st, part == kTrainBackwardSaved ? 0 : route_launches(T, o));
+        if (part != kTrainBackwardSaved && launch_route(logits, T, E, k, o, st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    {
+        ProfScope ps(fwd ? MOE_KERNEL_QUANT : MOE_KERNEL_BWD_AUX, st);
         SlotGatherArgs g{};
-        g.x = static_cast<const __nv_bfloat16*>(x);
-        g.dy = static_cast<const __nv_bfloat16*>(dy);
+        g.x = part == kTrainBackwardSaved ? nullptr : static_cast<const __nv_bfloat16*>(x);
+        g.dy = bwd ? static_cast<const __nv_bfloat16*>(dy) : nullptr;
         g.num_mtiles = o.num_mtiles;
         g.mt_max = L.MT_max;
         g.slot_assign = o.slot_assign;
@@ -870,26 +884,29 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         g.dog = reinterpret_cast<__nv_bfloat16*>(breg(kBwDOG));
         g.status = status;
         if (launch_slot_gather(g, S, st) != cudaSuccess) return MOE_ERR_CUDA;
-        if (cudaMemsetAsync(dx32, 0, (size_t)T * H * 4, st) != cudaSuccess ||
-            cudaMemsetAsync(dwa, 0, (size_t)L.A * 4, st) != cudaSuccess)
-            return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(rows32, 0, (size_t)T * H * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+        if (bwd && cudaMemsetAsync(dwa, 0, (size_t)L.A * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     }
 
     // tensor maps: 64-element x 128-row boxes for K-major operands, 64 x 64
     // for MN-major ones (all bf16, 128-byte swizzle)
-    CUtensorMap mXg, mW1, mW3, mDyg, mW2mn, mDgu, mW1mn, mW3mn, mDogmn, mHmn, mDgumn, mXgmn;
+    CUtensorMap mXg, mW1, mW3, mH, mW2k, mDyg, mW2mn, mDgu, mW1mn, mW3mn, mDogmn, mHmn, mDgumn, mXgmn;
     if (!make_map(&mXg, reg(MOE_WS_XG), S, H, p2H, 2, 128) ||
         !make_map(&mW1, w1, (size_t)E * F, H, (size_t)H * 2, 2, 128) ||
-        !make_map(&mW3, w3, (size_t)E * F, H, (size_t)H * 2, 2, 128) ||
-        !make_map(&mDyg, breg(kBwDYG), S, H, p2H, 2, 128) ||
-        !make_map(&mW2mn, w2, (size_t)E * H, F, (size_t)F * 2, 2, 64) ||
-        !make_map(&mDgu, breg(kBwDGU), S, 2L * F, p4F, 2, 128) ||
-        !make_map(&mW1mn, w1, (size_t)E * F, H, (size_t)H * 2, 2, 64) ||
-        !make_map(&mW3mn, w3, (size_t)E * F, H, (size_t)H * 2, 2, 64) ||
-        !make_map(&mDogmn, breg(kBwDOG), S, H, p2H, 2, 64) ||
-        !make_map(&mHmn, reg(MOE_WS_H), S, F, p2F, 2, 64) ||
-        !make_map(&mDgumn, breg(kBwDGU), S, 2L * F, p4F, 2, 64) ||
-        !make_map(&mXgmn, reg(MOE_WS_XG), S, H, p2H, 2, 64))
+        !make_map(&mW3, w3, (size_t)E * F, H, (size_t)H * 2, 2, 128))
+        return MOE_ERR_CUDA;
+    if (fwd && (!make_map(&mH, reg(MOE_WS_H), S, F, p2F, 2, 128) ||
+                !make_map(&mW2k, w2, (size_t)E * H, F, (size_t)F * 2, 2, 128)))
+        return MOE_ERR_CUDA;
+    if (bwd && (!make_map(&mDyg, breg(kBwDYG), S, H, p2H, 2, 128) ||
+                !make_map(&mW2mn, w2, (size_t)E * H, F, (size_t)F * 2, 2, 64) ||
+                !make_map(&mDgu, breg(kBwDGU), S, 2L * F, p4F, 2, 128) ||
+                !make_map(&mW1mn, w1, (size_t)E * F, H, (size_t)H * 2, 2, 64) ||
+                !make_map(&mW3mn, w3, (size_t)E * F, H, (size_t)H * 2, 2, 64) ||
+                !make_map(&mDogmn, breg(kBwDOG), S, H, p2H, 2, 64) ||
+                !make_map(&mHmn, reg(MOE_WS_H), S, F, p2F, 2, 64) ||
+                !make_map(&mDgumn, breg(kBwDGU), S, 2L * F, p4F, 2, 64) ||
+                !make_map(&mXgmn, reg(MOE_WS_XG), S, H, p2H, 2, 64)))
         return MOE_ERR_CUDA;
 
     BwdArgs base{};
@@ -912,8 +929,8 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
     auto pairs_for = [&](int mode) {
         if (opt_path >= 2) return 0;
         static std::mutex mu;
-        static unsigned long long key[4] = {0, 0, 0, 0};
-        static int val[4] = {0, 0, 0, 0};
+        static unsigned long long key[5] = {0, 0, 0, 0, 0};
+        static int val[5] = {0, 0, 0, 0, 0};
         std::lock_guard<std::mutex> lock(mu);
         if (key[mode] != ctx.ctx_id) {
             val[mode] = bwd_max_pairs(mode);
@@ -927,8 +944,8 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
     };
     const long mt_pairs = (L.MT_max + 1) / 2 + E;  // upper bound of the m-tile pairs over all experts
 
-    // 2. g, u, h recomputed
-    {
+    // 2. g, u (fp32, kept for the backward) and h = bf16(silu(g) u)
+    if (fwd || recompute) {
         BwdArgs a = base;
         a.n_tiles = F / 128;
         a.k_tiles = H / 64;
@@ -938,10 +955,29 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         a.out2 = reg(MOE_WS_H);
         a.out2_pitch = p2F;
         const bool pair = pairs_for(kBwdGU) > 0;
-        ProfScope ps(MOE_KERNEL_BWD_GU, st);
+        ProfScope ps(fwd ? MOE_KERNEL_STAGE1 : MOE_KERNEL_BWD_GU, st);
         if (launch_bwd_gemm(kBwdGU, 256, pair, mXg, mW1, mW3, a,
                             grid_for(kBwdGU, pair, (pair ? mt_pairs : L.MT_max) * a.n_tiles), st) != cudaSuccess)
             return MOE_ERR_CUDA;
+    }
+    if (fwd) {
+        // 3. the forward's second GEMM: w_a (h . W2_e^T) added into the token's fp32 row, then bf16
+        const int bn = (H % 256 == 0) ? 256 : 128;
+        BwdArgs a = base;
+        a.n_tiles = H / bn;
+        a.k_tiles = F / 64;
+        a.b_rows = H;
+        a.out = rows32;
+        a.out_pitch = (long)H * 4;
+        const bool pair = bn == 256 && pairs_for(kFwdW2) > 0;
+        {
+            ProfScope ps(MOE_KERNEL_STAGE2, st);
+            if (launch_bwd_gemm(kFwdW2, bn, pair, mH, mW2k, mW2k, a,
+                                grid_for(kFwdW2, pair, (pair ? mt_pairs : L.MT_max) * a.n_tiles), st) != cudaSuccess)
+                return MOE_ERR_CUDA;
+        }
+        ProfScope ps(MOE_KERNEL_FINALIZE, st);
+        return launch_status(launch_finalize(rows32, static_cast<__nv_bfloat16*>(out), (size_t)T * H, num_sms, st));
     }
     // 3. dh = w_a W2^T dy -> dg, du and the routing-weight gradients
     {
@@ -969,7 +1005,7 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         BwdArgs a = base;
         a.n_tiles = H / bn;
         a.k_tiles = 2 * F / 64;
-        a.out = dx32;
+        a.out = rows32;
         a.out_pitch = (long)H * 4;
         const bool pair = bn == 256 && pairs_for(kBwdDX) > 0;
         ProfScope ps(MOE_KERNEL_BWD_DX, st);
@@ -979,7 +1015,7 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
     }
     {
         ProfScope ps(MOE_KERNEL_BWD_AUX, st);
-        if (launch_finalize(dx32, static_cast<__nv_bfloat16*>(dx), (size_t)T * H, num_sms, st) != cudaSuccess)
+        if (launch_finalize(rows32, static_cast<__nv_bfloat16*>(dx), (size_t)T * H, num_sms, st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
     // 5. dW2_e = (w dy)^T h and [dW1_e; dW3_e] = [dg; du]^T x over each expert's slots
@@ -1024,6 +1060,35 @@ int moe_ffn_backward(const void* x, const float* logits, const void* w1, const v
         if (launch_dlogits(o.topk_ids, o.topk_w, dwa, T, E, k, dlogits, st) != cudaSuccess) return MOE_ERR_CUDA;
     }
     return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_backward_workspace_size(int T, int H, int F, int E, int k) {
+    if (!bwd_dims_ok(T, H, F, E, k)) return 0;
+    return make_bwd_layout(T, H, F, E, k).total;
+}
+
+int moe_ffn_forward_train(const void* x, const float* logits, const void* w1, const void* w3, const void* w2, int T,
+                          int H, int F, int E, int k, void* out, void* ws, size_t ws_bytes, void* stream) {
+    return train_impl(kTrainForward, x, logits, w1, w3, w2, nullptr, T, H, F, E, k, out, nullptr, nullptr, nullptr,
+                      nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+int moe_ffn_backward_saved(const void* w1, const void* w3, const void* w2, const void* dy, int T, int H, int F, int E,
+                           int k, void* dx, void* dw1, void* dw3, void* dw2, float* dlogits, void* ws, size_t ws_bytes,
+                           void* stream) {
+    return train_impl(kTrainBackwardSaved, nullptr, nullptr, w1, w3, w2, dy, T, H, F, E, k, nullptr, dx, dw1, dw3,
+                      dw2, dlogits, ws, ws_bytes, stream);
+}
+
+int moe_ffn_backward(const void* x, const float* logits, const void* w1, const void* w3, const void* w2,
+                     const void* dy, int T, int H, int F, int E, int k, void* dx, void* dw1, void* dw3, void* dw2,
+                     float* dlogits, void* ws, size_t ws_bytes, void* stream) {
+    return train_impl(kTrainBackward, x, logits, w1, w3, w2, dy, T, H, F, E, k, nullptr, dx, dw1, dw3, dw2, dlogits,
+                      ws, ws_bytes, stream);
 }
 
 }  // extern "C"

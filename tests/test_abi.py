@@ -182,3 +182,17 @@ def test_backward_entry_checks(moe):
                                 None) == -3
     n = moe.moe_backward_workspace_size(16, 256, 512, 8, 2)
     assert moe.moe_ffn_backward(P, P, P, P, P, P, 16, 256, 512, 8, 2, P, P, P, P, P, P, n - 1, None) == -4
+
+
+def test_training_entries_check_arguments(moe):
+    """The training forward and the saved backward refuse bad shapes,
+    pointers, alignment and a short workspace before any launch."""
+    P = 4096
+    n = moe.moe_backward_workspace_size(16, 256, 512, 8, 2)
+    assert moe.moe_ffn_forward_train(P, P, P, P, P, 16, 4000, 512, 8, 2, P, P, n, None) == -1  # d_model
+    assert moe.moe_ffn_forward_train(P, P, P, P, P, 16, 256, 512, 8, 2, None, P, n, None) == -1  # no output
+    assert moe.moe_ffn_forward_train(P, P, P + 8, P, P, 16, 256, 512, 8, 2, P, P, n, None) == -3
+    assert moe.moe_ffn_forward_train(P, P, P, P, P, 16, 256, 512, 8, 2, P, P, n - 1, None) == -4
+    assert moe.moe_ffn_backward_saved(P, P, P, None, 16, 256, 512, 8, 2, P, P, P, P, P, P, n, None) == -1  # no dy
+    assert moe.moe_ffn_backward_saved(P, P, P, P, 16, 256, 512, 8, 2, P + 4, P, P, P, P, P, n, None) == -3
+    assert moe.moe_ffn_backward_saved(P, P, P, P, 16, 256, 512, 8, 2, P, P, P, P, P, P, n - 1, None) == -4

@@ -178,3 +178,44 @@ def test_backward_full_size_sampled(moe):
         close(f64(out["dw1"][e, n]), ref["dw1"][q], ref["dw1_abs"][q], "dw1", f"dw1[{e}, {n}, :]")
         close(f64(out["dw3"][e, n]), ref["dw3"][q], ref["dw3_abs"][q], "dw3", f"dw3[{e}, {n}, :]")
         close(f64(out["dw2"][e, :, n]), ref["dw2"][q], ref["dw2_abs"][q], "dw2", f"dw2[{e}, :, {n}]")
+
+
+TRAIN = [
+    # (T, H, F, E, k, seed, skew)
+    (64, 256, 512, 8, 2, 61, False),
+    (300, 256, 512, 8, 2, 62, True),      # big and empty experts
+    (129, 384, 640, 4, 3, 63, False),     # 128-wide tiles
+    (700, 256, 512, 4, 2, 64, False),
+]
+
+
+@pytest.mark.parametrize("path", [0, 3], ids=["pair_tiles", "one_sm_tiles"])
+@pytest.mark.parametrize("p", TRAIN, ids=lambda p: f"T{p[0]}_H{p[1]}_F{p[2]}_E{p[3]}_k{p[4]}" + ("_skew" if p[6] else ""))
+def test_training_pair(moe, p, path):
+    """moe_ffn_forward_train: the BF16 layer from the row-major weights, held
+    to the forward's own check (every output against the oracle, h flips
+    validated); moe_ffn_backward_saved from what it kept: the backward's
+    check against the oracle, and the same gradients as moe_ffn_backward."""
+    from helpers import verify_layer
+    T, H, F, E, k, seed, skew = p
+    moe.moe_set_option(moe.OPT_PATH, path)
+    case = moe_inputs.make_case(T, H, F, E, k, "bf16", seed, skew)
+    dy = moe_inputs.make_dy(T, H, seed).cuda()
+    x, lg = case["x"].cuda(), case["logits"].cuda()
+    w1, w3, w2 = case["w1"].cuda(), case["w3"].cuda(), case["w2"].cuda()
+    out, ws = moe.ffn_forward_train(x, lg, w1, w3, w2, k)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(None) == 0
+    verify_layer(moe, ws, out, case, what=f"training forward T={T} F={F}")
+    saved = moe.ffn_backward_saved(w1, w3, w2, dy, k, ws)
+    again = moe.ffn_backward(x, lg, w1, w3, w2, dy, k)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(None) == 0
+    ref = oracle.ffn_bwd64(*oracle_inputs(case, dy.cpu()), k, round_h=True, round_inter=True, want_abs=True)
+    for name in ("dx", "dw1", "dw3", "dw2", "dlogits"):
+        close(f64(saved[name]), ref[name], ref[name + "_abs"], name, f"saved {name} T={T} F={F}")
+        close(f64(again[name]), ref[name], ref[name + "_abs"], name, f"recomputed {name} T={T} F={F}")
+    # the same g, u, h either way: the weight gradients without cross-tile
+    # atomics match bit for bit
+    for name in ("dw1", "dw3", "dw2"):
+        assert torch.equal(saved[name], again[name]), name
