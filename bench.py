@@ -251,17 +251,18 @@ class ClockSampler:
         return rec
 
 
-def source_sha(kernel="stage1_w13_swiglu"):
+def source_sha(kernel="stage1_w13_swiglu", workload=""):
     """Hash of the code a kernel is compiled from (the grouped GEMMs of the
-    forward: gemm.cu; of the backward: bwd.cu and bwd.cuh; both with the
-    library headers they include -- the public header gives them only status
-    codes), comments and blank space removed, so that an edit to a comment
-    keeps the recorded counters."""
+    forward: gemm.cu; of the backward and of the training forward -- every
+    GEMM of a train_* workload: bwd.cu and bwd.cuh; both with the library
+    headers they include -- the public header gives them only status codes),
+    comments and blank space removed, so that an edit to a comment keeps the
+    recorded counters."""
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixture_experts_routed_02_b200", "csrc")
-    files = ("bwd.cu", "bwd.cuh", "kernels.cuh", "ptx.cuh") if kernel.startswith("bwd") else (
-        "gemm.cu", "kernels.cuh", "ptx.cuh")
+    files = ("bwd.cu", "bwd.cuh", "kernels.cuh", "ptx.cuh") if kernel.startswith("bwd") or workload.startswith(
+        "train") else ("gemm.cu", "kernels.cuh", "ptx.cuh")
     for path in [os.path.join(csrc, n) for n in files]:
         with open(path) as f:
             code = f.read()
@@ -280,7 +281,7 @@ def recorded_traffic(kernel, workload):
             recs = json.load(f)
     except (OSError, ValueError):
         return None
-    sha = source_sha(kernel)
+    sha = source_sha(kernel, workload)
     for r in recs:
         if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == sha:
             return r.get("dram_bytes_per_launch")

@@ -43,7 +43,7 @@ def test_bf16_weights_count_two_bytes_and_no_scales():
 
 def test_recorded_traffic_needs_the_same_kernel_code(monkeypatch):
     assert bench.recorded_traffic("stage1_w13_swiglu", "no-such-workload") is None
-    monkeypatch.setattr(bench, "source_sha", lambda kernel="": "0000000000000000")
+    monkeypatch.setattr(bench, "source_sha", lambda kernel="", workload="": "0000000000000000")
     assert bench.recorded_traffic("stage1_w13_swiglu", "decode") is None
 
 
@@ -132,3 +132,12 @@ def test_mxfp4_weight_bytes():
     fp8 = bench.algorithmic(DECODE, [4] * 8)
     assert 0.5 < w["layer_bytes"] / fp8["layer_bytes"] < 0.55
     assert w["layer_flops"] == fp8["layer_flops"]
+
+
+def test_training_kernels_hash_the_backward_sources():
+    """Every GEMM of a training workload (the training forward's too) comes
+    from the backward's translation unit: its recorded counters are keyed to
+    that unit's hash, the forward layer's to the forward GEMM's."""
+    fwd = bench.source_sha("stage1_w13_swiglu", "prefill")
+    assert bench.source_sha("stage1_w13_swiglu", "train_prefill") == bench.source_sha("bwd_dw13", "train_prefill")
+    assert bench.source_sha("stage1_w13_swiglu", "train_prefill") != fwd
