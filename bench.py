@@ -162,7 +162,17 @@ def algorithmic(spec, counts):
                 s1_bytes=float(s1_bytes), s2_bytes=float(s2_bytes), layer_bytes=float(layer_bytes), active=active)
 
 
-def roofline(spec, alg, dom, dom_ms, window_ms, peaks, peak_kind, name):
+def power_capped(window_ms, clk):
+    """Whether the timed work ran in the sustained regime: a timed region of a
+    second or more, or SM clocks sampled well below their maximum (the power
+    cap pulls a long tensor-core run to about 1.3 GHz).  The sustained GEMM
+    peak is the denominator then, the burst one otherwise."""
+    if window_ms >= 1000.0:
+        return True
+    return bool(clk) and clk.get("sm_mhz", 0) < 0.9 * clk.get("sm_max_mhz", 0)
+
+
+def roofline(spec, alg, dom, dom_ms, window_ms, peaks, peak_kind, name, clk=None):
     """Roofline record of the dominant kernel: algorithmic bytes (HBM-bound
     shapes) or FLOPs (tensor-bound shapes) per launch over its average launch
     time, against the measured peak."""
@@ -182,8 +192,7 @@ def roofline(spec, alg, dom, dom_ms, window_ms, peaks, peak_kind, name):
                 "algorithmic_per_launch": alg[per + "_bytes"]}
     else:
         ach = alg[per + "_flops"] / (dom_ms / 1e3) / 1e12
-        # a timed region of a second or more runs under the power cap: sustained peak; else burst
-        long_run = window_ms >= 1000.0
+        long_run = power_capped(window_ms, clk)
         key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
         base = float(peaks.get(key, FALLBACK_PEAKS[key]))
         peak = base * (FP8_PER_BF16 if fp8 else 1.0)
@@ -570,7 +579,7 @@ def run_gpu_config(args, moe, name, spec, case, weights, dev, world, rank, cpu_s
     names = moe.FWD_KERNELS
     dom = max(names, key=lambda n: kern[n][0])
     dom_ms = kern[dom][0] / max(1, kern[dom][1])
-    roof = roofline(spec, alg, dom, dom_ms, ms_total, peaks, peak_kind, name)
+    roof = roofline(spec, alg, dom, dom_ms, ms_total, peaks, peak_kind, name, clk)
     launches = sum(v[1] for v in kern.values())  # K steps, the same count as the timed region
     rec = {
         "value": value, "unit": "tokens/s", "ms_per_step": ms_step, "steps": args.steps, "warmup": args.warmup,
@@ -741,7 +750,7 @@ def run_gpu_train(args, moe, name, spec, case, dev, world, rank, cpu_seconds):
     dom = max(kflops, key=lambda n: kern[n][0])
     dom_ms = kern[dom][0] / max(1, kern[dom][1])
     peaks, peak_kind = load_peaks()
-    long_run = ms_total >= 1000.0
+    long_run = power_capped(ms_total, clk)
     key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
     peak = float(peaks.get(key, FALLBACK_PEAKS[key]))
     ach = kflops[dom] / (dom_ms / 1e3) / 1e12

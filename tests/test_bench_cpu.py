@@ -141,3 +141,19 @@ def test_training_kernels_hash_the_backward_sources():
     fwd = bench.source_sha("stage1_w13_swiglu", "prefill")
     assert bench.source_sha("stage1_w13_swiglu", "train_prefill") == bench.source_sha("bwd_dw13", "train_prefill")
     assert bench.source_sha("stage1_w13_swiglu", "train_prefill") != fwd
+
+
+def test_power_capped_clocks_select_the_sustained_peak():
+    """A tensor-bound run whose sampled SM clock sat well below its maximum
+    (the power cap) is measured against the sustained GEMM rate even when its
+    timed region is short; at full clock against the burst rate."""
+    spec = dict(T=4096, H=4096, F=14336, E=8, k=2, dtype="fp8", skew=False)
+    alg = bench.algorithmic(spec, [1024] * 8)
+    peaks = {"hbm_gbs": 6540.0, "bf16_tflops": 1633.0, "bf16_tflops_sustained": 1374.0}
+    capped = {"sm_mhz": 1263.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    full = {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.roofline(spec, alg, "stage1_w13_swiglu", 1.0, 300.0, peaks, "measured", "prefill",
+                          capped)["peak"] == 2 * 1374.0
+    assert bench.roofline(spec, alg, "stage1_w13_swiglu", 1.0, 300.0, peaks, "measured", "prefill",
+                          full)["peak"] == 2 * 1633.0
+    assert bench.power_capped(1500.0, None) and not bench.power_capped(10.0, None)
