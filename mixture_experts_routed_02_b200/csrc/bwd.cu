@@ -30,6 +30,9 @@
 //        operands MN-major: dW2_e = dO^T h with dO = w_a dy_t gathered per
 //        slot, and [dW1_e; dW3_e] = dGU^T xg (padding slots are zero in dO,
 //        h, dGU and xg, so they add nothing).
+// The training forward is built from the same kernel: GU (keeping g, u, h for
+// the backward) and FwdW2 [slots x H] = h . W2_e^T, K = F, W2_e rows K-major,
+// with the routing weight applied in the scatter-add of its epilogue.
 // Warp roles as in the forward GEMM: warp 0 lane 0 issues the TMA copies into
 // an NST-deep ring, warp 1 owns TMEM and issues the MMAs, warps 2..5 drain the
 // two TMEM accumulators (the epilogue of one tile overlaps the next tile's
