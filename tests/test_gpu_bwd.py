@@ -219,3 +219,40 @@ def test_training_pair(moe, p, path):
     # atomics match bit for bit
     for name in ("dw1", "dw3", "dw2"):
         assert torch.equal(saved[name], again[name]), name
+
+
+def test_training_pair_in_a_cuda_graph(moe):
+    """The training forward and the saved backward allocate nothing and
+    synchronise nothing: a CUDA graph captured from them replays the same
+    step, bit for bit on the outputs without cross-tile atomics."""
+    T, H, F, E, k = 200, 256, 512, 8, 2
+    case = moe_inputs.make_case(T, H, F, E, k, "bf16", 65)
+    x, lg = case["x"].cuda(), case["logits"].cuda()
+    w1, w3, w2 = case["w1"].cuda(), case["w3"].cuda(), case["w2"].cuda()
+    dy = moe_inputs.make_dy(T, H, 65).cuda()
+    out, ws = moe.ffn_forward_train(x, lg, w1, w3, w2, k)
+    grads = moe.ffn_backward_saved(w1, w3, w2, dy, k, ws)
+    torch.cuda.synchronize()
+    eager = {n: v.clone() for n, v in grads.items()}
+    eager_out = out.clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        moe.ffn_forward_train(x, lg, w1, w3, w2, k, ws=ws, out=out, stream=s)  # warm up on the capture stream
+        moe.ffn_backward_saved(w1, w3, w2, dy, k, ws, out=grads, stream=s)
+        s.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            moe.ffn_forward_train(x, lg, w1, w3, w2, k, ws=ws, out=out, stream=s)
+            moe.ffn_backward_saved(w1, w3, w2, dy, k, ws, out=grads, stream=s)
+    for v in list(grads.values()) + [out]:
+        v.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(None) == 0
+    assert torch.equal(out, eager_out)
+    for n in ("dw1", "dw3", "dw2"):
+        assert torch.equal(grads[n], eager[n]), n
+    for n in ("dx", "dlogits"):
+        torch.testing.assert_close(grads[n], eager[n], rtol=1e-6, atol=1e-6)
+    del g
