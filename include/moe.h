@@ -358,7 +358,8 @@ typedef enum {
     MOE_KERNEL_STAGE1 = 2, /* group GEMM with w1/w3 + SwiGLU */
     MOE_KERNEL_STAGE2 = 3, /* group GEMM with w2 + weighted scatter-add */
     MOE_KERNEL_FINALIZE = 4,
-    MOE_KERNEL_BWD_GU = 5,   /* backward: g, u, h recomputed (group GEMM with w1/w3) */
+    MOE_KERNEL_BWD_GU = 5,   /* backward: g, u, h recomputed (group GEMM with w1/w3); the training forward
+                              * counts its two GEMMs as STAGE1 and STAGE2 */
     MOE_KERNEL_BWD_DH = 6,   /* backward: dh = W2^T dy -> dg, du, routing-weight gradients */
     MOE_KERNEL_BWD_DX = 7,   /* backward: dx = W1^T dg + W3^T du, scatter-add per token */
     MOE_KERNEL_BWD_DW2 = 8,  /* backward: dW2 per expert */

@@ -24,6 +24,12 @@ Use (FP8: e4m3 weights with fp32 per-output-channel scales)::
 ``moe_set_option(OPT_PATH, n)`` forces the tile configuration (0 = by size,
 1 = CTA pairs, 2 = weight streaming, 3 = 128 x 256 tiles, 4 = tiny batches);
 ``moe_profile_enable``/``moe_profile_read`` time each kernel of the layer.
+
+Training (BF16, the row-major weights as they are)::
+
+    out, ws = moe.ffn_forward_train(x, logits, w1, w3, w2, k)   # keeps g, u, h in ws
+    grads = moe.ffn_backward_saved(w1, w3, w2, dy, k, ws)         # dx, dw1, dw3, dw2, dlogits
+    grads = moe.ffn_backward(x, logits, w1, w3, w2, dy, k)        # the same, recomputing g and u
 """
 import ctypes
 import os
@@ -32,7 +38,8 @@ __all__ = [
     "lib", "MOE_OK", "MOE_BF16", "MOE_FP8_E4M3", "WS", "MoeError", "moe_workspace_size", "moe_workspace_region",
     "moe_prepare_weights", "moe_route", "moe_ffn_forward", "moe_get_status", "moe_set_option", "prepare_weights",
     "route", "ffn_forward", "workspace", "ws_view", "EXPORTS", "KERNELS", "moe_profile_enable",
-    "moe_profile_read",
+    "moe_profile_read", "backward_workspace", "ffn_backward", "ffn_forward_train", "ffn_backward_saved",
+    "moe_backward_workspace_size", "moe_ffn_backward", "moe_ffn_forward_train", "moe_ffn_backward_saved",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))

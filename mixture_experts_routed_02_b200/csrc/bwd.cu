@@ -17,9 +17,10 @@
 // expert-padded slot layout -- and read by the MMA K-major (K contiguous) or
 // MN-major (M or N contiguous), as it lies, so nothing is transposed:
 //   GU   [slots x 2F]: xg . [W1_e; W3_e]^T, K = H, both K-major -- g and u
-//        recomputed (activation recomputation: the forward keeps nothing but
-//        its output); the epilogue stores g and u in fp32 and h =
-//        bf16(silu(g) u), zero rows for padding slots;
+//        recomputed (the layer's own forward keeps nothing but its output),
+//        or computed once by the training forward and kept; the epilogue
+//        stores g and u in fp32 and h = bf16(silu(g) u), zero rows for
+//        padding slots;
 //   DH   [slots x F]:  dyg . W2_e, K = H, W2_e [H, F] MN-major -- epilogue:
 //        dw_a (the tile's sum of dh_unweighted * h, one fp32 atomic per row
 //        and tile), dh = w_a * acc, then dg and du into dGU [slots x 2F];
