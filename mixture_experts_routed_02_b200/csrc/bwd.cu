@@ -109,7 +109,7 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// SiLU and the logistic function (the fast division and exponential, as in the
+// The logistic function (the fast division and exponential, as in the
 // forward epilogue: far below the bf16 roundings around them)
 __device__ __forceinline__ float logistic(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 
