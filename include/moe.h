@@ -322,6 +322,8 @@ long long moe_workspace_region(int T, int H, int F, int E, int k, int dtype, int
  *                     tiles (both read by both GEMMs).  The kernel that reads it records
  *                     MOE_ERR_DEVICE_BOUNDS and skips the access; the call's
  *                     outputs are undefined and the context stays usable.
+ *                     Also applies to moe_ffn_backward and
+ *                     moe_ffn_forward_train (after their routing).
  *                     0 (default) = off.
  *   MOE_OPT_GATHER:   how the first group GEMM gets each expert's token rows:
  *                     0 = automatic (currently 2), 1 = the GEMM gathers them

@@ -866,6 +866,13 @@ int train_impl(int part, const void* x, const float* logits, const void* w1, con
         ProfScope ps(fwd ? MOE_KERNEL_ROUTE : MOE_KERNEL_BWD_AUX, st, part == kTrainBackwardSaved ? 0 : route_launches(T, o));
         if (part != kTrainBackwardSaved && launch_route(logits, T, E, k, o, st) != cudaSuccess) return MOE_ERR_CUDA;
     }
+    // failure-detection test hook (as in the forward): one routing-table entry
+    // overwritten with an index far out of range after the routing
+    const int corrupt = g_opt_test_corrupt.load();
+    if (corrupt && part != kTrainBackwardSaved) {
+        void* target = corrupt == 1 ? (void*)o.slot_assign : corrupt == 2 ? (void*)o.mtile_expert : (void*)o.num_mtiles;
+        if (cudaMemsetAsync(target, 0x7F, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     {
         ProfScope ps(fwd ? MOE_KERNEL_QUANT : MOE_KERNEL_BWD_AUX, st);
         SlotGatherArgs g{};

@@ -256,3 +256,28 @@ def test_training_pair_in_a_cuda_graph(moe):
     for n in ("dx", "dlogits"):
         torch.testing.assert_close(grads[n], eager[n], rtol=1e-6, atol=1e-6)
     del g
+
+
+@pytest.mark.parametrize("table", [1, 3], ids=["slot_assign", "num_mtiles"])
+@pytest.mark.parametrize("path", [0, 3], ids=["pair_tiles", "one_sm_tiles"])
+def test_backward_catches_corrupted_routing(moe, table, path):
+    """A routing-table entry far out of range (written on the host side of the
+    call, after routing) is caught by the backward's kernels: the status word
+    says MOE_ERR_DEVICE_BOUNDS, nothing faults, and the next call is correct."""
+    T, H, F, E, k = 64, 256, 512, 8, 2
+    case = moe_inputs.make_case(T, H, F, E, k, "bf16", 66)
+    dy = moe_inputs.make_dy(T, H, 66)
+    moe.moe_set_option(moe.OPT_PATH, path)
+    x, lg = case["x"].cuda(), case["logits"].cuda()
+    w1, w3, w2 = case["w1"].cuda(), case["w3"].cuda(), case["w2"].cuda()
+    old = moe.moe_set_option(moe.OPT_TEST_CORRUPT, table)
+    try:
+        moe.ffn_backward(x, lg, w1, w3, w2, dy.cuda(), k)
+        st = moe.moe_get_status(None)
+        assert st == -7, f"expected MOE_ERR_DEVICE_BOUNDS, got {moe.STATUS_NAMES.get(st, st)}"
+    finally:
+        moe.moe_set_option(moe.OPT_TEST_CORRUPT, old)
+    out = run_bwd(moe, case, dy)
+    ref = oracle.ffn_bwd64(*oracle_inputs(case, dy), k, round_h=True, round_inter=True, want_abs=True)
+    for name in ("dx", "dw1", "dw3", "dw2", "dlogits"):
+        close(f64(out[name]), ref[name], ref[name + "_abs"], name, f"{name} after a corrupted table {table}")
