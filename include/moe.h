@@ -194,7 +194,7 @@ int moe_ffn_forward(const void* x, const float* logits, const void* w13, const v
  *   process exits.  This call allocates nothing.
  *   Returns MOE_ERR_WORKSPACE, before enqueuing anything, when the problem
  *   needs more than that (moe_workspace_size(T,H,F,E,k,dtype) bytes); decode
- *   batches of Mixtral-8x7B experts fit (T = 16: about 18 MB FP8, 34 MB BF16).
+ *   batches of Mixtral-8x7B experts fit (T = 16: about 22 MB FP8, 43 MB BF16).
  *   The first call in each CUDA context looks up the array's device address
  *   (cudaGetSymbolAddress) with that context current; make that first call
  *   before capturing a stream.  A device reset (cudaDeviceReset) ends the

@@ -143,6 +143,17 @@ def test_static_entry_checks_arguments_before_size(moe):
     assert moe.moe_ffn_forward_static(P, P, P, P, P, P, T, H, F, E, k, dt, P, None) == -4
 
 
+def test_static_workspace_holds_the_decode_layer(moe):
+    """The built-in workspace (64 MiB) holds the Mixtral-shaped decode layer
+    (T = 16) in every weight format; the header's figures for it are about
+    22 MB in FP8 and 43 MB in BF16."""
+    cap = moe.moe_static_workspace_bytes()
+    assert cap == 64 << 20
+    need = {d: moe.moe_workspace_size(16, 4096, 14336, 8, 2, moe.dtype_code(d)) for d in ("fp8", "bf16", "mxfp4")}
+    assert all(n <= cap for n in need.values())
+    assert round(need["fp8"] / 1e6) == 22 and round(need["bf16"] / 1e6) == 43
+
+
 def test_test_hook_options_range(moe):
     assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, 4) == -1
     assert moe.moe_set_option(moe.OPT_TEST_CORRUPT, -1) == -1
