@@ -66,7 +66,12 @@ struct Cfg {
     static constexpr int B_ROW_TX = MXW ? 0 : 128;
     static constexpr int STG_BYTES = MXW ? B_ROWS * 64 : 0;
     static constexpr int NCONV = MXW ? 2 : 0;               // converter warps (6, 7)
-    static constexpr int THREADS = 192 + 32 * NCONV;
+    // epilogue warps: 4 (one per TMEM lane quarter), or 8 for the block-scaled
+    // second GEMM with its single accumulator (two warps per lane quarter,
+    // each with half the columns in registers, so the accumulator is free for
+    // the next tile before any atomic is issued)
+    static constexpr int EPI = (STAGE == 2 && NACC == 1 && !MXW) ? 8 : 4;
+    static constexpr int THREADS = 64 + 32 * EPI + 32 * NCONV;
     static constexpr int SFA_BYTES = SFA_VAR ? 512 : 0;
     static constexpr int SFB_BYTES = SFB_VAR ? 512 * (B_ROWS / 128) : 0;
     // bytes that complete one stage: both CTAs' copies count on the even CTA's barrier
@@ -153,7 +158,7 @@ __global__ void __launch_bounds__(Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR, MXW>:
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], PAIR ? 8 : 4);  // the epilogue warps of both CTAs release a pair tile
+            mbar_init(&tempty[i], PAIR ? 2 * C::EPI : C::EPI);  // the epilogue warps of both CTAs release a pair tile
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -692,8 +697,9 @@ __global__ void __launch_bounds__(Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR, MXW>:
             }
         }
         __syncwarp();
-    } else if (warp < 6) {
-        // ---------------- epilogue warps 2..5
+    } else if (warp < 2 + C::EPI) {
+        // ---------------- epilogue warps 2..5 (2..9: warps w and w + 4 share
+        // a lane quarter and split its columns)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;
         int acc = 0;
@@ -823,52 +829,67 @@ __global__ void __launch_bounds__(Cfg<STAGE, FP8, BN, NST, NACC, PAIR, AR, MXW>:
                                                     (size_t)(t - g * args.rows_per_rank) * args.out_pitch);
                     remote = g != args.rank;
                 }
-                // 64 columns per TMEM wait; the accumulator is released as soon as
-                // the last columns are in registers, before their atomics
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 64) {
-                    uint32_t r[64];
-                    tmem_ld_32cols(tbase + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-                    tmem_ld_32cols(tbase + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+                // 64 columns of the accumulator (in registers) into the combine
+                // row: the weighted (and, FP8, channel-scaled) values first, all
+                // scale loads in flight together; then one branch around two
+                // straight runs of atomics (a branch inside the run keeps the
+                // compiler from hoisting the loads)
+                auto emit64 = [&](const uint32_t* r, int col) {
+                    float4 v[16];
+#pragma unroll
+                    for (int i4 = 0; i4 < 16; ++i4)
+                        v[i4] = make_float4(__uint_as_float(r[4 * i4]) * wgt, __uint_as_float(r[4 * i4 + 1]) * wgt,
+                                            __uint_as_float(r[4 * i4 + 2]) * wgt, __uint_as_float(r[4 * i4 + 3]) * wgt);
+                    if constexpr (FP8 && !MXW) {
+                        const float4* cs4 = reinterpret_cast<const float4*>(args.col_scale + (size_t)e * args.rows_b + col);
+#pragma unroll
+                        for (int i4 = 0; i4 < 16; ++i4) {
+                            const float4 sc = __ldg(cs4 + i4);
+                            v[i4].x *= sc.x;
+                            v[i4].y *= sc.y;
+                            v[i4].z *= sc.z;
+                            v[i4].w *= sc.w;
+                        }
+                    }
+                    if (!remote) {
+#pragma unroll
+                        for (int i4 = 0; i4 < 16; ++i4) atomicAdd(reinterpret_cast<float4*>(orow + col + 4 * i4), v[i4]);
+                    } else {  // scalar atomics through peer memory
+#pragma unroll
+                        for (int i4 = 0; i4 < 16; ++i4) {
+                            atomicAdd(orow + col + 4 * i4, v[i4].x);
+                            atomicAdd(orow + col + 4 * i4 + 1, v[i4].y);
+                            atomicAdd(orow + col + 4 * i4 + 2, v[i4].z);
+                            atomicAdd(orow + col + 4 * i4 + 3, v[i4].w);
+                        }
+                    }
+                };
+                if constexpr (C::EPI == 8) {
+                    // this warp's half of the columns, all in registers before the
+                    // (single) accumulator is released; the next tile's MMAs then
+                    // run under this tile's atomics
+                    const int c_lo = ((warp - 2) >> 2) * (BN / 2);
+                    uint32_t r[BN / 2];
+#pragma unroll
+                    for (int j = 0; j < BN / 64; ++j)
+                        tmem_ld_32cols(tbase + c_lo + 32 * j, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * j]));
                     tmem_ld_wait();
-                    if (c0 + 64 == BN) release(acc);
+                    release(acc);
                     if (t >= 0) {
-                        // the 64 weighted (and, FP8, channel-scaled) values first, all
-                        // scale loads in flight together; then one branch around two
-                        // straight runs of atomics (a branch inside the run keeps the
-                        // compiler from hoisting the loads)
-                        const int col = n * BN + c0;
-                        float4 v[16];
 #pragma unroll
-                        for (int i4 = 0; i4 < 16; ++i4)
-                            v[i4] = make_float4(__uint_as_float(r[4 * i4]) * wgt, __uint_as_float(r[4 * i4 + 1]) * wgt,
-                                                __uint_as_float(r[4 * i4 + 2]) * wgt,
-                                                __uint_as_float(r[4 * i4 + 3]) * wgt);
-                        if constexpr (FP8 && !MXW) {
-                            const float4* cs4 =
-                                reinterpret_cast<const float4*>(args.col_scale + (size_t)e * args.rows_b + col);
-#pragma unroll
-                            for (int i4 = 0; i4 < 16; ++i4) {
-                                const float4 sc = __ldg(cs4 + i4);
-                                v[i4].x *= sc.x;
-                                v[i4].y *= sc.y;
-                                v[i4].z *= sc.z;
-                                v[i4].w *= sc.w;
-                            }
-                        }
-                        if (!remote) {
-#pragma unroll
-                            for (int i4 = 0; i4 < 16; ++i4)
-                                atomicAdd(reinterpret_cast<float4*>(orow + col + 4 * i4), v[i4]);
-                        } else {  // scalar atomics through peer memory
-#pragma unroll
-                            for (int i4 = 0; i4 < 16; ++i4) {
-                                atomicAdd(orow + col + 4 * i4, v[i4].x);
-                                atomicAdd(orow + col + 4 * i4 + 1, v[i4].y);
-                                atomicAdd(orow + col + 4 * i4 + 2, v[i4].z);
-                                atomicAdd(orow + col + 4 * i4 + 3, v[i4].w);
-                            }
-                        }
+                        for (int j = 0; j < BN / 128; ++j) emit64(r + 64 * j, n * BN + c_lo + 64 * j);
+                    }
+                } else {
+                    // 64 columns per TMEM wait; the accumulator is released as soon as
+                    // the last columns are in registers, before their atomics
+#pragma unroll 1
+                    for (int c0 = 0; c0 < BN; c0 += 64) {
+                        uint32_t r[64];
+                        tmem_ld_32cols(tbase + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+                        tmem_ld_32cols(tbase + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+                        tmem_ld_wait();
+                        if (c0 + 64 == BN) release(acc);
+                        if (t >= 0) emit64(r, n * BN + c0);
                     }
                 }
             }
