@@ -20,9 +20,12 @@
 // Warp roles (192 threads): warp 0 lane 0 issues TMA loads into an NST-deep
 // shared-memory ring; warp 1 owns TMEM and lane 0 issues the MMAs; warps 2..5
 // drain the TMEM accumulators (double buffered where TMEM has room, so the
-// epilogue of one tile overlaps the main loop of the next).  With MX FP4
-// weights warps 6 and 7 (256 threads) spread each stage's packed weight rows
-// into the 4-bit operand form before the stage counts as full.
+// epilogue of one tile overlaps the main loop of the next; the block-scaled
+// FP8 second GEMM, whose single accumulator leaves TMEM room only for the
+// scales, runs warps 2..9 (320 threads) instead and frees the accumulator
+// before its atomics).  With MX FP4 weights warps 6 and 7 (256 threads)
+// spread each stage's packed weight rows into the 4-bit operand form before
+// the stage counts as full.
 //
 // CTA pairs (PAIR): a cluster of two CTAs on two SMs computes a 256 x BN tile
 // with tcgen05.mma.cta_group::2.  Its two 128-row halves are two m-tiles of
